@@ -1,0 +1,396 @@
+"""Benchmark of the CSA / HCA compressed-attention decode step on B200.
+
+One step = one decode step of one layer for a batch of requests: compressor
+append of the new token (csa_compress_append), lightning-indexer scores
+(csa_index_scores), top-k (csa_topk) and multi-query attention
+(csa_hca_decode_attn), all through the C ABI.  Inputs are seeded synthetic
+data of the workload's shapes; caches are filled through the same append
+path before timing.
+
+Default workload: CSA Pro-like decode at 1M context (1,048,576 tokens =
+262,144 compressed entries per request), batch 4, 128 query heads x 512, 64
+RoPE dims, indexer 64 x 128 MXFP4, top-1024, window 128.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference] [--no-cpu-baseline]
+
+Prints one JSON line (rank 0).  For N > 1 run under torch.distributed.run:
+each rank serves its own batch (requests shard across GPUs, no collective on
+the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from compressed_sparse_long_hca_b200 import inputs as I  # noqa: E402
+
+METRIC = "CSA/HCA decode queries/s per layer at 128K–1M ctx; HBM GB/s vs ~8 TB/s"
+UNIT = "queries/s"
+KEY_BYTES = 68          # one MXFP4 index key: 64 B codes + 4 B scales (d_I = 128)
+ROW_BYTES = 580         # one KV row: 448 B FP8 + 128 B BF16 + 4 B scale (D = 512)
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], "measured", d
+    return 6650.0, "fallback", {}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        import torch
+        try:
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
+        except Exception:
+            self.gpu = str(gpu_index)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from compressed_sparse_long_hca_b200.api import Cache, topk
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    wl = I.WORKLOADS[args.workload]
+    B, T0 = wl.batch, wl.context
+    csa = wl.kind == "csa"
+    steps, warm = args.steps, args.warmup
+    cap = T0 + steps + warm + 256
+    nb = (cap + 127) // 128
+    layer = 0
+    b_kv, b_idx, sink = I.layer_params(wl.seed, layer, wl.kind, wl.D, wl.d_I or 32, wl.H)
+    cache = Cache(n_csa=1 if csa else 0, n_hca=0 if csa else 1, H=wl.H, D=wl.D, D_rope=wl.R,
+                  H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=B, max_blocks_per_request=nb,
+                  pool_blocks=nb * B, b_pos_csa=b_kv[None] if csa else None,
+                  b_pos_idx=b_idx[None] if csa else None, b_pos_hca=None if csa else b_kv[None])
+    rid = torch.arange(B, dtype=torch.int32, device="cuda")
+    for r in range(B):
+        cache.request_alloc(r, cap)
+    # ---- fill the caches to the workload's context through the append path
+    dI = wl.d_I if csa else 0
+    t = 0
+    while t < T0:
+        n_tok = min(I.CHUNK, T0 - t)
+        chunk = t // I.CHUNK
+        parts = [I.device_token_inputs(wl.seed + 7919 * rank, layer, r, chunk, wl.D, dI) for r in range(B)]
+        st = lambda k: torch.stack([p[k][:n_tok] for p in parts]).contiguous() if parts[0][k] is not None else None
+        cache.compress_append(layer, rid, st(0), st(1), st(2), st(3))
+        t += n_tok
+    torch.cuda.synchronize()
+    cache.check_device_error()
+    # ---- per-step inputs (device), generated up front
+    total_steps = steps + warm
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl.seed * 31 + rank)
+    step_c = torch.randn((total_steps, B, 1, wl.D), generator=g, device="cuda")
+    step_z = torch.randn((total_steps, B, 1, wl.D), generator=g, device="cuda")
+    step_ci = torch.randn((total_steps, B, 1, dI), generator=g, device="cuda") if csa else None
+    step_zi = torch.randn((total_steps, B, 1, dI), generator=g, device="cuda") if csa else None
+    q = torch.randn((B, wl.H, wl.D), generator=g, device="cuda").to(torch.bfloat16)
+    qi = torch.randn((B, wl.H_I, dI), generator=g, device="cuda") if csa else None
+    w = torch.randn((B, wl.H_I), generator=g, device="cuda") if csa else None
+    sink_d = torch.from_numpy(sink).cuda()
+    ld = (cap // 4 + 127) // 128 * 128
+    scores = torch.empty((B, ld), device="cuda") if csa else None
+    nv = torch.empty(B, dtype=torch.int32, device="cuda")
+    idx = torch.empty((B, max(wl.k, 1)), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")    # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step(s, ev_idx=None):
+        cache.compress_append(layer, rid, step_c[s], step_z[s], step_ci[s] if csa else None,
+                              step_zi[s] if csa else None)
+        if csa:
+            if ev_idx:
+                ev_idx[0].record(stream)
+            cache.index_scores(layer, rid, qi, w, scores, nv)
+            if ev_idx:
+                ev_idx[1].record(stream)
+            topk(scores, nv, wl.k, idx)
+            cache.decode_attn(layer, rid, q, idx, sink_d, out)
+        else:
+            cache.decode_attn(layer, rid, q, None, sink_d, out)
+
+    launches_per_step = 3 + (3 if csa else 1)
+    for s in range(warm):
+        step(s)
+    torch.cuda.synchronize()
+    cache.check_device_error()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    evi = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s in range(steps):
+        flush.zero_()                       # L2 flushed between timed steps (not timed)
+        ev[s][0].record(stream)
+        step(warm + s, evi[s] if csa else None)
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev)
+    idx_ms = sum(a.elapsed_time(b) for a, b in evi) / steps if csa else None
+    # ---- end to end through the public API with host buffers
+    pin = lambda t: t.cpu().pin_memory() if t is not None else None
+    h_c, h_z, h_ci, h_zi = pin(step_c[:steps]), pin(step_z[:steps]), pin(step_ci[:steps] if csa else None), \
+        pin(step_zi[:steps] if csa else None)
+    h_q, h_qi, h_w = pin(q), pin(qi), pin(w)
+    h_out = torch.empty((B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory()
+    d_c, d_z = torch.empty_like(step_c[0]), torch.empty_like(step_z[0])
+    d_ci = torch.empty_like(step_ci[0]) if csa else None
+    d_zi = torch.empty_like(step_zi[0]) if csa else None
+    d_q, d_qi, d_w = torch.empty_like(q), torch.empty_like(qi) if csa else None, torch.empty_like(w) if csa else None
+    h2d = 0
+    e2e_ms = 0.0
+    for s in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        d_c.copy_(h_c[s], non_blocking=True)
+        d_z.copy_(h_z[s], non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        if csa:
+            d_ci.copy_(h_ci[s], non_blocking=True)
+            d_zi.copy_(h_zi[s], non_blocking=True)
+            d_qi.copy_(h_qi, non_blocking=True)
+            d_w.copy_(h_w, non_blocking=True)
+        cache.compress_append(layer, rid, d_c, d_z, d_ci, d_zi)
+        if csa:
+            cache.index_scores(layer, rid, d_qi, d_w, scores, nv)
+            topk(scores, nv, wl.k, idx)
+            cache.decode_attn(layer, rid, d_q, idx, sink_d, out)
+        else:
+            cache.decode_attn(layer, rid, d_q, None, sink_d, out)
+        h_out.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    copied = [d_c, d_z, d_q] + ([d_ci, d_zi, d_qi, d_w] if csa else [])
+    h2d = sum(t.numel() * t.element_size() for t in copied)
+    d2h = h_out.numel() * h_out.element_size()
+    clk = clocks.stop()
+    cache.check_device_error()
+    # ---- max over ranks
+    tt = torch.tensor([step_ms, e2e_ms, idx_ms or 0.0], dtype=torch.float64, device="cuda")
+    if ws > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    step_ms, e2e_ms, idx_ms = tt.tolist()
+    value = ws * B * steps / (step_ms / 1e3)
+    e2e_value = ws * B * steps / (e2e_ms / 1e3)
+    peak, peak_kind, _ = _peaks()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
+        "ms_per_step": step_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 on mxfp4/fp8/bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "context": T0, "batch_per_gpu": B, "heads": wl.H,
+                   "head_dim": wl.D, "rope_dims": wl.R, "indexer": f"{wl.H_I}x{wl.d_I}",
+                   "topk": wl.k, "window": wl.W, "layers_per_step": 1,
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"request-sharded x{ws}"},
+        "gpu_launches": launches_per_step * steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "clocks": clk,
+    }
+    if csa:
+        n_c = T0 // 4 + (warm + steps // 2) // 4
+        alg = B * (n_c * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
+        ach = alg / (idx_ms / 1e3) / 1e9
+        line["roofline"] = {"bound": "hbm", "kernel": "csa_index_scores", "achieved": ach, "peak": peak,
+                            "unit": "GB/s", "frac": ach / peak, "traffic": None,
+                            "peak_source": peak_kind, "ms_per_launch": idx_ms,
+                            "algorithmic_bytes_per_launch": alg}
+    if rank == 0 and args.cpu_baseline and ws == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+
+def _oracle_cache(wl, rng):
+    """Stored rows in the oracle's format for one request of the workload
+    (random valid codes: the oracle's cost does not depend on the values)."""
+    from oracle import csa_oracle as O
+    T = wl.context + 1
+    N = T // 4 if wl.kind == "csa" else T // 128
+    fp8 = rng.integers(0, 0x7E, (N, wl.D - wl.R), dtype=np.uint8) | (rng.integers(0, 2, (N, 1)) << 7).astype(np.uint8)
+    rope = O.bf16_bits_from_f32(rng.standard_normal((N, wl.R)).astype(np.float32))
+    scale = (np.abs(rng.standard_normal(N)) / 448 + 1e-3).astype(np.float32)
+    kv = O.KVRow(fp8=fp8, rope=rope, scale=scale)
+    keys = None
+    if wl.kind == "csa":
+        keys = O.MXFP4(codes=rng.integers(0, 16, (N, wl.d_I), dtype=np.uint8),
+                       scales=rng.integers(124, 130, (N, wl.d_I // 32), dtype=np.uint8))
+    win = O.quantize_kv(rng.standard_normal((min(T, 128), wl.D)), wl.R)
+    return kv, keys, win, T
+
+
+def oracle_setup(wl):
+    """Untimed set-up of the oracle arm: one request's stored rows."""
+    from oracle import csa_oracle as O
+    rng = np.random.default_rng(wl.seed)
+    kv, keys, win, T = _oracle_cache(wl, rng)
+    p = O.LayerParams(wl.kind, wl.D, wl.R, np.zeros((8, wl.D)), np.zeros((8, wl.d_I or 32)),
+                      m=4 if wl.kind == "csa" else 128)
+    return dict(p=p, kv=kv, keys=keys, win=win, T=T, rng=rng)
+
+
+def oracle_queries(wl, setup, n: int | None = None, budget_s: float | None = None):
+    """Run the fp64 oracle, as it stands, on decode queries of the workload
+    (index scan, top-k and attention over one request's stored rows).
+    Returns (queries done, seconds)."""
+    from oracle import csa_oracle as O
+    rng = setup["rng"]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        q = I.bf16_grid(rng.standard_normal((wl.H, wl.D)).astype(np.float32))
+        qi = rng.standard_normal((wl.H_I, wl.d_I)).astype(np.float32) if wl.kind == "csa" else None
+        w = rng.standard_normal(wl.H_I).astype(np.float32) if wl.kind == "csa" else None
+        O.decode_query(setup["p"], None, q, rng.standard_normal(wl.H), k=wl.k, q_idx=qi, w=w,
+                       entries=(setup["kv"], setup["keys"]), window=setup["win"], T=setup["T"])
+        done += 1
+        el = time.perf_counter() - t0
+        if (n is not None and done >= n) or (n is None and el >= budget_s):
+            return done, el
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return int(max([d.get("num_threads", 1) for d in threadpool_info()] + [1]))
+    except Exception:
+        return os.cpu_count()
+
+
+def _sample_text(wl, done, el):
+    n_ent = (wl.context + 1) // 4 if wl.kind == "csa" else (wl.context + 1) // 128
+    return (f"{done} decode queries of the {wl.name} workload on one request's stored rows "
+            f"({n_ent} compressed entries + 128-token window; index scan, top-k and attention in "
+            f"fp64 numpy), {el:.1f} s")
+
+
+def cpu_baseline(wl, budget_s: float = 15.0):
+    setup = oracle_setup(wl)
+    done, el = oracle_queries(wl, setup, budget_s=budget_s)
+    return {"value": done / el, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": _sample_text(wl, done, el)}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    wl = I.WORKLOADS[args.workload]
+    setup = oracle_setup(wl)
+    oracle_queries(wl, setup, n=args.warmup)                  # untimed warm-up queries
+    done, el = oracle_queries(wl, setup, n=args.steps * wl.batch)
+    value = done / el
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "context": wl.context, "batch_per_gpu": wl.batch, "heads": wl.H,
+                       "head_dim": wl.D, "topk": wl.k},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                             "sample": _sample_text(wl, done, el)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="csa-pro-1m", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+"""Thin Python binding over the C ABI (include/csa.h).
+
+PyTorch supplies device memory and streams; every step of the decode path
+runs in libcsa's CUDA kernels.  Functions here only check tensor shapes,
+dtypes and devices and pass raw pointers.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import CsaCfg, check
+
+VARIANTS = {"auto": _lib.VARIANT_AUTO, "high": _lib.VARIANT_HIGH_OCC, "low": _lib.VARIANT_LOW_OCC}
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream or None
+
+
+def _need(t, dtype, shape=None, name="tensor"):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+class Cache:
+    """A CSA/HCA cache living in one caller-owned device buffer (the arena).
+
+    Layers 0 .. n_csa-1 are CSA layers, n_csa .. n_csa+n_hca-1 HCA layers."""
+
+    def __init__(self, *, n_csa: int, n_hca: int, H: int, D: int, D_rope: int, H_I: int, d_I: int,
+                 max_requests: int, max_blocks_per_request: int, pool_blocks: int,
+                 b_pos_csa=None, b_pos_idx=None, b_pos_hca=None, rope_base: float = 10000.0,
+                 device: str | torch.device = "cuda"):
+        self.lib = _lib.load()
+        self.cfg = CsaCfg(n_csa, n_hca, H, D, D_rope, H_I if n_csa else 0, d_I if n_csa else 0, 128,
+                          max_requests, max_blocks_per_request, pool_blocks, rope_base)
+        nbytes = self.lib.csa_cache_required_bytes(ctypes.byref(self.cfg))
+        if nbytes == 0:
+            raise ValueError("invalid cache configuration")
+        self.nbytes = nbytes
+        self.arena = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = self.arena.data_ptr()
+        aligned = (base + 255) // 256 * 256
+        self.n_csa, self.n_hca = n_csa, n_hca
+        self.H, self.D, self.D_rope, self.H_I, self.d_I = H, D, D_rope, H_I, d_I
+
+        def host(a, shape):
+            if a is None:
+                return None, None
+            arr = np.ascontiguousarray(np.asarray(a, dtype=np.float32).reshape(shape))
+            return arr, arr.ctypes.data
+
+        self._bkv, p_bkv = host(b_pos_csa, (n_csa, 8, D)) if n_csa else (None, None)
+        self._bix, p_bix = host(b_pos_idx, (n_csa, 8, d_I)) if n_csa else (None, None)
+        self._bh, p_bh = host(b_pos_hca, (n_hca, 128, D)) if n_hca else (None, None)
+        handle = ctypes.c_void_p()
+        torch.cuda.synchronize()
+        check(self.lib.csa_cache_init(ctypes.byref(self.cfg), aligned, nbytes, p_bkv, p_bix, p_bh,
+                                      ctypes.byref(handle)), "csa_cache_init")
+        self.handle = handle
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            self.lib.csa_cache_destroy(h)
+            self.handle = None
+
+    # ------------------------------------------------------------ requests
+    def request_alloc(self, req: int, capacity_tokens: int) -> None:
+        check(self.lib.csa_request_alloc(self.handle, req, capacity_tokens), "csa_request_alloc")
+
+    def request_free(self, req: int) -> None:
+        check(self.lib.csa_request_free(self.handle, req), "csa_request_free")
+
+    # ------------------------------------------------------------ the path
+    def compress_append(self, layer: int, req_ids: torch.Tensor, kv_cand, kv_gate,
+                        idx_cand=None, idx_gate=None, stream=None) -> None:
+        n = req_ids.numel()
+        _need(req_ids, torch.int32, name="req_ids")
+        n_tok = kv_cand.shape[1] if n else 0
+        _need(kv_cand, torch.float32, (n, n_tok, self.D), "kv_cand")
+        _need(kv_gate, torch.float32, (n, n_tok, self.D), "kv_gate")
+        if layer < self.n_csa:
+            _need(idx_cand, torch.float32, (n, n_tok, self.d_I), "idx_cand")
+            _need(idx_gate, torch.float32, (n, n_tok, self.d_I), "idx_gate")
+        check(self.lib.csa_compress_append(self.handle, layer, n, _ptr(req_ids), n_tok, _ptr(kv_cand),
+                                           _ptr(kv_gate), _ptr(idx_cand), _ptr(idx_gate),
+                                           _stream(stream)), "csa_compress_append")
+
+    def index_scores(self, layer: int, req_ids, q_idx, w, scores, n_valid, variant="auto",
+                     stream=None) -> None:
+        n = req_ids.numel()
+        _need(req_ids, torch.int32, name="req_ids")
+        _need(q_idx, torch.float32, (n, self.H_I, self.d_I), "q_idx")
+        _need(w, torch.float32, (n, self.H_I), "w")
+        _need(scores, torch.float32, name="scores")
+        _need(n_valid, torch.int32, (n,), "n_valid")
+        if scores.dim() != 2 or scores.shape[0] != n:
+            raise ValueError("scores must be [n, ld]")
+        check(self.lib.csa_index_scores(self.handle, layer, n, _ptr(req_ids), _ptr(q_idx), _ptr(w),
+                                        _ptr(scores), scores.shape[1], _ptr(n_valid),
+                                        VARIANTS[variant], _stream(stream)), "csa_index_scores")
+
+    def decode_attn(self, layer: int, req_ids, q, topk_idx, sink, out, scale=None,
+                    variant="auto", stream=None) -> None:
+        n = req_ids.numel()
+        _need(req_ids, torch.int32, name="req_ids")
+        _need(q, torch.bfloat16, (n, self.H, self.D), "q")
+        _need(out, torch.bfloat16, (n, self.H, self.D), "out")
+        _need(sink, torch.float32, (self.H,), "sink")
+        k = 0
+        if topk_idx is not None:
+            _need(topk_idx, torch.int32, name="topk_idx")
+            k = topk_idx.shape[1]
+        if scale is None:
+            scale = 1.0 / float(np.sqrt(self.D))
+        check(self.lib.csa_hca_decode_attn(self.handle, layer, n, _ptr(req_ids), _ptr(q), _ptr(topk_idx),
+                                           k, _ptr(sink), scale, _ptr(out), VARIANTS[variant],
+                                           _stream(stream)), "csa_hca_decode_attn")
+
+    def check_device_error(self, stream=None) -> None:
+        check(self.lib.csa_check_device_error(self.handle, _stream(stream)), "device")
+
+    # ------------------------------------------------------------ test helpers
+    def row_bytes(self, region: int) -> int:
+        return self.lib.csa_debug_row_bytes(self.handle, region)
+
+    def read_rows(self, layer: int, req: int, region: int, first: int, count: int) -> np.ndarray:
+        buf = np.zeros((count, self.row_bytes(region)), dtype=np.uint8)
+        check(self.lib.csa_debug_rows(self.handle, layer, req, region, first, count,
+                                      buf.ctypes.data, 0), "csa_debug_rows(read)")
+        return buf
+
+    def write_rows(self, layer: int, req: int, region: int, first: int, rows: np.ndarray) -> None:
+        rows = np.ascontiguousarray(rows, dtype=np.uint8)
+        assert rows.shape[1] == self.row_bytes(region)
+        check(self.lib.csa_debug_rows(self.handle, layer, req, region, first, rows.shape[0],
+                                      rows.ctypes.data, 1), "csa_debug_rows(write)")
+
+    def set_length(self, layer: int, req: int, length: int) -> None:
+        check(self.lib.csa_debug_set_length(self.handle, layer, req, length), "csa_debug_set_length")
+
+    def get_length(self, layer: int, req: int) -> int:
+        return int(self.lib.csa_debug_get_length(self.handle, layer, req))
+
+
+def topk(scores: torch.Tensor, n_valid: torch.Tensor, k: int, out: torch.Tensor,
+         variant="auto", stream=None) -> None:
+    lib = _lib.load()
+    _need(scores, torch.float32, name="scores")
+    _need(n_valid, torch.int32, name="n_valid")
+    n = scores.shape[0]
+    _need(out, torch.int32, (n, k), "out")
+    check(lib.csa_topk(_ptr(scores), scores.shape[1], _ptr(n_valid), n, k, _ptr(out),
+                       VARIANTS[variant], _stream(stream)), "csa_topk")
+
+
+# ---------------------------------------------------------------- host row formats
+
+def pack_kv_rows(fp8: np.ndarray, rope_bf16_bits: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """Packed host rows for REGION_KV / REGION_WINDOW: codes | BF16 | fp32 scale."""
+    n = fp8.shape[0]
+    return np.concatenate([fp8.astype(np.uint8).reshape(n, -1),
+                           np.ascontiguousarray(rope_bf16_bits.astype(np.uint16)).view(np.uint8).reshape(n, -1),
+                           np.ascontiguousarray(scale.astype(np.float32)).view(np.uint8).reshape(n, 4)], axis=1)
+
+
+def unpack_kv_rows(rows: np.ndarray, D: int, R: int):
+    fp8 = rows[:, : D - R].copy()
+    bf = np.ascontiguousarray(rows[:, D - R: D - R + 2 * R]).view(np.uint16).reshape(-1, R)
+    sc = np.ascontiguousarray(rows[:, D + R: D + R + 4]).view(np.float32).reshape(-1)
+    return fp8, bf, sc
+
+
+def pack_index_rows(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Packed host rows for REGION_INDEX: E2M1 pairs (element 2i low nibble) | E8M0."""
+    c = codes.astype(np.uint8)
+    packed = (c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)
+    return np.concatenate([packed.astype(np.uint8), scales.astype(np.uint8)], axis=1)
+
+
+def unpack_index_rows(rows: np.ndarray, d_I: int):
+    packed = rows[:, : d_I // 2]
+    codes = np.empty((rows.shape[0], d_I), dtype=np.uint8)
+    codes[:, 0::2] = packed & 0xF
+    codes[:, 1::2] = packed >> 4
+    return codes, rows[:, d_I // 2:].copy()

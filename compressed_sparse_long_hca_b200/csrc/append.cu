@@ -1,0 +1,272 @@
+// Token-level compressor and cache write (csa_compress_append).
+//
+// Page "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力": a token-level
+// compressor turns every 4 tokens' KV into one entry, and the lightning
+// indexer keeps compressed index keys; section "HCA——重度压缩注意力": HCA
+// compresses 128 tokens into one entry, the state cache keeps the latest 128
+// raw tokens and the unfinished tails, the classic cache keeps entries in
+// 128-token blocks.  Page "深度解读DeepSeek V4 看清Benchmark以外的三个范式创新",
+// section 01 "混合注意力的精细解剖": CSA windows overlap so that meaning is not cut
+// at block edges.
+//
+// Entry j of CSA pools tokens [4j-4, 4j+4) (those >= 0), of HCA tokens
+// [128j, 128j+128); per channel the weights are softmax over the window's
+// tokens of (gate logit + position bias of the token's window slot).
+//
+// Three launches per call, stream-ordered:
+//   1. entries: every entry completed by the new tokens (reads tails + input)
+//   2. tokens:  window-ring rows and tail slots of the new tokens
+//   3. length:  L += n_tok
+// Launch 1 reads the tails before launch 2 overwrites them.
+#include "common.cuh"
+
+namespace csa {
+
+struct AppendArgs {
+  Layout L;
+  int layer;
+  int n;
+  const int32_t* req_ids;
+  int n_tok;
+  const float* c;
+  const float* z;
+  const float* ci;
+  const float* zi;
+};
+
+// Fetch channel `ch` of token `tau` (which the entry's window needs) from the
+// new-token input (tau >= L0) or from the request's tail ring.
+__device__ __forceinline__ void fetch_tok(const AppendArgs& a, int i, int64_t L0, int64_t tau, int ch,
+                                          int dim, const float* in_c, const float* in_z,
+                                          const float* tail_c, const float* tail_z, int ring,
+                                          float& c, float& z) {
+  if (tau >= L0) {
+    const int64_t o = ((int64_t)i * a.n_tok + (tau - L0)) * dim + ch;
+    c = in_c[o];
+    z = in_z[o];
+  } else {
+    const int64_t o = (int64_t)(tau % ring) * dim + ch;
+    c = tail_c[o];
+    z = tail_z[o];
+  }
+}
+
+__device__ __forceinline__ bool load_request(const AppendArgs& a, int i, int& req, int64_t& L0) {
+  req = a.req_ids[i];
+  if (req < 0 || req >= a.L.max_req) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) set_err(a.L, kErrBounds, i);
+    return false;
+  }
+  L0 = a.L.lengths()[(int64_t)a.layer * a.L.max_req + req];
+  const int64_t cap = (int64_t)a.L.capacity()[req] * kBlockTokens;
+  if (L0 + a.n_tok > cap) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) set_err(a.L, kErrCapacity, req);
+    return false;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------- launch 1
+
+__global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  const Layout& L = a.L;
+  const int D = L.D, R = L.R, dI = L.dI;
+  float* row = sm;            // [D]
+  float* key = sm + D;        // [dI]
+  float* red = key + dI;      // [32]
+  const int i = blockIdx.x;
+  int req;
+  int64_t L0;
+  if (!load_request(a, i, req, L0)) return;
+  const int64_t n_done = (L0 + a.n_tok) / kCsaM;    // entries complete after the call
+  const float* tc = reinterpret_cast<const float*>(L.tail(req, a.layer));
+  const float* tz = tc + kCsaWin * D;
+  const float* tci = tz + kCsaWin * D;
+  const float* tzi = tci + kCsaWin * dI;
+  const float* bkv = L.bpos_csa(a.layer);
+  const float* bix = L.bpos_idx(a.layer);
+  for (int64_t j = L0 / kCsaM + blockIdx.y; j < n_done; j += gridDim.y) {
+    const int64_t t0 = kCsaM * j - kCsaM;          // first window token (may be < 0)
+    for (int ch = threadIdx.x; ch < D + dI; ch += blockDim.x) {
+      const bool is_kv = ch < D;
+      const int cc = is_kv ? ch : ch - D;
+      const int dim = is_kv ? D : dI;
+      const float* b = is_kv ? bkv : bix;
+      float cv[kCsaWin], lg[kCsaWin];
+      float mx = -INFINITY;
+      for (int s = 0; s < kCsaWin; ++s) {
+        const int64_t tau = t0 + s;
+        if (tau < 0) { lg[s] = -INFINITY; cv[s] = 0.f; continue; }
+        float c, z;
+        fetch_tok(a, i, L0, tau, cc, dim, is_kv ? a.c : a.ci, is_kv ? a.z : a.zi,
+                  is_kv ? tc : tci, is_kv ? tz : tzi, kCsaWin, c, z);
+        cv[s] = c;
+        lg[s] = z + b[s * dim + cc];
+        mx = fmaxf(mx, lg[s]);
+      }
+      float num = 0.f, den = 0.f;
+      for (int s = 0; s < kCsaWin; ++s) {
+        if (lg[s] == -INFINITY) continue;
+        const float e = expf(lg[s] - mx);
+        den += e;
+        num = fmaf(e, cv[s], num);
+      }
+      const float v = __fdiv_rn(num, den);
+      if (is_kv) row[cc] = v; else key[cc] = v;
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
+      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, kCsaM * j, L.rope_base);
+    __syncthreads();
+    const int64_t lb = j / kCsaPerBlock;
+    const int s = (int)(j % kCsaPerBlock);
+    const int32_t blk = L.block_table(req)[lb];
+    char* bp = L.block(blk, a.layer);
+    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(bp) + (int64_t)s * (D - R),
+                 reinterpret_cast<uint16_t*>(bp + L.blk_kv_bf16) + (int64_t)s * R,
+                 reinterpret_cast<float*>(bp + L.blk_kv_scale) + s, red);
+    store_index_key(key, dI, s, reinterpret_cast<uint8_t*>(bp + L.blk_idx_codes),
+                    reinterpret_cast<uint8_t*>(bp + L.blk_idx_scale));
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  const Layout& L = a.L;
+  const int D = L.D, R = L.R;
+  float* row = sm;
+  float* red = sm + D;
+  const int i = blockIdx.x;
+  int req;
+  int64_t L0;
+  if (!load_request(a, i, req, L0)) return;
+  const int64_t n_done = (L0 + a.n_tok) / kHcaM;
+  const float* tc = reinterpret_cast<const float*>(L.tail(req, a.layer));
+  const float* tz = tc + kHcaM * D;
+  const float* b = L.bpos_hca(a.layer - L.n_csa);
+  for (int64_t j = L0 / kHcaM + blockIdx.y; j < n_done; j += gridDim.y) {
+    const int64_t t0 = kHcaM * j;
+    for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
+      float mx = -INFINITY;
+      for (int s = 0; s < kHcaM; ++s) {
+        float c, z;
+        fetch_tok(a, i, L0, t0 + s, ch, D, a.c, a.z, tc, tz, kHcaM, c, z);
+        mx = fmaxf(mx, z + b[s * D + ch]);
+      }
+      float num = 0.f, den = 0.f;
+      for (int s = 0; s < kHcaM; ++s) {
+        float c, z;
+        fetch_tok(a, i, L0, t0 + s, ch, D, a.c, a.z, tc, tz, kHcaM, c, z);
+        const float e = expf(z + b[s * D + ch] - mx);
+        den += e;
+        num = fmaf(e, c, num);
+      }
+      row[ch] = __fdiv_rn(num, den);
+    }
+    __syncthreads();
+    for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
+      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, kHcaM * j, L.rope_base);
+    __syncthreads();
+    const int32_t blk = L.block_table(req)[j];
+    char* bp = L.block(blk, a.layer);
+    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(bp),
+                 reinterpret_cast<uint16_t*>(bp + L.blk_hca_bf16),
+                 reinterpret_cast<float*>(bp + L.blk_hca_scale), red);
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- launch 2
+
+__global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  const Layout& L = a.L;
+  const int D = L.D, R = L.R, dI = L.dI;
+  const bool csa = a.layer < L.n_csa;
+  float* row = sm;
+  float* red = sm + D;
+  const int i = blockIdx.x;
+  int req;
+  int64_t L0;
+  if (!load_request(a, i, req, L0)) return;
+  const int64_t L1 = L0 + a.n_tok;
+  char* st = L.state(req, a.layer);
+  // window ring rows for positions max(L0, L1-128) .. L1-1
+  const int64_t r0 = L1 - kWindow > L0 ? L1 - kWindow : L0;
+  for (int64_t pos = r0 + blockIdx.y; pos < L1; pos += gridDim.y) {
+    const float* src = a.c + ((int64_t)i * a.n_tok + (pos - L0)) * D;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) row[d] = src[d];
+    __syncthreads();
+    for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
+      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, pos, L.rope_base);
+    __syncthreads();
+    const int slot = (int)(pos % kWindow);
+    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),
+                 reinterpret_cast<uint16_t*>(st + L.ring_bf16) + (int64_t)slot * R,
+                 reinterpret_cast<float*>(st + L.ring_scale) + slot, red);
+    __syncthreads();
+  }
+  // tail slots
+  float* tail = reinterpret_cast<float*>(L.tail(req, a.layer));
+  const int ring = csa ? kCsaWin : kHcaM;
+  int64_t t_lo = csa ? L1 - kCsaWin : (L1 / kHcaM) * kHcaM;
+  if (t_lo < L0) t_lo = L0;
+  for (int64_t pos = t_lo + blockIdx.y; pos < L1; pos += gridDim.y) {
+    const int slot = (int)(pos % ring);
+    const int64_t src = (int64_t)i * a.n_tok + (pos - L0);
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      tail[(int64_t)slot * D + d] = a.c[src * D + d];
+      tail[(int64_t)ring * D + (int64_t)slot * D + d] = a.z[src * D + d];
+    }
+    if (csa) {
+      float* ti = tail + 2 * (int64_t)ring * D;
+      for (int d = threadIdx.x; d < dI; d += blockDim.x) {
+        ti[(int64_t)slot * dI + d] = a.ci[src * dI + d];
+        ti[(int64_t)ring * dI + (int64_t)slot * dI + d] = a.zi[src * dI + d];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- launch 3
+
+__global__ void length_kernel(AppendArgs a) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.n) return;
+  const int req = a.req_ids[i];
+  if (req < 0 || req >= a.L.max_req) return;
+  int64_t* len = a.L.lengths() + (int64_t)a.layer * a.L.max_req + req;
+  const int64_t cap = (int64_t)a.L.capacity()[req] * kBlockTokens;
+  if (*len + a.n_tok <= cap) *len += a.n_tok;
+}
+
+cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok,
+                          const float* c, const float* z, const float* ci, const float* zi,
+                          cudaStream_t st) {
+  AppendArgs a{L, layer, n, req_ids, n_tok, c, z, ci, zi};
+  const bool csa = layer < L.n_csa;
+  const int threads = 256;
+  // entries completed by n_tok new tokens: at most n_tok/m + 1 per request
+  const int64_t emax = csa ? n_tok / kCsaM + 1 : n_tok / kHcaM + 1;
+  dim3 g1(n, (unsigned)(emax < 1024 ? emax : 1024));
+  if (csa) {
+    const size_t sm = (size_t)(L.D + L.dI + 32) * sizeof(float);
+    csa_entries_kernel<<<g1, threads, sm, st>>>(a);
+  } else {
+    const size_t sm = (size_t)(L.D + 32) * sizeof(float);
+    hca_entries_kernel<<<g1, threads, sm, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int rows = n_tok < kWindow ? n_tok : kWindow;
+  dim3 g2(n, (unsigned)rows);
+  tokens_kernel<<<g2, threads, (size_t)(L.D + 32) * sizeof(float), st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  length_kernel<<<(n + 127) / 128, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

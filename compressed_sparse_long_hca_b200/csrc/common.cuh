@@ -1,0 +1,133 @@
+// Device helpers shared by the kernels: error word, number formats, partial
+// RoPE.  Format rules (the pages name the formats but not their scaling):
+//   KV row   first D-R dims FP8 E4M3 with one fp32 scale s = amax/448 per row
+//            (s = 1 for an all-zero row), code = E4M3_rn_satfinite(x / s);
+//            last R dims BF16 (round to nearest even).  Page "V4终于终于终于终于
+//            是来了", section "HCA——重度压缩注意力": RoPE dims BF16, others FP8.
+//   MXFP4    per 32 values one E8M0 scale 2^e, e = floor(log2 amax) - 2
+//            clamped to [-127, 127] (e = 0 for an all-zero block), element
+//            code = E2M1_rn_satfinite(x * 2^-e).  Podcast summary page,
+//            section "2.1 推理与计算效率": FP4 on the indexer path.
+//   RoPE     pairs (2i, 2i+1) of the last R dims, angle pos * base^(-2i/R),
+//            computed in fp64 so that positions up to 2^20 keep full accuracy.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "layout.cuh"
+
+namespace csa {
+
+__device__ __forceinline__ void set_err(const Layout& L, int32_t code, int32_t detail) {
+  int32_t* e = L.err();
+  if (atomicCAS(e, 0, code) == 0) e[1] = detail;
+}
+
+__device__ __forceinline__ uint8_t e4m3_rn(float y) {
+  return (uint8_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float e4m3_val(uint8_t c) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+__device__ __forceinline__ uint16_t bf16_rn(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ float bf16_val(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+// Two E2M1 codes in one byte: `lo` in bits 0-3, `hi` in bits 4-7.
+__device__ __forceinline__ uint8_t e2m1x2_rn(float lo, float hi) {
+  return (uint8_t)__nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest);
+}
+
+// E2M1 value of a 4-bit code, exact.
+__device__ __forceinline__ float e2m1_val(uint32_t c) {
+  const uint32_t mag = c & 7u;
+  // magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 as (mag < 2 ? mag*0.5 : (2 + (mag&1)) * 2^((mag>>1) - 2))
+  float v = (mag < 2u) ? 0.5f * (float)mag : (float)(2u + (mag & 1u)) * __int_as_float((127 + (int)(mag >> 1) - 2) << 23);
+  return (c & 8u) ? -v : v;
+}
+
+// Shared exponent of one MX block from its amax (see the rule above).
+__device__ __forceinline__ int mx_exponent(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int e = ilogbf(amax) - 2;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+__device__ __forceinline__ float exp2i(int e) {  // 2^e for -126 <= e <= 127, exact
+  return __int_as_float((e + 127) << 23);
+}
+
+// Multiply by 2^-e exactly (two steps keep every factor a normal fp32).
+__device__ __forceinline__ float scale_pow2(float x, int e) {
+  const int a = -e / 2, b = -e - a;
+  return (x * exp2i(a)) * exp2i(b);
+}
+
+// Rotate the pair (x0, x1) at dim pair i of R rope dims by position pos.
+__device__ __forceinline__ void rope_pair(float& x0, float& x1, int i, int R, int64_t pos, float base) {
+  const double theta = pow((double)base, -2.0 * (double)i / (double)R);
+  double s, c;
+  sincos((double)pos * theta, &s, &c);
+  const double a = x0, b = x1;
+  x0 = (float)(a * c - b * s);
+  x1 = (float)(a * s + b * c);
+}
+
+// Block-wide max of non-negative values; `red` holds >= 32 floats.
+__device__ __forceinline__ float block_max_nonneg(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  const int nw = (blockDim.x + 31) >> 5;
+  v = (l < nw) ? red[l] : 0.f;
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;  // every thread holds the result
+}
+
+// Quantise a row held in shared memory (fp32, already rotated) into the KV
+// format and store it.  All threads of the block take part.
+__device__ __forceinline__ void store_kv_row(const float* row, int D, int R, uint8_t* fp8,
+                                             uint16_t* bf16, float* scale, float* red) {
+  float amax = 0.f;
+  for (int d = threadIdx.x; d < D - R; d += blockDim.x) amax = fmaxf(amax, fabsf(row[d]));
+  amax = block_max_nonneg(amax, red);
+  const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  for (int d = threadIdx.x; d < D - R; d += blockDim.x) fp8[d] = e4m3_rn(__fdiv_rn(row[d], s));
+  for (int d = threadIdx.x; d < R; d += blockDim.x) bf16[d] = bf16_rn(row[D - R + d]);
+  if (threadIdx.x == 0) *scale = s;
+}
+
+// Quantise an index key held in shared memory (fp32, d_I values) to MXFP4 and
+// store it at slot `s` of a block (interleaved code layout, see layout.cuh).
+// One warp per 32-value chunk.
+__device__ __forceinline__ void store_index_key(const float* key, int dI, int s, uint8_t* codes,
+                                                uint8_t* scales) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int CH = dI / 32;
+  for (int c = w; c < CH; c += blockDim.x >> 5) {
+    const float x = key[c * 32 + l];
+    float a = fabsf(x);
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const int e = mx_exponent(a);
+    const float y = scale_pow2(x, e);
+    const float y_hi = __shfl_down_sync(0xffffffffu, y, 1);
+    if ((l & 1) == 0) {
+      const uint8_t b = e2m1x2_rn(y, y_hi);
+      codes[(s >> 3) * (CH * 128) + c * 128 + (s & 7) * 16 + (l >> 1)] = b;
+    }
+    if (l == 0) scales[s * CH + c] = (uint8_t)(e + 127);
+  }
+}
+
+}  // namespace csa

@@ -1,0 +1,417 @@
+// Host side of the C ABI declared in include/csa.h: configuration checks,
+// arena layout, the host-side block allocator, launches and test helpers.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/csa.h"
+#include "layout.cuh"
+
+namespace csa {
+cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok,
+                          const float* c, const float* z, const float* ci, const float* zi,
+                          cudaStream_t st);
+cudaError_t launch_index_simt(const Layout& L, int layer, int n, const int32_t* req_ids,
+                              const float* q_idx, const float* w, float* scores, int64_t ld,
+                              int32_t* n_valid, int tiles_per_cta, cudaStream_t st);
+cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
+                        int32_t* out, int32_t* err, cudaStream_t st);
+cudaError_t launch_attn_simt(const Layout& L, int layer, int n, const int32_t* req_ids,
+                             const uint16_t* q, const int32_t* topk, int k, const float* sink,
+                             float scale, uint16_t* out, int heads_per_cta, cudaStream_t st);
+}  // namespace csa
+
+using csa::Layout;
+
+struct csa_cache {
+  csa_cfg cfg;
+  Layout L;
+  std::vector<int32_t> free_blocks;               // pool blocks not held by a request
+  std::vector<std::vector<int32_t>> req_blocks;   // blocks held by each request
+};
+
+namespace {
+
+thread_local std::string g_err;
+
+csa_status fail(csa_status s, const std::string& msg) {
+  g_err = msg;
+  return s;
+}
+
+csa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(CSA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool cfg_ok(const csa_cfg* c, std::string* why) {
+  auto bad = [&](const char* m) { if (why) *why = m; return false; };
+  if (!c) return bad("cfg is NULL");
+  if (c->n_csa_layers < 0 || c->n_hca_layers < 0 || c->n_csa_layers + c->n_hca_layers < 1)
+    return bad("need at least one layer");
+  if (c->H < 1 || c->H > 128) return bad("H must be in [1, 128]");
+  if (c->D < 64 || c->D > 512 || c->D % 32) return bad("D must be a multiple of 32 in [64, 512]");
+  if (c->D_rope < 16 || c->D_rope % 2 || c->D_rope >= c->D || (c->D - c->D_rope) % 16)
+    return bad("D_rope must be even, >= 16, < D, with D - D_rope a multiple of 16");
+  if (c->n_csa_layers > 0) {
+    if (c->H_I < 1 || c->H_I > 64) return bad("H_I must be in [1, 64]");
+    if (c->d_I < 32 || c->d_I > 128 || c->d_I % 32) return bad("d_I must be 32, 64, 96 or 128");
+  }
+  if (c->window != csa::kWindow) return bad("window must be 128");
+  if (c->max_requests < 1) return bad("max_requests must be >= 1");
+  if (c->max_blocks_per_request < 1) return bad("max_blocks_per_request must be >= 1");
+  if (c->pool_blocks < 1) return bad("pool_blocks must be >= 1");
+  if (!(c->rope_base > 1.f)) return bad("rope_base must be > 1");
+  return true;
+}
+
+Layout make_layout(const csa_cfg& c) {
+  using csa::align_up;
+  const int64_t A = csa::kAlign;
+  Layout L{};
+  L.H = c.H; L.D = c.D; L.R = c.D_rope;
+  L.HI = c.n_csa_layers ? c.H_I : 0;
+  L.dI = c.n_csa_layers ? c.d_I : 32;
+  L.n_csa = c.n_csa_layers; L.n_hca = c.n_hca_layers; L.n_layers = c.n_csa_layers + c.n_hca_layers;
+  L.max_req = c.max_requests; L.max_blocks_per_req = c.max_blocks_per_request;
+  L.pool_blocks = c.pool_blocks; L.rope_base = c.rope_base;
+  L.kv_fp8_bytes = c.D - c.D_rope;
+  L.kv_bf16_bytes = 2 * (int64_t)c.D_rope;
+  // window ring
+  L.ring_fp8 = 0;
+  L.ring_bf16 = align_up(csa::kWindow * L.kv_fp8_bytes, 128);
+  L.ring_scale = L.ring_bf16 + align_up(csa::kWindow * L.kv_bf16_bytes, 128);
+  L.ring_bytes = L.ring_scale + align_up(csa::kWindow * 4, 128);
+  L.csa_tail_bytes = align_up((int64_t)csa::kCsaWin * (2 * c.D + 2 * L.dI) * 4, 128);
+  L.hca_tail_bytes = align_up((int64_t)csa::kHcaM * 2 * c.D * 4, 128);
+  L.state_csa_layer = L.ring_bytes + L.csa_tail_bytes;
+  L.state_hca_layer = L.ring_bytes + L.hca_tail_bytes;
+  L.state_req = align_up(L.n_csa * L.state_csa_layer + L.n_hca * L.state_hca_layer, A);
+  // classic-cache block sections
+  const int P = csa::kCsaPerBlock;
+  L.blk_kv_bf16 = align_up(P * L.kv_fp8_bytes, 128);
+  L.blk_kv_scale = L.blk_kv_bf16 + align_up(P * L.kv_bf16_bytes, 128);
+  L.blk_idx_codes = L.blk_kv_scale + align_up(P * 4, 128);
+  L.blk_idx_scale = L.blk_idx_codes + align_up(P * (L.dI / 2), 128);
+  L.blk_csa_bytes = L.blk_idx_scale + align_up(P * (L.dI / 32), 128);
+  L.blk_hca_bf16 = L.kv_fp8_bytes;                   // one row: fp8 | bf16 | scale
+  L.blk_hca_scale = L.blk_hca_bf16 + L.kv_bf16_bytes;
+  L.blk_hca_bytes = align_up(L.blk_hca_scale + 4, 128);
+  L.block_bytes = align_up(L.n_csa * L.blk_csa_bytes + L.n_hca * L.blk_hca_bytes, A);
+  // arena sections
+  int64_t o = 0;
+  L.off_err = o; o += A;
+  L.off_len = o; o = align_up(o + (int64_t)L.n_layers * L.max_req * 8, A);
+  L.off_cap = o; o = align_up(o + (int64_t)L.max_req * 4, A);
+  L.off_bt = o; o = align_up(o + (int64_t)L.max_req * L.max_blocks_per_req * 4, A);
+  L.off_bkv = o; o = align_up(o + (int64_t)L.n_csa * csa::kCsaWin * c.D * 4, A);
+  L.off_bidx = o; o = align_up(o + (int64_t)L.n_csa * csa::kCsaWin * L.dI * 4, A);
+  L.off_bhca = o; o = align_up(o + (int64_t)L.n_hca * csa::kHcaM * c.D * 4, A);
+  L.off_state = o; o = align_up(o + (int64_t)L.max_req * L.state_req, A);
+  L.off_pool = o; o = align_up(o + (int64_t)L.pool_blocks * L.block_bytes, A);
+  L.total_bytes = o;
+  L.base = nullptr;
+  return L;
+}
+
+bool layer_ok(const csa_cache* c, int32_t layer) { return c && layer >= 0 && layer < c->L.n_layers; }
+
+}  // namespace
+
+extern "C" {
+
+size_t csa_cache_required_bytes(const csa_cfg* cfg) {
+  if (!cfg_ok(cfg, nullptr)) return 0;
+  return (size_t)make_layout(*cfg).total_bytes;
+}
+
+csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes, const float* b_pos_csa,
+                          const float* b_pos_idx, const float* b_pos_hca, csa_cache_t** out) {
+  std::string why;
+  if (!out) return fail(CSA_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (!cfg_ok(cfg, &why)) return fail(CSA_ERR_ARG, why);
+  if (!dev_mem || (reinterpret_cast<uintptr_t>(dev_mem) % csa::kAlign))
+    return fail(CSA_ERR_ARG, "dev_mem must be a 256-byte aligned device pointer");
+  Layout L = make_layout(*cfg);
+  if ((int64_t)bytes < L.total_bytes) return fail(CSA_ERR_CAPACITY, "arena smaller than required bytes");
+  if (cfg->n_csa_layers > 0 && (!b_pos_csa || !b_pos_idx)) return fail(CSA_ERR_ARG, "CSA position biases missing");
+  if (cfg->n_hca_layers > 0 && !b_pos_hca) return fail(CSA_ERR_ARG, "HCA position biases missing");
+  L.base = static_cast<char*>(dev_mem);
+  cudaError_t e = cudaMemset(L.base, 0, (size_t)L.off_bkv);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(arena header)");
+  if (L.n_csa) {
+    e = cudaMemcpy(L.base + L.off_bkv, b_pos_csa, (size_t)L.n_csa * csa::kCsaWin * L.D * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(L.base + L.off_bidx, b_pos_idx, (size_t)L.n_csa * csa::kCsaWin * L.dI * 4, cudaMemcpyHostToDevice);
+  }
+  if (e == cudaSuccess && L.n_hca)
+    e = cudaMemcpy(L.base + L.off_bhca, b_pos_hca, (size_t)L.n_hca * csa::kHcaM * L.D * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(position biases)");
+  csa_cache* c = new (std::nothrow) csa_cache();
+  if (!c) return fail(CSA_ERR_CAPACITY, "host allocation failed");
+  c->cfg = *cfg;
+  c->L = L;
+  c->req_blocks.assign(cfg->max_requests, {});
+  // Hand pool blocks out in a fixed pseudo-random order, so that a request's
+  // blocks are scattered through the pool and every access goes through the
+  // block table.
+  c->free_blocks.resize(cfg->pool_blocks);
+  for (int32_t b = 0; b < cfg->pool_blocks; ++b) c->free_blocks[b] = b;
+  uint64_t s = 0x9E3779B97F4A7C15ull;
+  for (int32_t b = cfg->pool_blocks - 1; b > 0; --b) {
+    s ^= s << 13; s ^= s >> 7; s ^= s << 17;
+    std::swap(c->free_blocks[b], c->free_blocks[s % (uint64_t)(b + 1)]);
+  }
+  *out = c;
+  return CSA_OK;
+}
+
+void csa_cache_destroy(csa_cache_t* cache) { delete cache; }
+
+static csa_status reset_lengths(csa_cache* c, int32_t req) {
+  const Layout& L = c->L;
+  for (int l = 0; l < L.n_layers; ++l) {
+    cudaError_t e = cudaMemset(L.lengths() + (int64_t)l * L.max_req + req, 0, 8);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(length)");
+  }
+  return CSA_OK;
+}
+
+csa_status csa_request_free(csa_cache_t* c, int32_t req) {
+  if (!c || req < 0 || req >= c->L.max_req) return fail(CSA_ERR_ARG, "bad request id");
+  auto& held = c->req_blocks[req];
+  c->free_blocks.insert(c->free_blocks.end(), held.rbegin(), held.rend());
+  held.clear();
+  cudaError_t e = cudaMemset(c->L.capacity() + req, 0, 4);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(capacity)");
+  return reset_lengths(c, req);
+}
+
+csa_status csa_request_alloc(csa_cache_t* c, int32_t req, int64_t capacity_tokens) {
+  if (!c || req < 0 || req >= c->L.max_req) return fail(CSA_ERR_ARG, "bad request id");
+  if (capacity_tokens < 1) return fail(CSA_ERR_ARG, "capacity_tokens must be >= 1");
+  csa_status s = csa_request_free(c, req);
+  if (s != CSA_OK) return s;
+  const int64_t nb = (capacity_tokens + csa::kBlockTokens - 1) / csa::kBlockTokens;
+  if (nb > c->L.max_blocks_per_req) return fail(CSA_ERR_CAPACITY, "capacity exceeds max_blocks_per_request");
+  if (nb > (int64_t)c->free_blocks.size()) return fail(CSA_ERR_CAPACITY, "block pool exhausted");
+  auto& held = c->req_blocks[req];
+  held.assign(c->free_blocks.end() - nb, c->free_blocks.end());
+  std::reverse(held.begin(), held.end());
+  c->free_blocks.resize(c->free_blocks.size() - nb);
+  cudaError_t e = cudaMemcpy(c->L.block_table(req), held.data(), nb * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(block table)");
+  const int32_t nb32 = (int32_t)nb;
+  e = cudaMemcpy(c->L.capacity() + req, &nb32, 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(capacity)");
+  return CSA_OK;
+}
+
+csa_status csa_compress_append(csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                               int32_t n_tok, const float* kv_cand, const float* kv_gate,
+                               const float* idx_cand, const float* idx_gate, csa_stream_t stream) {
+  if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
+  if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
+  if (n == 0) return CSA_OK;
+  if (n_tok < 1) return fail(CSA_ERR_ARG, "n_tok must be >= 1");
+  if (!req_ids || !kv_cand || !kv_gate) return fail(CSA_ERR_ARG, "NULL input");
+  const bool is_csa = layer < c->L.n_csa;
+  if (is_csa && (!idx_cand || !idx_gate)) return fail(CSA_ERR_ARG, "CSA layer needs index-key inputs");
+  cudaError_t e = csa::launch_append(c->L, layer, n, req_ids, n_tok, kv_cand, kv_gate,
+                                     idx_cand, idx_gate, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return CSA_OK;
+}
+
+csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                            const float* q_idx, const float* w, float* scores, int64_t ld,
+                            int32_t* n_valid, csa_variant variant, csa_stream_t stream) {
+  if (!layer_ok(c, layer) || layer >= c->L.n_csa) return fail(CSA_ERR_ARG, "index scores need a CSA layer");
+  if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
+  if (n == 0) return CSA_OK;
+  if (!req_ids || !q_idx || !w || !scores || !n_valid) return fail(CSA_ERR_ARG, "NULL argument");
+  if (ld < 1) return fail(CSA_ERR_ARG, "ld must be >= 1");
+  if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
+  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 16);
+  cudaError_t e = csa::launch_index_simt(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid,
+                                         low ? 1 : 4, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "index launch");
+  return CSA_OK;
+}
+
+csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int32_t n, int32_t k,
+                    int32_t* idx_out, csa_variant variant, csa_stream_t stream) {
+  if (n < 0 || n > 2147483647) return fail(CSA_ERR_ARG, "bad n");
+  if (n == 0) return CSA_OK;
+  if (!scores || !n_valid || !idx_out) return fail(CSA_ERR_ARG, "NULL argument");
+  if (k < 1 || ld < 1) return fail(CSA_ERR_ARG, "k and ld must be >= 1");
+  if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
+  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "topk launch");
+  return CSA_OK;
+}
+
+csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                               const uint16_t* q, const int32_t* topk_idx, int32_t k, const float* sink,
+                               float scale, uint16_t* out, csa_variant variant, csa_stream_t stream) {
+  if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
+  if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
+  if (n == 0) return CSA_OK;
+  if (!req_ids || !q || !sink || !out) return fail(CSA_ERR_ARG, "NULL argument");
+  const bool is_csa = layer < c->L.n_csa;
+  if (is_csa && (!topk_idx || k < 1)) return fail(CSA_ERR_ARG, "CSA layer needs topk_idx and k >= 1");
+  if (!is_csa && topk_idx) return fail(CSA_ERR_ARG, "HCA layer takes topk_idx == NULL");
+  if (!(scale > 0.f)) return fail(CSA_ERR_ARG, "scale must be > 0");
+  if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
+  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 16);
+  int hpc = low ? 4 : 8;
+  while (c->L.H % hpc) hpc >>= 1;
+  cudaError_t e = csa::launch_attn_simt(c->L, layer, n, req_ids, q, topk_idx, is_csa ? k : 0, sink,
+                                        scale, out, hpc, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return CSA_OK;
+}
+
+csa_status csa_check_device_error(csa_cache_t* c, csa_stream_t stream) {
+  if (!c) return fail(CSA_ERR_ARG, "cache is NULL");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int32_t w[2] = {0, 0};
+  e = cudaMemcpy(w, c->L.err(), 8, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
+  if (w[0] == 0) return CSA_OK;
+  const int32_t zero[2] = {0, 0};
+  e = cudaMemcpy(c->L.err(), zero, 8, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word reset)");
+  char msg[160];
+  switch (w[0]) {
+    case csa::kErrBounds:
+      snprintf(msg, sizeof msg, "device: index out of range (detail %d)", w[1]);
+      return fail(CSA_ERR_DEVICE_BOUNDS, msg);
+    case csa::kErrCapacity:
+      snprintf(msg, sizeof msg, "device: append beyond the capacity of request %d", w[1]);
+      return fail(CSA_ERR_CAPACITY, msg);
+    case csa::kErrLd:
+      snprintf(msg, sizeof msg, "device: score row too short for query %d", w[1]);
+      return fail(CSA_ERR_DEVICE_BOUNDS, msg);
+    case csa::kErrTimeout:
+      snprintf(msg, sizeof msg, "device: bounded wait gave up (detail %d)", w[1]);
+      return fail(CSA_ERR_DEVICE_TIMEOUT, msg);
+    default:
+      snprintf(msg, sizeof msg, "device: error %d (detail %d)", w[0], w[1]);
+      return fail(CSA_ERR_DEVICE_BOUNDS, msg);
+  }
+}
+
+const char* csa_last_error(void) { return g_err.c_str(); }
+
+size_t csa_debug_row_bytes(const csa_cache_t* c, int32_t region) {
+  if (!c) return 0;
+  const Layout& L = c->L;
+  if (region == CSA_REGION_KV || region == CSA_REGION_WINDOW) return (size_t)(L.D + L.R + 4);
+  if (region == CSA_REGION_INDEX) return (size_t)(L.dI / 2 + L.dI / 32);
+  return 0;
+}
+
+int64_t csa_debug_get_length(csa_cache_t* c, int32_t layer, int32_t req) {
+  if (!layer_ok(c, layer) || req < 0 || req >= c->L.max_req) return -1;
+  int64_t v = -1;
+  if (cudaMemcpy(&v, c->L.lengths() + (int64_t)layer * c->L.max_req + req, 8, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return -1;
+  return v;
+}
+
+csa_status csa_debug_set_length(csa_cache_t* c, int32_t layer, int32_t req, int64_t len) {
+  if (!layer_ok(c, layer) || req < 0 || req >= c->L.max_req) return fail(CSA_ERR_ARG, "bad layer/request");
+  if (len < 0 || len > (int64_t)c->req_blocks[req].size() * csa::kBlockTokens)
+    return fail(CSA_ERR_CAPACITY, "length beyond the request's capacity");
+  cudaError_t e = cudaMemcpy(c->L.lengths() + (int64_t)layer * c->L.max_req + req, &len, 8, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(length)");
+  return CSA_OK;
+}
+
+// Copy `bytes` between host and device in the requested direction.
+static cudaError_t xfer(void* dev, void* host, size_t bytes, bool write) {
+  return write ? cudaMemcpy(dev, host, bytes, cudaMemcpyHostToDevice)
+               : cudaMemcpy(host, dev, bytes, cudaMemcpyDeviceToHost);
+}
+
+// Rows are moved block by block: a whole block section is copied to host
+// memory, rows are packed or unpacked there, and (for writes) the section is
+// copied back.
+csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t region, int64_t first,
+                          int64_t count, void* host, int32_t write) {
+  if (!layer_ok(c, layer) || req < 0 || req >= c->L.max_req) return fail(CSA_ERR_ARG, "bad layer/request");
+  if (!host || first < 0 || count < 0) return fail(CSA_ERR_ARG, "bad rows");
+  const Layout& L = c->L;
+  const bool is_csa = layer < L.n_csa;
+  const int64_t fp8b = L.kv_fp8_bytes, bfb = L.kv_bf16_bytes;
+  const size_t rb = csa_debug_row_bytes(c, region);
+  if (rb == 0) return fail(CSA_ERR_ARG, "bad region");
+  if (region == CSA_REGION_INDEX && !is_csa) return fail(CSA_ERR_ARG, "index keys exist on CSA layers only");
+  auto& held = c->req_blocks[req];
+  char* h = static_cast<char*>(host);
+  const bool wr = write != 0;
+  if (region == CSA_REGION_WINDOW) {
+    char* st = L.state(req, layer);
+    std::vector<char> ring(L.ring_bytes);
+    cudaError_t e = xfer(st, ring.data(), L.ring_bytes, false);
+    if (e != cudaSuccess) return cuda_fail(e, "debug ring read");
+    for (int64_t r = 0; r < count; ++r) {
+      const int slot = (int)((first + r) % csa::kWindow);
+      char* row = h + r * rb;
+      char* a = ring.data() + L.ring_fp8 + slot * fp8b;
+      char* b = ring.data() + L.ring_bf16 + slot * bfb;
+      char* s = ring.data() + L.ring_scale + slot * 4;
+      if (wr) { memcpy(a, row, fp8b); memcpy(b, row + fp8b, bfb); memcpy(s, row + fp8b + bfb, 4); }
+      else { memcpy(row, a, fp8b); memcpy(row + fp8b, b, bfb); memcpy(row + fp8b + bfb, s, 4); }
+    }
+    if (wr) {
+      e = xfer(st, ring.data(), L.ring_bytes, true);
+      if (e != cudaSuccess) return cuda_fail(e, "debug ring write");
+    }
+    return CSA_OK;
+  }
+  const int64_t per_blk = is_csa ? csa::kCsaPerBlock : 1;
+  const int64_t sec = is_csa ? L.blk_csa_bytes : L.blk_hca_bytes;
+  std::vector<char> buf(sec);
+  const int CH = L.dI / 32;
+  int64_t r = 0;
+  while (r < count) {
+    const int64_t j0 = first + r;
+    const int64_t lb = j0 / per_blk;
+    if (lb >= (int64_t)held.size()) return fail(CSA_ERR_ARG, "entry beyond the request's blocks");
+    char* bp = L.block(held[lb], layer);
+    cudaError_t e = xfer(bp, buf.data(), sec, false);
+    if (e != cudaSuccess) return cuda_fail(e, "debug block read");
+    for (; r < count && (first + r) / per_blk == lb; ++r) {
+      const int s = (int)((first + r) % per_blk);
+      char* row = h + r * rb;
+      if (region == CSA_REGION_KV) {
+        char* a = buf.data() + (is_csa ? s * fp8b : 0);
+        char* b = buf.data() + (is_csa ? L.blk_kv_bf16 + s * bfb : L.blk_hca_bf16);
+        char* sc = buf.data() + (is_csa ? L.blk_kv_scale + s * 4 : L.blk_hca_scale);
+        if (wr) { memcpy(a, row, fp8b); memcpy(b, row + fp8b, bfb); memcpy(sc, row + fp8b + bfb, 4); }
+        else { memcpy(row, a, fp8b); memcpy(row + fp8b, b, bfb); memcpy(row + fp8b + bfb, sc, 4); }
+      } else {
+        for (int ch = 0; ch < CH; ++ch) {
+          char* cp = buf.data() + L.blk_idx_codes + (s >> 3) * (CH * 128) + ch * 128 + (s & 7) * 16;
+          if (wr) memcpy(cp, row + ch * 16, 16); else memcpy(row + ch * 16, cp, 16);
+        }
+        char* sp = buf.data() + L.blk_idx_scale + s * CH;
+        if (wr) memcpy(sp, row + L.dI / 2, CH); else memcpy(row + L.dI / 2, sp, CH);
+      }
+    }
+    if (wr) {
+      e = xfer(bp, buf.data(), sec, true);
+      if (e != cudaSuccess) return cuda_fail(e, "debug block write");
+    }
+  }
+  return CSA_OK;
+}
+
+}  // extern "C"

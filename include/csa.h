@@ -1,0 +1,263 @@
+/*
+ * csa.h -- C ABI of libcsa: the compressed-attention decode step of
+ * DeepSeek-V4-style CSA / HCA layers on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (one decode step of one layer for a batch of requests):
+ *
+ *   csa_compress_append   token-level compressor + cache write
+ *       Source: page "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力"
+ *       (every 4 tokens' KV become one entry) and section "HCA——重度压缩注意力"
+ *       (128 tokens become one entry; state cache holds the last 128 raw
+ *       tokens and the unfinished tails; classic cache blocks of 128 raw
+ *       tokens hold 32 CSA entries and 1 HCA entry); page "深度解读DeepSeek V4
+ *       看清Benchmark以外的三个范式创新", section 01, "混合注意力的精细解剖"
+ *       (CSA windows overlap).
+ *   csa_index_scores      lightning indexer, FP4 query x FP4 keys
+ *       Source: page "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力"
+ *       (down/up-projected index queries, ReLU, scores against compressed
+ *       index keys); podcast summary page, section "2.1 推理与计算效率" (FP4
+ *       on the indexer path).
+ *   csa_topk              top-k selector
+ *       Source: page "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力"
+ *       (top 512 / 1024 compressed entries).
+ *   csa_hca_decode_attn   multi-query attention over the selected (CSA) or all
+ *                         (HCA) compressed entries plus the 128-token raw
+ *                         window, with a per-head sink logit
+ *       Source: page "V4终于终于终于终于是来了", sections "CSA——压缩稀疏注意力"
+ *       and "HCA——重度压缩注意力" (MQA core, sliding window, sink logit in the
+ *       denominator, RoPE on the last 64 dims, FP8 + BF16 KV).
+ *
+ * The precise definition of every step (gating form, overlap geometry,
+ * quantiser rules, RoPE pairing and positions, tie-break, visibility) is the
+ * specification shipped with this library; the points the pages leave open
+ * are settled there and repeated in the comments below.
+ *
+ * Conventions that hold for every function:
+ *   - All device pointers are CUDA device memory owned by the caller; they
+ *     must stay valid until the work queued on `stream` has finished.
+ *   - The library never allocates device memory.  The caller hands one
+ *     device buffer (the arena) to csa_cache_init; the library carves the
+ *     state cache, the classic-cache block pool, block tables and lengths out
+ *     of it.  Host memory owned by the library: the handle and its host-side
+ *     block allocator.
+ *   - Every compute call is asynchronous on `stream` (NULL = legacy default
+ *     stream).  Argument errors are detected on the host and returned before
+ *     anything is launched.  Errors found on the device (request id out of
+ *     range, capacity exceeded, a top-k index out of range) are recorded in a
+ *     device error word, the offending work item is skipped, and
+ *     csa_check_device_error reports them.  No kernel traps.
+ *   - No C++ exception crosses the ABI.  csa_last_error() returns a
+ *     thread-local message for the last failing call.
+ *   - Results are batch-invariant: a request's outputs do not depend on the
+ *     batch size, its position in the batch or the other requests, and the
+ *     two launch variants (csa_variant) return identical bits.
+ *   - BF16 values are passed as uint16_t bit patterns.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct csa_cache csa_cache_t;          /* opaque host-side handle        */
+typedef struct CUstream_st* csa_stream_t;      /* same type as cudaStream_t      */
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_ARG = -1,             /* invalid argument (host-side check)             */
+  CSA_ERR_CAPACITY = -2,        /* block pool or request capacity exhausted       */
+  CSA_ERR_CUDA = -3,            /* a CUDA runtime call failed                     */
+  CSA_ERR_DEVICE_TIMEOUT = -4,  /* a bounded device-side wait gave up             */
+  CSA_ERR_DEVICE_BOUNDS = -5    /* a device-side index check failed               */
+} csa_status;
+
+typedef enum {
+  CSA_VARIANT_AUTO = 0,         /* library picks by batch size                    */
+  CSA_VARIANT_HIGH_OCC = 1,     /* launch shape for a well-fed GPU (large batch)  */
+  CSA_VARIANT_LOW_OCC = 2       /* launch shape for an under-fed GPU (small batch)*/
+} csa_variant;                  /* both return identical bits                     */
+
+/* Regions addressed by csa_debug_rows. */
+typedef enum {
+  CSA_REGION_KV = 0,            /* compressed KV entries, by entry index          */
+  CSA_REGION_INDEX = 1,         /* compressed index keys (CSA layers), by entry   */
+  CSA_REGION_WINDOW = 2         /* raw-token window rows, by token position       */
+} csa_region;
+
+/*
+ * Layer configuration, shared by all layers of the cache.  Layers
+ * 0 .. n_csa_layers-1 are CSA layers, the next n_hca_layers are HCA layers.
+ *   H        query heads (one shared KV head: multi-query attention), <= 128
+ *   D        head dim, multiple of 32, 64 <= D <= 512
+ *   D_rope   RoPE dims (the last D_rope dims of q and KV), even, 16 <= D_rope,
+ *            D - D_rope a multiple of 16
+ *   H_I      indexer heads, 1 <= H_I <= 64 (ignored when n_csa_layers == 0)
+ *   d_I      index dim, one of 32, 64, 96, 128
+ *   window   raw-token sliding window; must be 128
+ *   max_requests            request slots
+ *   max_blocks_per_request  classic-cache blocks a request may hold
+ *                           (a block = 128 raw tokens)
+ *   pool_blocks             blocks in the shared pool
+ *   rope_base               RoPE frequency base (10000)
+ * Entry geometry (fixed): CSA m = 4 with windows of 8 tokens overlapping by 4;
+ * HCA m = 128, no overlap.
+ */
+typedef struct {
+  int32_t n_csa_layers;
+  int32_t n_hca_layers;
+  int32_t H;
+  int32_t D;
+  int32_t D_rope;
+  int32_t H_I;
+  int32_t d_I;
+  int32_t window;
+  int32_t max_requests;
+  int32_t max_blocks_per_request;
+  int32_t pool_blocks;
+  float rope_base;
+} csa_cfg;
+
+/* Bytes of device memory the arena must have for `cfg` (0 if cfg invalid). */
+size_t csa_cache_required_bytes(const csa_cfg* cfg);
+
+/*
+ * Initialise a cache in the caller's device buffer `dev_mem` (256-byte
+ * aligned, `bytes` >= csa_cache_required_bytes).  Position biases of the
+ * compressor gates are copied in from host memory:
+ *   b_pos_csa  float [n_csa_layers][8][D]    bias of KV gates, CSA window slot
+ *   b_pos_idx  float [n_csa_layers][8][d_I]  bias of index-key gates
+ *   b_pos_hca  float [n_hca_layers][128][D]  bias of KV gates, HCA window slot
+ * (NULL allowed when the corresponding layer count is 0).  Synchronous.  All
+ * request lengths start at 0 and no blocks are allocated.
+ */
+csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes,
+                          const float* b_pos_csa, const float* b_pos_idx,
+                          const float* b_pos_hca, csa_cache_t** out);
+
+/* Release the host handle (the arena stays the caller's). */
+void csa_cache_destroy(csa_cache_t* cache);
+
+/*
+ * Give request slot `req` room for `capacity_tokens` raw tokens: blocks are
+ * taken from the pool (in the allocator's order, so a request's blocks are
+ * not contiguous) and its block table is written; every layer's length is
+ * reset to 0.  A slot that already holds blocks is released first.
+ * Synchronous (device copies on the legacy stream).  CSA_ERR_CAPACITY when
+ * the pool or max_blocks_per_request is too small.
+ */
+csa_status csa_request_alloc(csa_cache_t* cache, int32_t req, int64_t capacity_tokens);
+
+/* Return request slot `req`'s blocks to the pool; its lengths become 0. */
+csa_status csa_request_free(csa_cache_t* cache, int32_t req);
+
+/*
+ * Compressor + cache write for `n_tok` new tokens of each of `n` requests of
+ * layer `layer`.  Request i appends tokens at positions L_i .. L_i+n_tok-1,
+ * L_i its current length (held on the device).
+ *   req_ids   device int32 [n]               request slots (distinct)
+ *   kv_cand   device float [n][n_tok][D]     KV candidates c_t
+ *   kv_gate   device float [n][n_tok][D]     gate logits z_t
+ *   idx_cand  device float [n][n_tok][d_I]   index-key candidates (CSA only)
+ *   idx_gate  device float [n][n_tok][d_I]   index-key gate logits (CSA only)
+ * For every completed CSA entry j (4j+3 < L_i+n_tok) the gated pool
+ *   e = sum_t softmax_t(z_t + b_pos[t-4j+4]) * c_t over t in [4j-4, 4j+4), t >= 0
+ * is rotated (RoPE at position 4j on the last D_rope dims) and stored as FP8
+ * E4M3 (first D-D_rope dims, one fp32 scale amax/448 per row) + BF16 (RoPE
+ * dims) in block j/32, slot j%32; the index key pools (idx_cand, idx_gate)
+ * the same way without RoPE and is stored as MXFP4 (E2M1 + one E8M0 scale
+ * per 32 values).  HCA entry j pools t in [128j, 128j+128) and is rotated at
+ * 128j.  Each token's own KV, rotated at its position, is written to the raw
+ * window ring; the unfinished tails are kept in the state cache.
+ * Returns before the work runs.  Capacity overflow and bad request ids are
+ * device errors (the request's append is skipped).
+ */
+csa_status csa_compress_append(csa_cache_t* cache, int32_t layer, int32_t n,
+                               const int32_t* req_ids, int32_t n_tok,
+                               const float* kv_cand, const float* kv_gate,
+                               const float* idx_cand, const float* idx_gate,
+                               csa_stream_t stream);
+
+/*
+ * Lightning-indexer scores of each query against every completed index key
+ * of its request (CSA layers only).  For query i (request req_ids[i], whose
+ * length is T = L after the step's append, N = floor(T/4) entries):
+ *   scores[i*ld + j] = sum_h w[i][h] * max(0, q^_h . k^_j),   j < N
+ * where q^_h is q_idx[i][h] quantised to MXFP4 in the kernel and k^_j the
+ * stored MXFP4 key.  Entries j >= N of the row are not written.
+ *   q_idx    device float [n][H_I][d_I]
+ *   w        device float [n][H_I]
+ *   scores   device float [n][ld]   (ld >= the largest N; checked on device)
+ *   n_valid  device int32 [n]       receives N per query
+ */
+csa_status csa_index_scores(const csa_cache_t* cache, int32_t layer, int32_t n,
+                            const int32_t* req_ids, const float* q_idx, const float* w,
+                            float* scores, int64_t ld, int32_t* n_valid,
+                            csa_variant variant, csa_stream_t stream);
+
+/*
+ * Top-k per query row: the k largest of scores[i*ld + 0 .. n_valid[i]-1];
+ * equal scores go to the lower index; -0.0 equals +0.0; output ascending,
+ * padded with -1 when n_valid[i] < k.
+ *   idx_out  device int32 [n][k]
+ * Scores must not be NaN (a NaN is ordered above +inf).
+ */
+csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int32_t n,
+                    int32_t k, int32_t* idx_out, csa_variant variant, csa_stream_t stream);
+
+/*
+ * Multi-query attention of each query over its rows: for CSA layers the
+ * entries listed in topk_idx[i][0..k) (-1 = none), for HCA layers
+ * (topk_idx == NULL) every completed entry, plus the raw window of positions
+ * max(0, t-127) .. t, t = L-1 the query's own position.  K = V = the stored
+ * row (FP8 x scale, BF16).  With q rotated at t:
+ *   u_hr = scale * q_h . K_r,  mu_h = max(max_r u_hr, sink_h)
+ *   out_h = sum_r e^{u_hr-mu_h} V_r / (sum_r e^{u_hr-mu_h} + e^{sink_h-mu_h})
+ *   q     device uint16 (BF16) [n][H][D]   before RoPE
+ *   sink  device float [H]
+ *   out   device uint16 (BF16) [n][H][D]
+ * Rows are visited in a fixed order (selected entries ascending, then the
+ * window ascending); one query's reduction is never split across thread
+ * blocks.
+ */
+csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t n,
+                               const int32_t* req_ids, const uint16_t* q,
+                               const int32_t* topk_idx, int32_t k, const float* sink,
+                               float scale, uint16_t* out, csa_variant variant,
+                               csa_stream_t stream);
+
+/*
+ * Read and clear the device error word (synchronises `stream`).  Returns
+ * CSA_OK or the first device error recorded since the last check;
+ * csa_last_error() then describes it.
+ */
+csa_status csa_check_device_error(csa_cache_t* cache, csa_stream_t stream);
+
+/* Thread-local description of the last failing call ("" if none). */
+const char* csa_last_error(void);
+
+/* ---------------------------------------------------------------------
+ * Test helpers (synchronous).  They move rows between host memory and the
+ * cache in a packed host format, so that tests can fill a cache from
+ * known codes and read back what the kernels stored.
+ *   CSA_REGION_KV / CSA_REGION_WINDOW rows: D-D_rope bytes E4M3 codes, then
+ *     D_rope BF16 values (2 bytes each, little endian), then one fp32 scale.
+ *   CSA_REGION_INDEX rows: d_I/2 bytes of packed E2M1 codes (element 2i in
+ *     the low nibble of byte i), then d_I/32 E8M0 scale bytes.
+ * `first`/`count` are entry indices (KV, INDEX) or token positions (WINDOW;
+ * only the last 128 positions of the current length are held).
+ * ------------------------------------------------------------------- */
+size_t     csa_debug_row_bytes(const csa_cache_t* cache, int32_t region);
+csa_status csa_debug_rows(csa_cache_t* cache, int32_t layer, int32_t req, int32_t region,
+                          int64_t first, int64_t count, void* host, int32_t write);
+csa_status csa_debug_set_length(csa_cache_t* cache, int32_t layer, int32_t req, int64_t len);
+int64_t    csa_debug_get_length(csa_cache_t* cache, int32_t layer, int32_t req);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* CSA_H_ */

@@ -467,21 +467,22 @@ def bf16_round(x) -> np.ndarray:
     return bf16_value(bf16_bits_from_f32(f32(x)))
 
 
-def decode_query(p: LayerParams, st: RequestState, q, sink, k: int | None = None,
+def decode_query(p: LayerParams, st: RequestState | None, q, sink, k: int | None = None,
                  q_idx=None, w=None, scale: float | None = None,
-                 entries=None, window=None):
+                 entries=None, window=None, T: int | None = None):
     """Full decode step for the query at position t = T - 1 (the token just
     appended): index scores, top-k and attention for CSA; dense attention
     over all entries for HCA.  q: [H, D] BF16 values before RoPE.
-    Returns a dict with the intermediate results."""
-    t = st.T - 1
+    `entries` / `window` may hand in stored rows directly (then `st` may be
+    None and T gives the context length).  Returns a dict with the
+    intermediate results."""
+    t = (st.T if T is None else T) - 1
     if scale is None:
         scale = 1.0 / math.sqrt(p.D)
     if entries is None:
         entries = stored_entries(p, st)
     kvq, keyq = entries
     win = window if window is not None else stored_window(p, st, t)
-    kv_rows = dequantize_kv(kvq)
     out = {}
     if p.kind == "csa":
         qi = dequantize_mxfp4(quantize_mxfp4(q_idx))
@@ -491,9 +492,10 @@ def decode_query(p: LayerParams, st: RequestState, q, sink, k: int | None = None
         # scores (comparison tolerance covers the difference)
         sel = topk(s, k)
         out["topk"] = sel
-        rows = kv_rows[sel[sel >= 0]]
+        j = sel[sel >= 0]
+        rows = dequantize_kv(KVRow(fp8=kvq.fp8[j], rope=kvq.rope[j], scale=kvq.scale[j]))
     else:
-        rows = kv_rows
+        rows = dequantize_kv(kvq)
     rows = np.concatenate([rows, dequantize_kv(win)], axis=0)
     qr = rope(np.asarray(q, np.float64), t, p.R, p.base)
     out["out"] = mqa_attention(qr, rows, sink, scale)

