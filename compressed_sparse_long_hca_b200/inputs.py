@@ -140,7 +140,7 @@ def device_token_inputs(seed: int, layer: int, req: int, chunk: int, D: int, d_I
     filling long contexts quickly.  Returns c, z, ci, zi as fp32 tensors."""
     import torch
     g = torch.Generator(device=device)
-    g.manual_seed(((seed * 1_000_003 + layer) * 1_000_033 + req) * 1_000_037 + chunk)
+    g.manual_seed((((seed * 1_000_003 + layer) * 1_000_033 + req) * 1_000_037 + chunk) % (2**62))
     c = torch.randn((CHUNK, D), generator=g, device=device)
     z = torch.randn((CHUNK, D), generator=g, device=device)
     if d_I:

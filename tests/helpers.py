@@ -13,23 +13,25 @@ from compressed_sparse_long_hca_b200 import inputs as I
 from oracle import csa_oracle as O
 
 # ---------------------------------------------------------------- tolerances
-# Attention output (BF16, O(1) after normalising by the reference's RMS):
-ATT_MAX_ABS = 1e-2      # max |gpu - ref| / rms(ref)
-ATT_MAX_REL = 2e-2      # |gpu - ref| / |ref| for elements with |ref| >= rms(ref)
+# Attention output (BF16).  Outputs are compared after scaling them to O(1)
+# by the reference's RMS sigma, elementwise in the allclose form
+#     |gpu - ref| <= ATT_ATOL * sigma + ATT_RTOL * |ref|.
+ATT_ATOL = 1e-2
+ATT_RTOL = 2e-2
 TOPK_TIE_REL = 1e-3     # oracle scores within this of the k-th score are a tie zone
 
 
-def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "attention") -> None:
+def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "attention") -> float:
+    """Returns the largest |gpu - ref| / sigma seen."""
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
-    rms = math.sqrt(float(np.mean(ref ** 2))) or 1.0
+    sigma = math.sqrt(float(np.mean(ref ** 2))) or 1.0
     err = np.abs(gpu - ref)
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
-    assert err.max() / rms <= ATT_MAX_ABS, f"{what}: max abs err {err.max() / rms:.3e} x rms"
-    big = np.abs(ref) >= rms
-    if big.any():
-        rel = (err[big] / np.abs(ref[big])).max()
-        assert rel <= ATT_MAX_REL, f"{what}: max rel err {rel:.3e}"
+    bad = err > ATT_ATOL * sigma + ATT_RTOL * np.abs(ref)
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements outside tolerance; worst "
+                           f"|err|/sigma {err.max() / sigma:.3e}")
+    return float(err.max() / sigma)
 
 
 def check_kv_rounding(gpu_rows: np.ndarray, ref_vals: np.ndarray, D: int, R: int, what="kv",
