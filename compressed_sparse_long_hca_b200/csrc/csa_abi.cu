@@ -18,6 +18,9 @@ cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_
 cudaError_t launch_index_simt(const Layout& L, int layer, int n, const int32_t* req_ids,
                               const float* q_idx, const float* w, float* scores, int64_t ld,
                               int32_t* n_valid, int tiles_per_cta, cudaStream_t st);
+cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
+                            const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
+                            cudaStream_t st);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
                         int32_t* out, int32_t* err, cudaStream_t st);
 cudaError_t launch_attn_simt(const Layout& L, int layer, int n, const int32_t* req_ids,
@@ -115,6 +118,13 @@ Layout make_layout(const csa_cfg& c) {
   L.total_bytes = o;
   L.base = nullptr;
   return L;
+}
+
+int sm_count() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return v;
 }
 
 bool layer_ok(const csa_cache* c, int32_t layer) { return c && layer >= 0 && layer < c->L.n_layers; }
@@ -236,9 +246,12 @@ csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, cons
   if (!req_ids || !q_idx || !w || !scores || !n_valid) return fail(CSA_ERR_ARG, "NULL argument");
   if (ld < 1) return fail(CSA_ERR_ARG, "ld must be >= 1");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
-  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 16);
-  cudaError_t e = csa::launch_index_simt(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid,
-                                         low ? 1 : 4, (cudaStream_t)stream);
+  const int sms = sm_count();
+  if (sms <= 0) return fail(CSA_ERR_CUDA, "cannot query the SM count");
+  // HIGH: two resident CTAs per SM; LOW: one.  Per-key arithmetic is identical.
+  const bool low = variant == CSA_VARIANT_LOW_OCC;
+  cudaError_t e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid,
+                                       low ? sms : 2 * sms, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "index launch");
   return CSA_OK;
 }
