@@ -129,12 +129,12 @@ def run_gpu(args):
     csa = wl.kind == "csa"
     steps, warm = args.steps, args.warmup
     cap = T0 + steps + warm + 256
-    nb = (cap + 127) // 128
+    nb = (cap + 511) // 512
     layer = 0
     b_kv, b_idx, sink = I.layer_params(wl.seed, layer, wl.kind, wl.D, wl.d_I or 32, wl.H)
     cache = Cache(n_csa=1 if csa else 0, n_hca=0 if csa else 1, H=wl.H, D=wl.D, D_rope=wl.R,
-                  H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=B, max_blocks_per_request=nb,
-                  pool_blocks=nb * B, b_pos_csa=b_kv[None] if csa else None,
+                  H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=B, max_pages_per_request=nb,
+                  pool_pages=nb * B, b_pos_csa=b_kv[None] if csa else None,
                   b_pos_idx=b_idx[None] if csa else None, b_pos_hca=None if csa else b_kv[None])
     rid = torch.arange(B, dtype=torch.int32, device="cuda")
     for r in range(B):

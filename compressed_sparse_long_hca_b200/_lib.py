@@ -22,8 +22,8 @@ class CsaCfg(ctypes.Structure):
     _fields_ = [("n_csa_layers", ctypes.c_int32), ("n_hca_layers", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("D", ctypes.c_int32), ("D_rope", ctypes.c_int32),
                 ("H_I", ctypes.c_int32), ("d_I", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("max_requests", ctypes.c_int32), ("max_blocks_per_request", ctypes.c_int32),
-                ("pool_blocks", ctypes.c_int32), ("rope_base", ctypes.c_float)]
+                ("max_requests", ctypes.c_int32), ("max_pages_per_request", ctypes.c_int32),
+                ("pool_pages", ctypes.c_int32), ("rope_base", ctypes.c_float)]
 
 
 # exported symbol -> (restype, argtypes)

@@ -41,15 +41,17 @@ def _need(t, dtype, shape=None, name="tensor"):
 class Cache:
     """A CSA/HCA cache living in one caller-owned device buffer (the arena).
 
+    Pool pages hold 512 raw tokens (4 classic-cache blocks) of one request.
+
     Layers 0 .. n_csa-1 are CSA layers, n_csa .. n_csa+n_hca-1 HCA layers."""
 
     def __init__(self, *, n_csa: int, n_hca: int, H: int, D: int, D_rope: int, H_I: int, d_I: int,
-                 max_requests: int, max_blocks_per_request: int, pool_blocks: int,
+                 max_requests: int, max_pages_per_request: int, pool_pages: int,
                  b_pos_csa=None, b_pos_idx=None, b_pos_hca=None, rope_base: float = 10000.0,
                  device: str | torch.device = "cuda"):
         self.lib = _lib.load()
         self.cfg = CsaCfg(n_csa, n_hca, H, D, D_rope, H_I if n_csa else 0, d_I if n_csa else 0, 128,
-                          max_requests, max_blocks_per_request, pool_blocks, rope_base)
+                          max_requests, max_pages_per_request, pool_pages, rope_base)
         nbytes = self.lib.csa_cache_required_bytes(ctypes.byref(self.cfg))
         if nbytes == 0:
             raise ValueError("invalid cache configuration")

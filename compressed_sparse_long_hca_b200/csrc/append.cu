@@ -58,7 +58,7 @@ __device__ __forceinline__ bool load_request(const AppendArgs& a, int i, int& re
     return false;
   }
   L0 = a.L.lengths()[(int64_t)a.layer * a.L.max_req + req];
-  const int64_t cap = (int64_t)a.L.capacity()[req] * kBlockTokens;
+  const int64_t cap = (int64_t)a.L.capacity()[req] * kPageTokens;
   if (L0 + a.n_tok > cap) {
     if (threadIdx.x == 0 && blockIdx.y == 0) set_err(a.L, kErrCapacity, req);
     return false;
@@ -119,15 +119,13 @@ __global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
       rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, kCsaM * j, L.rope_base);
     __syncthreads();
-    const int64_t lb = j / kCsaPerBlock;
-    const int s = (int)(j % kCsaPerBlock);
-    const int32_t blk = L.block_table(req)[lb];
-    char* bp = L.block(blk, a.layer);
-    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(bp) + (int64_t)s * (D - R),
-                 reinterpret_cast<uint16_t*>(bp + L.blk_kv_bf16) + (int64_t)s * R,
-                 reinterpret_cast<float*>(bp + L.blk_kv_scale) + s, red);
-    store_index_key(key, dI, s, reinterpret_cast<uint8_t*>(bp + L.blk_idx_codes),
-                    reinterpret_cast<uint8_t*>(bp + L.blk_idx_scale));
+    const int s = (int)(j % kCsaPerPage);
+    char* pp = L.page(L.page_table(req)[j / kCsaPerPage], a.layer);
+    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(pp) + (int64_t)s * (D - R),
+                 reinterpret_cast<uint16_t*>(pp + L.pg_csa_bf16) + (int64_t)s * R,
+                 reinterpret_cast<float*>(pp + L.pg_csa_scale) + s, red);
+    store_index_key(L, key, s, reinterpret_cast<uint8_t*>(pp + L.pg_idx_codes),
+                    reinterpret_cast<uint8_t*>(pp + L.pg_idx_sf));
     __syncthreads();
   }
 }
@@ -169,11 +167,11 @@ __global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
       rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, kHcaM * j, L.rope_base);
     __syncthreads();
-    const int32_t blk = L.block_table(req)[j];
-    char* bp = L.block(blk, a.layer);
-    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(bp),
-                 reinterpret_cast<uint16_t*>(bp + L.blk_hca_bf16),
-                 reinterpret_cast<float*>(bp + L.blk_hca_scale), red);
+    const int s = (int)(j % kHcaPerPage);
+    char* pp = L.page(L.page_table(req)[j / kHcaPerPage], a.layer);
+    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(pp) + (int64_t)s * (D - R),
+                 reinterpret_cast<uint16_t*>(pp + L.pg_hca_bf16) + (int64_t)s * R,
+                 reinterpret_cast<float*>(pp + L.pg_hca_scale) + s, red);
     __syncthreads();
   }
 }
@@ -238,7 +236,7 @@ __global__ void length_kernel(AppendArgs a) {
   const int req = a.req_ids[i];
   if (req < 0 || req >= a.L.max_req) return;
   int64_t* len = a.L.lengths() + (int64_t)a.layer * a.L.max_req + req;
-  const int64_t cap = (int64_t)a.L.capacity()[req] * kBlockTokens;
+  const int64_t cap = (int64_t)a.L.capacity()[req] * kPageTokens;
   if (*len + a.n_tok <= cap) *len += a.n_tok;
 }
 

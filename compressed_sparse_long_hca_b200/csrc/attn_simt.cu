@@ -80,7 +80,6 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
 #pragma unroll
   for (int x = 0; x < 16; ++x) o[x] = 0.f;
   float m = -INFINITY, l = 0.f;
-  const int32_t* bt = L.block_table(req);
   const char* st = L.state(req, a.layer);
   // walk the rows: list slots 0..n_sel-1, then window rows
   const int64_t total = n_sel + n_win;
@@ -91,6 +90,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
       const int64_t r = r0 + rr;
       const uint8_t* fp8 = nullptr;
       const uint16_t* bf = nullptr;
+      const float* scp = nullptr;
       float sc = 0.f;
       bool ok = false;
       if (r < n_sel) {
@@ -99,18 +99,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
           if (j >= n_entries) {
             if (lane == 0) set_err(L, kErrBounds, 2000000 + i);
           } else {
-            const int64_t lb = csa ? j / kCsaPerBlock : j;
-            const int s = csa ? (int)(j % kCsaPerBlock) : 0;
-            const char* bp = L.block(bt[lb], a.layer);
-            if (csa) {
-              fp8 = reinterpret_cast<const uint8_t*>(bp) + (int64_t)s * (D - R);
-              bf = reinterpret_cast<const uint16_t*>(bp + L.blk_kv_bf16) + (int64_t)s * R;
-              sc = reinterpret_cast<const float*>(bp + L.blk_kv_scale)[s];
-            } else {
-              fp8 = reinterpret_cast<const uint8_t*>(bp);
-              bf = reinterpret_cast<const uint16_t*>(bp + L.blk_hca_bf16);
-              sc = *reinterpret_cast<const float*>(bp + L.blk_hca_scale);
-            }
+            L.entry_row(req, a.layer, j, &fp8, &bf, &scp);
+            sc = *scp;
             ok = true;
           }
         }

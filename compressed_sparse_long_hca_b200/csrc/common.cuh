@@ -109,24 +109,27 @@ __device__ __forceinline__ void store_kv_row(const float* row, int D, int R, uin
 }
 
 // Quantise an index key held in shared memory (fp32, d_I values) to MXFP4 and
-// store it at slot `s` of a block (interleaved code layout, see layout.cuh).
-// One warp per 32-value chunk.
-__device__ __forceinline__ void store_index_key(const float* key, int dI, int s, uint8_t* codes,
-                                                uint8_t* scales) {
+// store it as key `s` of a page's index tile (code and scale layout in
+// layout.cuh).  One warp per 32-value chunk; padding chunks and scales are
+// written by the warps that own them.
+__device__ __forceinline__ void store_index_key(const Layout& L, const float* key, int s, uint8_t* tile,
+                                                uint8_t* sfchunk) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  const int CH = dI / 32;
-  for (int c = w; c < CH; c += blockDim.x >> 5) {
-    const float x = key[c * 32 + l];
-    float a = fabsf(x);
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    const int e = mx_exponent(a);
-    const float y = scale_pow2(x, e);
-    const float y_hi = __shfl_down_sync(0xffffffffu, y, 1);
-    if ((l & 1) == 0) {
-      const uint8_t b = e2m1x2_rn(y, y_hi);
-      codes[(s >> 3) * (CH * 128) + c * 128 + (s & 7) * 16 + (l >> 1)] = b;
+  const int CH = L.dI / 32;
+  for (int c = w; c < 4; c += blockDim.x >> 5) {
+    if (c < CH) {
+      const float x = key[c * 32 + l];
+      float a = fabsf(x);
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      const int e = mx_exponent(a);
+      const float y = scale_pow2(x, e);
+      const float y_hi = __shfl_down_sync(0xffffffffu, y, 1);
+      if ((l & 1) == 0) tile[L.idx_code_off(s, c) + (l >> 1)] = e2m1x2_rn(y, y_hi);
+      if (l == 0) sfchunk[Layout::idx_sf_off(s, c)] = (uint8_t)(e + 127);
+    } else {
+      if (c < L.CHs && l < 16) tile[L.idx_code_off(s, c) + l] = 0;
+      if (l == 0) sfchunk[Layout::idx_sf_off(s, c)] = 127;
     }
-    if (l == 0) scales[s * CH + c] = (uint8_t)(e + 127);
   }
 }
 

@@ -1,5 +1,5 @@
 // Host side of the C ABI declared in include/csa.h: configuration checks,
-// arena layout, the host-side block allocator, launches and test helpers.
+// arena layout, the host-side page allocator, launches and test helpers.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -8,7 +8,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/csa.h"
+#include "csa.h"
 #include "layout.cuh"
 
 namespace csa {
@@ -33,8 +33,8 @@ using csa::Layout;
 struct csa_cache {
   csa_cfg cfg;
   Layout L;
-  std::vector<int32_t> free_blocks;               // pool blocks not held by a request
-  std::vector<std::vector<int32_t>> req_blocks;   // blocks held by each request
+  std::vector<int32_t> free_pages;                // pool pages not held by a request
+  std::vector<std::vector<int32_t>> req_pages;    // pages held by each request
 };
 
 namespace {
@@ -65,8 +65,8 @@ bool cfg_ok(const csa_cfg* c, std::string* why) {
   }
   if (c->window != csa::kWindow) return bad("window must be 128");
   if (c->max_requests < 1) return bad("max_requests must be >= 1");
-  if (c->max_blocks_per_request < 1) return bad("max_blocks_per_request must be >= 1");
-  if (c->pool_blocks < 1) return bad("pool_blocks must be >= 1");
+  if (c->max_pages_per_request < 1) return bad("max_pages_per_request must be >= 1");
+  if (c->pool_pages < 1) return bad("pool_pages must be >= 1");
   if (!(c->rope_base > 1.f)) return bad("rope_base must be > 1");
   return true;
 }
@@ -79,8 +79,8 @@ Layout make_layout(const csa_cfg& c) {
   L.HI = c.n_csa_layers ? c.H_I : 0;
   L.dI = c.n_csa_layers ? c.d_I : 32;
   L.n_csa = c.n_csa_layers; L.n_hca = c.n_hca_layers; L.n_layers = c.n_csa_layers + c.n_hca_layers;
-  L.max_req = c.max_requests; L.max_blocks_per_req = c.max_blocks_per_request;
-  L.pool_blocks = c.pool_blocks; L.rope_base = c.rope_base;
+  L.max_req = c.max_requests; L.max_pages_per_req = c.max_pages_per_request;
+  L.pool_pages = c.pool_pages; L.rope_base = c.rope_base;
   L.kv_fp8_bytes = c.D - c.D_rope;
   L.kv_bf16_bytes = 2 * (int64_t)c.D_rope;
   // window ring
@@ -93,28 +93,30 @@ Layout make_layout(const csa_cfg& c) {
   L.state_csa_layer = L.ring_bytes + L.csa_tail_bytes;
   L.state_hca_layer = L.ring_bytes + L.hca_tail_bytes;
   L.state_req = align_up(L.n_csa * L.state_csa_layer + L.n_hca * L.state_hca_layer, A);
-  // classic-cache block sections
-  const int P = csa::kCsaPerBlock;
-  L.blk_kv_bf16 = align_up(P * L.kv_fp8_bytes, 128);
-  L.blk_kv_scale = L.blk_kv_bf16 + align_up(P * L.kv_bf16_bytes, 128);
-  L.blk_idx_codes = L.blk_kv_scale + align_up(P * 4, 128);
-  L.blk_idx_scale = L.blk_idx_codes + align_up(P * (L.dI / 2), 128);
-  L.blk_csa_bytes = L.blk_idx_scale + align_up(P * (L.dI / 32), 128);
-  L.blk_hca_bf16 = L.kv_fp8_bytes;                   // one row: fp8 | bf16 | scale
-  L.blk_hca_scale = L.blk_hca_bf16 + L.kv_bf16_bytes;
-  L.blk_hca_bytes = align_up(L.blk_hca_scale + 4, 128);
-  L.block_bytes = align_up(L.n_csa * L.blk_csa_bytes + L.n_hca * L.blk_hca_bytes, A);
+  // classic-cache page sections (a page = 4 blocks = 512 raw tokens)
+  L.CHs = (L.dI / 32 + 1) / 2 * 2;
+  const int64_t P = csa::kCsaPerPage, PH = csa::kHcaPerPage;
+  L.pg_csa_bf16 = align_up(P * L.kv_fp8_bytes, 128);
+  L.pg_csa_scale = L.pg_csa_bf16 + align_up(P * L.kv_bf16_bytes, 128);
+  L.pg_idx_codes = L.pg_csa_scale + align_up(P * 4, 128);
+  L.pg_idx_sf = L.pg_idx_codes + P * L.CHs * 16;          // codes and scales are adjacent
+  L.idx_tile_bytes = P * L.CHs * 16 + csa::kSfChunk;
+  L.pg_csa_bytes = align_up(L.pg_idx_codes + L.idx_tile_bytes, 128);
+  L.pg_hca_bf16 = align_up(PH * L.kv_fp8_bytes, 16);
+  L.pg_hca_scale = L.pg_hca_bf16 + align_up(PH * L.kv_bf16_bytes, 16);
+  L.pg_hca_bytes = align_up(L.pg_hca_scale + PH * 4, 128);
+  L.page_bytes = align_up(L.n_csa * L.pg_csa_bytes + L.n_hca * L.pg_hca_bytes, A);
   // arena sections
   int64_t o = 0;
   L.off_err = o; o += A;
   L.off_len = o; o = align_up(o + (int64_t)L.n_layers * L.max_req * 8, A);
   L.off_cap = o; o = align_up(o + (int64_t)L.max_req * 4, A);
-  L.off_bt = o; o = align_up(o + (int64_t)L.max_req * L.max_blocks_per_req * 4, A);
+  L.off_pt = o; o = align_up(o + (int64_t)L.max_req * L.max_pages_per_req * 4, A);
   L.off_bkv = o; o = align_up(o + (int64_t)L.n_csa * csa::kCsaWin * c.D * 4, A);
   L.off_bidx = o; o = align_up(o + (int64_t)L.n_csa * csa::kCsaWin * L.dI * 4, A);
   L.off_bhca = o; o = align_up(o + (int64_t)L.n_hca * csa::kHcaM * c.D * 4, A);
   L.off_state = o; o = align_up(o + (int64_t)L.max_req * L.state_req, A);
-  L.off_pool = o; o = align_up(o + (int64_t)L.pool_blocks * L.block_bytes, A);
+  L.off_pool = o; o = align_up(o + (int64_t)L.pool_pages * L.page_bytes, A);
   L.total_bytes = o;
   L.base = nullptr;
   return L;
@@ -165,16 +167,16 @@ csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes, const
   if (!c) return fail(CSA_ERR_CAPACITY, "host allocation failed");
   c->cfg = *cfg;
   c->L = L;
-  c->req_blocks.assign(cfg->max_requests, {});
-  // Hand pool blocks out in a fixed pseudo-random order, so that a request's
-  // blocks are scattered through the pool and every access goes through the
-  // block table.
-  c->free_blocks.resize(cfg->pool_blocks);
-  for (int32_t b = 0; b < cfg->pool_blocks; ++b) c->free_blocks[b] = b;
+  c->req_pages.assign(cfg->max_requests, {});
+  // Hand pool pages out in a fixed pseudo-random order, so that a request's
+  // pages are scattered through the pool and every access goes through the
+  // page table.
+  c->free_pages.resize(cfg->pool_pages);
+  for (int32_t b = 0; b < cfg->pool_pages; ++b) c->free_pages[b] = b;
   uint64_t s = 0x9E3779B97F4A7C15ull;
-  for (int32_t b = cfg->pool_blocks - 1; b > 0; --b) {
+  for (int32_t b = cfg->pool_pages - 1; b > 0; --b) {
     s ^= s << 13; s ^= s >> 7; s ^= s << 17;
-    std::swap(c->free_blocks[b], c->free_blocks[s % (uint64_t)(b + 1)]);
+    std::swap(c->free_pages[b], c->free_pages[s % (uint64_t)(b + 1)]);
   }
   *out = c;
   return CSA_OK;
@@ -193,8 +195,8 @@ static csa_status reset_lengths(csa_cache* c, int32_t req) {
 
 csa_status csa_request_free(csa_cache_t* c, int32_t req) {
   if (!c || req < 0 || req >= c->L.max_req) return fail(CSA_ERR_ARG, "bad request id");
-  auto& held = c->req_blocks[req];
-  c->free_blocks.insert(c->free_blocks.end(), held.rbegin(), held.rend());
+  auto& held = c->req_pages[req];
+  c->free_pages.insert(c->free_pages.end(), held.rbegin(), held.rend());
   held.clear();
   cudaError_t e = cudaMemset(c->L.capacity() + req, 0, 4);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(capacity)");
@@ -206,15 +208,15 @@ csa_status csa_request_alloc(csa_cache_t* c, int32_t req, int64_t capacity_token
   if (capacity_tokens < 1) return fail(CSA_ERR_ARG, "capacity_tokens must be >= 1");
   csa_status s = csa_request_free(c, req);
   if (s != CSA_OK) return s;
-  const int64_t nb = (capacity_tokens + csa::kBlockTokens - 1) / csa::kBlockTokens;
-  if (nb > c->L.max_blocks_per_req) return fail(CSA_ERR_CAPACITY, "capacity exceeds max_blocks_per_request");
-  if (nb > (int64_t)c->free_blocks.size()) return fail(CSA_ERR_CAPACITY, "block pool exhausted");
-  auto& held = c->req_blocks[req];
-  held.assign(c->free_blocks.end() - nb, c->free_blocks.end());
+  const int64_t nb = (capacity_tokens + csa::kPageTokens - 1) / csa::kPageTokens;
+  if (nb > c->L.max_pages_per_req) return fail(CSA_ERR_CAPACITY, "capacity exceeds max_pages_per_request");
+  if (nb > (int64_t)c->free_pages.size()) return fail(CSA_ERR_CAPACITY, "page pool exhausted");
+  auto& held = c->req_pages[req];
+  held.assign(c->free_pages.end() - nb, c->free_pages.end());
   std::reverse(held.begin(), held.end());
-  c->free_blocks.resize(c->free_blocks.size() - nb);
-  cudaError_t e = cudaMemcpy(c->L.block_table(req), held.data(), nb * 4, cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(block table)");
+  c->free_pages.resize(c->free_pages.size() - nb);
+  cudaError_t e = cudaMemcpy(c->L.page_table(req), held.data(), nb * 4, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(page table)");
   const int32_t nb32 = (int32_t)nb;
   e = cudaMemcpy(c->L.capacity() + req, &nb32, 4, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(capacity)");
@@ -248,10 +250,10 @@ csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, cons
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
   const int sms = sm_count();
   if (sms <= 0) return fail(CSA_ERR_CUDA, "cannot query the SM count");
-  // HIGH: two resident CTAs per SM; LOW: one.  Per-key arithmetic is identical.
-  const bool low = variant == CSA_VARIANT_LOW_OCC;
-  cudaError_t e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid,
-                                       low ? sms : 2 * sms, (cudaStream_t)stream);
+  // One persistent CTA per SM for either variant; the per-key arithmetic
+  // does not depend on the grid.
+  cudaError_t e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, sms,
+                                       (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "index launch");
   return CSA_OK;
 }
@@ -340,7 +342,7 @@ int64_t csa_debug_get_length(csa_cache_t* c, int32_t layer, int32_t req) {
 
 csa_status csa_debug_set_length(csa_cache_t* c, int32_t layer, int32_t req, int64_t len) {
   if (!layer_ok(c, layer) || req < 0 || req >= c->L.max_req) return fail(CSA_ERR_ARG, "bad layer/request");
-  if (len < 0 || len > (int64_t)c->req_blocks[req].size() * csa::kBlockTokens)
+  if (len < 0 || len > (int64_t)c->req_pages[req].size() * csa::kPageTokens)
     return fail(CSA_ERR_CAPACITY, "length beyond the request's capacity");
   cudaError_t e = cudaMemcpy(c->L.lengths() + (int64_t)layer * c->L.max_req + req, &len, 8, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(length)");
@@ -353,7 +355,7 @@ static cudaError_t xfer(void* dev, void* host, size_t bytes, bool write) {
                : cudaMemcpy(host, dev, bytes, cudaMemcpyDeviceToHost);
 }
 
-// Rows are moved block by block: a whole block section is copied to host
+// Rows are moved page by page: a whole page section is copied to host
 // memory, rows are packed or unpacked there, and (for writes) the section is
 // copied back.
 csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t region, int64_t first,
@@ -366,7 +368,7 @@ csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t re
   const size_t rb = csa_debug_row_bytes(c, region);
   if (rb == 0) return fail(CSA_ERR_ARG, "bad region");
   if (region == CSA_REGION_INDEX && !is_csa) return fail(CSA_ERR_ARG, "index keys exist on CSA layers only");
-  auto& held = c->req_blocks[req];
+  auto& held = c->req_pages[req];
   char* h = static_cast<char*>(host);
   const bool wr = write != 0;
   if (region == CSA_REGION_WINDOW) {
@@ -389,39 +391,45 @@ csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t re
     }
     return CSA_OK;
   }
-  const int64_t per_blk = is_csa ? csa::kCsaPerBlock : 1;
-  const int64_t sec = is_csa ? L.blk_csa_bytes : L.blk_hca_bytes;
+  const int64_t per_pg = L.rows_per_page(layer);
+  const int64_t sec = is_csa ? L.pg_csa_bytes : L.pg_hca_bytes;
   std::vector<char> buf(sec);
   const int CH = L.dI / 32;
   int64_t r = 0;
   while (r < count) {
     const int64_t j0 = first + r;
-    const int64_t lb = j0 / per_blk;
-    if (lb >= (int64_t)held.size()) return fail(CSA_ERR_ARG, "entry beyond the request's blocks");
-    char* bp = L.block(held[lb], layer);
-    cudaError_t e = xfer(bp, buf.data(), sec, false);
-    if (e != cudaSuccess) return cuda_fail(e, "debug block read");
-    for (; r < count && (first + r) / per_blk == lb; ++r) {
-      const int s = (int)((first + r) % per_blk);
+    const int64_t lp = j0 / per_pg;
+    if (lp >= (int64_t)held.size()) return fail(CSA_ERR_ARG, "entry beyond the request's pages");
+    char* pp = L.page(held[lp], layer);
+    cudaError_t e = xfer(pp, buf.data(), sec, false);
+    if (e != cudaSuccess) return cuda_fail(e, "debug page read");
+    for (; r < count && (first + r) / per_pg == lp; ++r) {
+      const int s = (int)((first + r) % per_pg);
       char* row = h + r * rb;
       if (region == CSA_REGION_KV) {
-        char* a = buf.data() + (is_csa ? s * fp8b : 0);
-        char* b = buf.data() + (is_csa ? L.blk_kv_bf16 + s * bfb : L.blk_hca_bf16);
-        char* sc = buf.data() + (is_csa ? L.blk_kv_scale + s * 4 : L.blk_hca_scale);
+        char* a = buf.data() + s * fp8b;
+        char* b = buf.data() + (is_csa ? L.pg_csa_bf16 : L.pg_hca_bf16) + s * bfb;
+        char* sc = buf.data() + (is_csa ? L.pg_csa_scale : L.pg_hca_scale) + s * 4;
         if (wr) { memcpy(a, row, fp8b); memcpy(b, row + fp8b, bfb); memcpy(sc, row + fp8b + bfb, 4); }
         else { memcpy(row, a, fp8b); memcpy(row + fp8b, b, bfb); memcpy(row + fp8b + bfb, sc, 4); }
       } else {
-        for (int ch = 0; ch < CH; ++ch) {
-          char* cp = buf.data() + L.blk_idx_codes + (s >> 3) * (CH * 128) + ch * 128 + (s & 7) * 16;
-          if (wr) memcpy(cp, row + ch * 16, 16); else memcpy(row + ch * 16, cp, 16);
+        char* tile = buf.data() + L.pg_idx_codes;
+        for (int ch = 0; ch < L.CHs; ++ch) {
+          char* cp = tile + L.idx_code_off(s, ch);
+          if (ch < CH) { if (wr) memcpy(cp, row + ch * 16, 16); else memcpy(row + ch * 16, cp, 16); }
+          else if (wr) memset(cp, 0, 16);
         }
-        char* sp = buf.data() + L.blk_idx_scale + s * CH;
-        if (wr) memcpy(sp, row + L.dI / 2, CH); else memcpy(row + L.dI / 2, sp, CH);
+        char* sf = buf.data() + L.pg_idx_sf;
+        for (int k = 0; k < 4; ++k) {
+          char* sp = sf + Layout::idx_sf_off(s, k);
+          if (k < CH) { if (wr) *sp = row[L.dI / 2 + k]; else row[L.dI / 2 + k] = *sp; }
+          else if (wr) *sp = 127;
+        }
       }
     }
     if (wr) {
-      e = xfer(bp, buf.data(), sec, true);
-      if (e != cudaSuccess) return cuda_fail(e, "debug block write");
+      e = xfer(pp, buf.data(), sec, true);
+      if (e != cudaSuccess) return cuda_fail(e, "debug page write");
     }
   }
   return CSA_OK;

@@ -6,22 +6,28 @@
 // summary page, section "2.1 推理与计算效率": the indexer path runs in FP4.
 //   s_j = sum_h w_h * max(0, q^_h . k^_j),   q^, k^ MXFP4 (E2M1, E8M0 per 32)
 //
-// Shape of the work: per query a [N x d_I] x [d_I x H_I] product with N up to
-// 262,144 keys and H_I = 64, i.e. an FP4 GEMM whose A operand (the keys) is
-// streamed once from HBM.  Each CTA owns a contiguous range of 128-key tiles
-// (4 classic-cache blocks) of the flattened (query, tile) list:
-//   * thread 0 streams each tile's codes and E8M0 scales from the paged cache
-//     into a ring of shared-memory stages with bulk async copies (one per
-//     block section; the cache stores codes in the no-swizzle K-major core
-//     matrix order, so the copy lands ready for the MMA);
-//   * the tile's key scales go to TMEM (tcgen05.st) and thread 0 issues the
-//     block-scaled MMA  D[128 keys x 64 heads] = K^ Q^T  (kind::mxf4,
-//     M=128, N=64, K=64 per instruction) into one of two TMEM accumulators;
-//   * while the tensor core works on tile t, all four warps read tile t-1's
-//     accumulator (one TMEM lane = one key, 64 columns = its 64 head dot
-//     products) and reduce sum_h w_h max(0, d_h) in fixed head order.
-// Every key's score is produced by the same instruction sequence whatever the
+// Shape of the work: per query an FP4 product [N keys x d_I] x [d_I x H_I]
+// with N up to 262,144 and H_I = 64 whose A operand (the keys, 68 B each) is
+// streamed once from HBM.  The cache stores the index keys of every 512-token
+// page as one ready-made operand tile (codes in the no-swizzle K-major
+// core-matrix order, scales in the 32 x 128-bit order of tcgen05.cp), so a
+// 128-key tile is one bulk copy.  One persistent CTA per SM owns a contiguous
+// range of tiles of the flattened (query, tile) list and runs three roles:
+//   * producer (warp 0): one bulk async copy per tile into a ring of
+//     shared-memory stages;
+//   * MMA (warp 1): one thread copies the tile's key scales into TMEM
+//     (tcgen05.cp) and issues the block-scaled MMA
+//     D[128 keys x 64 heads] = K^ Q^T (kind::mxf4, M=128, N=64, K=64 per
+//     instruction) into one of four TMEM accumulators;
+//   * epilogue (warps 2-9, two groups of four taking alternate tiles): read a
+//     finished accumulator (one TMEM lane = one key, 64 columns = its 64 head
+//     dot products) and reduce sum_h w_h max(0, d_h) in a fixed order.  At a
+//     query boundary they quantise the next query's index heads to MXFP4 (the
+//     B operand and its scale chunk).
+// Every key's score comes from the same instruction sequence whatever the
 // grid, so launch variants and batch compositions return identical bits.
+// All waits are bounded: a stuck pipeline records a timeout in the device
+// error word, lets in-flight copies land, frees TMEM and returns.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -29,25 +35,37 @@ namespace csa {
 
 namespace {
 
-constexpr int kStages = 6;
-constexpr int kThreads = 128;
-constexpr int kTileKeys = 128;
+constexpr int kStages = 8;             // shared-memory stages of key tiles
+constexpr int kNA = 4;                 // TMEM accumulators (and key-scale buffers)
+constexpr int kEpiGroups = 2;
+constexpr int kEpiThreads = 128 * kEpiGroups;
+constexpr int kThreads = 64 + kEpiThreads;   // warp 0 producer, warp 1 MMA, warps 2.. epilogue
 constexpr int kHeadsN = 64;            // MMA N (index heads, zero padded)
 constexpr int kMaxCh = 4;              // d_I / 32 <= 4
-// TMEM columns (allocation of 256)
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kAcc0 = 0, kAcc1 = 64, kSfa0 = 128, kSfa1 = 132, kSfb = 136;
+constexpr int kTileBytes = kCsaPerPage * kMaxCh * 16 + kSfChunk;   // codes + scale chunk
+constexpr int kPassTiles = 512;        // tiles per pass (page-table window in smem)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfaCol = 256;      // + 4 * accumulator index
+constexpr uint32_t kSfbCol = 272;
 
 struct IdxSmem {
-  uint8_t codes[kStages][kTileKeys * kMaxCh * 16];   // 128 keys x up to 64 B, core-matrix order
-  uint8_t sfs[kStages][kTileKeys * kMaxCh];          // per block: [32 keys][CH] bytes
+  uint8_t tiles[kStages][kTileBytes];                // one page's index tile per stage
   uint8_t qb[kHeadsN * kMaxCh * 16];                 // query codes, core-matrix order
-  uint8_t sfq[kHeadsN][kMaxCh];
-  float w[kHeadsN];
-  uint64_t full[kStages];
-  uint64_t mdone[2];
+  uint8_t qsf[kSfChunk];                             // query scales, tcgen05.cp order
+  alignas(16) float w[kHeadsN];
+  int32_t pgs[kPassTiles];                           // pool page of every tile of the pass
+  // segments of the pass: one per query touched
+  int32_t seg_q[kPassTiles];
+  int32_t seg_n[kPassTiles];
+  int64_t seg_t0[kPassTiles];
+  int64_t seg_N[kPassTiles];
+  int32_t n_seg;
+  uint64_t full[kStages], stage_empty[kStages];
+  uint64_t acc_full[kNA], acc_empty[kNA];
+  uint64_t q_ready;
+  uint64_t drain;
   uint32_t tmem_base;
-  int abort;
+  volatile int abort;
 };
 
 struct IndexTcArgs {
@@ -62,7 +80,7 @@ struct IndexTcArgs {
   int32_t* n_valid;
 };
 
-// Number of 128-key tiles of query i (0 for an invalid query).
+// Number of 128-key tiles of query i (0 for an invalid query); N = its keys.
 __device__ __forceinline__ int64_t query_tiles(const IndexTcArgs& a, int i, int64_t* n_keys, int* req_out) {
   const int req = a.req_ids[i];
   *req_out = req;
@@ -70,22 +88,36 @@ __device__ __forceinline__ int64_t query_tiles(const IndexTcArgs& a, int i, int6
   const int64_t N = a.L.lengths()[(int64_t)a.layer * a.L.max_req + req] / kCsaM;
   *n_keys = N;
   if (N > a.ld) return 0;
-  return (N + kTileKeys - 1) / kTileKeys;
+  return (N + kCsaPerPage - 1) / kCsaPerPage;
+}
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(IdxSmem& sm, uint64_t* bar, uint32_t parity) {
+  if (tc::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = tc::globaltimer_ns();
+  for (uint32_t spin = 0;; ++spin) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if ((spin & 127u) == 127u) {
+      if (sm.abort) return false;
+      if (tc::globaltimer_ns() - t0 > 2000000000ull) { sm.abort = 1; return false; }
+    }
+  }
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 2) index_tc_kernel(IndexTcArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout& L = a.L;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int HI = L.HI, dI = L.dI, CH = dI / 32;
-  const int CHs = (CH + 1) / 2 * 2;                 // chunks per key in smem (multiple of 2)
+  const int HI = L.HI, dI = L.dI, CH = dI / 32, CHs = L.CHs;
   const int n_mma = CHs / 2;                        // K = 64 per instruction
   const uint32_t sbo = (uint32_t)CHs * 128;
+  const uint32_t tile_bytes = (uint32_t)L.idx_tile_bytes;
+  const uint32_t sf_off = (uint32_t)(kCsaPerPage * CHs * 16);
 
-  // ---- per-query bookkeeping (every CTA computes the same prefix)
+  // ---- per-query bookkeeping; every CTA computes the same tile prefix
   if (blockIdx.x == 0) {
     for (int i = tid; i < a.n; i += kThreads) {
       int64_t N;
@@ -105,200 +137,230 @@ __global__ void __launch_bounds__(kThreads, 2) index_tc_kernel(IndexTcArgs a) {
   const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
   if (g0 >= g1) return;
 
-  // ---- set-up: TMEM, barriers, zero padding
-  if (warp == 0) {
+  // ---- set-up
+  if (warp == 1) {
     tc::tmem_alloc(&sm.tmem_base, kTmemCols);
     tc::tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) tc::mbar_init(&sm.full[s], 1);
-    tc::mbar_init(&sm.mdone[0], 1);
-    tc::mbar_init(&sm.mdone[1], 1);
+    for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.stage_empty[s], 1); }
+    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], 128); }
+    tc::mbar_init(&sm.q_ready, 1);
+    tc::mbar_init(&sm.drain, 1);
     sm.abort = 0;
     tc::fence_mbar_init();
-  }
-  if (CHs != CH) {   // chunks past d_I stay zero for the whole kernel
-    for (int x = tid; x < kStages * kTileKeys * kMaxCh * 16 / 16; x += kThreads)
-      reinterpret_cast<uint4*>(&sm.codes[0][0])[x] = make_uint4(0, 0, 0, 0);
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
 
-  // locate the first tile of this CTA
+  // role state (each role only uses its own)
+  uint32_t u_base = 0;       // CTA-wide tile counter at the start of the pass (barrier phases)
+  uint32_t seg_count = 0;    // segments processed (q_ready phases)
+  uint32_t last_issue[kStages];
+  for (int s = 0; s < kStages; ++s) last_issue[s] = 0xFFFFFFFFu;
   int qi = 0;
-  int64_t before = 0, Nq = 0;
-  int req = 0;
-  for (;; ++qi) {
-    const int64_t t = query_tiles(a, qi, &Nq, &req);
-    if (before + t > g0) break;
-    before += t;
-  }
+  int64_t before = 0;        // tiles of queries < qi
   int64_t g = g0;
-  uint32_t cnt = 0;                 // tiles processed by this CTA (barrier phases)
-  bool ok = true;
-  uint32_t pending = 0;             // thread 0: stages with a copy in flight
-  uint32_t pend_par = 0;            //           and the parity that copy completes
 
-  auto issue_load = [&](int stage, uint32_t gidx, int qry_req, int64_t tile, int64_t N) {
-    const int32_t* bt = L.block_table(qry_req);
-    uint32_t bytes = 0;
-    for (int bb = 0; bb < 4; ++bb) {
-      const int64_t lb = tile * 4 + bb;
-      if (lb * kCsaPerBlock < N) bytes += 4u * (uint32_t)CH * 128u + 32u * (uint32_t)CH;
-    }
-    tc::mbar_arrive_expect_tx(&sm.full[stage], bytes);
-    for (int bb = 0; bb < 4; ++bb) {
-      const int64_t lb = tile * 4 + bb;
-      if (lb * kCsaPerBlock >= N) continue;
-      const char* bp = L.block(bt[lb], a.layer);
-      uint8_t* dst = &sm.codes[stage][bb * 4 * CHs * 128];
-      if (CHs == CH) {
-        tc::bulk_g2s(dst, bp + L.blk_idx_codes, 4u * CH * 128u, &sm.full[stage]);
-      } else {
-        for (int rg = 0; rg < 4; ++rg)
-          tc::bulk_g2s(dst + rg * CHs * 128, bp + L.blk_idx_codes + rg * CH * 128, (uint32_t)CH * 128u,
-                       &sm.full[stage]);
-      }
-      tc::bulk_g2s(&sm.sfs[stage][bb * 32 * CH], bp + L.blk_idx_scale, 32u * CH, &sm.full[stage]);
-    }
-    pending |= 1u << stage;
-    pend_par = (pend_par & ~(1u << stage)) | ((((gidx / kStages) & 1u)) << stage);
-  };
-
-  while (g < g1 && ok) {
-    // ---- segment: tiles of query qi inside [g, g1)
-    int64_t nt_q;
-    while ((nt_q = query_tiles(a, qi, &Nq, &req)) == 0 || before + nt_q <= g) { before += nt_q; ++qi; }
-    const int64_t t_first = g - before;
-    const int64_t t_end = (g1 - before < nt_q) ? g1 - before : nt_q;
-    const int64_t n_t = t_end - t_first;
-    // quantise this query's index heads to MXFP4 in shared memory
-    for (int x = tid; x < kHeadsN * CHs * 16 / 16; x += kThreads)
-      reinterpret_cast<uint4*>(sm.qb)[x] = make_uint4(0, 0, 0, 0);
+  while (g < g1 && !sm.abort) {
+    // ---- pass prologue: segment table and page window (all threads)
     __syncthreads();
-    const float* q = a.q_idx + (int64_t)qi * HI * dI;
-    for (int blk = warp; blk < HI * CH; blk += kThreads / 32) {
-      const int h = blk / CH, c = blk % CH;
-      const float x = q[h * dI + c * 32 + lane];
-      float am = fabsf(x);
-      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      const int e = mx_exponent(am);
-      const float y = scale_pow2(x, e);
-      const float y1 = __shfl_down_sync(0xffffffffu, y, 1);
-      if ((lane & 1) == 0) sm.qb[(h >> 3) * sbo + c * 128 + (h & 7) * 16 + (lane >> 1)] = e2m1x2_rn(y, y1);
-      if (lane == 0) sm.sfq[h][c] = (uint8_t)(e + 127);
+    if (tid == 0) {
+      int ns = 0;
+      int64_t gg = g, used = 0;
+      while (gg < g1 && used < kPassTiles) {
+        int64_t N;
+        int req;
+        const int64_t nt = query_tiles(a, qi, &N, &req);
+        if (nt == 0 || before + nt <= gg) { before += nt; ++qi; continue; }
+        const int64_t t0 = gg - before;
+        int64_t cnt = (g1 - before < nt ? g1 - before : nt) - t0;
+        if (cnt > kPassTiles - used) cnt = kPassTiles - used;
+        sm.seg_q[ns] = qi;
+        sm.seg_t0[ns] = t0;
+        sm.seg_n[ns] = (int32_t)cnt;
+        sm.seg_N[ns] = N;
+        ++ns;
+        used += cnt;
+        gg += cnt;
+      }
+      sm.n_seg = ns;
     }
-    for (int h = tid; h < kHeadsN; h += kThreads) sm.w[h] = h < HI ? a.w[(int64_t)qi * HI + h] : 0.f;
     __syncthreads();
     {
-      uint32_t wq[2];
-      for (int k = 0; k < 2; ++k) {
-        const int h = lane + 32 * k;
-        uint32_t word = 0;
-        for (int c = 0; c < 4; ++c) word |= (uint32_t)((h < HI && c < CH) ? sm.sfq[h][c] : 127) << (8 * c);
-        wq[k] = word;
+      int base = 0;
+      for (int sg = 0; sg < sm.n_seg; ++sg) {
+        const int32_t* pt = L.page_table(a.req_ids[sm.seg_q[sg]]);
+        for (int x = tid; x < sm.seg_n[sg]; x += kThreads) sm.pgs[base + x] = pt[sm.seg_t0[sg] + x];
+        base += sm.seg_n[sg];
       }
-      tc::tmem_st_x2(tmem + lane_base + kSfb, wq[0], wq[1]);
-      tc::tmem_wait_st();
     }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
     __syncthreads();
-    tc::tc_fence_after();
-    if (tid == 0)
-      for (int64_t p = 0; p < n_t && p < kStages; ++p)
-        issue_load((int)((cnt + p) % kStages), cnt + (uint32_t)p, req, t_first + p, Nq);
-    float* out = a.scores + (int64_t)qi * a.ld;
-    // read tile `tile`'s accumulator (global tile counter gt) and store its scores
-    auto epilogue = [&](uint32_t gt, int64_t tile) -> bool {
-      const int b = gt & 1;
-      if (!tc::mbar_wait(&sm.mdone[b], (gt >> 1) & 1)) return false;
-      tc::tc_fence_after();
-      uint32_t r[64];
-      const uint32_t col = tmem + lane_base + (b ? kAcc1 : kAcc0);
-      tc::tmem_ld_x16(col + 0, r);
-      tc::tmem_ld_x16(col + 16, r + 16);
-      tc::tmem_ld_x16(col + 32, r + 32);
-      tc::tmem_ld_x16(col + 48, r + 48);
-      tc::tmem_wait_ld();
-      float s = 0.f;
+    const int n_seg = sm.n_seg;
+    int pass_tiles = 0;
+    for (int sg = 0; sg < n_seg; ++sg) pass_tiles += sm.seg_n[sg];
+
+    if (warp == 0) {
+      // ================= producer: one bulk copy per tile =================
+      if (lane == 0) {
+        for (int k = 0; k < pass_tiles; ++k) {
+          const uint32_t u = u_base + (uint32_t)k;
+          const int s = u % kStages;
+          if (u >= (uint32_t)kStages && !wait_or_abort(sm, &sm.stage_empty[s], ((u / kStages) - 1) & 1)) break;
+          tc::mbar_arrive_expect_tx(&sm.full[s], tile_bytes);
+          tc::bulk_g2s(&sm.tiles[s][0], L.page(sm.pgs[k], a.layer) + L.pg_idx_codes, tile_bytes, &sm.full[s]);
+          last_issue[s] = u;
+        }
+      }
+    } else if (warp == 1) {
+      // ================= MMA issuer =================
+      if (lane == 0) {
+        uint32_t u = u_base;
+        bool ok = true;
+        for (int sg = 0; sg < n_seg && ok; ++sg) {
+          ok = wait_or_abort(sm, &sm.q_ready, seg_count & 1);
+          ++seg_count;
+          if (!ok) break;
+          tc::tc_fence_after();
+          tc::tmem_cp_32x128b_x4(tmem + kSfbCol, tc::smem_desc(tc::smem_u32(sm.qsf), 128, 128));
+          for (int k = 0; k < sm.seg_n[sg]; ++k, ++u) {
+            const int s = u % kStages, na = u % kNA;
+            ok = wait_or_abort(sm, &sm.full[s], (u / kStages) & 1) &&
+                 (u < (uint32_t)kNA || wait_or_abort(sm, &sm.acc_empty[na], ((u / kNA) - 1) & 1));
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t a_base = tc::smem_u32(&sm.tiles[s][0]);
+            const uint32_t b_base = tc::smem_u32(sm.qb);
+            const uint32_t sfa_col = tmem + kSfaCol + 4 * na;
+            tc::tmem_cp_32x128b_x4(sfa_col, tc::smem_desc(a_base + sf_off, 128, 128));
+            for (int m = 0; m < n_mma; ++m) {
+              const uint64_t ad = tc::smem_desc(a_base + m * 256, 128, sbo);
+              const uint64_t bd = tc::smem_desc(b_base + m * 256, 128, sbo);
+              const uint32_t id = tc::idesc_mxf4(128, kHeadsN, 2 * m, 2 * m);
+              tc::mma_mxf4(tmem + 64 * na, ad, bd, id, sfa_col | ((uint32_t)(2 * m) << 30),
+                           (tmem + kSfbCol) | ((uint32_t)(2 * m) << 30), m > 0 ? 1u : 0u);
+            }
+            tc::mma_commit(&sm.acc_full[na]);
+            tc::mma_commit(&sm.stage_empty[s]);
+          }
+        }
+      }
+      __syncwarp();
+    } else {
+      // ================= epilogue warps =================
+      const int et = tid - 64;                       // 0 .. kEpiThreads-1
+      const int grp = (warp - 2) >> 2;               // tiles u with u % 2 == grp
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const int key_in_tile = (warp & 3) * 32 + lane;
+      uint32_t u = u_base;
+      bool ok = true;
+      // Every epilogue thread walks all segments and reaches every named
+      // barrier, also after an abort (the work is then skipped), so that no
+      // thread can be left waiting at a barrier another thread has left.
+      for (int sg = 0; sg < n_seg; ++sg) {
+        const int qq = sm.seg_q[sg];
+        const int nt = sm.seg_n[sg];
+        const int64_t t0 = sm.seg_t0[sg], N = sm.seg_N[sg];
+        // -- all tiles of earlier segments are finished: every MMA that read
+        //    the previous query's operands has completed.  Quantise this
+        //    query's index heads: B operand codes and its scale chunk.
+        tc::named_bar_sync(1, kEpiThreads);
+        for (int x = et; x < kHeadsN * CHs; x += kEpiThreads)
+          reinterpret_cast<uint4*>(sm.qb)[x] = make_uint4(0, 0, 0, 0);
+        for (int x = et; x < kSfChunk / 4; x += kEpiThreads)
+          reinterpret_cast<uint32_t*>(sm.qsf)[x] = 0x7F7F7F7Fu;        // scale 1.0 for padding
+        tc::named_bar_sync(1, kEpiThreads);
+        const float* q = a.q_idx + (int64_t)qq * HI * dI;
+        for (int blk = et; blk < HI * CH; blk += kEpiThreads) {
+          const int h = blk / CH, c = blk % CH;
+          const float4* src = reinterpret_cast<const float4*>(q + h * dI + c * 32);
+          float v[32];
 #pragma unroll
-      for (int h = 0; h < kHeadsN; ++h)
-        if (h < HI) s = fmaf(sm.w[h], fmaxf(__uint_as_float(r[h]), 0.f), s);
-      const int64_t j = tile * kTileKeys + warp * 32 + lane;
-      if (j < Nq) out[j] = s;
-      return true;
-    };
-    for (int64_t t = 0; t < n_t; ++t) {
-      const uint32_t gt = cnt + (uint32_t)t;
-      const int s = gt % kStages, b = gt & 1;
-      const bool full_ok = tc::mbar_wait(&sm.full[s], (gt / kStages) & 1);
-      if (full_ok) {
-        if (tid == 0) pending &= ~(1u << s);
-        // key scales of this tile -> TMEM (lane = key mod 32, column = key / 32)
-        uint32_t wd[4];
-        for (int m1 = 0; m1 < 4; ++m1) {
-          const uint8_t* p = &sm.sfs[s][m1 * 32 * CH + lane * CH];
-          uint32_t word = 0;
-          for (int c = 0; c < 4; ++c) word |= (uint32_t)(c < CH ? p[c] : 127) << (8 * c);
-          wd[m1] = word;
+          for (int x = 0; x < 8; ++x) {
+            const float4 f = src[x];
+            v[4 * x] = f.x; v[4 * x + 1] = f.y; v[4 * x + 2] = f.z; v[4 * x + 3] = f.w;
+          }
+          float am = 0.f;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) am = fmaxf(am, fabsf(v[x]));
+          const int e = mx_exponent(am);
+          uint32_t pk[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            pk[x >> 2] |= (uint32_t)e2m1x2_rn(scale_pow2(v[2 * x], e), scale_pow2(v[2 * x + 1], e)) << (8 * (x & 3));
+          *reinterpret_cast<uint4*>(&sm.qb[(h >> 3) * sbo + c * 128 + (h & 7) * 16]) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          sm.qsf[Layout::idx_sf_off(h, c)] = (uint8_t)(e + 127);
         }
-        tc::tmem_st_x4(tmem + lane_base + (b ? kSfa1 : kSfa0), wd[0], wd[1], wd[2], wd[3]);
-        tc::tmem_wait_st();
-      }
-      tc::tc_fence_before();
-      ok = __syncthreads_and(ok && full_ok) != 0;
-      tc::tc_fence_after();
-      if (!ok) break;
-      if (tid == 0) {
-        const uint32_t a_base = tc::smem_u32(&sm.codes[s][0]);
-        const uint32_t b_base = tc::smem_u32(sm.qb);
-        for (int k = 0; k < n_mma; ++k) {
-          const uint64_t ad = tc::smem_desc(a_base + k * 256, 128, sbo);
-          const uint64_t bd = tc::smem_desc(b_base + k * 256, 128, sbo);
-          const uint32_t id = tc::idesc_mxf4(128, kHeadsN, 2 * k, 2 * k);
-          const uint32_t sfa = (tmem + (b ? kSfa1 : kSfa0)) | ((uint32_t)(2 * k) << 30);
-          const uint32_t sfb = (tmem + kSfb) | ((uint32_t)(2 * k) << 30);
-          tc::mma_mxf4(tmem + (b ? kAcc1 : kAcc0), ad, bd, id, sfa, sfb, k > 0 ? 1u : 0u);
+        for (int h = et; h < kHeadsN; h += kEpiThreads) sm.w[h] = h < HI ? a.w[(int64_t)qq * HI + h] : 0.f;
+        tc::fence_proxy_async_smem();
+        tc::named_bar_sync(1, kEpiThreads);
+        if (et == 0) tc::mbar_arrive(&sm.q_ready);
+        float* out = a.scores + (int64_t)qq * a.ld;
+        for (int k = 0; k < nt && ok; ++k) {
+          const uint32_t uk = u + (uint32_t)k;
+          if ((int)(uk & 1) != grp) continue;
+          const int na = uk % kNA;
+          if (!(ok = wait_or_abort(sm, &sm.acc_full[na], (uk / kNA) & 1))) break;
+          tc::tc_fence_after();
+          uint32_t r[64];
+          const uint32_t col = tmem + lane_base + 64 * na;
+          tc::tmem_ld_x16(col + 0, r);
+          tc::tmem_ld_x16(col + 16, r + 16);
+          tc::tmem_ld_x16(col + 32, r + 32);
+          tc::tmem_ld_x16(col + 48, r + 48);
+          tc::tmem_wait_ld();
+          tc::tc_fence_before();
+          tc::mbar_arrive(&sm.acc_empty[na]);
+          // four interleaved partial sums (heads h = 4i + p), combined in a fixed order
+          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+          const float4* w4 = reinterpret_cast<const float4*>(sm.w);
+#pragma unroll
+          for (int h4 = 0; h4 < kHeadsN / 4; ++h4) {
+            if (h4 * 4 < HI) {
+              const float4 wv = w4[h4];
+              p0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), p0);
+              p1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), p1);
+              p2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), p2);
+              p3 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), p3);
+            }
+          }
+          const int64_t j = (t0 + k) * kCsaPerPage + key_in_tile;
+          if (j < N) out[j] = (p0 + p1) + (p2 + p3);
         }
-        tc::mma_commit(&sm.mdone[b]);
-      }
-      if (t > 0) {
-        ok = epilogue(gt - 1, t_first + t - 1);
-        // tile t-1's MMA has completed: its stage can take tile t-1+kStages
-        if (ok && tid == 0 && t - 1 + kStages < n_t)
-          issue_load((int)((gt - 1) % kStages), gt - 1 + kStages, req, t_first + t - 1 + kStages, Nq);
+        u += (uint32_t)nt;
+        if (!ok) sm.abort = 1;
       }
     }
-    if (ok) ok = epilogue(cnt + (uint32_t)n_t - 1, t_first + n_t - 1);
-    cnt += (uint32_t)n_t;
-    g += n_t;
-    tc::tc_fence_before();
-    ok = __syncthreads_and(ok) != 0;
-    tc::tc_fence_after();
+    u_base += (uint32_t)pass_tiles;
+    g += pass_tiles;
+    __syncthreads();
   }
-  if (!ok) {
+  if (tid == 32 && u_base > 0) {
+    // every tcgen05 operation this CTA issued has finished before TMEM is released
+    tc::mma_commit(&sm.drain);
+    tc::mbar_wait(&sm.drain, 0, 200000000ull);
+  }
+  if (sm.abort) {
     if (tid == 0) {
       set_err(L, kErrTimeout, blockIdx.x);
       // let copies already in flight land before the shared memory goes away
       for (int s = 0; s < kStages; ++s)
-        if (pending & (1u << s)) tc::mbar_wait(&sm.full[s], (pend_par >> s) & 1u, 200000000ull);
+        if (last_issue[s] != 0xFFFFFFFFu) tc::mbar_wait(&sm.full[s], (last_issue[s] / kStages) & 1, 200000000ull);
     }
-    __syncthreads();
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Requesting ~100 KB keeps at most two CTAs on an SM, so that their two
-// 256-column TMEM allocations always fit in the SM's 512 columns.
+// More than half of the SM's shared memory: one CTA per SM, so that the
+// 512-column TMEM allocation never waits for another CTA of this kernel.
 size_t index_tc_smem_bytes() {
   const size_t need = sizeof(IdxSmem) + 1024;
-  return need > 100 * 1024 ? need : 100 * 1024;
+  return need > 120 * 1024 ? need : 120 * 1024;
 }
 
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,

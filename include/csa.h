@@ -37,9 +37,9 @@
  *     must stay valid until the work queued on `stream` has finished.
  *   - The library never allocates device memory.  The caller hands one
  *     device buffer (the arena) to csa_cache_init; the library carves the
- *     state cache, the classic-cache block pool, block tables and lengths out
+ *     state cache, the classic-cache page pool, page tables and lengths out
  *     of it.  Host memory owned by the library: the handle and its host-side
- *     block allocator.
+ *     page allocator.
  *   - Every compute call is asynchronous on `stream` (NULL = legacy default
  *     stream).  Argument errors are detected on the host and returned before
  *     anything is launched.  Errors found on the device (request id out of
@@ -69,7 +69,7 @@ typedef struct CUstream_st* csa_stream_t;      /* same type as cudaStream_t     
 typedef enum {
   CSA_OK = 0,
   CSA_ERR_ARG = -1,             /* invalid argument (host-side check)             */
-  CSA_ERR_CAPACITY = -2,        /* block pool or request capacity exhausted       */
+  CSA_ERR_CAPACITY = -2,        /* page pool or request capacity exhausted        */
   CSA_ERR_CUDA = -3,            /* a CUDA runtime call failed                     */
   CSA_ERR_DEVICE_TIMEOUT = -4,  /* a bounded device-side wait gave up             */
   CSA_ERR_DEVICE_BOUNDS = -5    /* a device-side index check failed               */
@@ -99,9 +99,10 @@ typedef enum {
  *   d_I      index dim, one of 32, 64, 96, 128
  *   window   raw-token sliding window; must be 128
  *   max_requests            request slots
- *   max_blocks_per_request  classic-cache blocks a request may hold
- *                           (a block = 128 raw tokens)
- *   pool_blocks             blocks in the shared pool
+ *   max_pages_per_request   pool pages a request may hold
+ *   pool_pages              pages in the shared pool
+ *                           (a page = 4 classic-cache blocks = 512 raw tokens:
+ *                           128 CSA entries and 4 HCA entries per layer)
  *   rope_base               RoPE frequency base (10000)
  * Entry geometry (fixed): CSA m = 4 with windows of 8 tokens overlapping by 4;
  * HCA m = 128, no overlap.
@@ -116,8 +117,8 @@ typedef struct {
   int32_t d_I;
   int32_t window;
   int32_t max_requests;
-  int32_t max_blocks_per_request;
-  int32_t pool_blocks;
+  int32_t max_pages_per_request;
+  int32_t pool_pages;
   float rope_base;
 } csa_cfg;
 
@@ -132,7 +133,7 @@ size_t csa_cache_required_bytes(const csa_cfg* cfg);
  *   b_pos_idx  float [n_csa_layers][8][d_I]  bias of index-key gates
  *   b_pos_hca  float [n_hca_layers][128][D]  bias of KV gates, HCA window slot
  * (NULL allowed when the corresponding layer count is 0).  Synchronous.  All
- * request lengths start at 0 and no blocks are allocated.
+ * request lengths start at 0 and no pages are allocated.
  */
 csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes,
                           const float* b_pos_csa, const float* b_pos_idx,
@@ -142,16 +143,16 @@ csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes,
 void csa_cache_destroy(csa_cache_t* cache);
 
 /*
- * Give request slot `req` room for `capacity_tokens` raw tokens: blocks are
- * taken from the pool (in the allocator's order, so a request's blocks are
- * not contiguous) and its block table is written; every layer's length is
- * reset to 0.  A slot that already holds blocks is released first.
+ * Give request slot `req` room for `capacity_tokens` raw tokens: pages are
+ * taken from the pool (in the allocator's order, so a request's pages are
+ * not contiguous) and its page table is written; every layer's length is
+ * reset to 0.  A slot that already holds pages is released first.
  * Synchronous (device copies on the legacy stream).  CSA_ERR_CAPACITY when
- * the pool or max_blocks_per_request is too small.
+ * the pool or max_pages_per_request is too small.
  */
 csa_status csa_request_alloc(csa_cache_t* cache, int32_t req, int64_t capacity_tokens);
 
-/* Return request slot `req`'s blocks to the pool; its lengths become 0. */
+/* Return request slot `req`'s pages to the pool; its lengths become 0. */
 csa_status csa_request_free(csa_cache_t* cache, int32_t req);
 
 /*
@@ -167,7 +168,7 @@ csa_status csa_request_free(csa_cache_t* cache, int32_t req);
  *   e = sum_t softmax_t(z_t + b_pos[t-4j+4]) * c_t over t in [4j-4, 4j+4), t >= 0
  * is rotated (RoPE at position 4j on the last D_rope dims) and stored as FP8
  * E4M3 (first D-D_rope dims, one fp32 scale amax/448 per row) + BF16 (RoPE
- * dims) in block j/32, slot j%32; the index key pools (idx_cand, idx_gate)
+ * dims) in classic-cache block j/32 (page j/128); the index key pools (idx_cand, idx_gate)
  * the same way without RoPE and is stored as MXFP4 (E2M1 + one E8M0 scale
  * per 32 values).  HCA entry j pools t in [128j, 128j+128) and is rotated at
  * 128j.  Each token's own KV, rotated at its position, is written to the raw

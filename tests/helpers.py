@@ -120,10 +120,10 @@ class Pair:
                 bix.append(bi)
             else:
                 bh.append(b)
-        nb = (capacity + 127) // 128
+        nb = (capacity + 511) // 512
         self.cache = Cache(n_csa=n_csa, n_hca=n_hca, H=wl.H, D=wl.D, D_rope=wl.R,
                            H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=max_req,
-                           max_blocks_per_request=nb, pool_blocks=pool_blocks or nb * max_req,
+                           max_pages_per_request=nb, pool_pages=pool_blocks or nb * max_req,
                            b_pos_csa=np.stack(bkv) if bkv else None,
                            b_pos_idx=np.stack(bix) if bix else None,
                            b_pos_hca=np.stack(bh) if bh else None)

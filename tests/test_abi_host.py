@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol(cuda_lib):
 
 def _cfg(**kw):
     base = dict(n_csa_layers=1, n_hca_layers=1, H=128, D=512, D_rope=64, H_I=64, d_I=128, window=128,
-                max_requests=4, max_blocks_per_request=8192, pool_blocks=4 * 8192, rope_base=10000.0)
+                max_requests=4, max_pages_per_request=2048, pool_pages=4 * 2048, rope_base=10000.0)
     base.update(kw)
     return _lib.CsaCfg(**base)
 
@@ -45,7 +45,7 @@ def test_required_bytes_and_validation(cuda_lib):
     assert nbytes >= 32768 * (32 * 580 + 32 * 68 + 580)
     assert nbytes < 32768 * 24000 + 64 * 2**20
     for bad in (dict(D=500), dict(D_rope=15), dict(window=64), dict(d_I=48), dict(H=0),
-                dict(H_I=65), dict(n_csa_layers=0, n_hca_layers=0), dict(pool_blocks=0)):
+                dict(H_I=65), dict(n_csa_layers=0, n_hca_layers=0), dict(pool_pages=0)):
         assert cuda_lib.csa_cache_required_bytes(ctypes.byref(_cfg(**bad))) == 0, bad
 
 
