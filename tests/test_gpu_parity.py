@@ -356,9 +356,9 @@ def test_device_errors_are_reported_not_trapped():
         pair.cache.check_device_error()
     assert e.value.status == -5
     pair.cache.check_device_error()          # the word was cleared
-    # capacity: 256 tokens allowed, appending 300 is refused on the device
-    toks = pair.gen_tokens(0, 0, 0, 300)
-    pair.append(0, [0], {0: toks}, 300, oracle=False)
+    # capacity: one 512-token page allowed, appending 600 is refused on the device
+    toks = pair.gen_tokens(0, 0, 0, 600)
+    pair.append(0, [0], {0: toks}, 600, oracle=False)
     with pytest.raises(CsaError) as e:
         pair.cache.check_device_error()
     assert e.value.status == -2
