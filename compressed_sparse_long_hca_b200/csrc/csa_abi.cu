@@ -250,9 +250,9 @@ csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, cons
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
   const int sms = sm_count();
   if (sms <= 0) return fail(CSA_ERR_CUDA, "cannot query the SM count");
-  // One persistent CTA per SM for either variant; the per-key arithmetic
+  // Two persistent CTAs per SM for either variant; the per-key arithmetic
   // does not depend on the grid.
-  cudaError_t e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, sms,
+  cudaError_t e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, 2 * sms,
                                        (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "index launch");
   return CSA_OK;

@@ -11,16 +11,16 @@
 // streamed once from HBM.  The cache stores the index keys of every 512-token
 // page as one ready-made operand tile (codes in the no-swizzle K-major
 // core-matrix order, scales in the 32 x 128-bit order of tcgen05.cp), so a
-// 128-key tile is one bulk copy.  One persistent CTA per SM owns a contiguous
-// range of tiles of the flattened (query, tile) list and runs three roles:
+// 128-key tile is one bulk copy.  Two persistent CTAs per SM (their tcgen05
+// issue latencies overlap) each own a contiguous range of tiles of the
+// flattened (query, tile) list and run three roles:
 //   * producer (warp 0): one bulk async copy per tile into a ring of
 //     shared-memory stages;
 //   * MMA (warp 1): one thread copies the tile's key scales into TMEM
 //     (tcgen05.cp) and issues the block-scaled MMA
 //     D[128 keys x 64 heads] = K^ Q^T (kind::mxf4, M=128, N=64, K=64 per
 //     instruction) into one of four TMEM accumulators;
-//   * epilogue (warps 2-9, two groups of four taking alternate tiles): read a
-//     finished accumulator (one TMEM lane = one key, 64 columns = its 64 head
+//   * epilogue (warps 2-5): read a finished accumulator (one TMEM lane = one key, 64 columns = its 64 head
 //     dot products) and reduce sum_h w_h max(0, d_h) in a fixed order.  At a
 //     query boundary they quantise the next query's index heads to MXFP4 (the
 //     B operand and its scale chunk).
@@ -36,17 +36,18 @@ namespace csa {
 namespace {
 
 constexpr int kStages = 8;             // shared-memory stages of key tiles
-constexpr int kNA = 4;                 // TMEM accumulators (and key-scale buffers)
-constexpr int kEpiGroups = 2;
-constexpr int kEpiThreads = 128 * kEpiGroups;
-constexpr int kThreads = 64 + kEpiThreads;   // warp 0 producer, warp 1 MMA, warps 2.. epilogue
+constexpr int kNA = 3;                 // TMEM accumulators (and key-scale buffers)
+constexpr int kEpiThreads = 128;
+constexpr int kThreads = 64 + kEpiThreads;   // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+constexpr int kCtasPerSm = 2;          // two CTAs per SM overlap their issue latencies
 constexpr int kHeadsN = 64;            // MMA N (index heads, zero padded)
 constexpr int kMaxCh = 4;              // d_I / 32 <= 4
 constexpr int kTileBytes = kCsaPerPage * kMaxCh * 16 + kSfChunk;   // codes + scale chunk
 constexpr int kPassTiles = 512;        // tiles per pass (page-table window in smem)
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfaCol = 256;      // + 4 * accumulator index
-constexpr uint32_t kSfbCol = 272;
+constexpr int kMaxSeg = 64;            // queries per pass
+constexpr uint32_t kTmemCols = 256;    // per CTA; two CTAs fill the SM's 512 columns
+constexpr uint32_t kSfaCol = 192;      // + 4 * accumulator index
+constexpr uint32_t kSfbCol = 204;
 
 struct IdxSmem {
   uint8_t tiles[kStages][kTileBytes];                // one page's index tile per stage
@@ -55,10 +56,10 @@ struct IdxSmem {
   alignas(16) float w[kHeadsN];
   int32_t pgs[kPassTiles];                           // pool page of every tile of the pass
   // segments of the pass: one per query touched
-  int32_t seg_q[kPassTiles];
-  int32_t seg_n[kPassTiles];
-  int64_t seg_t0[kPassTiles];
-  int64_t seg_N[kPassTiles];
+  int32_t seg_q[kMaxSeg];
+  int32_t seg_n[kMaxSeg];
+  int64_t seg_t0[kMaxSeg];
+  int64_t seg_N[kMaxSeg];
   int32_t n_seg;
   uint64_t full[kStages], stage_empty[kStages];
   uint64_t acc_full[kNA], acc_empty[kNA];
@@ -106,7 +107,7 @@ __device__ __forceinline__ bool wait_or_abort(IdxSmem& sm, uint64_t* bar, uint32
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout& L = a.L;
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.stage_empty[s], 1); }
-    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], 128); }
+    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], kEpiThreads); }
     tc::mbar_init(&sm.q_ready, 1);
     tc::mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
     if (tid == 0) {
       int ns = 0;
       int64_t gg = g, used = 0;
-      while (gg < g1 && used < kPassTiles) {
+      while (gg < g1 && used < kPassTiles && ns < kMaxSeg) {
         int64_t N;
         int req;
         const int64_t nt = query_tiles(a, qi, &N, &req);
@@ -204,36 +205,46 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
 
     if (warp == 0) {
       // ================= producer: one bulk copy per tile =================
-      if (lane == 0) {
-        for (int k = 0; k < pass_tiles; ++k) {
-          const uint32_t u = u_base + (uint32_t)k;
-          const int s = u % kStages;
-          if (u >= (uint32_t)kStages && !wait_or_abort(sm, &sm.stage_empty[s], ((u / kStages) - 1) & 1)) break;
+      // The whole warp walks the loop; one elected lane issues.
+      for (int k = 0; k < pass_tiles; ++k) {
+        const uint32_t u = u_base + (uint32_t)k;
+        const int s = u % kStages;
+        const bool ok = u < (uint32_t)kStages || wait_or_abort(sm, &sm.stage_empty[s], ((u / kStages) - 1) & 1);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const char* src = L.page(sm.pgs[k], a.layer) + L.pg_idx_codes;
+        if (tc::elect_one()) {
           tc::mbar_arrive_expect_tx(&sm.full[s], tile_bytes);
-          tc::bulk_g2s(&sm.tiles[s][0], L.page(sm.pgs[k], a.layer) + L.pg_idx_codes, tile_bytes, &sm.full[s]);
-          last_issue[s] = u;
+          tc::bulk_g2s(&sm.tiles[s][0], src, tile_bytes, &sm.full[s]);
         }
+        __syncwarp();
+        last_issue[s] = u;
       }
     } else if (warp == 1) {
       // ================= MMA issuer =================
-      if (lane == 0) {
-        uint32_t u = u_base;
-        bool ok = true;
-        for (int sg = 0; sg < n_seg && ok; ++sg) {
-          ok = wait_or_abort(sm, &sm.q_ready, seg_count & 1);
-          ++seg_count;
+      // The whole warp walks the loop; one elected lane issues the tcgen05
+      // operations, whose operands are warp-uniform.
+      uint32_t u = u_base;
+      bool ok = true;
+      for (int sg = 0; sg < n_seg && ok; ++sg) {
+        ok = wait_or_abort(sm, &sm.q_ready, seg_count & 1);
+        ++seg_count;
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc::tc_fence_after();
+        if (tc::elect_one()) tc::tmem_cp_32x128b_x4(tmem + kSfbCol, tc::smem_desc(tc::smem_u32(sm.qsf), 128, 128));
+        __syncwarp();
+        const int nt = sm.seg_n[sg];
+        for (int k = 0; k < nt; ++k, ++u) {
+          const int s = u % kStages, na = u % kNA;
+          ok = wait_or_abort(sm, &sm.full[s], (u / kStages) & 1) &&
+               (u < (uint32_t)kNA || wait_or_abort(sm, &sm.acc_empty[na], ((u / kNA) - 1) & 1));
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc::tc_fence_after();
-          tc::tmem_cp_32x128b_x4(tmem + kSfbCol, tc::smem_desc(tc::smem_u32(sm.qsf), 128, 128));
-          for (int k = 0; k < sm.seg_n[sg]; ++k, ++u) {
-            const int s = u % kStages, na = u % kNA;
-            ok = wait_or_abort(sm, &sm.full[s], (u / kStages) & 1) &&
-                 (u < (uint32_t)kNA || wait_or_abort(sm, &sm.acc_empty[na], ((u / kNA) - 1) & 1));
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t a_base = tc::smem_u32(&sm.tiles[s][0]);
-            const uint32_t b_base = tc::smem_u32(sm.qb);
-            const uint32_t sfa_col = tmem + kSfaCol + 4 * na;
+          const uint32_t a_base = tc::smem_u32(&sm.tiles[s][0]);
+          const uint32_t b_base = tc::smem_u32(sm.qb);
+          const uint32_t sfa_col = tmem + kSfaCol + 4 * na;
+          if (tc::elect_one()) {
             tc::tmem_cp_32x128b_x4(sfa_col, tc::smem_desc(a_base + sf_off, 128, 128));
             for (int m = 0; m < n_mma; ++m) {
               const uint64_t ad = tc::smem_desc(a_base + m * 256, 128, sbo);
@@ -245,13 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
             tc::mma_commit(&sm.acc_full[na]);
             tc::mma_commit(&sm.stage_empty[s]);
           }
+          __syncwarp();
         }
       }
-      __syncwarp();
     } else {
       // ================= epilogue warps =================
       const int et = tid - 64;                       // 0 .. kEpiThreads-1
-      const int grp = (warp - 2) >> 2;               // tiles u with u % 2 == grp
       const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
       const int key_in_tile = (warp & 3) * 32 + lane;
       uint32_t u = u_base;
@@ -301,7 +311,6 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
         float* out = a.scores + (int64_t)qq * a.ld;
         for (int k = 0; k < nt && ok; ++k) {
           const uint32_t uk = u + (uint32_t)k;
-          if ((int)(uk & 1) != grp) continue;
           const int na = uk % kNA;
           if (!(ok = wait_or_abort(sm, &sm.acc_full[na], (uk / kNA) & 1))) break;
           tc::tc_fence_after();
@@ -338,9 +347,10 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
     g += pass_tiles;
     __syncthreads();
   }
-  if (tid == 32 && u_base > 0) {
+  if (warp == 1 && u_base > 0) {
     // every tcgen05 operation this CTA issued has finished before TMEM is released
-    tc::mma_commit(&sm.drain);
+    if (tc::elect_one()) tc::mma_commit(&sm.drain);
+    __syncwarp();
     tc::mbar_wait(&sm.drain, 0, 200000000ull);
   }
   if (sm.abort) {
@@ -356,11 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_tc_kernel(IndexTcArgs a) {
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// More than half of the SM's shared memory: one CTA per SM, so that the
-// 512-column TMEM allocation never waits for another CTA of this kernel.
+// Sized so that exactly two CTAs share an SM: their two 256-column TMEM
+// allocations then always fit the SM's 512 columns.
 size_t index_tc_smem_bytes() {
   const size_t need = sizeof(IdxSmem) + 1024;
-  return need > 120 * 1024 ? need : 120 * 1024;
+  return need > 80 * 1024 ? need : 80 * 1024;
 }
 
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
