@@ -22,10 +22,10 @@ cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* re
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
                             cudaStream_t st);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
-                        int32_t* out, int32_t* err, cudaStream_t st);
-cudaError_t launch_attn_simt(const Layout& L, int layer, int n, const int32_t* req_ids,
-                             const uint16_t* q, const int32_t* topk, int k, const float* sink,
-                             float scale, uint16_t* out, int heads_per_cta, cudaStream_t st);
+                        int32_t* out, int32_t* err, int cluster, cudaStream_t st);
+cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
+                           const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
+                           cudaStream_t st);
 }  // namespace csa
 
 using csa::Layout;
@@ -260,12 +260,16 @@ csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, cons
 
 csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int32_t n, int32_t k,
                     int32_t* idx_out, csa_variant variant, csa_stream_t stream) {
-  if (n < 0 || n > 2147483647) return fail(CSA_ERR_ARG, "bad n");
+  if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
   if (n == 0) return CSA_OK;
   if (!scores || !n_valid || !idx_out) return fail(CSA_ERR_ARG, "NULL argument");
   if (k < 1 || ld < 1) return fail(CSA_ERR_ARG, "k and ld must be >= 1");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
-  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, (cudaStream_t)stream);
+  // One thread-block cluster per query: 8 CTAs for an under-fed GPU, 4 for a
+  // well-fed one.  The selection is exact, so both return identical indices.
+  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 37);
+  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, low ? 8 : 4,
+                                   (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "topk launch");
   return CSA_OK;
 }
@@ -282,11 +286,13 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
   if (!is_csa && topk_idx) return fail(CSA_ERR_ARG, "HCA layer takes topk_idx == NULL");
   if (!(scale > 0.f)) return fail(CSA_ERR_ARG, "scale must be > 0");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
+  if (is_csa && k > 8192) return fail(CSA_ERR_ARG, "k must be <= 8192");
+  // Heads per CTA: 32 for a well-fed GPU, 16 for an under-fed one (twice the
+  // CTAs per query).  Every per-head operation is independent of the grouping.
   const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 16);
-  int hpc = low ? 4 : 8;
-  while (c->L.H % hpc) hpc >>= 1;
-  cudaError_t e = csa::launch_attn_simt(c->L, layer, n, req_ids, q, topk_idx, is_csa ? k : 0, sink,
-                                        scale, out, hpc, (cudaStream_t)stream);
+  const int G = (low || c->L.H <= 16) ? 16 : 32;
+  cudaError_t e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, is_csa ? k : 0, sink, scale,
+                                      out, G, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
 }

@@ -5,15 +5,32 @@
 // entries.  Selection rule (fixed here): the k largest scores, equal scores
 // going to the lower index, -0.0 == +0.0, output ascending, -1 padding.
 //
-// Method: an exact radix select on order-preserving 32-bit keys.  Four 8-bit
-// passes of shared-memory histograms narrow the k-th largest key to one value
-// T and give the number of ties at T that still fit; a final ordered pass
-// emits every index with key > T and the first `ties` indices with key == T,
-// in ascending order, through block-wide prefix sums.  Integer histograms and
-// ordered prefix sums make the result independent of thread scheduling.
+// Method: an exact radix select on order-preserving 32-bit keys, run by one
+// thread-block cluster per query.  Each CTA of the cluster owns a contiguous
+// slice of the query's scores (kept in shared memory when it fits).  Three
+// passes (11, 11 and 10 bits) build shared-memory histograms of the keys
+// that still match the prefix found so far; the cluster adds its histograms
+// through distributed shared memory and every CTA reads off the same digit.
+// The passes end with the k-th largest key T and the number of ties at T
+// that still fit.  The output pass exchanges per-CTA counts, so that each
+// CTA writes its selected indices (all keys > T, then ties at T in index
+// order) at the right place of the ascending list.  Integer histograms and
+// ordered prefix sums make the result independent of thread scheduling and
+// of the cluster's launch shape; the cluster barriers are hardware barriers,
+// no thread spins on memory.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace csa {
+
+namespace {
+
+constexpr int kTopkThreads = 1024;
+constexpr int kBins = 2048;                // 11-bit digits
+constexpr int kMaxCluster = 8;
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   const uint32_t b = __float_as_uint(s + 0.0f);       // -0.0 -> +0.0
@@ -27,11 +44,13 @@ struct TopkArgs {
   int n;
   int k;
   int32_t* out;
-  int32_t* err;   // device error word (may be null)
+  int32_t* err;          // device error word (may be null)
+  int cache_keys;        // slices fit in shared memory
+  int64_t slice_cap;     // keys per CTA slice buffer
 };
 
-// Exclusive block prefix sum of `v` (blockDim.x == 1024); also returns the total.
-__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int& total) {
+// Exclusive block-wide prefix sum over kTopkThreads threads; returns the total.
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int x = v;
   for (int o = 1; o < 32; o <<= 1) {
@@ -46,81 +65,174 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int& total) {
       const int y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    wsum[lane] = s;   // inclusive over warps
+    wsum[lane] = s;
   }
   __syncthreads();
-  total = wsum[31];
+  *total = wsum[31];
   const int before = (w > 0 ? wsum[w - 1] : 0) + x - v;
   __syncthreads();
   return before;
 }
 
-__global__ void __launch_bounds__(1024) topk_radix_kernel(TopkArgs a) {
-  __shared__ int hist[256];
-  __shared__ int wsum[32];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_remaining;
-  const int i = blockIdx.x;
+struct TopkShared {
+  int hist[kBins];          // this CTA's histogram
+  int slice_sum[kBins];     // reduce-scatter: summed bins owned by this CTA
+  int full[kBins];          // the cluster's summed histogram
+  int wsum[32];
+  int cnt[2];               // this CTA's (count > T, count == T)
+  uint32_t digit;
+  int remaining;
+};
+
+}  // namespace
+
+template <int C>
+__global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int i = blockIdx.y;
+  const int tid = threadIdx.x;
   const float* s = a.scores + (int64_t)i * a.ld;
   int32_t* out = a.out + (int64_t)i * a.k;
   int64_t N = a.n_valid[i];
   if (N < 0 || N > a.ld) {
-    if (threadIdx.x == 0 && a.err) {
+    if (rank == 0 && tid == 0 && a.err) {
       if (atomicCAS(a.err, 0, (int32_t)kErrLd) == 0) a.err[1] = i;
     }
     N = 0;
   }
   const int k = a.k;
-  if (N <= k) {
-    for (int64_t j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < N ? (int32_t)j : -1;
-    return;
+  if (N <= k) {   // every entry is selected: indices in order, then -1
+    for (int64_t j = (int64_t)rank * kTopkThreads + tid; j < k; j += (int64_t)C * kTopkThreads)
+      out[j] = j < N ? (int32_t)j : -1;
+    return;       // uniform for the whole cluster (N is the cluster's)
   }
-  if (threadIdx.x == 0) { s_prefix = 0; s_mask = 0; s_remaining = k; }
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[b] = 0;
+  const int64_t chunk = (N + C - 1) / C;
+  const int64_t lo = (int64_t)rank * chunk;
+  const int64_t hi = lo + chunk < N ? lo + chunk : N;
+  const int64_t len = hi > lo ? hi - lo : 0;
+  auto key_at = [&](int64_t x) -> uint32_t { return a.cache_keys ? keys[x] : order_key(s[lo + x]); };
+  if (a.cache_keys)
+    for (int64_t x = tid; x < len; x += kTopkThreads) keys[x] = order_key(s[lo + x]);
+  if (tid == 0) { sh.digit = 0; sh.remaining = k; }
+  uint32_t prefix = 0;
+  int remaining = k;
+  const int shifts[3] = {21, 10, 0};
+  const int widths[3] = {11, 11, 10};
+  for (int p = 0; p < 3; ++p) {
+    const int shift = shifts[p], width = widths[p];
+    const uint32_t mask = (1u << width) - 1;
+    for (int b = tid; b < kBins; b += kTopkThreads) sh.hist[b] = 0;
     __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int64_t j = threadIdx.x; j < N; j += blockDim.x) {
-      const uint32_t key = order_key(s[j]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 0xFF], 1);
+    for (int64_t x = tid; x < len; x += kTopkThreads) {
+      const uint32_t key = key_at(x);
+      if (p == 0 || (key >> (shift + width)) == prefix) atomicAdd(&sh.hist[(key >> shift) & mask], 1);
     }
+    // cluster reduce-scatter: CTA r sums bins [r*kBins/C, (r+1)*kBins/C)
+    cluster.sync();
+    constexpr int per = kBins / C;
+    for (int b = tid; b < per; b += kTopkThreads) {
+      int t = 0;
+      for (int r = 0; r < C; ++r) t += cluster.map_shared_rank(&sh.hist[0], r)[rank * per + b];
+      sh.slice_sum[b] = t;
+    }
+    cluster.sync();
+    for (int b = tid; b < kBins; b += kTopkThreads)
+      sh.full[b] = cluster.map_shared_rank(&sh.slice_sum[0], b / per)[b % per];
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int rem = s_remaining;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (hist[d] >= rem) break;
-        rem -= hist[d];
+    // digit d: the largest d with (count of digits > d) < remaining <= (count of digits >= d)
+    {
+      // suffix sums over bins, 2 bins per thread (kBins = 2 * kTopkThreads)
+      const int b0 = kBins - 2 - 2 * tid;        // thread 0 owns the top bins
+      const int c1 = sh.full[b0 + 1], c0 = sh.full[b0];
+      int tot;
+      const int before = block_excl_scan(c1 + c0, sh.wsum, &tot);   // counts of bins above b0 + 1
+      if (before < remaining && before + c1 >= remaining) { sh.digit = (uint32_t)(b0 + 1); sh.remaining = remaining - before; }
+      else if (before + c1 < remaining && before + c1 + c0 >= remaining) {
+        sh.digit = (uint32_t)b0;
+        sh.remaining = remaining - before - c1;
       }
-      s_remaining = rem;
-      s_prefix = prefix | ((uint32_t)d << shift);
-      s_mask = mask | (0xFFu << shift);
+      __syncthreads();
     }
-    __syncthreads();
+    prefix = (prefix << width) | sh.digit;
+    remaining = sh.remaining;
+    // the histogram buffers are read remotely until every CTA has its copy
+    cluster.sync();
   }
-  const uint32_t T = s_prefix;
-  const int ties = s_remaining;        // indices with key == T still to take
-  int sel_base = 0, eq_base = 0;
-  for (int64_t j0 = 0; j0 < N; j0 += blockDim.x) {
-    const int64_t j = j0 + threadIdx.x;
-    uint32_t key = 0;
-    if (j < N) key = order_key(s[j]);
-    const int eq = (j < N && key == T) ? 1 : 0;
-    int eq_total;
-    const int eq_before = block_excl_scan(eq, wsum, eq_total);
-    const int take = (j < N) && (key > T || (eq && eq_base + eq_before < ties)) ? 1 : 0;
-    int sel_total;
-    const int pos = block_excl_scan(take, wsum, sel_total);
-    if (take) out[sel_base + pos] = (int32_t)j;
-    sel_base += sel_total;
-    eq_base += eq_total;
+  const uint32_t T = prefix;        // the k-th largest key
+  const int ties_needed = remaining;
+  // ---- output: per-thread contiguous sub-slices in index order
+  const int64_t per_thr = (len + kTopkThreads - 1) / kTopkThreads;
+  const int64_t t_lo = tid * per_thr < len ? tid * per_thr : len;
+  const int64_t t_hi = t_lo + per_thr < len ? t_lo + per_thr : len;
+  int gt = 0, eq = 0;
+  for (int64_t x = t_lo; x < t_hi; ++x) {
+    const uint32_t key = key_at(x);
+    gt += key > T;
+    eq += key == T;
   }
+  int gt_tot, eq_tot;
+  const int gt_before = block_excl_scan(gt, sh.wsum, &gt_tot);
+  const int eq_before = block_excl_scan(eq, sh.wsum, &eq_tot);
+  if (tid == 0) { sh.cnt[0] = gt_tot; sh.cnt[1] = eq_tot; }
+  cluster.sync();
+  int sel_before = 0, ties_before = 0, take_cta = 0;
+  {
+    int tb = 0;
+    for (int r = 0; r < C; ++r) {
+      const int* c = cluster.map_shared_rank(&sh.cnt[0], r);
+      const int g = c[0], e = c[1];
+      int take = ties_needed - tb;
+      take = take < 0 ? 0 : (take > e ? e : take);
+      if (r < rank) { sel_before += g + take; ties_before += e; }
+      if (r == rank) take_cta = take;
+      tb += e;
+    }
+  }
+  // ties this thread may take: those among the CTA's first take_cta ties
+  int my_take_ties = take_cta - eq_before;
+  my_take_ties = my_take_ties < 0 ? 0 : (my_take_ties > eq ? eq : my_take_ties);
+  int tot_sel;
+  const int pos0 = block_excl_scan(gt + my_take_ties, sh.wsum, &tot_sel);
+  int pos = sel_before + pos0;
+  int ties_left = my_take_ties;
+  for (int64_t x = t_lo; x < t_hi; ++x) {
+    const uint32_t key = key_at(x);
+    if (key > T || (key == T && ties_left > 0)) {
+      if (key == T) --ties_left;
+      out[pos++] = (int32_t)(lo + x);
+    }
+  }
+  (void)ties_before;
+  // no CTA may leave while others still read its shared memory
+  cluster.sync();
 }
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
-                        int32_t* out, int32_t* err, cudaStream_t st) {
-  TopkArgs a{scores, ld, n_valid, n, k, out, err};
-  topk_radix_kernel<<<n, 1024, 0, st>>>(a);
+                        int32_t* out, int32_t* err, int cluster, cudaStream_t st) {
+  if (n > 65535) return cudaErrorInvalidValue;
+  const int64_t slice = (ld + cluster - 1) / cluster;
+  const size_t base = sizeof(TopkShared);
+  const size_t cap = 200 * 1024;
+  const bool cache = base + (size_t)slice * 4 <= cap;
+  const size_t sm = cache ? base + (size_t)slice * 4 : base;
+  TopkArgs a{scores, ld, n_valid, n, k, out, err, cache ? 1 : 0, slice};
+  dim3 grid(cluster, n);
+  cudaError_t e;
+  if (cluster == 8) {
+    e = cudaFuncSetAttribute(topk_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+    if (e != cudaSuccess) return e;
+    topk_cluster_kernel<8><<<grid, kTopkThreads, sm, st>>>(a);
+  } else if (cluster == 4) {
+    e = cudaFuncSetAttribute(topk_cluster_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+    if (e != cudaSuccess) return e;
+    topk_cluster_kernel<4><<<grid, kTopkThreads, sm, st>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 
