@@ -58,7 +58,7 @@ struct AttnTcArgs {
 
 struct AttnSmemLayout {
   int Dp;           // head dim padded to a multiple of 128
-  int64_t tile, qs, pt, stage, sel, stats, bars, total;
+  int64_t tile, qs, pt, stage, sel, rsc, stats, bars, total;
 };
 
 __host__ __device__ inline AttnSmemLayout attn_smem_layout(int D, int G, int k) {
@@ -67,9 +67,10 @@ __host__ __device__ inline AttnSmemLayout attn_smem_layout(int D, int G, int k) 
   int64_t o = 0;
   s.tile = o;  o += (int64_t)kTileRows * s.Dp * 2;           // BF16 rows, core-matrix order
   s.qs = o;    o += (int64_t)G * s.Dp * 2;                   // BF16 query heads
-  s.pt = o;    o += (int64_t)kTileRows * G * 2;              // BF16 P^T (MN-major)
+  s.pt = o;    o += (int64_t)kTileRows * G * 2 * 2;          // BF16 P^T and (P*scale)^T (MN-major)
   s.stage = o; o += (int64_t)kTileRows * (G + 1) * 4;        // fp32 logits / p for reductions
   s.sel = o;   o += (int64_t)(k > 0 ? k : 1) * 4;            // compacted selected entries
+  s.rsc = o;   o += (int64_t)kTileRows * 4;                  // per-row FP8 scale of the tile
   o = (o + 15) / 16 * 16;
   s.stats = o; o += (int64_t)(6 * 32 + 4 * 32) * 4;          // m, l, corr, mt, den, cm; partials [4][32]
   o = (o + 15) / 16 * 16;
@@ -93,6 +94,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
   uint8_t* pt = sm + S.pt;
   float* stage = reinterpret_cast<float*>(sm + S.stage);
   int32_t* sel = reinterpret_cast<int32_t*>(sm + S.sel);
+  float* rsc = reinterpret_cast<float*>(sm + S.rsc);
+  uint8_t* ptm = pt + kTileRows * G * 2;                   // (P * row scale)^T for the FP8 dims
   float* m_run = reinterpret_cast<float*>(sm + S.stats);
   float* l_run = m_run + 32;
   float* corr = l_run + 32;
@@ -189,8 +192,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t col_s = 0, col_o = 32;
+  // TMEM columns: S_fp8 (logit part over the FP8 dims, before the row
+  // scale), S_bf16 (RoPE dims), then per 128-dim chunk of the output an
+  // accumulator for the FP8 dims (B = (P*scale)^T) and, where the chunk
+  // holds RoPE dims, one for those (B = P^T).
+  const uint32_t col_s = 0, col_sr = 32, col_o = 64;
   const int n_dc = Dp / 128;
+  const int dmain = D - R;
+  const int dc_r0 = dmain / 128;                            // first chunk holding RoPE dims
   const int64_t total = n_sel + n_win;
   const int n_tiles = (int)((total + kTileRows - 1) / kTileRows);
   const char* st_ring = L.state(req, a.layer);
@@ -224,6 +233,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
       }
       const int nch = Dp / 8;
       const int c0 = (tid >> 7) * (nch / 2), c1 = c0 + nch / 2;
+      if (tid < kTileRows) rsc[r] = sc;
       uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
       for (int c = c0; c < c1; ++c) {
         uint4 o = make_uint4(0, 0, 0, 0);
@@ -236,7 +246,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
               const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
               const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
               const float2 f = __half22float2(__half2(h2));
-              pk[e] = (uint32_t)bf16_rn(f.x * sc) | ((uint32_t)bf16_rn(f.y * sc) << 16);
+              pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);   // exact
             }
             o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           } else {
@@ -254,9 +264,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     if (warp == 0) {
       if (tc::elect_one()) {
         const uint32_t ta = tc::smem_u32(tile), tq = tc::smem_u32(qs);
-        for (int ks = 0; ks < Dp / 16; ++ks)
-          tc::mma_bf16(tmem + col_s, tc::smem_desc(ta + ks * 256, 128, sbo_rows),
-                       tc::smem_desc(tq + ks * 256, 128, sbo_rows), id_qk, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < Dp / 16; ++ks) {
+          const bool main = 16 * ks < dmain;                  // (D - R) is a multiple of 16
+          const int k0 = main ? 0 : dmain / 16;
+          tc::mma_bf16(tmem + (main ? col_s : col_sr), tc::smem_desc(ta + ks * 256, 128, sbo_rows),
+                       tc::smem_desc(tq + ks * 256, 128, sbo_rows), id_qk, ks > k0 ? 1u : 0u);
+        }
         tc::mma_commit(bar_qk);
       }
       __syncwarp();
@@ -268,12 +281,19 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     if (warp < 4) {
       ok = tc::mbar_wait(bar_qk, tt & 1);
       tc::tc_fence_after();
-      uint32_t sv[32];
+      uint32_t sv[32], sr[32];
       tc::tmem_ld_x16(tmem + lane_base + col_s, sv);
-      if (G > 16) tc::tmem_ld_x16(tmem + lane_base + col_s + 16, sv + 16);
+      tc::tmem_ld_x16(tmem + lane_base + col_sr, sr);
+      if (G > 16) {
+        tc::tmem_ld_x16(tmem + lane_base + col_s + 16, sv + 16);
+        tc::tmem_ld_x16(tmem + lane_base + col_sr + 16, sr + 16);
+      }
       tc::tmem_wait_ld();
+      const float rs = rsc[r];
       for (int h = 0; h < 32; ++h) {
-        u[h] = (h < G && rr < total) ? __uint_as_float(sv[h]) * a.scale : -INFINITY;
+        u[h] = (h < G && rr < total)
+                   ? fmaf(rs, __uint_as_float(sv[h]), __uint_as_float(sr[h])) * a.scale
+                   : -INFINITY;
         if (h < G) stage[r * (G + 1) + h] = u[h];
       }
     }
@@ -304,7 +324,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     __syncthreads();
     // -- rescale the accumulator columns of heads whose running max moved
     if (s_flag && warp < 4) {
-      for (int dc = 0; dc < n_dc; ++dc) {
+      for (int dc = 0; dc < n_dc + (n_dc - dc_r0); ++dc) {
         for (int hb = 0; hb < G; hb += 16) {
           uint32_t ov[16];
           const uint32_t addr = tmem + lane_base + col_o + dc * 32 + hb;
@@ -318,8 +338,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     }
     // -- p = exp(u - m_run): P^T (BF16, MN-major) for PV, fp32 copy for the sums
     if (warp < 4) {
+      const float rs = rsc[r];
       for (int hg = 0; hg < G / 8; ++hg) {
-        uint32_t pk[4];
+        uint32_t pk[4], pm[4];
         for (int e = 0; e < 8; e += 2) {
           const int h = hg * 8 + e;
           const float p0 = expf(u[h] - m_run[h]);
@@ -327,9 +348,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
           stage[r * (G + 1) + h] = p0;
           stage[r * (G + 1) + h + 1] = p1;
           pk[e >> 1] = (uint32_t)bf16_rn(p0) | ((uint32_t)bf16_rn(p1) << 16);
+          pm[e >> 1] = (uint32_t)bf16_rn(p0 * rs) | ((uint32_t)bf16_rn(p1 * rs) << 16);
         }
         *reinterpret_cast<uint4*>(pt + hg * 2048 + (r >> 3) * 128 + (r & 7) * 16) =
             make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(ptm + hg * 2048 + (r >> 3) * 128 + (r & 7) * 16) =
+            make_uint4(pm[0], pm[1], pm[2], pm[3]);
       }
     }
     tc::fence_proxy_async_smem();
@@ -339,11 +363,16 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     // -- PV: O^T[dims x heads] += V^T P^T
     if (warp == 0) {
       if (tc::elect_one()) {
-        const uint32_t ta = tc::smem_u32(tile), tp = tc::smem_u32(pt);
-        for (int dc = 0; dc < n_dc; ++dc)
+        const uint32_t ta = tc::smem_u32(tile), tp = tc::smem_u32(pt), tpm = tc::smem_u32(ptm);
+        // FP8 dims: chunks 0 .. n_dc-1 with B = (P*scale)^T; RoPE dims: chunks
+        // dc_r0 .. n_dc-1 again with B = P^T, into their own accumulators
+        for (int x = 0; x < n_dc + (n_dc - dc_r0); ++x) {
+          const bool main = x < n_dc;
+          const int dc = main ? x : dc_r0 + (x - n_dc);
           for (int ks = 0; ks < kTileRows / 16; ++ks)
-            tc::mma_bf16(tmem + col_o + dc * 32, tc::smem_desc(ta + dc * 16 * 128 + ks * 2 * sbo_rows, sbo_rows, 128),
-                         tc::smem_desc(tp + ks * 256, 128, 2048), id_pv, (tt > 0 || ks > 0) ? 1u : 0u);
+            tc::mma_bf16(tmem + col_o + x * 32, tc::smem_desc(ta + dc * 16 * 128 + ks * 2 * sbo_rows, sbo_rows, 128),
+                         tc::smem_desc((main ? tpm : tp) + ks * 256, 128, 2048), id_pv, (tt > 0 || ks > 0) ? 1u : 0u);
+        }
         tc::mma_commit(bar_pv);
       }
       __syncwarp();
@@ -374,9 +403,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     if (warp < 4) {
       for (int dc = 0; dc < n_dc; ++dc) {
         const int d = dc * 128 + tid;
+        // FP8 dims read the scaled accumulator, RoPE dims their own
+        const int x = d < dmain ? dc : n_dc + (dc - dc_r0);
         for (int hb = 0; hb < G; hb += 16) {
           uint32_t ov[16];
-          tc::tmem_ld_x16(tmem + lane_base + col_o + dc * 32 + hb, ov);
+          tc::tmem_ld_x16(tmem + lane_base + col_o + x * 32 + hb, ov);
           tc::tmem_wait_ld();
           for (int e = 0; e < 16; ++e) {
             const int h = h0 + hb + e;
