@@ -403,17 +403,20 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     if (warp < 4) {
       for (int dc = 0; dc < n_dc; ++dc) {
         const int d = dc * 128 + tid;
-        // FP8 dims read the scaled accumulator, RoPE dims their own
-        const int x = d < dmain ? dc : n_dc + (dc - dc_r0);
+        // FP8 dims read the scaled accumulator, RoPE dims their own.  TMEM
+        // loads are warp-collective, so a chunk that holds both kinds loads
+        // both and every lane keeps its own.
+        const bool has_rope = dc >= dc_r0;
         for (int hb = 0; hb < G; hb += 16) {
-          uint32_t ov[16];
-          tc::tmem_ld_x16(tmem + lane_base + col_o + x * 32 + hb, ov);
+          uint32_t om[16], orp[16];
+          tc::tmem_ld_x16(tmem + lane_base + col_o + dc * 32 + hb, om);
+          if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_o + (n_dc + dc - dc_r0) * 32 + hb, orp);
           tc::tmem_wait_ld();
           for (int e = 0; e < 16; ++e) {
             const int h = h0 + hb + e;
+            const float ov = __uint_as_float(d < dmain ? om[e] : orp[e]);
             if (h < H && d < D)
-              a.out[((int64_t)i * H + h) * D + d] =
-                  bf16_rn(__fdiv_rn(__uint_as_float(ov[e]) * cmul[hb + e], den[hb + e]));
+              a.out[((int64_t)i * H + h) * D + d] = bf16_rn(__fdiv_rn(ov * cmul[hb + e], den[hb + e]));
           }
         }
       }
