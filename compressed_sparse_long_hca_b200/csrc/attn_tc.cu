@@ -231,30 +231,48 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
         bf = reinterpret_cast<const uint16_t*>(st_ring + L.ring_bf16) + (int64_t)slot * R;
         sc = reinterpret_cast<const float*>(st_ring + L.ring_scale)[slot];
       }
-      const int nch = Dp / 8;
-      const int c0 = (tid >> 7) * (nch / 2), c1 = c0 + nch / 2;
       if (tid < kTileRows) rsc[r] = sc;
-      uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
-      for (int c = c0; c < c1; ++c) {
-        uint4 o = make_uint4(0, 0, 0, 0);
-        if (f8 != nullptr && 8 * c < D) {
-          if (8 * c < D - R) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(f8 + 8 * c);
-            const uint32_t wv[2] = {raw.x, raw.y};
-            uint32_t pk[4];
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-              const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
-              const float2 f = __half22float2(__half2(h2));
-              pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);   // exact
-            }
-            o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          } else {
-            o = *reinterpret_cast<const uint4*>(bf + (8 * c - (D - R)));
-          }
+      // This thread covers dims [lo, hi) of the row.  Issue every global load
+      // first (16-byte units: 16 FP8 dims or 8 BF16 dims), then convert.
+      const int lo = (tid >> 7) * (Dp / 2), hi = lo + Dp / 2;
+      const int f_lo = lo < D - R ? lo : D - R, f_hi = hi < D - R ? hi : D - R;          // FP8 dims
+      const int r_lo = lo > D - R ? (lo < D ? lo : D) : D - R, r_hi = hi < D ? hi : D;   // RoPE dims
+      const int nf = f_hi > f_lo ? (f_hi - f_lo) / 16 : 0;
+      const int nr = r_hi > r_lo ? (r_hi - r_lo) / 8 : 0;
+      constexpr int kMaxUnits = 24;
+      uint4 buf[kMaxUnits];
+#pragma unroll
+      for (int x = 0; x < kMaxUnits; ++x) {
+        buf[x] = make_uint4(0, 0, 0, 0);
+        if (f8 != nullptr) {
+          if (x < nf) buf[x] = *reinterpret_cast<const uint4*>(f8 + f_lo + 16 * x);
+          else if (x < nf + nr) buf[x] = *reinterpret_cast<const uint4*>(bf + (r_lo - (D - R)) + 8 * (x - nf));
         }
-        *reinterpret_cast<uint4*>(dst + c * 128) = o;
       }
+      uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
+#pragma unroll
+      for (int x = 0; x < kMaxUnits; ++x) {
+        if (x < nf) {   // 16 FP8 values -> two 8-dim BF16 chunks (exact conversion)
+          const uint32_t wv[4] = {buf[x].x, buf[x].y, buf[x].z, buf[x].w};
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
+            const float2 f = __half22float2(__half2(h2));
+            pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);
+          }
+          const int c = (f_lo + 16 * x) / 8;
+          *reinterpret_cast<uint4*>(dst + c * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(dst + (c + 1) * 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else if (x < nf + nr) {
+          const int c = (r_lo + 8 * (x - nf)) / 8;
+          *reinterpret_cast<uint4*>(dst + c * 128) = buf[x];
+        }
+      }
+      // dims past D (padding up to a multiple of 128) are zero
+      for (int c = (D > lo ? (D < hi ? D : hi) : lo) / 8; c < hi / 8; ++c)
+        *reinterpret_cast<uint4*>(dst + c * 128) = make_uint4(0, 0, 0, 0);
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();

@@ -57,8 +57,8 @@ bool cfg_ok(const csa_cfg* c, std::string* why) {
     return bad("need at least one layer");
   if (c->H < 1 || c->H > 128) return bad("H must be in [1, 128]");
   if (c->D < 64 || c->D > 512 || c->D % 32) return bad("D must be a multiple of 32 in [64, 512]");
-  if (c->D_rope < 16 || c->D_rope % 2 || c->D_rope >= c->D || (c->D - c->D_rope) % 16)
-    return bad("D_rope must be even, >= 16, < D, with D - D_rope a multiple of 16");
+  if (c->D_rope < 16 || c->D_rope > 64 || c->D_rope % 2 || c->D_rope >= c->D || (c->D - c->D_rope) % 16)
+    return bad("D_rope must be even, in [16, 64], < D, with D - D_rope a multiple of 16");
   if (c->n_csa_layers > 0) {
     if (c->H_I < 1 || c->H_I > 64) return bad("H_I must be in [1, 64]");
     if (c->d_I < 32 || c->d_I > 128 || c->d_I % 32) return bad("d_I must be 32, 64, 96 or 128");

@@ -115,8 +115,22 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   const int64_t hi = lo + chunk < N ? lo + chunk : N;
   const int64_t len = hi > lo ? hi - lo : 0;
   auto key_at = [&](int64_t x) -> uint32_t { return a.cache_keys ? keys[x] : order_key(s[lo + x]); };
-  if (a.cache_keys)
-    for (int64_t x = tid; x < len; x += kTopkThreads) keys[x] = order_key(s[lo + x]);
+  if (a.cache_keys) {
+    // eight loads in flight per thread before any of them is used
+    for (int64_t x0 = tid; x0 < len; x0 += 8 * kTopkThreads) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t x = x0 + (int64_t)u * kTopkThreads;
+        v[u] = x < len ? s[lo + x] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t x = x0 + (int64_t)u * kTopkThreads;
+        if (x < len) keys[x] = order_key(v[u]);
+      }
+    }
+  }
   if (tid == 0) { sh.digit = 0; sh.remaining = k; }
   uint32_t prefix = 0;
   int remaining = k;

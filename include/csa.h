@@ -93,8 +93,8 @@ typedef enum {
  * 0 .. n_csa_layers-1 are CSA layers, the next n_hca_layers are HCA layers.
  *   H        query heads (one shared KV head: multi-query attention), <= 128
  *   D        head dim, multiple of 32, 64 <= D <= 512
- *   D_rope   RoPE dims (the last D_rope dims of q and KV), even, 16 <= D_rope,
- *            D - D_rope a multiple of 16
+ *   D_rope   RoPE dims (the last D_rope dims of q and KV), even, 16 <= D_rope
+ *            <= 64, D - D_rope a multiple of 16
  *   H_I      indexer heads, 1 <= H_I <= 64 (ignored when n_csa_layers == 0)
  *   d_I      index dim, one of 32, 64, 96, 128
  *   window   raw-token sliding window; must be 128
