@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
     }
     __syncthreads();
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
-      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, kCsaM * j, L.rope_base);
+      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], L.theta()[p], kCsaM * j);
     __syncthreads();
     const int s = (int)(j % kCsaPerPage);
     char* pp = L.page(L.page_table(req)[j / kCsaPerPage], a.layer);
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
     }
     __syncthreads();
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
-      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, kHcaM * j, L.rope_base);
+      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], L.theta()[p], kHcaM * j);
     __syncthreads();
     const int s = (int)(j % kHcaPerPage);
     char* pp = L.page(L.page_table(req)[j / kHcaPerPage], a.layer);
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
     for (int d = threadIdx.x; d < D; d += blockDim.x) row[d] = src[d];
     __syncthreads();
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
-      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], p, R, pos, L.rope_base);
+      rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], L.theta()[p], pos);
     __syncthreads();
     const int slot = (int)(pos % kWindow);
     store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),

@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
       float v[8];
       for (int e = 0; e < 8; ++e) v[e] = (8 * c + e < D) ? bf16_val(qh[8 * c + e]) : 0.f;
       if (8 * c >= D - R && 8 * c < D) {
-        for (int e = 0; e < 8; e += 2) rope_pair(v[e], v[e + 1], (8 * c + e - (D - R)) / 2, R, t, L.rope_base);
+        for (int e = 0; e < 8; e += 2) rope_pair(v[e], v[e + 1], L.theta()[(8 * c + e - (D - R)) / 2], t);
       }
       for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
     }

@@ -72,11 +72,18 @@ __device__ __forceinline__ float scale_pow2(float x, int e) {
   return (x * exp2i(a)) * exp2i(b);
 }
 
-// Rotate the pair (x0, x1) at dim pair i of R rope dims by position pos.
-__device__ __forceinline__ void rope_pair(float& x0, float& x1, int i, int R, int64_t pos, float base) {
-  const double theta = pow((double)base, -2.0 * (double)i / (double)R);
+// Rotate the pair (x0, x1) by angle pos * theta, in fp64 (positions reach
+// 2^20, so an fp32 angle would be off by up to 0.06 rad).  The angle is
+// first reduced to [-pi, pi] by subtracting the nearest multiple of 2*pi,
+// given as a two-double constant, which keeps sin/cos on their short path.
+__device__ __forceinline__ void rope_pair(float& x0, float& x1, double theta, int64_t pos) {
+  constexpr double kTwoPiHi = 6.283185307179586;           // 2*pi rounded to double
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;      // 2*pi - kTwoPiHi
+  const double ang = (double)pos * theta;
+  const double kq = rint(ang * (1.0 / kTwoPiHi));
+  const double r = fma(-kq, kTwoPiHi, ang) - kq * kTwoPiLo;
   double s, c;
-  sincos((double)pos * theta, &s, &c);
+  sincos(r, &s, &c);
   const double a = x0, b = x1;
   x0 = (float)(a * c - b * s);
   x1 = (float)(a * s + b * c);

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -112,6 +113,7 @@ Layout make_layout(const csa_cfg& c) {
   L.off_len = o; o = align_up(o + (int64_t)L.n_layers * L.max_req * 8, A);
   L.off_cap = o; o = align_up(o + (int64_t)L.max_req * 4, A);
   L.off_pt = o; o = align_up(o + (int64_t)L.max_req * L.max_pages_per_req * 4, A);
+  L.off_theta = o; o = align_up(o + (int64_t)(L.R / 2) * 8, A);
   L.off_bkv = o; o = align_up(o + (int64_t)L.n_csa * csa::kCsaWin * c.D * 4, A);
   L.off_bidx = o; o = align_up(o + (int64_t)L.n_csa * csa::kCsaWin * L.dI * 4, A);
   L.off_bhca = o; o = align_up(o + (int64_t)L.n_hca * csa::kHcaM * c.D * 4, A);
@@ -163,6 +165,12 @@ csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes, const
   if (e == cudaSuccess && L.n_hca)
     e = cudaMemcpy(L.base + L.off_bhca, b_pos_hca, (size_t)L.n_hca * csa::kHcaM * L.D * 4, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(position biases)");
+  {
+    std::vector<double> th(L.R / 2);
+    for (int i = 0; i < L.R / 2; ++i) th[i] = std::pow((double)cfg->rope_base, -2.0 * i / (double)L.R);
+    e = cudaMemcpy(L.base + L.off_theta, th.data(), th.size() * 8, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(rope frequencies)");
+  }
   csa_cache* c = new (std::nothrow) csa_cache();
   if (!c) return fail(CSA_ERR_CAPACITY, "host allocation failed");
   c->cfg = *cfg;

@@ -16,6 +16,7 @@
 //   lengths     int64 [n_layers][max_req]         tokens appended so far
 //   capacity    int32 [max_req]                   pages held by the request
 //   page table  int32 [max_req][max_pages_per_req]  logical -> pool page
+//   theta       fp64 [R/2]                        RoPE frequencies
 //   b_pos       fp32 [n_csa][8][D], [n_csa][8][d_I], [n_hca][128][D]
 //   state       per request, per layer:
 //                 window ring: fp8 [128][D-R] | bf16 [128][R] | fp32 [128]
@@ -64,7 +65,7 @@ struct Layout {
   // arena base
   char* base;
   // section offsets from base
-  int64_t off_err, off_len, off_cap, off_pt, off_bkv, off_bidx, off_bhca, off_state, off_pool;
+  int64_t off_err, off_len, off_cap, off_pt, off_theta, off_bkv, off_bidx, off_bhca, off_state, off_pool;
   // row sections
   int64_t kv_fp8_bytes;     // D - R
   int64_t kv_bf16_bytes;    // 2R
@@ -85,6 +86,8 @@ struct Layout {
     return reinterpret_cast<int32_t*>(base + off_pt) + (int64_t)req * max_pages_per_req;
   }
   __host__ __device__ int32_t* err() const { return reinterpret_cast<int32_t*>(base + off_err); }
+  // RoPE frequencies base^(-2i/R), i < R/2, in fp64 (written at initialisation)
+  __host__ __device__ const double* theta() const { return reinterpret_cast<const double*>(base + off_theta); }
   __host__ __device__ const float* bpos_csa(int layer) const {
     return reinterpret_cast<const float*>(base + off_bkv) + (int64_t)layer * kCsaWin * D;
   }

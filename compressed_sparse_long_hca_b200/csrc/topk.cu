@@ -141,9 +141,15 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     const uint32_t mask = (1u << width) - 1;
     for (int b = tid; b < kBins; b += kTopkThreads) sh.hist[b] = 0;
     __syncthreads();
-    for (int64_t x = tid; x < len; x += kTopkThreads) {
-      const uint32_t key = key_at(x);
-      if (p == 0 || (key >> (shift + width)) == prefix) atomicAdd(&sh.hist[(key >> shift) & mask], 1);
+    // lanes that hit the same bin add once (score distributions pile up in a
+    // few top-bit bins, where per-lane atomics would serialise)
+    for (int64_t x0 = tid - (tid & 31); x0 < len; x0 += kTopkThreads) {
+      const int64_t x = x0 + (tid & 31);
+      const uint32_t key = x < len ? key_at(x) : 0u;
+      const bool hit = x < len && (p == 0 || (key >> (shift + width)) == prefix);
+      const uint32_t bin = hit ? (key >> shift) & mask : 0xFFFFFFFFu;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (hit && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
     }
     // cluster reduce-scatter: CTA r sums bins [r*kBins/C, (r+1)*kBins/C)
     cluster.sync();
