@@ -170,6 +170,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
     __syncthreads();
     n_sel = s_nsel;
   }
+  // cos/sin of the query position for each RoPE pair, shared by all heads
+  float2* cs = reinterpret_cast<float2*>(stage);
+  for (int p = tid; p < R / 2; p += kAttThreads) {
+    float c = 1.f, sn = 0.f;
+    rope_pair(c, sn, L.theta()[p], t);      // rotating (1, 0) gives (cos, sin)
+    cs[p] = make_float2(c, sn);
+  }
+  __syncthreads();
   // query heads h0 .. h0+G-1, rotated at t, as BF16 in K-major core-matrix order
   for (int x = tid; x < G * (Dp / 8); x += kAttThreads) {
     const int hh = x / (Dp / 8), c = x % (Dp / 8);
@@ -180,7 +188,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
       float v[8];
       for (int e = 0; e < 8; ++e) v[e] = (8 * c + e < D) ? bf16_val(qh[8 * c + e]) : 0.f;
       if (8 * c >= D - R && 8 * c < D) {
-        for (int e = 0; e < 8; e += 2) rope_pair(v[e], v[e + 1], L.theta()[(8 * c + e - (D - R)) / 2], t);
+        for (int e = 0; e < 8; e += 2) {
+          const float2 w = cs[(8 * c + e - (D - R)) / 2];
+          const float x0 = v[e], x1 = v[e + 1];
+          v[e] = x0 * w.x - x1 * w.y;
+          v[e + 1] = x0 * w.y + x1 * w.x;
+        }
       }
       for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
     }

@@ -148,6 +148,7 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
       const uint32_t key = x < len ? key_at(x) : 0u;
       const bool hit = x < len && (p == 0 || (key >> (shift + width)) == prefix);
       const uint32_t bin = hit ? (key >> shift) & mask : 0xFFFFFFFFu;
+      if (!__any_sync(0xffffffffu, hit)) continue;
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
       if (hit && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
     }
@@ -184,22 +185,28 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   }
   const uint32_t T = prefix;        // the k-th largest key
   const int ties_needed = remaining;
-  // ---- output: per-thread contiguous sub-slices in index order
-  const int64_t per_thr = (len + kTopkThreads - 1) / kTopkThreads;
-  const int64_t t_lo = tid * per_thr < len ? tid * per_thr : len;
-  const int64_t t_hi = t_lo + per_thr < len ? t_lo + per_thr : len;
-  int gt = 0, eq = 0;
-  for (int64_t x = t_lo; x < t_hi; ++x) {
-    const uint32_t key = key_at(x);
-    gt += key > T;
-    eq += key == T;
+  // ---- output: each warp owns a contiguous sub-slice, walked 32 keys at a
+  //      time (lane l reads key base + l: conflict-free), so that ballots
+  //      give ordered positions.
+  const int lane = tid & 31, wid = tid >> 5;
+  constexpr int kWarps = kTopkThreads / 32;
+  const int64_t per_w = ((len + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t w_lo = (int64_t)wid * per_w < len ? (int64_t)wid * per_w : len;
+  const int64_t w_hi = w_lo + per_w < len ? w_lo + per_w : len;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  int gt = 0, eq = 0;   // warp totals (uniform across the warp)
+  for (int64_t x0 = w_lo; x0 < w_hi; x0 += 32) {
+    const int64_t x = x0 + lane;
+    const uint32_t key = x < w_hi ? key_at(x) : 0u;
+    gt += __popc(__ballot_sync(0xffffffffu, x < w_hi && key > T));
+    eq += __popc(__ballot_sync(0xffffffffu, x < w_hi && key == T));
   }
   int gt_tot, eq_tot;
-  const int gt_before = block_excl_scan(gt, sh.wsum, &gt_tot);
-  const int eq_before = block_excl_scan(eq, sh.wsum, &eq_tot);
+  const int gt_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? gt : 0, sh.wsum, &gt_tot), 0);
+  const int eq_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? eq : 0, sh.wsum, &eq_tot), 0);
   if (tid == 0) { sh.cnt[0] = gt_tot; sh.cnt[1] = eq_tot; }
   cluster.sync();
-  int sel_before = 0, ties_before = 0, take_cta = 0;
+  int sel_before = 0, take_cta = 0;
   {
     int tb = 0;
     for (int r = 0; r < C; ++r) {
@@ -207,26 +214,31 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
       const int g = c[0], e = c[1];
       int take = ties_needed - tb;
       take = take < 0 ? 0 : (take > e ? e : take);
-      if (r < rank) { sel_before += g + take; ties_before += e; }
+      if (r < rank) sel_before += g + take;
       if (r == rank) take_cta = take;
       tb += e;
     }
   }
-  // ties this thread may take: those among the CTA's first take_cta ties
-  int my_take_ties = take_cta - eq_before;
-  my_take_ties = my_take_ties < 0 ? 0 : (my_take_ties > eq ? eq : my_take_ties);
+  // ties this warp may take: those among the CTA's first take_cta ties
+  int w_ties = take_cta - eq_before;
+  w_ties = w_ties < 0 ? 0 : (w_ties > eq ? eq : w_ties);
   int tot_sel;
-  const int pos0 = block_excl_scan(gt + my_take_ties, sh.wsum, &tot_sel);
-  int pos = sel_before + pos0;
-  int ties_left = my_take_ties;
-  for (int64_t x = t_lo; x < t_hi; ++x) {
-    const uint32_t key = key_at(x);
-    if (key > T || (key == T && ties_left > 0)) {
-      if (key == T) --ties_left;
-      out[pos++] = (int32_t)(lo + x);
-    }
+  const int w_pos0 = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? gt + w_ties : 0, sh.wsum, &tot_sel), 0);
+  int pos = sel_before + w_pos0;
+  int ties_seen = 0;
+  for (int64_t x0 = w_lo; x0 < w_hi; x0 += 32) {
+    const int64_t x = x0 + lane;
+    const uint32_t key = x < w_hi ? key_at(x) : 0u;
+    const bool is_eq = x < w_hi && key == T;
+    const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
+    const int tie_rank = ties_seen + __popc(eqb & lt_mask);
+    const bool take = x < w_hi && (key > T || (is_eq && tie_rank < w_ties));
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos + __popc(tb & lt_mask)] = (int32_t)(lo + x);
+    pos += __popc(tb);
+    ties_seen += __popc(eqb);
   }
-  (void)ties_before;
+  (void)gt_before;
   // no CTA may leave while others still read its shared memory
   cluster.sync();
 }
