@@ -57,6 +57,27 @@ def _dist():
     return ws, rank, local
 
 
+def rank_seed(wl, rank: int) -> int:
+    """Seed of the requests a rank owns: ranks hold disjoint requests."""
+    return wl.seed + 7919 * rank
+
+
+def max_over_ranks(vals, ws: int, device) -> list:
+    """Element-wise maximum of per-rank device timings (all ranks call it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(ws: int, batch_per_rank: int, steps: int, ms: float) -> float:
+    """Queries per second of the whole job: every rank's queries over the
+    slowest rank's time."""
+    return ws * batch_per_rank * steps / (ms / 1e3)
+
+
 class Clocks:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -117,6 +138,7 @@ def run_gpu(args):
     import torch
     import torch.distributed as dist
 
+    from compressed_sparse_long_hca_b200 import _lib
     from compressed_sparse_long_hca_b200.api import Cache, topk
 
     ws, rank, local = _dist()
@@ -145,7 +167,7 @@ def run_gpu(args):
     while t < T0:
         n_tok = min(I.CHUNK, T0 - t)
         chunk = t // I.CHUNK
-        parts = [I.device_token_inputs(wl.seed + 7919 * rank, layer, r, chunk, wl.D, dI) for r in range(B)]
+        parts = [I.device_token_inputs(rank_seed(wl, rank), layer, r, chunk, wl.D, dI) for r in range(B)]
         st = lambda k: torch.stack([p[k][:n_tok] for p in parts]).contiguous() if parts[0][k] is not None else None
         cache.compress_append(layer, rid, st(0), st(1), st(2), st(3))
         t += n_tok
@@ -154,7 +176,7 @@ def run_gpu(args):
     # ---- per-step inputs (device), generated up front
     total_steps = steps + warm
     g = torch.Generator(device="cuda")
-    g.manual_seed(wl.seed * 31 + rank)
+    g.manual_seed(rank_seed(wl, rank) * 31)
     step_c = torch.randn((total_steps, B, 1, wl.D), generator=g, device="cuda")
     step_z = torch.randn((total_steps, B, 1, wl.D), generator=g, device="cuda")
     step_ci = torch.randn((total_steps, B, 1, dI), generator=g, device="cuda") if csa else None
@@ -185,7 +207,6 @@ def run_gpu(args):
         else:
             cache.decode_attn(layer, rid, q, None, sink_d, out)
 
-    launches_per_step = 3 + (3 if csa else 1)
     for s in range(warm):
         step(s)
     torch.cuda.synchronize()
@@ -197,12 +218,15 @@ def run_gpu(args):
     clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     evi = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    lib = _lib.load()
+    launches0 = lib.csa_launch_count()
     for s in range(steps):
         flush.zero_()                       # L2 flushed between timed steps (not timed)
         ev[s][0].record(stream)
         step(warm + s, evi[s] if csa else None)
         ev[s][1].record(stream)
     torch.cuda.synchronize()
+    launches = lib.csa_launch_count() - launches0     # libcsa kernels queued in the timed region
     step_ms = sum(a.elapsed_time(b) for a, b in ev)
     idx_ms = sum(a.elapsed_time(b) for a, b in evi) / steps if csa else None
     # ---- end to end through the public API with host buffers
@@ -246,12 +270,9 @@ def run_gpu(args):
     clk = clocks.stop()
     cache.check_device_error()
     # ---- max over ranks
-    tt = torch.tensor([step_ms, e2e_ms, idx_ms or 0.0], dtype=torch.float64, device="cuda")
-    if ws > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    step_ms, e2e_ms, idx_ms = tt.tolist()
-    value = ws * B * steps / (step_ms / 1e3)
-    e2e_value = ws * B * steps / (e2e_ms / 1e3)
+    step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms or 0.0], ws, "cuda")
+    value = whole_job_rate(ws, B, steps, step_ms)
+    e2e_value = whole_job_rate(ws, B, steps, e2e_ms)
     peak, peak_kind, _ = _peaks()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
@@ -262,7 +283,7 @@ def run_gpu(args):
                    "topk": wl.k, "window": wl.W, "layers_per_step": 1,
                    "l2": "flushed (256 MB write) before every timed step",
                    "parallelism": f"request-sharded x{ws}"},
-        "gpu_launches": launches_per_step * steps,
+        "gpu_launches": launches,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "clocks": clk,
     }

@@ -119,8 +119,21 @@ class Cache:
                                         _ptr(scores), scores.shape[1], _ptr(n_valid),
                                         VARIANTS[variant], _stream(stream)), "csa_index_scores")
 
+    def attn_workspace_bytes(self, layer: int, n: int, k: int = 0) -> int:
+        return int(self.lib.csa_attn_workspace_bytes(self.handle, layer, n, k))
+
+    def _workspace(self, nbytes: int, device) -> torch.Tensor:
+        ws = getattr(self, "_ws", None)
+        if ws is None or ws.numel() < nbytes or ws.device != device:
+            ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+            self._ws = ws
+        return ws
+
     def decode_attn(self, layer: int, req_ids, q, topk_idx, sink, out, scale=None,
-                    variant="auto", stream=None) -> None:
+                    variant="auto", stream=None, workspace: torch.Tensor | None = None) -> None:
+        """Attention of each query over its rows.  The split (low-occupancy)
+        launch needs scratch; unless `workspace` is given, a buffer owned by
+        this Cache object is grown to the size the library asks for."""
         n = req_ids.numel()
         _need(req_ids, torch.int32, name="req_ids")
         _need(q, torch.bfloat16, (n, self.H, self.D), "q")
@@ -132,9 +145,16 @@ class Cache:
             k = topk_idx.shape[1]
         if scale is None:
             scale = 1.0 / float(np.sqrt(self.D))
+        ws_ptr, ws_bytes = None, 0
+        if variant != "high" and n > 0:
+            need = self.attn_workspace_bytes(layer, n, k)
+            if workspace is None:
+                workspace = self._workspace(need, q.device)
+            _need(workspace, torch.uint8, name="workspace")
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
         check(self.lib.csa_hca_decode_attn(self.handle, layer, n, _ptr(req_ids), _ptr(q), _ptr(topk_idx),
-                                           k, _ptr(sink), scale, _ptr(out), VARIANTS[variant],
-                                           _stream(stream)), "csa_hca_decode_attn")
+                                           k, _ptr(sink), scale, _ptr(out), ws_ptr, ws_bytes,
+                                           VARIANTS[variant], _stream(stream)), "csa_hca_decode_attn")
 
     def check_device_error(self, stream=None) -> None:
         check(self.lib.csa_check_device_error(self.handle, _stream(stream)), "device")

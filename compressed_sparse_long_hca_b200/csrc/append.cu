@@ -252,18 +252,22 @@ cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_
   if (csa) {
     const size_t sm = (size_t)(L.D + L.dI + 32) * sizeof(float);
     csa_entries_kernel<<<g1, threads, sm, st>>>(a);
+    note_launch();
   } else {
     const size_t sm = (size_t)(L.D + 32) * sizeof(float);
     hca_entries_kernel<<<g1, threads, sm, st>>>(a);
+    note_launch();
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int rows = n_tok < kWindow ? n_tok : kWindow;
   dim3 g2(n, (unsigned)rows);
   tokens_kernel<<<g2, threads, (size_t)(L.D + 32) * sizeof(float), st>>>(a);
+  note_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   length_kernel<<<(n + 127) / 128, 128, 0, st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -9,27 +9,42 @@
 // to the softmax denominator, RoPE acts on the last 64 dims only, and the
 // stored KV is FP8 (non-RoPE dims) + BF16 (RoPE dims).
 //
-// Per query the rows are: selected entries (ascending; HCA: all entries)
-// then the window (ascending positions); K = V = the stored row.  Because
-// the KV head is shared, QK^T and PV are dense products.  A CTA owns one
-// query and a group of G heads and walks the rows in tiles of 128:
-//   * all threads gather the tile's rows from the paged cache and the ring,
-//     dequantise them to BF16 and store them in shared memory in the
-//     no-swizzle core-matrix order;
-//   * QK: S^T[128 rows x G heads] = K_tile Q^T on tcgen05 (kind::f16,
-//     M = 128 rows, N = G heads, K = 16 dims per instruction) into TMEM;
-//   * softmax: one thread per row reads its G logits; per-head maxima and
-//     sums go through shared memory in a fixed order.  The running maximum
-//     of a head is only raised when a tile exceeds it by more than 8 (then
-//     the head's accumulator column is rescaled), so most tiles need no
-//     rescale; every decision depends on the query's own data only;
-//   * PV: O^T[dims x G] += V_tile^T P^T on tcgen05, the same shared-memory
-//     tile read as an MN-major A operand, P^T (BF16) as an MN-major B operand;
-//   * the sink enters at the end: out = O e^{m-mu} / (l e^{m-mu} + e^{sink-mu}),
-//     mu = max(m, sink).
-// A query's reduction over rows is never split across CTAs.  Launch
-// variants differ only in G (heads per CTA); every per-head operation is
-// independent of G, so the variants return identical bits.
+// Rows of a query: the entries of its top-k list in list order (HCA: every
+// completed entry), then the window in ascending position; a -1 in the list
+// is an empty row.  K = V = the stored row.  Because the KV head is shared,
+// QK^T and PV are dense products.
+//
+// Reduction order (fixed by the query alone).  The rows are cut into tiles
+// of 128.  Each tile gives a partial result
+//     m_t = max_r u_r,  l_t = sum_r e^{u_r - m_t},  O_t = sum_r e^{u_r - m_t} V_r
+// and the partials are folded in tile order,
+//     m' = max(m, m_t),  l' = l e^{m-m'} + l_t e^{m_t-m'},  O' = O e^{m-m'} + O_t e^{m_t-m'};
+// the sink enters last: out = O e^{m-mu} / (l e^{m-mu} + e^{sink-mu}),
+// mu = max(m, sink).  Page "DeepSeek不惜代价保住它！V4关键特性被挖出来了",
+// section "牺牲了什么" (and page "DeepSeek V4 底层逻辑全解析：从 V3 到 V4，真正
+// 升级了什么？", section "升级点 3"): the authors give up split-KV because its
+// reduction path changes with the batch, and ship two attention kernels (for
+// a well-fed and an under-fed GPU) that agree bit for bit.  Here both launch variants
+// compute the same tiles with the same code and fold them with the same
+// arithmetic:
+//   * whole-query launch (well-fed GPU): one CTA per (query, head group)
+//     walks the tiles and folds each into a running accumulator in TMEM;
+//   * split launch (under-fed GPU): one CTA per (query, head group, tile)
+//     writes its partial to the caller's workspace, and attn_fold_kernel
+//     folds them in tile order, one thread per output element.
+// Nothing in either path depends on the batch.
+//
+// Per tile, in a CTA of 8 warps:
+//   * the rows' addresses are resolved (page table, ring slot) into shared
+//     memory; all threads then gather the rows, 8 rows x 4 16-byte chunks per
+//     warp instruction, dequantise the FP8 codes exactly to BF16 and store
+//     them in the no-swizzle core-matrix order;
+//   * QK: S^T[128 rows x G heads] = K_tile Q^T (kind::f16, M = 128 rows,
+//     N = G heads) into TMEM, in two accumulators: the FP8 dims (scaled by
+//     the row's FP8 scale afterwards) and the BF16 RoPE dims;
+//   * softmax statistics of the tile: one thread per (row, 16 heads);
+//   * PV: O_t^T[dims x G] = V^T P^T, P^T in BF16; the FP8 dims use
+//     (P * row scale)^T, the RoPE dims P^T, each into its own accumulator.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -37,12 +52,12 @@ namespace csa {
 
 namespace {
 
-constexpr int kAttThreads = 256;       // warps 0-3: TMEM lanes / softmax; all: gather
+constexpr int kAttThreads = 256;
 constexpr int kTileRows = 128;
-constexpr float kSlack = 8.f;          // stale running maximum allowed below a tile's max
-constexpr int kMaxK = 8192;
+constexpr int kMaxLoads = 18;      // 16-byte loads per thread per tile (D <= 512)
+constexpr int kFoldBatch = 8;      // partials loaded at once by the fold kernel
 
-struct AttnTcArgs {
+struct AttnArgs {
   Layout L;
   int layer;
   int n;
@@ -53,406 +68,512 @@ struct AttnTcArgs {
   const float* sink;
   float scale;
   uint16_t* out;
-  int G;            // heads per CTA (MMA N), 16 or 32
+  int G;              // heads per CTA (MMA N), 16 or 32
+  // split launch only: partials of (query i, tile t, head h)
+  float* ws_o;        // [n][tiles_max][H][D]
+  float2* ws_ml;      // [n][tiles_max][H]   (m_t, l_t); m_t = -inf: empty tile
+  int tiles_max;
 };
 
-struct AttnSmemLayout {
-  int Dp;           // head dim padded to a multiple of 128
-  int64_t tile, qs, pt, stage, sel, rsc, stats, bars, total;
+struct QueryGeom {
+  int req;
+  bool csa;
+  int64_t t;          // query position
+  int64_t n_entries, w0, n_win, n_list, total;
+  int n_tiles;
 };
 
-__host__ __device__ inline AttnSmemLayout attn_smem_layout(int D, int G, int k) {
-  AttnSmemLayout s{};
+__device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& g, bool report) {
+  const Layout& L = a.L;
+  g.req = a.req_ids[i];
+  if (g.req < 0 || g.req >= L.max_req) {
+    if (report) set_err(L, kErrBounds, i);
+    return false;
+  }
+  g.csa = a.layer < L.n_csa;
+  const int64_t T = L.lengths()[(int64_t)a.layer * L.max_req + g.req];
+  if (T <= 0) {
+    if (report) set_err(L, kErrBounds, 1000000 + i);
+    return false;
+  }
+  g.t = T - 1;
+  g.n_entries = g.csa ? T / kCsaM : T / kHcaM;
+  g.w0 = g.t - (kWindow - 1) > 0 ? g.t - (kWindow - 1) : 0;
+  g.n_win = g.t - g.w0 + 1;
+  g.n_list = g.csa ? a.k : g.n_entries;
+  g.total = g.n_list + g.n_win;
+  g.n_tiles = (int)((g.total + kTileRows - 1) / kTileRows);
+  return true;
+}
+
+// The fold of one partial into a running (m, l, O); shared by both launch
+// variants so that they round identically.
+__device__ __forceinline__ void fold_coef(float m, float mt, float& mn, float& al, float& be) {
+  mn = fmaxf(m, mt);
+  al = (m == -INFINITY) ? 0.f : expf(m - mn);
+  be = expf(mt - mn);
+}
+__device__ __forceinline__ float fold_val(float o, float al, float ot, float be) {
+  const float b = __fmul_rn(ot, be);
+  return al == 0.f ? b : __fmaf_rn(o, al, b);
+}
+__device__ __forceinline__ void finish_coef(float m, float sk, float l, float& cm, float& den) {
+  const float mu = fmaxf(m, sk);
+  cm = expf(m - mu);
+  den = __fmaf_rn(l, cm, expf(sk - mu));
+}
+__device__ __forceinline__ uint16_t finish_val(float o, float cm, float den) {
+  return bf16_rn(__fdiv_rn(__fmul_rn(o, cm), den));
+}
+
+struct AttnSmem {
+  int Dp;             // head dim padded to a multiple of 128
+  int64_t tile, qs, pt, stage, rowf8, rowbf, rsc, stats, bars, total;
+};
+
+__host__ __device__ inline AttnSmem attn_smem(int D, int G) {
+  AttnSmem s{};
   s.Dp = (D + 127) / 128 * 128;
   int64_t o = 0;
   s.tile = o;  o += (int64_t)kTileRows * s.Dp * 2;           // BF16 rows, core-matrix order
   s.qs = o;    o += (int64_t)G * s.Dp * 2;                   // BF16 query heads
-  s.pt = o;    o += (int64_t)kTileRows * G * 2 * 2;          // BF16 P^T and (P*scale)^T (MN-major)
-  s.stage = o; o += (int64_t)kTileRows * (G + 1) * 4;        // fp32 logits / p for reductions
-  s.sel = o;   o += (int64_t)(k > 0 ? k : 1) * 4;            // compacted selected entries
-  s.rsc = o;   o += (int64_t)kTileRows * 4;                  // per-row FP8 scale of the tile
-  o = (o + 15) / 16 * 16;
-  s.stats = o; o += (int64_t)(6 * 32 + 4 * 32) * 4;          // m, l, corr, mt, den, cm; partials [4][32]
+  s.pt = o;    o += (int64_t)kTileRows * G * 2 * 2;          // BF16 P^T and (P*scale)^T
+  s.stage = o; o += (int64_t)kTileRows * (G + 1) * 4;        // fp32 logits / p
+  s.rowf8 = o; o += (int64_t)kTileRows * 8;                  // row addresses (FP8 part)
+  s.rowbf = o; o += (int64_t)kTileRows * 8;                  // row addresses (BF16 part)
+  s.rsc = o;   o += (int64_t)kTileRows * 4;                  // row FP8 scales
+  s.stats = o; o += (int64_t)12 * 32 * 4;
   o = (o + 15) / 16 * 16;
   s.bars = o;  o += 64;
   s.total = o;
   return s;
 }
 
+__device__ __forceinline__ uint4 ld_nc16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// Address of row `r` of tile `tt`; returns whether the row exists.
+__device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& g, int i, int tt, int r,
+                                            uint64_t* rowf8, uint64_t* rowbf, float* rsc) {
+  const Layout& L = a.L;
+  const int64_t rr = (int64_t)tt * kTileRows + r;
+  const uint8_t* f8 = nullptr;
+  const uint16_t* bf = nullptr;
+  float sc = 0.f;
+  if (rr < g.n_list) {
+    int64_t j = g.csa ? (int64_t)a.topk[(int64_t)i * a.k + rr] : rr;
+    if (j >= g.n_entries) {
+      set_err(L, kErrBounds, 2000000 + i);
+      j = -1;
+    }
+    if (j >= 0) {
+      const float* scp;
+      L.entry_row(g.req, a.layer, j, &f8, &bf, &scp);
+      sc = *scp;
+    }
+  } else if (rr < g.total) {
+    const char* st = L.state(g.req, a.layer);
+    const int slot = (int)((g.w0 + (rr - g.n_list)) % kWindow);
+    f8 = reinterpret_cast<const uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (L.D - L.R);
+    bf = reinterpret_cast<const uint16_t*>(st + L.ring_bf16) + (int64_t)slot * L.R;
+    sc = reinterpret_cast<const float*>(st + L.ring_scale)[slot];
+  }
+  rowf8[r] = reinterpret_cast<uint64_t>(f8);
+  rowbf[r] = reinterpret_cast<uint64_t>(bf);
+  rsc[r] = sc;
+  return f8 != nullptr;
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
+// Both launch variants.  kSplit: grid (tiles_max, head groups, n), one tile
+// per CTA, partials to the workspace.  Otherwise grid (n, head groups).
+template <bool kSplit>
+__global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout& L = a.L;
   const int D = L.D, R = L.R, H = L.H, G = a.G;
-  const AttnSmemLayout S = attn_smem_layout(D, G, a.k);
+  const AttnSmem S = attn_smem(D, G);
   const int Dp = S.Dp;
   const uint32_t sbo_rows = (uint32_t)Dp * 16;        // bytes between 8-row groups of the tile
   uint8_t* tile = sm + S.tile;
   uint8_t* qs = sm + S.qs;
   uint8_t* pt = sm + S.pt;
+  uint8_t* ptm = pt + kTileRows * G * 2;               // (P * row scale)^T for the FP8 dims
   float* stage = reinterpret_cast<float*>(sm + S.stage);
-  int32_t* sel = reinterpret_cast<int32_t*>(sm + S.sel);
+  uint64_t* rowf8 = reinterpret_cast<uint64_t*>(sm + S.rowf8);
+  uint64_t* rowbf = reinterpret_cast<uint64_t*>(sm + S.rowbf);
   float* rsc = reinterpret_cast<float*>(sm + S.rsc);
-  uint8_t* ptm = pt + kTileRows * G * 2;                   // (P * row scale)^T for the FP8 dims
-  float* m_run = reinterpret_cast<float*>(sm + S.stats);
+  float* m_t = reinterpret_cast<float*>(sm + S.stats);
+  float* l_t = m_t + 32;
+  float* m_run = l_t + 32;
   float* l_run = m_run + 32;
-  float* corr = l_run + 32;
-  float* m_tile = corr + 32;
-  float* den = m_tile + 32;
-  float* cmul = den + 32;
-  float* part = cmul + 32;                                  // [4][32]
+  float* alpha = l_run + 32;
+  float* beta = alpha + 32;
+  float* cmul = beta + 32;
+  float* den = cmul + 32;
+  float* part = den + 32;                                // [4][32]
   uint64_t* bar_qk = reinterpret_cast<uint64_t*>(sm + S.bars);
   uint64_t* bar_pv = bar_qk + 1;
   uint64_t* bar_drain = bar_qk + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_qk + 3);
-  __shared__ int s_nsel, s_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i = blockIdx.x;
+  const int i = kSplit ? (int)blockIdx.z : (int)blockIdx.x;
   const int h0 = blockIdx.y * G;
-  const int req = a.req_ids[i];
-  if (req < 0 || req >= L.max_req) {
-    if (tid == 0 && blockIdx.y == 0) set_err(L, kErrBounds, i);
-    return;
+  const int tt0 = kSplit ? (int)blockIdx.x : 0;
+  QueryGeom g;
+  const bool reporter = tid == 0 && blockIdx.y == 0 && (!kSplit || blockIdx.x == 0);
+  if (!query_geom(a, i, g, reporter)) return;
+  if (kSplit) {
+    if (g.n_tiles > a.tiles_max) {
+      if (reporter) set_err(L, kErrBounds, 4000000 + i);
+      return;
+    }
+    if (tt0 >= g.n_tiles) return;
   }
-  const bool csa = a.layer < L.n_csa;
-  const int64_t T = L.lengths()[(int64_t)a.layer * L.max_req + req];
-  if (T <= 0) {
-    if (tid == 0 && blockIdx.y == 0) set_err(L, kErrBounds, 1000000 + i);
-    return;
-  }
-  const int64_t t = T - 1;
-  const int64_t n_entries = csa ? T / kCsaM : T / kHcaM;
-  const int64_t w0 = t - (kWindow - 1) > 0 ? t - (kWindow - 1) : 0;
-  const int64_t n_win = t - w0 + 1;
+  const int tt_end = kSplit ? tt0 + 1 : g.n_tiles;
 
-  // ---- set-up: TMEM (S^T: G columns, O^T: Dp/128 chunks of G columns), barriers
+  // TMEM columns: S over the FP8 dims, S over the RoPE dims, the tile's
+  // output accumulators (per 128-dim chunk one for the FP8 dims and, where
+  // the chunk holds RoPE dims, one for those), then (whole-query launch) the
+  // running output, one accumulator per chunk.
+  const int n_dc = Dp / 128;
+  const int dmain = D - R;
+  const int dc_r0 = dmain / 128;                        // first chunk holding RoPE dims
+  const int n_acc = n_dc + (n_dc - dc_r0);
+  const uint32_t col_s = 0, col_sr = G, col_ot = 2 * G, col_orun = 2 * G + n_acc * G;
+  const int cols_needed = kSplit ? (int)col_orun : (int)col_orun + n_dc * G;
+  uint32_t n_cols = 32;
+  while ((int)n_cols < cols_needed) n_cols <<= 1;
+
   if (warp == 0) {
-    tc::tmem_alloc(tmem_slot, 256);
+    tc::tmem_alloc(tmem_slot, n_cols);
     tc::tmem_relinquish();
   }
-  if (tid == 0) {
+  if (tid == 32) {
     tc::mbar_init(bar_qk, 1);
     tc::mbar_init(bar_pv, 1);
     tc::mbar_init(bar_drain, 1);
     tc::fence_mbar_init();
   }
   if (tid < 32) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; }
-  // compact the selected list (CSA) in order, dropping -1 and out-of-range entries
-  int64_t n_sel = csa ? 0 : n_entries;
-  if (csa) {
-    if (tid == 0) s_nsel = 0;
-    __syncthreads();
-    for (int base = 0; base < a.k; base += kAttThreads) {
-      const int x = base + tid;
-      int j = x < a.k ? a.topk[(int64_t)i * a.k + x] : -1;
-      if (j >= n_entries) { set_err(L, kErrBounds, 2000000 + i); j = -1; }
-      const int v = j >= 0 ? 1 : 0;
-      // ordered compaction of this chunk of 256
-      const unsigned ballot = __ballot_sync(0xffffffffu, v);
-      const int wcount = __popc(ballot);
-      const int wpre = __popc(ballot & ((1u << lane) - 1));
-      __syncthreads();
-      if (lane == 0) part[warp] = (float)wcount;            // reuse as scratch (counts < 2^24)
-      __syncthreads();
-      int before = s_nsel;
-      for (int w = 0; w < warp; ++w) before += (int)part[w];
-      if (v) sel[before + wpre] = j;
-      __syncthreads();
-      if (tid == 0) {
-        int tot = 0;
-        for (int w = 0; w < kAttThreads / 32; ++w) tot += (int)part[w];
-        s_nsel += tot;
-      }
+  int any = 0;
+  if (warp < 4) {
+    any = resolve_row(a, g, i, tt0, tid, rowf8, rowbf, rsc) ? 1 : 0;
+  } else {
+    // warps 4-7: the query heads h0 .. h0+G-1 rotated at t, BF16, K-major core order
+    const int qt = tid - 128;
+    float2* cs = reinterpret_cast<float2*>(stage);
+    for (int p = qt; p < R / 2; p += 128) {
+      float c = 1.f, sn = 0.f;
+      rope_pair(c, sn, L.theta()[p], g.t);       // rotating (1, 0) gives (cos, sin)
+      cs[p] = make_float2(c, sn);
     }
-    __syncthreads();
-    n_sel = s_nsel;
-  }
-  // cos/sin of the query position for each RoPE pair, shared by all heads
-  float2* cs = reinterpret_cast<float2*>(stage);
-  for (int p = tid; p < R / 2; p += kAttThreads) {
-    float c = 1.f, sn = 0.f;
-    rope_pair(c, sn, L.theta()[p], t);      // rotating (1, 0) gives (cos, sin)
-    cs[p] = make_float2(c, sn);
-  }
-  __syncthreads();
-  // query heads h0 .. h0+G-1, rotated at t, as BF16 in K-major core-matrix order
-  for (int x = tid; x < G * (Dp / 8); x += kAttThreads) {
-    const int hh = x / (Dp / 8), c = x % (Dp / 8);
-    const int h = h0 + hh;
-    uint32_t pk[4] = {0, 0, 0, 0};
-    if (h < H) {
-      const uint16_t* qh = a.q + ((int64_t)i * H + h) * D;
-      float v[8];
-      for (int e = 0; e < 8; ++e) v[e] = (8 * c + e < D) ? bf16_val(qh[8 * c + e]) : 0.f;
-      if (8 * c >= D - R && 8 * c < D) {
-        for (int e = 0; e < 8; e += 2) {
-          const float2 w = cs[(8 * c + e - (D - R)) / 2];
-          const float x0 = v[e], x1 = v[e + 1];
-          v[e] = x0 * w.x - x1 * w.y;
-          v[e + 1] = x0 * w.y + x1 * w.x;
+    tc::named_bar_sync(1, 128);
+    for (int x = qt; x < G * (Dp / 8); x += 128) {
+      const int hh = x / (Dp / 8), c = x % (Dp / 8);
+      const int h = h0 + hh;
+      uint32_t pk[4] = {0, 0, 0, 0};
+      if (h < H && 8 * c < D) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(a.q + ((int64_t)i * H + h) * D + 8 * c);
+        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
+        float v[8];
+        for (int e = 0; e < 8; ++e) v[e] = bf16_val((uint16_t)(rw[e >> 1] >> (16 * (e & 1))));
+        if (8 * c >= dmain) {
+          for (int e = 0; e < 8; e += 2) {
+            const float2 w = cs[(8 * c + e - dmain) / 2];
+            const float x0 = v[e], x1 = v[e + 1];
+            v[e] = x0 * w.x - x1 * w.y;
+            v[e + 1] = x0 * w.y + x1 * w.x;
+          }
         }
+        for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
       }
-      for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
+      *reinterpret_cast<uint4*>(qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-    *reinterpret_cast<uint4*>(qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    // padding dims [D, Dp) of the tile stay zero
+    const int npad = (Dp - D) / 8;
+    for (int x = qt; x < kTileRows * npad; x += 128) {
+      const int r = x % kTileRows, c = D / 8 + x / kTileRows;
+      *reinterpret_cast<uint4*>(tile + (r >> 3) * sbo_rows + c * 128 + (r & 7) * 16) = make_uint4(0, 0, 0, 0);
+    }
   }
-  tc::tc_fence_before();
-  __syncthreads();
+  bool tile_valid = __syncthreads_count(any) > 0;
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  // TMEM columns: S_fp8 (logit part over the FP8 dims, before the row
-  // scale), S_bf16 (RoPE dims), then per 128-dim chunk of the output an
-  // accumulator for the FP8 dims (B = (P*scale)^T) and, where the chunk
-  // holds RoPE dims, one for those (B = P^T).
-  const uint32_t col_s = 0, col_sr = 32, col_o = 64;
-  const int n_dc = Dp / 128;
-  const int dmain = D - R;
-  const int dc_r0 = dmain / 128;                            // first chunk holding RoPE dims
-  const int64_t total = n_sel + n_win;
-  const int n_tiles = (int)((total + kTileRows - 1) / kTileRows);
-  const char* st_ring = L.state(req, a.layer);
+  const bool tw = warp < 4 * (G / 16);                  // this warp reads TMEM: lanes (warp%4)*32.., heads hb..hb+15
+  const int hb = 16 * (warp >> 2);
   const uint32_t id_qk = tc::idesc_bf16(128, G, false, false);
   const uint32_t id_pv = tc::idesc_bf16(128, G, true, true);
+  // gather geometry: chunks of a row are FP8 (16 dims) then BF16 (8 dims)
+  const int nc8 = dmain / 16, nc = nc8 + R / 8;
+  const int n_items = 16 * ((nc + 3) / 4);
   bool ok = true;
+  int n_done = 0;                                        // tiles whose PV has been issued
+  bool pend_fold = false;
 
-  for (int tt = 0; tt < n_tiles && ok; ++tt) {
-    // -- the previous tile's PV has finished: tile and P^T buffers are free
-    if (tt > 0) ok = tc::mbar_wait(bar_pv, (tt - 1) & 1);
-    ok = __syncthreads_and(ok) != 0;
-    if (!ok) break;
-    tc::tc_fence_after();
-    // -- gather + dequantise: thread handles row (tid % 128), half of the chunks
-    {
-      const int r = tid & (kTileRows - 1);
-      const int64_t rr = (int64_t)tt * kTileRows + r;
-      const uint8_t* f8 = nullptr;
-      const uint16_t* bf = nullptr;
-      float sc = 0.f;
-      if (rr < n_sel) {
-        const int64_t j = csa ? (int64_t)sel[rr] : rr;
-        const float* scp;
-        L.entry_row(req, a.layer, j, &f8, &bf, &scp);
-        sc = *scp;
-      } else if (rr < total) {
-        const int slot = (int)((w0 + (rr - n_sel)) % kWindow);
-        f8 = reinterpret_cast<const uint8_t*>(st_ring + L.ring_fp8) + (int64_t)slot * (D - R);
-        bf = reinterpret_cast<const uint16_t*>(st_ring + L.ring_bf16) + (int64_t)slot * R;
-        sc = reinterpret_cast<const float*>(st_ring + L.ring_scale)[slot];
-      }
-      if (tid < kTileRows) rsc[r] = sc;
-      // This thread covers dims [lo, hi) of the row.  Issue every global load
-      // first (16-byte units: 16 FP8 dims or 8 BF16 dims), then convert.
-      const int lo = (tid >> 7) * (Dp / 2), hi = lo + Dp / 2;
-      const int f_lo = lo < D - R ? lo : D - R, f_hi = hi < D - R ? hi : D - R;          // FP8 dims
-      const int r_lo = lo > D - R ? (lo < D ? lo : D) : D - R, r_hi = hi < D ? hi : D;   // RoPE dims
-      const int nf = f_hi > f_lo ? (f_hi - f_lo) / 16 : 0;
-      const int nr = r_hi > r_lo ? (r_hi - r_lo) / 8 : 0;
-      constexpr int kMaxUnits = 24;
-      uint4 buf[kMaxUnits];
-#pragma unroll
-      for (int x = 0; x < kMaxUnits; ++x) {
-        buf[x] = make_uint4(0, 0, 0, 0);
-        if (f8 != nullptr) {
-          if (x < nf) buf[x] = *reinterpret_cast<const uint4*>(f8 + f_lo + 16 * x);
-          else if (x < nf + nr) buf[x] = *reinterpret_cast<const uint4*>(bf + (r_lo - (D - R)) + 8 * (x - nf));
-        }
-      }
-      uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
-#pragma unroll
-      for (int x = 0; x < kMaxUnits; ++x) {
-        if (x < nf) {   // 16 FP8 values -> two 8-dim BF16 chunks (exact conversion)
-          const uint32_t wv[4] = {buf[x].x, buf[x].y, buf[x].z, buf[x].w};
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-            const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
-            const float2 f = __half22float2(__half2(h2));
-            pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);
-          }
-          const int c = (f_lo + 16 * x) / 8;
-          *reinterpret_cast<uint4*>(dst + c * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(dst + (c + 1) * 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        } else if (x < nf + nr) {
-          const int c = (r_lo + 8 * (x - nf)) / 8;
-          *reinterpret_cast<uint4*>(dst + c * 128) = buf[x];
-        }
-      }
-      // dims past D (padding up to a multiple of 128) are zero
-      for (int c = (D > lo ? (D < hi ? D : hi) : lo) / 8; c < hi / 8; ++c)
-        *reinterpret_cast<uint4*>(dst + c * 128) = make_uint4(0, 0, 0, 0);
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    // -- QK: S^T[rows x heads]
-    if (warp == 0) {
-      if (tc::elect_one()) {
-        const uint32_t ta = tc::smem_u32(tile), tq = tc::smem_u32(qs);
-        for (int ks = 0; ks < Dp / 16; ++ks) {
-          const bool main = 16 * ks < dmain;                  // (D - R) is a multiple of 16
-          const int k0 = main ? 0 : dmain / 16;
-          tc::mma_bf16(tmem + (main ? col_s : col_sr), tc::smem_desc(ta + ks * 256, 128, sbo_rows),
-                       tc::smem_desc(tq + ks * 256, 128, sbo_rows), id_qk, ks > k0 ? 1u : 0u);
-        }
-        tc::mma_commit(bar_qk);
-      }
-      __syncwarp();
-    }
-    // -- softmax statistics (warps 0-3 own the 128 TMEM lanes = rows)
-    const int r = tid;                       // valid for warps 0-3
-    const int64_t rr = (int64_t)tt * kTileRows + r;
-    float u[32];
-    if (warp < 4) {
-      ok = tc::mbar_wait(bar_qk, tt & 1);
+  for (int tt = tt0; tt < tt_end && ok; ++tt) {
+    if (tile_valid) {
+      // the previous PV has finished: tile buffer, P^T and O_t are free
+      if (n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
+      ok = __syncthreads_and(ok) != 0;
+      if (!ok) break;
       tc::tc_fence_after();
-      uint32_t sv[32], sr[32];
-      tc::tmem_ld_x16(tmem + lane_base + col_s, sv);
-      tc::tmem_ld_x16(tmem + lane_base + col_sr, sr);
-      if (G > 16) {
-        tc::tmem_ld_x16(tmem + lane_base + col_s + 16, sv + 16);
-        tc::tmem_ld_x16(tmem + lane_base + col_sr + 16, sr + 16);
+      // -- gather: issue every load of this thread first
+      uint4 buf[kMaxLoads];
+#pragma unroll
+      for (int u = 0; u < kMaxLoads; ++u) {
+        const int it = warp + 8 * u;
+        buf[u] = make_uint4(0, 0, 0, 0);
+        if (it < n_items) {
+          const int r = 8 * (it & 15) + (lane & 7), c = 4 * (it >> 4) + (lane >> 3);
+          if (c < nc8) {
+            const uint8_t* p = reinterpret_cast<const uint8_t*>(rowf8[r]);
+            if (p != nullptr) buf[u] = ld_nc16(p + 16 * c);
+          } else if (c < nc) {
+            const uint16_t* p = reinterpret_cast<const uint16_t*>(rowbf[r]);
+            if (p != nullptr) buf[u] = ld_nc16(p + 8 * (c - nc8));
+          }
+        }
       }
-      tc::tmem_wait_ld();
-      const float rs = rsc[r];
-      for (int h = 0; h < 32; ++h) {
-        u[h] = (h < G && rr < total)
-                   ? fmaf(rs, __uint_as_float(sv[h]), __uint_as_float(sr[h])) * a.scale
-                   : -INFINITY;
-        if (h < G) stage[r * (G + 1) + h] = u[h];
+      // -- whole-query launch: fold the previous tile while the loads fly
+      if (!kSplit && pend_fold) {
+        if (tid < G) {
+          float mn, al, be;
+          fold_coef(m_run[tid], m_t[tid], mn, al, be);
+          alpha[tid] = al;
+          beta[tid] = be;
+          m_run[tid] = mn;
+          l_run[tid] = fold_val(l_run[tid], al, l_t[tid], be);
+        }
+        __syncthreads();
+        if (tw) {
+          for (int dc = 0; dc < n_dc; ++dc) {
+            const int d = dc * 128 + (warp & 3) * 32 + lane;
+            const bool has_rope = dc >= dc_r0;
+            uint32_t om[16], orp[16], orun[16];
+            tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om);
+            if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp);
+            tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float ot = __uint_as_float(d < dmain ? om[e] : orp[e]);
+              orun[e] = __float_as_uint(fold_val(__uint_as_float(orun[e]), alpha[hb + e], ot, beta[hb + e]));
+            }
+            tc::tmem_st_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+          }
+          tc::tmem_wait_st();
+        }
+        pend_fold = false;
       }
-    }
-    ok = __syncthreads_and(ok) != 0;
-    if (!ok) break;
-    if (warp < 4) {   // warp w, lane h: max over rows 32w .. 32w+31 of head h
-      if (lane < G) {
+      // -- dequantise and store the tile (FP8 -> BF16 is exact)
+#pragma unroll
+      for (int u = 0; u < kMaxLoads; ++u) {
+        const int it = warp + 8 * u;
+        if (it < n_items) {
+          const int r = 8 * (it & 15) + (lane & 7), c = 4 * (it >> 4) + (lane >> 3);
+          uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
+          if (c < nc8) {
+            const uint32_t wv[4] = {buf[u].x, buf[u].y, buf[u].z, buf[u].w};
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+              const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
+              const float2 f = __half22float2(__half2(h2));
+              pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);
+            }
+            *reinterpret_cast<uint4*>(dst + (2 * c) * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(dst + (2 * c + 1) * 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          } else if (c < nc) {
+            *reinterpret_cast<uint4*>(dst + (dmain / 8 + c - nc8) * 128) = buf[u];
+          }
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      tc::tc_fence_after();
+      // -- QK: S^T[rows x heads]
+      if (warp == 0) {
+        if (tc::elect_one()) {
+          const uint32_t ta = tc::smem_u32(tile), tq = tc::smem_u32(qs);
+          for (int ks = 0; ks < Dp / 16; ++ks) {
+            const bool main = 16 * ks < dmain;                // dmain is a multiple of 16
+            const int k0 = main ? 0 : dmain / 16;
+            tc::mma_bf16(tmem + (main ? col_s : col_sr), tc::smem_desc(ta + ks * 256, 128, sbo_rows),
+                         tc::smem_desc(tq + ks * 256, 128, sbo_rows), id_qk, ks > k0 ? 1u : 0u);
+          }
+          tc::mma_commit(bar_qk);
+        }
+        __syncwarp();
+      }
+      // -- logits u = scale * (row scale * S_fp8 + S_rope); empty rows -inf
+      const int r = (warp & 3) * 32 + lane;
+      float u[16];
+      if (tw) {
+        ok = tc::mbar_wait(bar_qk, n_done & 1);
+        tc::tc_fence_after();
+        uint32_t sv[16], sr[16];
+        tc::tmem_ld_x16(tmem + lane_base + col_s + hb, sv);
+        tc::tmem_ld_x16(tmem + lane_base + col_sr + hb, sr);
+        tc::tmem_wait_ld();
+        const bool valid = rowf8[r] != 0;
+        const float rs = rsc[r];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          u[e] = valid ? fmaf(rs, __uint_as_float(sv[e]), __uint_as_float(sr[e])) * a.scale : -INFINITY;
+          stage[r * (G + 1) + hb + e] = u[e];
+        }
+      }
+      ok = __syncthreads_and(ok) != 0;
+      if (!ok) break;
+      if (warp < 4 && lane < G) {   // warp w, lane h: max over rows 32w .. 32w+31 of head h
         float mx = -INFINITY;
         for (int x = 0; x < 32; ++x) mx = fmaxf(mx, stage[(warp * 32 + x) * (G + 1) + lane]);
         part[warp * 32 + lane] = mx;
       }
-    }
-    __syncthreads();
-    if (tid < G) {
-      const float mt = fmaxf(fmaxf(part[tid], part[32 + tid]), fmaxf(part[64 + tid], part[96 + tid]));
-      const float mo = m_run[tid];
-      float c = 1.f;
-      if (mt > mo + kSlack || (mo == -INFINITY && mt > -INFINITY)) {
-        c = (mo == -INFINITY) ? 0.f : expf(mo - mt);
-        m_run[tid] = mt;
-      }
-      corr[tid] = c;
-      l_run[tid] *= c;
-    }
-    if (tid == 0) s_flag = 0;
-    __syncthreads();
-    if (tid < G && corr[tid] != 1.f && tt > 0) s_flag = 1;
-    __syncthreads();
-    // -- rescale the accumulator columns of heads whose running max moved
-    if (s_flag && warp < 4) {
-      for (int dc = 0; dc < n_dc + (n_dc - dc_r0); ++dc) {
-        for (int hb = 0; hb < G; hb += 16) {
-          uint32_t ov[16];
-          const uint32_t addr = tmem + lane_base + col_o + dc * 32 + hb;
-          tc::tmem_ld_x16(addr, ov);
-          tc::tmem_wait_ld();
-          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr[hb + e]);
-          tc::tmem_st_x16(addr, ov);
-        }
-      }
-      tc::tmem_wait_st();
-    }
-    // -- p = exp(u - m_run): P^T (BF16, MN-major) for PV, fp32 copy for the sums
-    if (warp < 4) {
-      const float rs = rsc[r];
-      for (int hg = 0; hg < G / 8; ++hg) {
-        uint32_t pk[4], pm[4];
-        for (int e = 0; e < 8; e += 2) {
-          const int h = hg * 8 + e;
-          const float p0 = expf(u[h] - m_run[h]);
-          const float p1 = expf(u[h + 1] - m_run[h + 1]);
-          stage[r * (G + 1) + h] = p0;
-          stage[r * (G + 1) + h + 1] = p1;
-          pk[e >> 1] = (uint32_t)bf16_rn(p0) | ((uint32_t)bf16_rn(p1) << 16);
-          pm[e >> 1] = (uint32_t)bf16_rn(p0 * rs) | ((uint32_t)bf16_rn(p1 * rs) << 16);
-        }
-        *reinterpret_cast<uint4*>(pt + hg * 2048 + (r >> 3) * 128 + (r & 7) * 16) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(ptm + hg * 2048 + (r >> 3) * 128 + (r & 7) * 16) =
-            make_uint4(pm[0], pm[1], pm[2], pm[3]);
-      }
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    // -- PV: O^T[dims x heads] += V^T P^T
-    if (warp == 0) {
-      if (tc::elect_one()) {
-        const uint32_t ta = tc::smem_u32(tile), tp = tc::smem_u32(pt), tpm = tc::smem_u32(ptm);
-        // FP8 dims: chunks 0 .. n_dc-1 with B = (P*scale)^T; RoPE dims: chunks
-        // dc_r0 .. n_dc-1 again with B = P^T, into their own accumulators
-        for (int x = 0; x < n_dc + (n_dc - dc_r0); ++x) {
-          const bool main = x < n_dc;
-          const int dc = main ? x : dc_r0 + (x - n_dc);
-          for (int ks = 0; ks < kTileRows / 16; ++ks)
-            tc::mma_bf16(tmem + col_o + x * 32, tc::smem_desc(ta + dc * 16 * 128 + ks * 2 * sbo_rows, sbo_rows, 128),
-                         tc::smem_desc((main ? tpm : tp) + ks * 256, 128, 2048), id_pv, (tt > 0 || ks > 0) ? 1u : 0u);
-        }
-        tc::mma_commit(bar_pv);
-      }
-      __syncwarp();
-    }
-    // -- row sums of p for each head (warp w: rows 32w..32w+31), fixed order
-    if (warp < 4 && lane < G) {
-      float sum = 0.f;
-      for (int x = 0; x < 32; ++x) sum += stage[(warp * 32 + x) * (G + 1) + lane];
-      part[warp * 32 + lane] = sum;
-    }
-    __syncthreads();
-    if (tid < G) l_run[tid] += ((part[tid] + part[32 + tid]) + part[64 + tid]) + part[96 + tid];
-  }
-  // ---- finish: out = O e^{m-mu} / (l e^{m-mu} + e^{sink-mu})
-  if (ok && n_tiles > 0) ok = tc::mbar_wait(bar_pv, (n_tiles - 1) & 1);
-  ok = __syncthreads_and(ok) != 0;
-  if (ok) {
-    tc::tc_fence_after();
-    if (tid < G) {
-      const int h = h0 + tid;
-      const float sk = h < H ? a.sink[h] : 0.f;
-      const float mf = fmaxf(m_run[tid], sk);
-      const float cm = expf(m_run[tid] - mf);
-      cmul[tid] = cm;
-      den[tid] = l_run[tid] * cm + expf(sk - mf);
-    }
-    __syncthreads();
-    if (warp < 4) {
-      for (int dc = 0; dc < n_dc; ++dc) {
-        const int d = dc * 128 + tid;
-        // FP8 dims read the scaled accumulator, RoPE dims their own.  TMEM
-        // loads are warp-collective, so a chunk that holds both kinds loads
-        // both and every lane keeps its own.
-        const bool has_rope = dc >= dc_r0;
-        for (int hb = 0; hb < G; hb += 16) {
-          uint32_t om[16], orp[16];
-          tc::tmem_ld_x16(tmem + lane_base + col_o + dc * 32 + hb, om);
-          if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_o + (n_dc + dc - dc_r0) * 32 + hb, orp);
-          tc::tmem_wait_ld();
-          for (int e = 0; e < 16; ++e) {
-            const int h = h0 + hb + e;
-            const float ov = __uint_as_float(d < dmain ? om[e] : orp[e]);
-            if (h < H && d < D)
-              a.out[((int64_t)i * H + h) * D + d] = bf16_rn(__fdiv_rn(ov * cmul[hb + e], den[hb + e]));
+      __syncthreads();
+      if (tid < G) m_t[tid] = fmaxf(fmaxf(part[tid], part[32 + tid]), fmaxf(part[64 + tid], part[96 + tid]));
+      __syncthreads();
+      // -- p = exp(u - m_t): P^T and (P * row scale)^T in BF16 for PV, fp32 p for the sums
+      if (tw) {
+        const float rs = rsc[r];
+#pragma unroll
+        for (int hg = 0; hg < 2; ++hg) {
+          uint32_t pk[4], pm[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int h = hb + hg * 8 + e;
+            const float p0 = expf(u[hg * 8 + e] - m_t[h]);
+            const float p1 = expf(u[hg * 8 + e + 1] - m_t[h + 1]);
+            stage[r * (G + 1) + h] = p0;
+            stage[r * (G + 1) + h + 1] = p1;
+            pk[e >> 1] = (uint32_t)bf16_rn(p0) | ((uint32_t)bf16_rn(p1) << 16);
+            pm[e >> 1] = (uint32_t)bf16_rn(p0 * rs) | ((uint32_t)bf16_rn(p1 * rs) << 16);
           }
+          const int hgl = (hb >> 3) + hg;
+          *reinterpret_cast<uint4*>(pt + hgl * 2048 + (r >> 3) * 128 + (r & 7) * 16) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(ptm + hgl * 2048 + (r >> 3) * 128 + (r & 7) * 16) =
+              make_uint4(pm[0], pm[1], pm[2], pm[3]);
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncthreads();
+      tc::tc_fence_after();
+      // -- PV: O_t^T[dims x heads] = V^T P^T
+      if (warp == 0) {
+        if (tc::elect_one()) {
+          const uint32_t ta = tc::smem_u32(tile), tp = tc::smem_u32(pt), tpm = tc::smem_u32(ptm);
+          for (int x = 0; x < n_acc; ++x) {
+            const bool main = x < n_dc;
+            const int dc = main ? x : dc_r0 + (x - n_dc);
+            for (int ks = 0; ks < kTileRows / 16; ++ks)
+              tc::mma_bf16(tmem + col_ot + x * G,
+                           tc::smem_desc(ta + dc * 16 * 128 + ks * 2 * sbo_rows, sbo_rows, 128),
+                           tc::smem_desc((main ? tpm : tp) + ks * 256, 128, 2048), id_pv, ks > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(bar_pv);
+        }
+        __syncwarp();
+      }
+      ++n_done;
+      // -- l_t: row sums of p per head, fixed order
+      if (warp < 4 && lane < G) {
+        float sum = 0.f;
+        for (int x = 0; x < 32; ++x) sum += stage[(warp * 32 + x) * (G + 1) + lane];
+        part[warp * 32 + lane] = sum;
+      }
+      __syncthreads();
+      if (tid < G) l_t[tid] = ((part[tid] + part[32 + tid]) + part[64 + tid]) + part[96 + tid];
+      pend_fold = true;
+    } else if (kSplit && tid < G && h0 + tid < H) {
+      // a tile without rows: an empty partial
+      a.ws_ml[((int64_t)i * a.tiles_max + tt) * H + h0 + tid] = make_float2(-INFINITY, 0.f);
+    }
+    // -- whole-query launch: addresses of the next tile's rows
+    if (!kSplit && tt + 1 < tt_end) {
+      int nany = 0;
+      if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc) ? 1 : 0;
+      tile_valid = __syncthreads_count(nany) > 0;
+    }
+  }
+
+  if (ok && n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
+  ok = __syncthreads_and(ok) != 0;
+  if (ok && kSplit && n_done > 0) {
+    // ---- split launch: the tile's partial to the workspace
+    tc::tc_fence_after();
+    if (tid < G && h0 + tid < H)
+      a.ws_ml[((int64_t)i * a.tiles_max + tt0) * H + h0 + tid] = make_float2(m_t[tid], l_t[tid]);
+    if (tw) {
+      float* wo = a.ws_o + ((int64_t)i * a.tiles_max + tt0) * H * D;
+      for (int dc = 0; dc < n_dc; ++dc) {
+        const int d = dc * 128 + (warp & 3) * 32 + lane;
+        const bool has_rope = dc >= dc_r0;
+        uint32_t om[16], orp[16];
+        tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om);
+        if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int h = h0 + hb + e;
+          if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(d < dmain ? om[e] : orp[e]);
         }
       }
     }
-  } else if (tid == 0) {
+  } else if (ok && !kSplit) {
+    // ---- whole-query launch: fold the last tile, then out = O e^{m-mu} / (l e^{m-mu} + e^{sink-mu})
+    tc::tc_fence_after();
+    if (tid < G) {
+      float mr = m_run[tid], lr = l_run[tid];
+      if (pend_fold) {
+        float mn, al, be;
+        fold_coef(mr, m_t[tid], mn, al, be);
+        alpha[tid] = al;
+        beta[tid] = be;
+        lr = fold_val(lr, al, l_t[tid], be);
+        mr = mn;
+      }
+      const int h = h0 + tid;
+      float cm, dn;
+      finish_coef(mr, h < H ? a.sink[h] : 0.f, lr, cm, dn);
+      cmul[tid] = cm;
+      den[tid] = dn;
+    }
+    __syncthreads();
+    if (tw) {
+      for (int dc = 0; dc < n_dc; ++dc) {
+        const int d = dc * 128 + (warp & 3) * 32 + lane;
+        const bool has_rope = dc >= dc_r0;
+        uint32_t om[16], orp[16], orun[16];
+        tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+        if (pend_fold) {
+          tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om);
+          if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp);
+        }
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int h = h0 + hb + e;
+          float o = __uint_as_float(orun[e]);
+          if (pend_fold) o = fold_val(o, alpha[hb + e], __uint_as_float(d < dmain ? om[e] : orp[e]), beta[hb + e]);
+          if (h < H && d < D) a.out[((int64_t)i * H + h) * D + d] = finish_val(o, cmul[hb + e], den[hb + e]);
+        }
+      }
+    }
+  } else if (!ok && tid == 0) {
     set_err(L, kErrTimeout, 3000000 + i);
   }
   if (warp == 0) {   // no tcgen05 operation of this CTA is in flight when TMEM is released
@@ -462,21 +583,94 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnTcArgs a) {
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(tmem, 256);
+  if (warp == 0) tc::tmem_dealloc(tmem, n_cols);
 }
 
-size_t attn_tc_smem_bytes(int D, int G, int k) { return (size_t)attn_smem_layout(D, G, k).total + 1024; }
+// Split launch, second step: fold the partials of (query blockIdx.y, head
+// blockIdx.x) in tile order; thread x owns dims 4x .. 4x+3.
+__global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
+  const Layout& L = a.L;
+  const int h = blockIdx.x, i = blockIdx.y, H = L.H, D = L.D;
+  const int d4 = threadIdx.x;
+  if (4 * d4 >= D) return;
+  QueryGeom g;
+  if (!query_geom(a, i, g, false)) return;             // recorded by the partial kernel
+  if (g.n_tiles > a.tiles_max) return;
+  float m = -INFINITY, l = 0.f;
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  const int64_t base = (int64_t)i * a.tiles_max;
+  for (int t0 = 0; t0 < g.n_tiles; t0 += kFoldBatch) {
+    float2 ml[kFoldBatch];
+    float4 v[kFoldBatch];
+#pragma unroll
+    for (int x = 0; x < kFoldBatch; ++x) {
+      if (t0 + x < g.n_tiles) {
+        ml[x] = a.ws_ml[(base + t0 + x) * H + h];
+        v[x] = reinterpret_cast<const float4*>(a.ws_o + ((base + t0 + x) * H + h) * D)[d4];
+      } else {
+        ml[x] = make_float2(-INFINITY, 0.f);
+        v[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < kFoldBatch; ++x) {
+      if (ml[x].x == -INFINITY) continue;
+      float mn, al, be;
+      fold_coef(m, ml[x].x, mn, al, be);
+      l = fold_val(l, al, ml[x].y, be);
+      o[0] = fold_val(o[0], al, v[x].x, be);
+      o[1] = fold_val(o[1], al, v[x].y, be);
+      o[2] = fold_val(o[2], al, v[x].z, be);
+      o[3] = fold_val(o[3], al, v[x].w, be);
+      m = mn;
+    }
+  }
+  float cm, dn;
+  finish_coef(m, a.sink[h], l, cm, dn);
+  uint2 pk;
+  pk.x = (uint32_t)finish_val(o[0], cm, dn) | ((uint32_t)finish_val(o[1], cm, dn) << 16);
+  pk.y = (uint32_t)finish_val(o[2], cm, dn) | ((uint32_t)finish_val(o[3], cm, dn) << 16);
+  *reinterpret_cast<uint2*>(a.out + ((int64_t)i * H + h) * D + 4 * d4) = pk;
+}
+
+size_t attn_tc_smem_bytes(int D, int G) { return (size_t)attn_smem(D, G).total + 1024; }
+
+int attn_tiles_max(const Layout& L, int layer, int k) {
+  const int64_t rows = (layer < L.n_csa ? (int64_t)k : (int64_t)L.max_pages_per_req * kHcaPerPage) + kWindow;
+  return (int)((rows + kTileRows - 1) / kTileRows);
+}
+
+size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k) {
+  const int64_t units = (int64_t)n * attn_tiles_max(L, layer, k) * L.H;
+  return (size_t)(units * L.D * 4 + units * 8);
+}
 
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
-                           cudaStream_t st) {
-  const size_t sm = attn_tc_smem_bytes(L.D, G, k);
+                           void* ws, cudaStream_t st) {
+  const size_t sm = attn_tc_smem_bytes(L.D, G);
   if (sm > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  const bool split = ws != nullptr;
+  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0};
+  const int n_hg = (L.H + G - 1) / G;
+  if (!split) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    attn_tc_kernel<false><<<dim3(n, n_hg), kAttThreads, sm, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+  }
+  a.tiles_max = attn_tiles_max(L, layer, k);
+  a.ws_o = static_cast<float*>(ws);
+  a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + (int64_t)n * a.tiles_max * L.H * L.D * 4);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  AttnTcArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G};
-  dim3 grid(n, (L.H + G - 1) / G);
-  attn_tc_kernel<<<grid, kAttThreads, sm, st>>>(a);
+  attn_tc_kernel<true><<<dim3(a.tiles_max, n_hg, n), kAttThreads, sm, st>>>(a);
+  note_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_fold_kernel<<<dim3(L.H, n), (L.D / 4 + 31) / 32 * 32, 0, st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -16,9 +17,6 @@ namespace csa {
 cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok,
                           const float* c, const float* z, const float* ci, const float* zi,
                           cudaStream_t st);
-cudaError_t launch_index_simt(const Layout& L, int layer, int n, const int32_t* req_ids,
-                              const float* q_idx, const float* w, float* scores, int64_t ld,
-                              int32_t* n_valid, int tiles_per_cta, cudaStream_t st);
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
                             cudaStream_t st);
@@ -26,8 +24,15 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st);
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
-                           cudaStream_t st);
+                           void* ws, cudaStream_t st);
+size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k);
 }  // namespace csa
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void csa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 using csa::Layout;
 
@@ -282,9 +287,17 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
   return CSA_OK;
 }
 
+size_t csa_attn_workspace_bytes(const csa_cache_t* c, int32_t layer, int32_t n, int32_t k) {
+  if (!layer_ok(c, layer) || n < 0 || n > 65535) return 0;
+  const bool is_csa = layer < c->L.n_csa;
+  if (is_csa && (k < 1 || k > 8192)) return 0;
+  return csa::attn_workspace_bytes(c->L, layer, n, is_csa ? k : 0);
+}
+
 csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
                                const uint16_t* q, const int32_t* topk_idx, int32_t k, const float* sink,
-                               float scale, uint16_t* out, csa_variant variant, csa_stream_t stream) {
+                               float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
+                               csa_variant variant, csa_stream_t stream) {
   if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
   if (n == 0) return CSA_OK;
@@ -295,15 +308,26 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
   if (!(scale > 0.f)) return fail(CSA_ERR_ARG, "scale must be > 0");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
   if (is_csa && k > 8192) return fail(CSA_ERR_ARG, "k must be <= 8192");
-  // Heads per CTA: 32 for a well-fed GPU, 16 for an under-fed one (twice the
-  // CTAs per query).  Every per-head operation is independent of the grouping.
-  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 16);
-  const int G = (low || c->L.H <= 16) ? 16 : 32;
-  cudaError_t e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, is_csa ? k : 0, sink, scale,
-                                      out, G, (cudaStream_t)stream);
+  const int kk = is_csa ? k : 0;
+  const size_t need = csa::attn_workspace_bytes(c->L, layer, n, kk);
+  const bool ws_ok = workspace != nullptr && workspace_bytes >= need &&
+                     reinterpret_cast<uintptr_t>(workspace) % 16 == 0;
+  if (variant == CSA_VARIANT_LOW_OCC && !ws_ok)
+    return fail(CSA_ERR_ARG, "the split launch needs a 16-byte aligned workspace of csa_attn_workspace_bytes");
+  // 32 heads per CTA (16 when H <= 16).  Whole-query launch when one CTA per
+  // (query, head group) already covers the SMs, split launch otherwise.  Both
+  // compute the same tiles and fold them in the same order.
+  const int G = c->L.H <= 16 ? 16 : 32;
+  const int ctas = n * ((c->L.H + G - 1) / G);
+  const bool split = variant == CSA_VARIANT_LOW_OCC ||
+                     (variant == CSA_VARIANT_AUTO && ws_ok && ctas < sm_count());
+  cudaError_t e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, kk, sink, scale, out, G,
+                                      split ? workspace : nullptr, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
 }
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 csa_status csa_check_device_error(csa_cache_t* c, csa_stream_t stream) {
   if (!c) return fail(CSA_ERR_ARG, "cache is NULL");

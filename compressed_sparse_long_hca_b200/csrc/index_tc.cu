@@ -385,6 +385,7 @@ cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* re
   }
   IndexTcArgs a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid};
   index_tc_kernel<<<ctas, kThreads, index_tc_smem_bytes(), st>>>(a);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -132,6 +132,9 @@ struct Layout {
   __host__ __device__ static int idx_sf_off(int s, int k) { return 16 * (s & 31) + 4 * (s >> 5) + k; }
 };
 
+// Counts the kernels libcsa has queued (csa_launch_count).
+void note_launch();
+
 // Device error word: first error wins.
 enum DevErr : int32_t {
   kErrNone = 0,

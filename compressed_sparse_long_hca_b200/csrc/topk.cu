@@ -258,10 +258,12 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid,
     e = cudaFuncSetAttribute(topk_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
     if (e != cudaSuccess) return e;
     topk_cluster_kernel<8><<<grid, kTopkThreads, sm, st>>>(a);
+    note_launch();
   } else if (cluster == 4) {
     e = cudaFuncSetAttribute(topk_cluster_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
     if (e != cudaSuccess) return e;
     topk_cluster_kernel<4><<<grid, kTopkThreads, sm, st>>>(a);
+    note_launch();
   } else {
     return cudaErrorInvalidValue;
   }

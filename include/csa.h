@@ -211,23 +211,44 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
 
 /*
  * Multi-query attention of each query over its rows: for CSA layers the
- * entries listed in topk_idx[i][0..k) (-1 = none), for HCA layers
- * (topk_idx == NULL) every completed entry, plus the raw window of positions
- * max(0, t-127) .. t, t = L-1 the query's own position.  K = V = the stored
- * row (FP8 x scale, BF16).  With q rotated at t:
+ * entries listed in topk_idx[i][0..k) in list order (-1 = an empty row), for
+ * HCA layers (topk_idx == NULL) every completed entry in order, then the raw
+ * window of positions max(0, t-127) .. t, t = L-1 the query's own position.
+ * K = V = the stored row (FP8 x scale, BF16).  With q rotated at t:
  *   u_hr = scale * q_h . K_r,  mu_h = max(max_r u_hr, sink_h)
  *   out_h = sum_r e^{u_hr-mu_h} V_r / (sum_r e^{u_hr-mu_h} + e^{sink_h-mu_h})
  *   q     device uint16 (BF16) [n][H][D]   before RoPE
  *   sink  device float [H]
  *   out   device uint16 (BF16) [n][H][D]
- * Rows are visited in a fixed order (selected entries ascending, then the
- * window ascending); one query's reduction is never split across thread
- * blocks.
+ * Source: page "V4终于终于终于终于是来了", sections "CSA——压缩稀疏注意力"
+ * and "HCA——重度压缩注意力".
+ *
+ * Reduction order: the rows are cut into tiles of 128; each tile yields
+ * (max, sum of exponentials, weighted sum of V) and the tiles are folded in
+ * order.  The order depends on the query alone, never on the batch.
+ *
+ * Launch variants (page "DeepSeek不惜代价保住它！V4关键特性被挖出来了",
+ * section "牺牲了什么": two decode-attention kernels for a well-fed and an
+ * under-fed GPU that agree bit for bit):
+ *   CSA_VARIANT_HIGH_OCC  one thread block per (query, 32 heads) walks all
+ *                         tiles; `workspace` is not used (may be NULL).
+ *   CSA_VARIANT_LOW_OCC   one thread block per (query, 32 heads, tile); the
+ *                         tiles' partials go to `workspace` and a second
+ *                         kernel folds them.  Needs workspace_bytes >=
+ *                         csa_attn_workspace_bytes(cache, layer, n, k) and a
+ *                         16-byte aligned workspace, else CSA_ERR_ARG.
+ *   CSA_VARIANT_AUTO      LOW_OCC when the workspace suffices and HIGH_OCC
+ *                         would leave SMs idle, else HIGH_OCC.
+ * All three return identical bits.  The workspace is scratch owned by the
+ * caller; its contents before and after the call are irrelevant, and it must
+ * not be used by other work on the stream until the call's kernels finish.
  */
+size_t     csa_attn_workspace_bytes(const csa_cache_t* cache, int32_t layer, int32_t n, int32_t k);
 csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t n,
                                const int32_t* req_ids, const uint16_t* q,
                                const int32_t* topk_idx, int32_t k, const float* sink,
-                               float scale, uint16_t* out, csa_variant variant,
+                               float scale, uint16_t* out, void* workspace,
+                               size_t workspace_bytes, csa_variant variant,
                                csa_stream_t stream);
 
 /*
@@ -236,6 +257,11 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
  * csa_last_error() then describes it.
  */
 csa_status csa_check_device_error(csa_cache_t* cache, csa_stream_t stream);
+
+/* Number of CUDA kernels libcsa has queued since it was loaded (all
+ * threads, all caches).  A library-side count for measurement, not a
+ * device-side event: the kernels may still be pending. */
+uint64_t   csa_launch_count(void);
 
 /* Thread-local description of the last failing call ("" if none). */
 const char* csa_last_error(void);

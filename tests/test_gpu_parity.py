@@ -260,6 +260,50 @@ def test_attention_on_oracle_written_rows(H, D, R):
             Hp.check_attention(outs[0][i], ref, f"layer {layer} len {T}")
 
 
+@pytest.mark.parametrize("H,D,R", [(32, 160, 32), (128, 512, 64)])
+def test_attention_many_tiles_and_empty_rows(H, D, R):
+    """Rows spanning many 128-row tiles, -1 holes inside the list, tiles with
+    no row at all, and a padded head dim; every launch variant returns the
+    same bits and matches the oracle."""
+    wl = I.Workload("att-tiles", "csa", H=H, D=D, R=R, H_I=4, d_I=32, k=700, W=128, context=0, batch=0,
+                    seed=556)
+    lens = [3000, 40000, 9001]
+    pair = Hp.Pair(wl, 1, 1, max_req=len(lens), capacity=max(lens) + 8)
+    rng = np.random.default_rng(H * D)
+    n = len(lens)
+    q = I.bf16_grid(rng.standard_normal((n, H, D)).astype(np.float32))
+    for layer in (0, 1):
+        csa = layer == 0
+        sink = pair.params[layer]["sink"]
+        ents, wins, sels = [], [], np.full((n, wl.k), -1, np.int32)
+        for i, T in enumerate(lens):
+            if layer == 0:
+                pair.cache.request_alloc(i, T + 8)
+            e, wv = _write_cache_rows(pair, layer, i, T, rng, csa)
+            ents.append(e)
+            wins.append(wv)
+            if csa:
+                N = e.shape[0]
+                pick = np.sort(rng.choice(N, size=min(N, wl.k), replace=False)).astype(np.int32)
+                sels[i, : len(pick)] = pick
+        if csa:
+            sels[0, rng.random(wl.k) < 0.3] = -1               # holes inside the list
+            sels[2, :384] = -1                                 # three tiles without a row
+        outs = []
+        for variant in ("high", "low", "auto"):
+            out = torch.empty((n, H, D), dtype=torch.bfloat16, device="cuda")
+            pair.cache.decode_attn(layer, _t(np.arange(n, dtype=np.int32)), _t(q, torch.bfloat16),
+                                   _t(sels) if csa else None, _t(sink), out, variant=variant)
+            pair.cache.check_device_error()
+            outs.append(out.float().cpu().numpy())
+        assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2]), "variants differ"
+        for i, T in enumerate(lens):
+            rows = ents[i][sels[i][sels[i] >= 0]] if csa else ents[i]
+            rows = np.concatenate([rows, wins[i]], axis=0)
+            ref = O.mqa_attention(O.rope(q[i].astype(np.float64), T - 1, R), rows, sink, 1.0 / math.sqrt(D))
+            Hp.check_attention(outs[0][i], ref, f"layer {layer} len {T}")
+
+
 # ---------------------------------------------------------------- HCA end to end
 
 def test_hca_end_to_end_small():
