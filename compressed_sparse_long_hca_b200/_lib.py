@@ -39,6 +39,7 @@ SIGNATURES = {
     "csa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _I32, _P]),
     "csa_attn_workspace_bytes": (_SZ, [_P, _I32, _I32, _I32]),
     "csa_hca_decode_attn": (_I32, [_P, _I32, _I32, _P, _P, _P, _I32, _P, _F, _P, _P, _SZ, _I32, _P]),
+    "csa_hca_decode_attn_noalloc": (_I32, [_P, _I32, _I32, _P, _P, _P, _I32, _P, _F, _P, _P]),
     "csa_check_device_error": (_I32, [_P, _P]),
     "csa_last_error": (ctypes.c_char_p, []),
     "csa_launch_count": (ctypes.c_uint64, []),

@@ -45,6 +45,8 @@
 //   * softmax statistics of the tile: one thread per (row, 16 heads);
 //   * PV: O_t^T[dims x G] = V^T P^T, P^T in BF16; the FP8 dims use
 //     (P * row scale)^T, the RoPE dims P^T, each into its own accumulator.
+#include <mutex>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -672,6 +674,42 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   attn_fold_kernel<<<dim3(L.H, n), (L.D / 4 + 31) / 32 * 32, 0, st>>>(a);
   note_launch();
   return cudaGetLastError();
+}
+
+// ---- scratch for csa_hca_decode_attn_noalloc
+//
+// For callers that must not allocate device memory: the split launch's
+// partials go to this file-scope array instead of a caller workspace.  Every
+// GPU that loads the library holds it until the process exits.  All calls
+// share it: the partial kernel writes every (tile, head) slot the fold kernel
+// reads, so nothing needs clearing between calls, but calls whose kernels
+// overlap on the GPU race on it.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+constexpr int kNoAllocMaxDevices = 64;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+size_t attn_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress, once per device (by the first call on it), with
+// that device current.
+cudaError_t attn_noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[kNoAllocMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace csa

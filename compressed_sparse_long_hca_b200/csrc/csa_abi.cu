@@ -26,6 +26,8 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
                            void* ws, cudaStream_t st);
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k);
+size_t attn_noalloc_scratch_bytes();
+cudaError_t attn_noalloc_scratch(void** out);
 }  // namespace csa
 
 namespace {
@@ -323,6 +325,36 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
                      (variant == CSA_VARIANT_AUTO && ws_ok && ctas < sm_count());
   cudaError_t e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, kk, sink, scale, out, G,
                                       split ? workspace : nullptr, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return CSA_OK;
+}
+
+csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* c, int32_t layer, int32_t n,
+                                       const int32_t* req_ids, const uint16_t* q, const int32_t* topk_idx,
+                                       int32_t k, const float* sink, float scale, uint16_t* out,
+                                       csa_stream_t stream) {
+  if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
+  if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
+  if (n == 0) return CSA_OK;
+  if (!req_ids || !q || !sink || !out) return fail(CSA_ERR_ARG, "NULL argument");
+  const bool is_csa = layer < c->L.n_csa;
+  if (is_csa && (!topk_idx || k < 1)) return fail(CSA_ERR_ARG, "CSA layer needs topk_idx and k >= 1");
+  if (!is_csa && topk_idx) return fail(CSA_ERR_ARG, "HCA layer takes topk_idx == NULL");
+  if (!(scale > 0.f)) return fail(CSA_ERR_ARG, "scale must be > 0");
+  if (is_csa && k > 8192) return fail(CSA_ERR_ARG, "k must be <= 8192");
+  const int kk = is_csa ? k : 0;
+  const size_t need = csa::attn_workspace_bytes(c->L, layer, n, kk);
+  if (need > csa::attn_noalloc_scratch_bytes())
+    return fail(CSA_ERR_CAPACITY, "this batch needs " + std::to_string(need) +
+                                      " bytes of scratch; the built-in array holds " +
+                                      std::to_string(csa::attn_noalloc_scratch_bytes()) +
+                                      " (use a smaller batch or csa_hca_decode_attn with a workspace)");
+  void* ws = nullptr;
+  cudaError_t e = csa::attn_noalloc_scratch(&ws);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+  const int G = c->L.H <= 16 ? 16 : 32;
+  e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, kk, sink, scale, out, G, ws,
+                          (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
 }

@@ -252,6 +252,33 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
                                csa_stream_t stream);
 
 /*
+ * csa_hca_decode_attn without a caller workspace, for callers that cannot
+ * allocate device memory: an engine whose memory planner hands out every
+ * device buffer ahead of time and forbids allocation while serving, or a
+ * plugin that only receives device pointers and has no allocator of its own.
+ * (The source pages have no counterpart; this is a library convenience.)
+ *
+ * Same arguments and results as csa_hca_decode_attn with
+ * CSA_VARIANT_LOW_OCC (identical bits), except that the tiles' partials go
+ * to a 16 MiB array built into the library instead of `workspace`:
+ *   - every GPU that loads libcsa holds those 16 MiB until the process exits;
+ *   - a batch whose scratch (csa_attn_workspace_bytes) exceeds 16 MiB is
+ *     rejected with CSA_ERR_CAPACITY before anything is launched (C4-sized
+ *     batches of 4 queries x 128 heads x k = 1024 need about 9.5 MiB);
+ *   - the first call on each device looks up the array's device address;
+ *     make that first call before any stream capture;
+ *   - all calls share the array: calls whose kernels may overlap on the GPU
+ *     (different streams, or different threads on one device) race on it and
+ *     must be ordered by the caller.  Nothing in it needs clearing between
+ *     calls.
+ * The call allocates no device memory.
+ */
+csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* cache, int32_t layer, int32_t n,
+                                       const int32_t* req_ids, const uint16_t* q,
+                                       const int32_t* topk_idx, int32_t k, const float* sink,
+                                       float scale, uint16_t* out, csa_stream_t stream);
+
+/*
  * Read and clear the device error word (synchronises `stream`).  Returns
  * CSA_OK or the first device error recorded since the last check;
  * csa_last_error() then describes it.
