@@ -13,11 +13,18 @@
 // [128j, 128j+128); per channel the weights are softmax over the window's
 // tokens of (gate logit + position bias of the token's window slot).
 //
-// Three launches per call, stream-ordered:
+// General call (any n_tok): three launches, stream-ordered:
 //   1. entries: every entry completed by the new tokens (reads tails + input)
 //   2. tokens:  window-ring rows and tail slots of the new tokens
 //   3. length:  L += n_tok
 // Launch 1 reads the tails before launch 2 overwrites them.
+// Decode call (n_tok == 1): one launch, two CTAs per request (the token's
+// ring row and tail slot; the entry it completes, if any).  With one new
+// token the tail slot it overwrites is never one the completed entry reads
+// (the entry's older tokens sit in the other slots of the ring), so the two
+// roles can run concurrently.  Every CTA reads the lengths first and then
+// takes a ticket; the CTA with the last ticket advances the lengths and
+// resets the ticket for the next call.
 #include "common.cuh"
 
 namespace csa {
@@ -68,14 +75,12 @@ __device__ __forceinline__ bool load_request(const AppendArgs& a, int i, int& re
 
 // ---------------------------------------------------------------- launch 1
 
-__global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
-  extern __shared__ float sm[];
+__device__ void csa_entries_body(const AppendArgs& a, int i, int y0, int ystride, float* sm) {
   const Layout& L = a.L;
   const int D = L.D, R = L.R, dI = L.dI;
   float* row = sm;            // [D]
   float* key = sm + D;        // [dI]
   float* red = key + dI;      // [32]
-  const int i = blockIdx.x;
   int req;
   int64_t L0;
   if (!load_request(a, i, req, L0)) return;
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
   const float* tzi = tci + kCsaWin * dI;
   const float* bkv = L.bpos_csa(a.layer);
   const float* bix = L.bpos_idx(a.layer);
-  for (int64_t j = L0 / kCsaM + blockIdx.y; j < n_done; j += gridDim.y) {
+  for (int64_t j = L0 / kCsaM + y0; j < n_done; j += ystride) {
     const int64_t t0 = kCsaM * j - kCsaM;          // first window token (may be < 0)
     for (int ch = threadIdx.x; ch < D + dI; ch += blockDim.x) {
       const bool is_kv = ch < D;
@@ -130,13 +135,11 @@ __global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
   }
 }
 
-__global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
-  extern __shared__ float sm[];
+__device__ void hca_entries_body(const AppendArgs& a, int i, int y0, int ystride, float* sm) {
   const Layout& L = a.L;
   const int D = L.D, R = L.R;
   float* row = sm;
   float* red = sm + D;
-  const int i = blockIdx.x;
   int req;
   int64_t L0;
   if (!load_request(a, i, req, L0)) return;
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
   const float* tc = reinterpret_cast<const float*>(L.tail(req, a.layer));
   const float* tz = tc + kHcaM * D;
   const float* b = L.bpos_hca(a.layer - L.n_csa);
-  for (int64_t j = L0 / kHcaM + blockIdx.y; j < n_done; j += gridDim.y) {
+  for (int64_t j = L0 / kHcaM + y0; j < n_done; j += ystride) {
     const int64_t t0 = kHcaM * j;
     for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
       float mx = -INFINITY;
@@ -176,16 +179,24 @@ __global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  csa_entries_body(a, blockIdx.x, blockIdx.y, gridDim.y, sm);
+}
+
+__global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  hca_entries_body(a, blockIdx.x, blockIdx.y, gridDim.y, sm);
+}
+
 // ---------------------------------------------------------------- launch 2
 
-__global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
-  extern __shared__ float sm[];
+__device__ void tokens_body(const AppendArgs& a, int i, int y0, int ystride, float* sm) {
   const Layout& L = a.L;
   const int D = L.D, R = L.R, dI = L.dI;
   const bool csa = a.layer < L.n_csa;
   float* row = sm;
   float* red = sm + D;
-  const int i = blockIdx.x;
   int req;
   int64_t L0;
   if (!load_request(a, i, req, L0)) return;
@@ -193,7 +204,7 @@ __global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
   char* st = L.state(req, a.layer);
   // window ring rows for positions max(L0, L1-128) .. L1-1
   const int64_t r0 = L1 - kWindow > L0 ? L1 - kWindow : L0;
-  for (int64_t pos = r0 + blockIdx.y; pos < L1; pos += gridDim.y) {
+  for (int64_t pos = r0 + y0; pos < L1; pos += ystride) {
     const float* src = a.c + ((int64_t)i * a.n_tok + (pos - L0)) * D;
     for (int d = threadIdx.x; d < D; d += blockDim.x) row[d] = src[d];
     __syncthreads();
@@ -211,7 +222,7 @@ __global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
   const int ring = csa ? kCsaWin : kHcaM;
   int64_t t_lo = csa ? L1 - kCsaWin : (L1 / kHcaM) * kHcaM;
   if (t_lo < L0) t_lo = L0;
-  for (int64_t pos = t_lo + blockIdx.y; pos < L1; pos += gridDim.y) {
+  for (int64_t pos = t_lo + y0; pos < L1; pos += ystride) {
     const int slot = (int)(pos % ring);
     const int64_t src = (int64_t)i * a.n_tok + (pos - L0);
     for (int d = threadIdx.x; d < D; d += blockDim.x) {
@@ -228,6 +239,11 @@ __global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
   }
 }
 
+__global__ void __launch_bounds__(256) tokens_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  tokens_body(a, blockIdx.x, blockIdx.y, gridDim.y, sm);
+}
+
 // ---------------------------------------------------------------- launch 3
 
 __global__ void length_kernel(AppendArgs a) {
@@ -240,12 +256,49 @@ __global__ void length_kernel(AppendArgs a) {
   if (*len + a.n_tok <= cap) *len += a.n_tok;
 }
 
+// ---------------------------------------------------------------- decode: one launch
+
+// grid (n, 2): blockIdx.y 0 = the token's ring row and tail slot, 1 = the
+// entry it completes (if any).  n_tok == 1.
+__global__ void __launch_bounds__(256) append_decode_kernel(AppendArgs a) {
+  extern __shared__ float sm[];
+  __shared__ int s_last;
+  const Layout& L = a.L;
+  const int i = blockIdx.x;
+  if (blockIdx.y == 0) tokens_body(a, i, 0, 1, sm);
+  else if (a.layer < L.n_csa) csa_entries_body(a, i, 0, 1, sm);
+  else hca_entries_body(a, i, 0, 1, sm);
+  // every read of the lengths by this CTA is done; the last ticket advances them
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(L.ticket(a.layer), 1) == (int)(gridDim.x * gridDim.y) - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int x = threadIdx.x; x < a.n; x += blockDim.x) {
+    const int req = a.req_ids[x];
+    if (req < 0 || req >= L.max_req) continue;
+    int64_t* len = L.lengths() + (int64_t)a.layer * L.max_req + req;
+    const int64_t cap = (int64_t)L.capacity()[req] * kPageTokens;
+    if (*len + a.n_tok <= cap) *len += a.n_tok;
+  }
+  if (threadIdx.x == 0) *L.ticket(a.layer) = 0;
+}
+
 cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok,
                           const float* c, const float* z, const float* ci, const float* zi,
                           cudaStream_t st) {
   AppendArgs a{L, layer, n, req_ids, n_tok, c, z, ci, zi};
   const bool csa = layer < L.n_csa;
   const int threads = 256;
+  if (n_tok == 1) {
+    const size_t sm = (size_t)(L.D + (csa ? L.dI : 0) + 32) * sizeof(float);
+    append_decode_kernel<<<dim3(n, 2), threads, sm, st>>>(a);
+    note_launch();
+    return cudaGetLastError();
+  }
   // entries completed by n_tok new tokens: at most n_tok/m + 1 per request
   const int64_t emax = csa ? n_tok / kCsaM + 1 : n_tok / kHcaM + 1;
   dim3 g1(n, (unsigned)(emax < 1024 ? emax : 1024));

@@ -278,25 +278,35 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       cs[p] = make_float2(c, sn);
     }
     tc::named_bar_sync(1, 128);
-    for (int x = qt; x < G * (Dp / 8); x += 128) {
+    // every load of this thread first (G * Dp / 8 <= 2048 chunks, 16 per thread)
+    constexpr int kQPer = 16;
+    uint4 raw[kQPer];
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+      const int x = qt + 128 * u;
       const int hh = x / (Dp / 8), c = x % (Dp / 8);
-      const int h = h0 + hh;
-      uint32_t pk[4] = {0, 0, 0, 0};
-      if (h < H && 8 * c < D) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(a.q + ((int64_t)i * H + h) * D + 8 * c);
-        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
-        float v[8];
-        for (int e = 0; e < 8; ++e) v[e] = bf16_val((uint16_t)(rw[e >> 1] >> (16 * (e & 1))));
-        if (8 * c >= dmain) {
-          for (int e = 0; e < 8; e += 2) {
-            const float2 w = cs[(8 * c + e - dmain) / 2];
-            const float x0 = v[e], x1 = v[e + 1];
-            v[e] = x0 * w.x - x1 * w.y;
-            v[e + 1] = x0 * w.y + x1 * w.x;
-          }
+      raw[u] = make_uint4(0, 0, 0, 0);
+      if (x < G * (Dp / 8) && h0 + hh < H && 8 * c < D)
+        raw[u] = *reinterpret_cast<const uint4*>(a.q + ((int64_t)i * H + h0 + hh) * D + 8 * c);
+    }
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+      const int x = qt + 128 * u;
+      if (x >= G * (Dp / 8)) break;
+      const int hh = x / (Dp / 8), c = x % (Dp / 8);
+      const uint32_t rw[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      float v[8];
+      for (int e = 0; e < 8; ++e) v[e] = bf16_val((uint16_t)(rw[e >> 1] >> (16 * (e & 1))));
+      if (8 * c >= dmain && 8 * c < D) {
+        for (int e = 0; e < 8; e += 2) {
+          const float2 w = cs[(8 * c + e - dmain) / 2];
+          const float x0 = v[e], x1 = v[e + 1];
+          v[e] = x0 * w.x - x1 * w.y;
+          v[e + 1] = x0 * w.y + x1 * w.x;
         }
-        for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
       }
+      uint32_t pk[4];
+      for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
       *reinterpret_cast<uint4*>(qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16) =
           make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }

@@ -20,10 +20,11 @@
 //     (tcgen05.cp) and issues the block-scaled MMA
 //     D[128 keys x 64 heads] = K^ Q^T (kind::mxf4, M=128, N=64, K=64 per
 //     instruction) into one of four TMEM accumulators;
-//   * epilogue (warps 2-5): read a finished accumulator (one TMEM lane = one key, 64 columns = its 64 head
-//     dot products) and reduce sum_h w_h max(0, d_h) in a fixed order.  At a
-//     query boundary they quantise the next query's index heads to MXFP4 (the
-//     B operand and its scale chunk).
+//   * epilogue (warps 2-9, two groups of four warps taking alternate tiles):
+//     read a finished accumulator (one TMEM lane = one key, 64 columns = its
+//     64 head dot products) and reduce sum_h w_h max(0, d_h) in a fixed
+//     order.  At a query boundary they quantise the next query's index heads
+//     to MXFP4 (the B operand and its scale chunk).
 // Every key's score comes from the same instruction sequence whatever the
 // grid, so launch variants and batch compositions return identical bits.
 // All waits are bounded: a stuck pipeline records a timeout in the device
@@ -37,8 +38,10 @@ namespace {
 
 constexpr int kStages = 8;             // shared-memory stages of key tiles
 constexpr int kNA = 3;                 // TMEM accumulators (and key-scale buffers)
-constexpr int kEpiThreads = 128;
-constexpr int kThreads = 64 + kEpiThreads;   // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+constexpr int kEpiGroups = 2;          // epilogue groups, alternate tiles
+constexpr int kGroupThreads = 128;     // one thread per key of a tile
+constexpr int kEpiThreads = kEpiGroups * kGroupThreads;
+constexpr int kThreads = 64 + kEpiThreads;   // warp 0 producer, warp 1 MMA, warps 2-9 epilogue
 constexpr int kCtasPerSm = 2;          // two CTAs per SM overlap their issue latencies
 constexpr int kHeadsN = 64;            // MMA N (index heads, zero padded)
 constexpr int kMaxCh = 4;              // d_I / 32 <= 4
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.stage_empty[s], 1); }
-    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], kEpiThreads); }
+    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], kGroupThreads); }
     tc::mbar_init(&sm.q_ready, 1);
     tc::mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -262,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
     } else {
       // ================= epilogue warps =================
       const int et = tid - 64;                       // 0 .. kEpiThreads-1
+      const int grp = et / kGroupThreads;            // this group takes tiles u with u % kEpiGroups == grp
       const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
       const int key_in_tile = (warp & 3) * 32 + lane;
       uint32_t u = u_base;
@@ -309,31 +313,36 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
         tc::named_bar_sync(1, kEpiThreads);
         if (et == 0) tc::mbar_arrive(&sm.q_ready);
         float* out = a.scores + (int64_t)qq * a.ld;
-        for (int k = 0; k < nt && ok; ++k) {
+        for (int k = (int)((grp + kEpiGroups - (int)(u % kEpiGroups)) % kEpiGroups); k < nt && ok;
+             k += kEpiGroups) {
           const uint32_t uk = u + (uint32_t)k;
           const int na = uk % kNA;
           if (!(ok = wait_or_abort(sm, &sm.acc_full[na], (uk / kNA) & 1))) break;
           tc::tc_fence_after();
-          uint32_t r[64];
+          // two halves of 32 head columns (fewer live registers); four
+          // interleaved partial sums (heads h = 4i + p), combined in a fixed order
           const uint32_t col = tmem + lane_base + 64 * na;
-          tc::tmem_ld_x16(col + 0, r);
-          tc::tmem_ld_x16(col + 16, r + 16);
-          tc::tmem_ld_x16(col + 32, r + 32);
-          tc::tmem_ld_x16(col + 48, r + 48);
-          tc::tmem_wait_ld();
-          tc::tc_fence_before();
-          tc::mbar_arrive(&sm.acc_empty[na]);
-          // four interleaved partial sums (heads h = 4i + p), combined in a fixed order
-          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
           const float4* w4 = reinterpret_cast<const float4*>(sm.w);
+          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
-          for (int h4 = 0; h4 < kHeadsN / 4; ++h4) {
-            if (h4 * 4 < HI) {
-              const float4 wv = w4[h4];
-              p0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), p0);
-              p1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), p1);
-              p2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), p2);
-              p3 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), p3);
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r[32];
+            tc::tmem_ld_x16(col + 32 * half, r);
+            tc::tmem_ld_x16(col + 32 * half + 16, r + 16);
+            tc::tmem_wait_ld();
+            if (half == 1) {
+              tc::tc_fence_before();
+              tc::mbar_arrive(&sm.acc_empty[na]);
+            }
+#pragma unroll
+            for (int h4 = 0; h4 < 8; ++h4) {
+              if (32 * half + h4 * 4 < HI) {
+                const float4 wv = w4[8 * half + h4];
+                p0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), p0);
+                p1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), p1);
+                p2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), p2);
+                p3 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), p3);
+              }
             }
           }
           const int64_t j = (t0 + k) * kCsaPerPage + key_in_tile;

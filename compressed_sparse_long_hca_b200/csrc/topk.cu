@@ -5,22 +5,37 @@
 // entries.  Selection rule (fixed here): the k largest scores, equal scores
 // going to the lower index, -0.0 == +0.0, output ascending, -1 padding.
 //
-// Method: an exact radix select on order-preserving 32-bit keys, run by one
-// thread-block cluster per query.  Each CTA of the cluster owns a contiguous
-// slice of the query's scores (kept in shared memory when it fits).  Three
-// passes (11, 11 and 10 bits) build shared-memory histograms of the keys
-// that still match the prefix found so far; the cluster adds its histograms
-// through distributed shared memory and every CTA reads off the same digit.
-// The passes end with the k-th largest key T and the number of ties at T
-// that still fit.  The output pass exchanges per-CTA counts, so that each
-// CTA writes its selected indices (all keys > T, then ties at T in index
-// order) at the right place of the ascending list.  Integer histograms and
-// ordered prefix sums make the result independent of thread scheduling and
-// of the cluster's launch shape; the cluster barriers are hardware barriers,
-// no thread spins on memory.
+// Scores become order-preserving 32-bit keys.  One thread-block cluster per
+// query; each CTA owns a contiguous slice of the query's keys, which one bulk
+// copy brings into shared memory when it fits.
+//
+// Filter path (the usual case).
+//   1. Threshold.  Every CTA reads the same strided sample of S keys and
+//      takes tau = the sample's r-th largest key, r chosen so that with
+//      overwhelming probability fewer than r sampled keys lie above the
+//      query's k-th key; then every key of the top k is >= tau, and about
+//      r N / S keys pass, whatever the scores' distribution.  (Correctness
+//      never depends on the sample: step 3 checks that at least k keys pass.)
+//   2. Filter.  Each CTA counts its keys >= tau (warp ballots), the cluster
+//      exchanges the counts through distributed shared memory, and each CTA
+//      writes its passing (key, index) pairs, in index order, into the leader
+//      CTA's candidate list at its offset.
+//   3. Select.  If between k and kCandCap keys passed, the leader finds the
+//      k-th largest candidate key T: one histogram of the candidates over
+//      2048 equal bins of [tau, max] finds T's bin, and the few keys in that
+//      bin are ranked against each other.  It then writes, in index order,
+//      every candidate > T and the first k - #(> T) candidates == T.
+// Radix path (when the filter does not apply, e.g. a tie class larger than
+// kCandCap): an exact three-pass radix select (11, 11, 10 bits) with
+// cluster-summed histograms, then an ordered output walk over the slices.
+// Both paths are exact, so they return the same indices; integer counts and
+// ordered prefix sums make the result independent of scheduling and of the
+// cluster's size.  Cluster barriers are hardware barriers; the one wait on
+// memory (the bulk copy's mbarrier) gives up after a time limit.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -29,8 +44,12 @@ namespace csa {
 namespace {
 
 constexpr int kTopkThreads = 1024;
+constexpr int kWarps = kTopkThreads / 32;
 constexpr int kBins = 2048;                // 11-bit digits
-constexpr int kMaxCluster = 8;
+constexpr int kSample = 4096;              // sampled keys for the threshold
+constexpr int kSamplePer = kSample / kTopkThreads;
+constexpr int kCandCap = 8192;             // candidate list capacity
+constexpr int kCandPer = kCandCap / kTopkThreads;
 
 __device__ __forceinline__ uint32_t order_key(float s) {
   const uint32_t b = __float_as_uint(s + 0.0f);       // -0.0 -> +0.0
@@ -45,8 +64,31 @@ struct TopkArgs {
   int k;
   int32_t* out;
   int32_t* err;          // device error word (may be null)
-  int cache_keys;        // slices fit in shared memory
-  int64_t slice_cap;     // keys per CTA slice buffer
+  int cache_keys;        // every CTA's slice fits in shared memory
+};
+
+struct RadixBufs {
+  int hist[kBins];          // this CTA's histogram
+  int slice_sum[kBins];     // summed bins owned by this CTA
+  int full[kBins];          // the cluster's summed histogram
+};
+
+struct TopkShared {
+  union {
+    uint2 cand[kCandCap];   // filter path (leader): (key, index) of the candidates, index order
+    RadixBufs rx;           // radix path
+  } u;
+  int sel_hist[kBins];      // histogram of block_select
+  uint32_t list[kTopkThreads];  // block_select: the keys of one bin
+  int wsum[32];
+  uint32_t mm[2][32];       // per-warp min / max
+  int cnt[2];               // radix path: this CTA's (count > T, count == T)
+  int n_cand;               // filter path: this CTA's keys >= tau
+  int n_list;
+  int bin_count;
+  uint32_t digit;
+  int remaining;
+  uint64_t bar;             // bulk copy of the slice
 };
 
 // Exclusive block-wide prefix sum over kTopkThreads threads; returns the total.
@@ -74,63 +116,113 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   return before;
 }
 
-struct TopkShared {
-  int hist[kBins];          // this CTA's histogram
-  int slice_sum[kBins];     // reduce-scatter: summed bins owned by this CTA
-  int full[kBins];          // the cluster's summed histogram
-  int wsum[32];
-  int cnt[2];               // this CTA's (count > T, count == T)
-  uint32_t digit;
-  int remaining;
-};
+// Block-wide (min, max) of E keys per thread (flags mark the valid ones).
+template <int E>
+__device__ __forceinline__ void block_minmax(const uint32_t (&v)[E], const bool (&ok)[E], uint32_t (*mm)[32],
+                                             uint32_t* mn, uint32_t* mx) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t a = 0xFFFFFFFFu, b = 0u;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (ok[e]) { a = min(a, v[e]); b = max(b, v[e]); }
+  a = __reduce_min_sync(0xffffffffu, a);
+  b = __reduce_max_sync(0xffffffffu, b);
+  if (lane == 0) { mm[0][w] = a; mm[1][w] = b; }
+  __syncthreads();
+  *mn = __reduce_min_sync(0xffffffffu, mm[0][lane]);
+  *mx = __reduce_max_sync(0xffffffffu, mm[1][lane]);
+  __syncthreads();
+}
 
-}  // namespace
-
-template <int C>
-__global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(TopkArgs a) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int i = blockIdx.y;
+// The r-th largest of the valid keys (1 <= r <= #valid, every valid key in
+// [kmin, kmax]), exactly: returns T and sets *ties = r - #{keys > T}.  Each
+// round histograms the keys of the current range over up to 2048 equal
+// bins and keeps the bin that holds the r-th key; once that bin holds at
+// most kTopkThreads keys they are ranked against each other.  With
+// exact == false the first round's bin is kept and its lower edge returned
+// (then #{keys >= result} >= r).
+template <int E>
+__device__ uint32_t block_select(const uint32_t (&v)[E], const bool (&ok)[E], int r, uint32_t kmin, uint32_t kmax,
+                                 bool exact, TopkShared& sh, int* ties) {
   const int tid = threadIdx.x;
-  const float* s = a.scores + (int64_t)i * a.ld;
-  int32_t* out = a.out + (int64_t)i * a.k;
-  int64_t N = a.n_valid[i];
-  if (N < 0 || N > a.ld) {
-    if (rank == 0 && tid == 0 && a.err) {
-      if (atomicCAS(a.err, 0, (int32_t)kErrLd) == 0) a.err[1] = i;
-    }
-    N = 0;
-  }
-  const int k = a.k;
-  if (N <= k) {   // every entry is selected: indices in order, then -1
-    for (int64_t j = (int64_t)rank * kTopkThreads + tid; j < k; j += (int64_t)C * kTopkThreads)
-      out[j] = j < N ? (int32_t)j : -1;
-    return;       // uniform for the whole cluster (N is the cluster's)
-  }
-  const int64_t chunk = (N + C - 1) / C;
-  const int64_t lo = (int64_t)rank * chunk;
-  const int64_t hi = lo + chunk < N ? lo + chunk : N;
-  const int64_t len = hi > lo ? hi - lo : 0;
-  auto key_at = [&](int64_t x) -> uint32_t { return a.cache_keys ? keys[x] : order_key(s[lo + x]); };
-  if (a.cache_keys) {
-    // eight loads in flight per thread before any of them is used
-    for (int64_t x0 = tid; x0 < len; x0 += 8 * kTopkThreads) {
-      float v[8];
+  uint64_t base = kmin, width = (uint64_t)kmax - kmin + 1;
+  int remaining = r;
+  while (true) {
+    int shift = 0;
+    while (((width - 1) >> shift) >= (uint64_t)kBins) ++shift;
+    for (int b = tid; b < kBins; b += kTopkThreads) sh.sel_hist[b] = 0;
+    __syncthreads();
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t x = x0 + (int64_t)u * kTopkThreads;
-        v[u] = x < len ? s[lo + x] : 0.f;
+    for (int e = 0; e < E; ++e)
+      if (ok[e] && (uint64_t)v[e] >= base && (uint64_t)v[e] - base < width)
+        atomicAdd(&sh.sel_hist[((uint64_t)v[e] - base) >> shift], 1);
+    __syncthreads();
+    {   // bin d: (count in bins > d) < remaining <= (count in bins >= d); 2 bins per thread, top first
+      const int b0 = kBins - 2 - 2 * tid;
+      const int c1 = sh.sel_hist[b0 + 1], c0 = sh.sel_hist[b0];
+      int tot;
+      const int before = block_excl_scan(c1 + c0, sh.wsum, &tot);
+      if (before < remaining && before + c1 >= remaining) {
+        sh.digit = (uint32_t)(b0 + 1);
+        sh.remaining = remaining - before;
+        sh.bin_count = c1;
+      } else if (before + c1 < remaining && before + c1 + c0 >= remaining) {
+        sh.digit = (uint32_t)b0;
+        sh.remaining = remaining - before - c1;
+        sh.bin_count = c0;
       }
+      __syncthreads();
+    }
+    const uint64_t d = sh.digit;
+    const int in_bin = sh.bin_count;
+    remaining = sh.remaining;
+    base += d << shift;
+    const uint64_t left = width - (d << shift);
+    width = left < ((uint64_t)1 << shift) ? left : ((uint64_t)1 << shift);
+    if (shift == 0) {
+      *ties = remaining;
+      return (uint32_t)base;
+    }
+    if (!exact) {
+      *ties = 0;
+      return (uint32_t)base;
+    }
+    if (in_bin <= kTopkThreads) {   // rank the bin's keys against each other
+      if (tid == 0) sh.n_list = 0;
+      __syncthreads();
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t x = x0 + (int64_t)u * kTopkThreads;
-        if (x < len) keys[x] = order_key(v[u]);
+      for (int e = 0; e < E; ++e)
+        if (ok[e] && (uint64_t)v[e] >= base && (uint64_t)v[e] - base < width) sh.list[atomicAdd(&sh.n_list, 1)] = v[e];
+      __syncthreads();
+      const int m = sh.n_list;
+      if (tid < m) {
+        const uint32_t x = sh.list[tid];
+        int gt = 0, ge = 0;
+        for (int y = 0; y < m; ++y) {
+          const uint32_t z = sh.list[y];
+          gt += z > x ? 1 : 0;
+          ge += z >= x ? 1 : 0;
+        }
+        if (gt < remaining && remaining <= ge) {   // equal keys write equal values
+          sh.digit = x;
+          sh.remaining = remaining - gt;
+        }
       }
+      __syncthreads();
+      *ties = sh.remaining;
+      const uint32_t T = sh.digit;
+      __syncthreads();
+      return T;
     }
   }
+}
+
+// Radix path: the k-th largest key of the query (all CTAs of the cluster)
+// and how many keys equal to it are selected.
+template <int C>
+__device__ void radix_select(cg::cluster_group& cluster, TopkShared& sh, const float* s, int64_t lo, int64_t len,
+                             int k, uint32_t* T_out, int* ties_out) {
+  const int tid = threadIdx.x, rank = (int)cluster.block_rank();
   if (tid == 0) { sh.digit = 0; sh.remaining = k; }
   uint32_t prefix = 0;
   int remaining = k;
@@ -139,40 +231,40 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   for (int p = 0; p < 3; ++p) {
     const int shift = shifts[p], width = widths[p];
     const uint32_t mask = (1u << width) - 1;
-    for (int b = tid; b < kBins; b += kTopkThreads) sh.hist[b] = 0;
+    for (int b = tid; b < kBins; b += kTopkThreads) sh.u.rx.hist[b] = 0;
     __syncthreads();
-    // lanes that hit the same bin add once (score distributions pile up in a
-    // few top-bit bins, where per-lane atomics would serialise)
+    // lanes that hit the same bin add once
     for (int64_t x0 = tid - (tid & 31); x0 < len; x0 += kTopkThreads) {
       const int64_t x = x0 + (tid & 31);
-      const uint32_t key = x < len ? key_at(x) : 0u;
+      const uint32_t key = x < len ? order_key(s[lo + x]) : 0u;
       const bool hit = x < len && (p == 0 || (key >> (shift + width)) == prefix);
       const uint32_t bin = hit ? (key >> shift) & mask : 0xFFFFFFFFu;
       if (!__any_sync(0xffffffffu, hit)) continue;
       const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (hit && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
+      if (hit && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.u.rx.hist[bin], __popc(peers));
     }
     // cluster reduce-scatter: CTA r sums bins [r*kBins/C, (r+1)*kBins/C)
     cluster.sync();
     constexpr int per = kBins / C;
     for (int b = tid; b < per; b += kTopkThreads) {
       int t = 0;
-      for (int r = 0; r < C; ++r) t += cluster.map_shared_rank(&sh.hist[0], r)[rank * per + b];
-      sh.slice_sum[b] = t;
+      for (int r = 0; r < C; ++r) t += cluster.map_shared_rank(&sh.u.rx.hist[0], r)[rank * per + b];
+      sh.u.rx.slice_sum[b] = t;
     }
     cluster.sync();
     for (int b = tid; b < kBins; b += kTopkThreads)
-      sh.full[b] = cluster.map_shared_rank(&sh.slice_sum[0], b / per)[b % per];
+      sh.u.rx.full[b] = cluster.map_shared_rank(&sh.u.rx.slice_sum[0], b / per)[b % per];
     __syncthreads();
     // digit d: the largest d with (count of digits > d) < remaining <= (count of digits >= d)
     {
-      // suffix sums over bins, 2 bins per thread (kBins = 2 * kTopkThreads)
-      const int b0 = kBins - 2 - 2 * tid;        // thread 0 owns the top bins
-      const int c1 = sh.full[b0 + 1], c0 = sh.full[b0];
+      const int b0 = kBins - 2 - 2 * tid;        // 2 bins per thread, thread 0 owns the top bins
+      const int c1 = sh.u.rx.full[b0 + 1], c0 = sh.u.rx.full[b0];
       int tot;
-      const int before = block_excl_scan(c1 + c0, sh.wsum, &tot);   // counts of bins above b0 + 1
-      if (before < remaining && before + c1 >= remaining) { sh.digit = (uint32_t)(b0 + 1); sh.remaining = remaining - before; }
-      else if (before + c1 < remaining && before + c1 + c0 >= remaining) {
+      const int before = block_excl_scan(c1 + c0, sh.wsum, &tot);
+      if (before < remaining && before + c1 >= remaining) {
+        sh.digit = (uint32_t)(b0 + 1);
+        sh.remaining = remaining - before;
+      } else if (before + c1 < remaining && before + c1 + c0 >= remaining) {
         sh.digit = (uint32_t)b0;
         sh.remaining = remaining - before - c1;
       }
@@ -180,29 +272,32 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     }
     prefix = (prefix << width) | sh.digit;
     remaining = sh.remaining;
-    // the histogram buffers are read remotely until every CTA has its copy
-    cluster.sync();
+    cluster.sync();   // histograms are read remotely until every CTA has its copy
   }
-  const uint32_t T = prefix;        // the k-th largest key
-  const int ties_needed = remaining;
-  // ---- output: each warp owns a contiguous sub-slice, walked 32 keys at a
-  //      time (lane l reads key base + l: conflict-free), so that ballots
-  //      give ordered positions.
+  *T_out = prefix;
+  *ties_out = remaining;
+}
+
+// Radix path output: each warp owns a contiguous sub-slice, walked 32 keys
+// at a time, so that ballots give ordered positions.
+template <int C>
+__device__ void radix_output(cg::cluster_group& cluster, TopkShared& sh, const float* s, int64_t lo, int64_t len,
+                             uint32_t T, int ties_needed, int32_t* out) {
+  const int tid = threadIdx.x, rank = (int)cluster.block_rank();
   const int lane = tid & 31, wid = tid >> 5;
-  constexpr int kWarps = kTopkThreads / 32;
   const int64_t per_w = ((len + kWarps - 1) / kWarps + 31) / 32 * 32;
   const int64_t w_lo = (int64_t)wid * per_w < len ? (int64_t)wid * per_w : len;
   const int64_t w_hi = w_lo + per_w < len ? w_lo + per_w : len;
   const unsigned lt_mask = (1u << lane) - 1u;
-  int gt = 0, eq = 0;   // warp totals (uniform across the warp)
+  int gt = 0, eq = 0;
   for (int64_t x0 = w_lo; x0 < w_hi; x0 += 32) {
     const int64_t x = x0 + lane;
-    const uint32_t key = x < w_hi ? key_at(x) : 0u;
+    const uint32_t key = x < w_hi ? order_key(s[lo + x]) : 0u;
     gt += __popc(__ballot_sync(0xffffffffu, x < w_hi && key > T));
     eq += __popc(__ballot_sync(0xffffffffu, x < w_hi && key == T));
   }
   int gt_tot, eq_tot;
-  const int gt_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? gt : 0, sh.wsum, &gt_tot), 0);
+  (void)block_excl_scan(lane == 0 ? gt : 0, sh.wsum, &gt_tot);
   const int eq_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? eq : 0, sh.wsum, &eq_tot), 0);
   if (tid == 0) { sh.cnt[0] = gt_tot; sh.cnt[1] = eq_tot; }
   cluster.sync();
@@ -219,7 +314,6 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
       tb += e;
     }
   }
-  // ties this warp may take: those among the CTA's first take_cta ties
   int w_ties = take_cta - eq_before;
   w_ties = w_ties < 0 ? 0 : (w_ties > eq ? eq : w_ties);
   int tot_sel;
@@ -228,7 +322,7 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   int ties_seen = 0;
   for (int64_t x0 = w_lo; x0 < w_hi; x0 += 32) {
     const int64_t x = x0 + lane;
-    const uint32_t key = x < w_hi ? key_at(x) : 0u;
+    const uint32_t key = x < w_hi ? order_key(s[lo + x]) : 0u;
     const bool is_eq = x < w_hi && key == T;
     const unsigned eqb = __ballot_sync(0xffffffffu, is_eq);
     const int tie_rank = ties_seen + __popc(eqb & lt_mask);
@@ -238,29 +332,204 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     pos += __popc(tb);
     ties_seen += __popc(eqb);
   }
-  (void)gt_before;
-  // no CTA may leave while others still read its shared memory
+}
+
+}  // namespace
+
+template <int C>
+__global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) topk_cluster_kernel(TopkArgs a) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + (sizeof(TopkShared) + 127) / 128 * 128);
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int i = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const float* s = a.scores + (int64_t)i * a.ld;
+  int32_t* out = a.out + (int64_t)i * a.k;
+  int64_t N = a.n_valid[i];
+  if (N < 0 || N > a.ld) {
+    if (rank == 0 && tid == 0 && a.err) {
+      if (atomicCAS(a.err, 0, (int32_t)kErrLd) == 0) a.err[1] = i;
+    }
+    N = 0;
+  }
+  const int k = a.k;
+  if (N <= k) {   // every entry is selected: indices in order, then -1
+    for (int64_t j = (int64_t)rank * kTopkThreads + tid; j < k; j += (int64_t)C * kTopkThreads)
+      out[j] = j < N ? (int32_t)j : -1;
+    return;       // uniform for the whole cluster (N is the cluster's)
+  }
+  const int64_t chunk = ((N + C - 1) / C + 3) / 4 * 4;
+  const int64_t lo = (int64_t)rank * chunk < N ? (int64_t)rank * chunk : N;
+  const int64_t hi = lo + chunk < N ? lo + chunk : N;
+  const int64_t len = hi - lo;
+
+  // ---- slice -> shared memory: one bulk copy of the 16-byte aligned part
+  const bool cached = a.cache_keys != 0;
+  const bool bulk = cached && ((reinterpret_cast<uintptr_t>(s + lo) & 15) == 0);
+  const int64_t nbulk = bulk ? len / 4 * 4 : 0;
+  if (cached && tid == 0) {
+    tc::mbar_init(&sh.bar, 1);
+    tc::fence_mbar_init();
+    tc::mbar_arrive_expect_tx(&sh.bar, (uint32_t)(nbulk * 4));
+    for (int64_t x = 0; x < nbulk; x += 8192) {
+      const int64_t m = nbulk - x < 8192 ? nbulk - x : 8192;
+      tc::bulk_g2s(keys + x, s + lo + x, (uint32_t)(m * 4), &sh.bar);
+    }
+  }
+  if (cached)
+    for (int64_t x = nbulk + tid; x < len; x += kTopkThreads) keys[x] = __float_as_uint(s[lo + x]);
+  __syncthreads();   // the mbarrier is initialised before anyone waits on it
+
+  // ---- 1. threshold from a strided sample (the same sample in every CTA)
+  const int S = N < kSample ? (int)N : kSample;
+  uint32_t sv[kSamplePer];
+  bool sok[kSamplePer];
+#pragma unroll
+  for (int e = 0; e < kSamplePer; ++e) {
+    const int x = tid + e * kTopkThreads;
+    sok[e] = x < S;
+    sv[e] = sok[e] ? order_key(s[(int64_t)x * N / S]) : 0u;
+  }
+  const float lam = (float)k * (float)S / (float)N;     // expected sampled keys above the k-th
+  const int r = (int)ceilf(lam + 6.f * sqrtf(lam) + 8.f);
+  uint32_t tau = 0;
+  if (r <= S) {
+    uint32_t smin, smax;
+    int unused;
+    block_minmax(sv, sok, sh.mm, &smin, &smax);
+    tau = block_select(sv, sok, r, smin, smax, true, sh, &unused);
+  }
+  if (cached) {
+    // all threads observe the copy's completion (bounded wait)
+    const bool arrived = __syncthreads_and(tc::mbar_wait(&sh.bar, 0)) != 0;
+    if (!arrived) {
+      if (tid == 0 && a.err && atomicCAS(a.err, 0, (int32_t)kErrTimeout) == 0) a.err[1] = i;
+      return;
+    }
+  }
+  auto key_at = [&](int64_t x) -> uint32_t { return cached ? order_key(__uint_as_float(keys[x])) : order_key(s[lo + x]); };
+
+  // ---- 2. filter: count, exchange counts, write candidates to the leader
+  const int64_t per_w = ((len + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t w_lo = (int64_t)wid * per_w < len ? (int64_t)wid * per_w : len;
+  const int64_t w_hi = w_lo + per_w < len ? w_lo + per_w : len;
+  int wc = 0;
+  for (int64_t x0 = w_lo; x0 < w_hi; x0 += 8 * 32) {
+    uint32_t kv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t x = x0 + u * 32 + lane;
+      kv[u] = x < w_hi ? key_at(x) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t x = x0 + u * 32 + lane;
+      wc += __popc(__ballot_sync(0xffffffffu, x < w_hi && kv[u] >= tau));
+    }
+  }
+  int cta_cnt;
+  const int w_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? wc : 0, sh.wsum, &cta_cnt), 0);
+  if (tid == 0) sh.n_cand = cta_cnt;
   cluster.sync();
+  int base = 0, total = 0;
+  for (int q = 0; q < C; ++q) {
+    const int c = *cluster.map_shared_rank(&sh.n_cand, q);
+    if (q < rank) base += c;
+    total += c;
+  }
+  const bool filter = total >= k && total <= kCandCap;   // the same in every CTA
+  if (filter) {
+    uint2* lc = cluster.map_shared_rank(&sh.u.cand[0], 0);
+    int pos = base + w_before;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int64_t x0 = w_lo; x0 < w_hi; x0 += 8 * 32) {
+      uint32_t kv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t x = x0 + u * 32 + lane;
+        kv[u] = x < w_hi ? key_at(x) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t x = x0 + u * 32 + lane;
+        const bool pass = x < w_hi && kv[u] >= tau;
+        const unsigned b = __ballot_sync(0xffffffffu, pass);
+        if (pass) lc[pos + __popc(b & lt_mask)] = make_uint2(kv[u], (uint32_t)(lo + x));
+        pos += __popc(b);
+      }
+    }
+    cluster.sync();   // the leader's list is complete; nobody reads another CTA after this
+    if (rank != 0) return;
+
+    // ---- 3. exact selection among the candidates (leader)
+    const int M = total;
+    uint32_t cv[kCandPer];
+    bool cok[kCandPer];
+    const int e0 = tid * kCandPer;                     // contiguous run, index order
+#pragma unroll
+    for (int e = 0; e < kCandPer; ++e) {
+      cok[e] = e0 + e < M;
+      cv[e] = cok[e] ? sh.u.cand[e0 + e].x : 0u;
+    }
+    uint32_t cmin, cmax;
+    block_minmax(cv, cok, sh.mm, &cmin, &cmax);
+    int ties_needed;
+    const uint32_t T = block_select(cv, cok, k, tau, cmax, true, sh, &ties_needed);
+    int neq = 0;
+#pragma unroll
+    for (int e = 0; e < kCandPer; ++e) neq += (cok[e] && cv[e] == T) ? 1 : 0;
+    int eq_tot;
+    const int eq_before = block_excl_scan(neq, sh.wsum, &eq_tot);
+    int take = 0, seen = eq_before;
+    unsigned take_bits = 0;
+#pragma unroll
+    for (int e = 0; e < kCandPer; ++e) {
+      const bool is_eq = cok[e] && cv[e] == T;
+      const bool t = cok[e] && (cv[e] > T || (is_eq && seen < ties_needed));
+      seen += is_eq ? 1 : 0;
+      if (t) { take_bits |= 1u << e; ++take; }
+    }
+    int tot_sel;
+    int p = block_excl_scan(take, sh.wsum, &tot_sel);
+#pragma unroll
+    for (int e = 0; e < kCandPer; ++e)
+      if (take_bits & (1u << e)) out[p++] = (int32_t)sh.u.cand[e0 + e].y;
+    return;
+  }
+
+  // ---- radix path (every CTA of the cluster)
+  uint32_t T;
+  int ties_needed;
+  radix_select<C>(cluster, sh, s, lo, len, k, &T, &ties_needed);
+  radix_output<C>(cluster, sh, s, lo, len, T, ties_needed, out);
+  cluster.sync();   // no CTA may leave while others still read its shared memory
+}
+
+size_t topk_smem_bytes(int64_t ld, int cluster, bool* cache) {
+  const int64_t chunk = ((ld + cluster - 1) / cluster + 3) / 4 * 4;
+  const size_t base = (sizeof(TopkShared) + 127) / 128 * 128;
+  const size_t with = base + (size_t)chunk * 4;
+  *cache = with <= 227 * 1024;
+  return *cache ? with : base;
 }
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st) {
   if (n > 65535) return cudaErrorInvalidValue;
-  const int64_t slice = (ld + cluster - 1) / cluster;
-  const size_t base = sizeof(TopkShared);
-  const size_t cap = 200 * 1024;
-  const bool cache = base + (size_t)slice * 4 <= cap;
-  const size_t sm = cache ? base + (size_t)slice * 4 : base;
-  TopkArgs a{scores, ld, n_valid, n, k, out, err, cache ? 1 : 0, slice};
+  bool cache = false;
+  const size_t sm = topk_smem_bytes(ld, cluster, &cache);
+  TopkArgs a{scores, ld, n_valid, n, k, out, err, cache ? 1 : 0};
   dim3 grid(cluster, n);
   cudaError_t e;
   if (cluster == 8) {
-    e = cudaFuncSetAttribute(topk_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+    e = cudaFuncSetAttribute(topk_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     topk_cluster_kernel<8><<<grid, kTopkThreads, sm, st>>>(a);
     note_launch();
   } else if (cluster == 4) {
-    e = cudaFuncSetAttribute(topk_cluster_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cap);
+    e = cudaFuncSetAttribute(topk_cluster_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     topk_cluster_kernel<4><<<grid, kTopkThreads, sm, st>>>(a);
     note_launch();

@@ -202,6 +202,24 @@ def test_topk_exact_large(N, k):
     _topk_case([a, b], k)
 
 
+def test_topk_rows_that_defeat_or_stress_the_sample_filter():
+    """The selector estimates a threshold from a strided sample (every
+    N/4096-th score).  Rows whose sample lies about the top k must still
+    come out exact: a sample made of the largest scores (too few pass the
+    threshold), a top k hidden between the sampled positions, and a tie
+    class at the k-th score."""
+    N, k = 262144, 1024
+    r = np.random.default_rng(99)
+    base = r.standard_normal(N).astype(np.float32)
+    lying = base.copy()
+    lying[::64] = 100.0 + np.arange(N // 64, dtype=np.float32)      # the sample sees only these
+    hidden = base.copy()
+    hidden[1::64][:k] = 50.0 + r.random(k).astype(np.float32)       # never sampled
+    ties = base.copy()
+    ties[r.choice(N, 3000, replace=False)] = 3.0                     # the k-th score is a 3000-way tie
+    _topk_case([lying, hidden, ties], k)
+
+
 # ---------------------------------------------------------------- stage: attention
 
 def _write_cache_rows(pair, layer, req, T, rng, csa=True):
