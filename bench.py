@@ -79,31 +79,70 @@ def whole_job_rate(ws: int, batch_per_rank: int, steps: int, ms: float) -> float
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clock and clock-event reasons of this rank's GPU, sampled every
+    millisecond through NVML (read-only queries) by a background thread
+    during the timed region; nvidia-smi polling when NVML is unavailable."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
     def __init__(self, gpu_index: int):
         import torch
         try:
-            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
         except Exception:
-            self.gpu = str(gpu_index)
+            self.uuid = None
+        self.gpu_index = gpu_index
         self.proc = None
+        self.thread = None
+        self.samples = []
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
 
+    def _nvml_loop(self, handle, nv):
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((sm, mx, rs))
+            except Exception:
+                pass
+            time.sleep(0.001)
+
     def start(self):
+        self.stop_flag = False
+        try:
+            import pynvml as nv
+            import threading
+            nv.nvmlInit()
+            handle = nv.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else nv.nvmlDeviceGetHandleByIndex(self.gpu_index)
+            self.nv = nv
+            self.thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.uuid or self.gpu_index), f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            if not self.samples:
+                return None
+            sm = [x[0] for x in self.samples]
+            reasons = sorted({nm for _, _, rs in self.samples for bit, nm in self.REASONS.items() if rs & bit})
+            return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(x[1] for x in self.samples)),
+                    "reasons": reasons, "samples": len(sm), "source": "nvml, 1 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -129,7 +168,7 @@ class Clocks:
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, 100 ms"}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -228,40 +267,40 @@ def run_gpu(args):
     torch.cuda.synchronize()
     cache.check_device_error()
     lib = _lib.load()
-    graphs = []
+    # one CUDA graph per step; the index kernel is bracketed by events inside it
+    ev_i0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev_i1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
     launches0 = lib.csa_launch_count()
-    for f in parts:
-        gph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gph):
-            f()
-        graphs.append(gph)
-    kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graphs
+    with torch.cuda.graph(graph):
+        part_append()
+        if csa:
+            ev_i0.record()
+            part_index()
+            ev_i1.record()
+        part_post()
+    kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graph
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = Clocks(local)
     clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    evi = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms, idx_sum = 0.0, 0.0
     for s in range(steps):
         load_inputs(warm + s)
         flush.zero_()                       # L2 flushed between timed steps (not timed)
-        ev[s][0].record(stream)
-        graphs[0].replay()
+        ev0.record(stream)
+        graph.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+        step_ms += ev0.elapsed_time(ev1)
         if csa:
-            evi[s][0].record(stream)
-            graphs[1].replay()
-            evi[s][1].record(stream)
-            graphs[2].replay()
-        else:
-            graphs[1].replay()
-        ev[s][1].record(stream)
-    torch.cuda.synchronize()
+            idx_sum += ev_i0.elapsed_time(ev_i1)
     launches = kernels_per_step * steps               # libcsa kernels run in the timed region
-    step_ms = sum(a.elapsed_time(b) for a, b in ev)
-    idx_ms = sum(a.elapsed_time(b) for a, b in evi) / steps if csa else None
-    del graphs
+    idx_ms = idx_sum / steps if csa else None
+    del graph
     # ---- end to end through the public API with host buffers
     pin = lambda t: t.cpu().pin_memory() if t is not None else None
     h_c, h_z, h_ci, h_zi = pin(step_c[:steps]), pin(step_z[:steps]), pin(step_ci[:steps] if csa else None), \

@@ -294,21 +294,18 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       const int x = qt + 128 * u;
       if (x >= G * (Dp / 8)) break;
       const int hh = x / (Dp / 8), c = x % (Dp / 8);
-      const uint32_t rw[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-      float v[8];
-      for (int e = 0; e < 8; ++e) v[e] = bf16_val((uint16_t)(rw[e >> 1] >> (16 * (e & 1))));
-      if (8 * c >= dmain && 8 * c < D) {
+      uint4 o = raw[u];                               // non-RoPE dims: the BF16 input as is
+      if (8 * c >= dmain && 8 * c < D) {              // RoPE dims: rotate, round to BF16
+        const uint32_t rw[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+        uint32_t pk[4];
         for (int e = 0; e < 8; e += 2) {
           const float2 w = cs[(8 * c + e - dmain) / 2];
-          const float x0 = v[e], x1 = v[e + 1];
-          v[e] = x0 * w.x - x1 * w.y;
-          v[e + 1] = x0 * w.y + x1 * w.x;
+          const float x0 = bf16_val((uint16_t)(rw[e >> 1] & 0xFFFFu)), x1 = bf16_val((uint16_t)(rw[e >> 1] >> 16));
+          pk[e >> 1] = (uint32_t)bf16_rn(x0 * w.x - x1 * w.y) | ((uint32_t)bf16_rn(x0 * w.y + x1 * w.x) << 16);
         }
+        o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      uint32_t pk[4];
-      for (int e = 0; e < 4; ++e) pk[e] = (uint32_t)bf16_rn(v[2 * e]) | ((uint32_t)bf16_rn(v[2 * e + 1]) << 16);
-      *reinterpret_cast<uint4*>(qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16) =
-          make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16) = o;
     }
     // padding dims [D, Dp) of the tile stay zero
     const int npad = (Dp - D) / 8;
@@ -530,18 +527,29 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (tid < G && h0 + tid < H)
       a.ws_ml[((int64_t)i * a.tiles_max + tt0) * H + h0 + tid] = make_float2(m_t[tid], l_t[tid]);
     if (tw) {
+      // two 128-dim chunks per TMEM wait
       float* wo = a.ws_o + ((int64_t)i * a.tiles_max + tt0) * H * D;
-      for (int dc = 0; dc < n_dc; ++dc) {
-        const int d = dc * 128 + (warp & 3) * 32 + lane;
-        const bool has_rope = dc >= dc_r0;
-        uint32_t om[16], orp[16];
-        tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om);
-        if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp);
+      for (int dc0 = 0; dc0 < n_dc; dc0 += 2) {
+        uint32_t om[2][16], orp[2][16];
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const int dc = dc0 + q2;
+          if (dc < n_dc) {
+            tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om[q2]);
+            if (dc >= dc_r0) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp[q2]);
+          }
+        }
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int h = h0 + hb + e;
-          if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(d < dmain ? om[e] : orp[e]);
+        for (int q2 = 0; q2 < 2; ++q2) {
+          const int dc = dc0 + q2;
+          if (dc >= n_dc) break;
+          const int d = dc * 128 + (warp & 3) * 32 + lane;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int h = h0 + hb + e;
+            if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(d < dmain ? om[q2][e] : orp[q2][e]);
+          }
         }
       }
     }

@@ -281,10 +281,11 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
   if (!scores || !n_valid || !idx_out) return fail(CSA_ERR_ARG, "NULL argument");
   if (k < 1 || ld < 1) return fail(CSA_ERR_ARG, "k and ld must be >= 1");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
-  // One thread-block cluster per query: 8 CTAs for an under-fed GPU, 4 for a
-  // well-fed one.  The selection is exact, so both return identical indices.
-  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 37);
-  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, low ? 8 : 4,
+  // One thread-block cluster per query: 16 CTAs for an under-fed GPU (8 where
+  // the device cannot co-schedule 16), 8 for a well-fed one.  The selection
+  // is exact, so both return identical indices.
+  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 10);
+  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, low ? 16 : 8,
                                    (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "topk launch");
   return CSA_OK;

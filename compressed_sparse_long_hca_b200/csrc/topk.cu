@@ -365,6 +365,16 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   const int64_t hi = lo + chunk < N ? lo + chunk : N;
   const int64_t len = hi - lo;
 
+  // ---- 1. threshold from a strided sample (the same sample in every CTA)
+  const int S = N < kSample ? (int)N : kSample;
+  float sraw[kSamplePer];         // loads issued here, used after the bulk copy is on its way
+  bool sok[kSamplePer];
+#pragma unroll
+  for (int e = 0; e < kSamplePer; ++e) {
+    const int x = tid + e * kTopkThreads;
+    sok[e] = x < S;
+    sraw[e] = sok[e] ? s[(int64_t)x * N / S] : 0.f;
+  }
   // ---- slice -> shared memory: one bulk copy of the 16-byte aligned part
   const bool cached = a.cache_keys != 0;
   const bool bulk = cached && ((reinterpret_cast<uintptr_t>(s + lo) & 15) == 0);
@@ -382,16 +392,9 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     for (int64_t x = nbulk + tid; x < len; x += kTopkThreads) keys[x] = __float_as_uint(s[lo + x]);
   __syncthreads();   // the mbarrier is initialised before anyone waits on it
 
-  // ---- 1. threshold from a strided sample (the same sample in every CTA)
-  const int S = N < kSample ? (int)N : kSample;
   uint32_t sv[kSamplePer];
-  bool sok[kSamplePer];
 #pragma unroll
-  for (int e = 0; e < kSamplePer; ++e) {
-    const int x = tid + e * kTopkThreads;
-    sok[e] = x < S;
-    sv[e] = sok[e] ? order_key(s[(int64_t)x * N / S]) : 0u;
-  }
+  for (int e = 0; e < kSamplePer; ++e) sv[e] = sok[e] ? order_key(sraw[e]) : 0u;
   const float lam = (float)k * (float)S / (float)N;     // expected sampled keys above the k-th
   const int r = (int)ceilf(lam + 6.f * sqrtf(lam) + 8.f);
   uint32_t tau = 0;
@@ -409,55 +412,100 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
       return;
     }
   }
-  auto key_at = [&](int64_t x) -> uint32_t { return cached ? order_key(__uint_as_float(keys[x])) : order_key(s[lo + x]); };
 
   // ---- 2. filter: count, exchange counts, write candidates to the leader
-  const int64_t per_w = ((len + kWarps - 1) / kWarps + 31) / 32 * 32;
+  // Each warp owns a contiguous sub-slice (a multiple of 128 keys when the
+  // slice is in shared memory: each lane then reads 4 keys per 16-byte load).
+  const int64_t per_w = cached ? ((len + kWarps - 1) / kWarps + 127) / 128 * 128
+                               : ((len + kWarps - 1) / kWarps + 31) / 32 * 32;
   const int64_t w_lo = (int64_t)wid * per_w < len ? (int64_t)wid * per_w : len;
   const int64_t w_hi = w_lo + per_w < len ? w_lo + per_w : len;
-  int wc = 0;
-  for (int64_t x0 = w_lo; x0 < w_hi; x0 += 8 * 32) {
-    uint32_t kv[8];
+  const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+  auto load4 = [&](int64_t x, uint32_t (&kv)[4], bool (&pass)[4]) {
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (x < w_hi) v = k4[x >> 2];
+    const uint32_t raw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t x = x0 + u * 32 + lane;
-      kv[u] = x < w_hi ? key_at(x) : 0u;
+    for (int e = 0; e < 4; ++e) {
+      kv[e] = order_key(__uint_as_float(raw[e]));
+      pass[e] = x + e < w_hi && kv[e] >= tau;
     }
+  };
+  int wc = 0;
+  if (cached) {
+    int c = 0;
+    for (int64_t x0 = w_lo; x0 < w_hi; x0 += 128) {
+      uint32_t kv[4];
+      bool pass[4];
+      load4(x0 + 4 * lane, kv, pass);
+      c += (int)pass[0] + (int)pass[1] + (int)pass[2] + (int)pass[3];
+    }
+    wc = __reduce_add_sync(0xffffffffu, c);
+  } else {
+    for (int64_t x0 = w_lo; x0 < w_hi; x0 += 8 * 32) {
+      uint32_t kv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t x = x0 + u * 32 + lane;
-      wc += __popc(__ballot_sync(0xffffffffu, x < w_hi && kv[u] >= tau));
+      for (int u = 0; u < 8; ++u) {
+        const int64_t x = x0 + u * 32 + lane;
+        kv[u] = x < w_hi ? order_key(s[lo + x]) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t x = x0 + u * 32 + lane;
+        wc += __popc(__ballot_sync(0xffffffffu, x < w_hi && kv[u] >= tau));
+      }
     }
   }
   int cta_cnt;
   const int w_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? wc : 0, sh.wsum, &cta_cnt), 0);
   if (tid == 0) sh.n_cand = cta_cnt;
   cluster.sync();
-  int base = 0, total = 0;
-  for (int q = 0; q < C; ++q) {
-    const int c = *cluster.map_shared_rank(&sh.n_cand, q);
-    if (q < rank) base += c;
-    total += c;
+  int base, total;
+  {   // lane q reads CTA q's count (all remote reads in flight at once)
+    const int c = lane < C ? *cluster.map_shared_rank(&sh.n_cand, lane) : 0;
+    base = __reduce_add_sync(0xffffffffu, lane < rank ? c : 0);
+    total = __reduce_add_sync(0xffffffffu, c);
   }
   const bool filter = total >= k && total <= kCandCap;   // the same in every CTA
   if (filter) {
     uint2* lc = cluster.map_shared_rank(&sh.u.cand[0], 0);
     int pos = base + w_before;
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int64_t x0 = w_lo; x0 < w_hi; x0 += 8 * 32) {
-      uint32_t kv[8];
+    if (cached) {
+      for (int64_t x0 = w_lo; x0 < w_hi; x0 += 128) {
+        const int64_t x = x0 + 4 * lane;
+        uint32_t kv[4];
+        bool pass[4];
+        load4(x, kv, pass);
+        const int cnt = (int)pass[0] + (int)pass[1] + (int)pass[2] + (int)pass[3];
+        int incl = cnt;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t x = x0 + u * 32 + lane;
-        kv[u] = x < w_hi ? key_at(x) : 0u;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int p = pos + incl - cnt;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (pass[e]) lc[p++] = make_uint2(kv[e], (uint32_t)(lo + x + e));
+        pos += __shfl_sync(0xffffffffu, incl, 31);
       }
+    } else {
+      for (int64_t x0 = w_lo; x0 < w_hi; x0 += 8 * 32) {
+        uint32_t kv[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t x = x0 + u * 32 + lane;
-        const bool pass = x < w_hi && kv[u] >= tau;
-        const unsigned b = __ballot_sync(0xffffffffu, pass);
-        if (pass) lc[pos + __popc(b & lt_mask)] = make_uint2(kv[u], (uint32_t)(lo + x));
-        pos += __popc(b);
+        for (int u = 0; u < 8; ++u) {
+          const int64_t x = x0 + u * 32 + lane;
+          kv[u] = x < w_hi ? order_key(s[lo + x]) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t x = x0 + u * 32 + lane;
+          const bool pass = x < w_hi && kv[u] >= tau;
+          const unsigned b = __ballot_sync(0xffffffffu, pass);
+          if (pass) lc[pos + __popc(b & lt_mask)] = make_uint2(kv[u], (uint32_t)(lo + x));
+          pos += __popc(b);
+        }
       }
     }
     cluster.sync();   // the leader's list is complete; nobody reads another CTA after this
@@ -477,22 +525,26 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     block_minmax(cv, cok, sh.mm, &cmin, &cmax);
     int ties_needed;
     const uint32_t T = block_select(cv, cok, k, tau, cmax, true, sh, &ties_needed);
-    int neq = 0;
+    // one scan of (count > T, count == T) packed in 16-bit halves (counts <= kCandCap)
+    int ngt = 0, neq = 0;
 #pragma unroll
-    for (int e = 0; e < kCandPer; ++e) neq += (cok[e] && cv[e] == T) ? 1 : 0;
-    int eq_tot;
-    const int eq_before = block_excl_scan(neq, sh.wsum, &eq_tot);
-    int take = 0, seen = eq_before;
+    for (int e = 0; e < kCandPer; ++e) {
+      ngt += (cok[e] && cv[e] > T) ? 1 : 0;
+      neq += (cok[e] && cv[e] == T) ? 1 : 0;
+    }
+    int packed_tot;
+    const int packed = block_excl_scan(ngt | (neq << 16), sh.wsum, &packed_tot);
+    const int gt_before = packed & 0xFFFF, eq_before = packed >> 16;
+    int seen = eq_before;
     unsigned take_bits = 0;
 #pragma unroll
     for (int e = 0; e < kCandPer; ++e) {
       const bool is_eq = cok[e] && cv[e] == T;
       const bool t = cok[e] && (cv[e] > T || (is_eq && seen < ties_needed));
       seen += is_eq ? 1 : 0;
-      if (t) { take_bits |= 1u << e; ++take; }
+      if (t) take_bits |= 1u << e;
     }
-    int tot_sel;
-    int p = block_excl_scan(take, sh.wsum, &tot_sel);
+    int p = gt_before + (eq_before < ties_needed ? eq_before : ties_needed);
 #pragma unroll
     for (int e = 0; e < kCandPer; ++e)
       if (take_bits & (1u << e)) out[p++] = (int32_t)sh.u.cand[e0 + e].y;
@@ -515,28 +567,67 @@ size_t topk_smem_bytes(int64_t ld, int cluster, bool* cache) {
   return *cache ? with : base;
 }
 
+namespace {
+
+template <int C>
+cudaError_t launch_topk_c(const TopkArgs& a, size_t sm, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(topk_cluster_kernel<C>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  topk_cluster_kernel<C><<<dim3(C, a.n), kTopkThreads, sm, st>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// Whether this device can co-schedule a 16-CTA cluster of the kernel with
+// `sm` bytes of shared memory (asked once per device and size).
+bool cluster16_ok(size_t sm) {
+  static int cached_dev = -1;
+  static size_t cached_sm = 0;
+  static bool cached_ok = false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev == cached_dev && sm == cached_sm) return cached_ok;
+  bool ok = false;
+  if (cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+      cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) ==
+          cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = sm;
+    int nclusters = 0;
+    ok = cudaOccupancyMaxActiveClusters(&nclusters, topk_cluster_kernel<16>, &cfg) == cudaSuccess && nclusters > 0;
+  }
+  cudaGetLastError();
+  cached_dev = dev;
+  cached_sm = sm;
+  cached_ok = ok;
+  return ok;
+}
+
+}  // namespace
+
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st) {
   if (n > 65535) return cudaErrorInvalidValue;
+  if (cluster == 16) {
+    bool cache16 = false;
+    const size_t sm16 = topk_smem_bytes(ld, 16, &cache16);
+    if (!cluster16_ok(sm16)) cluster = 8;
+  }
   bool cache = false;
   const size_t sm = topk_smem_bytes(ld, cluster, &cache);
   TopkArgs a{scores, ld, n_valid, n, k, out, err, cache ? 1 : 0};
-  dim3 grid(cluster, n);
-  cudaError_t e;
-  if (cluster == 8) {
-    e = cudaFuncSetAttribute(topk_cluster_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    topk_cluster_kernel<8><<<grid, kTopkThreads, sm, st>>>(a);
-    note_launch();
-  } else if (cluster == 4) {
-    e = cudaFuncSetAttribute(topk_cluster_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    topk_cluster_kernel<4><<<grid, kTopkThreads, sm, st>>>(a);
-    note_launch();
-  } else {
-    return cudaErrorInvalidValue;
+  switch (cluster) {
+    case 16: return launch_topk_c<16>(a, sm, st);
+    case 8: return launch_topk_c<8>(a, sm, st);
+    case 4: return launch_topk_c<4>(a, sm, st);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace csa
