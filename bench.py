@@ -57,6 +57,27 @@ def _dist():
     return ws, rank, local
 
 
+def _profiled_traffic():
+    """DRAM bytes (read + write) per index-kernel launch from the committed
+    ncu summary, or None when the kernel's sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "index_tc_csa-pro-1m.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path, encoding="utf-8"):
+        k, _, v = line.strip().partition(": ")
+        if k in ("sources_sha256", "traffic_bytes_per_launch"):
+            fields[k] = v.strip()
+    h = hashlib.sha256()
+    for f in ("index_tc.cu", "layout.cuh", "tc.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "compressed_sparse_long_hca_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if fields.get("sources_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def rank_seed(wl, rank: int) -> int:
     """Seed of the requests a rank owns: ranks hold disjoint requests."""
     return wl.seed + 7919 * rank
@@ -230,6 +251,15 @@ def run_gpu(args):
     idx = torch.empty((B, max(wl.k, 1)), dtype=torch.int32, device="cuda")
     out = torch.empty((B, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")    # > 126 MB L2
+    flush_rd = torch.ones(256 * 2**20 // 4, dtype=torch.int32, device="cuda")
+
+    def flush_l2():
+        """Evict the step's inputs from L2 (not timed): write a buffer larger
+        than L2, then read another one, so that the lines left in L2 are
+        clean and the step is not charged for the flush's own write-backs."""
+        flush.zero_()
+        flush_rd.sum()
+
     stream = torch.cuda.current_stream()
 
     # Static per-step inputs: the timed steps replay CUDA graphs of the step
@@ -252,33 +282,30 @@ def run_gpu(args):
     def part_index():
         cache.index_scores(layer, rid, qi, w, scores, nv)
 
-    def part_post():
-        if csa:
-            topk(scores, nv, wl.k, idx)
-            cache.decode_attn(layer, rid, q, idx, sink_d, out)
-        else:
-            cache.decode_attn(layer, rid, q, None, sink_d, out)
+    def part_topk():
+        topk(scores, nv, wl.k, idx)
 
-    parts = [part_append] + ([part_index] if csa else []) + [part_post]
+    def part_attn():
+        cache.decode_attn(layer, rid, q, idx if csa else None, sink_d, out)
+
+    parts = [("append", part_append)] + ([("index", part_index), ("topk", part_topk)] if csa else []) + \
+        [("attention", part_attn)]
     for s in range(warm):                   # eager warm-up (also sizes the attention workspace)
         load_inputs(s)
-        for f in parts:
+        for _, f in parts:
             f()
     torch.cuda.synchronize()
     cache.check_device_error()
     lib = _lib.load()
-    # one CUDA graph per step; the index kernel is bracketed by events inside it
-    ev_i0 = torch.cuda.Event(enable_timing=True, external=True)
-    ev_i1 = torch.cuda.Event(enable_timing=True, external=True)
+    # one CUDA graph per step; every part is bracketed by events inside it
+    evp = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
     graph = torch.cuda.CUDAGraph()
     launches0 = lib.csa_launch_count()
     with torch.cuda.graph(graph):
-        part_append()
-        if csa:
-            ev_i0.record()
-            part_index()
-            ev_i1.record()
-        part_post()
+        for x, (_, f) in enumerate(parts):
+            evp[x].record()
+            f()
+        evp[len(parts)].record()
     kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graph
     torch.cuda.synchronize()
     if ws > 1:
@@ -287,19 +314,21 @@ def run_gpu(args):
     clocks = Clocks(local)
     clocks.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ms, idx_sum = 0.0, 0.0
+    step_ms = 0.0
+    part_ms = {nm: 0.0 for nm, _ in parts}
     for s in range(steps):
         load_inputs(warm + s)
-        flush.zero_()                       # L2 flushed between timed steps (not timed)
+        flush_l2()                          # L2 flushed between timed steps (not timed)
         ev0.record(stream)
         graph.replay()
         ev1.record(stream)
         ev1.synchronize()
         step_ms += ev0.elapsed_time(ev1)
-        if csa:
-            idx_sum += ev_i0.elapsed_time(ev_i1)
+        for x, (nm, _) in enumerate(parts):
+            part_ms[nm] += evp[x].elapsed_time(evp[x + 1])
     launches = kernels_per_step * steps               # libcsa kernels run in the timed region
-    idx_ms = idx_sum / steps if csa else None
+    idx_ms = part_ms["index"] / steps if csa else None
+    breakdown = {nm: round(v / steps * 1e3, 2) for nm, v in part_ms.items()}
     del graph
     # ---- end to end through the public API with host buffers
     pin = lambda t: t.cpu().pin_memory() if t is not None else None
@@ -314,7 +343,7 @@ def run_gpu(args):
     h2d = 0
     e2e_ms = 0.0
     for s in range(steps):
-        flush.zero_()
+        flush_l2()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         d_c.copy_(h_c[s], non_blocking=True)
@@ -353,9 +382,10 @@ def run_gpu(args):
         "config": {"workload": wl.name, "context": T0, "batch_per_gpu": B, "heads": wl.H,
                    "head_dim": wl.D, "rope_dims": wl.R, "indexer": f"{wl.H_I}x{wl.d_I}",
                    "topk": wl.k, "window": wl.W, "layers_per_step": 1,
-                   "l2": "flushed (256 MB write) before every timed step",
+                   "l2": "flushed before every timed step: 256 MB written, then 256 MB read (not timed)",
                    "parallelism": f"request-sharded x{ws}"},
         "gpu_launches": launches,
+        "step_breakdown_us": breakdown,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "clocks": clk,
     }
@@ -364,7 +394,7 @@ def run_gpu(args):
         alg = B * (n_c * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
         ach = alg / (idx_ms / 1e3) / 1e9
         line["roofline"] = {"bound": "hbm", "kernel": "csa_index_scores", "achieved": ach, "peak": peak,
-                            "unit": "GB/s", "frac": ach / peak, "traffic": None,
+                            "unit": "GB/s", "frac": ach / peak, "traffic": _profiled_traffic(),
                             "peak_source": peak_kind, "ms_per_launch": idx_ms,
                             "algorithmic_bytes_per_launch": alg}
     if rank == 0 and args.cpu_baseline and ws == 1:

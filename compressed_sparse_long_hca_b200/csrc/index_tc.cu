@@ -46,8 +46,9 @@ constexpr int kCtasPerSm = 2;          // two CTAs per SM overlap their issue la
 constexpr int kHeadsN = 64;            // MMA N (index heads, zero padded)
 constexpr int kMaxCh = 4;              // d_I / 32 <= 4
 constexpr int kTileBytes = kCsaPerPage * kMaxCh * 16 + kSfChunk;   // codes + scale chunk
-constexpr int kPassTiles = 512;        // tiles per pass (page-table window in smem)
+constexpr int kPassTiles = 128;        // tiles per pass (page-table window in smem)
 constexpr int kMaxSeg = 64;            // queries per pass
+constexpr int kMaxQ = 256;             // queries whose tile counts are kept in shared memory
 constexpr uint32_t kTmemCols = 256;    // per CTA; two CTAs fill the SM's 512 columns
 constexpr uint32_t kSfaCol = 192;      // + 4 * accumulator index
 constexpr uint32_t kSfbCol = 204;
@@ -64,6 +65,9 @@ struct IdxSmem {
   int64_t seg_t0[kMaxSeg];
   int64_t seg_N[kMaxSeg];
   int32_t n_seg;
+  int32_t q_tiles[kMaxQ];                            // tiles of query i (i < kMaxQ)
+  int64_t q_N[kMaxQ];                                // keys of query i
+  int64_t red[kThreads / 32];
   uint64_t full[kStages], stage_empty[kStages];
   uint64_t acc_full[kNA], acc_empty[kNA];
   uint64_t q_ready;
@@ -111,8 +115,8 @@ __device__ __forceinline__ bool wait_or_abort(IdxSmem& sm, uint64_t* bar, uint32
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const Layout& L = a.L;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int HI = L.HI, dI = L.dI, CH = dI / 32, CHs = L.CHs;
@@ -121,22 +125,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
   const uint32_t tile_bytes = (uint32_t)L.idx_tile_bytes;
   const uint32_t sf_off = (uint32_t)(kCsaPerPage * CHs * 16);
 
-  // ---- per-query bookkeeping; every CTA computes the same tile prefix
-  if (blockIdx.x == 0) {
+  // ---- per-query bookkeeping (one thread per query); every CTA computes
+  //      the same tile total
+  int64_t total = 0;
+  {
+    int64_t part = 0;
     for (int i = tid; i < a.n; i += kThreads) {
       int64_t N;
       int req;
-      query_tiles(a, i, &N, &req);
-      if (req < 0 || req >= L.max_req) { set_err(L, kErrBounds, i); a.n_valid[i] = 0; continue; }
-      a.n_valid[i] = (int32_t)N;
-      if (N > a.ld) set_err(L, kErrLd, i);
+      const int64_t nt = query_tiles(a, i, &N, &req);
+      if (i < kMaxQ) { sm.q_tiles[i] = (int32_t)nt; sm.q_N[i] = N; }
+      part += nt;
+      if (blockIdx.x == 0) {
+        if (req < 0 || req >= L.max_req) { set_err(L, kErrBounds, i); a.n_valid[i] = 0; continue; }
+        a.n_valid[i] = (int32_t)N;
+        if (N > a.ld) set_err(L, kErrLd, i);
+      }
     }
-  }
-  int64_t total = 0;
-  for (int i = 0; i < a.n; ++i) {
-    int64_t N;
-    int req;
-    total += query_tiles(a, i, &N, &req);
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) sm.red[warp] = part;
+    __syncthreads();
+    for (int w = 0; w < kThreads / 32; ++w) total += sm.red[w];
   }
   const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
   if (g0 >= g1) return;
@@ -175,9 +184,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
       int ns = 0;
       int64_t gg = g, used = 0;
       while (gg < g1 && used < kPassTiles && ns < kMaxSeg) {
-        int64_t N;
-        int req;
-        const int64_t nt = query_tiles(a, qi, &N, &req);
+        int64_t N, nt;
+        if (qi < kMaxQ) {
+          nt = sm.q_tiles[qi];
+          N = sm.q_N[qi];
+        } else {
+          int req;
+          nt = query_tiles(a, qi, &N, &req);
+        }
         if (nt == 0 || before + nt <= gg) { before += nt; ++qi; continue; }
         const int64_t t0 = gg - before;
         int64_t cnt = (g1 - before < nt ? g1 - before : nt) - t0;
@@ -375,10 +389,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Sized so that exactly two CTAs share an SM: their two 256-column TMEM
-// allocations then always fit the SM's 512 columns.
+// Sized so that exactly two CTAs share an SM (at most 113 KB each): their
+// two 256-column TMEM allocations then always fit the SM's 512 columns.
 size_t index_tc_smem_bytes() {
-  const size_t need = sizeof(IdxSmem) + 1024;
+  const size_t need = sizeof(IdxSmem) + 128;
   return need > 80 * 1024 ? need : 80 * 1024;
 }
 

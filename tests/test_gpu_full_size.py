@@ -1,0 +1,200 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration that
+bench.py times (AUTO variants, the same batch shapes).
+
+Caches are filled through csa_compress_append with device-generated inputs,
+then one decode step runs (append -> index -> top-k -> attention).  The
+oracle checks every index score against the keys read back from the cache,
+the top-k index set against its own top-k of its own scores, and every
+attention output over the rows the GPU selected (read back); the same step is
+re-run in another batch order and with both launch variants, bit-exact.
+
+A bounded ragged sweep (Pro-like CSA and HCA layers, contexts log-uniform in
+[4K, 256K]) checks that a request's bits do not depend on the batch it is in.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from compressed_sparse_long_hca_b200 import inputs as I
+from compressed_sparse_long_hca_b200.api import topk, unpack_index_rows, unpack_kv_rows
+from oracle import csa_oracle as O
+from tests import helpers as Hp
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_lib):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return cuda_lib
+
+
+def _fill(cache, layer, reqs, lengths, seed, D, dI):
+    """Append tokens 0 .. lengths[r]-1 of every request (chunks of 4096;
+    requests that are already full drop out of later calls)."""
+    t = 0
+    while True:
+        live = [r for r in reqs if lengths[r] > t]
+        if not live:
+            break
+        n_tok = min(min(lengths[r] for r in live) - t, I.CHUNK - t % I.CHUNK)
+        parts = [I.device_token_inputs(seed, layer, r, t // I.CHUNK, D, dI) for r in live]
+        lo = t % I.CHUNK
+        st = lambda k: (torch.stack([p[k][lo:lo + n_tok] for p in parts]).contiguous()
+                        if parts[0][k] is not None else None)
+        cache.compress_append(layer, torch.tensor(live, dtype=torch.int32, device="cuda"), st(0), st(1), st(2), st(3))
+        t += n_tok
+    torch.cuda.synchronize()
+    cache.check_device_error()
+
+
+def _host(seed, *shape):
+    return np.random.default_rng(seed).standard_normal(shape).astype(np.float32)
+
+
+def _step(cache, wl, layer, order, q, qi, w, sink, variant="auto"):
+    """Index, top-k and attention for the requests in `order`; results are
+    returned in request order (dicts keyed by request)."""
+    csa = wl.kind == "csa"
+    n = len(order)
+    rid = torch.tensor(order, dtype=torch.int32, device="cuda")
+    dq = torch.from_numpy(q[order]).cuda().to(torch.bfloat16)
+    out = torch.empty((n, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    res = {}
+    if csa:
+        ld = max(cache.get_length(layer, r) for r in order) // 4 + 128
+        scores = torch.full((n, ld), float("nan"), device="cuda")
+        nv = torch.zeros(n, dtype=torch.int32, device="cuda")
+        cache.index_scores(layer, rid, torch.from_numpy(qi[order]).cuda(), torch.from_numpy(w[order]).cuda(), scores,
+                           nv, variant=variant)
+        idx = torch.empty((n, wl.k), dtype=torch.int32, device="cuda")
+        topk(scores, nv, wl.k, idx, variant=variant)
+        cache.decode_attn(layer, rid, dq, idx, torch.from_numpy(sink).cuda(), out, variant=variant)
+        cache.check_device_error()
+        sc, nvh, ih = scores.cpu().numpy(), nv.cpu().numpy(), idx.cpu().numpy()
+        for x, r in enumerate(order):
+            res[r] = dict(scores=sc[x, : nvh[x]].copy(), idx=ih[x].copy())
+    else:
+        cache.decode_attn(layer, rid, dq, None, torch.from_numpy(sink).cuda(), out, variant=variant)
+        cache.check_device_error()
+    oh = out.cpu()
+    for x, r in enumerate(order):
+        res.setdefault(r, {})["out"] = oh[x].view(torch.int16).numpy().copy()
+        res[r]["out_f"] = oh[x].float().numpy()
+    return res
+
+
+def _oracle_check(cache, wl, layer, r, T, q, qi, w, sink, got):
+    """Oracle parity of one request's decode step (T tokens stored)."""
+    csa = wl.kind == "csa"
+    t = T - 1
+    N = T // 4 if csa else T // 128
+    if csa:
+        codes, scales = unpack_index_rows(cache.read_rows(layer, r, 1, 0, N), wl.d_I)
+        kd = O.dequantize_mxfp4(O.MXFP4(codes=codes, scales=scales))
+        qd = O.dequantize_mxfp4(O.quantize_mxfp4(qi[r]))
+        ref = O.index_scores(qd, w[r], kd)
+        mag = np.abs(kd @ qd.T) @ np.abs(w[r])
+        assert got["scores"].shape[0] == N
+        assert np.all(np.abs(got["scores"].astype(np.float64) - ref) <= 1e-5 * mag + 1e-6), f"scores, request {r}"
+        Hp.check_topk(got["idx"], ref, wl.k, N, what=f"topk request {r}")
+        sel = got["idx"][got["idx"] >= 0]
+    else:
+        sel = np.arange(N)
+    kv = cache.read_rows(layer, r, 0, 0, N) if N else np.zeros((0, cache.row_bytes(0)), np.uint8)
+    fp8, bf, sc = unpack_kv_rows(kv[sel] if len(sel) else kv[:0], wl.D, wl.R)
+    ent = O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc))
+    wp = O.window_positions(t)
+    fp8, bf, sc = unpack_kv_rows(cache.read_rows(layer, r, 2, wp[0], len(wp)), wl.D, wl.R)
+    win = O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc))
+    rows = np.concatenate([ent, win], axis=0)
+    ref_out = O.mqa_attention(O.rope(q[r].astype(np.float64), t, wl.R), rows, sink, 1.0 / math.sqrt(wl.D))
+    Hp.check_attention(got["out_f"], ref_out, f"attention request {r}")
+
+
+@pytest.mark.parametrize("name", ["csa-pro-1m", "csa-flash-128k", "hca-128k"])
+def test_full_size_decode_step(name):
+    wl = I.WORKLOADS[name]
+    csa = wl.kind == "csa"
+    B, T0 = wl.batch, wl.context
+    pair = Hp.Pair(wl, 1 if csa else 0, 0 if csa else 1, max_req=B, capacity=T0 + 512)
+    cache = pair.cache
+    for r in range(B):
+        cache.request_alloc(r, T0 + 512)
+    dI = wl.d_I if csa else 0
+    _fill(cache, 0, list(range(B)), {r: T0 for r in range(B)}, wl.seed, wl.D, dI)
+    # the decode step's own token (host-generated), then the read path
+    c, z = _host(wl.seed + 1, B, 1, wl.D), _host(wl.seed + 2, B, 1, wl.D)
+    ci = _host(wl.seed + 3, B, 1, dI) if csa else None
+    zi = _host(wl.seed + 4, B, 1, dI) if csa else None
+    dev = lambda a: torch.from_numpy(a).cuda() if a is not None else None
+    cache.compress_append(0, torch.arange(B, dtype=torch.int32, device="cuda"), dev(c), dev(z), dev(ci), dev(zi))
+    q = I.bf16_grid(_host(wl.seed + 5, B, wl.H, wl.D))
+    qi = _host(wl.seed + 6, B, wl.H_I, wl.d_I) if csa else None
+    w = _host(wl.seed + 7, B, wl.H_I) if csa else None
+    sink = pair.params[0]["sink"]
+    base = _step(cache, wl, 0, list(range(B)), q, qi, w, sink)
+    # oracle parity: every request of the small batches, four of the large ones
+    check = list(range(B)) if B <= 4 else [0, 7, 18, B - 1]
+    for r in check:
+        _oracle_check(cache, wl, 0, r, T0 + 1, q, qi, w, sink, base[r])
+    # the same requests in another order, and both launch variants: bit-exact
+    order = list(np.random.default_rng(wl.seed).permutation(B))
+    for variant in ("high", "low"):
+        again = _step(cache, wl, 0, [int(x) for x in order], q, qi, w, sink, variant)
+        for r in range(B):
+            assert np.array_equal(again[r]["out"], base[r]["out"]), f"request {r} ({variant})"
+            if csa:
+                assert np.array_equal(again[r]["idx"], base[r]["idx"]), f"request {r} ({variant})"
+                assert np.array_equal(again[r]["scores"].view(np.uint32), base[r]["scores"].view(np.uint32))
+
+
+def test_ragged_sweep_batch_invariance():
+    """Pro-like CSA (top-1024) and HCA layers, 16 requests with contexts
+    log-uniform in [4K, 256K], three decode steps; each step runs the whole
+    batch and sampled sub-batches (sizes 1 .. 16, shuffled positions, both
+    variants): every request's bits agree across all of them."""
+    wl_c, wl_h = I.C5_CSA, I.C5_HCA
+    n_req = 16
+    ctx = I.sweep_contexts(wl_c.seed, n_req, lo=4096, hi=1 << 18)
+    cap = int(ctx.max()) + 512
+    pair = Hp.Pair(wl_c, 1, 1, max_req=n_req, capacity=cap)
+    cache = pair.cache
+    for r in range(n_req):
+        cache.request_alloc(r, int(ctx[r]) + 512)
+    lens = {r: int(ctx[r]) for r in range(n_req)}
+    _fill(cache, 0, list(range(n_req)), lens, wl_c.seed, wl_c.D, wl_c.d_I)
+    _fill(cache, 1, list(range(n_req)), lens, wl_c.seed + 1, wl_c.D, 0)
+    rng = np.random.default_rng(55)
+    allr = list(range(n_req))
+    for step in range(3):
+        for layer, wl in ((0, wl_c), (1, wl_h)):
+            csa = layer == 0
+            c, z = _host(900 + step * 2 + layer, n_req, 1, wl.D), _host(950 + step * 2 + layer, n_req, 1, wl.D)
+            ci = _host(990 + step, n_req, 1, wl.d_I) if csa else None
+            zi = _host(995 + step, n_req, 1, wl.d_I) if csa else None
+            dev = lambda a: torch.from_numpy(a).cuda() if a is not None else None
+            cache.compress_append(layer, torch.arange(n_req, dtype=torch.int32, device="cuda"), dev(c), dev(z),
+                                  dev(ci), dev(zi))
+            q = I.bf16_grid(_host(700 + step * 2 + layer, n_req, wl.H, wl.D))
+            qi = _host(800 + step, n_req, wl.H_I, wl.d_I) if csa else None
+            w = _host(850 + step, n_req, wl.H_I) if csa else None
+            sink = pair.params[layer]["sink"]
+            base = _step(cache, wl, layer, allr, q, qi, w, sink)
+            if step == 0:   # oracle parity on the shortest request of each layer
+                r = int(np.argmin(ctx))
+                _oracle_check(cache, wl, layer, r, lens[r] + 1, q, qi, w, sink, base[r])
+            for size in (1, 3, 7, 16):
+                sub = [int(x) for x in rng.choice(n_req, size=size, replace=False)]
+                variant = ("high", "low", "auto")[int(rng.integers(0, 3))]
+                again = _step(cache, wl, layer, sub, q, qi, w, sink, variant)
+                for r in sub:
+                    assert np.array_equal(again[r]["out"], base[r]["out"]), f"step {step} layer {layer} req {r}"
+                    if csa:
+                        assert np.array_equal(again[r]["idx"], base[r]["idx"])
+        for r in allr:
+            lens[r] += 1
