@@ -210,7 +210,7 @@ def run_gpu(args):
     B, T0 = wl.batch, wl.context
     csa = wl.kind == "csa"
     steps, warm = args.steps, args.warmup
-    cap = T0 + steps + warm + 256
+    cap = T0 + 4 * steps + warm + 256
     nb = (cap + 511) // 512
     layer = 0
     b_kv, b_idx, sink = I.layer_params(wl.seed, layer, wl.kind, wl.D, wl.d_I or 32, wl.H)
@@ -234,7 +234,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     cache.check_device_error()
     # ---- per-step inputs (device), generated up front
-    total_steps = steps + warm
+    total_steps = 3 * steps + warm
     g = torch.Generator(device="cuda")
     g.manual_seed(rank_seed(wl, rank) * 31)
     step_c = torch.randn((total_steps, B, 1, wl.D), generator=g, device="cuda")
@@ -297,39 +297,67 @@ def run_gpu(args):
     torch.cuda.synchronize()
     cache.check_device_error()
     lib = _lib.load()
-    # one CUDA graph per step; every part is bracketed by events inside it
-    evp = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
-    graph = torch.cuda.CUDAGraph()
+    # The step as CUDA graphs: plain (the headline), with events around the
+    # index kernel (its roofline), with events around every part (the
+    # breakdown).  Event nodes inside a graph cost a few microseconds each,
+    # so each figure comes from its own pass of `steps` timed steps.
+    def capture(marks):
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for x, (nm, f) in enumerate(parts):
+                if nm in marks or (x > 0 and parts[x - 1][0] in marks):
+                    evs[x].record()
+                f()
+            if parts[-1][0] in marks:
+                evs[len(parts)].record()
+        return g, evs
+
     launches0 = lib.csa_launch_count()
-    with torch.cuda.graph(graph):
-        for x, (_, f) in enumerate(parts):
-            evp[x].record()
-            f()
-        evp[len(parts)].record()
+    g_plain, _ = capture(())
     kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graph
+    g_idx, ev_idx = capture(("index",) if csa else ())
+    g_all, ev_all = capture(tuple(nm for nm, _ in parts))
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed_pass(g, first, after=None):
+        total = 0.0
+        for s in range(steps):
+            load_inputs(first + s)
+            flush_l2()                      # L2 flushed between timed steps (not timed)
+            ev0.record(stream)
+            g.replay()
+            ev1.record(stream)
+            ev1.synchronize()
+            total += ev0.elapsed_time(ev1)
+            if after:
+                after()
+        return total
+
     clocks = Clocks(local)
     clocks.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ms = 0.0
-    part_ms = {nm: 0.0 for nm, _ in parts}
-    for s in range(steps):
-        load_inputs(warm + s)
-        flush_l2()                          # L2 flushed between timed steps (not timed)
-        ev0.record(stream)
-        graph.replay()
-        ev1.record(stream)
-        ev1.synchronize()
-        step_ms += ev0.elapsed_time(ev1)
-        for x, (nm, _) in enumerate(parts):
-            part_ms[nm] += evp[x].elapsed_time(evp[x + 1])
+    step_ms = timed_pass(g_plain, warm)
+    clk = clocks.stop()
     launches = kernels_per_step * steps               # libcsa kernels run in the timed region
-    idx_ms = part_ms["index"] / steps if csa else None
+    idx_sum = [0.0]
+    names = [nm for nm, _ in parts]
+    if csa:
+        x = names.index("index")
+        timed_pass(g_idx, warm + steps, lambda: idx_sum.__setitem__(0, idx_sum[0] + ev_idx[x].elapsed_time(ev_idx[x + 1])))
+    part_ms = {nm: 0.0 for nm in names}
+
+    def add_parts():
+        for x, nm in enumerate(names):
+            part_ms[nm] += ev_all[x].elapsed_time(ev_all[x + 1])
+
+    timed_pass(g_all, warm + 2 * steps, add_parts)
+    idx_ms = idx_sum[0] / steps if csa else None
     breakdown = {nm: round(v / steps * 1e3, 2) for nm, v in part_ms.items()}
-    del graph
+    del g_plain, g_idx, g_all
     # ---- end to end through the public API with host buffers
     pin = lambda t: t.cpu().pin_memory() if t is not None else None
     h_c, h_z, h_ci, h_zi = pin(step_c[:steps]), pin(step_z[:steps]), pin(step_ci[:steps] if csa else None), \
@@ -368,7 +396,6 @@ def run_gpu(args):
     copied = [d_c, d_z, d_q] + ([d_ci, d_zi, d_qi, d_w] if csa else [])
     h2d = sum(t.numel() * t.element_size() for t in copied)
     d2h = h_out.numel() * h_out.element_size()
-    clk = clocks.stop()
     cache.check_device_error()
     # ---- max over ranks
     step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms or 0.0], ws, "cuda")
