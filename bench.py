@@ -78,6 +78,15 @@ def _profiled_traffic():
     return int(fields["traffic_bytes_per_launch"])
 
 
+def workload_config(wl, ws: int) -> dict:
+    """The `config` object both arms print."""
+    return {"workload": wl.name, "context": wl.context, "batch_per_gpu": wl.batch, "heads": wl.H,
+            "head_dim": wl.D, "rope_dims": wl.R, "indexer": f"{wl.H_I}x{wl.d_I}", "topk": wl.k,
+            "window": wl.W, "layers_per_step": 1,
+            "l2": "flushed before every timed step: 256 MB written, then 256 MB read (not timed)",
+            "parallelism": f"request-sharded x{ws}"}
+
+
 def rank_seed(wl, rank: int) -> int:
     """Seed of the requests a rank owns: ranks hold disjoint requests."""
     return wl.seed + 7919 * rank
@@ -406,11 +415,7 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
         "ms_per_step": step_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32 on mxfp4/fp8/bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "context": T0, "batch_per_gpu": B, "heads": wl.H,
-                   "head_dim": wl.D, "rope_dims": wl.R, "indexer": f"{wl.H_I}x{wl.d_I}",
-                   "topk": wl.k, "window": wl.W, "layers_per_step": 1,
-                   "l2": "flushed before every timed step: 256 MB written, then 256 MB read (not timed)",
-                   "parallelism": f"request-sharded x{ws}"},
+        "config": workload_config(wl, ws),
         "gpu_launches": launches,
         "step_breakdown_us": breakdown,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
@@ -505,21 +510,25 @@ def cpu_baseline(wl, budget_s: float = 15.0):
 
 
 def run_reference(args):
+    """The oracle, as it stands, timed on the host cores.  A step is a
+    bounded sample of the workload: q queries of one request (q <= batch,
+    chosen from the warm-up so that the whole run stays within ~3 minutes)."""
     ws, rank, _ = _dist()
     if rank != 0:
         return
     wl = I.WORKLOADS[args.workload]
     setup = oracle_setup(wl)
-    oracle_queries(wl, setup, n=args.warmup)                  # untimed warm-up queries
-    done, el = oracle_queries(wl, setup, n=args.steps * wl.batch)
+    _, el_w = oracle_queries(wl, setup, n=args.warmup)       # untimed warm-up queries
+    per_q = el_w / max(args.warmup, 1)
+    q_step = max(1, min(wl.batch, int(180.0 / max(per_q * args.steps, 1e-9))))
+    done, el = oracle_queries(wl, setup, n=args.steps * q_step)
     value = done / el
+    sample = _sample_text(wl, done, el) + f"; {q_step} quer{'y' if q_step == 1 else 'ies'} per step"
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "context": wl.context, "batch_per_gpu": wl.batch, "heads": wl.H,
-                       "head_dim": wl.D, "topk": wl.k},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-                             "sample": _sample_text(wl, done, el)},
+            "config": workload_config(wl, ws),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
