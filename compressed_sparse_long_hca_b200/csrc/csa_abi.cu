@@ -306,6 +306,7 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
   if (n == 0) return CSA_OK;
   if (!req_ids || !q || !sink || !out) return fail(CSA_ERR_ARG, "NULL argument");
+  if (reinterpret_cast<uintptr_t>(q) % 16) return fail(CSA_ERR_ARG, "q must be 16-byte aligned");
   const bool is_csa = layer < c->L.n_csa;
   if (is_csa && (!topk_idx || k < 1)) return fail(CSA_ERR_ARG, "CSA layer needs topk_idx and k >= 1");
   if (!is_csa && topk_idx) return fail(CSA_ERR_ARG, "HCA layer takes topk_idx == NULL");
@@ -339,6 +340,7 @@ csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* c, int32_t layer, int3
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
   if (n == 0) return CSA_OK;
   if (!req_ids || !q || !sink || !out) return fail(CSA_ERR_ARG, "NULL argument");
+  if (reinterpret_cast<uintptr_t>(q) % 16) return fail(CSA_ERR_ARG, "q must be 16-byte aligned");
   const bool is_csa = layer < c->L.n_csa;
   if (is_csa && (!topk_idx || k < 1)) return fail(CSA_ERR_ARG, "CSA layer needs topk_idx and k >= 1");
   if (!is_csa && topk_idx) return fail(CSA_ERR_ARG, "HCA layer takes topk_idx == NULL");

@@ -217,7 +217,7 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
  * K = V = the stored row (FP8 x scale, BF16).  With q rotated at t:
  *   u_hr = scale * q_h . K_r,  mu_h = max(max_r u_hr, sink_h)
  *   out_h = sum_r e^{u_hr-mu_h} V_r / (sum_r e^{u_hr-mu_h} + e^{sink_h-mu_h})
- *   q     device uint16 (BF16) [n][H][D]   before RoPE
+ *   q     device uint16 (BF16) [n][H][D]   before RoPE; 16-byte aligned
  *   sink  device float [H]
  *   out   device uint16 (BF16) [n][H][D]
  * Source: page "V4终于终于终于终于是来了", sections "CSA——压缩稀疏注意力"
