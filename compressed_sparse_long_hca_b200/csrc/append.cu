@@ -22,9 +22,11 @@
 // ring row and tail slot; the entry it completes, if any).  With one new
 // token the tail slot it overwrites is never one the completed entry reads
 // (the entry's older tokens sit in the other slots of the ring), so the two
-// roles can run concurrently.  Every CTA reads the lengths first and then
-// takes a ticket; the CTA with the last ticket advances the lengths and
-// resets the ticket for the next call.
+// roles can run concurrently.  Both CTAs of a request read its length first
+// and then take a ticket of the request; the second one advances the length
+// (with the value both read) and resets the ticket for the next call.  The
+// token CTA loads its inputs before the request's state, so that the two
+// round trips overlap.
 #include "common.cuh"
 
 namespace csa {
@@ -75,15 +77,12 @@ __device__ __forceinline__ bool load_request(const AppendArgs& a, int i, int& re
 
 // ---------------------------------------------------------------- launch 1
 
-__device__ void csa_entries_body(const AppendArgs& a, int i, int y0, int ystride, float* sm) {
+__device__ void csa_entries_body(const AppendArgs& a, int i, int req, int64_t L0, int y0, int ystride, float* sm) {
   const Layout& L = a.L;
   const int D = L.D, R = L.R, dI = L.dI;
   float* row = sm;            // [D]
   float* key = sm + D;        // [dI]
   float* red = key + dI;      // [32]
-  int req;
-  int64_t L0;
-  if (!load_request(a, i, req, L0)) return;
   const int64_t n_done = (L0 + a.n_tok) / kCsaM;    // entries complete after the call
   const float* tc = reinterpret_cast<const float*>(L.tail(req, a.layer));
   const float* tz = tc + kCsaWin * D;
@@ -135,14 +134,11 @@ __device__ void csa_entries_body(const AppendArgs& a, int i, int y0, int ystride
   }
 }
 
-__device__ void hca_entries_body(const AppendArgs& a, int i, int y0, int ystride, float* sm) {
+__device__ void hca_entries_body(const AppendArgs& a, int i, int req, int64_t L0, int y0, int ystride, float* sm) {
   const Layout& L = a.L;
   const int D = L.D, R = L.R;
   float* row = sm;
   float* red = sm + D;
-  int req;
-  int64_t L0;
-  if (!load_request(a, i, req, L0)) return;
   const int64_t n_done = (L0 + a.n_tok) / kHcaM;
   const float* tc = reinterpret_cast<const float*>(L.tail(req, a.layer));
   const float* tz = tc + kHcaM * D;
@@ -181,12 +177,18 @@ __device__ void hca_entries_body(const AppendArgs& a, int i, int y0, int ystride
 
 __global__ void __launch_bounds__(256) csa_entries_kernel(AppendArgs a) {
   extern __shared__ float sm[];
-  csa_entries_body(a, blockIdx.x, blockIdx.y, gridDim.y, sm);
+  int req;
+  int64_t L0;
+  if (!load_request(a, blockIdx.x, req, L0)) return;
+  csa_entries_body(a, blockIdx.x, req, L0, blockIdx.y, gridDim.y, sm);
 }
 
 __global__ void __launch_bounds__(256) hca_entries_kernel(AppendArgs a) {
   extern __shared__ float sm[];
-  hca_entries_body(a, blockIdx.x, blockIdx.y, gridDim.y, sm);
+  int req;
+  int64_t L0;
+  if (!load_request(a, blockIdx.x, req, L0)) return;
+  hca_entries_body(a, blockIdx.x, req, L0, blockIdx.y, gridDim.y, sm);
 }
 
 // ---------------------------------------------------------------- launch 2
@@ -258,33 +260,86 @@ __global__ void length_kernel(AppendArgs a) {
 
 // ---------------------------------------------------------------- decode: one launch
 
+// The decode token (n_tok == 1) of request slot i: its ring row and tail
+// slot.  The token's inputs and RoPE frequencies are loaded before the
+// request's state; returns false when the request is skipped.
+__device__ bool token1_body(const AppendArgs& a, int i, float* sm, int& req, int64_t& L0) {
+  const Layout& L = a.L;
+  const int D = L.D, R = L.R, dI = L.dI;
+  const bool csa = a.layer < L.n_csa;
+  float* row = sm;
+  float* red = sm + D;
+  const int t = threadIdx.x;                 // 256 threads, D <= 512
+  const float* c = a.c + (int64_t)i * D;
+  const float* z = a.z + (int64_t)i * D;
+  const float c0 = t < D ? c[t] : 0.f, c1 = t + 256 < D ? c[t + 256] : 0.f;
+  const float z0 = t < D ? z[t] : 0.f, z1 = t + 256 < D ? z[t + 256] : 0.f;
+  float ci0 = 0.f, zi0 = 0.f;
+  if (csa && t < dI) {
+    ci0 = a.ci[(int64_t)i * dI + t];
+    zi0 = a.zi[(int64_t)i * dI + t];
+  }
+  const double th = t < R / 2 ? L.theta()[t] : 0.0;
+  if (!load_request(a, i, req, L0)) return false;
+  const int64_t pos = L0;
+  if (t < D) row[t] = c0;
+  if (t + 256 < D) row[t + 256] = c1;
+  __syncthreads();
+  if (t < R / 2) rope_pair(row[D - R + 2 * t], row[D - R + 2 * t + 1], th, pos);
+  __syncthreads();
+  char* st = L.state(req, a.layer);
+  const int slot = (int)(pos % kWindow);
+  store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),
+               reinterpret_cast<uint16_t*>(st + L.ring_bf16) + (int64_t)slot * R,
+               reinterpret_cast<float*>(st + L.ring_scale) + slot, red);
+  // tail slot (an HCA block completed by this token needs no tail)
+  if (csa || (pos + 1) % kHcaM != 0) {
+    float* tail = reinterpret_cast<float*>(L.tail(req, a.layer));
+    const int ring = csa ? kCsaWin : kHcaM;
+    const int ts = (int)(pos % ring);
+    if (t < D) { tail[(int64_t)ts * D + t] = c0; tail[(int64_t)ring * D + (int64_t)ts * D + t] = z0; }
+    if (t + 256 < D) {
+      tail[(int64_t)ts * D + t + 256] = c1;
+      tail[(int64_t)ring * D + (int64_t)ts * D + t + 256] = z1;
+    }
+    if (csa && t < dI) {
+      float* ti = tail + 2 * (int64_t)ring * D;
+      ti[(int64_t)ts * dI + t] = ci0;
+      ti[(int64_t)ring * dI + (int64_t)ts * dI + t] = zi0;
+    }
+  }
+  return true;
+}
+
 // grid (n, 2): blockIdx.y 0 = the token's ring row and tail slot, 1 = the
-// entry it completes (if any).  n_tok == 1.
+// entry it completes (if any).  n_tok == 1, request slots distinct.
 __global__ void __launch_bounds__(256) append_decode_kernel(AppendArgs a) {
   extern __shared__ float sm[];
-  __shared__ int s_last;
   const Layout& L = a.L;
   const int i = blockIdx.x;
-  if (blockIdx.y == 0) tokens_body(a, i, 0, 1, sm);
-  else if (a.layer < L.n_csa) csa_entries_body(a, i, 0, 1, sm);
-  else hca_entries_body(a, i, 0, 1, sm);
-  // every read of the lengths by this CTA is done; the last ticket advances them
+  int req;
+  int64_t L0;
+  bool ok;
+  if (blockIdx.y == 0) {
+    ok = token1_body(a, i, sm, req, L0);
+  } else {
+    ok = load_request(a, i, req, L0);
+    if (ok) {
+      if (a.layer < L.n_csa) csa_entries_body(a, i, req, L0, 0, 1, sm);
+      else hca_entries_body(a, i, req, L0, 0, 1, sm);
+    }
+  }
+  if (!ok) return;   // both CTAs of the request skip it alike
+  // both CTAs of the request have read its length; the second advances it
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    s_last = atomicAdd(L.ticket(a.layer), 1) == (int)(gridDim.x * gridDim.y) - 1;
+    int32_t* tk = L.ticket(a.layer, req);
+    if (atomicAdd(tk, 1) == 1) {
+      *tk = 0;
+      L.lengths()[(int64_t)a.layer * L.max_req + req] = L0 + a.n_tok;
+    }
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int x = threadIdx.x; x < a.n; x += blockDim.x) {
-    const int req = a.req_ids[x];
-    if (req < 0 || req >= L.max_req) continue;
-    int64_t* len = L.lengths() + (int64_t)a.layer * L.max_req + req;
-    const int64_t cap = (int64_t)L.capacity()[req] * kPageTokens;
-    if (*len + a.n_tok <= cap) *len += a.n_tok;
-  }
-  if (threadIdx.x == 0) *L.ticket(a.layer) = 0;
 }
 
 cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok,

@@ -117,7 +117,7 @@ Layout make_layout(const csa_cfg& c) {
   // arena sections
   int64_t o = 0;
   L.off_err = o; o += A;
-  L.off_tick = o; o = align_up(o + (int64_t)L.n_layers * 4, A);
+  L.off_tick = o; o = align_up(o + (int64_t)L.n_layers * L.max_req * 4, A);
   L.off_len = o; o = align_up(o + (int64_t)L.n_layers * L.max_req * 8, A);
   L.off_cap = o; o = align_up(o + (int64_t)L.max_req * 4, A);
   L.off_pt = o; o = align_up(o + (int64_t)L.max_req * L.max_pages_per_req * 4, A);

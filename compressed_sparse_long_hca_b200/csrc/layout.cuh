@@ -13,7 +13,7 @@
 //
 // Arena (one caller-owned device buffer, every section 256-byte aligned):
 //   header      error word (int32 code, int32 detail, int64 info)
-//   tickets     int32 [n_layers]                  CTA tickets of the one-launch append
+//   tickets     int32 [n_layers][max_req]         CTA tickets of the one-launch append
 //   lengths     int64 [n_layers][max_req]         tokens appended so far
 //   capacity    int32 [max_req]                   pages held by the request
 //   page table  int32 [max_req][max_pages_per_req]  logical -> pool page
@@ -87,7 +87,9 @@ struct Layout {
     return reinterpret_cast<int32_t*>(base + off_pt) + (int64_t)req * max_pages_per_req;
   }
   __host__ __device__ int32_t* err() const { return reinterpret_cast<int32_t*>(base + off_err); }
-  __host__ __device__ int32_t* ticket(int layer) const { return reinterpret_cast<int32_t*>(base + off_tick) + layer; }
+  __host__ __device__ int32_t* ticket(int layer, int req) const {
+    return reinterpret_cast<int32_t*>(base + off_tick) + (int64_t)layer * max_req + req;
+  }
   // RoPE frequencies base^(-2i/R), i < R/2, in fp64 (written at initialisation)
   __host__ __device__ const double* theta() const { return reinterpret_cast<const double*>(base + off_theta); }
   __host__ __device__ const float* bpos_csa(int layer) const {

@@ -81,7 +81,9 @@ struct TopkShared {
   int sel_hist[kBins];      // histogram of block_select
   uint32_t list[kTopkThreads];  // block_select: the keys of one bin
   int wsum[32];
-  uint32_t mm[2][32];       // per-warp min / max
+  int scan_a[32], scan_b[32];   // warp totals of the one-barrier scans (one buffer per call site)
+  int selw[2][32];          // block_select: warp totals of a round (alternating rounds)
+  uint32_t mm[2][2][32];    // per-warp min / max (one buffer per call site)
   int cnt[2];               // radix path: this CTA's (count > T, count == T)
   int n_cand;               // filter path: this CTA's keys >= tau
   int n_list;
@@ -116,7 +118,24 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
   return before;
 }
 
-// Block-wide (min, max) of E keys per thread (flags mark the valid ones).
+// Exclusive block-wide prefix sum with one barrier: warp scans, warp totals
+// through `buf`.  A later call must not reuse `buf` before another barrier.
+__device__ __forceinline__ int block_scan1(int v, int* buf, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) buf[w] = x;
+  __syncthreads();
+  const int tw = lane < kWarps ? buf[lane] : 0;
+  *total = __reduce_add_sync(0xffffffffu, tw);
+  return __reduce_add_sync(0xffffffffu, lane < w ? tw : 0) + x - v;
+}
+
+// Block-wide (min, max) of E keys per thread (flags mark the valid ones);
+// one barrier (each call site has its own buffer).
 template <int E>
 __device__ __forceinline__ void block_minmax(const uint32_t (&v)[E], const bool (&ok)[E], uint32_t (*mm)[32],
                                              uint32_t* mn, uint32_t* mx) {
@@ -131,37 +150,45 @@ __device__ __forceinline__ void block_minmax(const uint32_t (&v)[E], const bool 
   __syncthreads();
   *mn = __reduce_min_sync(0xffffffffu, mm[0][lane]);
   *mx = __reduce_max_sync(0xffffffffu, mm[1][lane]);
-  __syncthreads();
 }
 
 // The r-th largest of the valid keys (1 <= r <= #valid, every valid key in
 // [kmin, kmax]), exactly: returns T and sets *ties = r - #{keys > T}.  Each
 // round histograms the keys of the current range over up to 2048 equal
 // bins and keeps the bin that holds the r-th key; once that bin holds at
-// most kTopkThreads keys they are ranked against each other.  With
-// exact == false the first round's bin is kept and its lower edge returned
-// (then #{keys >= result} >= r).
+// most kTopkThreads keys they are ranked against each other.  sh.sel_hist
+// must be zero on entry and is zero again on return (each thread clears the
+// bins it has read); sh.n_list likewise.
 template <int E>
 __device__ uint32_t block_select(const uint32_t (&v)[E], const bool (&ok)[E], int r, uint32_t kmin, uint32_t kmax,
-                                 bool exact, TopkShared& sh, int* ties) {
-  const int tid = threadIdx.x;
+                                 TopkShared& sh, int* ties) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   uint64_t base = kmin, width = (uint64_t)kmax - kmin + 1;
   int remaining = r;
-  while (true) {
+  for (int round = 0;; ++round) {
     int shift = 0;
     while (((width - 1) >> shift) >= (uint64_t)kBins) ++shift;
-    for (int b = tid; b < kBins; b += kTopkThreads) sh.sel_hist[b] = 0;
-    __syncthreads();
 #pragma unroll
     for (int e = 0; e < E; ++e)
       if (ok[e] && (uint64_t)v[e] >= base && (uint64_t)v[e] - base < width)
         atomicAdd(&sh.sel_hist[((uint64_t)v[e] - base) >> shift], 1);
     __syncthreads();
-    {   // bin d: (count in bins > d) < remaining <= (count in bins >= d); 2 bins per thread, top first
-      const int b0 = kBins - 2 - 2 * tid;
-      const int c1 = sh.sel_hist[b0 + 1], c0 = sh.sel_hist[b0];
-      int tot;
-      const int before = block_excl_scan(c1 + c0, sh.wsum, &tot);
+    {   // bin d: (count in bins > d) < remaining <= (count in bins >= d).  Warp w
+        // owns bins 64w .. 64w+63, lane l the bins 64w+2l (c0) and 64w+2l+1 (c1).
+      const int b0 = 64 * w + 2 * lane;
+      const int c0 = sh.sel_hist[b0], c1 = sh.sel_hist[b0 + 1];
+      sh.sel_hist[b0] = 0;
+      sh.sel_hist[b0 + 1] = 0;
+      int x = c0 + c1;                                 // suffix sum over lanes >= l
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+      }
+      int* wt = sh.selw[round & 1];
+      if (lane == 0) wt[w] = x;                        // warp total
+      __syncthreads();
+      const int tw = lane < kWarps ? wt[lane] : 0;
+      const int before = __reduce_add_sync(0xffffffffu, lane > w ? tw : 0) + x - (c0 + c1);
       if (before < remaining && before + c1 >= remaining) {
         sh.digit = (uint32_t)(b0 + 1);
         sh.remaining = remaining - before;
@@ -183,13 +210,7 @@ __device__ uint32_t block_select(const uint32_t (&v)[E], const bool (&ok)[E], in
       *ties = remaining;
       return (uint32_t)base;
     }
-    if (!exact) {
-      *ties = 0;
-      return (uint32_t)base;
-    }
     if (in_bin <= kTopkThreads) {   // rank the bin's keys against each other
-      if (tid == 0) sh.n_list = 0;
-      __syncthreads();
 #pragma unroll
       for (int e = 0; e < E; ++e)
         if (ok[e] && (uint64_t)v[e] >= base && (uint64_t)v[e] - base < width) sh.list[atomicAdd(&sh.n_list, 1)] = v[e];
@@ -199,9 +220,9 @@ __device__ uint32_t block_select(const uint32_t (&v)[E], const bool (&ok)[E], in
         const uint32_t x = sh.list[tid];
         int gt = 0, ge = 0;
         for (int y = 0; y < m; ++y) {
-          const uint32_t z = sh.list[y];
-          gt += z > x ? 1 : 0;
-          ge += z >= x ? 1 : 0;
+          const uint32_t zz = sh.list[y];
+          gt += zz > x ? 1 : 0;
+          ge += zz >= x ? 1 : 0;
         }
         if (gt < remaining && remaining <= ge) {   // equal keys write equal values
           sh.digit = x;
@@ -211,7 +232,7 @@ __device__ uint32_t block_select(const uint32_t (&v)[E], const bool (&ok)[E], in
       __syncthreads();
       *ties = sh.remaining;
       const uint32_t T = sh.digit;
-      __syncthreads();
+      if (tid == 0) sh.n_list = 0;   // read above by every thread before the last barrier
       return T;
     }
   }
@@ -390,6 +411,8 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   }
   if (cached)
     for (int64_t x = nbulk + tid; x < len; x += kTopkThreads) keys[x] = __float_as_uint(s[lo + x]);
+  for (int b = tid; b < kBins; b += kTopkThreads) sh.sel_hist[b] = 0;   // block_select's invariant
+  if (tid == 0) sh.n_list = 0;
   __syncthreads();   // the mbarrier is initialised before anyone waits on it
 
   uint32_t sv[kSamplePer];
@@ -401,8 +424,8 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   if (r <= S) {
     uint32_t smin, smax;
     int unused;
-    block_minmax(sv, sok, sh.mm, &smin, &smax);
-    tau = block_select(sv, sok, r, smin, smax, true, sh, &unused);
+    block_minmax(sv, sok, sh.mm[0], &smin, &smax);
+    tau = block_select(sv, sok, r, smin, smax, sh, &unused);
   }
   if (cached) {
     // all threads observe the copy's completion (bounded wait)
@@ -457,7 +480,7 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     }
   }
   int cta_cnt;
-  const int w_before = __shfl_sync(0xffffffffu, block_excl_scan(lane == 0 ? wc : 0, sh.wsum, &cta_cnt), 0);
+  const int w_before = __shfl_sync(0xffffffffu, block_scan1(lane == 0 ? wc : 0, sh.scan_a, &cta_cnt), 0);
   if (tid == 0) sh.n_cand = cta_cnt;
   cluster.sync();
   int base, total;
@@ -522,9 +545,9 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
       cv[e] = cok[e] ? sh.u.cand[e0 + e].x : 0u;
     }
     uint32_t cmin, cmax;
-    block_minmax(cv, cok, sh.mm, &cmin, &cmax);
+    block_minmax(cv, cok, sh.mm[1], &cmin, &cmax);
     int ties_needed;
-    const uint32_t T = block_select(cv, cok, k, tau, cmax, true, sh, &ties_needed);
+    const uint32_t T = block_select(cv, cok, k, tau, cmax, sh, &ties_needed);
     // one scan of (count > T, count == T) packed in 16-bit halves (counts <= kCandCap)
     int ngt = 0, neq = 0;
 #pragma unroll
@@ -533,7 +556,7 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
       neq += (cok[e] && cv[e] == T) ? 1 : 0;
     }
     int packed_tot;
-    const int packed = block_excl_scan(ngt | (neq << 16), sh.wsum, &packed_tot);
+    const int packed = block_scan1(ngt | (neq << 16), sh.scan_b, &packed_tot);
     const int gt_before = packed & 0xFFFF, eq_before = packed >> 16;
     int seen = eq_before;
     unsigned take_bits = 0;
