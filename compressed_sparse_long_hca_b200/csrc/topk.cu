@@ -10,7 +10,8 @@
 // copy brings into shared memory when it fits.
 //
 // Filter path (the usual case).
-//   1. Threshold.  Every CTA reads the same strided sample of S keys and
+//   1. Threshold.  Every CTA reads the same sample of S keys (64 evenly
+//      spaced runs of 64 consecutive keys) and
 //      takes tau = the sample's r-th largest key, r chosen so that with
 //      overwhelming probability fewer than r sampled keys lie above the
 //      query's k-th key; then every key of the top k is >= tau, and about
@@ -386,15 +387,18 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   const int64_t hi = lo + chunk < N ? lo + chunk : N;
   const int64_t len = hi - lo;
 
-  // ---- 1. threshold from a strided sample (the same sample in every CTA)
+  // ---- 1. threshold from a sample (the same sample in every CTA)
   const int S = N < kSample ? (int)N : kSample;
   float sraw[kSamplePer];         // loads issued here, used after the bulk copy is on its way
   bool sok[kSamplePer];
+  // 64 evenly spaced runs of 64 consecutive scores (coalesced loads); all of
+  // them when N < 4096
 #pragma unroll
   for (int e = 0; e < kSamplePer; ++e) {
     const int x = tid + e * kTopkThreads;
     sok[e] = x < S;
-    sraw[e] = sok[e] ? s[(int64_t)x * N / S] : 0.f;
+    const int64_t pos = S < kSample ? (int64_t)x : (int64_t)(x / 64) * (N / 64) + (x % 64);
+    sraw[e] = sok[e] ? s[pos] : 0.f;
   }
   // ---- slice -> shared memory: one bulk copy of the 16-byte aligned part
   const bool cached = a.cache_keys != 0;

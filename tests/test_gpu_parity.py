@@ -203,20 +203,23 @@ def test_topk_exact_large(N, k):
 
 
 def test_topk_rows_that_defeat_or_stress_the_sample_filter():
-    """The selector estimates a threshold from a strided sample (every
-    N/4096-th score).  Rows whose sample lies about the top k must still
-    come out exact: a sample made of the largest scores (too few pass the
-    threshold), a top k hidden between the sampled positions, and a tie
-    class at the k-th score."""
+    """The selector estimates a threshold from a sample of the scores (64
+    evenly spaced runs of 64 consecutive scores).  Rows whose sample lies
+    about the top k must still come out exact: a sample made of the largest
+    scores (too few pass the threshold), a top k hidden outside the sample,
+    and a tie class at the k-th score."""
     N, k = 262144, 1024
+    x = np.arange(4096)
+    sampled = (x // 64) * (N // 64) + x % 64
+    unsampled = (x // 64) * (N // 64) + 64 + x % 64
     r = np.random.default_rng(99)
     base = r.standard_normal(N).astype(np.float32)
     lying = base.copy()
-    lying[::64] = 100.0 + np.arange(N // 64, dtype=np.float32)      # the sample sees only these
+    lying[sampled] = 100.0 + np.arange(4096, dtype=np.float32)        # the sample sees only these
     hidden = base.copy()
-    hidden[1::64][:k] = 50.0 + r.random(k).astype(np.float32)       # never sampled
+    hidden[unsampled[:k]] = 50.0 + r.random(k).astype(np.float32)     # never sampled
     ties = base.copy()
-    ties[r.choice(N, 3000, replace=False)] = 3.0                     # the k-th score is a 3000-way tie
+    ties[r.choice(N, 3000, replace=False)] = 3.0                       # the k-th score is a 3000-way tie
     _topk_case([lying, hidden, ties], k)
 
 
