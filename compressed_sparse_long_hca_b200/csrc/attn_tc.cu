@@ -158,6 +158,28 @@ __device__ __forceinline__ uint4 ld_nc16(const void* p) {
   return v;
 }
 
+// Reduction over the 32 lanes of a warp of 16 values per lane (lane = row,
+// value e = head e), by exchanging halves: 16 shuffles.  Lane l returns the
+// reduction for head l >> 1 (lanes 2h and 2h+1 hold the same value).  The
+// order of the operations is fixed.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce16(const float (&v)[16], int lane) {
+  auto op = [](float x, float y) { return kMax ? fmaxf(x, y) : x + y; };
+  float a8[8], a4[4], a2[2];
+  const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    a8[j] = op(u16 ? v[8 + j] : v[j], __shfl_xor_sync(0xffffffffu, u16 ? v[j] : v[8 + j], 16));
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    a4[j] = op(u8 ? a8[4 + j] : a8[j], __shfl_xor_sync(0xffffffffu, u8 ? a8[j] : a8[4 + j], 8));
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    a2[j] = op(u4 ? a4[2 + j] : a4[j], __shfl_xor_sync(0xffffffffu, u4 ? a4[j] : a4[2 + j], 4));
+  const float a1 = op(u2 ? a2[1] : a2[0], __shfl_xor_sync(0xffffffffu, u2 ? a2[0] : a2[1], 2));
+  return op(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+}
+
 // Address of row `r` of tile `tt`; returns whether the row exists.
 __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& g, int i, int tt, int r,
                                             uint64_t* rowf8, uint64_t* rowbf, float* rsc) {
@@ -439,22 +461,18 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
         const bool valid = rowf8[r] != 0;
         const float rs = rsc[r];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 16; ++e)
           u[e] = valid ? fmaf(rs, __uint_as_float(sv[e]), __uint_as_float(sr[e])) * a.scale : -INFINITY;
-          stage[r * (G + 1) + hb + e] = u[e];
-        }
+        // max over this warp's 32 rows, per head; then over the 4 row warps
+        const float mx = warp_reduce16<true>(u, lane);
+        if ((lane & 1) == 0) part[(warp & 3) * 32 + hb + (lane >> 1)] = mx;
       }
       ok = __syncthreads_and(ok) != 0;
       if (!ok) break;
-      if (warp < 4 && lane < G) {   // warp w, lane h: max over rows 32w .. 32w+31 of head h
-        float mx = -INFINITY;
-        for (int x = 0; x < 32; ++x) mx = fmaxf(mx, stage[(warp * 32 + x) * (G + 1) + lane]);
-        part[warp * 32 + lane] = mx;
-      }
-      __syncthreads();
       if (tid < G) m_t[tid] = fmaxf(fmaxf(part[tid], part[32 + tid]), fmaxf(part[64 + tid], part[96 + tid]));
       __syncthreads();
       // -- p = exp(u - m_t): P^T and (P * row scale)^T in BF16 for PV, fp32 p for the sums
+      float pv[16];
       if (tw) {
         const float rs = rsc[r];
 #pragma unroll
@@ -465,8 +483,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
             const int h = hb + hg * 8 + e;
             const float p0 = expf(u[hg * 8 + e] - m_t[h]);
             const float p1 = expf(u[hg * 8 + e + 1] - m_t[h + 1]);
-            stage[r * (G + 1) + h] = p0;
-            stage[r * (G + 1) + h + 1] = p1;
+            pv[hg * 8 + e] = p0;
+            pv[hg * 8 + e + 1] = p1;
             pk[e >> 1] = (uint32_t)bf16_rn(p0) | ((uint32_t)bf16_rn(p1) << 16);
             pm[e >> 1] = (uint32_t)bf16_rn(p0 * rs) | ((uint32_t)bf16_rn(p1 * rs) << 16);
           }
@@ -498,11 +516,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
         __syncwarp();
       }
       ++n_done;
-      // -- l_t: row sums of p per head, fixed order
-      if (warp < 4 && lane < G) {
-        float sum = 0.f;
-        for (int x = 0; x < 32; ++x) sum += stage[(warp * 32 + x) * (G + 1) + lane];
-        part[warp * 32 + lane] = sum;
+      // -- l_t: row sums of p per head, in a fixed order (warp tree, then the 4 row warps)
+      if (tw) {
+        const float sm_ = warp_reduce16<false>(pv, lane);
+        if ((lane & 1) == 0) part[(warp & 3) * 32 + hb + (lane >> 1)] = sm_;
       }
       __syncthreads();
       if (tid < G) l_t[tid] = ((part[tid] + part[32 + tid]) + part[64 + tid]) + part[96 + tid];
