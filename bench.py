@@ -208,7 +208,7 @@ def run_gpu(args):
     import torch.distributed as dist
 
     from compressed_sparse_long_hca_b200 import _lib
-    from compressed_sparse_long_hca_b200.api import Cache, topk
+    from compressed_sparse_long_hca_b200.api import Cache, DecodeStep, topk
 
     ws, rank, local = _dist()
     torch.cuda.set_device(local)
@@ -219,7 +219,7 @@ def run_gpu(args):
     B, T0 = wl.batch, wl.context
     csa = wl.kind == "csa"
     steps, warm = args.steps, args.warmup
-    cap = T0 + 4 * steps + warm + 256
+    cap = T0 + 5 * steps + warm + 256       # every timed or warm-up step appends one token
     nb = (cap + 511) // 512
     layer = 0
     b_kv, b_idx, sink = I.layer_params(wl.seed, layer, wl.kind, wl.D, wl.d_I or 32, wl.H)
@@ -367,44 +367,47 @@ def run_gpu(args):
     idx_ms = idx_sum[0] / steps if csa else None
     breakdown = {nm: round(v / steps * 1e3, 2) for nm, v in part_ms.items()}
     del g_plain, g_idx, g_all
-    # ---- end to end through the public API with host buffers
-    pin = lambda t: t.cpu().pin_memory() if t is not None else None
-    h_c, h_z, h_ci, h_zi = pin(step_c[:steps]), pin(step_z[:steps]), pin(step_ci[:steps] if csa else None), \
-        pin(step_zi[:steps] if csa else None)
-    h_q, h_qi, h_w = pin(q), pin(qi), pin(w)
-    h_out = torch.empty((B, wl.H, wl.D), dtype=torch.bfloat16).pin_memory()
-    d_c, d_z = torch.empty_like(step_c[0]), torch.empty_like(step_z[0])
-    d_ci = torch.empty_like(step_ci[0]) if csa else None
-    d_zi = torch.empty_like(step_zi[0]) if csa else None
-    d_q, d_qi, d_w = torch.empty_like(q), torch.empty_like(qi) if csa else None, torch.empty_like(w) if csa else None
-    h2d = 0
+    # ---- end to end through the public API with host buffers: DecodeStep
+    # copies each step's packed inputs from pinned host memory in one
+    # transfer, replays the step and copies the output back in one transfer
+    e2e = DecodeStep(cache, layer, list(range(B)), wl.k if csa else 0, sink_d)
+    host_in = []
+    for s in range(steps):                  # each step's own inputs, packed up front (not timed)
+        buf = e2e.new_host_inputs()
+        v = e2e.views(buf)
+        v["q"].copy_(q.cpu())
+        v["c"].copy_(step_c[s].cpu())
+        v["z"].copy_(step_z[s].cpu())
+        if csa:
+            v["ci"].copy_(step_ci[s].cpu())
+            v["zi"].copy_(step_zi[s].cpu())
+            v["q_idx"].copy_(qi.cpu())
+            v["w"].copy_(w.cpu())
+        host_in.append(buf)
     e2e_ms = 0.0
     for s in range(steps):
         flush_l2()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        d_c.copy_(h_c[s], non_blocking=True)
-        d_z.copy_(h_z[s], non_blocking=True)
-        d_q.copy_(h_q, non_blocking=True)
-        if csa:
-            d_ci.copy_(h_ci[s], non_blocking=True)
-            d_zi.copy_(h_zi[s], non_blocking=True)
-            d_qi.copy_(h_qi, non_blocking=True)
-            d_w.copy_(h_w, non_blocking=True)
-        cache.compress_append(layer, rid, d_c, d_z, d_ci, d_zi)
-        if csa:
-            cache.index_scores(layer, rid, d_qi, d_w, scores, nv)
-            topk(scores, nv, wl.k, idx)
-            cache.decode_attn(layer, rid, d_q, idx, sink_d, out)
-        else:
-            cache.decode_attn(layer, rid, d_q, None, sink_d, out)
-        h_out.copy_(out, non_blocking=True)
+        e2e(host_in[s])
         b.record(stream)
         b.synchronize()
         e2e_ms += a.elapsed_time(b)
-    copied = [d_c, d_z, d_q] + ([d_ci, d_zi, d_qi, d_w] if csa else [])
-    h2d = sum(t.numel() * t.element_size() for t in copied)
-    d2h = h_out.numel() * h_out.element_size()
+    # the same again with marks between the phases (input copy, step, output copy)
+    phase = [0.0, 0.0, 0.0]
+    for s in range(steps):
+        flush_l2()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        e2e(host_in[s], marks=(ev[1], ev[2]))
+        ev[3].record(stream)
+        ev[3].synchronize()
+        for x in range(3):
+            phase[x] += ev[x].elapsed_time(ev[x + 1])
+    e2e_phases = {nm: round(v / steps * 1e3, 2) for nm, v in zip(("h2d", "step", "d2h"), phase)}
+    h2d = e2e.input_bytes
+    d2h = e2e.host_out.numel() * e2e.host_out.element_size()
+    del e2e
     cache.check_device_error()
     # ---- max over ranks
     step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms or 0.0], ws, "cuda")
@@ -418,7 +421,8 @@ def run_gpu(args):
         "config": workload_config(wl, ws),
         "gpu_launches": launches,
         "step_breakdown_us": breakdown,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "phases_us": e2e_phases},
         "clocks": clk,
     }
     if csa:

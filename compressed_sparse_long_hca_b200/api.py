@@ -193,6 +193,132 @@ def topk(scores: torch.Tensor, n_valid: torch.Tensor, k: int, out: torch.Tensor,
                        VARIANTS[variant], _stream(stream)), "csa_topk")
 
 
+# ---------------------------------------------------------------- one decode step, replayed
+
+def decode_step_fields(n: int, H: int, D: int, H_I: int, d_I: int, csa: bool, align: int = 256):
+    """Packed layout of one decode step's inputs: a list of (name, dtype,
+    shape, byte offset, bytes) with every field starting on an `align`-byte
+    boundary, and the buffer's total size."""
+    fields = [("q", torch.bfloat16, (n, H, D)), ("c", torch.float32, (n, 1, D)),
+              ("z", torch.float32, (n, 1, D))]
+    if csa:
+        fields += [("ci", torch.float32, (n, 1, d_I)), ("zi", torch.float32, (n, 1, d_I)),
+                   ("q_idx", torch.float32, (n, H_I, d_I)), ("w", torch.float32, (n, H_I))]
+    out, off = [], 0
+    for name, dtype, shape in fields:
+        nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        out.append((name, dtype, shape, off, nbytes))
+        off += (nbytes + align - 1) // align * align
+    return out, off
+
+
+class DecodeStep:
+    """One decode step of a fixed batch of requests on one layer, captured
+    once as a CUDA graph and replayed every step.
+
+    The step appends each request's new token (csa_compress_append), then on
+    a CSA layer scores the index keys (csa_index_scores), selects the top k
+    (csa_topk) and attends (csa_hca_decode_attn); on an HCA layer it attends
+    over every compressed entry.  The step's inputs travel from one pinned
+    host buffer in one host-to-device copy, its output returns in one
+    device-to-host copy, all on one stream.
+
+    Inputs of a step, packed in a buffer from `new_host_inputs()` and filled
+    through `views(buf)`: q [n, H, D] bf16, c and z [n, 1, D] fp32 (the
+    token's KV candidate and gate logits), on a CSA layer also ci and zi
+    [n, 1, d_I] fp32, q_idx [n, H_I, d_I] fp32 and w [n, H_I] fp32.  Each
+    field starts on a 256-byte boundary.
+
+    The graph holds device pointers, so the batch (req_ids), k and the sink
+    logits are fixed at construction.  On a CSA layer construction runs the
+    index and top-k kernels once (they change nothing in the cache) so that
+    their one-time launch set-up happens before the capture."""
+
+    def __init__(self, cache: Cache, layer: int, req_ids, k: int, sink, variant: str = "auto",
+                 device: str | torch.device = "cuda"):
+        self.cache, self.layer, self.k, self.variant = cache, layer, int(k), variant
+        self.csa = layer < cache.n_csa
+        ids = [int(r) for r in req_ids]
+        n = self.n = len(ids)
+        if n == 0:
+            raise ValueError("a decode step needs at least one request")
+        if self.csa and self.k <= 0:
+            raise ValueError("a CSA layer needs k > 0")
+        H, D = cache.H, cache.D
+        self._fields, off = decode_step_fields(n, H, D, cache.H_I, cache.d_I, self.csa)
+        self.input_bytes = off
+        dev = torch.device(device)
+        self._dev_in = torch.zeros(off, dtype=torch.uint8, device=dev)
+        d = self.views(self._dev_in)
+        self._req = torch.tensor(ids, dtype=torch.int32, device=dev)
+        self._sink = (sink if isinstance(sink, torch.Tensor) else torch.from_numpy(np.asarray(sink, np.float32)))
+        self._sink = self._sink.to(device=dev, dtype=torch.float32).contiguous()
+        self.out = torch.empty((n, H, D), dtype=torch.bfloat16, device=dev)
+        self.host_out = torch.empty((n, H, D), dtype=torch.bfloat16).pin_memory()
+        self._ws = torch.empty(max(cache.attn_workspace_bytes(layer, n, self.k if self.csa else 0), 16),
+                               dtype=torch.uint8, device=dev)
+        if self.csa:
+            n_max = max(cache.cfg.max_pages_per_request * 128, 128)   # 512 tokens = 128 entries per page
+            self._scores = torch.empty((n, n_max), dtype=torch.float32, device=dev)
+            self._nv = torch.empty(n, dtype=torch.int32, device=dev)
+            self._idx = torch.empty((n, self.k), dtype=torch.int32, device=dev)
+
+        def select():
+            cache.index_scores(layer, self._req, d["q_idx"], d["w"], self._scores, self._nv, variant)
+            topk(self._scores, self._nv, self.k, self._idx, variant)
+
+        if self.csa:
+            # one eager pass of the selection kernels (valid on any cache
+            # state, an empty request included) does their one-time launch
+            # set-up (cluster-size query) outside the capture
+            select()
+            torch.cuda.synchronize(dev)
+            cache.check_device_error()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            cache.compress_append(layer, self._req, d["c"], d["z"], d.get("ci"), d.get("zi"))
+            if self.csa:
+                select()
+            cache.decode_attn(layer, self._req, d["q"], self._idx if self.csa else None, self._sink, self.out,
+                              variant=variant, workspace=self._ws)
+        torch.cuda.synchronize(dev)
+
+    def views(self, buf: torch.Tensor) -> dict:
+        """Typed views of the step's input fields inside a packed buffer."""
+        if buf.dtype != torch.uint8 or buf.numel() < self.input_bytes or not buf.is_contiguous():
+            raise ValueError(f"a packed input buffer is {self.input_bytes} contiguous bytes")
+        return {name: buf[off: off + nbytes].view(dtype).view(shape)
+                for name, dtype, shape, off, nbytes in self._fields}
+
+    def new_host_inputs(self) -> torch.Tensor:
+        """A pinned host buffer for one step's packed inputs."""
+        return torch.zeros(self.input_bytes, dtype=torch.uint8).pin_memory()
+
+    def __call__(self, host_inputs: torch.Tensor, marks=None) -> torch.Tensor:
+        """Enqueue one step on the current stream: copy the packed inputs in,
+        replay the step, copy the output [n, H, D] bf16 to `host_out` (pinned),
+        which is returned and is valid once the stream has reached this point.
+        `marks`, two torch.cuda.Events, are recorded after the input copy and
+        after the replay (to time the three phases)."""
+        if host_inputs.device.type != "cpu" or not host_inputs.is_pinned():
+            raise ValueError("host_inputs must be a pinned host buffer (new_host_inputs())")
+        if host_inputs.dtype != torch.uint8 or host_inputs.numel() != self.input_bytes:
+            raise ValueError(f"host_inputs must be {self.input_bytes} bytes")
+        self._dev_in.copy_(host_inputs, non_blocking=True)
+        if marks is not None:
+            marks[0].record()
+        self.graph.replay()
+        if marks is not None:
+            marks[1].record()
+        self.host_out.copy_(self.out, non_blocking=True)
+        return self.host_out
+
+    @property
+    def topk_idx(self) -> torch.Tensor | None:
+        """The last step's selected entries [n, k] (CSA layers)."""
+        return self._idx if self.csa else None
+
+
 # ---------------------------------------------------------------- host row formats
 
 def pack_kv_rows(fp8: np.ndarray, rope_bf16_bits: np.ndarray, scale: np.ndarray) -> np.ndarray:

@@ -60,3 +60,27 @@ def test_init_rejects_bad_arguments_without_launching(cuda_lib):
     # compute calls on a NULL handle fail on the host
     assert cuda_lib.csa_compress_append(None, 0, 1, None, 1, None, None, None, None, None) == -1
     assert cuda_lib.csa_topk(None, 1, None, 1, 1, None, 0, None) == -1
+
+
+def test_decode_step_packed_input_layout():
+    """DecodeStep's packed host buffer: the fields in order, each on a
+    256-byte boundary, sized by shape and dtype, none overlapping."""
+    import math
+
+    import torch
+
+    from compressed_sparse_long_hca_b200.api import decode_step_fields
+    for csa, names in ((True, ["q", "c", "z", "ci", "zi", "q_idx", "w"]), (False, ["q", "c", "z"])):
+        fields, total = decode_step_fields(4, 128, 512, 64, 128, csa)
+        assert [f[0] for f in fields] == names
+        end = 0
+        for name, dtype, shape, off, nbytes in fields:
+            assert off % 256 == 0 and off >= end, name
+            assert nbytes == math.prod(shape) * torch.empty((), dtype=dtype).element_size(), name
+            end = off + nbytes
+        assert total >= end and total % 256 == 0
+    fields, _ = decode_step_fields(4, 128, 512, 64, 128, True)
+    f = {x[0]: x for x in fields}
+    assert f["q"][4] == 4 * 128 * 512 * 2 and f["q"][1] == torch.bfloat16
+    assert f["q_idx"][2] == (4, 64, 128) and f["w"][2] == (4, 64)
+    assert f["c"][2] == (4, 1, 512) and f["ci"][2] == (4, 1, 128)
