@@ -38,7 +38,8 @@
 //   * the rows' addresses are resolved (page table, ring slot) into shared
 //     memory; all threads then gather the rows, 8 rows x 4 16-byte chunks per
 //     warp instruction, dequantise the FP8 codes exactly to BF16 and store
-//     them in the no-swizzle core-matrix order;
+//     them in the no-swizzle core-matrix order (the first tile is gathered by
+//     warps 0-3 alone, while warps 4-7 prepare the query heads);
 //   * QK: S^T[128 rows x G heads] = K_tile Q^T (kind::f16, M = 128 rows,
 //     N = G heads) into TMEM, in two accumulators: the FP8 dims (scaled by
 //     the row's FP8 scale afterwards) and the BF16 RoPE dims;
@@ -287,9 +288,63 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     tc::fence_mbar_init();
   }
   if (tid < 32) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; }
+
+  // gather geometry: chunks of a row are FP8 (16 dims) then BF16 (8 dims);
+  // item `it` of a tile = 8 rows x 4 chunks, one 16-byte load per lane
+  const int nc8 = dmain / 16, nc = nc8 + R / 8;
+  const int n_items = 16 * ((nc + 3) / 4);
+  auto gather_load = [&](int it) -> uint4 {
+    const int r = 8 * (it & 15) + (lane & 7), c = 4 * (it >> 4) + (lane >> 3);
+    if (c < nc8) {
+      const uint8_t* p = reinterpret_cast<const uint8_t*>(rowf8[r]);
+      if (p != nullptr) return ld_nc16(p + 16 * c);
+    } else if (c < nc) {
+      const uint16_t* p = reinterpret_cast<const uint16_t*>(rowbf[r]);
+      if (p != nullptr) return ld_nc16(p + 8 * (c - nc8));
+    }
+    return make_uint4(0, 0, 0, 0);
+  };
+  // dequantise (FP8 -> BF16 is exact) and store in the core-matrix order
+  auto gather_store = [&](int it, const uint4& v) {
+    const int r = 8 * (it & 15) + (lane & 7), c = 4 * (it >> 4) + (lane >> 3);
+    uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
+    if (c < nc8) {
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t pk[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+        const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
+        const float2 f = __half22float2(__half2(h2));
+        pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);
+      }
+      *reinterpret_cast<uint4*>(dst + (2 * c) * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(dst + (2 * c + 1) * 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    } else if (c < nc) {
+      *reinterpret_cast<uint4*>(dst + (dmain / 8 + c - nc8) * 128) = v;
+    }
+  };
+
   int any = 0;
   if (warp < 4) {
     any = resolve_row(a, g, i, tt0, tid, rowf8, rowbf, rsc) ? 1 : 0;
+    // the first tile's rows, gathered by warps 0-3 while warps 4-7 prepare
+    // the query: items warp, warp + 4, ... in two rounds of loads
+    tc::named_bar_sync(2, 128);
+#pragma unroll 1
+    for (int round = 0; round < 2; ++round) {
+      uint4 buf[kMaxLoads];
+#pragma unroll
+      for (int u = 0; u < kMaxLoads; ++u) {
+        const int it = warp + 4 * (round * kMaxLoads + u);
+        buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kMaxLoads; ++u) {
+        const int it = warp + 4 * (round * kMaxLoads + u);
+        if (it < n_items) gather_store(it, buf[u]);
+      }
+    }
   } else {
     // warps 4-7: the query heads h0 .. h0+G-1 rotated at t, BF16, K-major core order
     const int qt = tid - 128;
@@ -344,9 +399,6 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   const int hb = 16 * (warp >> 2);
   const uint32_t id_qk = tc::idesc_bf16(128, G, false, false);
   const uint32_t id_pv = tc::idesc_bf16(128, G, true, true);
-  // gather geometry: chunks of a row are FP8 (16 dims) then BF16 (8 dims)
-  const int nc8 = dmain / 16, nc = nc8 + R / 8;
-  const int n_items = 16 * ((nc + 3) / 4);
   bool ok = true;
   int n_done = 0;                                        // tiles whose PV has been issued
   bool pend_fold = false;
@@ -358,21 +410,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       ok = __syncthreads_and(ok) != 0;
       if (!ok) break;
       tc::tc_fence_after();
-      // -- gather: issue every load of this thread first
+      // -- gather: issue every load of this thread first (the first tile
+      //    was gathered in the prologue)
+      const bool fetch = tt != tt0;
       uint4 buf[kMaxLoads];
+      if (fetch) {
 #pragma unroll
-      for (int u = 0; u < kMaxLoads; ++u) {
-        const int it = warp + 8 * u;
-        buf[u] = make_uint4(0, 0, 0, 0);
-        if (it < n_items) {
-          const int r = 8 * (it & 15) + (lane & 7), c = 4 * (it >> 4) + (lane >> 3);
-          if (c < nc8) {
-            const uint8_t* p = reinterpret_cast<const uint8_t*>(rowf8[r]);
-            if (p != nullptr) buf[u] = ld_nc16(p + 16 * c);
-          } else if (c < nc) {
-            const uint16_t* p = reinterpret_cast<const uint16_t*>(rowbf[r]);
-            if (p != nullptr) buf[u] = ld_nc16(p + 8 * (c - nc8));
-          }
+        for (int u = 0; u < kMaxLoads; ++u) {
+          const int it = warp + 8 * u;
+          buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
         }
       }
       // -- whole-query launch: fold the previous tile while the loads fly
@@ -406,28 +452,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
         }
         pend_fold = false;
       }
-      // -- dequantise and store the tile (FP8 -> BF16 is exact)
+      // -- dequantise and store the tile
+      if (fetch) {
 #pragma unroll
-      for (int u = 0; u < kMaxLoads; ++u) {
-        const int it = warp + 8 * u;
-        if (it < n_items) {
-          const int r = 8 * (it & 15) + (lane & 7), c = 4 * (it >> 4) + (lane >> 3);
-          uint8_t* dst = tile + (r >> 3) * sbo_rows + (r & 7) * 16;
-          if (c < nc8) {
-            const uint32_t wv[4] = {buf[u].x, buf[u].y, buf[u].z, buf[u].w};
-            uint32_t pk[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t b2 = (wv[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
-              const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
-              const float2 f = __half22float2(__half2(h2));
-              pk[e] = (uint32_t)bf16_rn(f.x) | ((uint32_t)bf16_rn(f.y) << 16);
-            }
-            *reinterpret_cast<uint4*>(dst + (2 * c) * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(dst + (2 * c + 1) * 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          } else if (c < nc) {
-            *reinterpret_cast<uint4*>(dst + (dmain / 8 + c - nc8) * 128) = buf[u];
-          }
+        for (int u = 0; u < kMaxLoads; ++u) {
+          const int it = warp + 8 * u;
+          if (it < n_items) gather_store(it, buf[u]);
         }
       }
       tc::fence_proxy_async_smem();

@@ -125,6 +125,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
   const uint32_t tile_bytes = (uint32_t)L.idx_tile_bytes;
   const uint32_t sf_off = (uint32_t)(kCsaPerPage * CHs * 16);
 
+  // ---- set-up (overlaps the bookkeeping's global loads below)
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.stage_empty[s], 1); }
+    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], kGroupThreads); }
+    tc::mbar_init(&sm.q_ready, 1);
+    tc::mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    tc::fence_mbar_init();
+  }
+
   // ---- per-query bookkeeping (one thread per query); every CTA computes
   //      the same tile total
   int64_t total = 0;
@@ -144,29 +158,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
     }
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if (lane == 0) sm.red[warp] = part;
-    __syncthreads();
+    tc::tc_fence_before();
+    __syncthreads();                       // also publishes the TMEM address and the barriers
+    tc::tc_fence_after();
     for (int w = 0; w < kThreads / 32; ++w) total += sm.red[w];
   }
-  const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
-  if (g0 >= g1) return;
-
-  // ---- set-up
-  if (warp == 1) {
-    tc::tmem_alloc(&sm.tmem_base, kTmemCols);
-    tc::tmem_relinquish();
-  }
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) { tc::mbar_init(&sm.full[s], 1); tc::mbar_init(&sm.stage_empty[s], 1); }
-    for (int k = 0; k < kNA; ++k) { tc::mbar_init(&sm.acc_full[k], 1); tc::mbar_init(&sm.acc_empty[k], kGroupThreads); }
-    tc::mbar_init(&sm.q_ready, 1);
-    tc::mbar_init(&sm.drain, 1);
-    sm.abort = 0;
-    tc::fence_mbar_init();
-  }
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (g0 >= g1) {                          // no tiles for this CTA: nothing was issued
+    if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+    return;
+  }
 
   // role state (each role only uses its own)
   uint32_t u_base = 0;       // CTA-wide tile counter at the start of the pass (barrier phases)
