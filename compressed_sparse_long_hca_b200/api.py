@@ -198,12 +198,13 @@ def topk(scores: torch.Tensor, n_valid: torch.Tensor, k: int, out: torch.Tensor,
 def decode_step_fields(n: int, H: int, D: int, H_I: int, d_I: int, csa: bool, align: int = 256):
     """Packed layout of one decode step's inputs: a list of (name, dtype,
     shape, byte offset, bytes) with every field starting on an `align`-byte
-    boundary, and the buffer's total size."""
-    fields = [("q", torch.bfloat16, (n, H, D)), ("c", torch.float32, (n, 1, D)),
-              ("z", torch.float32, (n, 1, D))]
+    boundary, and the buffer's total size.  The attention query q comes last,
+    so that everything before it is one contiguous copy."""
+    fields = [("c", torch.float32, (n, 1, D)), ("z", torch.float32, (n, 1, D))]
     if csa:
         fields += [("ci", torch.float32, (n, 1, d_I)), ("zi", torch.float32, (n, 1, d_I)),
                    ("q_idx", torch.float32, (n, H_I, d_I)), ("w", torch.float32, (n, H_I))]
+    fields.append(("q", torch.bfloat16, (n, H, D)))
     out, off = [], 0
     for name, dtype, shape in fields:
         nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
@@ -214,22 +215,26 @@ def decode_step_fields(n: int, H: int, D: int, H_I: int, d_I: int, csa: bool, al
 
 class DecodeStep:
     """One decode step of a fixed batch of requests on one layer, captured
-    once as a CUDA graph and replayed every step.
+    once as two CUDA graphs and replayed every step.
 
     The step appends each request's new token (csa_compress_append), then on
-    a CSA layer scores the index keys (csa_index_scores), selects the top k
-    (csa_topk) and attends (csa_hca_decode_attn); on an HCA layer it attends
-    over every compressed entry.  The step's inputs travel from one pinned
-    host buffer in one host-to-device copy, its output returns in one
-    device-to-host copy, all on one stream.
+    a CSA layer scores the index keys (csa_index_scores) and selects the top
+    k (csa_topk) -- the first graph -- and attends (csa_hca_decode_attn) --
+    the second graph; on an HCA layer the first graph only appends and the
+    attention covers every compressed entry.
 
     Inputs of a step, packed in a buffer from `new_host_inputs()` and filled
-    through `views(buf)`: q [n, H, D] bf16, c and z [n, 1, D] fp32 (the
-    token's KV candidate and gate logits), on a CSA layer also ci and zi
-    [n, 1, d_I] fp32, q_idx [n, H_I, d_I] fp32 and w [n, H_I] fp32.  Each
+    through `views(buf)`: c and z [n, 1, D] fp32 (the token's KV candidate
+    and gate logits), on a CSA layer also ci and zi [n, 1, d_I] fp32, q_idx
+    [n, H_I, d_I] fp32 and w [n, H_I] fp32, and last q [n, H, D] bf16.  Each
     field starts on a 256-byte boundary.
 
-    The graph holds device pointers, so the batch (req_ids), k and the sink
+    Host transfers: the fields before q travel in one copy on the caller's
+    stream ahead of the first graph; q, which only the attention reads,
+    travels in one copy on a side stream while the first graph runs, and the
+    second graph waits for it; the output returns in one copy.
+
+    The graphs hold device pointers, so the batch (req_ids), k and the sink
     logits are fixed at construction.  On a CSA layer construction runs the
     index and top-k kernels once (they change nothing in the cache) so that
     their one-time launch set-up happens before the capture."""
@@ -247,7 +252,8 @@ class DecodeStep:
         H, D = cache.H, cache.D
         self._fields, off = decode_step_fields(n, H, D, cache.H_I, cache.d_I, self.csa)
         self.input_bytes = off
-        dev = torch.device(device)
+        self._q_off = next(f[3] for f in self._fields if f[0] == "q")
+        dev = self.device = torch.device(device)
         self._dev_in = torch.zeros(off, dtype=torch.uint8, device=dev)
         d = self.views(self._dev_in)
         self._req = torch.tensor(ids, dtype=torch.int32, device=dev)
@@ -257,6 +263,8 @@ class DecodeStep:
         self.host_out = torch.empty((n, H, D), dtype=torch.bfloat16).pin_memory()
         self._ws = torch.empty(max(cache.attn_workspace_bytes(layer, n, self.k if self.csa else 0), 16),
                                dtype=torch.uint8, device=dev)
+        self._side = torch.cuda.Stream(device=dev)
+        self._ev_start, self._ev_q = torch.cuda.Event(), torch.cuda.Event()
         if self.csa:
             n_max = max(cache.cfg.max_pages_per_request * 128, 128)   # 512 tokens = 128 entries per page
             self._scores = torch.empty((n, n_max), dtype=torch.float32, device=dev)
@@ -274,11 +282,13 @@ class DecodeStep:
             select()
             torch.cuda.synchronize(dev)
             cache.check_device_error()
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph):
+        self.graph_select = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_select):
             cache.compress_append(layer, self._req, d["c"], d["z"], d.get("ci"), d.get("zi"))
             if self.csa:
                 select()
+        self.graph_attn = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_attn):
             cache.decode_attn(layer, self._req, d["q"], self._idx if self.csa else None, self._sink, self.out,
                               variant=variant, workspace=self._ws)
         torch.cuda.synchronize(dev)
@@ -298,18 +308,30 @@ class DecodeStep:
         """Enqueue one step on the current stream: copy the packed inputs in,
         replay the step, copy the output [n, H, D] bf16 to `host_out` (pinned),
         which is returned and is valid once the stream has reached this point.
-        `marks`, two torch.cuda.Events, are recorded after the input copy and
-        after the replay (to time the three phases)."""
+        `marks`, two torch.cuda.Events, are recorded on the current stream
+        after the first input copy and after the second graph (to time the
+        three phases; the query's copy overlaps the first graph)."""
         if host_inputs.device.type != "cpu" or not host_inputs.is_pinned():
             raise ValueError("host_inputs must be a pinned host buffer (new_host_inputs())")
         if host_inputs.dtype != torch.uint8 or host_inputs.numel() != self.input_bytes:
             raise ValueError(f"host_inputs must be {self.input_bytes} bytes")
-        self._dev_in.copy_(host_inputs, non_blocking=True)
+        main = torch.cuda.current_stream(self.device)
+        qo = self._q_off
+        # the query's copy starts once everything queued before this step
+        # (the previous step's attention reads the same buffer) has run
+        self._ev_start.record(main)
+        self._side.wait_event(self._ev_start)
+        with torch.cuda.stream(self._side):
+            self._dev_in[qo:].copy_(host_inputs[qo:], non_blocking=True)
+            self._ev_q.record(self._side)
+        self._dev_in[:qo].copy_(host_inputs[:qo], non_blocking=True)
         if marks is not None:
-            marks[0].record()
-        self.graph.replay()
+            marks[0].record(main)
+        self.graph_select.replay()
+        main.wait_event(self._ev_q)
+        self.graph_attn.replay()
         if marks is not None:
-            marks[1].record()
+            marks[1].record(main)
         self.host_out.copy_(self.out, non_blocking=True)
         return self.host_out
 

@@ -63,14 +63,15 @@ def test_init_rejects_bad_arguments_without_launching(cuda_lib):
 
 
 def test_decode_step_packed_input_layout():
-    """DecodeStep's packed host buffer: the fields in order, each on a
-    256-byte boundary, sized by shape and dtype, none overlapping."""
+    """DecodeStep's packed host buffer: the fields in order (the attention
+    query last, copied on its own), each on a 256-byte boundary, sized by
+    shape and dtype, none overlapping."""
     import math
 
     import torch
 
     from compressed_sparse_long_hca_b200.api import decode_step_fields
-    for csa, names in ((True, ["q", "c", "z", "ci", "zi", "q_idx", "w"]), (False, ["q", "c", "z"])):
+    for csa, names in ((True, ["c", "z", "ci", "zi", "q_idx", "w", "q"]), (False, ["c", "z", "q"])):
         fields, total = decode_step_fields(4, 128, 512, 64, 128, csa)
         assert [f[0] for f in fields] == names
         end = 0
