@@ -325,7 +325,8 @@ def run_gpu(args):
     launches0 = lib.csa_launch_count()
     g_plain, _ = capture(())
     kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graph
-    g_idx, ev_idx = capture(("index",) if csa else ())
+    roof_part = "index" if csa else "attention"       # the kernel the roofline is reported for
+    g_idx, ev_idx = capture((roof_part,))
     g_all, ev_all = capture(tuple(nm for nm, _ in parts))
     torch.cuda.synchronize()
     if ws > 1:
@@ -354,9 +355,8 @@ def run_gpu(args):
     launches = kernels_per_step * steps               # libcsa kernels run in the timed region
     idx_sum = [0.0]
     names = [nm for nm, _ in parts]
-    if csa:
-        x = names.index("index")
-        timed_pass(g_idx, warm + steps, lambda: idx_sum.__setitem__(0, idx_sum[0] + ev_idx[x].elapsed_time(ev_idx[x + 1])))
+    x = names.index(roof_part)
+    timed_pass(g_idx, warm + steps, lambda: idx_sum.__setitem__(0, idx_sum[0] + ev_idx[x].elapsed_time(ev_idx[x + 1])))
     part_ms = {nm: 0.0 for nm in names}
 
     def add_parts():
@@ -364,7 +364,7 @@ def run_gpu(args):
             part_ms[nm] += ev_all[x].elapsed_time(ev_all[x + 1])
 
     timed_pass(g_all, warm + 2 * steps, add_parts)
-    idx_ms = idx_sum[0] / steps if csa else None
+    idx_ms = idx_sum[0] / steps
     breakdown = {nm: round(v / steps * 1e3, 2) for nm, v in part_ms.items()}
     del g_plain, g_idx, g_all
     # ---- end to end through the public API with host buffers: DecodeStep
@@ -410,10 +410,10 @@ def run_gpu(args):
     del e2e
     cache.check_device_error()
     # ---- max over ranks
-    step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms or 0.0], ws, "cuda")
+    step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms], ws, "cuda")
     value = whole_job_rate(ws, B, steps, step_ms)
     e2e_value = whole_job_rate(ws, B, steps, e2e_ms)
-    peak, peak_kind, _ = _peaks()
+    peak, peak_kind, peaks = _peaks()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
         "ms_per_step": step_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -433,6 +433,18 @@ def run_gpu(args):
                             "unit": "GB/s", "frac": ach / peak, "traffic": _profiled_traffic(),
                             "peak_source": peak_kind, "ms_per_launch": idx_ms,
                             "algorithmic_bytes_per_launch": alg}
+    else:
+        # HCA: the attention over every compressed entry is the dominant
+        # kernel; QK^T and PV are 2 * H * rows * D flops each per query
+        rows = (T0 + warm + steps + steps // 2) // 128 + wl.W     # mid-way through the pass that timed it
+        flops = B * 4.0 * wl.H * rows * wl.D
+        ach = flops / (idx_ms / 1e3) / 1e12
+        tpeak = peaks.get("bf16_tflops", 1590.0)
+        line["roofline"] = {"bound": "tensor", "kernel": "csa_hca_decode_attn", "achieved": ach, "peak": tpeak,
+                            "unit": "TFLOP/s", "frac": ach / tpeak, "traffic": None,
+                            "peak_source": "measured bf16 burst" if "bf16_tflops" in peaks else "fallback",
+                            "ms_per_launch": idx_ms, "algorithmic_flops_per_launch": flops,
+                            "rows_per_query": rows}
     if rank == 0 and args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if rank == 0:

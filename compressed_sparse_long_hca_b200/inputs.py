@@ -64,7 +64,12 @@ C5_CSA = Workload("sweep-csa", "csa", H=128, D=512, R=64, H_I=64, d_I=128, k=102
                   W=128, context=0, batch=0, seed=1005, hidden=7168)
 C5_HCA = Workload("sweep-hca", "hca", H=128, D=512, R=64, H_I=0, d_I=0, k=0,
                   W=128, context=0, batch=0, seed=1005, hidden=7168)
-WORKLOADS = {w.name: w for w in (C1, C2, C3, C4)}
+# The sweep's HCA layer at its longest context (1M tokens: 8192 compressed
+# entries + the window per query), batch 4: the attention over every entry is
+# the one contraction-heavy case of the path (about 430 flops per byte).
+C5_HCA_1M = Workload("hca-pro-1m", "hca", H=128, D=512, R=64, H_I=0, d_I=0, k=0, W=128,
+                     context=1048576, batch=4, seed=1006, hidden=7168)
+WORKLOADS = {w.name: w for w in (C1, C2, C3, C4, C5_HCA_1M)}
 
 
 def _rng(*key) -> np.random.Generator:

@@ -37,12 +37,18 @@ def _fill(cache, layer, reqs, lengths, seed, D, dI):
     """Append tokens 0 .. lengths[r]-1 of every request (chunks of 4096;
     requests that are already full drop out of later calls)."""
     t = 0
+    chunk, gen = -1, {}
     while True:
         live = [r for r in reqs if lengths[r] > t]
         if not live:
             break
         n_tok = min(min(lengths[r] for r in live) - t, I.CHUNK - t % I.CHUNK)
-        parts = [I.device_token_inputs(seed, layer, r, t // I.CHUNK, D, dI) for r in live]
+        if t // I.CHUNK != chunk:          # each request's chunk is generated once
+            chunk, gen = t // I.CHUNK, {}
+        for r in live:
+            if r not in gen:
+                gen[r] = I.device_token_inputs(seed, layer, r, chunk, D, dI)
+        parts = [gen[r] for r in live]
         lo = t % I.CHUNK
         st = lambda k: (torch.stack([p[k][lo:lo + n_tok] for p in parts]).contiguous()
                         if parts[0][k] is not None else None)
@@ -155,12 +161,12 @@ def test_full_size_decode_step(name):
 
 def test_ragged_sweep_batch_invariance():
     """Pro-like CSA (top-1024) and HCA layers, 16 requests with contexts
-    log-uniform in [4K, 256K], three decode steps; each step runs the whole
+    log-uniform in [4K, 1M], three decode steps; each step runs the whole
     batch and sampled sub-batches (sizes 1 .. 16, shuffled positions, both
     variants): every request's bits agree across all of them."""
     wl_c, wl_h = I.C5_CSA, I.C5_HCA
     n_req = 16
-    ctx = I.sweep_contexts(wl_c.seed, n_req, lo=4096, hi=1 << 18)
+    ctx = I.sweep_contexts(wl_c.seed, n_req, lo=4096, hi=1 << 20)
     cap = int(ctx.max()) + 512
     pair = Hp.Pair(wl_c, 1, 1, max_req=n_req, capacity=cap)
     cache = pair.cache
@@ -198,3 +204,49 @@ def test_ragged_sweep_batch_invariance():
                         assert np.array_equal(again[r]["idx"], base[r]["idx"])
         for r in allr:
             lens[r] += 1
+
+
+def test_batch_larger_than_the_indexer_query_table():
+    """300 requests in one batch (the indexer keeps per-query tile counts in
+    shared memory for the first 256 and recomputes them beyond), Pro-like CSA
+    and HCA layers, contexts log-uniform in [600, 20K]: the whole batch, its
+    reverse and sub-batches agree bit for bit per request, and three requests
+    (shortest, median, longest) match the oracle."""
+    wl_c, wl_h = I.C5_CSA, I.C5_HCA
+    n_req = 300
+    ctx = I.sweep_contexts(wl_c.seed + 300, n_req, lo=600, hi=20000)
+    cap = int(ctx.max()) + 64
+    pair = Hp.Pair(wl_c, 1, 1, max_req=n_req, capacity=cap)
+    cache = pair.cache
+    for r in range(n_req):
+        cache.request_alloc(r, int(ctx[r]) + 64)
+    lens = {r: int(ctx[r]) for r in range(n_req)}
+    _fill(cache, 0, list(range(n_req)), lens, wl_c.seed + 300, wl_c.D, wl_c.d_I)
+    _fill(cache, 1, list(range(n_req)), lens, wl_c.seed + 301, wl_c.D, 0)
+    allr = list(range(n_req))
+    order_ctx = [int(x) for x in np.argsort(ctx, kind="stable")]
+    probes = [order_ctx[0], order_ctx[n_req // 2], order_ctx[-1]]
+    rng = np.random.default_rng(300)
+    for layer, wl in ((0, wl_c), (1, wl_h)):
+        csa = layer == 0
+        c, z = _host(1300 + layer, n_req, 1, wl.D), _host(1350 + layer, n_req, 1, wl.D)
+        ci = _host(1390, n_req, 1, wl.d_I) if csa else None
+        zi = _host(1395, n_req, 1, wl.d_I) if csa else None
+        dev = lambda a: torch.from_numpy(a).cuda() if a is not None else None
+        cache.compress_append(layer, torch.arange(n_req, dtype=torch.int32, device="cuda"), dev(c), dev(z),
+                              dev(ci), dev(zi))
+        q = I.bf16_grid(_host(1400 + layer, n_req, wl.H, wl.D))
+        qi = _host(1450, n_req, wl.H_I, wl.d_I) if csa else None
+        w = _host(1460, n_req, wl.H_I) if csa else None
+        sink = pair.params[layer]["sink"]
+        base = _step(cache, wl, layer, allr, q, qi, w, sink)
+        for r in probes:
+            _oracle_check(cache, wl, layer, r, lens[r] + 1, q, qi, w, sink, base[r])
+        subs = [allr[::-1], [int(x) for x in rng.choice(n_req, size=40, replace=False)], probes]
+        for sub, variant in zip(subs, ("high", "low", "auto")):
+            again = _step(cache, wl, layer, sub, q, qi, w, sink, variant)
+            for r in sub:
+                assert np.array_equal(again[r]["out"], base[r]["out"]), f"layer {layer} req {r} ({variant})"
+                if csa:
+                    assert np.array_equal(again[r]["idx"], base[r]["idx"]), f"layer {layer} req {r}"
+                    assert np.array_equal(again[r]["scores"].view(np.uint32), base[r]["scores"].view(np.uint32))
