@@ -153,6 +153,14 @@ def test_index_scores_on_oracle_written_keys(HI, dI):
             first = got.copy()
         else:
             assert np.array_equal(np.nan_to_num(first, nan=7.0), np.nan_to_num(got, nan=7.0))
+    # the same queries in smaller batches and other positions: the same bits
+    for sub in ([5, 3, 0], [4, 5, 1, 2], [5], [3, 4, 5, 0]):
+        scores = torch.full((len(sub), ld), float("nan"), device="cuda")
+        nv = torch.zeros(len(sub), dtype=torch.int32, device="cuda")
+        pair.cache.index_scores(0, _t(np.array(sub, np.int32)), _t(qi[sub]), _t(w[sub]), scores, nv)
+        pair.cache.check_device_error()
+        got = scores.double().cpu().numpy()
+        assert np.array_equal(np.nan_to_num(first[sub], nan=7.0), np.nan_to_num(got, nan=7.0)), f"batch {sub}"
 
 
 # ---------------------------------------------------------------- stage: top-k
