@@ -58,7 +58,7 @@ namespace {
 constexpr int kAttThreads = 256;
 constexpr int kTileRows = 128;
 constexpr int kMaxLoads = 18;      // 16-byte loads per thread per tile (D <= 512)
-constexpr int kFoldBatch = 8;      // partials loaded at once by the fold kernel
+constexpr int kFoldBatch = 9;      // partials loaded at once by the fold kernel (a top-1024 query's 9 tiles)
 
 struct AttnArgs {
   Layout L;
