@@ -85,3 +85,34 @@ def test_decode_step_packed_input_layout():
     assert f["q"][4] == 4 * 128 * 512 * 2 and f["q"][1] == torch.bfloat16
     assert f["q_idx"][2] == (4, 64, 128) and f["w"][2] == (4, 64)
     assert f["c"][2] == (4, 1, 512) and f["ci"][2] == (4, 1, 128)
+
+
+def test_topk_argument_errors_are_returned_before_any_launch(cuda_lib):
+    """csa_topk needs no cache: every argument error comes back as
+    CSA_ERR_ARG from the host checks (the pointer below is never touched)."""
+    P = 0x10000
+    cases = [
+        ((P, 10, P, -1, 4, P, 0, None), b"n must be"),
+        ((P, 10, P, 70000, 4, P, 0, None), b"n must be"),
+        ((None, 10, P, 1, 4, P, 0, None), b"NULL"),
+        ((P, 10, None, 1, 4, P, 0, None), b"NULL"),
+        ((P, 10, P, 1, 4, None, 0, None), b"NULL"),
+        ((P, 10, P, 1, 0, P, 0, None), b"k and ld"),
+        ((P, 0, P, 1, 4, P, 0, None), b"k and ld"),
+        ((P, 10, P, 1, 4, P, 3, None), b"variant"),
+    ]
+    for args, msg in cases:
+        assert cuda_lib.csa_topk(*args) == -1, args
+        assert msg in cuda_lib.csa_last_error(), (args, cuda_lib.csa_last_error())
+    assert cuda_lib.csa_topk(P, 10, P, 0, 4, P, 0, None) == 0        # an empty batch is a no-op
+
+
+def test_cache_calls_on_a_null_handle_fail_on_the_host(cuda_lib):
+    P = 0x10000
+    assert cuda_lib.csa_index_scores(None, 0, 1, P, P, P, P, 8, P, 0, None) == -1
+    assert cuda_lib.csa_hca_decode_attn(None, 0, 1, P, P, P, 4, P, 1.0, P, P, 1 << 20, 0, None) == -1
+    assert cuda_lib.csa_hca_decode_attn_noalloc(None, 0, 1, P, P, P, 4, P, 1.0, P, None) == -1
+    assert cuda_lib.csa_attn_workspace_bytes(None, 0, 1, 4) == 0
+    assert cuda_lib.csa_request_alloc(None, 0, 16) == -1
+    assert cuda_lib.csa_request_free(None, 0) == -1
+    assert cuda_lib.csa_check_device_error(None, None) == -1
