@@ -307,7 +307,9 @@ class DecodeStep:
     def __call__(self, host_inputs: torch.Tensor, marks=None) -> torch.Tensor:
         """Enqueue one step on the current stream: copy the packed inputs in,
         replay the step, copy the output [n, H, D] bf16 to `host_out` (pinned),
-        which is returned and is valid once the stream has reached this point.
+        which is returned and is valid once the stream has reached this point
+        (the next call overwrites it).  The copies are asynchronous:
+        `host_inputs` must not change until the stream has passed them.
         `marks`, two torch.cuda.Events, are recorded on the current stream
         after the first input copy and after the second graph (to time the
         three phases; the query's copy overlaps the first graph)."""
