@@ -431,8 +431,12 @@ def run_gpu(args):
                 "phases_us": e2e_phases},
         "clocks": clk,
     }
+    # tokens per request half-way through the pass that timed the roofline
+    # kernel: eager warm-up steps, one untimed replay of each of the three
+    # graphs, the plain pass, then half of the timed pass
+    t_mid = T0 + warm + 3 + steps + steps // 2
     if csa:
-        n_c = T0 // 4 + (warm + steps // 2) // 4
+        n_c = t_mid // 4
         alg = B * (n_c * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
         ach = alg / (idx_ms / 1e3) / 1e9
         line["roofline"] = {"bound": "hbm", "kernel": "csa_index_scores", "achieved": ach, "peak": peak,
@@ -442,7 +446,7 @@ def run_gpu(args):
     else:
         # HCA: the attention over every compressed entry is the dominant
         # kernel; QK^T and PV are 2 * H * rows * D flops each per query
-        rows = (T0 + warm + steps + steps // 2) // 128 + wl.W     # mid-way through the pass that timed it
+        rows = t_mid // 128 + wl.W
         flops = B * 4.0 * wl.H * rows * wl.D
         ach = flops / (idx_ms / 1e3) / 1e12
         tpeak = peaks.get("bf16_tflops", 1590.0)
