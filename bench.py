@@ -128,7 +128,8 @@ class Clocks:
         self.proc = None
         self.thread = None
         self.samples = []
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"csa_bench_clocks_{os.getpid()}_{gpu_index}.csv")
 
     def _nvml_loop(self, handle, nv):
         while not self.stop_flag:
@@ -155,7 +156,6 @@ class Clocks:
         except Exception:
             self.thread = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.uuid or self.gpu_index), f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -455,6 +455,16 @@ def run_gpu(args):
                             "peak_source": "measured bf16 burst" if "bf16_tflops" in peaks else "fallback",
                             "ms_per_launch": idx_ms, "algorithmic_flops_per_launch": flops,
                             "rows_per_query": rows}
+    # the whole step against HBM: the algorithmic bytes of every part (index
+    # keys scanned, selected and window rows gathered, q in and out) over the
+    # step time, against the measured copy peak and the nominal 8 TB/s
+    rows_q = (wl.k if csa else t_mid // 128) + wl.W
+    step_bytes = B * ((t_mid // 4 * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4 if csa else 0)
+                      + rows_q * ROW_BYTES + 2 * wl.H * wl.D * 2)
+    step_gbs = step_bytes / (step_ms / steps / 1e3) / 1e9
+    line["step_roofline"] = {"bound": "hbm", "achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                             "frac": step_gbs / peak, "frac_of_8tbs": step_gbs / 8000.0,
+                             "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_kind}
     if rank == 0 and args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if rank == 0:

@@ -16,6 +16,7 @@ STATUS_NAMES = {0: "CSA_OK", -1: "CSA_ERR_ARG", -2: "CSA_ERR_CAPACITY", -3: "CSA
                 -4: "CSA_ERR_DEVICE_TIMEOUT", -5: "CSA_ERR_DEVICE_BOUNDS"}
 VARIANT_AUTO, VARIANT_HIGH_OCC, VARIANT_LOW_OCC = 0, 1, 2
 REGION_KV, REGION_INDEX, REGION_WINDOW = 0, 1, 2
+FMT_MIXED, FMT_F32 = 0, 1
 
 
 class CsaCfg(ctypes.Structure):
@@ -23,7 +24,7 @@ class CsaCfg(ctypes.Structure):
                 ("H", ctypes.c_int32), ("D", ctypes.c_int32), ("D_rope", ctypes.c_int32),
                 ("H_I", ctypes.c_int32), ("d_I", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("max_requests", ctypes.c_int32), ("max_pages_per_request", ctypes.c_int32),
-                ("pool_pages", ctypes.c_int32), ("rope_base", ctypes.c_float)]
+                ("pool_pages", ctypes.c_int32), ("rope_base", ctypes.c_float), ("fmt", ctypes.c_int32)]
 
 
 # exported symbol -> (restype, argtypes)
@@ -47,6 +48,7 @@ SIGNATURES = {
     "csa_debug_rows": (_I32, [_P, _I32, _I32, _I32, _I64, _I64, _P, _I32]),
     "csa_debug_set_length": (_I32, [_P, _I32, _I32, _I64]),
     "csa_debug_get_length": (_I64, [_P, _I32, _I32]),
+    "csa_debug_wait_timeout": (_I32, [_P, _I32, _P]),
 }
 
 _lib = None

@@ -123,13 +123,18 @@ __device__ void csa_entries_body(const AppendArgs& a, int i, int req, int64_t L0
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
       rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], L.theta()[p], kCsaM * j);
     __syncthreads();
-    const int s = (int)(j % kCsaPerPage);
-    char* pp = L.page(L.page_table(req)[j / kCsaPerPage], a.layer);
-    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(pp) + (int64_t)s * (D - R),
-                 reinterpret_cast<uint16_t*>(pp + L.pg_csa_bf16) + (int64_t)s * R,
-                 reinterpret_cast<float*>(pp + L.pg_csa_scale) + s, red);
-    store_index_key(L, key, s, reinterpret_cast<uint8_t*>(pp + L.pg_idx_codes),
-                    reinterpret_cast<uint8_t*>(pp + L.pg_idx_sf));
+    if (L.fmt == kFmtF32) {
+      store_f32_row(row, D, L.entry_row_f32(req, a.layer, j));
+      store_f32_row(key, dI, L.index_key_f32(req, a.layer, j));
+    } else {
+      const int s = (int)(j % kCsaPerPage);
+      char* pp = L.page(L.page_table(req)[j / kCsaPerPage], a.layer);
+      store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(pp) + (int64_t)s * (D - R),
+                   reinterpret_cast<uint16_t*>(pp + L.pg_csa_bf16) + (int64_t)s * R,
+                   reinterpret_cast<float*>(pp + L.pg_csa_scale) + s, red);
+      store_index_key(L, key, s, reinterpret_cast<uint8_t*>(pp + L.pg_idx_codes),
+                      reinterpret_cast<uint8_t*>(pp + L.pg_idx_sf));
+    }
     __syncthreads();
   }
 }
@@ -166,11 +171,15 @@ __device__ void hca_entries_body(const AppendArgs& a, int i, int req, int64_t L0
     for (int p = threadIdx.x; p < R / 2; p += blockDim.x)
       rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], L.theta()[p], kHcaM * j);
     __syncthreads();
-    const int s = (int)(j % kHcaPerPage);
-    char* pp = L.page(L.page_table(req)[j / kHcaPerPage], a.layer);
-    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(pp) + (int64_t)s * (D - R),
-                 reinterpret_cast<uint16_t*>(pp + L.pg_hca_bf16) + (int64_t)s * R,
-                 reinterpret_cast<float*>(pp + L.pg_hca_scale) + s, red);
+    if (L.fmt == kFmtF32) {
+      store_f32_row(row, D, L.entry_row_f32(req, a.layer, j));
+    } else {
+      const int s = (int)(j % kHcaPerPage);
+      char* pp = L.page(L.page_table(req)[j / kHcaPerPage], a.layer);
+      store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(pp) + (int64_t)s * (D - R),
+                   reinterpret_cast<uint16_t*>(pp + L.pg_hca_bf16) + (int64_t)s * R,
+                   reinterpret_cast<float*>(pp + L.pg_hca_scale) + s, red);
+    }
     __syncthreads();
   }
 }
@@ -214,9 +223,12 @@ __device__ void tokens_body(const AppendArgs& a, int i, int y0, int ystride, flo
       rope_pair(row[D - R + 2 * p], row[D - R + 2 * p + 1], L.theta()[p], pos);
     __syncthreads();
     const int slot = (int)(pos % kWindow);
-    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),
-                 reinterpret_cast<uint16_t*>(st + L.ring_bf16) + (int64_t)slot * R,
-                 reinterpret_cast<float*>(st + L.ring_scale) + slot, red);
+    if (L.fmt == kFmtF32)
+      store_f32_row(row, D, L.ring_row_f32(req, a.layer, slot));
+    else
+      store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),
+                   reinterpret_cast<uint16_t*>(st + L.ring_bf16) + (int64_t)slot * R,
+                   reinterpret_cast<float*>(st + L.ring_scale) + slot, red);
     __syncthreads();
   }
   // tail slots
@@ -289,9 +301,12 @@ __device__ bool token1_body(const AppendArgs& a, int i, float* sm, int& req, int
   __syncthreads();
   char* st = L.state(req, a.layer);
   const int slot = (int)(pos % kWindow);
-  store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),
-               reinterpret_cast<uint16_t*>(st + L.ring_bf16) + (int64_t)slot * R,
-               reinterpret_cast<float*>(st + L.ring_scale) + slot, red);
+  if (L.fmt == kFmtF32)
+    store_f32_row(row, D, L.ring_row_f32(req, a.layer, slot));
+  else
+    store_kv_row(row, D, R, reinterpret_cast<uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (D - R),
+                 reinterpret_cast<uint16_t*>(st + L.ring_bf16) + (int64_t)slot * R,
+                 reinterpret_cast<float*>(st + L.ring_scale) + slot, red);
   // tail slot (an HCA block completed by this token needs no tail)
   if (csa || (pos + 1) % kHcaM != 0) {
     float* tail = reinterpret_cast<float*>(L.tail(req, a.layer));

@@ -1,0 +1,98 @@
+// Pieces of the decode attention shared by the tensor-core kernel (the
+// mixed FP8 / BF16 storage format) and the CUDA-core kernel (the fp32
+// storage format): arguments, the rows of a query, and the fold of per-tile
+// partials.
+//
+// Page "V4终于终于终于终于是来了", sections "CSA——压缩稀疏注意力" and
+// "HCA——重度压缩注意力": a query attends to its selected (CSA) or all (HCA)
+// compressed entries, then the 128 latest raw tokens; each head's sink logit
+// enters the softmax denominator.  The rows are cut into tiles of 128; each
+// tile gives (m_t, l_t, O_t) and the tiles are folded in order, the sink
+// last.  Both storage formats and both launch variants use the fold below,
+// so that the order and the rounding of the reduction depend on the query
+// alone.
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+constexpr int kTileRows = 128;
+constexpr int kFoldBatch = 9;      // partials loaded at once by the fold kernel (a top-1024 query's 9 tiles)
+
+struct AttnArgs {
+  Layout L;
+  int layer;
+  int n;
+  const int32_t* req_ids;
+  const void* q;       // BF16 (mixed format) or fp32 (fp32 format) [n][H][D]
+  const int32_t* topk;
+  int k;
+  const float* sink;
+  float scale;
+  void* out;           // BF16 or fp32 [n][H][D], as q
+  int G;              // heads per CTA (MMA N), 16 or 32
+  // split launch only: partials of (query i, tile t, head h)
+  float* ws_o;        // [n][tiles_max][H][D]
+  float2* ws_ml;      // [n][tiles_max][H]   (m_t, l_t); m_t = -inf: empty tile
+  int tiles_max;
+  int f32;            // fp32 storage format: fp32 q and out
+};
+
+struct QueryGeom {
+  int req;
+  bool csa;
+  int64_t t;          // query position
+  int64_t n_entries, w0, n_win, n_list, total;
+  int n_tiles;
+};
+
+__device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& g, bool report) {
+  const Layout& L = a.L;
+  g.req = a.req_ids[i];
+  if (g.req < 0 || g.req >= L.max_req) {
+    if (report) set_err(L, kErrBounds, i);
+    return false;
+  }
+  g.csa = a.layer < L.n_csa;
+  const int64_t T = L.lengths()[(int64_t)a.layer * L.max_req + g.req];
+  if (T <= 0) {
+    if (report) set_err(L, kErrBounds, 1000000 + i);
+    return false;
+  }
+  g.t = T - 1;
+  g.n_entries = g.csa ? T / kCsaM : T / kHcaM;
+  g.w0 = g.t - (kWindow - 1) > 0 ? g.t - (kWindow - 1) : 0;
+  g.n_win = g.t - g.w0 + 1;
+  g.n_list = g.csa ? a.k : g.n_entries;
+  g.total = g.n_list + g.n_win;
+  g.n_tiles = (int)((g.total + kTileRows - 1) / kTileRows);
+  return true;
+}
+
+// The fold of one partial into a running (m, l, O); shared by both launch
+// variants so that they round identically.
+__device__ __forceinline__ void fold_coef(float m, float mt, float& mn, float& al, float& be) {
+  mn = fmaxf(m, mt);
+  al = (m == -INFINITY) ? 0.f : expf(m - mn);
+  be = expf(mt - mn);
+}
+__device__ __forceinline__ float fold_val(float o, float al, float ot, float be) {
+  const float b = __fmul_rn(ot, be);
+  return al == 0.f ? b : __fmaf_rn(o, al, b);
+}
+__device__ __forceinline__ void finish_coef(float m, float sk, float l, float& cm, float& den) {
+  const float mu = fmaxf(m, sk);
+  cm = expf(m - mu);
+  den = __fmaf_rn(l, cm, expf(sk - mu));
+}
+__device__ __forceinline__ float finish_f32(float o, float cm, float den) {
+  return __fdiv_rn(__fmul_rn(o, cm), den);
+}
+__device__ __forceinline__ uint16_t finish_val(float o, float cm, float den) {
+  return bf16_rn(finish_f32(o, cm, den));
+}
+
+int attn_tiles_max(const Layout& L, int layer, int k);
+cudaError_t launch_attn_fold(const AttnArgs& a, cudaStream_t st);
+
+}  // namespace csa

@@ -48,6 +48,7 @@
 //     (P * row scale)^T, the RoPE dims P^T, each into its own accumulator.
 #include <mutex>
 
+#include "attn_common.cuh"
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -56,78 +57,7 @@ namespace csa {
 namespace {
 
 constexpr int kAttThreads = 256;
-constexpr int kTileRows = 128;
 constexpr int kMaxLoads = 18;      // 16-byte loads per thread per tile (D <= 512)
-constexpr int kFoldBatch = 9;      // partials loaded at once by the fold kernel (a top-1024 query's 9 tiles)
-
-struct AttnArgs {
-  Layout L;
-  int layer;
-  int n;
-  const int32_t* req_ids;
-  const uint16_t* q;
-  const int32_t* topk;
-  int k;
-  const float* sink;
-  float scale;
-  uint16_t* out;
-  int G;              // heads per CTA (MMA N), 16 or 32
-  // split launch only: partials of (query i, tile t, head h)
-  float* ws_o;        // [n][tiles_max][H][D]
-  float2* ws_ml;      // [n][tiles_max][H]   (m_t, l_t); m_t = -inf: empty tile
-  int tiles_max;
-};
-
-struct QueryGeom {
-  int req;
-  bool csa;
-  int64_t t;          // query position
-  int64_t n_entries, w0, n_win, n_list, total;
-  int n_tiles;
-};
-
-__device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& g, bool report) {
-  const Layout& L = a.L;
-  g.req = a.req_ids[i];
-  if (g.req < 0 || g.req >= L.max_req) {
-    if (report) set_err(L, kErrBounds, i);
-    return false;
-  }
-  g.csa = a.layer < L.n_csa;
-  const int64_t T = L.lengths()[(int64_t)a.layer * L.max_req + g.req];
-  if (T <= 0) {
-    if (report) set_err(L, kErrBounds, 1000000 + i);
-    return false;
-  }
-  g.t = T - 1;
-  g.n_entries = g.csa ? T / kCsaM : T / kHcaM;
-  g.w0 = g.t - (kWindow - 1) > 0 ? g.t - (kWindow - 1) : 0;
-  g.n_win = g.t - g.w0 + 1;
-  g.n_list = g.csa ? a.k : g.n_entries;
-  g.total = g.n_list + g.n_win;
-  g.n_tiles = (int)((g.total + kTileRows - 1) / kTileRows);
-  return true;
-}
-
-// The fold of one partial into a running (m, l, O); shared by both launch
-// variants so that they round identically.
-__device__ __forceinline__ void fold_coef(float m, float mt, float& mn, float& al, float& be) {
-  mn = fmaxf(m, mt);
-  al = (m == -INFINITY) ? 0.f : expf(m - mn);
-  be = expf(mt - mn);
-}
-__device__ __forceinline__ float fold_val(float o, float al, float ot, float be) {
-  const float b = __fmul_rn(ot, be);
-  return al == 0.f ? b : __fmaf_rn(o, al, b);
-}
-__device__ __forceinline__ void finish_coef(float m, float sk, float l, float& cm, float& den) {
-  const float mu = fmaxf(m, sk);
-  cm = expf(m - mu);
-  den = __fmaf_rn(l, cm, expf(sk - mu));
-}
-__device__ __forceinline__ uint16_t finish_val(float o, float cm, float den) {
-  return bf16_rn(__fdiv_rn(__fmul_rn(o, cm), den));
-}
 
 struct AttnSmem {
   int Dp;             // head dim padded to a multiple of 128
@@ -364,7 +294,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       const int hh = x / (Dp / 8), c = x % (Dp / 8);
       raw[u] = make_uint4(0, 0, 0, 0);
       if (x < G * (Dp / 8) && h0 + hh < H && 8 * c < D)
-        raw[u] = *reinterpret_cast<const uint4*>(a.q + ((int64_t)i * H + h0 + hh) * D + 8 * c);
+        raw[u] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) + ((int64_t)i * H + h0 + hh) * D + 8 * c);
     }
 #pragma unroll
     for (int u = 0; u < kQPer; ++u) {
@@ -636,7 +566,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
           const int h = h0 + hb + e;
           float o = __uint_as_float(orun[e]);
           if (pend_fold) o = fold_val(o, alpha[hb + e], __uint_as_float(d < dmain ? om[e] : orp[e]), beta[hb + e]);
-          if (h < H && d < D) a.out[((int64_t)i * H + h) * D + d] = finish_val(o, cmul[hb + e], den[hb + e]);
+          if (h < H && d < D)
+            static_cast<uint16_t*>(a.out)[((int64_t)i * H + h) * D + d] = finish_val(o, cmul[hb + e], den[hb + e]);
         }
       }
     }
@@ -694,10 +625,22 @@ __global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
   }
   float cm, dn;
   finish_coef(m, a.sink[h], l, cm, dn);
+  if (a.f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + ((int64_t)i * H + h) * D + 4 * d4) =
+        make_float4(finish_f32(o[0], cm, dn), finish_f32(o[1], cm, dn), finish_f32(o[2], cm, dn),
+                    finish_f32(o[3], cm, dn));
+    return;
+  }
   uint2 pk;
   pk.x = (uint32_t)finish_val(o[0], cm, dn) | ((uint32_t)finish_val(o[1], cm, dn) << 16);
   pk.y = (uint32_t)finish_val(o[2], cm, dn) | ((uint32_t)finish_val(o[3], cm, dn) << 16);
-  *reinterpret_cast<uint2*>(a.out + ((int64_t)i * H + h) * D + 4 * d4) = pk;
+  *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + ((int64_t)i * H + h) * D + 4 * d4) = pk;
+}
+
+cudaError_t launch_attn_fold(const AttnArgs& a, cudaStream_t st) {
+  attn_fold_kernel<<<dim3(a.L.H, a.n), (a.L.D / 4 + 31) / 32 * 32, 0, st>>>(a);
+  note_launch();
+  return cudaGetLastError();
 }
 
 size_t attn_tc_smem_bytes(int D, int G) { return (size_t)attn_smem(D, G).total + 1024; }
@@ -718,7 +661,7 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   const size_t sm = attn_tc_smem_bytes(L.D, G);
   if (sm > 227 * 1024) return cudaErrorInvalidValue;
   const bool split = ws != nullptr;
-  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0};
+  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0, 0};
   const int n_hg = (L.H + G - 1) / G;
   if (!split) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -736,9 +679,7 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   note_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_fold_kernel<<<dim3(L.H, n), (L.D / 4 + 31) / 32 * 32, 0, st>>>(a);
-  note_launch();
-  return cudaGetLastError();
+  return launch_attn_fold(a, st);
 }
 
 // ---- scratch for csa_hca_decode_attn_noalloc

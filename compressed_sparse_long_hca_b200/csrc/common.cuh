@@ -115,6 +115,12 @@ __device__ __forceinline__ void store_kv_row(const float* row, int D, int R, uin
   if (threadIdx.x == 0) *scale = s;
 }
 
+// fp32 storage format: copy a row held in shared memory (already rotated) to
+// its stored place as it is.  All threads of the block take part.
+__device__ __forceinline__ void store_f32_row(const float* row, int n, float* dst) {
+  for (int d = threadIdx.x; d < n; d += blockDim.x) dst[d] = row[d];
+}
+
 // Quantise an index key held in shared memory (fp32, d_I values) to MXFP4 and
 // store it as key `s` of a page's index tile (code and scale layout in
 // layout.cuh).  One warp per 32-value chunk; padding chunks and scales are

@@ -28,6 +28,13 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k);
 size_t attn_noalloc_scratch_bytes();
 cudaError_t attn_noalloc_scratch(void** out);
+cudaError_t launch_wait_probe(const Layout& L, uint64_t limit_ns, cudaStream_t st);
+cudaError_t launch_index_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
+                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas_per_query,
+                             cudaStream_t st);
+cudaError_t launch_attn_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q,
+                            const int32_t* topk, int k, const float* sink, float scale, float* out, void* ws,
+                            cudaStream_t st);
 }  // namespace csa
 
 namespace {
@@ -76,6 +83,7 @@ bool cfg_ok(const csa_cfg* c, std::string* why) {
   if (c->max_pages_per_request < 1) return bad("max_pages_per_request must be >= 1");
   if (c->pool_pages < 1) return bad("pool_pages must be >= 1");
   if (!(c->rope_base > 1.f)) return bad("rope_base must be > 1");
+  if (c->fmt != CSA_FMT_MIXED && c->fmt != CSA_FMT_F32) return bad("fmt must be CSA_FMT_MIXED or CSA_FMT_F32");
   return true;
 }
 
@@ -89,6 +97,8 @@ Layout make_layout(const csa_cfg& c) {
   L.n_csa = c.n_csa_layers; L.n_hca = c.n_hca_layers; L.n_layers = c.n_csa_layers + c.n_hca_layers;
   L.max_req = c.max_requests; L.max_pages_per_req = c.max_pages_per_request;
   L.pool_pages = c.pool_pages; L.rope_base = c.rope_base;
+  L.fmt = c.fmt;
+  const bool f32 = c.fmt == CSA_FMT_F32;
   L.kv_fp8_bytes = c.D - c.D_rope;
   L.kv_bf16_bytes = 2 * (int64_t)c.D_rope;
   // window ring
@@ -96,6 +106,7 @@ Layout make_layout(const csa_cfg& c) {
   L.ring_bf16 = align_up(csa::kWindow * L.kv_fp8_bytes, 128);
   L.ring_scale = L.ring_bf16 + align_up(csa::kWindow * L.kv_bf16_bytes, 128);
   L.ring_bytes = L.ring_scale + align_up(csa::kWindow * 4, 128);
+  if (f32) L.ring_bytes = align_up((int64_t)csa::kWindow * c.D * 4, 128);
   L.csa_tail_bytes = align_up((int64_t)csa::kCsaWin * (2 * c.D + 2 * L.dI) * 4, 128);
   L.hca_tail_bytes = align_up((int64_t)csa::kHcaM * 2 * c.D * 4, 128);
   L.state_csa_layer = L.ring_bytes + L.csa_tail_bytes;
@@ -113,6 +124,12 @@ Layout make_layout(const csa_cfg& c) {
   L.pg_hca_bf16 = align_up(PH * L.kv_fp8_bytes, 16);
   L.pg_hca_scale = L.pg_hca_bf16 + align_up(PH * L.kv_bf16_bytes, 16);
   L.pg_hca_bytes = align_up(L.pg_hca_scale + PH * 4, 128);
+  L.pg_idx_f32 = 0;
+  if (f32) {   // fp32 rows [P][D], then (CSA) fp32 keys [P][d_I]
+    L.pg_idx_f32 = align_up(P * c.D * 4, 128);
+    L.pg_csa_bytes = align_up(L.pg_idx_f32 + P * L.dI * 4, 128);
+    L.pg_hca_bytes = align_up(PH * c.D * 4, 128);
+  }
   L.page_bytes = align_up(L.n_csa * L.pg_csa_bytes + L.n_hca * L.pg_hca_bytes, A);
   // arena sections
   int64_t o = 0;
@@ -266,10 +283,20 @@ csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, cons
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
   const int sms = sm_count();
   if (sms <= 0) return fail(CSA_ERR_CUDA, "cannot query the SM count");
-  // Two persistent CTAs per SM for either variant; the per-key arithmetic
-  // does not depend on the grid.
-  cudaError_t e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, 2 * sms,
-                                       (cudaStream_t)stream);
+  cudaError_t e;
+  if (c->L.fmt == csa::kFmtF32) {
+    // fp32 keys on the CUDA cores: one thread per key; the variants only
+    // change how many CTAs share a query (the per-key arithmetic is fixed)
+    const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < sms);
+    const int per_q = low ? std::max(1, (4 * sms + n - 1) / n) : 1;
+    e = csa::launch_index_f32(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, std::min(per_q, 1024),
+                              (cudaStream_t)stream);
+  } else {
+    // Two persistent CTAs per SM for either variant; the per-key arithmetic
+    // does not depend on the grid.
+    e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, 2 * sms,
+                             (cudaStream_t)stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "index launch");
   return CSA_OK;
 }
@@ -299,8 +326,8 @@ size_t csa_attn_workspace_bytes(const csa_cache_t* c, int32_t layer, int32_t n, 
 }
 
 csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
-                               const uint16_t* q, const int32_t* topk_idx, int32_t k, const float* sink,
-                               float scale, uint16_t* out, void* workspace, size_t workspace_bytes,
+                               const void* q, const int32_t* topk_idx, int32_t k, const float* sink,
+                               float scale, void* out, void* workspace, size_t workspace_bytes,
                                csa_variant variant, csa_stream_t stream) {
   if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
@@ -326,15 +353,20 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
   const int ctas = n * ((c->L.H + G - 1) / G);
   const bool split = variant == CSA_VARIANT_LOW_OCC ||
                      (variant == CSA_VARIANT_AUTO && ws_ok && ctas < sm_count());
-  cudaError_t e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, kk, sink, scale, out, G,
-                                      split ? workspace : nullptr, (cudaStream_t)stream);
+  cudaError_t e =
+      c->L.fmt == csa::kFmtF32
+          ? csa::launch_attn_f32(c->L, layer, n, req_ids, static_cast<const float*>(q), topk_idx, kk, sink, scale,
+                                 static_cast<float*>(out), split ? workspace : nullptr, (cudaStream_t)stream)
+          : csa::launch_attn_tc(c->L, layer, n, req_ids, static_cast<const uint16_t*>(q), topk_idx, kk, sink,
+                                scale, static_cast<uint16_t*>(out), G, split ? workspace : nullptr,
+                                (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
 }
 
 csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* c, int32_t layer, int32_t n,
-                                       const int32_t* req_ids, const uint16_t* q, const int32_t* topk_idx,
-                                       int32_t k, const float* sink, float scale, uint16_t* out,
+                                       const int32_t* req_ids, const void* q, const int32_t* topk_idx,
+                                       int32_t k, const float* sink, float scale, void* out,
                                        csa_stream_t stream) {
   if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
@@ -357,8 +389,11 @@ csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* c, int32_t layer, int3
   cudaError_t e = csa::attn_noalloc_scratch(&ws);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
   const int G = c->L.H <= 16 ? 16 : 32;
-  e = csa::launch_attn_tc(c->L, layer, n, req_ids, q, topk_idx, kk, sink, scale, out, G, ws,
-                          (cudaStream_t)stream);
+  e = c->L.fmt == csa::kFmtF32
+          ? csa::launch_attn_f32(c->L, layer, n, req_ids, static_cast<const float*>(q), topk_idx, kk, sink, scale,
+                                 static_cast<float*>(out), ws, (cudaStream_t)stream)
+          : csa::launch_attn_tc(c->L, layer, n, req_ids, static_cast<const uint16_t*>(q), topk_idx, kk, sink,
+                                scale, static_cast<uint16_t*>(out), G, ws, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
 }
@@ -398,11 +433,20 @@ csa_status csa_check_device_error(csa_cache_t* c, csa_stream_t stream) {
 
 const char* csa_last_error(void) { return g_err.c_str(); }
 
+csa_status csa_debug_wait_timeout(csa_cache_t* c, int32_t limit_us, csa_stream_t stream) {
+  if (!c) return fail(CSA_ERR_ARG, "cache is NULL");
+  if (limit_us < 1 || limit_us > 1000000) return fail(CSA_ERR_ARG, "limit_us must be in [1, 1000000]");
+  cudaError_t e = csa::launch_wait_probe(c->L, (uint64_t)limit_us * 1000ull, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe launch");
+  return CSA_OK;
+}
+
 size_t csa_debug_row_bytes(const csa_cache_t* c, int32_t region) {
   if (!c) return 0;
   const Layout& L = c->L;
-  if (region == CSA_REGION_KV || region == CSA_REGION_WINDOW) return (size_t)(L.D + L.R + 4);
-  if (region == CSA_REGION_INDEX) return (size_t)(L.dI / 2 + L.dI / 32);
+  const bool f32 = L.fmt == csa::kFmtF32;
+  if (region == CSA_REGION_KV || region == CSA_REGION_WINDOW) return f32 ? (size_t)L.D * 4 : (size_t)(L.D + L.R + 4);
+  if (region == CSA_REGION_INDEX) return f32 ? (size_t)L.dI * 4 : (size_t)(L.dI / 2 + L.dI / 32);
   return 0;
 }
 
@@ -445,6 +489,7 @@ csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t re
   auto& held = c->req_pages[req];
   char* h = static_cast<char*>(host);
   const bool wr = write != 0;
+  const bool f32 = L.fmt == csa::kFmtF32;
   if (region == CSA_REGION_WINDOW) {
     char* st = L.state(req, layer);
     std::vector<char> ring(L.ring_bytes);
@@ -453,6 +498,11 @@ csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t re
     for (int64_t r = 0; r < count; ++r) {
       const int slot = (int)((first + r) % csa::kWindow);
       char* row = h + r * rb;
+      if (f32) {
+        char* a = ring.data() + (int64_t)slot * rb;
+        if (wr) memcpy(a, row, rb); else memcpy(row, a, rb);
+        continue;
+      }
       char* a = ring.data() + L.ring_fp8 + slot * fp8b;
       char* b = ring.data() + L.ring_bf16 + slot * bfb;
       char* s = ring.data() + L.ring_scale + slot * 4;
@@ -480,6 +530,11 @@ csa_status csa_debug_rows(csa_cache_t* c, int32_t layer, int32_t req, int32_t re
     for (; r < count && (first + r) / per_pg == lp; ++r) {
       const int s = (int)((first + r) % per_pg);
       char* row = h + r * rb;
+      if (f32) {   // fp32 rows [P][D] then (CSA) fp32 keys [P][d_I]
+        char* a = buf.data() + (region == CSA_REGION_KV ? 0 : L.pg_idx_f32) + (int64_t)s * rb;
+        if (wr) memcpy(a, row, rb); else memcpy(row, a, rb);
+        continue;
+      }
       if (region == CSA_REGION_KV) {
         char* a = buf.data() + s * fp8b;
         char* b = buf.data() + (is_csa ? L.pg_csa_bf16 : L.pg_hca_bf16) + s * bfb;

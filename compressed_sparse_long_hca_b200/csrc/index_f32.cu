@@ -1,0 +1,84 @@
+// Lightning-indexer scores for caches in the fp32 storage format
+// (csa_index_scores on a CSA_FMT_F32 cache), on the CUDA cores.
+//
+// Page "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力": the query's
+// index heads are scored against every compressed index key after a ReLU,
+//   s_j = sum_h w_h * max(0, q_h . k_j),
+// here with q and the stored keys in fp32 (no FP4 quantisation).  One thread
+// computes one key's score in a fixed order (d ascending inside a head, heads
+// ascending), so a score never depends on the grid, the batch or the launch
+// variant; the two variants only differ in how many CTAs share a query.
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kIdxF32Threads = 256;
+
+struct IndexF32Args {
+  Layout L;
+  int layer;
+  int n;
+  const int32_t* req_ids;
+  const float* q_idx;     // [n][H_I][d_I]
+  const float* w;         // [n][H_I]
+  float* scores;          // [n][ld]
+  int64_t ld;
+  int32_t* n_valid;
+};
+
+}  // namespace
+
+// grid (CTAs per query, n); the CTAs of a query stride over its keys.
+__global__ void __launch_bounds__(kIdxF32Threads) index_f32_kernel(IndexF32Args a) {
+  extern __shared__ __align__(16) float sm_f[];
+  const Layout& L = a.L;
+  const int HI = L.HI, dI = L.dI;
+  float* qs = sm_f;                 // [H_I][d_I]
+  float* ws = sm_f + HI * dI;       // [H_I]
+  const int i = blockIdx.y, tid = threadIdx.x;
+  const int req = a.req_ids[i];
+  if (req < 0 || req >= L.max_req) {
+    if (blockIdx.x == 0 && tid == 0) {
+      set_err(L, kErrBounds, i);
+      a.n_valid[i] = 0;
+    }
+    return;
+  }
+  const int64_t N = L.lengths()[(int64_t)a.layer * L.max_req + req] / kCsaM;
+  if (blockIdx.x == 0 && tid == 0) {
+    a.n_valid[i] = (int32_t)N;
+    if (N > a.ld) set_err(L, kErrLd, i);
+  }
+  if (N > a.ld) return;
+  for (int x = tid; x < HI * dI; x += kIdxF32Threads) qs[x] = a.q_idx[(int64_t)i * HI * dI + x];
+  for (int x = tid; x < HI; x += kIdxF32Threads) ws[x] = a.w[(int64_t)i * HI + x];
+  __syncthreads();
+  float* out = a.scores + (int64_t)i * a.ld;
+  for (int64_t j = (int64_t)blockIdx.x * kIdxF32Threads + tid; j < N; j += (int64_t)gridDim.x * kIdxF32Threads) {
+    const float* k = L.index_key_f32(req, a.layer, j);
+    float s = 0.f;
+    for (int h = 0; h < HI; ++h) {
+      const float* qh = qs + h * dI;
+      float dot = 0.f;
+      for (int d = 0; d < dI; ++d) dot = fmaf(qh[d], k[d], dot);
+      s = fmaf(ws[h], fmaxf(dot, 0.f), s);
+    }
+    out[j] = s;
+  }
+}
+
+cudaError_t launch_index_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
+                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas_per_query,
+                             cudaStream_t st) {
+  IndexF32Args a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid};
+  const size_t sm = (size_t)(L.HI * L.dI + L.HI) * 4;
+  cudaError_t e = cudaFuncSetAttribute(index_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  index_f32_kernel<<<dim3(ctas_per_query, n), kIdxF32Threads, sm, st>>>(a);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -30,6 +30,13 @@
 //                 codes: 16 groups of 8 keys x CHs 16-byte chunks
 //                 scale chunk: 512 bytes of E8M0 scales
 //
+// Storage formats (one per cache):
+//   mixed (the pages' formats): as above.
+//   fp32: every stored vector is plain fp32 -- a KV row is D floats (RoPE
+//         dims rotated), an index key d_I floats; the ring is [128][D] fp32,
+//         a CSA page section [128][D] fp32 rows then [128][d_I] fp32 keys,
+//         an HCA page section [4][D] fp32 rows.
+//
 // Index keys are stored as one ready-made tcgen05 operand tile per page.
 // Codes: key s, 16-byte chunk c (32 E2M1 values) at (s/8)*(CHs*128) + c*128 +
 // (s%8)*16, the K-major no-swizzle core-matrix order (CHs = d_I/32 rounded up
@@ -57,9 +64,13 @@ constexpr int kSfChunk = 512;
 constexpr int64_t kAlign = 256;
 __host__ __device__ constexpr int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
+constexpr int kFmtMixed = 0;      // FP8 + BF16 rows, MXFP4 index keys
+constexpr int kFmtF32 = 1;        // fp32 rows and index keys
+
 struct Layout {
   // shapes
   int H, D, R, HI, dI, CHs;
+  int fmt;                  // kFmtMixed or kFmtF32
   int n_csa, n_hca, n_layers;
   int max_req, max_pages_per_req, pool_pages;
   float rope_base;
@@ -78,6 +89,7 @@ struct Layout {
   int64_t pg_csa_bf16, pg_csa_scale, pg_idx_codes, pg_idx_sf, pg_csa_bytes;
   int64_t pg_hca_bf16, pg_hca_scale, pg_hca_bytes;
   int64_t idx_tile_bytes;   // codes + scale chunk of one page (one bulk copy)
+  int64_t pg_idx_f32;       // fp32 format: offset of the index keys in a CSA page section
   int64_t page_bytes;
   int64_t total_bytes;
 
@@ -127,6 +139,18 @@ struct Layout {
     *fp8 = reinterpret_cast<const uint8_t*>(pp) + (int64_t)s * kv_fp8_bytes;
     *bf16 = reinterpret_cast<const uint16_t*>(pp + (csa ? pg_csa_bf16 : pg_hca_bf16)) + (int64_t)s * R;
     *scale = reinterpret_cast<const float*>(pp + (csa ? pg_csa_scale : pg_hca_scale)) + s;
+  }
+  // fp32 format: stored row of compressed entry j, its index key, a ring row
+  __host__ __device__ float* entry_row_f32(int req, int layer, int64_t j) const {
+    const int P = rows_per_page(layer);
+    return reinterpret_cast<float*>(page(page_table(req)[j / P], layer)) + (j % P) * D;
+  }
+  __host__ __device__ float* index_key_f32(int req, int layer, int64_t j) const {
+    return reinterpret_cast<float*>(page(page_table(req)[j / kCsaPerPage], layer) + pg_idx_f32) +
+           (j % kCsaPerPage) * dI;
+  }
+  __host__ __device__ float* ring_row_f32(int req, int layer, int slot) const {
+    return reinterpret_cast<float*>(state(req, layer)) + (int64_t)slot * D;
   }
   // byte offset of chunk c of index key s inside a page's code tile
   __host__ __device__ int64_t idx_code_off(int s, int c) const {

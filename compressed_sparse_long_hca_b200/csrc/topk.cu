@@ -431,14 +431,12 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     block_minmax(sv, sok, sh.mm[0], &smin, &smax);
     tau = block_select(sv, sok, r, smin, smax, sh, &unused);
   }
-  if (cached) {
-    // all threads observe the copy's completion (bounded wait)
-    const bool arrived = __syncthreads_and(tc::mbar_wait(&sh.bar, 0)) != 0;
-    if (!arrived) {
-      if (tid == 0 && a.err && atomicCAS(a.err, 0, (int32_t)kErrTimeout) == 0) a.err[1] = i;
-      return;
-    }
-  }
+  // all threads observe the copy's completion (bounded wait).  A CTA whose
+  // copy did not arrive does not leave on its own: it reports a count of -1
+  // in the count exchange below, and the whole cluster then leaves together
+  // after one more cluster barrier, so that no CTA touches the shared memory
+  // of a CTA that has gone.
+  const bool arrived = !cached || __syncthreads_and(tc::mbar_wait(&sh.bar, 0)) != 0;
 
   // ---- 2. filter: count, exchange counts, write candidates to the leader
   // Each warp owns a contiguous sub-slice (a multiple of 128 keys when the
@@ -459,7 +457,9 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
     }
   };
   int wc = 0;
-  if (cached) {
+  if (!arrived) {
+    // nothing to count: the slice never reached shared memory
+  } else if (cached) {
     int c = 0;
     for (int64_t x0 = w_lo; x0 < w_hi; x0 += 128) {
       uint32_t kv[4];
@@ -485,13 +485,20 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   }
   int cta_cnt;
   const int w_before = __shfl_sync(0xffffffffu, block_scan1(lane == 0 ? wc : 0, sh.scan_a, &cta_cnt), 0);
-  if (tid == 0) sh.n_cand = cta_cnt;
+  if (tid == 0) sh.n_cand = arrived ? cta_cnt : -1;
   cluster.sync();
   int base, total;
+  bool abort_all;
   {   // lane q reads CTA q's count (all remote reads in flight at once)
     const int c = lane < C ? *cluster.map_shared_rank(&sh.n_cand, lane) : 0;
     base = __reduce_add_sync(0xffffffffu, lane < rank ? c : 0);
     total = __reduce_add_sync(0xffffffffu, c);
+    abort_all = __any_sync(0xffffffffu, c < 0);   // the same decision in every CTA
+  }
+  if (abort_all) {
+    if (!arrived && tid == 0 && a.err && atomicCAS(a.err, 0, (int32_t)kErrTimeout) == 0) a.err[1] = i;
+    cluster.sync();   // every CTA has read every count before any leaves
+    return;
   }
   const bool filter = total >= k && total <= kCandCap;   // the same in every CTA
   if (filter) {

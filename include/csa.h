@@ -52,6 +52,8 @@
  *     batch size, its position in the batch or the other requests, and the
  *     two launch variants (csa_variant) return identical bits.
  *   - BF16 values are passed as uint16_t bit patterns.
+ *   - A cache holds one storage format (csa_fmt): the pages' mixed FP8 /
+ *     BF16 / MXFP4 format, or plain fp32 for the tiny fp32 configuration.
  */
 #ifndef CSA_H_
 #define CSA_H_
@@ -81,6 +83,15 @@ typedef enum {
   CSA_VARIANT_LOW_OCC = 2       /* launch shape for an under-fed GPU (small batch)*/
 } csa_variant;                  /* both return identical bits                     */
 
+/* Storage format of a cache (csa_cfg.fmt). */
+typedef enum {
+  CSA_FMT_MIXED = 0,            /* the pages' formats: KV rows FP8 E4M3 (non-RoPE
+                                   dims, one fp32 scale per row) + BF16 (RoPE dims),
+                                   index keys MXFP4; queries and outputs BF16     */
+  CSA_FMT_F32 = 1               /* every stored vector, query and output in fp32
+                                   (the tiny fp32 configuration)                  */
+} csa_fmt;
+
 /* Regions addressed by csa_debug_rows. */
 typedef enum {
   CSA_REGION_KV = 0,            /* compressed KV entries, by entry index          */
@@ -104,6 +115,7 @@ typedef enum {
  *                           (a page = 4 classic-cache blocks = 512 raw tokens:
  *                           128 CSA entries and 4 HCA entries per layer)
  *   rope_base               RoPE frequency base (10000)
+ *   fmt                     storage format (csa_fmt); 0 = CSA_FMT_MIXED
  * Entry geometry (fixed): CSA m = 4 with windows of 8 tokens overlapping by 4;
  * HCA m = 128, no overlap.
  */
@@ -120,6 +132,7 @@ typedef struct {
   int32_t max_pages_per_request;
   int32_t pool_pages;
   float rope_base;
+  int32_t fmt;
 } csa_cfg;
 
 /* Bytes of device memory the arena must have for `cfg` (0 if cfg invalid). */
@@ -187,8 +200,11 @@ csa_status csa_compress_append(csa_cache_t* cache, int32_t layer, int32_t n,
  * of its request (CSA layers only).  For query i (request req_ids[i], whose
  * length is T = L after the step's append, N = floor(T/4) entries):
  *   scores[i*ld + j] = sum_h w[i][h] * max(0, q^_h . k^_j),   j < N
- * where q^_h is q_idx[i][h] quantised to MXFP4 in the kernel and k^_j the
- * stored MXFP4 key.  Entries j >= N of the row are not written.
+ * where, in the mixed format, q^_h is q_idx[i][h] quantised to MXFP4 in the
+ * kernel and k^_j the stored MXFP4 key (block-scaled FP4 tensor-core MMA,
+ * fp32 accumulation); in the fp32 format q^_h = q_idx[i][h] and k^_j the
+ * stored fp32 key (fp32 FMA, d ascending, heads ascending).  Entries j >= N
+ * of the row are not written.  Both variants return identical bits.
  *   q_idx    device float [n][H_I][d_I]
  *   w        device float [n][H_I]
  *   scores   device float [n][ld]   (ld >= the largest N; checked on device)
@@ -214,12 +230,17 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
  * entries listed in topk_idx[i][0..k) in list order (-1 = an empty row), for
  * HCA layers (topk_idx == NULL) every completed entry in order, then the raw
  * window of positions max(0, t-127) .. t, t = L-1 the query's own position.
- * K = V = the stored row (FP8 x scale, BF16).  With q rotated at t:
+ * K = V = the stored row (mixed format: FP8 x scale, BF16; fp32 format: the
+ * fp32 row).  With q rotated at t:
  *   u_hr = scale * q_h . K_r,  mu_h = max(max_r u_hr, sink_h)
  *   out_h = sum_r e^{u_hr-mu_h} V_r / (sum_r e^{u_hr-mu_h} + e^{sink_h-mu_h})
- *   q     device uint16 (BF16) [n][H][D]   before RoPE; 16-byte aligned
+ *   q     device [n][H][D] before RoPE, 16-byte aligned: BF16 bit patterns
+ *         (uint16) in the mixed format, fp32 in the fp32 format
  *   sink  device float [H]
- *   out   device uint16 (BF16) [n][H][D]
+ *   out   device [n][H][D], the type of q
+ * The mixed format runs QK^T and PV on the tensor cores (BF16 operands, fp32
+ * accumulation, P rounded to BF16); the fp32 format runs them as fp32 FMA
+ * chains on the CUDA cores (tf32 would keep only 10 mantissa bits).
  * Source: page "V4终于终于终于终于是来了", sections "CSA——压缩稀疏注意力"
  * and "HCA——重度压缩注意力".
  *
@@ -245,9 +266,9 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
  */
 size_t     csa_attn_workspace_bytes(const csa_cache_t* cache, int32_t layer, int32_t n, int32_t k);
 csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t n,
-                               const int32_t* req_ids, const uint16_t* q,
+                               const int32_t* req_ids, const void* q,
                                const int32_t* topk_idx, int32_t k, const float* sink,
-                               float scale, uint16_t* out, void* workspace,
+                               float scale, void* out, void* workspace,
                                size_t workspace_bytes, csa_variant variant,
                                csa_stream_t stream);
 
@@ -263,8 +284,14 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
  * to a 16 MiB array built into the library instead of `workspace`:
  *   - every GPU that loads libcsa holds those 16 MiB until the process exits;
  *   - a batch whose scratch (csa_attn_workspace_bytes) exceeds 16 MiB is
- *     rejected with CSA_ERR_CAPACITY before anything is launched (C4-sized
- *     batches of 4 queries x 128 heads x k = 1024 need about 9.5 MiB);
+ *     rejected with CSA_ERR_CAPACITY before anything is launched.  The
+ *     scratch is n x tiles x H x (4 D + 8) bytes; with H = 128 and D = 512
+ *     that allows n x tiles <= 63.  On CSA layers tiles = ceil((k + 128) / 128)
+ *     (k = 1024: up to 7 queries; 4 queries need about 9.5 MiB).  On HCA
+ *     layers the host does not know the lengths, so tiles follows the
+ *     cache's capacity: tiles = ceil(P / 32) + 1 for P = max_pages_per_request;
+ *     at H = 128, D = 512 one query fits up to P = 1984 (1,015,808 tokens),
+ *     and a cache sized for 1M tokens (P >= 2048) is refused even for n = 1;
  *   - the first call on each device looks up the array's device address;
  *     make that first call before any stream capture;
  *   - all calls share the array: calls whose kernels may overlap on the GPU
@@ -274,9 +301,9 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
  * The call allocates no device memory.
  */
 csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* cache, int32_t layer, int32_t n,
-                                       const int32_t* req_ids, const uint16_t* q,
+                                       const int32_t* req_ids, const void* q,
                                        const int32_t* topk_idx, int32_t k, const float* sink,
-                                       float scale, uint16_t* out, csa_stream_t stream);
+                                       float scale, void* out, csa_stream_t stream);
 
 /*
  * Read and clear the device error word (synchronises `stream`).  Returns
@@ -309,6 +336,18 @@ csa_status csa_debug_rows(csa_cache_t* cache, int32_t layer, int32_t req, int32_
                           int64_t first, int64_t count, void* host, int32_t write);
 csa_status csa_debug_set_length(csa_cache_t* cache, int32_t layer, int32_t req, int64_t len);
 int64_t    csa_debug_get_length(csa_cache_t* cache, int32_t layer, int32_t req);
+
+/*
+ * Test helper for the device-side failure path: queue one thread block that
+ * waits on a shared-memory barrier nothing arrives on, through the same
+ * bounded-wait routine the tensor-core kernels use, with a limit of
+ * `limit_us` microseconds (1 .. 1000000).  The wait gives up, the block
+ * records a timeout in the cache's device error word and returns, so that
+ * csa_check_device_error then reports CSA_ERR_DEVICE_TIMEOUT and the context
+ * stays usable.  Asynchronous on `stream`; CSA_ERR_ARG for a NULL cache or a
+ * limit out of range.
+ */
+csa_status csa_debug_wait_timeout(csa_cache_t* cache, int32_t limit_us, csa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -288,20 +288,25 @@ def n_hca_entries(T: int, m: int = 128) -> int:
 
 
 def csa_entry_vectors(c, z, ci, zi, b_kv, b_idx, j: int, D: int, R: int,
-                      m: int = 4, base: float = 10000.0):
+                      m: int = 4, base: float = 10000.0, offset: int = 0):
     """Pooled fp64 KV vector (after RoPE at 4j) and pooled index-key vector of
-    CSA entry j.  c, z: [T, D]; ci, zi: [T, d_I]; b_kv: [2m, D]; b_idx: [2m, d_I]."""
+    CSA entry j.  c, z: [T, D]; ci, zi: [T, d_I]; b_kv: [2m, D]; b_idx: [2m, d_I].
+    Row x of c, z, ci, zi holds token position offset + x."""
     taus, slots = csa_window(j, m)
-    kv = pool(c[taus], z[taus], b_kv[slots])
+    rows = [t - offset for t in taus]
+    kv = pool(c[rows], z[rows], b_kv[slots])
     kv = rope(kv, m * j, R, base)
-    key = pool(ci[taus], zi[taus], b_idx[slots])
+    key = pool(ci[rows], zi[rows], b_idx[slots])
     return kv, key
 
 
 def hca_entry_vector(c, z, b_kv, j: int, D: int, R: int, m: int = 128,
-                     base: float = 10000.0):
+                     base: float = 10000.0, offset: int = 0):
+    """Pooled fp64 KV vector of HCA entry j (after RoPE at 128j); row x of c, z
+    holds token position offset + x."""
     taus, slots = hca_window(j, m)
-    kv = pool(c[taus], z[taus], b_kv[slots])
+    rows = [t - offset for t in taus]
+    kv = pool(c[rows], z[rows], b_kv[slots])
     return rope(kv, m * j, R, base)
 
 

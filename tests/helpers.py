@@ -49,7 +49,14 @@ def check_kv_rounding(gpu_rows: np.ndarray, ref_vals: np.ndarray, D: int, R: int
     bound = (np.abs(x[:, : D - R]) * 2.0 ** -4 + ref.scale.astype(np.float64)[:, None] * 2.0 ** -10) * 1.001 + 1e-30
     assert np.all(nope_err <= bound), f"{what}: FP8 part outside the rounding bound"
     rope_err = np.abs(v[:, D - R:] - x[:, D - R:])
-    assert np.all(rope_err <= np.abs(x[:, D - R:]) * 2.0 ** -8 * 1.001 + 1e-30), f"{what}: BF16 part outside bound"
+    # BF16 rounds to half an ulp (2^-9 relative; 2^-8 allowed).  The kernels
+    # pool in fp32 and the oracle in fp64, so a pooled or rotated value near
+    # zero (cancellation) also carries an absolute error of a few fp32 ulps
+    # of the row's magnitudes: 2^-18 x the row's RMS covers it (simulated
+    # worst case on 25.6M values: 2.7e-7 x RMS).
+    rms = np.sqrt(np.mean(x ** 2, axis=1, keepdims=True))
+    assert np.all(rope_err <= np.abs(x[:, D - R:]) * 2.0 ** -8 * 1.001 + 2.0 ** -18 * rms + 1e-30), \
+        f"{what}: BF16 part outside bound"
     same = (fp8 == ref.fp8).all(1) & (bf == ref.rope).all(1) & (sc == ref.scale)
     frac_elem = ((fp8 == ref.fp8).mean() + (bf == ref.rope).mean()) / 2
     assert frac_elem >= min_exact, f"{what}: only {frac_elem:.5f} of codes equal the oracle's"
@@ -156,3 +163,28 @@ class Pair:
     def gen_tokens(self, layer: int, req: int, start: int, count: int):
         return I.token_inputs(self.wl.seed, layer, req, start, count, self.wl.D,
                               self.wl.d_I if layer < self.n_csa else 0)
+
+
+def attention_over_stored_rows(cache, layer: int, req: int, t: int, sel, q, sink, D: int, R: int,
+                               scale: float | None = None) -> np.ndarray:
+    """The oracle's attention for the query at position t over the rows the
+    GPU path attends to: the stored entries listed in `sel` (the GPU's own
+    top-k, -1 = none; for HCA every entry) and the stored window, read back
+    from the cache.  Checks the attention kernel whatever the selection
+    (also when a tie-zone swap makes the GPU's selection differ from the
+    oracle's)."""
+    from compressed_sparse_long_hca_b200.api import unpack_kv_rows
+    sel = np.asarray(sel)
+    sel = sel[sel >= 0]
+    rows = []
+    if len(sel):
+        kv = np.concatenate([cache.read_rows(layer, req, 0, int(j), 1) for j in sel])
+        fp8, bf, sc = unpack_kv_rows(kv, D, R)
+        rows.append(O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc)))
+    wp = O.window_positions(t)
+    fp8, bf, sc = unpack_kv_rows(cache.read_rows(layer, req, 2, wp[0], len(wp)), D, R)
+    rows.append(O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc)))
+    rows = np.concatenate(rows, axis=0)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    return O.mqa_attention(O.rope(np.asarray(q, np.float64), t, R), rows, sink, scale)
+

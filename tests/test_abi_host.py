@@ -116,3 +116,4 @@ def test_cache_calls_on_a_null_handle_fail_on_the_host(cuda_lib):
     assert cuda_lib.csa_request_alloc(None, 0, 16) == -1
     assert cuda_lib.csa_request_free(None, 0) == -1
     assert cuda_lib.csa_check_device_error(None, None) == -1
+    assert cuda_lib.csa_debug_wait_timeout(None, 1000, None) == -1

@@ -95,15 +95,23 @@ def test_decode_step_graph_matches_individual_calls(layer):
     p = pairs[0].oracle_params(layer)
     for i, r in enumerate(reqs):
         st = pairs[0].states[(layer, r)]
+        t = st.T - 1
         if csa:
             res = O.decode_query(p, st, q[i], sink, k=wl.k, q_idx=v["q_idx"][i].numpy(), w=v["w"][i].numpy())
             N = st.T // 4
             Hp.check_topk(got_idx[i].numpy(), res["scores"], wl.k, N, what=f"request {r}")
-            if set(got_idx[i].numpy().tolist()) != set(res["topk"].tolist()):
-                continue                 # a tie-zone swap: the attention rows differ legitimately
+            sel = got_idx[i].numpy()
         else:
             res = O.decode_query(p, st, q[i], sink)
-        Hp.check_attention(got[i].float().numpy(), res["out"], f"request {r}")
+            sel = np.arange(st.T // 128)
+        # the attention over the rows the GPU selected and stored, always
+        Hp.check_attention(got[i].float().numpy(),
+                           Hp.attention_over_stored_rows(pairs[0].cache, layer, r, t, sel, q[i], sink, wl.D, wl.R),
+                           f"request {r} (stored rows)")
+        if not csa or set(sel.tolist()) == set(res["topk"].tolist()):
+            # and end to end against the oracle's own rows (a tie-zone swap
+            # changes the rows legitimately, which the check above covers)
+            Hp.check_attention(got[i].float().numpy(), res["out"], f"request {r}")
 
 
 def test_decode_step_rejects_unpinned_or_mis_sized_inputs():

@@ -58,6 +58,62 @@ def _fill(cache, layer, reqs, lengths, seed, D, dI):
     cache.check_device_error()
 
 
+def _compressor_check(cache, wl, layer, r, seed, T0, c_dec, csa):
+    """The compressor at the workload's shapes against the oracle, on the
+    device-generated inputs the fill appended (copied back to the host): the
+    first entries, an entry whose 8-token window straddles two fill calls
+    (CSA), the last entries before the decode token (positions near T0), and
+    the window rows including the decode token's own (host-generated) row."""
+    dI = wl.d_I if csa else 0
+    m = 4 if csa else 128
+    N = T0 // m
+    chunks = {}
+
+    def tokens(lo, hi):
+        """c, z, ci, zi of positions lo .. hi-1 (hi <= T0), fp64 on the host."""
+        parts = {k: [] for k in range(4)}
+        for ch in range(lo // I.CHUNK, (hi - 1) // I.CHUNK + 1):
+            if ch not in chunks:
+                g = I.device_token_inputs(seed, layer, r, ch, wl.D, dI)
+                chunks[ch] = [x.double().cpu().numpy() if x is not None else None for x in g]
+            a, b = max(lo, ch * I.CHUNK) - ch * I.CHUNK, min(hi, (ch + 1) * I.CHUNK) - ch * I.CHUNK
+            for k in range(4):
+                if chunks[ch][k] is not None:
+                    parts[k].append(chunks[ch][k][a:b])
+        return [np.concatenate(parts[k]) if parts[k] else None for k in range(4)]
+
+    params = _PARAMS[(wl.name, layer)]
+    ents = [0, 1, N - 2, N - 1]
+    if csa and T0 >= 2 * I.CHUNK:
+        ents.append((T0 // I.CHUNK - 1) * (I.CHUNK // 4))     # window [4096c - 4, 4096c + 4)
+    ents = sorted(set(e for e in ents if 0 <= e < N))
+    got_kv = np.concatenate([cache.read_rows(layer, r, 0, j, 1) for j in ents])
+    ref_kv, ref_key = [], []
+    for j in ents:
+        lo = max(0, m * j - (4 if csa else 0))
+        c, z, ci, zi = tokens(lo, m * j + m)
+        if csa:
+            kv, key = O.csa_entry_vectors(c, z, ci, zi, params["b_kv"], params["b_idx"], j, wl.D, wl.R, offset=lo)
+            ref_key.append(key)
+        else:
+            kv = O.hca_entry_vector(c, z, params["b_kv"], j, wl.D, wl.R, offset=lo)
+        ref_kv.append(kv)
+    Hp.check_kv_rounding(got_kv, np.stack(ref_kv), wl.D, wl.R, f"{wl.name} entries {ents}", min_exact=0.998)
+    if csa:
+        got_key = np.concatenate([cache.read_rows(layer, r, 1, j, 1) for j in ents])
+        Hp.check_index_rounding(got_key, np.stack(ref_key), wl.d_I, f"{wl.name} index keys {ents}", min_exact=0.998)
+    # window: positions T0-127 .. T0, the last one the decode token
+    wp = O.window_positions(T0)
+    c = tokens(wp[0], T0)[0]
+    c = np.concatenate([c, np.asarray(c_dec, np.float64).reshape(1, -1)])
+    win_ref = np.stack([O.raw_token_row(c[x], wp[x], wl.R) for x in range(len(wp))])
+    Hp.check_kv_rounding(cache.read_rows(layer, r, 2, wp[0], len(wp)), win_ref, wl.D, wl.R,
+                         f"{wl.name} window", min_exact=0.998)
+
+
+_PARAMS = {}
+
+
 def _host(seed, *shape):
     return np.random.default_rng(seed).standard_normal(shape).astype(np.float32)
 
@@ -143,6 +199,11 @@ def test_full_size_decode_step(name):
     qi = _host(wl.seed + 6, B, wl.H_I, wl.d_I) if csa else None
     w = _host(wl.seed + 7, B, wl.H_I) if csa else None
     sink = pair.params[0]["sink"]
+    # the compressor at these shapes (D = 512, R = 64, d_I = 128), against
+    # the oracle on the same inputs, for the first and the last request
+    _PARAMS[(wl.name, 0)] = pair.params[0]
+    for r in (0, B - 1):
+        _compressor_check(cache, wl, 0, r, wl.seed, T0, c[r], csa)
     base = _step(cache, wl, 0, list(range(B)), q, qi, w, sink)
     # oracle parity: every request of the small batches, four of the large ones
     check = list(range(B)) if B <= 4 else [0, 7, 18, B - 1]

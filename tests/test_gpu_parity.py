@@ -98,8 +98,13 @@ def test_c1_end_to_end_from_hidden_states():
     ok = same_key
     assert np.all(np.abs(s_gpu - res["scores"])[ok] <= 1e-5 * mag[ok] + 1e-6)
     Hp.check_topk(idx[0].cpu().numpy(), res["scores"], wl.k, N, excused=np.where(~ok)[0])
+    got_out = out[0].float().cpu().numpy()
+    # the attention over the rows the GPU selected and stored, whatever the selection
+    Hp.check_attention(got_out, Hp.attention_over_stored_rows(pair.cache, 0, 1, T, idx[0].cpu().numpy(), q, sink,
+                                                              64, 16), "c1 attention (stored rows)")
     if set(idx[0].cpu().numpy().tolist()) == set(res["topk"].tolist()):
-        Hp.check_attention(out[0].float().cpu().numpy(), res["out"], "c1 attention")
+        # and end to end against the oracle's own rows
+        Hp.check_attention(got_out, res["out"], "c1 attention")
     # scales are fp32 divisions of amax values that differ by fp32 rounding only
     from compressed_sparse_long_hca_b200.api import unpack_kv_rows
     sc_gpu = unpack_kv_rows(pair.cache.read_rows(0, 1, 0, 0, N), 64, 16)[2]

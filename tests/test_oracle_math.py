@@ -329,3 +329,73 @@ def test_decode_brute_force_tiny():
         den = sum(math.exp(x - mu) for x in u) + math.exp(sink[h] - mu)
         o = sum(math.exp(u[i] - mu) * rows[i] for i in range(len(rows))) / den
         assert np.allclose(res["out"][h], o)
+
+
+def _hca_brute_step(c, z, bh, q, sink, T, D, R, W):
+    """The HCA step written out with loops: every completed 128-token entry
+    pooled per channel (softmax over the block's tokens), rotated at its
+    first token and stored; the window's raw tokens rotated at their own
+    positions and stored; attention of every head over entries then window,
+    with the sink in the denominator."""
+    t = T - 1
+    rows = []
+    for j in range(T // 128):                      # only blocks whose 128 tokens have all arrived
+        taus = list(range(128 * j, 128 * j + 128))
+        kv = _brute_rope(_brute_entry(c.tolist(), z.tolist(), bh.tolist(), taus, list(range(128))), 128 * j, R)
+        rows.append(O.dequantize_kv(O.quantize_kv(np.array(kv)[None], R))[0])
+    n_ent = len(rows)
+    for tau in range(max(0, t - W + 1), t + 1):
+        rows.append(O.dequantize_kv(O.quantize_kv(np.array(_brute_rope(c[tau], tau, R))[None], R))[0])
+    out = np.zeros((q.shape[0], D))
+    for h in range(q.shape[0]):
+        qr = np.array(_brute_rope(q[h], t, R))
+        u = [float(qr @ row) / math.sqrt(D) for row in rows]
+        mu = max(max(u), sink[h])
+        den = sum(math.exp(x - mu) for x in u) + math.exp(sink[h] - mu)
+        out[h] = sum(math.exp(u[i] - mu) * rows[i] for i in range(len(rows))) / den
+    return out, n_ent
+
+
+@pytest.mark.parametrize("T", [130, 255, 256, 300])
+def test_hca_decode_brute_force_tiny(T):
+    """The HCA branch of decode_query (dense over every completed 128:1 entry,
+    then the window) against loops: a block counts only once all its 128
+    tokens have arrived (T = 255 sees one entry, T = 256 two), and the window
+    is the last W raw tokens."""
+    r = _rng(16)
+    D, R, H = 16, 4, 2
+    p = _tiny_layer("hca", r, D, R)
+    p.W = 8
+    c, z = r.standard_normal((T, D)), r.standard_normal((T, D))
+    st = O.RequestState()
+    O.append_tokens(st, c, z)
+    q = O.bf16_round(r.standard_normal((H, D)))
+    sink = r.standard_normal(H)
+    res = O.decode_query(p, st, q, sink)
+    ref, n_ent = _hca_brute_step(c, z, p.b_kv, q, sink, T, D, R, p.W)
+    assert n_ent == T // 128
+    assert res["n_rows"] == n_ent + min(T, p.W)
+    assert np.allclose(res["out"], ref, atol=1e-12)
+
+
+def test_hca_equals_csa_with_k_at_least_entries():
+    """With the same stored entries and window, the HCA branch (dense) gives
+    exactly what the CSA branch gives when k >= the number of entries (every
+    entry selected, in index order)."""
+    r = _rng(17)
+    D, R, H, dI = 32, 8, 4, 32
+    N, T = 37, 37 * 128 + 50
+    ent = O.quantize_kv(r.standard_normal((N, D)), R)
+    win = O.quantize_kv(r.standard_normal((128, D)), R)
+    keys = O.quantize_mxfp4(r.standard_normal((N, dI)))
+    q = O.bf16_round(r.standard_normal((H, D)))
+    sink = r.standard_normal(H)
+    ph = _tiny_layer("hca", r, D, R)
+    pc = _tiny_layer("csa", r, D, R, dI)
+    oh = O.decode_query(ph, None, q, sink, entries=(ent, None), window=win, T=T)
+    for k in (N, N + 5):
+        oc = O.decode_query(pc, None, q, sink, k=k, q_idx=r.standard_normal((2, dI)), w=r.standard_normal(2),
+                            entries=(ent, keys), window=win, T=T)
+        assert list(oc["topk"][:N]) == list(range(N))
+        assert np.array_equal(oh["out"], oc["out"])
+        assert oh["n_rows"] == oc["n_rows"] == N + 128
