@@ -15,6 +15,7 @@ from . import _lib
 from ._lib import CsaCfg, check
 
 VARIANTS = {"auto": _lib.VARIANT_AUTO, "high": _lib.VARIANT_HIGH_OCC, "low": _lib.VARIANT_LOW_OCC}
+FORMATS = {"mixed": _lib.FMT_MIXED, "f32": _lib.FMT_F32}
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:
@@ -48,10 +49,16 @@ class Cache:
     def __init__(self, *, n_csa: int, n_hca: int, H: int, D: int, D_rope: int, H_I: int, d_I: int,
                  max_requests: int, max_pages_per_request: int, pool_pages: int,
                  b_pos_csa=None, b_pos_idx=None, b_pos_hca=None, rope_base: float = 10000.0,
-                 device: str | torch.device = "cuda"):
+                 fmt: str = "mixed", device: str | torch.device = "cuda"):
+        """fmt: "mixed" (FP8 + BF16 rows, MXFP4 index keys, BF16 q and out) or
+        "f32" (fp32 rows, keys, q and out)."""
         self.lib = _lib.load()
+        if fmt not in FORMATS:
+            raise ValueError(f"fmt must be one of {sorted(FORMATS)}")
+        self.fmt = fmt
+        self.qdtype = torch.float32 if fmt == "f32" else torch.bfloat16
         self.cfg = CsaCfg(n_csa, n_hca, H, D, D_rope, H_I if n_csa else 0, d_I if n_csa else 0, 128,
-                          max_requests, max_pages_per_request, pool_pages, rope_base)
+                          max_requests, max_pages_per_request, pool_pages, rope_base, FORMATS[fmt])
         nbytes = self.lib.csa_cache_required_bytes(ctypes.byref(self.cfg))
         if nbytes == 0:
             raise ValueError("invalid cache configuration")
@@ -136,8 +143,8 @@ class Cache:
         this Cache object is grown to the size the library asks for."""
         n = req_ids.numel()
         _need(req_ids, torch.int32, name="req_ids")
-        _need(q, torch.bfloat16, (n, self.H, self.D), "q")
-        _need(out, torch.bfloat16, (n, self.H, self.D), "out")
+        _need(q, self.qdtype, (n, self.H, self.D), "q")
+        _need(out, self.qdtype, (n, self.H, self.D), "out")
         _need(sink, torch.float32, (self.H,), "sink")
         k = 0
         if topk_idx is not None:
@@ -195,16 +202,18 @@ def topk(scores: torch.Tensor, n_valid: torch.Tensor, k: int, out: torch.Tensor,
 
 # ---------------------------------------------------------------- one decode step, replayed
 
-def decode_step_fields(n: int, H: int, D: int, H_I: int, d_I: int, csa: bool, align: int = 256):
+def decode_step_fields(n: int, H: int, D: int, H_I: int, d_I: int, csa: bool, align: int = 256,
+                       qdtype=torch.bfloat16):
     """Packed layout of one decode step's inputs: a list of (name, dtype,
     shape, byte offset, bytes) with every field starting on an `align`-byte
-    boundary, and the buffer's total size.  The attention query q comes last,
-    so that everything before it is one contiguous copy."""
+    boundary, and the buffer's total size.  The attention query q (BF16, or
+    fp32 for an fp32 cache) comes last, so that everything before it is one
+    contiguous copy."""
     fields = [("c", torch.float32, (n, 1, D)), ("z", torch.float32, (n, 1, D))]
     if csa:
         fields += [("ci", torch.float32, (n, 1, d_I)), ("zi", torch.float32, (n, 1, d_I)),
                    ("q_idx", torch.float32, (n, H_I, d_I)), ("w", torch.float32, (n, H_I))]
-    fields.append(("q", torch.bfloat16, (n, H, D)))
+    fields.append(("q", qdtype, (n, H, D)))
     out, off = [], 0
     for name, dtype, shape in fields:
         nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
@@ -250,7 +259,7 @@ class DecodeStep:
         if self.csa and self.k <= 0:
             raise ValueError("a CSA layer needs k > 0")
         H, D = cache.H, cache.D
-        self._fields, off = decode_step_fields(n, H, D, cache.H_I, cache.d_I, self.csa)
+        self._fields, off = decode_step_fields(n, H, D, cache.H_I, cache.d_I, self.csa, qdtype=cache.qdtype)
         self.input_bytes = off
         self._q_off = next(f[3] for f in self._fields if f[0] == "q")
         dev = self.device = torch.device(device)
@@ -259,8 +268,8 @@ class DecodeStep:
         self._req = torch.tensor(ids, dtype=torch.int32, device=dev)
         self._sink = (sink if isinstance(sink, torch.Tensor) else torch.from_numpy(np.asarray(sink, np.float32)))
         self._sink = self._sink.to(device=dev, dtype=torch.float32).contiguous()
-        self.out = torch.empty((n, H, D), dtype=torch.bfloat16, device=dev)
-        self.host_out = torch.empty((n, H, D), dtype=torch.bfloat16).pin_memory()
+        self.out = torch.empty((n, H, D), dtype=cache.qdtype, device=dev)
+        self.host_out = torch.empty((n, H, D), dtype=cache.qdtype).pin_memory()
         self._ws = torch.empty(max(cache.attn_workspace_bytes(layer, n, self.k if self.csa else 0), 16),
                                dtype=torch.uint8, device=dev)
         self._side = torch.cuda.Stream(device=dev)

@@ -426,6 +426,7 @@ class LayerParams:
     m: int = 4
     W: int = 128
     base: float = 10000.0
+    fmt: str = "mixed"        # "mixed": FP8 + BF16 rows, MXFP4 keys; "f32": fp32 storage
 
 
 @dataclass
@@ -449,22 +450,33 @@ def append_tokens(st: RequestState, c, z, ci=None, zi=None) -> None:
             st.zi.append(np.asarray(zi[i], np.float64))
 
 
+def store_f32(x) -> np.ndarray:
+    """fp32 storage format (the tiny configuration is described as fp32):
+    a stored vector is its value rounded to fp32, with no other quantiser."""
+    return f32(x).astype(np.float64)
+
+
 def stored_entries(p: LayerParams, st: RequestState):
-    """Quantised compressed entries of the context: KV rows and (CSA) index keys."""
+    """Stored compressed entries of the context: KV rows and (CSA) index keys,
+    quantised (mixed format) or rounded to fp32 (fp32 format)."""
     c = np.array(st.c)
     z = np.array(st.z)
     if p.kind == "csa":
         kv, key = csa_entries_all(c, z, np.array(st.ci), np.array(st.zi),
                                   p.b_kv, p.b_idx, p.R, p.m, p.base)
+        if p.fmt == "f32":
+            return store_f32(kv), store_f32(key)
         return quantize_kv(kv, p.R), quantize_mxfp4(key)
     kv = hca_entries_all(c, z, p.b_kv, p.R, p.m, p.base)
+    if p.fmt == "f32":
+        return store_f32(kv), None
     return quantize_kv(kv, p.R), None
 
 
-def stored_window(p: LayerParams, st: RequestState, t: int) -> KVRow:
+def stored_window(p: LayerParams, st: RequestState, t: int):
     pos = window_positions(t, p.W)
     rows = np.stack([raw_token_row(st.c[tau], tau, p.R, p.base) for tau in pos])
-    return quantize_kv(rows, p.R)
+    return store_f32(rows) if p.fmt == "f32" else quantize_kv(rows, p.R)
 
 
 def bf16_round(x) -> np.ndarray:
@@ -477,7 +489,9 @@ def decode_query(p: LayerParams, st: RequestState | None, q, sink, k: int | None
                  entries=None, window=None, T: int | None = None):
     """Full decode step for the query at position t = T - 1 (the token just
     appended): index scores, top-k and attention for CSA; dense attention
-    over all entries for HCA.  q: [H, D] BF16 values before RoPE.
+    over all entries for HCA.  q: [H, D] before RoPE (BF16 values in the
+    mixed format, fp32 values in the fp32 format, where the index query is
+    used as given instead of through MXFP4).
     `entries` / `window` may hand in stored rows directly (then `st` may be
     None and T gives the context length).  Returns a dict with the
     intermediate results."""
@@ -488,20 +502,25 @@ def decode_query(p: LayerParams, st: RequestState | None, q, sink, k: int | None
         entries = stored_entries(p, st)
     kvq, keyq = entries
     win = window if window is not None else stored_window(p, st, t)
+    f32_fmt = p.fmt == "f32"
+    value = (lambda rows: np.asarray(rows, np.float64)) if f32_fmt else dequantize_kv
     out = {}
     if p.kind == "csa":
-        qi = dequantize_mxfp4(quantize_mxfp4(q_idx))
-        s = index_scores(qi, w, dequantize_mxfp4(keyq))
+        if f32_fmt:
+            s = index_scores(store_f32(q_idx), w, keyq)
+        else:
+            qi = dequantize_mxfp4(quantize_mxfp4(q_idx))
+            s = index_scores(qi, w, dequantize_mxfp4(keyq))
         out["scores"] = s
         # the kernels select on fp32 scores; the oracle selects on its fp64
         # scores (comparison tolerance covers the difference)
         sel = topk(s, k)
         out["topk"] = sel
         j = sel[sel >= 0]
-        rows = dequantize_kv(KVRow(fp8=kvq.fp8[j], rope=kvq.rope[j], scale=kvq.scale[j]))
+        rows = kvq[j] if f32_fmt else dequantize_kv(KVRow(fp8=kvq.fp8[j], rope=kvq.rope[j], scale=kvq.scale[j]))
     else:
-        rows = dequantize_kv(kvq)
-    rows = np.concatenate([rows, dequantize_kv(win)], axis=0)
+        rows = value(kvq)
+    rows = np.concatenate([rows, value(win)], axis=0)
     qr = rope(np.asarray(q, np.float64), t, p.R, p.base)
     out["out"] = mqa_attention(qr, rows, sink, scale)
     out["n_rows"] = rows.shape[0]

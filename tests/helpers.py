@@ -19,16 +19,23 @@ from oracle import csa_oracle as O
 ATT_ATOL = 1e-2
 ATT_RTOL = 2e-2
 TOPK_TIE_REL = 1e-3     # oracle scores within this of the k-th score are a tie zone
+# Attention output in the fp32 storage format: fp32 operands and fp32 FMA
+# chains.  A logit's error is about D * 2^-24 * sum|q_d k_d| (< 1e-5 for the
+# tiny configuration), which moves an output by ~1e-5 relative; the bound
+# below leaves a factor of about 10.
+F32_ATT_ATOL = 1e-4
+F32_ATT_RTOL = 1e-4
 
 
-def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "attention") -> float:
+def check_attention(gpu: np.ndarray, ref: np.ndarray, what: str = "attention", fmt: str = "mixed") -> float:
     """Returns the largest |gpu - ref| / sigma seen."""
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)
     sigma = math.sqrt(float(np.mean(ref ** 2))) or 1.0
     err = np.abs(gpu - ref)
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
-    bad = err > ATT_ATOL * sigma + ATT_RTOL * np.abs(ref)
+    atol, rtol = (F32_ATT_ATOL, F32_ATT_RTOL) if fmt == "f32" else (ATT_ATOL, ATT_RTOL)
+    bad = err > atol * sigma + rtol * np.abs(ref)
     assert not bad.any(), (f"{what}: {int(bad.sum())} elements outside tolerance; worst "
                            f"|err|/sigma {err.max() / sigma:.3e}")
     return float(err.max() / sigma)
@@ -111,10 +118,11 @@ class Pair:
     """One CUDA cache plus the oracle's state for the same requests."""
 
     def __init__(self, wl: I.Workload, n_csa: int, n_hca: int, max_req: int, capacity: int,
-                 pool_blocks: int | None = None):
+                 pool_blocks: int | None = None, fmt: str = "mixed"):
         import torch
         from compressed_sparse_long_hca_b200.api import Cache
         self.wl = wl
+        self.fmt = fmt
         self.n_csa, self.n_hca = n_csa, n_hca
         self.params = []
         bkv, bix, bh = [], [], []
@@ -133,15 +141,15 @@ class Pair:
                            max_pages_per_request=nb, pool_pages=pool_blocks or nb * max_req,
                            b_pos_csa=np.stack(bkv) if bkv else None,
                            b_pos_idx=np.stack(bix) if bix else None,
-                           b_pos_hca=np.stack(bh) if bh else None)
+                           b_pos_hca=np.stack(bh) if bh else None, fmt=fmt)
         self.torch = torch
         self.states = {}   # (layer, req) -> O.RequestState
 
     def oracle_params(self, layer: int) -> O.LayerParams:
         p = self.params[layer]
         if p["kind"] == "csa":
-            return O.LayerParams("csa", self.wl.D, self.wl.R, p["b_kv"], p["b_idx"])
-        return O.LayerParams("hca", self.wl.D, self.wl.R, p["b_kv"], None, m=128)
+            return O.LayerParams("csa", self.wl.D, self.wl.R, p["b_kv"], p["b_idx"], fmt=self.fmt)
+        return O.LayerParams("hca", self.wl.D, self.wl.R, p["b_kv"], None, m=128, fmt=self.fmt)
 
     def append(self, layer: int, reqs, tokens: dict, n_tok: int, stream=None, oracle=True):
         """Append n_tok tokens to each request in `reqs`; tokens[req] = (c, z, ci, zi)."""
@@ -174,17 +182,38 @@ def attention_over_stored_rows(cache, layer: int, req: int, t: int, sel, q, sink
     (also when a tie-zone swap makes the GPU's selection differ from the
     oracle's)."""
     from compressed_sparse_long_hca_b200.api import unpack_kv_rows
+
+    def value(packed):
+        if cache.fmt == "f32":
+            return f32_rows_value(packed, D)
+        fp8, bf, sc = unpack_kv_rows(packed, D, R)
+        return O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc))
+
     sel = np.asarray(sel)
     sel = sel[sel >= 0]
     rows = []
     if len(sel):
-        kv = np.concatenate([cache.read_rows(layer, req, 0, int(j), 1) for j in sel])
-        fp8, bf, sc = unpack_kv_rows(kv, D, R)
-        rows.append(O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc)))
+        rows.append(value(np.concatenate([cache.read_rows(layer, req, 0, int(j), 1) for j in sel])))
     wp = O.window_positions(t)
-    fp8, bf, sc = unpack_kv_rows(cache.read_rows(layer, req, 2, wp[0], len(wp)), D, R)
-    rows.append(O.dequantize_kv(O.KVRow(fp8=fp8, rope=bf, scale=sc)))
+    rows.append(value(cache.read_rows(layer, req, 2, wp[0], len(wp))))
     rows = np.concatenate(rows, axis=0)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     return O.mqa_attention(O.rope(np.asarray(q, np.float64), t, R), rows, sink, scale)
+
+
+def check_f32_rows(gpu_rows: np.ndarray, ref_vals: np.ndarray, what="rows") -> None:
+    """fp32 storage format: stored rows (packed fp32 bytes) against the
+    oracle's fp64 values.  The kernels pool in fp32 (a few ulps; near-zero
+    values after cancellation carry a few ulps of the row's magnitudes), so
+    |gpu - ref| <= 2^-20 |ref| + 2^-18 rms(row)."""
+    g = np.ascontiguousarray(gpu_rows).view(np.float32).astype(np.float64).reshape(np.asarray(ref_vals).shape)
+    x = np.asarray(ref_vals, np.float64)
+    rms = np.sqrt(np.mean(x ** 2, axis=1, keepdims=True))
+    err = np.abs(g - x)
+    bad = err > 2.0 ** -20 * np.abs(x) + 2.0 ** -18 * rms + 1e-30
+    assert not bad.any(), f"{what}: {int(bad.sum())} values outside the fp32 bound; worst {err.max():.3e}"
+
+
+def f32_rows_value(gpu_rows: np.ndarray, d: int) -> np.ndarray:
+    return np.ascontiguousarray(gpu_rows).view(np.float32).astype(np.float64).reshape(-1, d)
 

@@ -285,13 +285,25 @@ def test_window_visibility():
     assert O.window_positions(1000) == list(range(873, 1001))
 
 
-def test_decode_brute_force_tiny():
+def _stored_value(x, R, fmt):
+    """What a stored vector stands for: its fp32 rounding (fp32 format), or
+    its FP8 + BF16 quantisation (mixed format)."""
+    x = np.asarray(x, np.float64)[None]
+    if fmt == "f32":
+        return np.array([float(np.float32(v)) for v in x[0]])
+    return O.dequantize_kv(O.quantize_kv(x, R))[0]
+
+
+@pytest.mark.parametrize("fmt", ["mixed", "f32"])
+def test_decode_brute_force_tiny(fmt):
     """The whole CSA step, written out with loops over positions for a tiny
-    context, against decode_query."""
+    context, against decode_query, in both storage formats (fp32: stored
+    vectors and the index query rounded to fp32, no quantiser)."""
     r = _rng(15)
     D, R, dI, H, HI, k, T = 32, 8, 32, 2, 2, 3, 45
     p = _tiny_layer("csa", r, D, R, dI)
     p.W = 8
+    p.fmt = fmt
     st = O.RequestState()
     c, z = r.standard_normal((T, D)), r.standard_normal((T, D))
     ci, zi = r.standard_normal((T, dI)), r.standard_normal((T, dI))
@@ -306,10 +318,16 @@ def test_decode_brute_force_tiny():
         taus = [x for x in range(4 * j - 4, 4 * j + 4) if x >= 0]
         slots = [x - (4 * j - 4) for x in taus]
         kv = _brute_rope(_brute_entry(c.tolist(), z.tolist(), p.b_kv.tolist(), taus, slots), 4 * j, R)
-        kvs.append(O.dequantize_kv(O.quantize_kv(np.array(kv)[None], R))[0])
+        kvs.append(_stored_value(kv, R, fmt))
         kk = _brute_entry(ci.tolist(), zi.tolist(), p.b_idx.tolist(), taus, slots)
-        keys.append(O.dequantize_mxfp4(O.quantize_mxfp4(np.array(kk)[None]))[0])
-    qd = O.dequantize_mxfp4(O.quantize_mxfp4(qi))
+        if fmt == "f32":
+            keys.append(np.array([float(np.float32(v)) for v in kk]))
+        else:
+            keys.append(O.dequantize_mxfp4(O.quantize_mxfp4(np.array(kk)[None]))[0])
+    if fmt == "f32":
+        qd = np.array([[float(np.float32(v)) for v in row] for row in qi])
+    else:
+        qd = O.dequantize_mxfp4(O.quantize_mxfp4(qi))
     scores = []
     for j in range(len(keys)):
         s = 0.0
@@ -321,7 +339,7 @@ def test_decode_brute_force_tiny():
     assert list(res["topk"]) == sel
     rows = [kvs[j] for j in sel]
     for tau in range(max(0, t - p.W + 1), t + 1):
-        rows.append(O.dequantize_kv(O.quantize_kv(np.array(_brute_rope(c[tau], tau, R))[None], R))[0])
+        rows.append(_stored_value(_brute_rope(c[tau], tau, R), R, fmt))
     qr = np.array([_brute_rope(q[h], t, R) for h in range(H)])
     for h in range(H):
         u = [qr[h] @ row / math.sqrt(D) for row in rows]
@@ -331,7 +349,7 @@ def test_decode_brute_force_tiny():
         assert np.allclose(res["out"][h], o)
 
 
-def _hca_brute_step(c, z, bh, q, sink, T, D, R, W):
+def _hca_brute_step(c, z, bh, q, sink, T, D, R, W, fmt="mixed"):
     """The HCA step written out with loops: every completed 128-token entry
     pooled per channel (softmax over the block's tokens), rotated at its
     first token and stored; the window's raw tokens rotated at their own
@@ -342,10 +360,10 @@ def _hca_brute_step(c, z, bh, q, sink, T, D, R, W):
     for j in range(T // 128):                      # only blocks whose 128 tokens have all arrived
         taus = list(range(128 * j, 128 * j + 128))
         kv = _brute_rope(_brute_entry(c.tolist(), z.tolist(), bh.tolist(), taus, list(range(128))), 128 * j, R)
-        rows.append(O.dequantize_kv(O.quantize_kv(np.array(kv)[None], R))[0])
+        rows.append(_stored_value(kv, R, fmt))
     n_ent = len(rows)
     for tau in range(max(0, t - W + 1), t + 1):
-        rows.append(O.dequantize_kv(O.quantize_kv(np.array(_brute_rope(c[tau], tau, R))[None], R))[0])
+        rows.append(_stored_value(_brute_rope(c[tau], tau, R), R, fmt))
     out = np.zeros((q.shape[0], D))
     for h in range(q.shape[0]):
         qr = np.array(_brute_rope(q[h], t, R))
@@ -356,8 +374,9 @@ def _hca_brute_step(c, z, bh, q, sink, T, D, R, W):
     return out, n_ent
 
 
+@pytest.mark.parametrize("fmt", ["mixed", "f32"])
 @pytest.mark.parametrize("T", [130, 255, 256, 300])
-def test_hca_decode_brute_force_tiny(T):
+def test_hca_decode_brute_force_tiny(T, fmt):
     """The HCA branch of decode_query (dense over every completed 128:1 entry,
     then the window) against loops: a block counts only once all its 128
     tokens have arrived (T = 255 sees one entry, T = 256 two), and the window
@@ -366,13 +385,14 @@ def test_hca_decode_brute_force_tiny(T):
     D, R, H = 16, 4, 2
     p = _tiny_layer("hca", r, D, R)
     p.W = 8
+    p.fmt = fmt
     c, z = r.standard_normal((T, D)), r.standard_normal((T, D))
     st = O.RequestState()
     O.append_tokens(st, c, z)
     q = O.bf16_round(r.standard_normal((H, D)))
     sink = r.standard_normal(H)
     res = O.decode_query(p, st, q, sink)
-    ref, n_ent = _hca_brute_step(c, z, p.b_kv, q, sink, T, D, R, p.W)
+    ref, n_ent = _hca_brute_step(c, z, p.b_kv, q, sink, T, D, R, p.W, fmt)
     assert n_ent == T // 128
     assert res["n_rows"] == n_ent + min(T, p.W)
     assert np.allclose(res["out"], ref, atol=1e-12)
