@@ -1,8 +1,8 @@
 """Benchmark of the CSA / HCA compressed-attention decode step on B200.
 
 One step = one decode step of one layer for a batch of requests: compressor
-append of the new token (csa_compress_append), lightning-indexer scores
-(csa_index_scores), top-k (csa_topk) and multi-query attention
+append of the new token (csa_compress_append), lightning-indexer scores and
+top-k in one launch (csa_index_topk) and multi-query attention
 (csa_hca_decode_attn), all through the C ABI.  Inputs are seeded synthetic
 data of the workload's shapes; caches are filled through the same append
 path before timing.
@@ -208,7 +208,7 @@ def run_gpu(args):
     import torch.distributed as dist
 
     from compressed_sparse_long_hca_b200 import _lib
-    from compressed_sparse_long_hca_b200.api import Cache, DecodeStep, topk
+    from compressed_sparse_long_hca_b200.api import Cache, DecodeStep
 
     ws, rank, local = _dist()
     torch.cuda.set_device(local)
@@ -288,16 +288,15 @@ def run_gpu(args):
     def part_append():
         cache.compress_append(layer, rid, in_c, in_z, in_ci, in_zi)
 
-    def part_index():
-        cache.index_scores(layer, rid, qi, w, scores, nv)
+    tk_ws = torch.empty(cache.index_topk_workspace_bytes(B, ld) + 256, dtype=torch.uint8, device="cuda") if csa else None
 
-    def part_topk():
-        topk(scores, nv, wl.k, idx)
+    def part_index_topk():
+        cache.index_topk(layer, rid, qi, w, scores, nv, wl.k, idx, workspace=tk_ws)
 
     def part_attn():
         cache.decode_attn(layer, rid, q, idx if csa else None, sink_d, out)
 
-    parts = [("append", part_append)] + ([("index", part_index), ("topk", part_topk)] if csa else []) + \
+    parts = [("append", part_append)] + ([("index_topk", part_index_topk)] if csa else []) + \
         [("attention", part_attn)]
     for s in range(warm):                   # eager warm-up (also sizes the attention workspace)
         load_inputs(s)
@@ -325,7 +324,7 @@ def run_gpu(args):
     launches0 = lib.csa_launch_count()
     g_plain, _ = capture(())
     kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graph
-    roof_part = "index" if csa else "attention"       # the kernel the roofline is reported for
+    roof_part = "index_topk" if csa else "attention"  # the kernel the roofline is reported for
     g_idx, ev_idx = capture((roof_part,))
     g_all, ev_all = capture(tuple(nm for nm, _ in parts))
     for gr in (g_plain, g_idx, g_all):      # a graph's first replay also uploads it: not timed
@@ -439,7 +438,7 @@ def run_gpu(args):
         n_c = t_mid // 4
         alg = B * (n_c * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
         ach = alg / (idx_ms / 1e3) / 1e9
-        line["roofline"] = {"bound": "hbm", "kernel": "csa_index_scores", "achieved": ach, "peak": peak,
+        line["roofline"] = {"bound": "hbm", "kernel": "csa_index_topk", "achieved": ach, "peak": peak,
                             "unit": "GB/s", "frac": ach / peak, "traffic": _profiled_traffic(),
                             "peak_source": peak_kind, "ms_per_launch": idx_ms,
                             "algorithmic_bytes_per_launch": alg}

@@ -19,6 +19,10 @@ REGION_KV, REGION_INDEX, REGION_WINDOW = 0, 1, 2
 FMT_MIXED, FMT_F32 = 0, 1
 
 
+class GemmOut(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int32), ("bf16", ctypes.c_int32), ("y", ctypes.c_void_p)]
+
+
 class CsaCfg(ctypes.Structure):
     _fields_ = [("n_csa_layers", ctypes.c_int32), ("n_hca_layers", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("D", ctypes.c_int32), ("D_rope", ctypes.c_int32),
@@ -38,6 +42,8 @@ SIGNATURES = {
     "csa_compress_append": (_I32, [_P, _I32, _I32, _P, _I32, _P, _P, _P, _P, _P]),
     "csa_index_scores": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _I64, _P, _I32, _P]),
     "csa_topk": (_I32, [_P, _I64, _P, _I32, _I32, _P, _I32, _P]),
+    "csa_index_topk_workspace_bytes": (_SZ, [_P, _I32, _I64]),
+    "csa_index_topk": (_I32, [_P, _I32, _I32, _P, _P, _P, _P, _I64, _P, _I32, _P, _P, _SZ, _I32, _P]),
     "csa_attn_workspace_bytes": (_SZ, [_P, _I32, _I32, _I32]),
     "csa_hca_decode_attn": (_I32, [_P, _I32, _I32, _P, _P, _P, _I32, _P, _F, _P, _P, _SZ, _I32, _P]),
     "csa_hca_decode_attn_noalloc": (_I32, [_P, _I32, _I32, _P, _P, _P, _I32, _P, _F, _P, _P]),
@@ -49,6 +55,11 @@ SIGNATURES = {
     "csa_debug_set_length": (_I32, [_P, _I32, _I32, _I64]),
     "csa_debug_get_length": (_I64, [_P, _I32, _I32]),
     "csa_debug_wait_timeout": (_I32, [_P, _I32, _P]),
+    "csa_gemm_weight_bytes": (_SZ, [_I32, _I32, _I32]),
+    "csa_gemm_pack_weight": (_I32, [_P, _I32, _I32, _I32, _P, _SZ]),
+    "csa_gemm_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32]),
+    "csa_gemm_bf16": (_I32, [_P, _I32, _I32, _I32, _P, _I32, _I32, _P, _P, _SZ, _P]),
+    "csa_gemm_check_device_error": (_I32, [_P]),
 }
 
 _lib = None

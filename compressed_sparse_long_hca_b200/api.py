@@ -126,6 +126,40 @@ class Cache:
                                         _ptr(scores), scores.shape[1], _ptr(n_valid),
                                         VARIANTS[variant], _stream(stream)), "csa_index_scores")
 
+    def index_topk(self, layer: int, req_ids, q_idx, w, scores, n_valid, k: int, idx_out, variant="auto",
+                   stream=None, workspace: torch.Tensor | None = None) -> None:
+        """Index scores and top-k in one launch (csa_index_topk): the same
+        results as index_scores followed by topk.  Unless `workspace` is
+        given, a buffer owned by this Cache object is grown to the size the
+        library asks for."""
+        n = req_ids.numel()
+        _need(req_ids, torch.int32, name="req_ids")
+        _need(q_idx, torch.float32, (n, self.H_I, self.d_I), "q_idx")
+        _need(w, torch.float32, (n, self.H_I), "w")
+        _need(scores, torch.float32, name="scores")
+        _need(n_valid, torch.int32, (n,), "n_valid")
+        _need(idx_out, torch.int32, (n, k), "idx_out")
+        if scores.dim() != 2 or scores.shape[0] != n:
+            raise ValueError("scores must be [n, ld]")
+        ws_ptr, ws_bytes = None, 0
+        if n > 0:
+            need = self.index_topk_workspace_bytes(n, scores.shape[1])
+            if workspace is None:
+                ws = getattr(self, "_tk_ws", None)
+                if ws is None or ws.numel() < need + 256 or ws.device != q_idx.device:
+                    ws = torch.empty(need + 256, dtype=torch.uint8, device=q_idx.device)
+                    self._tk_ws = ws
+                workspace = ws
+            _need(workspace, torch.uint8, name="workspace")
+            ws_ptr = (workspace.data_ptr() + 255) // 256 * 256
+            ws_bytes = workspace.numel() - (ws_ptr - workspace.data_ptr())
+        check(self.lib.csa_index_topk(self.handle, layer, n, _ptr(req_ids), _ptr(q_idx), _ptr(w), _ptr(scores),
+                                      scores.shape[1], _ptr(n_valid), k, _ptr(idx_out), ws_ptr, ws_bytes,
+                                      VARIANTS[variant], _stream(stream)), "csa_index_topk")
+
+    def index_topk_workspace_bytes(self, n: int, ld: int) -> int:
+        return int(self.lib.csa_index_topk_workspace_bytes(self.handle, n, ld))
+
     def attn_workspace_bytes(self, layer: int, n: int, k: int = 0) -> int:
         return int(self.lib.csa_attn_workspace_bytes(self.handle, layer, n, k))
 
@@ -227,9 +261,9 @@ class DecodeStep:
     once as two CUDA graphs and replayed every step.
 
     The step appends each request's new token (csa_compress_append), then on
-    a CSA layer scores the index keys (csa_index_scores) and selects the top
-    k (csa_topk) -- the first graph -- and attends (csa_hca_decode_attn) --
-    the second graph; on an HCA layer the first graph only appends and the
+    a CSA layer scores the index keys and selects the top k in one launch
+    (csa_index_topk) -- the first graph -- and attends (csa_hca_decode_attn)
+    -- the second graph; on an HCA layer the first graph only appends and the
     attention covers every compressed entry.
 
     Inputs of a step, packed in a buffer from `new_host_inputs()` and filled
@@ -245,8 +279,8 @@ class DecodeStep:
 
     The graphs hold device pointers, so the batch (req_ids), k and the sink
     logits are fixed at construction.  On a CSA layer construction runs the
-    index and top-k kernels once (they change nothing in the cache) so that
-    their one-time launch set-up happens before the capture."""
+    selection once (it changes nothing in the cache) so that its one-time
+    launch set-up happens before the capture."""
 
     def __init__(self, cache: Cache, layer: int, req_ids, k: int, sink, variant: str = "auto",
                  device: str | torch.device = "cuda"):
@@ -280,9 +314,13 @@ class DecodeStep:
             self._nv = torch.empty(n, dtype=torch.int32, device=dev)
             self._idx = torch.empty((n, self.k), dtype=torch.int32, device=dev)
 
+        if self.csa:
+            self._tk_ws = torch.empty(cache.index_topk_workspace_bytes(n, n_max) + 256, dtype=torch.uint8, device=dev)
+
         def select():
-            cache.index_scores(layer, self._req, d["q_idx"], d["w"], self._scores, self._nv, variant)
-            topk(self._scores, self._nv, self.k, self._idx, variant)
+            # index scores and top-k in one launch (csa_index_topk)
+            cache.index_topk(layer, self._req, d["q_idx"], d["w"], self._scores, self._nv, self.k, self._idx,
+                             variant, workspace=self._tk_ws)
 
         if self.csa:
             # one eager pass of the selection kernels (valid on any cache
@@ -382,3 +420,142 @@ def unpack_index_rows(rows: np.ndarray, d_I: int):
     codes[:, 0::2] = packed & 0xF
     codes[:, 1::2] = packed >> 4
     return codes, rows[:, d_I // 2:].copy()
+
+
+# ---------------------------------------------------------------- batch-invariant projection GEMM
+
+def bf16_bits(a) -> np.ndarray:
+    """BF16 bit patterns (uint16) of a host array (torch's round-to-nearest-even cast)."""
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(a, dtype=np.float32)))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+class Linear:
+    """A BF16 weight packed once for the batch-invariant projection GEMM
+    (csa_gemm_bf16): Y[t][o] = sum_k X[t][k] W[o][k], fp32 accumulation.
+
+    w: host array [n_out][k_in // groups] (BF16 bit patterns as uint16, or
+    real values, rounded to BF16 here).  With groups > 1 the weight is block
+    diagonal: group g's rows (n_out / groups, a multiple of 128) read the
+    columns [g k_in / groups, (g + 1) k_in / groups) of X."""
+
+    def __init__(self, w, groups: int = 1, device: str | torch.device = "cuda"):
+        self.lib = _lib.load()
+        w = np.ascontiguousarray(w)
+        if w.dtype != np.uint16:
+            w = bf16_bits(w)
+        self.n_out, kg = w.shape
+        self.groups = int(groups)
+        self.k_in = kg * self.groups
+        nbytes = self.lib.csa_gemm_weight_bytes(self.n_out, self.k_in, self.groups)
+        if nbytes == 0:
+            raise ValueError("invalid GEMM weight shape")
+        self.packed = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        check(self.lib.csa_gemm_pack_weight(w.ctypes.data, self.n_out, self.k_in, self.groups,
+                                            self.packed.data_ptr(), nbytes), "csa_gemm_pack_weight")
+        self._ws = None
+
+    def workspace_bytes(self, n_tok: int) -> int:
+        return int(self.lib.csa_gemm_workspace_bytes(self.n_out, self.k_in, self.groups, n_tok))
+
+    def __call__(self, x: torch.Tensor, outs, workspace: torch.Tensor | None = None, stream=None):
+        """x: CUDA BF16 [n_tok][k_in].  outs: one tensor or a list of CUDA
+        tensors [n_tok][rows_s] (BF16 or fp32, contiguous) whose rows add up
+        to n_out: rows [r_s, r_s + rows_s) of Y go to outs[s].  Returns outs."""
+        single = isinstance(outs, torch.Tensor)
+        segs = [outs] if single else list(outs)
+        n = x.shape[0] if x.dim() == 2 else -1
+        _need(x, torch.bfloat16, (n, self.k_in), "x")
+        arr = (_lib.GemmOut * len(segs))()
+        for s, t in enumerate(segs):
+            if t.dtype not in (torch.bfloat16, torch.float32):
+                raise ValueError("outputs must be BF16 or fp32")
+            _need(t, t.dtype, (n, t.shape[1] if t.dim() == 2 else -1), f"outs[{s}]")
+            arr[s] = _lib.GemmOut(t.shape[1], 1 if t.dtype == torch.bfloat16 else 0, t.data_ptr())
+        need = self.workspace_bytes(n) if n > 0 else 0
+        if workspace is None:
+            if self._ws is None or self._ws.numel() < need + 256 or self._ws.device != x.device:
+                self._ws = torch.empty(need + 256, dtype=torch.uint8, device=x.device)
+            workspace = self._ws
+        ws_ptr = (workspace.data_ptr() + 255) // 256 * 256
+        ws_bytes = workspace.numel() - (ws_ptr - workspace.data_ptr())
+        check(self.lib.csa_gemm_bf16(self.packed.data_ptr(), self.n_out, self.k_in, self.groups, _ptr(x), n,
+                                     len(segs), arr, ws_ptr, ws_bytes, _stream(stream)), "csa_gemm_bf16")
+        return outs
+
+    @staticmethod
+    def check_device_error(stream=None) -> None:
+        check(_lib.load().csa_gemm_check_device_error(_stream(stream)), "gemm device")
+
+
+class LayerProjections:
+    """The projections that feed one layer's decode step, from the token's
+    hidden state h (BF16 [n, d]) through the batch-invariant GEMM:
+
+      first call, one fused weight [W_c; W_z; (W_cI; W_zI; W_w;) W_dq]:
+        c, z [n, 1, D] fp32 (compressor candidate and gate logits),
+        on a CSA layer c_I, z_I [n, 1, d_I] and w [n, H_I] fp32,
+        c_q [n, d_c] BF16 (the query latent);
+      second call, [W_uq; (W_uqI)] on c_q:
+        q [n, H, D] BF16 (before RoPE), on a CSA layer q_I [n, H_I, d_I] fp32.
+
+    Weights are host arrays [out, in] (rounded to BF16 when packed)."""
+
+    def __init__(self, *, csa: bool, W_c, W_z, W_dq, W_uq, W_cI=None, W_zI=None, W_w=None, W_uqI=None,
+                 device: str | torch.device = "cuda"):
+        self.csa = bool(csa)
+        self.D = W_c.shape[0]
+        self.d = W_c.shape[1]
+        self.d_c = W_dq.shape[0]
+        first = [W_c, W_z] + ([W_cI, W_zI, W_w] if csa else []) + [W_dq]
+        self.rows1 = [int(w.shape[0]) for w in first]
+        self.W1 = Linear(np.concatenate([np.asarray(w, np.float32) for w in first]), device=device)
+        second = [W_uq] + ([W_uqI] if csa else [])
+        self.rows2 = [int(w.shape[0]) for w in second]
+        self.W2 = Linear(np.concatenate([np.asarray(w, np.float32) for w in second]), device=device)
+        self.d_I = int(W_cI.shape[0]) if csa else 0
+        self.H_I = int(W_w.shape[0]) if csa else 0
+        self.HD = int(W_uq.shape[0])
+
+    def new_outputs(self, n: int, H: int, device="cuda") -> dict:
+        f32, bf = torch.float32, torch.bfloat16
+        o = {"c": torch.empty((n, 1, self.D), dtype=f32, device=device),
+             "z": torch.empty((n, 1, self.D), dtype=f32, device=device),
+             "c_q": torch.empty((n, self.d_c), dtype=bf, device=device),
+             "q": torch.empty((n, H, self.HD // H), dtype=bf, device=device)}
+        if self.csa:
+            o.update(ci=torch.empty((n, 1, self.d_I), dtype=f32, device=device),
+                     zi=torch.empty((n, 1, self.d_I), dtype=f32, device=device),
+                     w=torch.empty((n, self.H_I), dtype=f32, device=device),
+                     q_idx=torch.empty((n, self.H_I, self.rows2[1] // self.H_I), dtype=f32, device=device))
+        return o
+
+    def __call__(self, h: torch.Tensor, outs: dict, stream=None) -> dict:
+        n = h.shape[0]
+        seg1 = [outs["c"].view(n, -1), outs["z"].view(n, -1)]
+        if self.csa:
+            seg1 += [outs["ci"].view(n, -1), outs["zi"].view(n, -1), outs["w"]]
+        seg1.append(outs["c_q"])
+        self.W1(h, seg1, stream=stream)
+        seg2 = [outs["q"].view(n, -1)] + ([outs["q_idx"].view(n, -1)] if self.csa else [])
+        self.W2(outs["c_q"], seg2, stream=stream)
+        return outs
+
+
+class OutputProjection:
+    """The grouped output projection after the attention: the H heads x D
+    output (BF16 [n, H, D]) is projected per group of H / groups heads by a
+    block-diagonal weight W_g [groups * d_g, (H / groups) * D] to a BF16
+    intermediate [n, groups * d_g], then to the model width by W_o
+    [d_model, groups * d_g] (fp32 output [n, d_model])."""
+
+    def __init__(self, W_g, W_o, groups: int, device: str | torch.device = "cuda"):
+        self.groups = int(groups)
+        self.Wg = Linear(W_g, groups=self.groups, device=device)
+        self.Wo = Linear(W_o, device=device)
+
+    def __call__(self, attn_out: torch.Tensor, mid: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+        n = attn_out.shape[0]
+        self.Wg(attn_out.view(n, -1), mid, stream=stream)
+        self.Wo(mid, out, stream=stream)
+        return out

@@ -59,9 +59,11 @@ namespace {
 constexpr int kAttThreads = 256;
 constexpr int kMaxLoads = 18;      // 16-byte loads per thread per tile (D <= 512)
 
+constexpr int kPgtCache = 4096;    // page-table entries of the query's request kept in shared memory
+
 struct AttnSmem {
   int Dp;             // head dim padded to a multiple of 128
-  int64_t tile, qs, pt, stage, rowf8, rowbf, rsc, stats, bars, total;
+  int64_t tile, qs, pt, stage, rowf8, rowbf, rsc, stats, pgt, bars, total;
 };
 
 __host__ __device__ inline AttnSmem attn_smem(int D, int G) {
@@ -76,6 +78,7 @@ __host__ __device__ inline AttnSmem attn_smem(int D, int G) {
   s.rowbf = o; o += (int64_t)kTileRows * 8;                  // row addresses (BF16 part)
   s.rsc = o;   o += (int64_t)kTileRows * 4;                  // row FP8 scales
   s.stats = o; o += (int64_t)12 * 32 * 4;
+  s.pgt = o;   o += (int64_t)kPgtCache * 4;                  // page table of the request (first entries)
   o = (o + 15) / 16 * 16;
   s.bars = o;  o += 64;
   s.total = o;
@@ -111,9 +114,12 @@ __device__ __forceinline__ float warp_reduce16(const float (&v)[16], int lane) {
   return op(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
 }
 
-// Address of row `r` of tile `tt`; returns whether the row exists.
+// Address of row `r` of tile `tt`; returns whether the row exists.  The
+// first n_pgt page-table entries of the request are read from `pgt`
+// (shared memory), the others from the arena.
 __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& g, int i, int tt, int r,
-                                            uint64_t* rowf8, uint64_t* rowbf, float* rsc) {
+                                            uint64_t* rowf8, uint64_t* rowbf, float* rsc, const int32_t* pgt,
+                                            int n_pgt) {
   const Layout& L = a.L;
   const int64_t rr = (int64_t)tt * kTileRows + r;
   const uint8_t* f8 = nullptr;
@@ -126,9 +132,13 @@ __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& 
       j = -1;
     }
     if (j >= 0) {
-      const float* scp;
-      L.entry_row(g.req, a.layer, j, &f8, &bf, &scp);
-      sc = *scp;
+      const int P = L.rows_per_page(a.layer);
+      const int64_t pi = j / P;
+      const int s = (int)(j % P);
+      const char* pp = L.page(pi < n_pgt ? pgt[pi] : L.page_table(g.req)[pi], a.layer);
+      f8 = reinterpret_cast<const uint8_t*>(pp) + (int64_t)s * L.kv_fp8_bytes;
+      bf = reinterpret_cast<const uint16_t*>(pp + (g.csa ? L.pg_csa_bf16 : L.pg_hca_bf16)) + (int64_t)s * L.R;
+      sc = reinterpret_cast<const float*>(pp + (g.csa ? L.pg_csa_scale : L.pg_hca_scale))[s];
     }
   } else if (rr < g.total) {
     const char* st = L.state(g.req, a.layer);
@@ -173,6 +183,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   float* cmul = beta + 32;
   float* den = cmul + 32;
   float* part = den + 32;                                // [4][32]
+  int32_t* pgt = reinterpret_cast<int32_t*>(sm + S.pgt);
   uint64_t* bar_qk = reinterpret_cast<uint64_t*>(sm + S.bars);
   uint64_t* bar_pv = bar_qk + 1;
   uint64_t* bar_drain = bar_qk + 2;
@@ -184,6 +195,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   const int tt0 = kSplit ? (int)blockIdx.x : 0;
   QueryGeom g;
   const bool reporter = tid == 0 && blockIdx.y == 0 && (!kSplit || blockIdx.x == 0);
+  // The kernel is launched with programmatic serialization: its CTAs may be
+  // resident before the previous grid on the stream (the top-k selection,
+  // or the append on an HCA layer) has finished.  Nothing it reads may be
+  // read before that grid is complete, so every thread waits here first.
+  tc::griddep_wait();
   if (!query_geom(a, i, g, reporter)) return;
   if (kSplit) {
     if (g.n_tiles > a.tiles_max) {
@@ -193,6 +209,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     if (tt0 >= g.n_tiles) return;
   }
   const int tt_end = kSplit ? tt0 + 1 : g.n_tiles;
+  const int64_t pages_needed = (g.n_entries + L.rows_per_page(a.layer) - 1) / L.rows_per_page(a.layer);
+  const int n_pgt = (int)(pages_needed < kPgtCache ? pages_needed : kPgtCache);
 
   // TMEM columns: S over the FP8 dims, S over the RoPE dims, the tile's
   // output accumulators (per 128-dim chunk one for the FP8 dims and, where
@@ -255,64 +273,46 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     }
   };
 
+  // The request's page-table entries and the query heads h0 .. h0+G-1 (in
+  // the K-major core-matrix order) go to shared memory by cp.async (no
+  // registers), issued first; warps 0-3 then resolve the first tile's row
+  // addresses while warps
+  // 4-7 tabulate cos / sin of the query position and clear the tile's padding
+  // dims.  All warps then gather the first tile in one round of loads, and
+  // the query's RoPE dims are rotated in place once its copies have landed.
+  {
+    // the request's page-table entries that hold its completed entries, one
+    // cp.async group (waited for before the rows are resolved)
+    const int32_t* ptg = L.page_table(g.req);
+    for (int x = tid; x < n_pgt; x += kAttThreads)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(pgt + x)), "l"(ptg + x) : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  {
+    const uint16_t* qg = static_cast<const uint16_t*>(a.q) + ((int64_t)i * H + h0) * D;
+    for (int x = tid; x < G * (Dp / 8); x += kAttThreads) {
+      const int hh = x / (Dp / 8), c = x % (Dp / 8);
+      uint8_t* dst = qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16;
+      if (h0 + hh < H && 8 * c < D)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(qg + (int64_t)hh * D + 8 * c)
+                     : "memory");
+      else
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  asm volatile("cp.async.wait_group 1;" ::: "memory");  // its page-table group has landed (the query's may not)
+  __syncthreads();
+  float2* cs = reinterpret_cast<float2*>(stage);
   int any = 0;
   if (warp < 4) {
-    any = resolve_row(a, g, i, tt0, tid, rowf8, rowbf, rsc) ? 1 : 0;
-    // the first tile's rows, gathered by warps 0-3 while warps 4-7 prepare
-    // the query: items warp, warp + 4, ... in two rounds of loads
-    tc::named_bar_sync(2, 128);
-#pragma unroll 1
-    for (int round = 0; round < 2; ++round) {
-      uint4 buf[kMaxLoads];
-#pragma unroll
-      for (int u = 0; u < kMaxLoads; ++u) {
-        const int it = warp + 4 * (round * kMaxLoads + u);
-        buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < kMaxLoads; ++u) {
-        const int it = warp + 4 * (round * kMaxLoads + u);
-        if (it < n_items) gather_store(it, buf[u]);
-      }
-    }
+    any = resolve_row(a, g, i, tt0, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
   } else {
-    // warps 4-7: the query heads h0 .. h0+G-1 rotated at t, BF16, K-major core order
     const int qt = tid - 128;
-    float2* cs = reinterpret_cast<float2*>(stage);
     for (int p = qt; p < R / 2; p += 128) {
       float c = 1.f, sn = 0.f;
       rope_pair(c, sn, L.theta()[p], g.t);       // rotating (1, 0) gives (cos, sin)
       cs[p] = make_float2(c, sn);
-    }
-    tc::named_bar_sync(1, 128);
-    // every load of this thread first (G * Dp / 8 <= 2048 chunks, 16 per thread)
-    constexpr int kQPer = 16;
-    uint4 raw[kQPer];
-#pragma unroll
-    for (int u = 0; u < kQPer; ++u) {
-      const int x = qt + 128 * u;
-      const int hh = x / (Dp / 8), c = x % (Dp / 8);
-      raw[u] = make_uint4(0, 0, 0, 0);
-      if (x < G * (Dp / 8) && h0 + hh < H && 8 * c < D)
-        raw[u] = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) + ((int64_t)i * H + h0 + hh) * D + 8 * c);
-    }
-#pragma unroll
-    for (int u = 0; u < kQPer; ++u) {
-      const int x = qt + 128 * u;
-      if (x >= G * (Dp / 8)) break;
-      const int hh = x / (Dp / 8), c = x % (Dp / 8);
-      uint4 o = raw[u];                               // non-RoPE dims: the BF16 input as is
-      if (8 * c >= dmain && 8 * c < D) {              // RoPE dims: rotate, round to BF16
-        const uint32_t rw[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-        uint32_t pk[4];
-        for (int e = 0; e < 8; e += 2) {
-          const float2 w = cs[(8 * c + e - dmain) / 2];
-          const float x0 = bf16_val((uint16_t)(rw[e >> 1] & 0xFFFFu)), x1 = bf16_val((uint16_t)(rw[e >> 1] >> 16));
-          pk[e >> 1] = (uint32_t)bf16_rn(x0 * w.x - x1 * w.y) | ((uint32_t)bf16_rn(x0 * w.y + x1 * w.x) << 16);
-        }
-        o = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      *reinterpret_cast<uint4*>(qs + (hh >> 3) * sbo_rows + c * 128 + (hh & 7) * 16) = o;
     }
     // padding dims [D, Dp) of the tile stay zero
     const int npad = (Dp - D) / 8;
@@ -322,6 +322,31 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     }
   }
   bool tile_valid = __syncthreads_count(any) > 0;
+  {   // the first tile: every warp, all its loads in flight at once
+    uint4 buf[kMaxLoads];
+#pragma unroll
+    for (int u = 0; u < kMaxLoads; ++u) {
+      const int it = warp + 8 * u;
+      buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kMaxLoads; ++u) {
+      const int it = warp + 8 * u;
+      if (it < n_items) gather_store(it, buf[u]);
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();                                      // every thread's query copies have landed
+  for (int x = tid; x < G * (R / 2); x += kAttThreads) {
+    // RoPE dims of the query: rotate the BF16 input at t, round to BF16
+    const int hh = x / (R / 2), p = x % (R / 2);
+    const int d = dmain + 2 * p;
+    uint32_t* wp = reinterpret_cast<uint32_t*>(qs + (hh >> 3) * sbo_rows + (d >> 3) * 128 + (hh & 7) * 16 + (d & 7) * 2);
+    const uint32_t v = *wp;
+    const float2 w = cs[p];
+    const float x0 = bf16_val((uint16_t)(v & 0xFFFFu)), x1 = bf16_val((uint16_t)(v >> 16));
+    *wp = (uint32_t)bf16_rn(x0 * w.x - x1 * w.y) | ((uint32_t)bf16_rn(x0 * w.y + x1 * w.x) << 16);
+  }
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -491,7 +516,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     // -- whole-query launch: addresses of the next tile's rows
     if (!kSplit && tt + 1 < tt_end) {
       int nany = 0;
-      if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc) ? 1 : 0;
+      if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
       tile_valid = __syncthreads_count(nany) > 0;
     }
   }
@@ -574,6 +599,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   } else if (!ok && tid == 0) {
     set_err(L, kErrTimeout, 3000000 + i);
   }
+  tc::griddep_launch_dependents();                      // the fold (or the next step) may start launching
   if (warp == 0) {   // no tcgen05 operation of this CTA is in flight when TMEM is released
     if (tc::elect_one()) tc::mma_commit(bar_drain);
     __syncwarp();
@@ -587,6 +613,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
 // Split launch, second step: fold the partials of (query blockIdx.y, head
 // blockIdx.x) in tile order; thread x owns dims 4x .. 4x+3.
 __global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
+  tc::griddep_wait();                                   // the partials are complete from here on
   const Layout& L = a.L;
   const int h = blockIdx.x, i = blockIdx.y, H = L.H, D = L.D;
   const int d4 = threadIdx.x;
@@ -638,8 +665,18 @@ __global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
 }
 
 cudaError_t launch_attn_fold(const AttnArgs& a, cudaStream_t st) {
-  attn_fold_kernel<<<dim3(a.L.H, a.n), (a.L.D / 4 + 31) / 32 * 32, 0, st>>>(a);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.L.H, a.n);
+  cfg.blockDim = dim3((a.L.D / 4 + 31) / 32 * 32);
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_fold_kernel, a);
   note_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -663,11 +700,24 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   const bool split = ws != nullptr;
   AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0, 0};
   const int n_hg = (L.H + G - 1) / G;
+  // programmatic dependent launch: the kernel may start before the previous
+  // grid on the stream ends and waits for it (griddepcontrol) where it must
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kAttThreads);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   if (!split) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<false><<<dim3(n, n_hg), kAttThreads, sm, st>>>(a);
+    cfg.gridDim = dim3(n, n_hg);
+    e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<false>, a);
     note_launch();
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
   a.tiles_max = attn_tiles_max(L, layer, k);
@@ -675,8 +725,10 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + (int64_t)n * a.tiles_max * L.H * L.D * 4);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  attn_tc_kernel<true><<<dim3(a.tiles_max, n_hg, n), kAttThreads, sm, st>>>(a);
+  cfg.gridDim = dim3(a.tiles_max, n_hg, n);
+  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, a);
   note_launch();
+  if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_attn_fold(a, st);

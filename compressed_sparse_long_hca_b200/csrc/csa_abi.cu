@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "csa.h"
+#include "gemm_out.cuh"
 #include "layout.cuh"
 
 namespace csa {
@@ -29,12 +30,25 @@ size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k);
 size_t attn_noalloc_scratch_bytes();
 cudaError_t attn_noalloc_scratch(void** out);
 cudaError_t launch_wait_probe(const Layout& L, uint64_t limit_ns, cudaStream_t st);
+size_t index_topk_workspace_bytes(int n, int64_t ld);
+cudaError_t launch_index_topk(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
+                              const float* w, float* scores, int64_t ld, int32_t* n_valid, int k, int32_t* idx_out,
+                              void* ws, int ctas, cudaStream_t st);
 cudaError_t launch_index_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                              const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas_per_query,
                              cudaStream_t st);
 cudaError_t launch_attn_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q,
                             const int32_t* topk, int k, const float* sink, float scale, float* out, void* ws,
                             cudaStream_t st);
+int gemm_row_tiles(int n_out);
+int gemm_k_tiles(int k_in, int groups);
+size_t gemm_weight_bytes(int n_out, int k_in, int groups);
+int gemm_max_tokens();
+size_t gemm_workspace_bytes(int n_out, int k_in, int groups, int n_tok, int sms);
+void gemm_pack_weight_host(const uint16_t* w, int n_out, int k_in, int groups, uint8_t* dst);
+cudaError_t launch_gemm_bf16(const void* w_packed, int n_out, int k_in, int groups, const uint16_t* x, int n_tok,
+                             const GemmOut& out, void* ws, int sms, cudaStream_t st);
+cudaError_t gemm_read_error(int32_t* code, int32_t* detail, cudaStream_t st);
 }  // namespace csa
 
 namespace {
@@ -318,6 +332,39 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
   return CSA_OK;
 }
 
+size_t csa_index_topk_workspace_bytes(const csa_cache_t* c, int32_t n, int64_t ld) {
+  if (!c || n < 1 || n > 65535 || ld < 1) return 0;
+  if (c->L.fmt == csa::kFmtF32) return 16;   // the fp32 format runs the two separate kernels
+  return csa::index_topk_workspace_bytes(n, ld);
+}
+
+csa_status csa_index_topk(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                          const float* q_idx, const float* w, float* scores, int64_t ld, int32_t* n_valid,
+                          int32_t k, int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                          csa_variant variant, csa_stream_t stream) {
+  if (!layer_ok(c, layer) || layer >= c->L.n_csa) return fail(CSA_ERR_ARG, "index scores need a CSA layer");
+  if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
+  if (n == 0) return CSA_OK;
+  if (!req_ids || !q_idx || !w || !scores || !n_valid || !idx_out) return fail(CSA_ERR_ARG, "NULL argument");
+  if (ld < 1 || k < 1) return fail(CSA_ERR_ARG, "k and ld must be >= 1");
+  if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
+  if (c->L.fmt == csa::kFmtF32) {   // fp32 keys: the CUDA-core indexer, then the top-k kernel
+    csa_status st = csa_index_scores(c, layer, n, req_ids, q_idx, w, scores, ld, n_valid, variant, stream);
+    if (st != CSA_OK) return st;
+    return csa_topk(scores, ld, n_valid, n, k, idx_out, variant, stream);
+  }
+  const size_t need = csa::index_topk_workspace_bytes(n, ld);
+  if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(CSA_ERR_ARG, "workspace must be 256-byte aligned and hold csa_index_topk_workspace_bytes");
+  const int sms = sm_count();
+  if (sms <= 0) return fail(CSA_ERR_CUDA, "cannot query the SM count");
+  // the same persistent grid for either variant (the selection is exact)
+  cudaError_t e = csa::launch_index_topk(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, k, idx_out,
+                                         workspace, 2 * sms, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fused index + top-k launch");
+  return CSA_OK;
+}
+
 size_t csa_attn_workspace_bytes(const csa_cache_t* c, int32_t layer, int32_t n, int32_t k) {
   if (!layer_ok(c, layer) || n < 0 || n > 65535) return 0;
   const bool is_csa = layer < c->L.n_csa;
@@ -404,17 +451,17 @@ csa_status csa_check_device_error(csa_cache_t* c, csa_stream_t stream) {
   if (!c) return fail(CSA_ERR_ARG, "cache is NULL");
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-  int32_t w[2] = {0, 0};
-  e = cudaMemcpy(w, c->L.err(), 8, cudaMemcpyDeviceToHost);
+  int32_t w[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(w, c->L.err(), 16, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
   if (w[0] == 0) return CSA_OK;
-  const int32_t zero[2] = {0, 0};
-  e = cudaMemcpy(c->L.err(), zero, 8, cudaMemcpyHostToDevice);
+  const int32_t zero[4] = {0, 0, 0, 0};
+  e = cudaMemcpy(c->L.err(), zero, 16, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word reset)");
   char msg[160];
   switch (w[0]) {
     case csa::kErrBounds:
-      snprintf(msg, sizeof msg, "device: index out of range (detail %d)", w[1]);
+      snprintf(msg, sizeof msg, "device: index out of range (detail %d; %d %d)", w[1], w[2], w[3]);
       return fail(CSA_ERR_DEVICE_BOUNDS, msg);
     case csa::kErrCapacity:
       snprintf(msg, sizeof msg, "device: append beyond the capacity of request %d", w[1]);
@@ -432,6 +479,91 @@ csa_status csa_check_device_error(csa_cache_t* c, csa_stream_t stream) {
 }
 
 const char* csa_last_error(void) { return g_err.c_str(); }
+
+// ---- batch-invariant projection GEMM
+
+static bool gemm_shape_ok(int32_t n_out, int32_t k_in, int32_t groups, std::string* why) {
+  if (n_out < 1 || k_in < 1 || groups < 1) { *why = "n_out, k_in and groups must be >= 1"; return false; }
+  if (n_out % groups || k_in % groups) { *why = "groups must divide n_out and k_in"; return false; }
+  if (groups > 1 && (n_out / groups) % 128) { *why = "a grouped weight needs a multiple of 128 rows per group"; return false; }
+  if ((k_in / groups) % 8) { *why = "k_in / groups must be a multiple of 8"; return false; }
+  return true;
+}
+
+size_t csa_gemm_weight_bytes(int32_t n_out, int32_t k_in, int32_t groups) {
+  std::string why;
+  if (!gemm_shape_ok(n_out, k_in, groups, &why)) return 0;
+  return csa::gemm_weight_bytes(n_out, k_in, groups);
+}
+
+csa_status csa_gemm_pack_weight(const uint16_t* w_host, int32_t n_out, int32_t k_in, int32_t groups, void* w_dev,
+                                size_t bytes) {
+  std::string why;
+  if (!gemm_shape_ok(n_out, k_in, groups, &why)) return fail(CSA_ERR_ARG, why);
+  if (!w_host || !w_dev || reinterpret_cast<uintptr_t>(w_dev) % 16) return fail(CSA_ERR_ARG, "NULL or unaligned pointer");
+  const size_t need = csa::gemm_weight_bytes(n_out, k_in, groups);
+  if (bytes < need) return fail(CSA_ERR_CAPACITY, "w_dev smaller than csa_gemm_weight_bytes");
+  std::vector<uint8_t> tiles;
+  try {
+    tiles.resize(need);
+  } catch (...) {
+    return fail(CSA_ERR_CAPACITY, "host allocation failed");
+  }
+  csa::gemm_pack_weight_host(w_host, n_out, k_in, groups, tiles.data());
+  cudaError_t e = cudaMemcpy(w_dev, tiles.data(), need, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(packed weight)");
+  return CSA_OK;
+}
+
+size_t csa_gemm_workspace_bytes(int32_t n_out, int32_t k_in, int32_t groups, int32_t n_tok) {
+  std::string why;
+  if (!gemm_shape_ok(n_out, k_in, groups, &why) || n_tok < 1 || n_tok > csa::gemm_max_tokens()) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return csa::gemm_workspace_bytes(n_out, k_in, groups, n_tok, sms);
+}
+
+csa_status csa_gemm_bf16(const void* w_packed, int32_t n_out, int32_t k_in, int32_t groups, const uint16_t* x,
+                         int32_t n_tok, int32_t n_seg, const csa_gemm_out* segs, void* workspace,
+                         size_t workspace_bytes, csa_stream_t stream) {
+  std::string why;
+  if (!gemm_shape_ok(n_out, k_in, groups, &why)) return fail(CSA_ERR_ARG, why);
+  if (n_tok < 0 || n_tok > csa::gemm_max_tokens()) return fail(CSA_ERR_ARG, "n_tok must be in [0, 256]");
+  if (n_seg < 1 || n_seg > csa::kGemmMaxSeg || !segs) return fail(CSA_ERR_ARG, "n_seg must be in [1, 8]");
+  csa::GemmOut out{};
+  out.n_seg = n_seg;
+  int rows = 0;
+  for (int s = 0; s < n_seg; ++s) {
+    if (segs[s].rows < 1 || !segs[s].y) return fail(CSA_ERR_ARG, "every output segment needs rows >= 1 and y");
+    rows += segs[s].rows;
+    out.seg_end[s] = rows;
+    out.y[s] = segs[s].y;
+    if (segs[s].bf16) out.bf16_mask |= 1u << s;
+  }
+  if (rows != n_out) return fail(CSA_ERR_ARG, "the segments' rows must add up to n_out");
+  if (n_tok == 0) return CSA_OK;
+  if (!w_packed || !x || !workspace) return fail(CSA_ERR_ARG, "NULL argument");
+  if (reinterpret_cast<uintptr_t>(w_packed) % 16 || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(CSA_ERR_ARG, "w_packed must be 16-byte and workspace 256-byte aligned");
+  const int sms = sm_count();
+  if (sms <= 0) return fail(CSA_ERR_CUDA, "cannot query the SM count");
+  if (workspace_bytes < csa::gemm_workspace_bytes(n_out, k_in, groups, n_tok, sms))
+    return fail(CSA_ERR_ARG, "workspace smaller than csa_gemm_workspace_bytes");
+  cudaError_t e = csa::launch_gemm_bf16(w_packed, n_out, k_in, groups, x, n_tok, out, workspace, sms,
+                                        (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return CSA_OK;
+}
+
+csa_status csa_gemm_check_device_error(csa_stream_t stream) {
+  int32_t code = 0, detail = 0;
+  cudaError_t e = csa::gemm_read_error(&code, &detail, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm error word");
+  if (code == 0) return CSA_OK;
+  char msg[120];
+  snprintf(msg, sizeof msg, "device: a GEMM pipeline wait gave up (row tile %d)", detail);
+  return fail(CSA_ERR_DEVICE_TIMEOUT, msg);
+}
 
 csa_status csa_debug_wait_timeout(csa_cache_t* c, int32_t limit_us, csa_stream_t stream) {
   if (!c) return fail(CSA_ERR_ARG, "cache is NULL");

@@ -42,7 +42,6 @@ constexpr int kEpiGroups = 2;          // epilogue groups, alternate tiles
 constexpr int kGroupThreads = 128;     // one thread per key of a tile
 constexpr int kEpiThreads = kEpiGroups * kGroupThreads;
 constexpr int kThreads = 64 + kEpiThreads;   // warp 0 producer, warp 1 MMA, warps 2-9 epilogue
-constexpr int kCtasPerSm = 2;          // two CTAs per SM overlap their issue latencies
 constexpr int kHeadsN = 64;            // MMA N (index heads, zero padded)
 constexpr int kMaxCh = 4;              // d_I / 32 <= 4
 constexpr int kTileBytes = kCsaPerPage * kMaxCh * 16 + kSfChunk;   // codes + scale chunk
@@ -52,9 +51,20 @@ constexpr int kMaxQ = 256;             // queries whose tile counts are kept in 
 constexpr uint32_t kTmemCols = 256;    // per CTA; two CTAs fill the SM's 512 columns
 constexpr uint32_t kSfaCol = 192;      // + 4 * accumulator index
 constexpr uint32_t kSfbCol = 204;
+// fused top-k (csa_index_topk)
+constexpr int kHistBits = 12;          // histogram of the score keys' top 12 bits
+constexpr int kHistBins = 1 << kHistBits;
+constexpr int kHistShift = 32 - kHistBits;
+constexpr int kCandCap = 8192;         // candidates the selecting CTA holds
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr int kScoreCache = 24576;     // scores of the CTA's own range kept in shared memory (fused top-k)
+constexpr int kBitmapKeys = kScoreCache / 2 * 32;   // keys the selection's two bitmaps cover (same region)
 
 struct IdxSmem {
-  uint8_t tiles[kStages][kTileBytes];                // one page's index tile per stage
+  union {
+    uint8_t tiles[kStages][kTileBytes];              // one page's index tile per stage
+    uint2 cand[kCandCap];                            // top-k: (key, index) of a query's candidates, index order
+  } u;
   uint8_t qb[kHeadsN * kMaxCh * 16];                 // query codes, core-matrix order
   uint8_t qsf[kSfChunk];                             // query scales, tcgen05.cp order
   alignas(16) float w[kHeadsN];
@@ -74,6 +84,15 @@ struct IdxSmem {
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort;
+  // fused top-k
+  uint32_t hist[kHistBins];                          // score-key histogram of the current segment
+  int32_t wt[2][kThreads / 32];                      // warp totals of block scans (alternating)
+  int32_t tk_q, tk_t0, tk_nt, tk_flag, tk_bin, tk_above, tk_M, tk_rem;
+  int64_t tk_N, tk_before;
+  uint32_t tk_digit;
+  int32_t n_pend;                                    // selections this CTA owes (it was a query's last CTA)
+  int32_t pend_q[64];
+  int64_t pend_N[64];
 };
 
 struct IndexTcArgs {
@@ -86,6 +105,15 @@ struct IndexTcArgs {
   float* scores;
   int64_t ld;
   int32_t* n_valid;
+  // fused top-k only
+  int k;
+  int32_t* idx_out;       // [n][k]
+  int32_t* hist_done;     // [n]  CTAs whose histogram of the query is flushed
+  int32_t* cand_done;     // [n]  CTAs whose candidates of the query are written
+  uint32_t* hist;         // [n][kHistBins]  the query's keys over their top 12 bits
+  uint32_t* hist2;        // [n][2048]       candidates in the k-th bin over key bits 9 .. 19
+  int32_t* qcount;        // [n]             candidates appended so far
+  uint2* cand;            // [n][ld]         candidates (key, index), in no particular order
 };
 
 // Number of 128-key tiles of query i (0 for an invalid query); N = its keys.
@@ -112,9 +140,556 @@ __device__ __forceinline__ bool wait_or_abort(IdxSmem& sm, uint64_t* bar, uint32
   }
 }
 
+
+// ---------------------------------------------------------------- fused top-k
+//
+// Selection rule (as csa_topk): the k largest scores, equal scores to the
+// lower index, -0.0 == +0.0, output ascending, -1 padding.  Scores become
+// order-preserving 32-bit keys; the kernel's CTAs build a histogram of each
+// query's keys over their top 12 bits while they score, wait (bounded) until
+// every CTA of the query has flushed its part, find the bin b holding the
+// k-th largest key, and write the keys of their own range with top bits >= b
+// (the candidates) compactly, in index order, into the window of the
+// candidate buffer that starts at their range's first key.  The last CTA to
+// finish a query gathers the windows in order and selects exactly; when more
+// than kCandCap keys fall in bins >= b (a huge tie class), it selects with a
+// radix select over the query's whole score row instead.  Both are exact, so
+// the indices equal csa_topk's.
+
+__device__ __forceinline__ uint32_t score_key(float s) {
+  const uint32_t b = __float_as_uint(s + 0.0f);       // -0.0 -> +0.0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// CTA that owns flattened tile g when `total` tiles are split over G CTAs as
+// [total * c / G, total * (c + 1) / G).
+__device__ __forceinline__ int owner_cta(int64_t g, int64_t total, int G) {
+  return (int)(((g + 1) * (int64_t)G - 1) / total);
+}
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Exclusive prefix sum over the CTA's threads in thread order; one barrier.
+// `wt` must not be reused before another barrier.
+__device__ __forceinline__ int cta_scan(int v, int32_t* wt, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wt[w] = x;
+  __syncthreads();
+  const int tw = lane < kThreads / 32 ? wt[lane] : 0;
+  *total = __reduce_add_sync(0xffffffffu, tw);
+  return __reduce_add_sync(0xffffffffu, lane < w ? tw : 0) + x - v;
+}
+
+// Among `nbins` counts (thread t < 256 owns bins nbins-PER*(t+1) .. nbins-PER*t-1,
+// highest first), find the bin d holding the r-th largest key: (count in bins
+// > d) < r <= (count in bins >= d).  Publishes d in sm.tk_digit, the count
+// above it in sm.tk_above and the count at or above it in sm.tk_M; returns
+// false when fewer than r keys are counted.  Two barriers.
+template <int PER>
+__device__ bool find_bin(const uint32_t* bins, int r, IdxSmem& sm) {
+  const int tid = threadIdx.x;
+  int c[PER];
+  int sum = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    const int b = 256 * PER - 1 - (PER * tid + e);     // descending
+    c[e] = tid < 256 ? (int)bins[b] : 0;
+    sum += c[e];
+  }
+  if (tid == 0) sm.tk_flag = 0;
+  int tot;
+  const int before = cta_scan(sum, sm.wt[0], &tot);
+  if (tid < 256 && before < r && before + sum >= r) {
+    int cum = before;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      if (cum < r && cum + c[e] >= r) {
+        sm.tk_digit = (uint32_t)(256 * PER - 1 - (PER * tid + e));
+        sm.tk_above = cum;
+        sm.tk_M = cum + c[e];
+        sm.tk_flag = 1;
+      }
+      cum += c[e];
+    }
+  }
+  __syncthreads();
+  return sm.tk_flag != 0;
+}
+
+// find_bin over the 256 PER counts of a global histogram: thread t < 256
+// loads its PER bins (256 PER - PER(t+1) .. 256 PER - PER t - 1) with PER / 4
+// vector loads, all in flight at once.
+template <int PER>
+__device__ bool find_bin_global(const uint32_t* gbins, int r, IdxSmem& sm) {
+  const int tid = threadIdx.x;
+  int c[PER];
+  int sum = 0;
+  if (tid < 256) {
+    const uint4* src = reinterpret_cast<const uint4*>(gbins + 256 * PER - PER * (tid + 1));
+    uint32_t v[PER];
+#pragma unroll
+    for (int x = 0; x < PER / 4; ++x) {
+      const uint4 w = __ldcg(src + x);
+      v[4 * x] = w.x; v[4 * x + 1] = w.y; v[4 * x + 2] = w.z; v[4 * x + 3] = w.w;
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) { c[e] = (int)v[PER - 1 - e]; sum += c[e]; }   // descending bins
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) c[e] = 0;
+  }
+  if (tid == 0) sm.tk_flag = 0;
+  int tot;
+  const int before = cta_scan(sum, sm.wt[0], &tot);
+  if (tid < 256 && before < r && before + sum >= r) {
+    int cum = before;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      if (cum < r && cum + c[e] >= r) {
+        sm.tk_digit = (uint32_t)(256 * PER - 1 - (PER * tid + e));
+        sm.tk_above = cum;
+        sm.tk_M = cum + c[e];
+        sm.tk_flag = 1;
+      }
+      cum += c[e];
+    }
+  }
+  __syncthreads();
+  return sm.tk_flag != 0;
+}
+
+// Histogram of the digit (key >> shift) & (2^bits - 1) over the keys whose
+// higher bits (key >> (shift + bits)) equal `prefix`, into sm.hist[0 .. 2^bits);
+// then find the bin of the r-th largest.  `keys(x)` yields key x of `count`.
+template <int BITS, typename F>
+__device__ bool digit_round(F keys, int64_t count, uint32_t prefix, int shift, int r, IdxSmem& sm) {
+  for (int b = threadIdx.x; b < (1 << BITS); b += kThreads) sm.hist[b] = 0;
+  __syncthreads();
+  for (int64_t x = threadIdx.x; x < count; x += kThreads) {
+    const uint32_t key = keys(x);
+    if ((key >> (shift + BITS)) == prefix) atomicAdd(&sm.hist[(key >> shift) & ((1u << BITS) - 1)], 1u);
+  }
+  __syncthreads();
+  return find_bin<(1 << BITS) / 256>(sm.hist, r, sm);
+}
+
+// The k-th largest key among `count` keys whose top 12 bits are >= `bin`,
+// given `above` keys with top bits > bin: returns T and sets *ties = the
+// number of keys == T that are selected.
+template <typename F>
+__device__ uint32_t exact_kth(F keys, int64_t count, uint32_t bin, int above, int k, IdxSmem& sm, int* ties,
+                              bool* ok) {
+  int r = k - above;
+  *ok = digit_round<11>(keys, count, bin, 9, r, sm);           // bits 9 .. 19
+  const uint32_t dA = sm.tk_digit;
+  r -= sm.tk_above;
+  const bool okB = digit_round<9>(keys, count, (bin << 11) | dA, 0, r, sm);   // bits 0 .. 8
+  *ok = *ok && okB;
+  const uint32_t dB = sm.tk_digit;
+  *ties = r - sm.tk_above;
+  __syncthreads();
+  return (bin << 20) | (dA << 9) | dB;
+}
+
+
+// Add this CTA's histogram of query q's keys to the query's global histogram
+// and clear it (epilogue thread et owns bins 16 et .. 16 et + 15).
+__device__ __forceinline__ void flush_hist(const IndexTcArgs& a, IdxSmem& sm, int q, int et) {
+  uint32_t* g = a.hist + (int64_t)q * kHistBins;
+#pragma unroll
+  for (int e = 0; e < kHistBins / kEpiThreads; ++e) {
+    const int b = et * (kHistBins / kEpiThreads) + e;
+    const uint32_t v = sm.hist[b];
+    if (v) {
+      atomicAdd(&g[b], v);
+      sm.hist[b] = 0;
+    }
+  }
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Inclusive prefix sum over the lanes of a warp.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// A shared-memory bitmap of nw words read in chunks of 32 consecutive words
+// (lane l of chunk c reads word 32 c + l, one word per bank), warp w owning
+// chunks [c0, c1) in order.  Returns the number of set bits in the chunks of
+// the warps before this one.  Two barriers; uses sm.wt[1].
+__device__ __forceinline__ int bitmap_warp_base(const uint32_t* bm, int nw, int c0, int c1, IdxSmem& sm) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int cnt = 0;
+  for (int c = c0; c < c1; ++c) {
+    const int x = c * 32 + lane;
+    cnt += x < nw ? __popc(bm[x]) : 0;
+  }
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) sm.wt[1][w] = cnt;
+  __syncthreads();
+  const int tw = lane < kThreads / 32 ? sm.wt[1][lane] : 0;
+  const int base = __reduce_add_sync(0xffffffffu, lane < w ? tw : 0);
+  __syncthreads();
+  return base;
+}
+
+// Write the selected indices of `count` keys (key(x), index(x) in index
+// order): every key > T and the first `ties` keys == T, ascending.
+template <typename FK, typename FI>
+__device__ void write_selection(FK key, FI index, int64_t count, uint32_t T, int ties, int32_t* out, IdxSmem& sm,
+                                const Layout& L, int req, int layer) {
+  const int tid = threadIdx.x;
+  const int64_t per = (count + kThreads - 1) / kThreads;
+  const int64_t e0 = tid * per, e1 = e0 + per < count ? e0 + per : count;
+  int ngt = 0, neq = 0;
+  for (int64_t x = e0; x < e1; ++x) {
+    const uint32_t v = key(x);
+    ngt += v > T ? 1 : 0;
+    neq += v == T ? 1 : 0;
+  }
+  int tot;
+  const int gt_before = cta_scan(ngt, sm.wt[0], &tot);
+  const int eq_before = cta_scan(neq, sm.wt[1], &tot);
+  int p = gt_before + (eq_before < ties ? eq_before : ties);
+  int seen = eq_before;
+  for (int64_t x = e0; x < e1; ++x) {
+    const uint32_t v = key(x);
+    const bool eq = v == T;
+    if (v > T || (eq && seen < ties)) out[p++] = index(x);
+    seen += eq ? 1 : 0;
+  }
+  __syncthreads();
+}
+
+// The query's raw-token window ring into L2 (the attention's last rows).
+__device__ __forceinline__ void prefetch_window(const Layout& L, int req, int layer) {
+  const char* st = L.state(req, layer);
+  for (int64_t o = threadIdx.x * 128; o < L.ring_bytes; o += (int64_t)kThreads * 128) prefetch_l2(st + o);
+}
+
+// The top-k part of csa_index_topk, by every thread of a CTA that scored the
+// tiles [g0, g1) of the flattened (query, tile) list (its histograms flushed).
+// The selection of query q by its last CTA (every CTA of q has flushed its
+// histogram and appended its candidates): indices ascending into idx_out.
+__device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N) {
+  const Layout& L = a.L;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __threadfence();
+  int32_t* out = a.idx_out + (int64_t)q * a.k;
+  const int req = a.req_ids[q];
+  const float* row = a.scores + (int64_t)q * a.ld;
+  const uint2* cq = a.cand + (int64_t)q * a.ld;
+  prefetch_window(L, req, a.layer);
+  if (N <= a.k) {                               // every entry is selected
+    for (int j = tid; j < a.k; j += kThreads) out[j] = j < N ? j : -1;
+    __syncthreads();
+    return;
+  }
+  // the k-th bin, as every CTA of q found it, from the complete histogram
+  if (!find_bin_global<kHistBins / 256>(a.hist + (int64_t)q * kHistBins, a.k, sm)) {
+    if (tid == 0) set_err(L, kErrBounds, 7300000 + q);
+    return;
+  }
+  const uint32_t bin = sm.tk_digit;
+  const int above = sm.tk_above, M = sm.tk_M;
+  __syncthreads();
+    if (M <= kCandCap && N <= kBitmapKeys) {
+      // first digit of the k-th key (bits 9 .. 19) from the candidates' hist2
+      const int r1 = a.k - above;
+      bool ok = find_bin_global<8>(a.hist2 + (int64_t)q * 2048, r1, sm);
+      const uint32_t dA = sm.tk_digit;
+      const int r2 = r1 - sm.tk_above;
+      const int Mtot = __ldcg(a.qcount + q);
+      __syncthreads();
+      if (!ok || Mtot != M) {                   // cannot happen unless a CTA skipped its part
+        if (tid == 0) {
+          int32_t* e = L.err();
+          if (atomicCAS(e, 0, (int32_t)kErrBounds) == 0) {
+            e[1] = 7000000 + q;
+            e[2] = M;
+            e[3] = Mtot | (ok ? 0 : (1 << 30));
+          }
+        }
+        return;
+      }
+      // the candidates to shared memory (no order needed), all loads in flight
+      constexpr int kB = 8;
+      for (int m0 = 0; m0 < Mtot; m0 += kThreads * kB) {
+        uint2 v[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int m = m0 + u * kThreads + tid;
+          v[u] = m < Mtot ? __ldcg(cq + m) : make_uint2(0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int m = m0 + u * kThreads + tid;
+          if (m < Mtot) sm.u.cand[m] = v[u];
+        }
+      }
+      __syncthreads();
+      // last digit (bits 0 .. 8) among the candidates that share T's upper 23 bits
+      const uint32_t pre = (bin << 11) | dA;
+      ok = digit_round<9>([&](int64_t x) { return sm.u.cand[x].x; }, Mtot, pre, 0, r2, sm);
+      const uint32_t T = (pre << 9) | sm.tk_digit;
+      const int ties = r2 - sm.tk_above;        // keys == T to take, lowest indices first
+      const int n_eq = sm.tk_M - sm.tk_above;   // keys == T among the candidates
+      __syncthreads();
+      if (!ok) {
+        if (tid == 0) set_err(L, kErrBounds, 7100000 + q);
+        return;
+      }
+      // bitmaps over the query's N keys: selected and (when only some of the
+      // keys == T are taken) the tied ones
+      uint32_t* mb = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(&sm) + (sizeof(IdxSmem) + 127) / 128 * 128);
+      uint32_t* tb = mb + kBitmapKeys / 32;
+      const int nw = (int)((N + 31) / 32);
+      const bool all_ties = ties == n_eq;       // the usual case: every key == T is taken
+      for (int x = tid; x < nw; x += kThreads) {
+        mb[x] = 0;
+        if (!all_ties) tb[x] = 0;
+      }
+      __syncthreads();
+      for (int m = tid; m < Mtot; m += kThreads) {
+        const uint2 c = sm.u.cand[m];
+        if (c.x > T || (all_ties && c.x == T)) atomicOr(mb + (c.y >> 5), 1u << (c.y & 31));
+        else if (c.x == T) atomicOr(tb + (c.y >> 5), 1u << (c.y & 31));
+      }
+      __syncthreads();
+      const int nc = (nw + 31) / 32;            // chunks of 32 words, lane l reads word 32 c + l
+      const int cpw = (nc + kThreads / 32 - 1) / (kThreads / 32);
+      const int c0 = min(warp * cpw, nc), c1 = min(c0 + cpw, nc);
+      if (!all_ties) {
+        // the `ties` lowest tied indices join the selection
+        int base = bitmap_warp_base(tb, nw, c0, c1, sm);
+        for (int c = c0; c < c1; ++c) {
+          const int x = c * 32 + lane;
+          uint32_t t = x < nw ? tb[x] : 0u;
+          const int n = __popc(t);
+          const int incl = warp_incl_scan(n, lane);
+          const int before = base + incl - n;
+          if (before >= ties) {
+            t = 0;
+          } else if (before + n > ties) {       // keep the lowest (ties - before) bits
+            uint32_t keep = 0;
+            for (int j = ties - before; j > 0; --j) {
+              keep |= t & (0u - t);
+              t &= t - 1;
+            }
+            t = keep;
+          }
+          if (x < nw) mb[x] |= t;
+          base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        __syncthreads();
+      }
+      // every selected index, ascending
+      int p = bitmap_warp_base(mb, nw, c0, c1, sm);
+      for (int c = c0; c < c1; ++c) {
+        const int x = c * 32 + lane;
+        uint32_t b = x < nw ? mb[x] : 0u;
+        const int n = __popc(b);
+        const int incl = warp_incl_scan(n, lane);
+        int o = p + incl - n;
+        while (b) {
+          out[o++] = x * 32 + (__ffs(b) - 1);
+          b &= b - 1;
+        }
+        p += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      __syncthreads();
+    } else {
+      // more keys than kCandCap at or above the bin (a huge tie class):
+      // radix select over the whole score row
+      int ties;
+      bool ok;
+      auto rk = [&](int64_t x) { return score_key(__ldcg(row + x)); };
+      const uint32_t T = exact_kth(rk, N, bin, above, a.k, sm, &ties, &ok);
+      if (!ok) {
+        if (tid == 0) set_err(L, kErrBounds, 7200000 + q);
+        return;
+      }
+      write_selection(rk, [&](int64_t x) { return (int32_t)x; }, N, T, ties, out, sm, L, req, a.layer);
+    }
+}
+
+__device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int64_t g0, int64_t g1,
+                           const float* sc_cache) {
+  const Layout& L = a.L;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int G = gridDim.x;
+  tc::griddep_launch_dependents();    // the next kernel may start launching while the selection runs
+  if (tid == 0) sm.n_pend = 0;
+  __threadfence();
+  __syncthreads();
+  // thread 0 walks the queries whose tiles overlap [g0, g1)
+  int walk_q = 0;
+  int64_t walk_before = 0;
+  auto next_covered = [&](int& q, int64_t& before, int& nt, int64_t& N) {
+    q = -1;
+    while (walk_q < a.n && walk_before < g1) {
+      int64_t n_keys;
+      int req;
+      const int64_t t = walk_q < kMaxQ ? sm.q_tiles[walk_q] : query_tiles(a, walk_q, &n_keys, &req);
+      if (walk_q < kMaxQ) n_keys = sm.q_N[walk_q];
+      const int64_t b0 = walk_before;
+      walk_before += t;
+      const int qq = walk_q++;
+      if (t > 0 && b0 + t > g0) {
+        q = qq; before = b0; nt = (int)t; N = n_keys;
+        return;
+      }
+    }
+  };
+  // 1. arrive on every covered query's histogram counter
+  if (tid == 0) {
+    int q, nt;
+    int64_t before, N;
+    for (next_covered(q, before, nt, N); q >= 0; next_covered(q, before, nt, N)) atomicAdd(&a.hist_done[q], 1);
+    walk_q = 0;
+    walk_before = 0;
+  }
+  // 2. per covered query: threshold, candidates, and the selection by the last CTA
+  for (;;) {
+    if (tid == 0) {
+      int q, nt;
+      int64_t before, N;
+      next_covered(q, before, nt, N);
+      sm.tk_q = q;
+      sm.tk_before = before;
+      sm.tk_nt = nt;
+      sm.tk_N = N;
+    }
+    __syncthreads();
+    const int q = sm.tk_q;
+    if (q < 0) break;
+    const int64_t before = sm.tk_before, N = sm.tk_N;
+    const int nt_q = sm.tk_nt;
+    // the CTAs holding tiles of q: owners of its first and last tile and every
+    // non-empty CTA between them (a CTA whose share rounds to no tile takes no part)
+    const int c_first = owner_cta(before, total, G), c_last = owner_cta(before + nt_q - 1, total, G);
+    int n_ctas;
+    {
+      const int c = c_first + tid;
+      const int64_t gs = total * c / G, ge = total * (c + 1) / G;
+      const bool holds = c <= c_last && gs < ge;
+      (void)cta_scan(holds ? 1 : 0, sm.wt[0], &n_ctas);
+      __syncthreads();
+    }
+    const int64_t lo_t = (g0 > before ? g0 : before) - before;
+    const int64_t hi_t = (g1 < before + nt_q ? g1 : before + nt_q) - before;
+    const bool all = N <= a.k;                 // every entry is selected
+    const float* row = a.scores + (int64_t)q * a.ld;
+    uint2* cq = a.cand + (int64_t)q * a.ld;
+    bool fine = true;
+    uint32_t bin = 0;
+    int M = 0;
+    if (!all) {
+      if (tid == 0) {
+        bool ok = ld_acquire(&a.hist_done[q]) >= n_ctas;
+        if (!ok) {
+          const uint64_t t0 = tc::globaltimer_ns();
+          while (!(ok = ld_acquire(&a.hist_done[q]) >= n_ctas) && tc::globaltimer_ns() - t0 < kWaitLimitNs)
+            __nanosleep(100);
+        }
+        if (!ok) set_err(L, kErrTimeout, 6000000 + q);
+        sm.tk_flag = ok ? 1 : 0;
+      }
+      __syncthreads();
+      fine = sm.tk_flag != 0;
+      __syncthreads();
+      if (fine) {
+        fine = find_bin_global<kHistBins / 256>(a.hist + (int64_t)q * kHistBins, a.k, sm);
+        bin = sm.tk_digit;
+        M = sm.tk_M;
+        __syncthreads();
+      }
+      if (fine && M <= kCandCap) {
+        // this CTA's keys of q with top bits >= bin (the candidates) are
+        // appended to the query's candidate array (warp-aggregated atomics,
+        // in no particular order); those in the k-th bin are also counted
+        // over key bits 9 .. 19 for the selection's first digit
+        const int64_t j_lo = lo_t * kCsaPerPage, j_hi = hi_t * kCsaPerPage < N ? hi_t * kCsaPerPage : N;
+        const int warp = tid >> 5;
+        const unsigned lt = (1u << lane) - 1u;
+        constexpr int kB = 8;                   // keys per lane in flight
+        // the CTA's own scores of q: in the shared-memory cache (local index of
+        // key j = (first local tile of q) * 128 + j - j_lo) or, past it, in L2
+        const float* cache = sc_cache != nullptr ? sc_cache + ((before + lo_t - g0) * kCsaPerPage - j_lo) : nullptr;
+        uint32_t* h2 = a.hist2 + (int64_t)q * 2048;
+        for (int64_t base = j_lo + (int64_t)warp * 32 * kB; base < j_hi; base += (int64_t)(kThreads / 32) * 32 * kB) {
+          float v[kB];
+#pragma unroll
+          for (int u = 0; u < kB; ++u) {
+            const int64_t j = base + u * 32 + lane;
+            v[u] = j < j_hi ? (cache != nullptr ? cache[j] : __ldcg(row + j)) : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < kB; ++u) {
+            const int64_t j = base + u * 32 + lane;
+            const uint32_t key = score_key(v[u]);
+            const bool pass = j < j_hi && (key >> kHistShift) >= bin;
+            const unsigned bal = __ballot_sync(0xffffffffu, pass);
+            if (bal == 0) continue;
+            int off = 0;
+            if (lane == 0) off = atomicAdd(a.qcount + q, __popc(bal));
+            off = __shfl_sync(0xffffffffu, off, 0);
+            if (pass) {
+              cq[off + __popc(bal & lt)] = make_uint2(key, (uint32_t)j);
+              if ((key >> kHistShift) == bin) atomicAdd(h2 + ((key >> 9) & 2047u), 1u);
+            }
+          }
+        }
+      }
+    }
+    // arrive; the last CTA of the query owes its selection, which runs
+    // after all this CTA's filters (the selection's bitmaps share shared
+    // memory with the score cache the filters read)
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sm.tk_flag = atomicAdd(&a.cand_done[q], 1) == n_ctas - 1 ? 1 : 0;
+    __syncthreads();
+    const bool last = sm.tk_flag != 0;
+    __syncthreads();
+    if (!last) continue;
+    if (sm.n_pend < 64) {
+      if (tid == 0) {
+        sm.pend_q[sm.n_pend] = q;
+        sm.pend_N[sm.n_pend] = N;
+        sm.n_pend = sm.n_pend + 1;
+      }
+      __syncthreads();
+      continue;
+    }
+    select_query(a, sm, q, N);                  // the list is full: select now ...
+    sc_cache = nullptr;                         // ... and read later scores from L2
+  }
+  // 3. the selections this CTA owes
+  for (int x = 0; x < sm.n_pend; ++x) select_query(a, sm, sm.pend_q[x], sm.pend_N[x]);
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcArgs a) {
+template <bool kTopk>
+__global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const Layout& L = a.L;
@@ -151,11 +726,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
       if (i < kMaxQ) { sm.q_tiles[i] = (int32_t)nt; sm.q_N[i] = N; }
       part += nt;
       if (blockIdx.x == 0) {
+        // a query without tiles takes no part in the fused selection: its row is all -1
+        if (kTopk && nt == 0)
+          for (int j = 0; j < a.k; ++j) a.idx_out[(int64_t)i * a.k + j] = -1;
         if (req < 0 || req >= L.max_req) { set_err(L, kErrBounds, i); a.n_valid[i] = 0; continue; }
         a.n_valid[i] = (int32_t)N;
         if (N > a.ld) set_err(L, kErrLd, i);
       }
     }
+    if (kTopk)
+      for (int b = tid; b < kHistBins; b += kThreads) sm.hist[b] = 0;
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if (lane == 0) sm.red[warp] = part;
     tc::tc_fence_before();
@@ -165,12 +745,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
   }
   const uint32_t tmem = sm.tmem_base;
   const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
+  // fused top-k: the scores of this CTA's range also go to shared memory when they fit
+  float* sc_cache = (kTopk && (g1 - g0) * kCsaPerPage <= kScoreCache)
+                        ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&sm) + (sizeof(IdxSmem) + 127) / 128 * 128)
+                        : nullptr;
   if (g0 >= g1) {                          // no tiles for this CTA: nothing was issued
     if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
     return;
   }
 
   // role state (each role only uses its own)
+  int hist_q = -1;           // epilogue, fused top-k: query whose keys sm.hist counts
   uint32_t u_base = 0;       // CTA-wide tile counter at the start of the pass (barrier phases)
   uint32_t seg_count = 0;    // segments processed (q_ready phases)
   uint32_t last_issue[kStages];
@@ -233,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
         const char* src = L.page(sm.pgs[k], a.layer) + L.pg_idx_codes;
         if (tc::elect_one()) {
           tc::mbar_arrive_expect_tx(&sm.full[s], tile_bytes);
-          tc::bulk_g2s(&sm.tiles[s][0], src, tile_bytes, &sm.full[s]);
+          tc::bulk_g2s(&sm.u.tiles[s][0], src, tile_bytes, &sm.full[s]);
         }
         __syncwarp();
         last_issue[s] = u;
@@ -260,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc::tc_fence_after();
-          const uint32_t a_base = tc::smem_u32(&sm.tiles[s][0]);
+          const uint32_t a_base = tc::smem_u32(&sm.u.tiles[s][0]);
           const uint32_t b_base = tc::smem_u32(sm.qb);
           const uint32_t sfa_col = tmem + kSfaCol + 4 * na;
           if (tc::elect_one()) {
@@ -297,6 +882,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
         //    the previous query's operands has completed.  Quantise this
         //    query's index heads: B operand codes and its scale chunk.
         tc::named_bar_sync(1, kEpiThreads);
+        if (kTopk && hist_q != qq) {             // a new query: hand the last one's counts on
+          if (hist_q >= 0) flush_hist(a, sm, hist_q, et);
+          hist_q = qq;
+        }
         for (int x = et; x < kHeadsN * CHs; x += kEpiThreads)
           reinterpret_cast<uint4*>(sm.qb)[x] = make_uint4(0, 0, 0, 0);
         for (int x = et; x < kSfChunk / 4; x += kEpiThreads)
@@ -335,25 +924,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
           const int na = uk % kNA;
           if (!(ok = wait_or_abort(sm, &sm.acc_full[na], (uk / kNA) & 1))) break;
           tc::tc_fence_after();
-          // two halves of 32 head columns (fewer live registers); four
+          // four quarters of 16 head columns (few live registers); four
           // interleaved partial sums (heads h = 4i + p), combined in a fixed order
           const uint32_t col = tmem + lane_base + 64 * na;
           const float4* w4 = reinterpret_cast<const float4*>(sm.w);
           float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t r[32];
-            tc::tmem_ld_x16(col + 32 * half, r);
-            tc::tmem_ld_x16(col + 32 * half + 16, r + 16);
+          for (int qtr = 0; qtr < 4; ++qtr) {
+            uint32_t r[16];
+            tc::tmem_ld_x16(col + 16 * qtr, r);
             tc::tmem_wait_ld();
-            if (half == 1) {
+            if (qtr == 3) {
               tc::tc_fence_before();
               tc::mbar_arrive(&sm.acc_empty[na]);
             }
 #pragma unroll
-            for (int h4 = 0; h4 < 8; ++h4) {
-              if (32 * half + h4 * 4 < HI) {
-                const float4 wv = w4[8 * half + h4];
+            for (int h4 = 0; h4 < 4; ++h4) {
+              if (16 * qtr + h4 * 4 < HI) {
+                const float4 wv = w4[4 * qtr + h4];
                 p0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), p0);
                 p1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), p1);
                 p2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), p2);
@@ -362,7 +950,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
             }
           }
           const int64_t j = (t0 + k) * kCsaPerPage + key_in_tile;
-          if (j < N) out[j] = (p0 + p1) + (p2 + p3);
+          if (j < N) {
+            const float sc = (p0 + p1) + (p2 + p3);
+            out[j] = sc;
+            if (kTopk) {
+              atomicAdd(&sm.hist[score_key(sc) >> kHistShift], 1u);
+              if (sc_cache != nullptr) sc_cache[(int64_t)uk * kCsaPerPage + key_in_tile] = sc;
+            }
+          }
         }
         u += (uint32_t)nt;
         if (!ok) sm.abort = 1;
@@ -389,10 +984,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) index_tc_kernel(IndexTcA
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+  if (kTopk && !sm.abort) {
+    if (warp >= 2 && hist_q >= 0) flush_hist(a, sm, hist_q, tid - 64);
+    topk_phase(a, sm, total, g0, g1, sc_cache);
+  }
 }
 
 // Sized so that exactly two CTAs share an SM (at most 113 KB each): their
 // two 256-column TMEM allocations then always fit the SM's 512 columns.
+static_assert(sizeof(IdxSmem) + 128 <= 112 * 1024, "two CTAs must share an SM");
+
 size_t index_tc_smem_bytes() {
   const size_t need = sizeof(IdxSmem) + 128;
   return need > 80 * 1024 ? need : 80 * 1024;
@@ -403,14 +1004,93 @@ cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* re
                             cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)index_tc_smem_bytes());
     if (e != cudaSuccess) return e;
     attr = true;
   }
   IndexTcArgs a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid};
-  index_tc_kernel<<<ctas, kThreads, index_tc_smem_bytes(), st>>>(a);
+  index_tc_kernel<false><<<ctas, kThreads, index_tc_smem_bytes(), st>>>(a);
   note_launch();
+  return cudaGetLastError();
+}
+
+// Workspace of the fused index + top-k: counters and histograms (cleared
+// before every launch), per-window candidate counts and the candidate buffer.
+struct TopkWs {
+  int64_t hist_done, cand_done, qcount, hist, hist2, cand, zero_bytes, total;
+};
+
+static TopkWs topk_ws(int n, int64_t ld) {
+  auto al = [](int64_t x) { return (x + 255) / 256 * 256; };
+  TopkWs w{};
+  w.hist_done = 0;
+  w.cand_done = al(4LL * n);
+  w.qcount = w.cand_done + al(4LL * n);
+  w.hist = w.qcount + al(4LL * n);
+  w.hist2 = w.hist + al(4LL * n * kHistBins);
+  w.zero_bytes = w.hist2 + al(4LL * n * 2048);
+  w.cand = w.zero_bytes;
+  w.total = w.cand + al(8LL * n * ld);
+  return w;
+}
+
+size_t index_topk_workspace_bytes(int n, int64_t ld) { return (size_t)topk_ws(n, ld).total; }
+
+// The fused kernel runs one CTA per SM (it allocates TMEM, and its CTAs wait
+// for one another, so the launch must fit the resident count the runtime
+// guarantees), which leaves room for the score cache.
+static size_t index_topk_smem_bytes() {
+  return (sizeof(IdxSmem) + 127) / 128 * 128 + 128 + (size_t)kScoreCache * 4;
+}
+
+int index_topk_max_ctas() { return kThreads; }
+
+cudaError_t launch_index_topk(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
+                              const float* w, float* scores, int64_t ld, int32_t* n_valid, int k, int32_t* idx_out,
+                              void* ws, int ctas, cudaStream_t st) {
+  static int occ = 0;                      // CTAs per SM that can be resident together
+  if (occ == 0) {
+    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)index_topk_smem_bytes());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(index_tc_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_tc_kernel<true>, kThreads, index_topk_smem_bytes());
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+  }
+  // the CTAs of a query wait for one another, so the grid never exceeds what
+  // is resident at once; the selection enumerates a query's CTAs one per thread
+  int dev = 0, sms = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e0 != cudaSuccess) return e0;
+  if (ctas > occ * sms) ctas = occ * sms;
+  if (ctas > kThreads) ctas = kThreads;
+  const TopkWs wl = topk_ws(n, ld);
+  char* base = static_cast<char*>(ws);
+  cudaError_t e = cudaMemsetAsync(base, 0, (size_t)wl.zero_bytes, st);
+  if (e != cudaSuccess) return e;
+  IndexTcArgs a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, k, idx_out,
+                reinterpret_cast<int32_t*>(base + wl.hist_done), reinterpret_cast<int32_t*>(base + wl.cand_done),
+                reinterpret_cast<uint32_t*>(base + wl.hist), reinterpret_cast<uint32_t*>(base + wl.hist2),
+                reinterpret_cast<int32_t*>(base + wl.qcount), reinterpret_cast<uint2*>(base + wl.cand)};
+  // the CTAs of a query wait for one another: all must be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = index_topk_smem_bytes();
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, index_tc_kernel<true>, a);
+  note_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

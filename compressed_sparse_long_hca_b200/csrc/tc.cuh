@@ -29,6 +29,17 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Wait until the grids this one depends on (launched before it on the
+// stream, with programmatic serialization allowed) have completed and their
+// memory is visible.  A no-op for a grid launched without that attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next grid on the stream (if launched with programmatic
+// serialization allowed) start before this one has finished.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -226,6 +226,40 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
                     int32_t k, int32_t* idx_out, csa_variant variant, csa_stream_t stream);
 
 /*
+ * csa_index_scores followed by csa_topk in one launch: the same scores,
+ * n_valid and indices, bit for bit (page "V4终于终于终于终于是来了", section
+ * "CSA——压缩稀疏注意力": the lightning indexer scores every compressed index
+ * key and the top-k selector keeps the best; podcast summary page, section
+ * "2.1 推理与计算效率": FP4 on the indexer path).
+ *
+ * While the indexer's thread blocks score their tiles they count each
+ * query's score keys (order-preserving 32-bit keys) over their top 12 bits;
+ * once every block of a query has added its counts they find the bin that
+ * holds the k-th largest key, write their own keys at or above that bin
+ * (the candidates, in index order) to the workspace, and the last block of
+ * the query selects exactly among the candidates (when more than 8192 keys
+ * fall at or above the bin, it radix-selects over the whole score row
+ * instead).  The scores are still written to `scores`.  The blocks wait for
+ * one another, so the kernel is launched cooperatively (all blocks resident);
+ * every wait is bounded (CSA_ERR_DEVICE_TIMEOUT).
+ *   q_idx, w, scores, ld, n_valid  as csa_index_scores
+ *   k          top-k, >= 1
+ *   idx_out    device int32 [n][k]: ascending, -1 padded, as csa_topk
+ *   workspace  device scratch of csa_index_topk_workspace_bytes(cache, n, ld)
+ *              bytes, 256-byte aligned, owned by the caller; the call clears
+ *              the part it needs (one memset queued on `stream`); it must not
+ *              be used by other work until the call's work has finished.
+ * Caches in the fp32 format run the two separate kernels instead (same
+ * results; the workspace is not used).
+ */
+size_t     csa_index_topk_workspace_bytes(const csa_cache_t* cache, int32_t n, int64_t ld);
+csa_status csa_index_topk(const csa_cache_t* cache, int32_t layer, int32_t n,
+                          const int32_t* req_ids, const float* q_idx, const float* w,
+                          float* scores, int64_t ld, int32_t* n_valid, int32_t k,
+                          int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                          csa_variant variant, csa_stream_t stream);
+
+/*
  * Multi-query attention of each query over its rows: for CSA layers the
  * entries listed in topk_idx[i][0..k) in list order (-1 = an empty row), for
  * HCA layers (topk_idx == NULL) every completed entry in order, then the raw
@@ -304,6 +338,63 @@ csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* cache, int32_t layer, 
                                        const int32_t* req_ids, const void* q,
                                        const int32_t* topk_idx, int32_t k, const float* sink,
                                        float scale, void* out, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------
+ * Batch-invariant projection GEMM:  Y[t][o] = sum_k X[t][k] W[o][k]
+ * (BF16 operands, fp32 accumulation), for the projections around the path:
+ * hidden state -> compressor candidates and gates, query down-projection to
+ * d_c and up-projection to the (index) query heads, index head weights
+ * (page "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力"); and the
+ * grouped output projection, 16 groups of 8 heads x 512 dims projected
+ * separately, then to the model width (page "深度解读DeepSeek V4 看清
+ * Benchmark以外的三个范式创新", section 01, "「精度补偿」的无限套娃游戏").
+ *
+ * Batch invariance (page "DeepSeek不惜代价保住它！V4关键特性被挖出来了",
+ * section "牺牲了什么"): a token's output never depends on the batch.  The
+ * weight rows are the MMA's M (128 per tile), the tokens its N, always in
+ * chunks of 32 (zero padded); the K order is fixed.  A weight with few row
+ * tiles has its K range cut into a number of parts that depends on the
+ * weight's shape alone, and the parts are summed in part order.
+ *
+ * Groups: with `groups` > 1 the weight is block diagonal; group g's rows
+ * (n_out / groups of them, a multiple of 128) read the columns
+ * [g k_in / groups, (g + 1) k_in / groups) of X, and the host weight holds
+ * only those k_in / groups columns per row: W is [n_out][k_in / groups].
+ *
+ *   csa_gemm_weight_bytes   device bytes of a packed weight (0 for a bad shape)
+ *   csa_gemm_pack_weight    host BF16 W (row-major, as above) -> packed
+ *                           device tiles; synchronous
+ *   csa_gemm_workspace_bytes  scratch of one call (packed activations, and
+ *                           the parts' partials when K is split)
+ *   csa_gemm_bf16           X device BF16 [n_tok][k_in], 1 <= n_tok <= 256.
+ *                           Y is written as n_seg (1 .. 8) row segments:
+ *                           rows [r_s, r_s + segs[s].rows) of Y go to the
+ *                           device buffer segs[s].y as a contiguous
+ *                           [n_tok][segs[s].rows] matrix, BF16 when
+ *                           segs[s].bf16 != 0, else fp32 (the rows add up
+ *                           to n_out; one fused weight then feeds several
+ *                           outputs).  `segs` is host memory.  workspace
+ *                           256-byte aligned, owned by the caller, not used
+ *                           by other work until the call's kernels finish.
+ *                           Asynchronous on `stream`.
+ *   csa_gemm_check_device_error  read and clear the GEMM's device error word
+ *                           (a bounded pipeline wait that gave up);
+ *                           synchronises `stream`.
+ * ------------------------------------------------------------------- */
+typedef struct {
+  int32_t rows;                 /* rows of Y in this segment                      */
+  int32_t bf16;                 /* nonzero: BF16 output, else fp32                */
+  void* y;                      /* device [n_tok][rows]                           */
+} csa_gemm_out;
+
+size_t     csa_gemm_weight_bytes(int32_t n_out, int32_t k_in, int32_t groups);
+csa_status csa_gemm_pack_weight(const uint16_t* w_host, int32_t n_out, int32_t k_in, int32_t groups,
+                                void* w_dev, size_t bytes);
+size_t     csa_gemm_workspace_bytes(int32_t n_out, int32_t k_in, int32_t groups, int32_t n_tok);
+csa_status csa_gemm_bf16(const void* w_packed, int32_t n_out, int32_t k_in, int32_t groups,
+                         const uint16_t* x, int32_t n_tok, int32_t n_seg, const csa_gemm_out* segs,
+                         void* workspace, size_t workspace_bytes, csa_stream_t stream);
+csa_status csa_gemm_check_device_error(csa_stream_t stream);
 
 /*
  * Read and clear the device error word (synchronises `stream`).  Returns

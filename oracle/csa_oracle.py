@@ -352,6 +352,32 @@ def raw_token_row(c_tau, tau, R: int, base: float = 10000.0) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Projections around the path.  [V4-来了] section "CSA——压缩稀疏注意力": the
+# token's hidden state is projected to the compressor's inputs, and the query
+# side down to a latent of width d_c (1024 in the Flash-like configuration)
+# and up to the (index) query heads.  [深度解读] section 01, "「精度补偿」的无限
+# 套娃游戏": the 128 heads x 512 attention output is projected in 16 groups
+# first, then to the model width.  A projection is a plain matrix product;
+# the grouped one is the same product with a block-diagonal weight.
+# ---------------------------------------------------------------------------
+
+def linear(x, W) -> np.ndarray:
+    """y = x W^T in fp64: x [n, K], W [n_out, K]."""
+    return np.asarray(x, np.float64) @ np.asarray(W, np.float64).T
+
+
+def grouped_linear(x, W, groups: int) -> np.ndarray:
+    """Block-diagonal projection: W [n_out, K / groups]; the rows of group g
+    (n_out / groups of them) see the columns [g K / groups, (g + 1) K / groups)
+    of x.  y[:, rows of g] = x[:, columns of g] W[rows of g]^T."""
+    x = np.asarray(x, np.float64)
+    W = np.asarray(W, np.float64)
+    n_out, kg = W.shape
+    rg = n_out // groups
+    return np.concatenate([x[:, g * kg:(g + 1) * kg] @ W[g * rg:(g + 1) * rg].T for g in range(groups)], axis=1)
+
+
+# ---------------------------------------------------------------------------
 # Lightning indexer.  [V4-来了] section "CSA——压缩稀疏注意力": the query's hidden
 # state is projected down and up to multi-head index queries, passed through
 # ReLU and scored against the compressed index keys.  Reading: the score is

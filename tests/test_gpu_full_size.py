@@ -136,7 +136,16 @@ def _step(cache, wl, layer, order, q, qi, w, sink, variant="auto"):
         idx = torch.empty((n, wl.k), dtype=torch.int32, device="cuda")
         topk(scores, nv, wl.k, idx, variant=variant)
         cache.decode_attn(layer, rid, dq, idx, torch.from_numpy(sink).cuda(), out, variant=variant)
+        # the fused index + top-k (the launch the bench times) gives the same bits
+        s2 = torch.full((n, ld), float("nan"), device="cuda")
+        nv2 = torch.zeros(n, dtype=torch.int32, device="cuda")
+        i2 = torch.empty((n, wl.k), dtype=torch.int32, device="cuda")
+        cache.index_topk(layer, rid, torch.from_numpy(qi[order]).cuda(), torch.from_numpy(w[order]).cuda(), s2, nv2,
+                         wl.k, i2, variant=variant)
         cache.check_device_error()
+        assert torch.equal(i2, idx), "fused top-k differs"
+        assert torch.equal(nv2, nv)
+        assert torch.equal(torch.nan_to_num(s2, nan=7.0).view(torch.int32), torch.nan_to_num(scores, nan=7.0).view(torch.int32))
         sc, nvh, ih = scores.cpu().numpy(), nv.cpu().numpy(), idx.cpu().numpy()
         for x, r in enumerate(order):
             res[r] = dict(scores=sc[x, : nvh[x]].copy(), idx=ih[x].copy())
@@ -311,3 +320,132 @@ def test_batch_larger_than_the_indexer_query_table():
                 if csa:
                     assert np.array_equal(again[r]["idx"], base[r]["idx"]), f"layer {layer} req {r}"
                     assert np.array_equal(again[r]["scores"].view(np.uint32), base[r]["scores"].view(np.uint32))
+
+
+def _pool_fill(cache, layer, reqs, lengths, pool, dI, group=32):
+    """Append tokens 0 .. lengths[r]-1 of every request: the inputs of
+    request r's chunk c (4096 tokens) are pool chunk (131 r + 7 c) mod P.
+    Requests go in groups so that one call's stacked inputs stay small."""
+    P = pool[0].shape[0]
+    for g0 in range(0, len(reqs), group):
+        grp = reqs[g0:g0 + group]
+        t = 0
+        while True:
+            live = [r for r in grp if lengths[r] > t]
+            if not live:
+                break
+            n_tok = min(min(lengths[r] for r in live) - t, I.CHUNK - t % I.CHUNK)
+            c, lo = t // I.CHUNK, t % I.CHUNK
+            idx = torch.tensor([(131 * r + 7 * c) % P for r in live], device="cuda")
+            st = lambda k: pool[k][idx, lo:lo + n_tok].contiguous() if pool[k] is not None else None
+            cache.compress_append(layer, torch.tensor(live, dtype=torch.int32, device="cuda"), st(0), st(1),
+                                  st(2) if dI else None, st(3) if dI else None)
+            t += n_tok
+    torch.cuda.synchronize()
+    cache.check_device_error()
+
+
+def test_c5_ragged_sweep_at_scale():
+    """The ragged batch-invariance sweep at its stated scale: interleaved
+    CSA (top-1024) and HCA layers with Pro-like shapes, 256 requests with
+    contexts log-uniform in [4K, 1M], 64 decode steps, each appending a token
+    to every request (entries complete every 4th / 128th token).  Every step
+    runs the whole batch, then sub-batches whose sizes span 1 .. 256 in
+    shuffled order with random launch variants: every request's scores,
+    indices and outputs must equal its whole-batch bits.  Eight probe
+    requests (shortest, longest, quantiles) are checked against the oracle on
+    the last step."""
+    wl_c, wl_h = I.C5_CSA, I.C5_HCA
+    n_req, n_steps = 256, 64
+    ctx = I.sweep_contexts(wl_c.seed, n_req, lo=4096, hi=1 << 20)
+    cap = int(ctx.max()) + n_steps + 512
+    pair = Hp.Pair(wl_c, 1, 1, max_req=n_req, capacity=cap,
+                   pool_blocks=int(sum((int(c) + n_steps + 8 + 511) // 512 for c in ctx)))
+    cache = pair.cache
+    for r in range(n_req):
+        cache.request_alloc(r, int(ctx[r]) + n_steps + 8)
+    lens = {r: int(ctx[r]) for r in range(n_req)}
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5005)
+    P = 24
+    pool_c = [torch.randn((P, I.CHUNK, wl_c.D), generator=g, device="cuda") for _ in range(2)]
+    pool_i = [torch.randn((P, I.CHUNK, wl_c.d_I), generator=g, device="cuda") for _ in range(2)]
+    _pool_fill(cache, 0, list(range(n_req)), lens, (pool_c[0], pool_c[1], pool_i[0], pool_i[1]), wl_c.d_I)
+    _pool_fill(cache, 1, list(range(n_req)), lens, (pool_c[1], pool_c[0], None, None), 0)
+    del pool_c, pool_i
+    order_ctx = [int(x) for x in np.argsort(ctx, kind="stable")]
+    probes = [order_ctx[int(round(qq * (n_req - 1)))] for qq in (0, 1 / 7, 2 / 7, 3 / 7, 4 / 7, 5 / 7, 6 / 7, 1)]
+    rng = np.random.default_rng(5)
+    allr = list(range(n_req))
+    sizes_seen = set()
+    for step in range(n_steps):
+        for layer, wl in ((0, wl_c), (1, wl_h)):
+            csa = layer == 0
+            gs = torch.Generator(device="cuda")
+            gs.manual_seed(10_000 + 2 * step + layer)
+            mk = lambda *shape: torch.randn(shape, generator=gs, device="cuda")
+            c, z = mk(n_req, 1, wl.D), mk(n_req, 1, wl.D)
+            ci = mk(n_req, 1, wl.d_I) if csa else None
+            zi = mk(n_req, 1, wl.d_I) if csa else None
+            cache.compress_append(layer, torch.arange(n_req, dtype=torch.int32, device="cuda"), c, z, ci, zi)
+            q = mk(n_req, wl.H, wl.D).to(torch.bfloat16)
+            qi = mk(n_req, wl.H_I, wl.d_I) if csa else None
+            w = mk(n_req, wl.H_I) if csa else None
+            sink = torch.from_numpy(pair.params[layer]["sink"]).cuda()
+
+            def run(sub, variant):
+                rid = torch.tensor(sub, dtype=torch.int32, device="cuda")
+                ix = torch.tensor(sub, device="cuda")
+                out = torch.empty((len(sub), wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+                res = {"out": out}
+                if csa:
+                    ld = max(lens[r] + 1 for r in sub) // 4 + 128
+                    sc = torch.full((len(sub), ld), float("nan"), device="cuda")
+                    nv = torch.zeros(len(sub), dtype=torch.int32, device="cuda")
+                    idx = torch.empty((len(sub), wl.k), dtype=torch.int32, device="cuda")
+                    cache.index_topk(layer, rid, qi[ix].contiguous(), w[ix].contiguous(), sc, nv, wl.k, idx,
+                                     variant=variant)
+                    cache.decode_attn(layer, rid, q[ix].contiguous(), idx, sink, out, variant=variant)
+                    res.update(sc=sc, nv=nv, idx=idx)
+                else:
+                    cache.decode_attn(layer, rid, q[ix].contiguous(), None, sink, out, variant=variant)
+                cache.check_device_error()
+                return res
+
+            base = run(allr, "auto")
+            n_sub = 3
+            for s_ in range(n_sub):
+                size = int([rng.integers(1, 9), rng.integers(9, 65), rng.integers(65, 257)][s_])
+                if step == 0 and s_ == 0:
+                    size = 1
+                sizes_seen.add(size)
+                sub = [int(x) for x in rng.choice(n_req, size=size, replace=False)]
+                variant = ("high", "low", "auto")[int(rng.integers(0, 3))]
+                got = run(sub, variant)
+                pos = torch.tensor(sub, device="cuda")
+                assert torch.equal(got["out"].view(torch.int16), base["out"][pos].view(torch.int16)), \
+                    f"step {step} layer {layer} size {size} {variant}: outputs differ"
+                if csa:
+                    assert torch.equal(got["idx"], base["idx"][pos]), f"step {step}: indices differ"
+                    assert torch.equal(got["nv"], base["nv"][pos])
+                    ldm = min(got["sc"].shape[1], base["sc"].shape[1])
+                    a_ = torch.nan_to_num(got["sc"][:, :ldm], nan=7.0).view(torch.int32)
+                    b_ = torch.nan_to_num(base["sc"][pos][:, :ldm], nan=7.0).view(torch.int32)
+                    assert torch.equal(a_, b_), f"step {step}: scores differ"
+            if step == n_steps - 1:
+                qh = q.float().cpu().numpy()
+                qih = qi.cpu().numpy() if csa else None
+                wh = w.cpu().numpy() if csa else None
+                got_h = {}
+                for r in probes:
+                    x = allr.index(r)
+                    d = {"out_f": base["out"][x].float().cpu().numpy()}
+                    if csa:
+                        nvr = int(base["nv"][x])
+                        d.update(scores=base["sc"][x, :nvr].cpu().numpy(), idx=base["idx"][x].cpu().numpy())
+                    got_h[r] = d
+                for r in probes:
+                    _oracle_check(cache, wl, layer, r, lens[r] + 1, qh, qih, wh, pair.params[layer]["sink"], got_h[r])
+        for r in allr:
+            lens[r] += 1
+    assert 1 in sizes_seen and max(sizes_seen) > 64

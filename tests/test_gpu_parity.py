@@ -462,3 +462,80 @@ def test_device_errors_are_reported_not_trapped():
     with pytest.raises(CsaError) as e:
         pair.cache.check_device_error()
     assert e.value.status == -5
+
+
+# ---------------------------------------------------------------- stage: fused index + top-k
+
+def _fused_vs_separate(pair, qi, w, k, reqs, ld, variant="auto"):
+    """csa_index_topk against csa_index_scores + csa_topk on the same inputs:
+    returns (scores, n_valid, idx) of the fused call after checking bits."""
+    from compressed_sparse_long_hca_b200.api import topk
+    n = len(reqs)
+    rid = _t(np.array(reqs, np.int32))
+    s1 = torch.full((n, ld), float("nan"), device="cuda")
+    nv1 = torch.zeros(n, dtype=torch.int32, device="cuda")
+    pair.cache.index_scores(0, rid, _t(qi[reqs]), _t(w[reqs]), s1, nv1, variant=variant)
+    i1 = torch.full((n, k), 777, dtype=torch.int32, device="cuda")
+    topk(s1, nv1, k, i1, variant=variant)
+    s2 = torch.full((n, ld), float("nan"), device="cuda")
+    nv2 = torch.zeros(n, dtype=torch.int32, device="cuda")
+    i2 = torch.full((n, k), 777, dtype=torch.int32, device="cuda")
+    pair.cache.index_topk(0, rid, _t(qi[reqs]), _t(w[reqs]), s2, nv2, k, i2, variant=variant)
+    pair.cache.check_device_error()
+    a1, a2 = s1.cpu().numpy(), s2.cpu().numpy()
+    assert np.array_equal(np.nan_to_num(a1, nan=7.0).view(np.uint32), np.nan_to_num(a2, nan=7.0).view(np.uint32))
+    assert torch.equal(nv1, nv2)
+    assert torch.equal(i1, i2), f"fused top-k differs from csa_topk (k={k}, reqs={reqs})"
+    return a2, nv2.cpu().numpy(), i2.cpu().numpy()
+
+
+@pytest.mark.parametrize("k", [1, 16, 512, 1024])
+def test_fused_index_topk_equals_separate_calls(k):
+    """csa_index_topk = csa_index_scores + csa_topk, bit for bit, on keys
+    written from oracle codes: ragged lengths (tile tails, N < k, N = 0), heavy
+    exact ties (integer-valued scores), an all-zero row (w = 0: one tie class
+    of 33,793 keys, which sends the selection to its radix path), and other
+    batch compositions; indices also against the oracle's top-k."""
+    from compressed_sparse_long_hca_b200.api import pack_index_rows
+    HI, dI = 64, 128
+    wl = I.Workload("fused", "csa", H=8, D=64, R=16, H_I=HI, d_I=dI, k=k, W=128, context=0, batch=0, seed=4243)
+    lens = [1, 3, 4, 517 * 4 + 1, 4000, 40000, 33 * 4096 + 5, 20000, 12345]
+    pair = Hp.Pair(wl, 1, 0, max_req=len(lens), capacity=max(lens) + 8)
+    r = np.random.default_rng(k + 7)
+    keys = {}
+    for i, T in enumerate(lens):
+        pair.cache.request_alloc(i, T + 8)
+        pair.cache.set_length(0, i, T)
+        N = T // 4
+        if i == 7:      # integer-valued dots: every element +-1 at scale 2^0
+            x = np.where(r.random((max(N, 1), dI)) < 0.5, -1.0, 1.0)
+        else:
+            x = r.standard_normal((max(N, 1), dI)) * np.exp2(r.integers(-3, 3, (max(N, 1), 1)))
+        kq = O.quantize_mxfp4(x)
+        if N:
+            pair.cache.write_rows(0, i, 1, 0, pack_index_rows(kq.codes[:N], kq.scales[:N]))
+        keys[i] = kq
+    n = len(lens)
+    qi = r.standard_normal((n, HI, dI)).astype(np.float32)
+    qi[7] = np.where(r.random((HI, dI)) < 0.5, -1.0, 1.0).astype(np.float32)
+    w = r.standard_normal((n, HI)).astype(np.float32)
+    w[5] = 0.0                         # all scores 0: one tie class of N = 33793 keys
+    w[7] = 1.0
+    ld = max(lens) // 4 + 5
+    allr = list(range(n))
+    sc, nv, idx = _fused_vs_separate(pair, qi, w, k, allr, ld)
+    for i, T in enumerate(lens):
+        N = T // 4
+        assert int(nv[i]) == N
+        if N == 0:
+            assert (idx[i] == -1).all()
+            continue
+        kd = O.dequantize_mxfp4(keys[i])[:N]
+        ref = O.index_scores(O.dequantize_mxfp4(O.quantize_mxfp4(qi[i])), w[i], kd)
+        Hp.check_topk(idx[i], ref, k, N, what=f"fused top-k len {T}")
+        # exactly the top-k of the GPU's own scores
+        assert np.array_equal(idx[i], O.topk(sc[i, :N].astype(np.float64), k)), f"len {T}"
+    for sub, variant in (([6, 2, 5], "high"), ([5], "low"), ([8, 7, 0, 3], "auto"), (allr[::-1], "low")):
+        _, _, idx2 = _fused_vs_separate(pair, qi, w, k, sub, ld, variant)
+        for x_, i in enumerate(sub):
+            assert np.array_equal(idx2[x_], idx[i]), (sub, i)

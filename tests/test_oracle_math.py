@@ -419,3 +419,29 @@ def test_hca_equals_csa_with_k_at_least_entries():
         assert list(oc["topk"][:N]) == list(range(N))
         assert np.array_equal(oh["out"], oc["out"])
         assert oh["n_rows"] == oc["n_rows"] == N + 128
+
+
+# ---------------------------------------------------------------- projections
+
+def test_linear_brute_force_and_one_hot():
+    r = _rng(18)
+    x, W = r.standard_normal((3, 7)), r.standard_normal((5, 7))
+    y = O.linear(x, W)
+    for t in range(3):
+        for o in range(5):
+            assert abs(y[t, o] - sum(x[t][k] * W[o][k] for k in range(7))) < 1e-12
+    P = np.zeros((4, 7))
+    for o, k in enumerate([6, 0, 3, 3]):
+        P[o, k] = 1.0                      # one-hot rows copy columns exactly
+    assert np.array_equal(O.linear(x, P), x[:, [6, 0, 3, 3]])
+
+
+def test_grouped_linear_is_block_diagonal_dense():
+    r = _rng(19)
+    groups, rg, kg = 4, 3, 5
+    x, W = r.standard_normal((2, groups * kg)), r.standard_normal((groups * rg, kg))
+    dense = np.zeros((groups * rg, groups * kg))
+    for g in range(groups):
+        dense[g * rg:(g + 1) * rg, g * kg:(g + 1) * kg] = W[g * rg:(g + 1) * rg]
+    assert np.allclose(O.grouped_linear(x, W, groups), O.linear(x, dense), atol=1e-12)
+    assert np.allclose(O.grouped_linear(x, W, 1)[:, :rg], O.linear(x[:, :kg], W[:rg]))
