@@ -12,7 +12,11 @@ Default workload: CSA Pro-like decode at 1M context (1,048,576 tokens =
 RoPE dims, indexer 64 x 128 MXFP4, top-1024, window 128.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl reference] [--no-cpu-baseline]
+                    [--impl reference] [--no-cpu-baseline] [--no-other-workloads]
+
+At N = 1 the line also carries `other_workloads`: the tiny fp32 CSA layer,
+HCA at 128K, CSA Flash-like at 128K and HCA at 1M, each with its own
+throughput, breakdown, rooflines and clock record (fewer steps each).
 
 Prints one JSON line (rank 0).  For N > 1 run under torch.distributed.run:
 each rank serves its own batch (requests shard across GPUs, no collective on
@@ -38,8 +42,6 @@ from compressed_sparse_long_hca_b200 import inputs as I  # noqa: E402
 
 METRIC = "CSA/HCA decode queries/s per layer at 128K–1M ctx; HBM GB/s vs ~8 TB/s"
 UNIT = "queries/s"
-KEY_BYTES = 68          # one MXFP4 index key: 64 B codes + 4 B scales (d_I = 128)
-ROW_BYTES = 580         # one KV row: 448 B FP8 + 128 B BF16 + 4 B scale (D = 512)
 
 
 def _peaks():
@@ -203,22 +205,35 @@ class Clocks:
 
 # ---------------------------------------------------------------- GPU arm
 
-def run_gpu(args):
+def key_bytes(wl, fmt: str) -> int:
+    """Bytes of one stored index key: MXFP4 codes + E8M0 scales, or fp32."""
+    return wl.d_I * 4 if fmt == "f32" else wl.d_I // 2 + wl.d_I // 32
+
+
+def row_bytes(wl, fmt: str) -> int:
+    """Bytes of one stored KV row: E4M3 non-RoPE part + BF16 RoPE part + fp32
+    scale, or fp32."""
+    return wl.D * 4 if fmt == "f32" else (wl.D - wl.R) + 2 * wl.R + 4
+
+
+def workload_fmt(wl) -> str:
+    """Storage format of a workload: the tiny configuration is the fp32 one."""
+    return "f32" if wl.name == "tiny-csa" else "mixed"
+
+
+def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> dict:
+    """Fill a cache of the workload through the append path, then time
+    `steps` decode steps (after `warm` eager warm-up steps) as CUDA graph
+    replays with the L2 flushed before each; returns the figures of the
+    bench line (times are this rank's; the caller takes the max over ranks)."""
     import torch
-    import torch.distributed as dist
 
     from compressed_sparse_long_hca_b200 import _lib
     from compressed_sparse_long_hca_b200.api import Cache, DecodeStep
 
-    ws, rank, local = _dist()
-    torch.cuda.set_device(local)
-    if ws > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    wl = I.WORKLOADS[args.workload]
     B, T0 = wl.batch, wl.context
     csa = wl.kind == "csa"
-    steps, warm = args.steps, args.warmup
+    fmt = workload_fmt(wl)
     cap = T0 + 5 * steps + warm + 256       # every timed or warm-up step (and graph warm-up) appends one token
     nb = (cap + 511) // 512
     layer = 0
@@ -226,7 +241,8 @@ def run_gpu(args):
     cache = Cache(n_csa=1 if csa else 0, n_hca=0 if csa else 1, H=wl.H, D=wl.D, D_rope=wl.R,
                   H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=B, max_pages_per_request=nb,
                   pool_pages=nb * B, b_pos_csa=b_kv[None] if csa else None,
-                  b_pos_idx=b_idx[None] if csa else None, b_pos_hca=None if csa else b_kv[None])
+                  b_pos_idx=b_idx[None] if csa else None, b_pos_hca=None if csa else b_kv[None], fmt=fmt)
+    qdt = cache.qdtype
     rid = torch.arange(B, dtype=torch.int32, device="cuda")
     for r in range(B):
         cache.request_alloc(r, cap)
@@ -250,7 +266,7 @@ def run_gpu(args):
     step_z = torch.randn((total_steps, B, 1, wl.D), generator=g, device="cuda")
     step_ci = torch.randn((total_steps, B, 1, dI), generator=g, device="cuda") if csa else None
     step_zi = torch.randn((total_steps, B, 1, dI), generator=g, device="cuda") if csa else None
-    q = torch.randn((B, wl.H, wl.D), generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn((B, wl.H, wl.D), generator=g, device="cuda").to(qdt)
     qi = torch.randn((B, wl.H_I, dI), generator=g, device="cuda") if csa else None
     w = torch.randn((B, wl.H_I), generator=g, device="cuda") if csa else None
     sink_d = torch.from_numpy(sink).cuda()
@@ -258,7 +274,7 @@ def run_gpu(args):
     scores = torch.empty((B, ld), device="cuda") if csa else None
     nv = torch.empty(B, dtype=torch.int32, device="cuda")
     idx = torch.empty((B, max(wl.k, 1)), dtype=torch.int32, device="cuda")
-    out = torch.empty((B, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((B, wl.H, wl.D), dtype=qdt, device="cuda")
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")    # > 126 MB L2
     flush_rd = torch.ones(256 * 2**20 // 4, dtype=torch.int32, device="cuda")
 
@@ -272,7 +288,7 @@ def run_gpu(args):
     stream = torch.cuda.current_stream()
 
     # Static per-step inputs: the timed steps replay CUDA graphs of the step
-    # (append | index | top-k + attention); before each replay the step's
+    # (append | index + top-k | attention); before each replay the step's
     # token inputs are copied into these buffers (outside the timed region).
     in_c, in_z = torch.empty_like(step_c[0]), torch.empty_like(step_z[0])
     in_ci = torch.empty_like(step_ci[0]) if csa else None
@@ -294,7 +310,8 @@ def run_gpu(args):
         cache.index_topk(layer, rid, qi, w, scores, nv, wl.k, idx, workspace=tk_ws)
 
     def part_attn():
-        cache.decode_attn(layer, rid, q, idx if csa else None, sink_d, out)
+        # on a CSA layer the call directly follows the step's index_topk
+        cache.decode_attn(layer, rid, q, idx if csa else None, sink_d, out, state_ready=csa)
 
     parts = [("append", part_append)] + ([("index_topk", part_index_topk)] if csa else []) + \
         [("attention", part_attn)]
@@ -306,9 +323,9 @@ def run_gpu(args):
     cache.check_device_error()
     lib = _lib.load()
     # The step as CUDA graphs: plain (the headline), with events around the
-    # index kernel (its roofline), with events around every part (the
-    # breakdown).  Event nodes inside a graph cost a few microseconds each,
-    # so each figure comes from its own pass of `steps` timed steps.
+    # roofline kernel, with events around every part (the breakdown).  Event
+    # nodes inside a graph cost a few microseconds each, so each figure comes
+    # from its own pass of `steps` timed steps.
     def capture(marks):
         evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
         g = torch.cuda.CUDAGraph()
@@ -333,6 +350,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     cache.check_device_error()
     if ws > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -351,11 +369,10 @@ def run_gpu(args):
                 after()
         return total
 
-    clocks = Clocks(local)
+    clocks = Clocks(torch.cuda.current_device())
     clocks.start()
     step_ms = timed_pass(g_plain, warm)
     clk = clocks.stop()
-    launches = kernels_per_step * steps               # libcsa kernels run in the timed region
     idx_sum = [0.0]
     names = [nm for nm, _ in parts]
     x = names.index(roof_part)
@@ -368,80 +385,82 @@ def run_gpu(args):
 
     timed_pass(g_all, warm + 2 * steps, add_parts)
     idx_ms = idx_sum[0] / steps
-    breakdown = {nm: round(v / steps * 1e3, 2) for nm, v in part_ms.items()}
+    res = {"step_ms": step_ms, "idx_ms": idx_ms, "clocks": clk, "launches": kernels_per_step * steps,
+           "breakdown": {nm: round(v / steps * 1e3, 2) for nm, v in part_ms.items()}, "e2e_ms": None}
     del g_plain, g_idx, g_all
-    # ---- end to end through the public API with host buffers: DecodeStep
-    # copies each step's packed inputs from pinned host memory in one
-    # transfer, replays the step and copies the output back in one transfer
-    e2e = DecodeStep(cache, layer, list(range(B)), wl.k if csa else 0, sink_d)
-    host_in = []
-    for s in range(steps):                  # each step's own inputs, packed up front (not timed)
-        buf = e2e.new_host_inputs()
-        v = e2e.views(buf)
-        v["q"].copy_(q.cpu())
-        v["c"].copy_(step_c[s].cpu())
-        v["z"].copy_(step_z[s].cpu())
-        if csa:
-            v["ci"].copy_(step_ci[s].cpu())
-            v["zi"].copy_(step_zi[s].cpu())
-            v["q_idx"].copy_(qi.cpu())
-            v["w"].copy_(w.cpu())
-        host_in.append(buf)
-    e2e(host_in[0])                         # first replay of the step's graphs: not timed
-    torch.cuda.synchronize()
-    e2e_ms = 0.0
-    for s in range(steps):
-        flush_l2()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        e2e(host_in[s])
-        b.record(stream)
-        b.synchronize()
-        e2e_ms += a.elapsed_time(b)
-    # the same again with marks between the phases (input copy, step, output copy)
-    phase = [0.0, 0.0, 0.0]
-    for s in range(steps):
-        flush_l2()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record(stream)
-        e2e(host_in[s], marks=(ev[1], ev[2]))
-        ev[3].record(stream)
-        ev[3].synchronize()
-        for x in range(3):
-            phase[x] += ev[x].elapsed_time(ev[x + 1])
-    e2e_phases = {nm: round(v / steps * 1e3, 2) for nm, v in zip(("h2d", "step", "d2h"), phase)}
-    h2d = e2e.input_bytes
-    d2h = e2e.host_out.numel() * e2e.host_out.element_size()
-    del e2e
+    if with_e2e:
+        # ---- end to end through the public API with host buffers: DecodeStep
+        # copies each step's packed inputs from pinned host memory in one
+        # transfer, replays the step and copies the output back in one transfer
+        e2e = DecodeStep(cache, layer, list(range(B)), wl.k if csa else 0, sink_d)
+        host_in = []
+        for s in range(steps):              # each step's own inputs, packed up front (not timed)
+            buf = e2e.new_host_inputs()
+            v = e2e.views(buf)
+            v["q"].copy_(q.cpu())
+            v["c"].copy_(step_c[s].cpu())
+            v["z"].copy_(step_z[s].cpu())
+            if csa:
+                v["ci"].copy_(step_ci[s].cpu())
+                v["zi"].copy_(step_zi[s].cpu())
+                v["q_idx"].copy_(qi.cpu())
+                v["w"].copy_(w.cpu())
+            host_in.append(buf)
+        e2e(host_in[0])                     # first replay of the step's graphs: not timed
+        torch.cuda.synchronize()
+        e2e_ms = 0.0
+        for s in range(steps):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e(host_in[s])
+            b.record(stream)
+            b.synchronize()
+            e2e_ms += a.elapsed_time(b)
+        # the same again with marks between the phases (input copy, step, output copy)
+        phase = [0.0, 0.0, 0.0]
+        for s in range(steps):
+            flush_l2()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record(stream)
+            e2e(host_in[s], marks=(ev[1], ev[2]))
+            ev[3].record(stream)
+            ev[3].synchronize()
+            for x in range(3):
+                phase[x] += ev[x].elapsed_time(ev[x + 1])
+        res["e2e_ms"] = e2e_ms
+        res["e2e_phases"] = {nm: round(v / steps * 1e3, 2) for nm, v in zip(("h2d", "step", "d2h"), phase)}
+        res["h2d"] = e2e.input_bytes
+        res["d2h"] = e2e.host_out.numel() * e2e.host_out.element_size()
+        del e2e
     cache.check_device_error()
-    # ---- max over ranks
-    step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms], ws, "cuda")
-    value = whole_job_rate(ws, B, steps, step_ms)
-    e2e_value = whole_job_rate(ws, B, steps, e2e_ms)
-    peak, peak_kind, peaks = _peaks()
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
-        "ms_per_step": step_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32 on mxfp4/fp8/bf16", "data": "synthetic",
-        "config": workload_config(wl, ws),
-        "gpu_launches": launches,
-        "step_breakdown_us": breakdown,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "phases_us": e2e_phases},
-        "clocks": clk,
-    }
     # tokens per request half-way through the pass that timed the roofline
     # kernel: eager warm-up steps, one untimed replay of each of the three
     # graphs, the plain pass, then half of the timed pass
-    t_mid = T0 + warm + 3 + steps + steps // 2
+    res["t_mid"] = T0 + warm + 3 + steps + steps // 2
+    del cache
+    return res
+
+
+def rooflines(wl, m: dict, steps: int) -> dict:
+    """The dominant kernel's roofline and the whole step's, from the
+    algorithmic bytes (or flops) of the workload."""
+    peak, peak_kind, peaks = _peaks()
+    csa = wl.kind == "csa"
+    fmt = workload_fmt(wl)
+    t_mid, idx_ms, step_ms = m["t_mid"], m["idx_ms"], m["step_ms"]
+    B = wl.batch
+    kb, rb = key_bytes(wl, fmt) if csa else 0, row_bytes(wl, fmt)
+    out = {}
     if csa:
         n_c = t_mid // 4
-        alg = B * (n_c * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
+        alg = B * (n_c * kb + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
         ach = alg / (idx_ms / 1e3) / 1e9
-        line["roofline"] = {"bound": "hbm", "kernel": "csa_index_topk", "achieved": ach, "peak": peak,
-                            "unit": "GB/s", "frac": ach / peak, "traffic": _profiled_traffic(),
-                            "peak_source": peak_kind, "ms_per_launch": idx_ms,
-                            "algorithmic_bytes_per_launch": alg}
+        out["roofline"] = {"bound": "hbm", "kernel": "csa_index_topk", "achieved": ach, "peak": peak,
+                           "unit": "GB/s", "frac": ach / peak,
+                           "traffic": _profiled_traffic() if wl.name == "csa-pro-1m" else None,
+                           "peak_source": peak_kind, "ms_per_launch": idx_ms,
+                           "algorithmic_bytes_per_launch": alg}
     else:
         # HCA: the attention over every compressed entry is the dominant
         # kernel; QK^T and PV are 2 * H * rows * D flops each per query
@@ -449,21 +468,79 @@ def run_gpu(args):
         flops = B * 4.0 * wl.H * rows * wl.D
         ach = flops / (idx_ms / 1e3) / 1e12
         tpeak = peaks.get("bf16_tflops", 1590.0)
-        line["roofline"] = {"bound": "tensor", "kernel": "csa_hca_decode_attn", "achieved": ach, "peak": tpeak,
-                            "unit": "TFLOP/s", "frac": ach / tpeak, "traffic": None,
-                            "peak_source": "measured bf16 burst" if "bf16_tflops" in peaks else "fallback",
-                            "ms_per_launch": idx_ms, "algorithmic_flops_per_launch": flops,
-                            "rows_per_query": rows}
+        out["roofline"] = {"bound": "tensor", "kernel": "csa_hca_decode_attn", "achieved": ach, "peak": tpeak,
+                           "unit": "TFLOP/s", "frac": ach / tpeak, "traffic": None,
+                           "peak_source": "measured bf16 burst" if "bf16_tflops" in peaks else "fallback",
+                           "ms_per_launch": idx_ms, "algorithmic_flops_per_launch": flops,
+                           "rows_per_query": rows}
     # the whole step against HBM: the algorithmic bytes of every part (index
     # keys scanned, selected and window rows gathered, q in and out) over the
     # step time, against the measured copy peak and the nominal 8 TB/s
     rows_q = (wl.k if csa else t_mid // 128) + wl.W
-    step_bytes = B * ((t_mid // 4 * KEY_BYTES + wl.H_I * wl.d_I * 4 + wl.H_I * 4 if csa else 0)
-                      + rows_q * ROW_BYTES + 2 * wl.H * wl.D * 2)
+    qb = 4 if fmt == "f32" else 2
+    step_bytes = B * ((t_mid // 4 * kb + wl.H_I * wl.d_I * 4 + wl.H_I * 4 if csa else 0)
+                      + rows_q * rb + 2 * wl.H * wl.D * qb)
     step_gbs = step_bytes / (step_ms / steps / 1e3) / 1e9
-    line["step_roofline"] = {"bound": "hbm", "achieved": step_gbs, "peak": peak, "unit": "GB/s",
-                             "frac": step_gbs / peak, "frac_of_8tbs": step_gbs / 8000.0,
-                             "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_kind}
+    out["step_roofline"] = {"bound": "hbm", "achieved": step_gbs, "peak": peak, "unit": "GB/s",
+                            "frac": step_gbs / peak, "frac_of_8tbs": step_gbs / 8000.0,
+                            "algorithmic_bytes_per_step": step_bytes, "peak_source": peak_kind}
+    return out
+
+
+# Configurations measured beside the headline at N = 1 (fewer steps each):
+# the tiny fp32 CSA layer, HCA at 128K (batch 32), CSA Flash-like at 128K
+# (batch 32) and the HCA layer at 1M (batch 4).
+OTHER_WORKLOADS = ("tiny-csa", "hca-128k", "csa-flash-128k", "hca-pro-1m")
+
+
+def run_gpu(args):
+    import gc
+
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    wl = I.WORKLOADS[args.workload]
+    steps, warm = args.steps, args.warmup
+    m = measure(wl, rank, ws, steps, warm, with_e2e=True)
+    # ---- max over ranks
+    step_ms, e2e_ms, idx_ms = max_over_ranks([m["step_ms"], m["e2e_ms"], m["idx_ms"]], ws, "cuda")
+    m.update(step_ms=step_ms, idx_ms=idx_ms)
+    value = whole_job_rate(ws, wl.batch, steps, step_ms)
+    e2e_value = whole_job_rate(ws, wl.batch, steps, e2e_ms)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
+        "ms_per_step": step_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 on fp32" if workload_fmt(wl) == "f32" else "f32 on mxfp4/fp8/bf16", "data": "synthetic",
+        "config": workload_config(wl, ws),
+        "gpu_launches": m["launches"],
+        "step_breakdown_us": m["breakdown"],
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(m["h2d"]),
+                "d2h_bytes_per_step": int(m["d2h"]), "phases_us": m["e2e_phases"]},
+        "clocks": m["clocks"],
+    }
+    line.update(rooflines(wl, m, steps))
+    if ws == 1 and args.others:
+        others = {}
+        o_steps = max(3, min(steps, 10))
+        for name in OTHER_WORKLOADS:
+            if name == wl.name:
+                continue
+            gc.collect()
+            torch.cuda.empty_cache()
+            wo = I.WORKLOADS[name]
+            mo = measure(wo, rank, ws, o_steps, 3, with_e2e=False)
+            rec = {"value": whole_job_rate(1, wo.batch, o_steps, mo["step_ms"]), "unit": UNIT,
+                   "ms_per_step": mo["step_ms"] / o_steps, "steps": o_steps, "warmup": 3,
+                   "config": workload_config(wo, 1), "step_breakdown_us": mo["breakdown"],
+                   "gpu_launches": mo["launches"], "clocks": mo["clocks"]}
+            rec.update(rooflines(wo, mo, o_steps))
+            others[name] = rec
+        line["other_workloads"] = others
     if rank == 0 and args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if rank == 0:
@@ -577,6 +654,8 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-other-workloads", dest="others", action="store_false",
+                    help="skip the other configurations measured beside the headline at N = 1")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

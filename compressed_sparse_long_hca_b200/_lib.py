@@ -15,6 +15,7 @@ CSA_OK = 0
 STATUS_NAMES = {0: "CSA_OK", -1: "CSA_ERR_ARG", -2: "CSA_ERR_CAPACITY", -3: "CSA_ERR_CUDA",
                 -4: "CSA_ERR_DEVICE_TIMEOUT", -5: "CSA_ERR_DEVICE_BOUNDS"}
 VARIANT_AUTO, VARIANT_HIGH_OCC, VARIANT_LOW_OCC = 0, 1, 2
+ATTN_STATE_READY = 0x100        # flag OR-ed into csa_hca_decode_attn's variant
 REGION_KV, REGION_INDEX, REGION_WINDOW = 0, 1, 2
 FMT_MIXED, FMT_F32 = 0, 1
 

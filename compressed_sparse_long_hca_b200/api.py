@@ -15,6 +15,7 @@ from . import _lib
 from ._lib import CsaCfg, check
 
 VARIANTS = {"auto": _lib.VARIANT_AUTO, "high": _lib.VARIANT_HIGH_OCC, "low": _lib.VARIANT_LOW_OCC}
+STATE_READY = _lib.ATTN_STATE_READY
 FORMATS = {"mixed": _lib.FMT_MIXED, "f32": _lib.FMT_F32}
 
 
@@ -171,10 +172,14 @@ class Cache:
         return ws
 
     def decode_attn(self, layer: int, req_ids, q, topk_idx, sink, out, scale=None,
-                    variant="auto", stream=None, workspace: torch.Tensor | None = None) -> None:
+                    variant="auto", stream=None, workspace: torch.Tensor | None = None,
+                    state_ready: bool = False) -> None:
         """Attention of each query over its rows.  The split (low-occupancy)
         launch needs scratch; unless `workspace` is given, a buffer owned by
-        this Cache object is grown to the size the library asks for."""
+        this Cache object is grown to the size the library asks for.
+        state_ready (CSA_ATTN_STATE_READY): the call directly follows this
+        step's index_topk on the stream, so the lengths, window rows and q
+        may be read before that kernel ends."""
         n = req_ids.numel()
         _need(req_ids, torch.int32, name="req_ids")
         _need(q, self.qdtype, (n, self.H, self.D), "q")
@@ -193,9 +198,10 @@ class Cache:
                 workspace = self._workspace(need, q.device)
             _need(workspace, torch.uint8, name="workspace")
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel()
+        flags = STATE_READY if state_ready else 0
         check(self.lib.csa_hca_decode_attn(self.handle, layer, n, _ptr(req_ids), _ptr(q), _ptr(topk_idx),
                                            k, _ptr(sink), scale, _ptr(out), ws_ptr, ws_bytes,
-                                           VARIANTS[variant], _stream(stream)), "csa_hca_decode_attn")
+                                           VARIANTS[variant] | flags, _stream(stream)), "csa_hca_decode_attn")
 
     def check_device_error(self, stream=None) -> None:
         check(self.lib.csa_check_device_error(self.handle, _stream(stream)), "device")
@@ -337,7 +343,7 @@ class DecodeStep:
         self.graph_attn = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph_attn):
             cache.decode_attn(layer, self._req, d["q"], self._idx if self.csa else None, self._sink, self.out,
-                              variant=variant, workspace=self._ws)
+                              variant=variant, workspace=self._ws, state_ready=self.csa)
         torch.cuda.synchronize(dev)
 
     def views(self, buf: torch.Tensor) -> dict:
@@ -458,19 +464,30 @@ class Linear:
     def workspace_bytes(self, n_tok: int) -> int:
         return int(self.lib.csa_gemm_workspace_bytes(self.n_out, self.k_in, self.groups, n_tok))
 
+    MAX_TOKENS = 256        # tokens per csa_gemm_bf16 call
+
     def __call__(self, x: torch.Tensor, outs, workspace: torch.Tensor | None = None, stream=None):
         """x: CUDA BF16 [n_tok][k_in].  outs: one tensor or a list of CUDA
         tensors [n_tok][rows_s] (BF16 or fp32, contiguous) whose rows add up
-        to n_out: rows [r_s, r_s + rows_s) of Y go to outs[s].  Returns outs."""
+        to n_out: rows [r_s, r_s + rows_s) of Y go to outs[s].  More than
+        MAX_TOKENS tokens are projected in consecutive calls of MAX_TOKENS
+        (a token's result does not depend on its batch).  Returns outs."""
         single = isinstance(outs, torch.Tensor)
         segs = [outs] if single else list(outs)
         n = x.shape[0] if x.dim() == 2 else -1
         _need(x, torch.bfloat16, (n, self.k_in), "x")
-        arr = (_lib.GemmOut * len(segs))()
         for s, t in enumerate(segs):
             if t.dtype not in (torch.bfloat16, torch.float32):
                 raise ValueError("outputs must be BF16 or fp32")
             _need(t, t.dtype, (n, t.shape[1] if t.dim() == 2 else -1), f"outs[{s}]")
+        for t0 in range(0, max(n, 1), self.MAX_TOKENS):
+            t1 = min(t0 + self.MAX_TOKENS, n)
+            self._call(x[t0:t1], [t[t0:t1] for t in segs], t1 - t0, workspace, stream)
+        return outs
+
+    def _call(self, x, segs, n, workspace, stream):
+        arr = (_lib.GemmOut * len(segs))()
+        for s, t in enumerate(segs):
             arr[s] = _lib.GemmOut(t.shape[1], 1 if t.dtype == torch.bfloat16 else 0, t.data_ptr())
         need = self.workspace_bytes(n) if n > 0 else 0
         if workspace is None:
@@ -481,7 +498,6 @@ class Linear:
         ws_bytes = workspace.numel() - (ws_ptr - workspace.data_ptr())
         check(self.lib.csa_gemm_bf16(self.packed.data_ptr(), self.n_out, self.k_in, self.groups, _ptr(x), n,
                                      len(segs), arr, ws_ptr, ws_bytes, _stream(stream)), "csa_gemm_bf16")
-        return outs
 
     @staticmethod
     def check_device_error(stream=None) -> None:

@@ -273,19 +273,20 @@ __global__ void length_kernel(AppendArgs a) {
 // ---------------------------------------------------------------- decode: one launch
 
 // The decode token (n_tok == 1) of request slot i: its ring row and tail
-// slot.  The token's inputs and RoPE frequencies are loaded before the
-// request's state; returns false when the request is skipped.
+// slot.  One thread per channel (blockDim >= D).  The token's inputs and
+// RoPE frequencies are loaded before the request's state; returns false
+// when the request is skipped.
 __device__ bool token1_body(const AppendArgs& a, int i, float* sm, int& req, int64_t& L0) {
   const Layout& L = a.L;
   const int D = L.D, R = L.R, dI = L.dI;
   const bool csa = a.layer < L.n_csa;
   float* row = sm;
   float* red = sm + D;
-  const int t = threadIdx.x;                 // 256 threads, D <= 512
+  const int t = threadIdx.x;
   const float* c = a.c + (int64_t)i * D;
   const float* z = a.z + (int64_t)i * D;
-  const float c0 = t < D ? c[t] : 0.f, c1 = t + 256 < D ? c[t + 256] : 0.f;
-  const float z0 = t < D ? z[t] : 0.f, z1 = t + 256 < D ? z[t + 256] : 0.f;
+  const float c0 = t < D ? c[t] : 0.f;
+  const float z0 = t < D ? z[t] : 0.f;
   float ci0 = 0.f, zi0 = 0.f;
   if (csa && t < dI) {
     ci0 = a.ci[(int64_t)i * dI + t];
@@ -295,7 +296,6 @@ __device__ bool token1_body(const AppendArgs& a, int i, float* sm, int& req, int
   if (!load_request(a, i, req, L0)) return false;
   const int64_t pos = L0;
   if (t < D) row[t] = c0;
-  if (t + 256 < D) row[t + 256] = c1;
   __syncthreads();
   if (t < R / 2) rope_pair(row[D - R + 2 * t], row[D - R + 2 * t + 1], th, pos);
   __syncthreads();
@@ -313,10 +313,6 @@ __device__ bool token1_body(const AppendArgs& a, int i, float* sm, int& req, int
     const int ring = csa ? kCsaWin : kHcaM;
     const int ts = (int)(pos % ring);
     if (t < D) { tail[(int64_t)ts * D + t] = c0; tail[(int64_t)ring * D + (int64_t)ts * D + t] = z0; }
-    if (t + 256 < D) {
-      tail[(int64_t)ts * D + t + 256] = c1;
-      tail[(int64_t)ring * D + (int64_t)ts * D + t + 256] = z1;
-    }
     if (csa && t < dI) {
       float* ti = tail + 2 * (int64_t)ring * D;
       ti[(int64_t)ts * dI + t] = ci0;
@@ -327,8 +323,10 @@ __device__ bool token1_body(const AppendArgs& a, int i, float* sm, int& req, int
 }
 
 // grid (n, 2): blockIdx.y 0 = the token's ring row and tail slot, 1 = the
-// entry it completes (if any).  n_tok == 1, request slots distinct.
-__global__ void __launch_bounds__(256) append_decode_kernel(AppendArgs a) {
+// entry it completes (if any).  n_tok == 1, request slots distinct.  One
+// thread per channel of the entry (D + d_I on CSA layers, D on HCA), so that
+// every channel's window loads are in flight at once.
+__global__ void __launch_bounds__(640) append_decode_kernel(AppendArgs a) {
   extern __shared__ float sm[];
   const Layout& L = a.L;
   const int i = blockIdx.x;
@@ -365,7 +363,8 @@ cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_
   const int threads = 256;
   if (n_tok == 1) {
     const size_t sm = (size_t)(L.D + (csa ? L.dI : 0) + 32) * sizeof(float);
-    append_decode_kernel<<<dim3(n, 2), threads, sm, st>>>(a);
+    const int dec_threads = (L.D + (csa ? L.dI : 0) + 31) / 32 * 32;   // <= 640
+    append_decode_kernel<<<dim3(n, 2), dec_threads, sm, st>>>(a);
     note_launch();
     return cudaGetLastError();
   }

@@ -7,8 +7,11 @@
 // "HCA——重度压缩注意力": a query attends to its selected (CSA) or all (HCA)
 // compressed entries, then the 128 latest raw tokens; each head's sink logit
 // enters the softmax denominator.  The rows are cut into tiles of 128; each
-// tile gives (m_t, l_t, O_t) and the tiles are folded in order, the sink
-// last.  Both storage formats and both launch variants use the fold below,
+// tile gives (m_t, l_t, O_t).  The tiles are grouped into chunks of C
+// consecutive tiles: the tiles of a chunk are folded in order into the
+// chunk's (m_c, l_c, O_c), then the chunks are folded in order, the sink
+// last.  C is fixed by the layer kind (attn_chunk_tiles), never by the
+// batch.  Both storage formats and both launch variants use the fold below,
 // so that the order and the rounding of the reduction depend on the query
 // alone.
 #pragma once
@@ -18,6 +21,13 @@ namespace csa {
 
 constexpr int kTileRows = 128;
 constexpr int kFoldBatch = 9;      // partials loaded at once by the fold kernel (a top-1024 query's 9 tiles)
+
+// Tiles per chunk of the reduction: 1 on CSA layers (a top-k query has a
+// handful of tiles, each a unit of parallel work), 8 on HCA layers (a query
+// at 1M tokens has 65 tiles: a thread block folds a chunk's tiles on chip
+// and writes one partial per chunk).  A chunk of one tile is that tile's
+// partial exactly (folding into an empty result scales by e^0 = 1).
+__host__ __device__ inline int attn_chunk_tiles(bool csa) { return csa ? 1 : 8; }
 
 struct AttnArgs {
   Layout L;
@@ -31,11 +41,15 @@ struct AttnArgs {
   float scale;
   void* out;           // BF16 or fp32 [n][H][D], as q
   int G;              // heads per CTA (MMA N), 16 or 32
-  // split launch only: partials of (query i, tile t, head h)
-  float* ws_o;        // [n][tiles_max][H][D]
-  float2* ws_ml;      // [n][tiles_max][H]   (m_t, l_t); m_t = -inf: empty tile
-  int tiles_max;
+  // split launch only: partials of (query i, chunk c, head h)
+  float* ws_o;        // [n][chunks_max][H][D]
+  float2* ws_ml;      // [n][chunks_max][H]   (m_c, l_c); m_c = -inf: empty chunk
+  int chunks_max;
   int f32;            // fp32 storage format: fp32 q and out
+  // The lengths, window rows, q and sink are final before the previous grid
+  // on the stream ends (that grid writes none of them): they may be read
+  // before griddepcontrol.wait.  Top-k lists and compressed entries never are.
+  int state_ready;
 };
 
 struct QueryGeom {
@@ -44,6 +58,8 @@ struct QueryGeom {
   int64_t t;          // query position
   int64_t n_entries, w0, n_win, n_list, total;
   int n_tiles;
+  int chunk;          // tiles per chunk
+  int n_chunks;
 };
 
 __device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& g, bool report) {
@@ -66,6 +82,8 @@ __device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& 
   g.n_list = g.csa ? a.k : g.n_entries;
   g.total = g.n_list + g.n_win;
   g.n_tiles = (int)((g.total + kTileRows - 1) / kTileRows);
+  g.chunk = attn_chunk_tiles(g.csa);
+  g.n_chunks = (g.n_tiles + g.chunk - 1) / g.chunk;
   return true;
 }
 
@@ -93,6 +111,7 @@ __device__ __forceinline__ uint16_t finish_val(float o, float cm, float den) {
 }
 
 int attn_tiles_max(const Layout& L, int layer, int k);
+int attn_chunks_max(const Layout& L, int layer, int k);
 cudaError_t launch_attn_fold(const AttnArgs& a, cudaStream_t st);
 
 }  // namespace csa

@@ -77,7 +77,7 @@ __host__ __device__ inline AttnSmem attn_smem(int D, int G) {
   s.rowf8 = o; o += (int64_t)kTileRows * 8;                  // row addresses (FP8 part)
   s.rowbf = o; o += (int64_t)kTileRows * 8;                  // row addresses (BF16 part)
   s.rsc = o;   o += (int64_t)kTileRows * 4;                  // row FP8 scales
-  s.stats = o; o += (int64_t)12 * 32 * 4;
+  s.stats = o; o += (int64_t)14 * 32 * 4;
   s.pgt = o;   o += (int64_t)kPgtCache * 4;                  // page table of the request (first entries)
   o = (o + 15) / 16 * 16;
   s.bars = o;  o += 64;
@@ -155,8 +155,11 @@ __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& 
 
 }  // namespace
 
-// Both launch variants.  kSplit: grid (tiles_max, head groups, n), one tile
-// per CTA, partials to the workspace.  Otherwise grid (n, head groups).
+// Both launch variants.  kSplit: grid (chunks_max, head groups, n), one chunk
+// of tiles per CTA, its partial to the workspace.  Otherwise grid (n, head
+// groups): the CTA walks every tile, folding the tiles of a chunk into a
+// chunk result and (chunks of more than one tile) the chunk results into a
+// total.
 template <bool kSplit>
 __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -183,6 +186,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   float* cmul = beta + 32;
   float* den = cmul + 32;
   float* part = den + 32;                                // [4][32]
+  float* m_tot = part + 128;                             // whole-query launch, chunks of > 1 tile
+  float* l_tot = m_tot + 32;
   int32_t* pgt = reinterpret_cast<int32_t*>(sm + S.pgt);
   uint64_t* bar_qk = reinterpret_cast<uint64_t*>(sm + S.bars);
   uint64_t* bar_pv = bar_qk + 1;
@@ -192,36 +197,46 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = kSplit ? (int)blockIdx.z : (int)blockIdx.x;
   const int h0 = blockIdx.y * G;
-  const int tt0 = kSplit ? (int)blockIdx.x : 0;
+  const int c0 = kSplit ? (int)blockIdx.x : 0;         // split launch: this CTA's chunk
   QueryGeom g;
   const bool reporter = tid == 0 && blockIdx.y == 0 && (!kSplit || blockIdx.x == 0);
   // The kernel is launched with programmatic serialization: its CTAs may be
   // resident before the previous grid on the stream (the top-k selection,
-  // or the append on an HCA layer) has finished.  Nothing it reads may be
-  // read before that grid is complete, so every thread waits here first.
-  tc::griddep_wait();
+  // or the append on an HCA layer) has finished.  Without state_ready every
+  // thread waits for that grid here.  With it, the query's length, q, the
+  // page table and the window rows are read first; the wait comes before
+  // the first top-k list or compressed entry is read (before the first
+  // tile's rows are resolved, or, for a tile of window rows only, once that
+  // tile has been gathered) and before anything is written.
+  const bool early = a.state_ready != 0;
+  if (!early) tc::griddep_wait();
   if (!query_geom(a, i, g, reporter)) return;
   if (kSplit) {
-    if (g.n_tiles > a.tiles_max) {
+    if (g.n_chunks > a.chunks_max) {
       if (reporter) set_err(L, kErrBounds, 4000000 + i);
       return;
     }
-    if (tt0 >= g.n_tiles) return;
+    if (c0 >= g.n_chunks) return;
   }
-  const int tt_end = kSplit ? tt0 + 1 : g.n_tiles;
+  const int tt0 = kSplit ? c0 * g.chunk : 0;
+  const int tt_end = kSplit ? min(tt0 + g.chunk, g.n_tiles) : g.n_tiles;
+  const bool multi = tt_end - tt0 > 1 || !kSplit;       // tiles are folded on chip
+  const bool two_level = !kSplit && g.chunk > 1;       // chunk results fold into a total on chip
   const int64_t pages_needed = (g.n_entries + L.rows_per_page(a.layer) - 1) / L.rows_per_page(a.layer);
   const int n_pgt = (int)(pages_needed < kPgtCache ? pages_needed : kPgtCache);
 
   // TMEM columns: S over the FP8 dims, S over the RoPE dims, the tile's
-  // output accumulators (per 128-dim chunk one for the FP8 dims and, where
-  // the chunk holds RoPE dims, one for those), then (whole-query launch) the
-  // running output, one accumulator per chunk.
+  // output accumulators (per 128-dim block one for the FP8 dims and, where
+  // the block holds RoPE dims, one for those), then (tiles folded on chip)
+  // the running output of the chunk, one accumulator per 128-dim block, and
+  // (two-level fold) the total.
   const int n_dc = Dp / 128;
   const int dmain = D - R;
   const int dc_r0 = dmain / 128;                        // first chunk holding RoPE dims
   const int n_acc = n_dc + (n_dc - dc_r0);
   const uint32_t col_s = 0, col_sr = G, col_ot = 2 * G, col_orun = 2 * G + n_acc * G;
-  const int cols_needed = kSplit ? (int)col_orun : (int)col_orun + n_dc * G;
+  const uint32_t col_otot = col_orun + n_dc * G;
+  const int cols_needed = (int)col_orun + (multi ? n_dc * G : 0) + (two_level ? n_dc * G : 0);
   uint32_t n_cols = 32;
   while ((int)n_cols < cols_needed) n_cols <<= 1;
 
@@ -235,7 +250,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     tc::mbar_init(bar_drain, 1);
     tc::fence_mbar_init();
   }
-  if (tid < 32) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; }
+  if (tid < 32) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; m_tot[tid] = -INFINITY; l_tot[tid] = 0.f; }
 
   // gather geometry: chunks of a row are FP8 (16 dims) then BF16 (8 dims);
   // item `it` of a tile = 8 rows x 4 chunks, one 16-byte load per lane
@@ -303,6 +318,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   }
   asm volatile("cp.async.wait_group 1;" ::: "memory");  // its page-table group has landed (the query's may not)
   __syncthreads();
+  const bool list_rows = (int64_t)tt0 * kTileRows < g.n_list;   // the first tile holds top-k / entry rows
+  if (early && list_rows) tc::griddep_wait();
   float2* cs = reinterpret_cast<float2*>(stage);
   int any = 0;
   if (warp < 4) {
@@ -347,6 +364,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     const float x0 = bf16_val((uint16_t)(v & 0xFFFFu)), x1 = bf16_val((uint16_t)(v >> 16));
     *wp = (uint32_t)bf16_rn(x0 * w.x - x1 * w.y) | ((uint32_t)bf16_rn(x0 * w.y + x1 * w.x) << 16);
   }
+  if (early && !list_rows) tc::griddep_wait();          // a window-only tile: gathered, nothing written yet
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -356,9 +374,89 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   const uint32_t id_pv = tc::idesc_bf16(128, G, true, true);
   bool ok = true;
   int n_done = 0;                                        // tiles whose PV has been issued
-  bool pend_fold = false;
+  bool pend_fold = false;                                // the last tile's (m_t, l_t, O_t) await their fold
+  bool chunk_has = false;                                // the current chunk holds a tile with rows
+
+  // Fold the pending tile into the chunk's running (m, l, O) (its PV has
+  // completed).  All threads.
+  auto fold_pending = [&]() {
+    if (tid < G) {
+      float mn, al, be;
+      fold_coef(m_run[tid], m_t[tid], mn, al, be);
+      alpha[tid] = al;
+      beta[tid] = be;
+      m_run[tid] = mn;
+      l_run[tid] = fold_val(l_run[tid], al, l_t[tid], be);
+    }
+    __syncthreads();
+    if (tw) {
+      for (int dc = 0; dc < n_dc; ++dc) {
+        const int d = dc * 128 + (warp & 3) * 32 + lane;
+        const bool has_rope = dc >= dc_r0;
+        uint32_t om[16], orp[16], orun[16];
+        tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om);
+        if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp);
+        tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float ot = __uint_as_float(d < dmain ? om[e] : orp[e]);
+          orun[e] = __float_as_uint(fold_val(__uint_as_float(orun[e]), alpha[hb + e], ot, beta[hb + e]));
+        }
+        tc::tmem_st_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+      }
+      tc::tmem_wait_st();
+    }
+    pend_fold = false;
+  };
+  // Two-level fold: the finished chunk's (m, l, O) into the total (an empty
+  // chunk is skipped, as the fold kernel skips its partial); the chunk
+  // result starts again empty.  All threads.
+  auto fold_chunk = [&]() {
+    __syncthreads();                                     // alpha / beta of the last tile fold are read
+    if (chunk_has) {
+      if (tid < G) {
+        float mn, al, be;
+        fold_coef(m_tot[tid], m_run[tid], mn, al, be);
+        alpha[tid] = al;
+        beta[tid] = be;
+        m_tot[tid] = mn;
+        l_tot[tid] = fold_val(l_tot[tid], al, l_run[tid], be);
+      }
+      __syncthreads();
+      if (tw) {
+        for (int dc = 0; dc < n_dc; ++dc) {
+          uint32_t orun[16], otot[16];
+          tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+          tc::tmem_ld_x16(tmem + lane_base + col_otot + dc * G + hb, otot);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            otot[e] = __float_as_uint(fold_val(__uint_as_float(otot[e]), alpha[hb + e], __uint_as_float(orun[e]),
+                                               beta[hb + e]));
+          tc::tmem_st_x16(tmem + lane_base + col_otot + dc * G + hb, otot);
+        }
+        tc::tmem_wait_st();
+      }
+      __syncthreads();
+    }
+    if (tid < G) { m_run[tid] = -INFINITY; l_run[tid] = 0.f; }
+    chunk_has = false;
+    __syncthreads();
+  };
 
   for (int tt = tt0; tt < tt_end && ok; ++tt) {
+    if (two_level && tt > tt0 && tt % g.chunk == 0) {
+      // a chunk ends before tile tt: its last tile and then the chunk fold in
+      if (pend_fold) {
+        if (n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        tc::tc_fence_after();
+        fold_pending();
+      }
+      fold_chunk();
+    }
     if (tile_valid) {
       // the previous PV has finished: tile buffer, P^T and O_t are free
       if (n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
@@ -376,37 +474,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
           buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
         }
       }
-      // -- whole-query launch: fold the previous tile while the loads fly
-      if (!kSplit && pend_fold) {
-        if (tid < G) {
-          float mn, al, be;
-          fold_coef(m_run[tid], m_t[tid], mn, al, be);
-          alpha[tid] = al;
-          beta[tid] = be;
-          m_run[tid] = mn;
-          l_run[tid] = fold_val(l_run[tid], al, l_t[tid], be);
-        }
-        __syncthreads();
-        if (tw) {
-          for (int dc = 0; dc < n_dc; ++dc) {
-            const int d = dc * 128 + (warp & 3) * 32 + lane;
-            const bool has_rope = dc >= dc_r0;
-            uint32_t om[16], orp[16], orun[16];
-            tc::tmem_ld_x16(tmem + lane_base + col_ot + dc * G + hb, om);
-            if (has_rope) tc::tmem_ld_x16(tmem + lane_base + col_ot + (n_dc + dc - dc_r0) * G + hb, orp);
-            tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float ot = __uint_as_float(d < dmain ? om[e] : orp[e]);
-              orun[e] = __float_as_uint(fold_val(__uint_as_float(orun[e]), alpha[hb + e], ot, beta[hb + e]));
-            }
-            tc::tmem_st_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
-          }
-          tc::tmem_wait_st();
-        }
-        pend_fold = false;
-      }
+      // -- fold the previous tile while the loads fly
+      if (pend_fold) fold_pending();
       // -- dequantise and store the tile
       if (fetch) {
 #pragma unroll
@@ -509,12 +578,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       __syncthreads();
       if (tid < G) l_t[tid] = ((part[tid] + part[32 + tid]) + part[64 + tid]) + part[96 + tid];
       pend_fold = true;
-    } else if (kSplit && tid < G && h0 + tid < H) {
-      // a tile without rows: an empty partial
-      a.ws_ml[((int64_t)i * a.tiles_max + tt) * H + h0 + tid] = make_float2(-INFINITY, 0.f);
+      chunk_has = true;
     }
-    // -- whole-query launch: addresses of the next tile's rows
-    if (!kSplit && tt + 1 < tt_end) {
+    // -- addresses of the next tile's rows
+    if (tt + 1 < tt_end) {
       int nany = 0;
       if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
       tile_valid = __syncthreads_count(nany) > 0;
@@ -523,14 +590,39 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
 
   if (ok && n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
   ok = __syncthreads_and(ok) != 0;
-  if (ok && kSplit && n_done > 0) {
-    // ---- split launch: the tile's partial to the workspace
+  if (ok && kSplit && n_done == 0) {
+    // ---- split launch, a chunk without rows: an empty partial
+    if (tid < G && h0 + tid < H) a.ws_ml[((int64_t)i * a.chunks_max + c0) * H + h0 + tid] = make_float2(-INFINITY, 0.f);
+  } else if (ok && kSplit && multi) {
+    // ---- split launch, a chunk of several tiles: fold its last tile, then
+    // the chunk's (m, l, O) to the workspace
+    tc::tc_fence_after();
+    if (pend_fold) fold_pending();
+    if (tid < G && h0 + tid < H)
+      a.ws_ml[((int64_t)i * a.chunks_max + c0) * H + h0 + tid] = make_float2(m_run[tid], l_run[tid]);
+    if (tw) {
+      float* wo = a.ws_o + ((int64_t)i * a.chunks_max + c0) * H * D;
+      for (int dc = 0; dc < n_dc; ++dc) {
+        uint32_t orun[16];
+        tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
+        tc::tmem_wait_ld();
+        const int d = dc * 128 + (warp & 3) * 32 + lane;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int h = h0 + hb + e;
+          if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(orun[e]);
+        }
+      }
+    }
+  } else if (ok && kSplit) {
+    // ---- split launch, a chunk of one tile: the tile's partial is the
+    // chunk's (folding into an empty result is exact)
     tc::tc_fence_after();
     if (tid < G && h0 + tid < H)
-      a.ws_ml[((int64_t)i * a.tiles_max + tt0) * H + h0 + tid] = make_float2(m_t[tid], l_t[tid]);
+      a.ws_ml[((int64_t)i * a.chunks_max + c0) * H + h0 + tid] = make_float2(m_t[tid], l_t[tid]);
     if (tw) {
-      // two 128-dim chunks per TMEM wait
-      float* wo = a.ws_o + ((int64_t)i * a.tiles_max + tt0) * H * D;
+      // two 128-dim blocks per TMEM wait
+      float* wo = a.ws_o + ((int64_t)i * a.chunks_max + c0) * H * D;
       for (int dc0 = 0; dc0 < n_dc; dc0 += 2) {
         uint32_t om[2][16], orp[2][16];
 #pragma unroll
@@ -552,6 +644,35 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
             const int h = h0 + hb + e;
             if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(d < dmain ? om[q2][e] : orp[q2][e]);
           }
+        }
+      }
+    }
+  } else if (ok && two_level) {
+    // ---- whole-query launch, two-level fold: the last tile, the last chunk,
+    // then out = O e^{m-mu} / (l e^{m-mu} + e^{sink-mu}) from the total
+    tc::tc_fence_after();
+    if (pend_fold) fold_pending();
+    fold_chunk();
+    if (tid < G) {
+      const int h = h0 + tid;
+      float cm, dn;
+      finish_coef(m_tot[tid], h < H ? a.sink[h] : 0.f, l_tot[tid], cm, dn);
+      cmul[tid] = cm;
+      den[tid] = dn;
+    }
+    __syncthreads();
+    if (tw) {
+      for (int dc = 0; dc < n_dc; ++dc) {
+        const int d = dc * 128 + (warp & 3) * 32 + lane;
+        uint32_t otot[16];
+        tc::tmem_ld_x16(tmem + lane_base + col_otot + dc * G + hb, otot);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int h = h0 + hb + e;
+          if (h < H && d < D)
+            static_cast<uint16_t*>(a.out)[((int64_t)i * H + h) * D + d] =
+                finish_val(__uint_as_float(otot[e]), cmul[hb + e], den[hb + e]);
         }
       }
     }
@@ -610,8 +731,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   if (warp == 0) tc::tmem_dealloc(tmem, n_cols);
 }
 
-// Split launch, second step: fold the partials of (query blockIdx.y, head
-// blockIdx.x) in tile order; thread x owns dims 4x .. 4x+3.
+// Split launch, second step: fold the chunk partials of (query blockIdx.y,
+// head blockIdx.x) in chunk order; thread x owns dims 4x .. 4x+3.
 __global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
   tc::griddep_wait();                                   // the partials are complete from here on
   const Layout& L = a.L;
@@ -620,16 +741,16 @@ __global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
   if (4 * d4 >= D) return;
   QueryGeom g;
   if (!query_geom(a, i, g, false)) return;             // recorded by the partial kernel
-  if (g.n_tiles > a.tiles_max) return;
+  if (g.n_chunks > a.chunks_max) return;
   float m = -INFINITY, l = 0.f;
   float o[4] = {0.f, 0.f, 0.f, 0.f};
-  const int64_t base = (int64_t)i * a.tiles_max;
-  for (int t0 = 0; t0 < g.n_tiles; t0 += kFoldBatch) {
+  const int64_t base = (int64_t)i * a.chunks_max;
+  for (int t0 = 0; t0 < g.n_chunks; t0 += kFoldBatch) {
     float2 ml[kFoldBatch];
     float4 v[kFoldBatch];
 #pragma unroll
     for (int x = 0; x < kFoldBatch; ++x) {
-      if (t0 + x < g.n_tiles) {
+      if (t0 + x < g.n_chunks) {
         ml[x] = a.ws_ml[(base + t0 + x) * H + h];
         v[x] = reinterpret_cast<const float4*>(a.ws_o + ((base + t0 + x) * H + h) * D)[d4];
       } else {
@@ -687,18 +808,23 @@ int attn_tiles_max(const Layout& L, int layer, int k) {
   return (int)((rows + kTileRows - 1) / kTileRows);
 }
 
+int attn_chunks_max(const Layout& L, int layer, int k) {
+  const int c = attn_chunk_tiles(layer < L.n_csa);
+  return (attn_tiles_max(L, layer, k) + c - 1) / c;
+}
+
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k) {
-  const int64_t units = (int64_t)n * attn_tiles_max(L, layer, k) * L.H;
+  const int64_t units = (int64_t)n * attn_chunks_max(L, layer, k) * L.H;
   return (size_t)(units * L.D * 4 + units * 8);
 }
 
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
-                           void* ws, cudaStream_t st) {
+                           void* ws, cudaStream_t st, bool state_ready) {
   const size_t sm = attn_tc_smem_bytes(L.D, G);
   if (sm > 227 * 1024) return cudaErrorInvalidValue;
   const bool split = ws != nullptr;
-  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0, 0};
+  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0, 0, state_ready ? 1 : 0};
   const int n_hg = (L.H + G - 1) / G;
   // programmatic dependent launch: the kernel may start before the previous
   // grid on the stream ends and waits for it (griddepcontrol) where it must
@@ -720,12 +846,12 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
-  a.tiles_max = attn_tiles_max(L, layer, k);
+  a.chunks_max = attn_chunks_max(L, layer, k);
   a.ws_o = static_cast<float*>(ws);
-  a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + (int64_t)n * a.tiles_max * L.H * L.D * 4);
+  a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + (int64_t)n * a.chunks_max * L.H * L.D * 4);
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  cfg.gridDim = dim3(a.tiles_max, n_hg, n);
+  cfg.gridDim = dim3(a.chunks_max, n_hg, n);
   e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, a);
   note_launch();
   if (e != cudaSuccess) return e;

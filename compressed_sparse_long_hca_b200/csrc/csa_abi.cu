@@ -25,7 +25,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st);
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
-                           void* ws, cudaStream_t st);
+                           void* ws, cudaStream_t st, bool state_ready = false);
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k);
 size_t attn_noalloc_scratch_bytes();
 cudaError_t attn_noalloc_scratch(void** out);
@@ -375,7 +375,10 @@ size_t csa_attn_workspace_bytes(const csa_cache_t* c, int32_t layer, int32_t n, 
 csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
                                const void* q, const int32_t* topk_idx, int32_t k, const float* sink,
                                float scale, void* out, void* workspace, size_t workspace_bytes,
-                               csa_variant variant, csa_stream_t stream) {
+                               csa_variant variant_flags, csa_stream_t stream) {
+  const int flags = (int)variant_flags & ~0xFF;
+  const csa_variant variant = (csa_variant)((int)variant_flags & 0xFF);
+  if (flags & ~CSA_ATTN_STATE_READY) return fail(CSA_ERR_ARG, "unknown variant flag");
   if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
   if (n == 0) return CSA_OK;
@@ -406,7 +409,7 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
                                  static_cast<float*>(out), split ? workspace : nullptr, (cudaStream_t)stream)
           : csa::launch_attn_tc(c->L, layer, n, req_ids, static_cast<const uint16_t*>(q), topk_idx, kk, sink,
                                 scale, static_cast<uint16_t*>(out), G, split ? workspace : nullptr,
-                                (cudaStream_t)stream);
+                                (cudaStream_t)stream, (flags & CSA_ATTN_STATE_READY) != 0);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
 }

@@ -57,12 +57,23 @@ __global__ void __launch_bounds__(kIdxF32Threads) index_f32_kernel(IndexF32Args 
   __syncthreads();
   float* out = a.scores + (int64_t)i * a.ld;
   for (int64_t j = (int64_t)blockIdx.x * kIdxF32Threads + tid; j < N; j += (int64_t)gridDim.x * kIdxF32Threads) {
-    const float* k = L.index_key_f32(req, a.layer, j);
+    const float4* k4 = reinterpret_cast<const float4*>(L.index_key_f32(req, a.layer, j));
     float s = 0.f;
     for (int h = 0; h < HI; ++h) {
       const float* qh = qs + h * dI;
       float dot = 0.f;
-      for (int d = 0; d < dI; ++d) dot = fmaf(qh[d], k[d], dot);
+      // 32 values of the key at a time, their loads in flight together (the
+      // first head brings the key into L1 for the others); d ascending
+      for (int d0 = 0; d0 < dI; d0 += 32) {
+        float kv[32];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float4 v = k4[d0 / 4 + x];
+          kv[4 * x] = v.x; kv[4 * x + 1] = v.y; kv[4 * x + 2] = v.z; kv[4 * x + 3] = v.w;
+        }
+#pragma unroll
+        for (int d = 0; d < 32; ++d) dot = fmaf(qh[d0 + d], kv[d], dot);
+      }
       s = fmaf(ws[h], fmaxf(dot, 0.f), s);
     }
     out[j] = s;

@@ -36,8 +36,13 @@ namespace csa {
 
 namespace {
 
-constexpr int kStages = 8;             // shared-memory stages of key tiles
-constexpr int kNA = 3;                 // TMEM accumulators (and key-scale buffers)
+constexpr int kStagesPlain = 8;        // shared-memory stages of key tiles, csa_index_scores (two CTAs per SM)
+constexpr int kStagesFused = 18;       // csa_index_topk (one CTA per SM: a tile's copy takes ~3 us to land,
+                                       // so an SM needs ~150 KB in flight to stream at the HBM rate)
+constexpr int kStagesMax = kStagesFused;
+constexpr int kNAPlain = 3;            // TMEM accumulators (and key-scale buffers), csa_index_scores
+constexpr int kNAFused = 6;            // csa_index_topk: one CTA per SM owns all 512 TMEM columns
+constexpr int kNAMax = kNAFused;
 constexpr int kEpiGroups = 2;          // epilogue groups, alternate tiles
 constexpr int kGroupThreads = 128;     // one thread per key of a tile
 constexpr int kEpiThreads = kEpiGroups * kGroupThreads;
@@ -48,23 +53,31 @@ constexpr int kTileBytes = kCsaPerPage * kMaxCh * 16 + kSfChunk;   // codes + sc
 constexpr int kPassTiles = 128;        // tiles per pass (page-table window in smem)
 constexpr int kMaxSeg = 64;            // queries per pass
 constexpr int kMaxQ = 256;             // queries whose tile counts are kept in shared memory
-constexpr uint32_t kTmemCols = 256;    // per CTA; two CTAs fill the SM's 512 columns
-constexpr uint32_t kSfaCol = 192;      // + 4 * accumulator index
-constexpr uint32_t kSfbCol = 204;
+// TMEM columns: accumulator na at 64 na, the keys' scales of accumulator na
+// at 64 NA + 4 na, the query's scales after them.  csa_index_scores: 256
+// columns per CTA (two CTAs fill the SM's 512); csa_index_topk: 512.
+template <int NA> struct TmemCols {
+  static constexpr uint32_t alloc = NA * 64 + 4 * NA + 4 <= 256 ? 256 : 512;
+  static constexpr uint32_t sfa = NA * 64;
+  static constexpr uint32_t sfb = NA * 64 + 4 * NA;
+};
+static_assert(TmemCols<kNAPlain>::alloc == 256 && TmemCols<kNAFused>::alloc == 512, "TMEM budget");
 // fused top-k (csa_index_topk)
 constexpr int kHistBits = 12;          // histogram of the score keys' top 12 bits
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kHistShift = 32 - kHistBits;
 constexpr int kCandCap = 8192;         // candidates the selecting CTA holds
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
-constexpr int kScoreCache = 24576;     // scores of the CTA's own range kept in shared memory (fused top-k)
-constexpr int kBitmapKeys = kScoreCache / 2 * 32;   // keys the selection's two bitmaps cover (same region)
+constexpr int kScoreCache = 8192;      // scores of the CTA's own range kept in shared memory (fused top-k)
+// The selection's candidates and its two bitmaps reuse the fused kernel's
+// tile stages (free once the CTA's scoring is done).
+constexpr int kBitmapWords = ((kStagesFused * kTileBytes - kCandCap * 8) / 8) & ~31;
+constexpr int64_t kBitmapKeys = (int64_t)kBitmapWords * 32;   // keys each bitmap covers
 
+// Dynamic shared memory: IdxSmem, then the tile stages (kTileBytes each),
+// then (fused top-k) the score cache.  In the top-k phase the stages hold
+// the selection's candidates (key, index) and its two bitmaps.
 struct IdxSmem {
-  union {
-    uint8_t tiles[kStages][kTileBytes];              // one page's index tile per stage
-    uint2 cand[kCandCap];                            // top-k: (key, index) of a query's candidates, index order
-  } u;
   uint8_t qb[kHeadsN * kMaxCh * 16];                 // query codes, core-matrix order
   uint8_t qsf[kSfChunk];                             // query scales, tcgen05.cp order
   alignas(16) float w[kHeadsN];
@@ -78,8 +91,8 @@ struct IdxSmem {
   int32_t q_tiles[kMaxQ];                            // tiles of query i (i < kMaxQ)
   int64_t q_N[kMaxQ];                                // keys of query i
   int64_t red[kThreads / 32];
-  uint64_t full[kStages], stage_empty[kStages];
-  uint64_t acc_full[kNA], acc_empty[kNA];
+  uint64_t full[kStagesMax], stage_empty[kStagesMax];
+  uint64_t acc_full[kNAMax], acc_empty[kNAMax];
   uint64_t q_ready;
   uint64_t drain;
   uint32_t tmem_base;
@@ -87,13 +100,19 @@ struct IdxSmem {
   // fused top-k
   uint32_t hist[kHistBins];                          // score-key histogram of the current segment
   int32_t wt[2][kThreads / 32];                      // warp totals of block scans (alternating)
+  int32_t flw[kEpiThreads / 32];                     // epilogue warp totals (histogram flush)
   int32_t tk_q, tk_t0, tk_nt, tk_flag, tk_bin, tk_above, tk_M, tk_rem;
   int64_t tk_N, tk_before;
   uint32_t tk_digit;
-  int32_t n_pend;                                    // selections this CTA owes (it was a query's last CTA)
-  int32_t pend_q[64];
-  int64_t pend_N[64];
 };
+
+constexpr size_t kSmemHead = (sizeof(IdxSmem) + 127) / 128 * 128;
+
+__device__ __forceinline__ uint8_t* smem_tiles(IdxSmem& sm) { return reinterpret_cast<uint8_t*>(&sm) + kSmemHead; }
+__device__ __forceinline__ uint2* smem_cand(IdxSmem& sm) { return reinterpret_cast<uint2*>(smem_tiles(sm)); }
+__device__ __forceinline__ uint32_t* smem_bitmaps(IdxSmem& sm) {
+  return reinterpret_cast<uint32_t*>(smem_tiles(sm) + (size_t)kCandCap * 8);
+}
 
 struct IndexTcArgs {
   Layout L;
@@ -303,18 +322,40 @@ __device__ uint32_t exact_kth(F keys, int64_t count, uint32_t bin, int above, in
 
 
 // Add this CTA's histogram of query q's keys to the query's global histogram
-// and clear it (epilogue thread et owns bins 16 et .. 16 et + 15).
+// and clear it (epilogue thread et owns bins 16 et .. 16 et + 15; all
+// epilogue threads call it).  Only the bins from the top down to the one
+// holding this CTA's k-th largest key are added: the query's k-th largest key
+// is at least as large as any CTA's k-th largest, so the global counts stay
+// exact in every bin at or above the query's k-th bin, which is all the
+// selection reads.
 __device__ __forceinline__ void flush_hist(const IndexTcArgs& a, IdxSmem& sm, int q, int et) {
+  constexpr int P = kHistBins / kEpiThreads;
+  const int lane = et & 31, w = et >> 5;
+  int mine = 0;
+#pragma unroll
+  for (int e = 0; e < P; ++e) mine += (int)sm.hist[et * P + e];
+  // keys in the bins of the epilogue threads after this one (higher bins)
+  int x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) sm.flw[w] = x;
+  tc::named_bar_sync(1, kEpiThreads);
+  int above = x - mine;
+  for (int v = w + 1; v < kEpiThreads / 32; ++v) above += sm.flw[v];
   uint32_t* g = a.hist + (int64_t)q * kHistBins;
 #pragma unroll
-  for (int e = 0; e < kHistBins / kEpiThreads; ++e) {
-    const int b = et * (kHistBins / kEpiThreads) + e;
-    const uint32_t v = sm.hist[b];
-    if (v) {
-      atomicAdd(&g[b], v);
-      sm.hist[b] = 0;
+  for (int e = P - 1; e >= 0; --e) {
+    const uint32_t c = sm.hist[et * P + e];
+    if (c) {
+      if (above < a.k) atomicAdd(&g[et * P + e], c);
+      sm.hist[et * P + e] = 0;
     }
+    above += (int)c;
   }
+  tc::named_bar_sync(1, kEpiThreads);                  // sm.flw may be reused
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
@@ -431,6 +472,7 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
         return;
       }
       // the candidates to shared memory (no order needed), all loads in flight
+      uint2* cand = smem_cand(sm);
       constexpr int kB = 8;
       for (int m0 = 0; m0 < Mtot; m0 += kThreads * kB) {
         uint2 v[kB];
@@ -442,13 +484,13 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
           const int m = m0 + u * kThreads + tid;
-          if (m < Mtot) sm.u.cand[m] = v[u];
+          if (m < Mtot) cand[m] = v[u];
         }
       }
       __syncthreads();
       // last digit (bits 0 .. 8) among the candidates that share T's upper 23 bits
       const uint32_t pre = (bin << 11) | dA;
-      ok = digit_round<9>([&](int64_t x) { return sm.u.cand[x].x; }, Mtot, pre, 0, r2, sm);
+      ok = digit_round<9>([&](int64_t x) { return cand[x].x; }, Mtot, pre, 0, r2, sm);
       const uint32_t T = (pre << 9) | sm.tk_digit;
       const int ties = r2 - sm.tk_above;        // keys == T to take, lowest indices first
       const int n_eq = sm.tk_M - sm.tk_above;   // keys == T among the candidates
@@ -459,8 +501,8 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
       }
       // bitmaps over the query's N keys: selected and (when only some of the
       // keys == T are taken) the tied ones
-      uint32_t* mb = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(&sm) + (sizeof(IdxSmem) + 127) / 128 * 128);
-      uint32_t* tb = mb + kBitmapKeys / 32;
+      uint32_t* mb = smem_bitmaps(sm);
+      uint32_t* tb = mb + kBitmapWords;
       const int nw = (int)((N + 31) / 32);
       const bool all_ties = ties == n_eq;       // the usual case: every key == T is taken
       for (int x = tid; x < nw; x += kThreads) {
@@ -469,7 +511,7 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
       }
       __syncthreads();
       for (int m = tid; m < Mtot; m += kThreads) {
-        const uint2 c = sm.u.cand[m];
+        const uint2 c = cand[m];
         if (c.x > T || (all_ties && c.x == T)) atomicOr(mb + (c.y >> 5), 1u << (c.y & 31));
         else if (c.x == T) atomicOr(tb + (c.y >> 5), 1u << (c.y & 31));
       }
@@ -537,7 +579,6 @@ __device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int
   const int tid = threadIdx.x, lane = tid & 31;
   const int G = gridDim.x;
   tc::griddep_launch_dependents();    // the next kernel may start launching while the selection runs
-  if (tid == 0) sm.n_pend = 0;
   __threadfence();
   __syncthreads();
   // thread 0 walks the queries whose tiles overlap [g0, g1)
@@ -660,38 +701,28 @@ __device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int
         }
       }
     }
-    // arrive; the last CTA of the query owes its selection, which runs
-    // after all this CTA's filters (the selection's bitmaps share shared
-    // memory with the score cache the filters read)
+    // arrive; the last CTA of the query selects (its candidates and bitmaps
+    // go to the tile stages, apart from the score cache later filters read)
     __threadfence();
     __syncthreads();
     if (tid == 0) sm.tk_flag = atomicAdd(&a.cand_done[q], 1) == n_ctas - 1 ? 1 : 0;
     __syncthreads();
     const bool last = sm.tk_flag != 0;
     __syncthreads();
-    if (!last) continue;
-    if (sm.n_pend < 64) {
-      if (tid == 0) {
-        sm.pend_q[sm.n_pend] = q;
-        sm.pend_N[sm.n_pend] = N;
-        sm.n_pend = sm.n_pend + 1;
-      }
-      __syncthreads();
-      continue;
-    }
-    select_query(a, sm, q, N);                  // the list is full: select now ...
-    sc_cache = nullptr;                         // ... and read later scores from L2
+    if (last) select_query(a, sm, q, N);
   }
-  // 3. the selections this CTA owes
-  for (int x = 0; x < sm.n_pend; ++x) select_query(a, sm, sm.pend_q[x], sm.pend_N[x]);
 }
 
 }  // namespace
 
 template <bool kTopk>
-__global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
+__global__ void __launch_bounds__(kThreads, kTopk ? 1 : 2) index_tc_kernel(IndexTcArgs a) {
+  constexpr int kStages = kTopk ? kStagesFused : kStagesPlain;
+  constexpr int kNA = kTopk ? kNAFused : kNAPlain;
+  constexpr uint32_t kTmemCols = TmemCols<kNA>::alloc, kSfaCol = TmemCols<kNA>::sfa, kSfbCol = TmemCols<kNA>::sfb;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* const tiles = smem_tiles(sm);
   const Layout& L = a.L;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int HI = L.HI, dI = L.dI, CH = dI / 32, CHs = L.CHs;
@@ -747,7 +778,7 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
   const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
   // fused top-k: the scores of this CTA's range also go to shared memory when they fit
   float* sc_cache = (kTopk && (g1 - g0) * kCsaPerPage <= kScoreCache)
-                        ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&sm) + (sizeof(IdxSmem) + 127) / 128 * 128)
+                        ? reinterpret_cast<float*>(tiles + (size_t)kStages * kTileBytes)
                         : nullptr;
   if (g0 >= g1) {                          // no tiles for this CTA: nothing was issued
     if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
@@ -758,8 +789,7 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
   int hist_q = -1;           // epilogue, fused top-k: query whose keys sm.hist counts
   uint32_t u_base = 0;       // CTA-wide tile counter at the start of the pass (barrier phases)
   uint32_t seg_count = 0;    // segments processed (q_ready phases)
-  uint32_t last_issue[kStages];
-  for (int s = 0; s < kStages; ++s) last_issue[s] = 0xFFFFFFFFu;
+  uint32_t n_issued = 0;     // producer: tiles whose copy has been issued (tiles 0 .. n_issued-1)
   int qi = 0;
   int64_t before = 0;        // tiles of queries < qi
   int64_t g = g0;
@@ -818,10 +848,10 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
         const char* src = L.page(sm.pgs[k], a.layer) + L.pg_idx_codes;
         if (tc::elect_one()) {
           tc::mbar_arrive_expect_tx(&sm.full[s], tile_bytes);
-          tc::bulk_g2s(&sm.u.tiles[s][0], src, tile_bytes, &sm.full[s]);
+          tc::bulk_g2s(tiles + (size_t)s * kTileBytes, src, tile_bytes, &sm.full[s]);
         }
         __syncwarp();
-        last_issue[s] = u;
+        n_issued = u + 1;
       }
     } else if (warp == 1) {
       // ================= MMA issuer =================
@@ -845,7 +875,7 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc::tc_fence_after();
-          const uint32_t a_base = tc::smem_u32(&sm.u.tiles[s][0]);
+          const uint32_t a_base = tc::smem_u32(tiles + (size_t)s * kTileBytes);
           const uint32_t b_base = tc::smem_u32(sm.qb);
           const uint32_t sfa_col = tmem + kSfaCol + 4 * na;
           if (tc::elect_one()) {
@@ -929,15 +959,7 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
           const uint32_t col = tmem + lane_base + 64 * na;
           const float4* w4 = reinterpret_cast<const float4*>(sm.w);
           float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-          for (int qtr = 0; qtr < 4; ++qtr) {
-            uint32_t r[16];
-            tc::tmem_ld_x16(col + 16 * qtr, r);
-            tc::tmem_wait_ld();
-            if (qtr == 3) {
-              tc::tc_fence_before();
-              tc::mbar_arrive(&sm.acc_empty[na]);
-            }
+          auto accumulate = [&](int qtr, const uint32_t* r) {
 #pragma unroll
             for (int h4 = 0; h4 < 4; ++h4) {
               if (16 * qtr + h4 * 4 < HI) {
@@ -947,6 +969,29 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
                 p2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), p2);
                 p3 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), p3);
               }
+            }
+          };
+          if constexpr (kTopk) {
+            // registers to spare (one CTA per SM): all four loads, one wait
+            uint32_t r[4][16];
+#pragma unroll
+            for (int qtr = 0; qtr < 4; ++qtr) tc::tmem_ld_x16(col + 16 * qtr, r[qtr]);
+            tc::tmem_wait_ld();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&sm.acc_empty[na]);
+#pragma unroll
+            for (int qtr = 0; qtr < 4; ++qtr) accumulate(qtr, r[qtr]);
+          } else {
+#pragma unroll
+            for (int qtr = 0; qtr < 4; ++qtr) {
+              uint32_t r[16];
+              tc::tmem_ld_x16(col + 16 * qtr, r);
+              tc::tmem_wait_ld();
+              if (qtr == 3) {
+                tc::tc_fence_before();
+                tc::mbar_arrive(&sm.acc_empty[na]);
+              }
+              accumulate(qtr, r);
             }
           }
           const int64_t j = (t0 + k) * kCsaPerPage + key_in_tile;
@@ -977,8 +1022,10 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
     if (tid == 0) {
       set_err(L, kErrTimeout, blockIdx.x);
       // let copies already in flight land before the shared memory goes away
-      for (int s = 0; s < kStages; ++s)
-        if (last_issue[s] != 0xFFFFFFFFu) tc::mbar_wait(&sm.full[s], (last_issue[s] / kStages) & 1, 200000000ull);
+      for (int s = 0; s < kStages && (uint32_t)s < n_issued; ++s) {
+        const uint32_t last = (uint32_t)s + kStages * ((n_issued - 1 - (uint32_t)s) / kStages);   // last tile of stage s
+        tc::mbar_wait(&sm.full[s], (last / kStages) & 1, 200000000ull);
+      }
     }
   }
   tc::tc_fence_before();
@@ -990,14 +1037,18 @@ __global__ void __maxnreg__(80) index_tc_kernel(IndexTcArgs a) {
   }
 }
 
-// Sized so that exactly two CTAs share an SM (at most 113 KB each): their
-// two 256-column TMEM allocations then always fit the SM's 512 columns.
-static_assert(sizeof(IdxSmem) + 128 <= 112 * 1024, "two CTAs must share an SM");
+// csa_index_scores: sized so that exactly two CTAs share an SM (at most
+// 113 KB each): their two 256-column TMEM allocations then always fit the
+// SM's 512 columns.
+constexpr size_t kSmemPlain = 128 + kSmemHead + (size_t)kStagesPlain * kTileBytes;
+static_assert(kSmemPlain <= 112 * 1024, "two CTAs must share an SM");
+// csa_index_topk: one CTA per SM, deeper stages and the score cache.
+constexpr size_t kSmemFused = 128 + kSmemHead + (size_t)kStagesFused * kTileBytes + (size_t)kScoreCache * 4;
+static_assert(kSmemFused <= 227 * 1024, "the fused kernel's shared memory exceeds one CTA's limit");
+static_assert((size_t)kCandCap * 8 + 2 * (size_t)kBitmapWords * 4 <= (size_t)kStagesFused * kTileBytes,
+              "the selection's candidates and bitmaps must fit the tile stages");
 
-size_t index_tc_smem_bytes() {
-  const size_t need = sizeof(IdxSmem) + 128;
-  return need > 80 * 1024 ? need : 80 * 1024;
-}
+size_t index_tc_smem_bytes() { return kSmemPlain > 80 * 1024 ? kSmemPlain : 80 * 1024; }
 
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
@@ -1040,9 +1091,7 @@ size_t index_topk_workspace_bytes(int n, int64_t ld) { return (size_t)topk_ws(n,
 // The fused kernel runs one CTA per SM (it allocates TMEM, and its CTAs wait
 // for one another, so the launch must fit the resident count the runtime
 // guarantees), which leaves room for the score cache.
-static size_t index_topk_smem_bytes() {
-  return (sizeof(IdxSmem) + 127) / 128 * 128 + 128 + (size_t)kScoreCache * 4;
-}
+static size_t index_topk_smem_bytes() { return kSmemFused; }
 
 int index_topk_max_ctas() { return kThreads; }
 

@@ -83,6 +83,18 @@ typedef enum {
   CSA_VARIANT_LOW_OCC = 2       /* launch shape for an under-fed GPU (small batch)*/
 } csa_variant;                  /* both return identical bits                     */
 
+/*
+ * Flag OR-ed into the variant of csa_hca_decode_attn: the attention may read
+ * the requests' lengths, their window rows, q and sink before the kernel
+ * queued directly ahead of it on the stream has finished (it still waits for
+ * that kernel before it reads a top-k list or a compressed entry, and before
+ * it writes anything).  Set it only when that kernel writes none of those
+ * inputs: in a decode step of a CSA layer, when the call directly follows
+ * the step's csa_index_topk (the step's csa_compress_append having been
+ * queued before it).  The results are the same with or without it.
+ */
+#define CSA_ATTN_STATE_READY 0x100
+
 /* Storage format of a cache (csa_cfg.fmt). */
 typedef enum {
   CSA_FMT_MIXED = 0,            /* the pages' formats: KV rows FP8 E4M3 (non-RoPE
@@ -279,24 +291,29 @@ csa_status csa_index_topk(const csa_cache_t* cache, int32_t layer, int32_t n,
  * and "HCA——重度压缩注意力".
  *
  * Reduction order: the rows are cut into tiles of 128; each tile yields
- * (max, sum of exponentials, weighted sum of V) and the tiles are folded in
- * order.  The order depends on the query alone, never on the batch.
+ * (max, sum of exponentials, weighted sum of V).  The tiles are grouped
+ * into chunks of consecutive tiles (one tile per chunk on CSA layers, 8 on
+ * HCA layers); the tiles of a chunk are folded in order into the chunk's
+ * result and the chunk results are folded in order, the sink last.  The
+ * order depends on the query and the layer kind alone, never on the batch.
  *
  * Launch variants (page "DeepSeek不惜代价保住它！V4关键特性被挖出来了",
  * section "牺牲了什么": two decode-attention kernels for a well-fed and an
  * under-fed GPU that agree bit for bit):
  *   CSA_VARIANT_HIGH_OCC  one thread block per (query, 32 heads) walks all
  *                         tiles; `workspace` is not used (may be NULL).
- *   CSA_VARIANT_LOW_OCC   one thread block per (query, 32 heads, tile); the
- *                         tiles' partials go to `workspace` and a second
+ *   CSA_VARIANT_LOW_OCC   one thread block per (query, 32 heads, chunk);
+ *                         the chunks' results go to `workspace` and a second
  *                         kernel folds them.  Needs workspace_bytes >=
  *                         csa_attn_workspace_bytes(cache, layer, n, k) and a
  *                         16-byte aligned workspace, else CSA_ERR_ARG.
  *   CSA_VARIANT_AUTO      LOW_OCC when the workspace suffices and HIGH_OCC
  *                         would leave SMs idle, else HIGH_OCC.
- * All three return identical bits.  The workspace is scratch owned by the
- * caller; its contents before and after the call are irrelevant, and it must
- * not be used by other work on the stream until the call's kernels finish.
+ * All three return identical bits.  Any of them may carry the flag
+ * CSA_ATTN_STATE_READY (defined with csa_variant above).  The workspace is
+ * scratch owned by the caller; its contents before and after the call are
+ * irrelevant, and it must not be used by other work on the stream until the
+ * call's kernels finish.
  */
 size_t     csa_attn_workspace_bytes(const csa_cache_t* cache, int32_t layer, int32_t n, int32_t k);
 csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t n,
@@ -319,13 +336,15 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
  *   - every GPU that loads libcsa holds those 16 MiB until the process exits;
  *   - a batch whose scratch (csa_attn_workspace_bytes) exceeds 16 MiB is
  *     rejected with CSA_ERR_CAPACITY before anything is launched.  The
- *     scratch is n x tiles x H x (4 D + 8) bytes; with H = 128 and D = 512
- *     that allows n x tiles <= 63.  On CSA layers tiles = ceil((k + 128) / 128)
- *     (k = 1024: up to 7 queries; 4 queries need about 9.5 MiB).  On HCA
- *     layers the host does not know the lengths, so tiles follows the
- *     cache's capacity: tiles = ceil(P / 32) + 1 for P = max_pages_per_request;
- *     at H = 128, D = 512 one query fits up to P = 1984 (1,015,808 tokens),
- *     and a cache sized for 1M tokens (P >= 2048) is refused even for n = 1;
+ *     scratch holds one partial per chunk of tiles: n x chunks x H x
+ *     (4 D + 8) bytes; with H = 128 and D = 512 that allows
+ *     n x chunks <= 63.  On CSA layers a chunk is one tile and chunks =
+ *     ceil((k + 128) / 128) (k = 1024: up to 7 queries; 4 queries need about
+ *     9.5 MiB).  On HCA layers a chunk is 8 tiles and, the host not knowing
+ *     the lengths, the count follows the cache's capacity: chunks =
+ *     ceil((ceil(P / 32) + 1) / 8) for P = max_pages_per_request; at H = 128,
+ *     D = 512 a cache sized for 1M tokens (P = 2048, 9 chunks) fits up to 7
+ *     queries, and one query fits up to P = 16,096 (8.2M tokens);
  *   - the first call on each device looks up the array's device address;
  *     make that first call before any stream capture;
  *   - all calls share the array: calls whose kernels may overlap on the GPU

@@ -390,19 +390,25 @@ def test_batch_invariance_and_variants():
     w = rng.standard_normal((n, 8)).astype(np.float32)
     sink = pair.params[0]["sink"]
 
-    def run(order, variant):
+    def run(order, variant, fused=False):
+        """fused: index_topk, then the attention directly after it with
+        state_ready (its lengths, window and q read before the top-k ends)."""
         order = list(order)
         rid = _t(np.array(order, np.int32))
         m = len(order)
         ld = max(lens) // 4 + 1
         scores = torch.zeros((m, ld), device="cuda")
         nv = torch.zeros(m, dtype=torch.int32, device="cuda")
-        pair.cache.index_scores(0, rid, _t(qi[order]), _t(w[order]), scores, nv, variant=variant)
         idx = torch.empty((m, wl.k), dtype=torch.int32, device="cuda")
-        from compressed_sparse_long_hca_b200.api import topk
-        topk(scores, nv, wl.k, idx, variant=variant)
+        qd = _t(q[order], torch.bfloat16)
+        if fused:
+            pair.cache.index_topk(0, rid, _t(qi[order]), _t(w[order]), scores, nv, wl.k, idx, variant=variant)
+        else:
+            pair.cache.index_scores(0, rid, _t(qi[order]), _t(w[order]), scores, nv, variant=variant)
+            from compressed_sparse_long_hca_b200.api import topk
+            topk(scores, nv, wl.k, idx, variant=variant)
         out = torch.empty((m, 16, 128), dtype=torch.bfloat16, device="cuda")
-        pair.cache.decode_attn(0, rid, _t(q[order], torch.bfloat16), idx, _t(sink), out, variant=variant)
+        pair.cache.decode_attn(0, rid, qd, idx, _t(sink), out, variant=variant, state_ready=fused)
         out_h = torch.empty((m, 16, 128), dtype=torch.bfloat16, device="cuda")
         pair.cache.decode_attn(1, rid, _t(q[order], torch.bfloat16), None, _t(sink), out_h, variant=variant)
         pair.cache.check_device_error()
@@ -412,8 +418,9 @@ def test_batch_invariance_and_variants():
                 for i, r in enumerate(order)}
 
     base = run(range(n), "high")
-    for order, variant in [([2], "low"), ([4, 2, 0], "high"), ([1, 3, 0, 4, 2], "low"), ([3, 3, 1], "auto")]:
-        got = run(order, variant)
+    for order, variant, fused in [([2], "low", False), ([4, 2, 0], "high", False), ([1, 3, 0, 4, 2], "low", False),
+                                  ([3, 3, 1], "auto", False), ([1, 3, 0, 4, 2], "low", True), ([4, 2, 0], "high", True)]:
+        got = run(order, variant, fused)
         for r in order:
             assert got[r] == base[r], f"request {r} differs in batch {order} ({variant})"
 

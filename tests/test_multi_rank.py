@@ -79,3 +79,24 @@ def test_reference_arm_only_rank0_prints(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(Args())
     assert buf.getvalue() == ""
+
+
+def test_bench_byte_counts_and_rooflines():
+    """Algorithmic bytes per stored key / row, and the two rooflines from a
+    made-up timing: 1 ms per step and per launch."""
+    import bench
+    from compressed_sparse_long_hca_b200 import inputs as I
+    assert bench.key_bytes(I.C4, "mixed") == 68          # 64 B E2M1 codes + 4 E8M0 scales
+    assert bench.row_bytes(I.C4, "mixed") == 580         # 448 E4M3 + 64 BF16 + fp32 scale
+    assert bench.key_bytes(I.C1, "f32") == 128 and bench.row_bytes(I.C1, "f32") == 256
+    assert bench.workload_fmt(I.C1) == "f32" and bench.workload_fmt(I.C4) == "mixed"
+    m = {"t_mid": 1 << 20, "idx_ms": 1.0, "step_ms": 1.0}
+    r = bench.rooflines(I.C4, m, steps=1)
+    keys = 4 * ((1 << 18) * 68 + 64 * 128 * 4 + 64 * 4)
+    assert r["roofline"]["algorithmic_bytes_per_launch"] == keys
+    assert r["roofline"]["achieved"] == pytest.approx(keys / 1e-3 / 1e9)
+    rows = 4 * ((1024 + 128) * 580 + 2 * 128 * 512 * 2)
+    assert r["step_roofline"]["algorithmic_bytes_per_step"] == keys + rows
+    h = bench.rooflines(I.C5_HCA_1M, m, steps=1)
+    assert h["roofline"]["bound"] == "tensor"
+    assert h["roofline"]["algorithmic_flops_per_launch"] == 4 * 4.0 * 128 * (8192 + 128) * 512

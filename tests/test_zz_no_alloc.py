@@ -108,21 +108,21 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
 
 def test_noalloc_hca_limit_follows_the_cache_capacity():
     """On an HCA layer the scratch is sized by the cache's capacity (the host
-    does not know the lengths): at H = 128, D = 512 one query fits up to 1984
-    pages per request, and a cache sized for 1M tokens (2048 pages) is refused
-    before any launch, even for a single query."""
+    does not know the lengths), one partial per chunk of 8 tiles: at H = 128,
+    D = 512 a cache sized for 1M tokens (2048 pages) fits 7 queries and not
+    8, one query fits up to 16,096 pages per request (8.2M tokens) and not
+    16,128; a batch that does not fit is refused before any launch."""
     wl = I.Workload("noalloc-hca", "hca", H=128, D=512, R=64, H_I=0, d_I=0, k=0, W=128, context=0,
                     batch=0, seed=779)
-    q = torch.zeros((1, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
     sink = torch.zeros(wl.H, device="cuda")
-    out = torch.zeros((1, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
-    rid = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for pages, expect in ((1984, True), (2048, False)):
+    for pages, n, expect in ((2048, 7, True), (2048, 8, False), (16096, 1, True), (16128, 1, False)):
         pair = Hp.Pair(wl, 0, 1, max_req=1, capacity=pages * 512)
-        fits = pair.cache.attn_workspace_bytes(0, 1, 0) <= 16 << 20
-        assert fits == expect, (pages, pair.cache.attn_workspace_bytes(0, 1, 0))
+        fits = pair.cache.attn_workspace_bytes(0, n, 0) <= 16 << 20
+        assert fits == expect, (pages, n, pair.cache.attn_workspace_bytes(0, n, 0))
         if not expect:
+            q = torch.zeros((n, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+            out = torch.zeros((n, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+            rid = torch.zeros(n, dtype=torch.int32, device="cuda")
             st = _noalloc(pair, 0, rid, q, None, 0, sink, out)
             assert st == -2, "expected CSA_ERR_CAPACITY"
             assert b"scratch" in _lib.load().csa_last_error()
-
