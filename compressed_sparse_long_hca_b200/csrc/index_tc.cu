@@ -430,7 +430,9 @@ __device__ __forceinline__ void prefetch_window(const Layout& L, int req, int la
 // tiles [g0, g1) of the flattened (query, tile) list (its histograms flushed).
 // The selection of query q by its last CTA (every CTA of q has flushed its
 // histogram and appended its candidates): indices ascending into idx_out.
-__device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N) {
+// bin / above / M: the k-th bin of the complete histogram, the keys above it
+// and at or above it, as this CTA found them for its own filter.
+__device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N, uint32_t bin, int above, int M) {
   const Layout& L = a.L;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __threadfence();
@@ -444,14 +446,6 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
     __syncthreads();
     return;
   }
-  // the k-th bin, as every CTA of q found it, from the complete histogram
-  if (!find_bin_global<kHistBins / 256>(a.hist + (int64_t)q * kHistBins, a.k, sm)) {
-    if (tid == 0) set_err(L, kErrBounds, 7300000 + q);
-    return;
-  }
-  const uint32_t bin = sm.tk_digit;
-  const int above = sm.tk_above, M = sm.tk_M;
-  __syncthreads();
     if (M <= kCandCap && N <= kBitmapKeys) {
       // first digit of the k-th key (bits 9 .. 19) from the candidates' hist2
       const int r1 = a.k - above;
@@ -543,7 +537,9 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
         }
         __syncthreads();
       }
-      // every selected index, ascending
+      // every selected index, ascending: staged in shared memory (the
+      // candidates are no longer needed), then written out coalesced
+      int32_t* staged = reinterpret_cast<int32_t*>(cand);
       int p = bitmap_warp_base(mb, nw, c0, c1, sm);
       for (int c = c0; c < c1; ++c) {
         const int x = c * 32 + lane;
@@ -552,11 +548,13 @@ __device__ void select_query(const IndexTcArgs& a, IdxSmem& sm, int q, int64_t N
         const int incl = warp_incl_scan(n, lane);
         int o = p + incl - n;
         while (b) {
-          out[o++] = x * 32 + (__ffs(b) - 1);
+          staged[o++] = x * 32 + (__ffs(b) - 1);
           b &= b - 1;
         }
         p += __shfl_sync(0xffffffffu, incl, 31);
       }
+      __syncthreads();
+      for (int x = tid; x < a.k; x += kThreads) out[x] = staged[x];
       __syncthreads();
     } else {
       // more keys than kCandCap at or above the bin (a huge tie class):
@@ -642,7 +640,7 @@ __device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int
     uint2* cq = a.cand + (int64_t)q * a.ld;
     bool fine = true;
     uint32_t bin = 0;
-    int M = 0;
+    int above = 0, M = 0;
     if (!all) {
       if (tid == 0) {
         bool ok = ld_acquire(&a.hist_done[q]) >= n_ctas;
@@ -660,14 +658,16 @@ __device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int
       if (fine) {
         fine = find_bin_global<kHistBins / 256>(a.hist + (int64_t)q * kHistBins, a.k, sm);
         bin = sm.tk_digit;
+        above = sm.tk_above;
         M = sm.tk_M;
         __syncthreads();
       }
       if (fine && M <= kCandCap) {
         // this CTA's keys of q with top bits >= bin (the candidates) are
-        // appended to the query's candidate array (warp-aggregated atomics,
-        // in no particular order); those in the k-th bin are also counted
-        // over key bits 9 .. 19 for the selection's first digit
+        // appended to the query's candidate array, in no particular order:
+        // a first pass counts them per warp, one global atomic reserves the
+        // CTA's range, a second pass writes them.  Those in the k-th bin are
+        // also counted over key bits 9 .. 19 for the selection's first digit.
         const int64_t j_lo = lo_t * kCsaPerPage, j_hi = hi_t * kCsaPerPage < N ? hi_t * kCsaPerPage : N;
         const int warp = tid >> 5;
         const unsigned lt = (1u << lane) - 1u;
@@ -676,27 +676,44 @@ __device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int
         // key j = (first local tile of q) * 128 + j - j_lo) or, past it, in L2
         const float* cache = sc_cache != nullptr ? sc_cache + ((before + lo_t - g0) * kCsaPerPage - j_lo) : nullptr;
         uint32_t* h2 = a.hist2 + (int64_t)q * 2048;
-        for (int64_t base = j_lo + (int64_t)warp * 32 * kB; base < j_hi; base += (int64_t)(kThreads / 32) * 32 * kB) {
-          float v[kB];
+        auto load = [&](int64_t base, float (&v)[kB]) {
 #pragma unroll
           for (int u = 0; u < kB; ++u) {
             const int64_t j = base + u * 32 + lane;
             v[u] = j < j_hi ? (cache != nullptr ? cache[j] : __ldcg(row + j)) : 0.f;
           }
+        };
+        const int64_t stride = (int64_t)(kThreads / 32) * 32 * kB;
+        int cnt = 0;
+        for (int64_t base = j_lo + (int64_t)warp * 32 * kB; base < j_hi; base += stride) {
+          float v[kB];
+          load(base, v);
+#pragma unroll
+          for (int u = 0; u < kB; ++u) {
+            const int64_t j = base + u * 32 + lane;
+            cnt += __popc(__ballot_sync(0xffffffffu, j < j_hi && (score_key(v[u]) >> kHistShift) >= bin));
+          }
+        }
+        // warp totals -> the warp's offset in the CTA's range, one atomic per CTA
+        int tot_c;
+        const int wbase = cta_scan(lane == 0 ? cnt : 0, sm.wt[1], &tot_c);
+        if (tid == 0) sm.tk_rem = tot_c > 0 ? atomicAdd(a.qcount + q, tot_c) : 0;
+        __syncthreads();
+        int off = sm.tk_rem + __shfl_sync(0xffffffffu, wbase, 0);
+        for (int64_t base = j_lo + (int64_t)warp * 32 * kB; base < j_hi; base += stride) {
+          float v[kB];
+          load(base, v);
 #pragma unroll
           for (int u = 0; u < kB; ++u) {
             const int64_t j = base + u * 32 + lane;
             const uint32_t key = score_key(v[u]);
             const bool pass = j < j_hi && (key >> kHistShift) >= bin;
             const unsigned bal = __ballot_sync(0xffffffffu, pass);
-            if (bal == 0) continue;
-            int off = 0;
-            if (lane == 0) off = atomicAdd(a.qcount + q, __popc(bal));
-            off = __shfl_sync(0xffffffffu, off, 0);
             if (pass) {
               cq[off + __popc(bal & lt)] = make_uint2(key, (uint32_t)j);
               if ((key >> kHistShift) == bin) atomicAdd(h2 + ((key >> 9) & 2047u), 1u);
             }
+            off += __popc(bal);
           }
         }
       }
@@ -709,7 +726,10 @@ __device__ void topk_phase(const IndexTcArgs& a, IdxSmem& sm, int64_t total, int
     __syncthreads();
     const bool last = sm.tk_flag != 0;
     __syncthreads();
-    if (last) select_query(a, sm, q, N);
+    if (last) {
+      if (all || fine) select_query(a, sm, q, N, bin, above, M);
+      else if (tid == 0) set_err(L, kErrBounds, 7300000 + q);   // the bin was never found
+    }
   }
 }
 
