@@ -2,8 +2,9 @@
 
 One step = one decode step of one layer for a batch of requests: compressor
 append of the new token (csa_compress_append), lightning-indexer scores and
-top-k in one launch (csa_index_topk) and multi-query attention
-(csa_hca_decode_attn), all through the C ABI.  Inputs are seeded synthetic
+top-k (csa_index_scores + csa_topk, or csa_index_topk in one launch with
+--select fused) and multi-query attention (csa_hca_decode_attn), all through
+the C ABI.  Inputs are seeded synthetic
 data of the workload's shapes; caches are filled through the same append
 path before timing.
 
@@ -59,11 +60,13 @@ def _dist():
     return ws, rank, local
 
 
-def _profiled_traffic():
-    """DRAM bytes (read + write) per index-kernel launch from the committed
-    ncu summary, or None when the kernel's sources changed since the capture."""
+def _profiled_traffic(select: str = "separate"):
+    """DRAM bytes (read + write) per launch of the roofline's kernel from the
+    committed ncu summary, or None when the kernel's sources changed since
+    the capture."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "index_tc_csa-pro-1m.md")
+    name = "index_topk_csa-pro-1m.md" if select == "fused" else "index_tc_csa-pro-1m.md"
+    path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
     fields = {}
@@ -80,13 +83,14 @@ def _profiled_traffic():
     return int(fields["traffic_bytes_per_launch"])
 
 
-def workload_config(wl, ws: int) -> dict:
+def workload_config(wl, ws: int, select: str = "separate") -> dict:
     """The `config` object both arms print."""
     return {"workload": wl.name, "context": wl.context, "batch_per_gpu": wl.batch, "heads": wl.H,
             "head_dim": wl.D, "rope_dims": wl.R, "indexer": f"{wl.H_I}x{wl.d_I}", "topk": wl.k,
             "window": wl.W, "layers_per_step": 1,
             "l2": "flushed before every timed step: 256 MB written, then 256 MB read (not timed)",
-            "parallelism": f"request-sharded x{ws}"}
+            "parallelism": f"request-sharded x{ws}",
+            "select": ("csa_index_topk" if select == "fused" else "csa_index_scores + csa_topk") if wl.kind == "csa" else None}
 
 
 def rank_seed(wl, rank: int) -> int:
@@ -221,7 +225,7 @@ def workload_fmt(wl) -> str:
     return "f32" if wl.name == "tiny-csa" else "mixed"
 
 
-def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> dict:
+def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool, select: str = "separate") -> dict:
     """Fill a cache of the workload through the append path, then time
     `steps` decode steps (after `warm` eager warm-up steps) as CUDA graph
     replays with the L2 flushed before each; returns the figures of the
@@ -229,7 +233,7 @@ def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> di
     import torch
 
     from compressed_sparse_long_hca_b200 import _lib
-    from compressed_sparse_long_hca_b200.api import Cache, DecodeStep
+    from compressed_sparse_long_hca_b200.api import Cache, DecodeStep, topk
 
     B, T0 = wl.batch, wl.context
     csa = wl.kind == "csa"
@@ -306,15 +310,22 @@ def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> di
 
     tk_ws = torch.empty(cache.index_topk_workspace_bytes(B, ld) + 256, dtype=torch.uint8, device="cuda") if csa else None
 
-    def part_index_topk():
+    def part_index_topk():                  # scores and selection in one launch
         cache.index_topk(layer, rid, qi, w, scores, nv, wl.k, idx, workspace=tk_ws)
+
+    def part_index():                       # scores materialised ...
+        cache.index_scores(layer, rid, qi, w, scores, nv)
+
+    def part_topk():                        # ... then selected
+        topk(scores, nv, wl.k, idx)
 
     def part_attn():
         # on a CSA layer the call directly follows the step's index_topk
         cache.decode_attn(layer, rid, q, idx if csa else None, sink_d, out, state_ready=csa)
 
-    parts = [("append", part_append)] + ([("index_topk", part_index_topk)] if csa else []) + \
-        [("attention", part_attn)]
+    sel_parts = ([("index_topk", part_index_topk)] if select == "fused" else
+                 [("index", part_index), ("topk", part_topk)]) if csa else []
+    parts = [("append", part_append)] + sel_parts + [("attention", part_attn)]
     for s in range(warm):                   # eager warm-up (also sizes the attention workspace)
         load_inputs(s)
         for _, f in parts:
@@ -341,7 +352,8 @@ def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> di
     launches0 = lib.csa_launch_count()
     g_plain, _ = capture(())
     kernels_per_step = lib.csa_launch_count() - launches0   # libcsa kernels inside the graph
-    roof_part = "index_topk" if csa else "attention"  # the kernel the roofline is reported for
+    # the kernel the roofline is reported for: the index scan (CSA), the attention (HCA)
+    roof_part = ("index_topk" if select == "fused" else "index") if csa else "attention"
     g_idx, ev_idx = capture((roof_part,))
     g_all, ev_all = capture(tuple(nm for nm, _ in parts))
     for gr in (g_plain, g_idx, g_all):      # a graph's first replay also uploads it: not timed
@@ -390,12 +402,12 @@ def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> di
     del g_plain, g_idx, g_all
     if with_e2e:
         # ---- end to end through the public API with host buffers: DecodeStep
-        # copies each step's packed inputs from pinned host memory in one
-        # transfer, replays the step and copies the output back in one transfer
-        e2e = DecodeStep(cache, layer, list(range(B)), wl.k if csa else 0, sink_d)
+        # replays one graph that copies the step's packed inputs from its
+        # pinned host buffer, runs the step and copies the output back
+        e2e = DecodeStep(cache, layer, list(range(B)), wl.k if csa else 0, sink_d, fused_select=select == "fused")
         host_in = []
         for s in range(steps):              # each step's own inputs, packed up front (not timed)
-            buf = e2e.new_host_inputs()
+            buf = torch.zeros(e2e.input_bytes, dtype=torch.uint8)
             v = e2e.views(buf)
             v["q"].copy_(q.cpu())
             v["c"].copy_(step_c[s].cpu())
@@ -406,30 +418,46 @@ def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> di
                 v["q_idx"].copy_(qi.cpu())
                 v["w"].copy_(w.cpu())
             host_in.append(buf)
-        e2e(host_in[0])                     # first replay of the step's graphs: not timed
+
+        def produce(s):
+            """The step's inputs written into the step's pinned buffer by
+            their producer (not timed; the transfer from it is)."""
+            e2e.host_in.copy_(host_in[s])
+
+        produce(0)
+        e2e()                               # first replay of the step's graph: not timed
+        e2e(timed=True)
         torch.cuda.synchronize()
         e2e_ms = 0.0
         for s in range(steps):
+            produce(s)
             flush_l2()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            e2e(host_in[s])
+            e2e()
             b.record(stream)
             b.synchronize()
             e2e_ms += a.elapsed_time(b)
-        # the same again with marks between the phases (input copy, step, output copy)
+        # the same again with marks between the phases (input copy, step,
+        # output copy) where the step is composed in Python (the C step's
+        # copies happen inside the one call)
         phase = [0.0, 0.0, 0.0]
-        for s in range(steps):
+        for s in range(steps if e2e.fused_select else 0):
+            produce(s)
             flush_l2()
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            ev[0].record(stream)
-            e2e(host_in[s], marks=(ev[1], ev[2]))
-            ev[3].record(stream)
-            ev[3].synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e(timed=True)
+            b.record(stream)
+            b.synchronize()
+            ev = [a, e2e.marks[0], e2e.marks[1], b]
             for x in range(3):
                 phase[x] += ev[x].elapsed_time(ev[x + 1])
         res["e2e_ms"] = e2e_ms
-        res["e2e_phases"] = {nm: round(v / steps * 1e3, 2) for nm, v in zip(("h2d", "step", "d2h"), phase)}
+        res["e2e_phases"] = ({nm: round(v / steps * 1e3, 2) for nm, v in zip(("h2d", "step", "d2h"), phase)}
+                             if e2e.fused_select else None)
+        res["e2e_api"] = "api.DecodeStep -> " + ("csa_compress_append + csa_index_topk + csa_hca_decode_attn"
+                                                 if e2e.fused_select else "csa_decode_step (host buffers)")
         res["h2d"] = e2e.input_bytes
         res["d2h"] = e2e.host_out.numel() * e2e.host_out.element_size()
         del e2e
@@ -442,7 +470,7 @@ def measure(wl, rank: int, ws: int, steps: int, warm: int, with_e2e: bool) -> di
     return res
 
 
-def rooflines(wl, m: dict, steps: int) -> dict:
+def rooflines(wl, m: dict, steps: int, select: str = "separate") -> dict:
     """The dominant kernel's roofline and the whole step's, from the
     algorithmic bytes (or flops) of the workload."""
     peak, peak_kind, peaks = _peaks()
@@ -456,9 +484,10 @@ def rooflines(wl, m: dict, steps: int) -> dict:
         n_c = t_mid // 4
         alg = B * (n_c * kb + wl.H_I * wl.d_I * 4 + wl.H_I * 4)
         ach = alg / (idx_ms / 1e3) / 1e9
-        out["roofline"] = {"bound": "hbm", "kernel": "csa_index_topk", "achieved": ach, "peak": peak,
+        out["roofline"] = {"bound": "hbm", "kernel": "csa_index_topk" if select == "fused" else "csa_index_scores",
+                           "achieved": ach, "peak": peak,
                            "unit": "GB/s", "frac": ach / peak,
-                           "traffic": _profiled_traffic() if wl.name == "csa-pro-1m" else None,
+                           "traffic": _profiled_traffic(select) if wl.name == "csa-pro-1m" else None,
                            "peak_source": peak_kind, "ms_per_launch": idx_ms,
                            "algorithmic_bytes_per_launch": alg}
     else:
@@ -506,7 +535,7 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     wl = I.WORKLOADS[args.workload]
     steps, warm = args.steps, args.warmup
-    m = measure(wl, rank, ws, steps, warm, with_e2e=True)
+    m = measure(wl, rank, ws, steps, warm, with_e2e=True, select=args.select)
     # ---- max over ranks
     step_ms, e2e_ms, idx_ms = max_over_ranks([m["step_ms"], m["e2e_ms"], m["idx_ms"]], ws, "cuda")
     m.update(step_ms=step_ms, idx_ms=idx_ms)
@@ -516,14 +545,14 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps, "warmup": warm,
         "ms_per_step": step_ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32 on fp32" if workload_fmt(wl) == "f32" else "f32 on mxfp4/fp8/bf16", "data": "synthetic",
-        "config": workload_config(wl, ws),
+        "config": workload_config(wl, ws, args.select),
         "gpu_launches": m["launches"],
         "step_breakdown_us": m["breakdown"],
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(m["h2d"]),
-                "d2h_bytes_per_step": int(m["d2h"]), "phases_us": m["e2e_phases"]},
+                "d2h_bytes_per_step": int(m["d2h"]), "phases_us": m["e2e_phases"], "through": m["e2e_api"]},
         "clocks": m["clocks"],
     }
-    line.update(rooflines(wl, m, steps))
+    line.update(rooflines(wl, m, steps, args.select))
     if ws == 1 and args.others:
         others = {}
         o_steps = max(3, min(steps, 10))
@@ -533,12 +562,12 @@ def run_gpu(args):
             gc.collect()
             torch.cuda.empty_cache()
             wo = I.WORKLOADS[name]
-            mo = measure(wo, rank, ws, o_steps, 3, with_e2e=False)
+            mo = measure(wo, rank, ws, o_steps, 3, with_e2e=False, select=args.select)
             rec = {"value": whole_job_rate(1, wo.batch, o_steps, mo["step_ms"]), "unit": UNIT,
                    "ms_per_step": mo["step_ms"] / o_steps, "steps": o_steps, "warmup": 3,
-                   "config": workload_config(wo, 1), "step_breakdown_us": mo["breakdown"],
+                   "config": workload_config(wo, 1, args.select), "step_breakdown_us": mo["breakdown"],
                    "gpu_launches": mo["launches"], "clocks": mo["clocks"]}
-            rec.update(rooflines(wo, mo, o_steps))
+            rec.update(rooflines(wo, mo, o_steps, args.select))
             others[name] = rec
         line["other_workloads"] = others
     if rank == 0 and args.cpu_baseline and ws == 1:
@@ -654,6 +683,9 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--select", default="separate", choices=["fused", "separate"],
+                    help="CSA selection: csa_index_scores + csa_topk (two launches, the faster on one "
+                         "B200) or csa_index_topk (one cooperative launch)")
     ap.add_argument("--no-other-workloads", dest="others", action="store_false",
                     help="skip the other configurations measured beside the headline at N = 1")
     args = ap.parse_args()

@@ -56,6 +56,9 @@ SIGNATURES = {
     "csa_debug_set_length": (_I32, [_P, _I32, _I32, _I64]),
     "csa_debug_get_length": (_I64, [_P, _I32, _I32]),
     "csa_debug_wait_timeout": (_I32, [_P, _I32, _P]),
+    "csa_decode_step_input_bytes": (_SZ, [_P, _I32, _I32]),
+    "csa_decode_step_dev_bytes": (_SZ, [_P, _I32, _I32, _I32]),
+    "csa_decode_step": (_I32, [_P, _I32, _I32, _P, _I32, _P, _F, _P, _P, _P, _SZ, _P]),
     "csa_gemm_weight_bytes": (_SZ, [_I32, _I32, _I32]),
     "csa_gemm_pack_weight": (_I32, [_P, _I32, _I32, _I32, _P, _SZ]),
     "csa_gemm_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32]),

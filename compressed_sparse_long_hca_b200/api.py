@@ -264,33 +264,36 @@ def decode_step_fields(n: int, H: int, D: int, H_I: int, d_I: int, csa: bool, al
 
 class DecodeStep:
     """One decode step of a fixed batch of requests on one layer, captured
-    once as two CUDA graphs and replayed every step.
+    once as a CUDA graph and replayed every step.
 
-    The step appends each request's new token (csa_compress_append), then on
-    a CSA layer scores the index keys and selects the top k in one launch
-    (csa_index_topk) -- the first graph -- and attends (csa_hca_decode_attn)
-    -- the second graph; on an HCA layer the first graph only appends and the
-    attention covers every compressed entry.
+    The step is the C ABI's csa_decode_step (host input copy, append, index
+    scores and top-k, attention, output copy, on one stream, the query's copy
+    on a second one); with fused_select=True it is composed here from
+    csa_compress_append, csa_index_topk (one launch) and csa_hca_decode_attn
+    instead.  The attention may start while the selection finishes.
 
-    Inputs of a step, packed in a buffer from `new_host_inputs()` and filled
-    through `views(buf)`: c and z [n, 1, D] fp32 (the token's KV candidate
-    and gate logits), on a CSA layer also ci and zi [n, 1, d_I] fp32, q_idx
-    [n, H_I, d_I] fp32 and w [n, H_I] fp32, and last q [n, H, D] bf16.  Each
-    field starts on a 256-byte boundary.
+    Inputs of a step, packed in the pinned host buffer `host_in` (owned by
+    the step) and filled through `views(step.host_in)`: c and z [n, 1, D] fp32
+    (the token's KV candidate and gate logits), on a CSA layer also ci and zi
+    [n, 1, d_I] fp32, q_idx [n, H_I, d_I] fp32 and w [n, H_I] fp32, and last
+    q [n, H, D] (bf16, fp32 in the fp32 format).  Each field starts on a
+    256-byte boundary.
 
-    Host transfers: the fields before q travel in one copy on the caller's
-    stream ahead of the first graph; q, which only the attention reads,
-    travels in one copy on a side stream while the first graph runs, and the
-    second graph waits for it; the output returns in one copy.
+    Host transfers are nodes of the graph: the fields before q in one copy
+    ahead of the append; q, which only the attention reads, in one copy on a
+    forked branch that runs beside the append and the selection and that the
+    attention waits for; the output [n, H, D] in one copy into `host_out`
+    (pinned) at the end.
 
-    The graphs hold device pointers, so the batch (req_ids), k and the sink
-    logits are fixed at construction.  On a CSA layer construction runs the
-    selection once (it changes nothing in the cache) so that its one-time
-    launch set-up happens before the capture."""
+    The graph holds device and host pointers, so the batch (req_ids), k, the
+    sink logits and the two host buffers are fixed at construction.  On a CSA
+    layer construction runs the selection once (it changes nothing in the
+    cache) so that its one-time launch set-up happens before the capture."""
 
     def __init__(self, cache: Cache, layer: int, req_ids, k: int, sink, variant: str = "auto",
-                 device: str | torch.device = "cuda"):
+                 device: str | torch.device = "cuda", fused_select: bool = False):
         self.cache, self.layer, self.k, self.variant = cache, layer, int(k), variant
+        self.fused_select = bool(fused_select)
         self.csa = layer < cache.n_csa
         ids = [int(r) for r in req_ids]
         n = self.n = len(ids)
@@ -300,11 +303,13 @@ class DecodeStep:
             raise ValueError("a CSA layer needs k > 0")
         H, D = cache.H, cache.D
         self._fields, off = decode_step_fields(n, H, D, cache.H_I, cache.d_I, self.csa, qdtype=cache.qdtype)
+        if int(cache.lib.csa_decode_step_input_bytes(cache.handle, layer, n)) != off:
+            raise RuntimeError("packed input layout differs from the library's")
         self.input_bytes = off
         self._q_off = next(f[3] for f in self._fields if f[0] == "q")
         dev = self.device = torch.device(device)
         self._dev_in = torch.zeros(off, dtype=torch.uint8, device=dev)
-        d = self.views(self._dev_in)
+        self.host_in = torch.zeros(off, dtype=torch.uint8).pin_memory()
         self._req = torch.tensor(ids, dtype=torch.int32, device=dev)
         self._sink = (sink if isinstance(sink, torch.Tensor) else torch.from_numpy(np.asarray(sink, np.float32)))
         self._sink = self._sink.to(device=dev, dtype=torch.float32).contiguous()
@@ -313,38 +318,103 @@ class DecodeStep:
         self._ws = torch.empty(max(cache.attn_workspace_bytes(layer, n, self.k if self.csa else 0), 16),
                                dtype=torch.uint8, device=dev)
         self._side = torch.cuda.Stream(device=dev)
-        self._ev_start, self._ev_q = torch.cuda.Event(), torch.cuda.Event()
-        if self.csa:
+        self._done = torch.cuda.Event()
+        self._dev_buf = None
+        if not self.fused_select:
+            nbytes = int(cache.lib.csa_decode_step_dev_bytes(cache.handle, layer, n, self.k if self.csa else 0))
+            if nbytes == 0:
+                raise ValueError("invalid decode step shape")
+            self._dev_buf = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+            # the C step holds its own copies of the inputs and the output
+            self._dev_in = None
+            self.out = None
+            if self.csa:
+                # one eager pass of the selection kernels on the C step's own
+                # scratch (it changes nothing in the cache) does their one-time
+                # launch set-up (cluster-size query) outside the capture
+                d = self.views(self._dev_buf[: self.input_bytes])
+                ld = max(cache.cfg.max_pages_per_request * 128, 128)
+                o = self.input_bytes
+                scores = self._dev_buf[o: o + n * ld * 4].view(torch.float32).view(n, ld)
+                o += (n * ld * 4 + 255) // 256 * 256
+                nv = self._dev_buf[o: o + n * 4].view(torch.int32)
+                cache.index_scores(layer, self._req, d["q_idx"], d["w"], scores, nv)
+                topk(scores, nv, self.k, self.topk_idx)
+                torch.cuda.synchronize(dev)
+                cache.check_device_error()
+        if self.csa and self.fused_select:
             n_max = max(cache.cfg.max_pages_per_request * 128, 128)   # 512 tokens = 128 entries per page
             self._scores = torch.empty((n, n_max), dtype=torch.float32, device=dev)
             self._nv = torch.empty(n, dtype=torch.int32, device=dev)
             self._idx = torch.empty((n, self.k), dtype=torch.int32, device=dev)
-
-        if self.csa:
-            self._tk_ws = torch.empty(cache.index_topk_workspace_bytes(n, n_max) + 256, dtype=torch.uint8, device=dev)
-
-        def select():
-            # index scores and top-k in one launch (csa_index_topk)
-            cache.index_topk(layer, self._req, d["q_idx"], d["w"], self._scores, self._nv, self.k, self._idx,
-                             variant, workspace=self._tk_ws)
-
-        if self.csa:
+            self._tk_ws = torch.empty(cache.index_topk_workspace_bytes(n, n_max) + 256, dtype=torch.uint8,
+                                      device=dev)
             # one eager pass of the selection kernels (valid on any cache
             # state, an empty request included) does their one-time launch
             # set-up (cluster-size query) outside the capture
-            select()
+            self._select(self.views(self._dev_in))
             torch.cuda.synchronize(dev)
             cache.check_device_error()
-        self.graph_select = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph_select):
+        self.graph = self._capture(None)
+        self.marks = None
+        self._graph_marked = None
+        torch.cuda.synchronize(dev)
+
+    def _select(self, d) -> None:
+        cache, layer, variant = self.cache, self.layer, self.variant
+        if self.fused_select:           # index scores and top-k in one launch (csa_index_topk)
+            cache.index_topk(layer, self._req, d["q_idx"], d["w"], self._scores, self._nv, self.k, self._idx,
+                             variant, workspace=self._tk_ws)
+        else:                           # csa_index_scores, then csa_topk
+            cache.index_scores(layer, self._req, d["q_idx"], d["w"], self._scores, self._nv, variant)
+            topk(self._scores, self._nv, self.k, self._idx, variant)
+
+    def _step_c(self, stream) -> None:
+        c = self.cache
+        check(c.lib.csa_decode_step(c.handle, self.layer, self.n, self._req.data_ptr(), self.k if self.csa else 0,
+                                    self._sink.data_ptr(), 1.0 / float(np.sqrt(c.D)), self.host_in.data_ptr(),
+                                    self.host_out.data_ptr(), self._dev_buf.data_ptr(), self._dev_buf.numel(),
+                                    stream.cuda_stream), "csa_decode_step")
+
+    def _capture(self, marks):
+        """The step as one graph; `marks` (two external timing events) are
+        recorded after the inputs are on the device and after the attention
+        (the composed step) or before and after the whole C step."""
+        cache, layer = self.cache, self.layer
+        if not self.fused_select:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                main = torch.cuda.current_stream(self.device)
+                if marks is not None:
+                    marks[0].record(main)
+                self._step_c(main)
+                if marks is not None:
+                    marks[1].record(main)
+            return g
+        d = self.views(self._dev_in)
+        qo = self._q_off
+        ev_fork, ev_q = torch.cuda.Event(), torch.cuda.Event()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            main = torch.cuda.current_stream(self.device)
+            ev_fork.record(main)
+            self._side.wait_event(ev_fork)
+            with torch.cuda.stream(self._side):
+                self._dev_in[qo:].copy_(self.host_in[qo:], non_blocking=True)
+                ev_q.record(self._side)
+            self._dev_in[:qo].copy_(self.host_in[:qo], non_blocking=True)
+            if marks is not None:
+                marks[0].record(main)
             cache.compress_append(layer, self._req, d["c"], d["z"], d.get("ci"), d.get("zi"))
             if self.csa:
-                select()
-        self.graph_attn = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph_attn):
+                self._select(d)
+            main.wait_event(ev_q)
             cache.decode_attn(layer, self._req, d["q"], self._idx if self.csa else None, self._sink, self.out,
-                              variant=variant, workspace=self._ws, state_ready=self.csa)
-        torch.cuda.synchronize(dev)
+                              variant=self.variant, workspace=self._ws, state_ready=self.csa)
+            if marks is not None:
+                marks[1].record(main)
+            self.host_out.copy_(self.out, non_blocking=True)
+        return g
 
     def views(self, buf: torch.Tensor) -> dict:
         """Typed views of the step's input fields inside a packed buffer."""
@@ -354,46 +424,66 @@ class DecodeStep:
                 for name, dtype, shape, off, nbytes in self._fields}
 
     def new_host_inputs(self) -> torch.Tensor:
-        """A pinned host buffer for one step's packed inputs."""
+        """A pinned host buffer for one step's packed inputs (for callers
+        that keep their own buffers; see __call__)."""
         return torch.zeros(self.input_bytes, dtype=torch.uint8).pin_memory()
 
-    def __call__(self, host_inputs: torch.Tensor, marks=None) -> torch.Tensor:
-        """Enqueue one step on the current stream: copy the packed inputs in,
-        replay the step, copy the output [n, H, D] bf16 to `host_out` (pinned),
-        which is returned and is valid once the stream has reached this point
-        (the next call overwrites it).  The copies are asynchronous:
-        `host_inputs` must not change until the stream has passed them.
-        `marks`, two torch.cuda.Events, are recorded on the current stream
-        after the first input copy and after the second graph (to time the
-        three phases; the query's copy overlaps the first graph)."""
-        if host_inputs.device.type != "cpu" or not host_inputs.is_pinned():
-            raise ValueError("host_inputs must be a pinned host buffer (new_host_inputs())")
-        if host_inputs.dtype != torch.uint8 or host_inputs.numel() != self.input_bytes:
-            raise ValueError(f"host_inputs must be {self.input_bytes} bytes")
-        main = torch.cuda.current_stream(self.device)
-        qo = self._q_off
-        # the query's copy starts once everything queued before this step
-        # (the previous step's attention reads the same buffer) has run
-        self._ev_start.record(main)
-        self._side.wait_event(self._ev_start)
-        with torch.cuda.stream(self._side):
-            self._dev_in[qo:].copy_(host_inputs[qo:], non_blocking=True)
-            self._ev_q.record(self._side)
-        self._dev_in[:qo].copy_(host_inputs[:qo], non_blocking=True)
-        if marks is not None:
-            marks[0].record(main)
-        self.graph_select.replay()
-        main.wait_event(self._ev_q)
-        self.graph_attn.replay()
-        if marks is not None:
-            marks[1].record(main)
-        self.host_out.copy_(self.out, non_blocking=True)
+    def __call__(self, host_inputs: torch.Tensor | None = None, timed: bool = False) -> torch.Tensor:
+        """Enqueue one step on the current stream and return `host_out` (the
+        output [n, H, D], valid once the stream has reached the end of the
+        step; the next call overwrites it).
+
+        The step reads its inputs from `host_in`: fill it through
+        `views(step.host_in)` and call with no argument.  It must not change
+        until the step's copy has run (`ready()`).  A caller's own pinned
+        buffer may be passed instead: the call then waits for the previous
+        step and copies it into `host_in` on the host first.
+
+        timed=True replays a second capture of the step that records the
+        events `marks` (after the input copy, after the attention) for
+        timing the phases."""
+        if host_inputs is not None and host_inputs.data_ptr() != self.host_in.data_ptr():
+            if host_inputs.device.type != "cpu" or host_inputs.dtype != torch.uint8 \
+                    or host_inputs.numel() != self.input_bytes:
+                raise ValueError(f"host_inputs must be {self.input_bytes} bytes on the host")
+            self._done.synchronize()
+            self.host_in.copy_(host_inputs)
+        if timed:
+            if self._graph_marked is None:
+                self.marks = (torch.cuda.Event(enable_timing=True, external=True),
+                              torch.cuda.Event(enable_timing=True, external=True))
+                self._graph_marked = self._capture(self.marks)
+            self._graph_marked.replay()
+        else:
+            self.graph.replay()
+        self._done.record(torch.cuda.current_stream(self.device))
         return self.host_out
+
+    def ready(self) -> bool:
+        """Whether the last step has finished (host_in may be refilled)."""
+        return self._done.query()
 
     @property
     def topk_idx(self) -> torch.Tensor | None:
         """The last step's selected entries [n, k] (CSA layers)."""
-        return self._idx if self.csa else None
+        if not self.csa:
+            return None
+        if self.fused_select:
+            return self._idx
+        off = self._step_dev_offsets()["idx"]
+        return self._dev_buf[off: off + self.n * self.k * 4].view(torch.int32).view(self.n, self.k)
+
+    def _step_dev_offsets(self) -> dict:
+        """Byte offsets in the C step's device scratch (csa_decode_step's
+        layout: the inputs, scores [n][ld], counts [n], indices [n][k], the
+        attention workspace, the output; each on a 256-byte boundary)."""
+        al = lambda x: (x + 255) // 256 * 256
+        c = self.cache
+        o = self.input_bytes
+        ld = max(c.cfg.max_pages_per_request * 128, 128) if self.csa else 0
+        o += al(self.n * ld * 4)                 # scores
+        o += al(self.n * 4)                      # counts
+        return {"idx": o}
 
 
 # ---------------------------------------------------------------- host row formats

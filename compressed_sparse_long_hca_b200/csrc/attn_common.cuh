@@ -10,8 +10,8 @@
 // tile gives (m_t, l_t, O_t).  The tiles are grouped into chunks of C
 // consecutive tiles: the tiles of a chunk are folded in order into the
 // chunk's (m_c, l_c, O_c), then the chunks are folded in order, the sink
-// last.  C is fixed by the layer kind (attn_chunk_tiles), never by the
-// batch.  Both storage formats and both launch variants use the fold below,
+// last.  C follows from the layer kind and the query's own tile count
+// (attn_chunk_tiles), never from the batch.  Both storage formats and both launch variants use the fold below,
 // so that the order and the rounding of the reduction depend on the query
 // alone.
 #pragma once
@@ -23,11 +23,16 @@ constexpr int kTileRows = 128;
 constexpr int kFoldBatch = 9;      // partials loaded at once by the fold kernel (a top-1024 query's 9 tiles)
 
 // Tiles per chunk of the reduction: 1 on CSA layers (a top-k query has a
-// handful of tiles, each a unit of parallel work), 8 on HCA layers (a query
-// at 1M tokens has 65 tiles: a thread block folds a chunk's tiles on chip
-// and writes one partial per chunk).  A chunk of one tile is that tile's
-// partial exactly (folding into an empty result scales by e^0 = 1).
-__host__ __device__ inline int attn_chunk_tiles(bool csa) { return csa ? 1 : 8; }
+// handful of tiles, each a unit of parallel work); on HCA layers the
+// query's n_tiles are cut into at most kHcaChunks chunks of
+// ceil(n_tiles / kHcaChunks) tiles (a query at 1M tokens has 65 tiles: a
+// thread block folds 9 of them on chip and writes one partial).  A chunk of
+// one tile is that tile's partial exactly (folding into an empty result
+// scales by e^0 = 1).
+constexpr int kHcaChunks = 8;
+__host__ __device__ inline int attn_chunk_tiles(bool csa, int n_tiles) {
+  return csa ? 1 : (n_tiles + kHcaChunks - 1) / kHcaChunks > 1 ? (n_tiles + kHcaChunks - 1) / kHcaChunks : 1;
+}
 
 struct AttnArgs {
   Layout L;
@@ -82,7 +87,7 @@ __device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& 
   g.n_list = g.csa ? a.k : g.n_entries;
   g.total = g.n_list + g.n_win;
   g.n_tiles = (int)((g.total + kTileRows - 1) / kTileRows);
-  g.chunk = attn_chunk_tiles(g.csa);
+  g.chunk = attn_chunk_tiles(g.csa, g.n_tiles);
   g.n_chunks = (g.n_tiles + g.chunk - 1) / g.chunk;
   return true;
 }

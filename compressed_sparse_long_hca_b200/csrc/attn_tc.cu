@@ -445,6 +445,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     __syncthreads();
   };
 
+  // The next tile's rows are resolved and their loads issued (into buf) as
+  // soon as the current tile's PV is issued, so that they fly during the row
+  // sums, the PV and the fold; buf_tile is the tile whose loads buf holds.
+  uint4 buf[kMaxLoads];
+  int buf_tile = tt0;                                    // the first tile was gathered in the prologue
+  bool next_resolved = false;
   for (int tt = tt0; tt < tt_end && ok; ++tt) {
     if (two_level && tt > tt0 && tt % g.chunk == 0) {
       // a chunk ends before tile tt: its last tile and then the chunk fold in
@@ -463,16 +469,16 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       ok = __syncthreads_and(ok) != 0;
       if (!ok) break;
       tc::tc_fence_after();
-      // -- gather: issue every load of this thread first (the first tile
-      //    was gathered in the prologue)
+      // -- gather: the loads were issued with the previous tile, unless it
+      //    had no rows (the first tile was gathered in the prologue)
       const bool fetch = tt != tt0;
-      uint4 buf[kMaxLoads];
-      if (fetch) {
+      if (fetch && buf_tile != tt) {
 #pragma unroll
         for (int u = 0; u < kMaxLoads; ++u) {
           const int it = warp + 8 * u;
           buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
         }
+        buf_tile = tt;
       }
       // -- fold the previous tile while the loads fly
       if (pend_fold) fold_pending();
@@ -570,6 +576,22 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
         __syncwarp();
       }
       ++n_done;
+      // -- the next tile: rows resolved (the current tile no longer reads
+      //    them) and loads issued now
+      if (tt + 1 < tt_end) {
+        int nany = 0;
+        if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
+        tile_valid = __syncthreads_count(nany) > 0;
+        next_resolved = true;
+        if (tile_valid) {
+#pragma unroll
+          for (int u = 0; u < kMaxLoads; ++u) {
+            const int it = warp + 8 * u;
+            buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
+          }
+          buf_tile = tt + 1;
+        }
+      }
       // -- l_t: row sums of p per head, in a fixed order (warp tree, then the 4 row warps)
       if (tw) {
         const float sm_ = warp_reduce16<false>(pv, lane);
@@ -580,12 +602,13 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       pend_fold = true;
       chunk_has = true;
     }
-    // -- addresses of the next tile's rows
-    if (tt + 1 < tt_end) {
+    // -- addresses of the next tile's rows (after a tile without rows)
+    if (tt + 1 < tt_end && !next_resolved) {
       int nany = 0;
       if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
       tile_valid = __syncthreads_count(nany) > 0;
     }
+    next_resolved = false;
   }
 
   if (ok && n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
@@ -809,8 +832,8 @@ int attn_tiles_max(const Layout& L, int layer, int k) {
 }
 
 int attn_chunks_max(const Layout& L, int layer, int k) {
-  const int c = attn_chunk_tiles(layer < L.n_csa);
-  return (attn_tiles_max(L, layer, k) + c - 1) / c;
+  const int t = attn_tiles_max(L, layer, k);
+  return layer < L.n_csa ? t : (t < kHcaChunks ? t : kHcaChunks);
 }
 
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k) {

@@ -64,6 +64,14 @@ struct csa_cache {
   Layout L;
   std::vector<int32_t> free_pages;                // pool pages not held by a request
   std::vector<std::vector<int32_t>> req_pages;    // pages held by each request
+  // csa_decode_step: the query's copy runs on a second stream (fork / join events)
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_q = nullptr;
+  ~csa_cache() {
+    if (ev_q) cudaEventDestroy(ev_q);
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (side) cudaStreamDestroy(side);
+  }
 };
 
 namespace {
@@ -215,6 +223,12 @@ csa_status csa_cache_init(const csa_cfg* cfg, void* dev_mem, size_t bytes, const
   c->cfg = *cfg;
   c->L = L;
   c->req_pages.assign(cfg->max_requests, {});
+  if ((e = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&c->ev_fork, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&c->ev_q, cudaEventDisableTiming)) != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "stream / event creation");
+  }
   // Hand pool pages out in a fixed pseudo-random order, so that a request's
   // pages are scattered through the pool and every access goes through the
   // page table.
@@ -482,6 +496,108 @@ csa_status csa_check_device_error(csa_cache_t* c, csa_stream_t stream) {
 }
 
 const char* csa_last_error(void) { return g_err.c_str(); }
+
+// ---- one decode step with host buffers
+
+namespace {
+
+// Byte layout of csa_decode_step's packed host input and of its device
+// scratch (every field on a 256-byte boundary).
+struct StepLayout {
+  int64_t c, z, ci, zi, qi, w, q, q_bytes, in_bytes;            // host input (and its device copy)
+  int64_t d_scores, d_nv, d_idx, d_ws, d_out, out_bytes, dev_bytes, ld;
+  size_t ws_bytes;
+};
+
+StepLayout step_layout(const csa_cache* c, int32_t layer, int32_t n, int32_t k) {
+  const Layout& L = c->L;
+  const bool csa = layer < L.n_csa;
+  const int64_t qb = L.fmt == csa::kFmtF32 ? 4 : 2;
+  auto al = [](int64_t x) { return (x + 255) / 256 * 256; };
+  StepLayout s{};
+  int64_t o = 0;
+  s.c = o;  o += al((int64_t)n * L.D * 4);
+  s.z = o;  o += al((int64_t)n * L.D * 4);
+  if (csa) {
+    s.ci = o; o += al((int64_t)n * L.dI * 4);
+    s.zi = o; o += al((int64_t)n * L.dI * 4);
+    s.qi = o; o += al((int64_t)n * L.HI * L.dI * 4);
+    s.w = o;  o += al((int64_t)n * L.HI * 4);
+  }
+  s.q = o;
+  s.q_bytes = (int64_t)n * L.H * L.D * qb;
+  o += al(s.q_bytes);
+  s.in_bytes = o;
+  s.ld = csa ? std::max<int64_t>((int64_t)L.max_pages_per_req * csa::kCsaPerPage, 128) : 0;
+  s.d_scores = o; o += al((int64_t)n * s.ld * 4);
+  s.d_nv = o;     o += al((int64_t)n * 4);
+  s.d_idx = o;    o += al((int64_t)n * (csa ? k : 0) * 4);
+  s.ws_bytes = csa::attn_workspace_bytes(L, layer, n, csa ? k : 0);
+  s.d_ws = o;     o += al((int64_t)s.ws_bytes);
+  s.out_bytes = s.q_bytes;
+  s.d_out = o;    o += al(s.out_bytes);
+  s.dev_bytes = o;
+  return s;
+}
+
+}  // namespace
+
+size_t csa_decode_step_input_bytes(const csa_cache_t* c, int32_t layer, int32_t n) {
+  if (!layer_ok(c, layer) || n < 1 || n > 65535) return 0;
+  return (size_t)step_layout(c, layer, n, 1).in_bytes;
+}
+
+size_t csa_decode_step_dev_bytes(const csa_cache_t* c, int32_t layer, int32_t n, int32_t k) {
+  if (!layer_ok(c, layer) || n < 1 || n > 65535) return 0;
+  if (layer < c->L.n_csa && (k < 1 || k > 8192)) return 0;
+  return (size_t)step_layout(c, layer, n, k).dev_bytes;
+}
+
+csa_status csa_decode_step(csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids, int32_t k,
+                           const float* sink, float scale, const void* host_in, void* host_out, void* dev_buf,
+                           size_t dev_bytes, csa_stream_t stream) {
+  if (!layer_ok(c, layer)) return fail(CSA_ERR_ARG, "bad layer");
+  if (n < 1 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [1, 65535]");
+  const bool csa = layer < c->L.n_csa;
+  if (csa && (k < 1 || k > 8192)) return fail(CSA_ERR_ARG, "a CSA layer needs 1 <= k <= 8192");
+  if (!req_ids || !sink || !host_in || !host_out || !dev_buf) return fail(CSA_ERR_ARG, "NULL argument");
+  if (reinterpret_cast<uintptr_t>(dev_buf) % 256) return fail(CSA_ERR_ARG, "dev_buf must be 256-byte aligned");
+  const StepLayout sl = step_layout(c, layer, n, csa ? k : 0);
+  if (dev_bytes < (size_t)sl.dev_bytes) return fail(CSA_ERR_ARG, "dev_buf smaller than csa_decode_step_dev_bytes");
+  char* d = static_cast<char*>(dev_buf);
+  const char* h = static_cast<const char*>(host_in);
+  cudaStream_t st = (cudaStream_t)stream;
+  // inputs before q in one copy; q, which only the attention reads, on the
+  // cache's second stream beside the append and the selection
+  cudaError_t e = cudaMemcpyAsync(d, h, (size_t)sl.q, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(c->side, c->ev_fork, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d + sl.q, h + sl.q, (size_t)sl.q_bytes, cudaMemcpyHostToDevice, c->side);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_q, c->side);
+  if (e != cudaSuccess) return cuda_fail(e, "decode step input copies");
+  csa_status r = csa_compress_append(c, layer, n, req_ids, 1, reinterpret_cast<const float*>(d + sl.c),
+                                     reinterpret_cast<const float*>(d + sl.z),
+                                     csa ? reinterpret_cast<const float*>(d + sl.ci) : nullptr,
+                                     csa ? reinterpret_cast<const float*>(d + sl.zi) : nullptr, stream);
+  int32_t* idx = csa ? reinterpret_cast<int32_t*>(d + sl.d_idx) : nullptr;
+  if (r == CSA_OK && csa) {
+    float* scores = reinterpret_cast<float*>(d + sl.d_scores);
+    int32_t* nv = reinterpret_cast<int32_t*>(d + sl.d_nv);
+    r = csa_index_scores(c, layer, n, req_ids, reinterpret_cast<const float*>(d + sl.qi),
+                         reinterpret_cast<const float*>(d + sl.w), scores, sl.ld, nv, CSA_VARIANT_AUTO, stream);
+    if (r == CSA_OK) r = csa_topk(scores, sl.ld, nv, n, k, idx, CSA_VARIANT_AUTO, stream);
+  }
+  if (r != CSA_OK) return r;
+  e = cudaStreamWaitEvent(st, c->ev_q, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "decode step join");
+  r = csa_hca_decode_attn(c, layer, n, req_ids, d + sl.q, idx, csa ? k : 0, sink, scale, d + sl.d_out,
+                          d + sl.d_ws, sl.ws_bytes, (csa_variant)(CSA_VARIANT_AUTO | (csa ? CSA_ATTN_STATE_READY : 0)),
+                          stream);
+  if (r != CSA_OK) return r;
+  e = cudaMemcpyAsync(host_out, d + sl.d_out, (size_t)sl.out_bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode step output copy");
+  return CSA_OK;
+}
 
 // ---- batch-invariant projection GEMM
 

@@ -1032,6 +1032,10 @@ __global__ void __launch_bounds__(kThreads, kTopk ? 1 : 2) index_tc_kernel(Index
     g += pass_tiles;
     __syncthreads();
   }
+  // csa_index_scores: the next kernel on the stream (the top-k, launched with
+  // programmatic serialization) may start launching; it waits for this grid
+  // before reading the scores
+  if (!kTopk) tc::griddep_launch_dependents();
   if (warp == 1 && u_base > 0) {
     // every tcgen05 operation this CTA issued has finished before TMEM is released
     if (tc::elect_one()) tc::mma_commit(&sm.drain);

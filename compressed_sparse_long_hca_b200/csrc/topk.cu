@@ -369,6 +369,13 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kTopkThreads, 1) top
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const float* s = a.scores + (int64_t)i * a.ld;
   int32_t* out = a.out + (int64_t)i * a.k;
+  // Launched with programmatic serialization after the index kernel: the
+  // scores and counts are read only once that grid has completed.  The next
+  // kernel on the stream (the attention, launched the same way) may become
+  // resident and start what does not depend on the indices; it waits for
+  // this grid before reading them.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   int64_t N = a.n_valid[i];
   if (N < 0 || N > a.ld) {
     if (rank == 0 && tid == 0 && a.err) {
@@ -611,8 +618,19 @@ cudaError_t launch_topk_c(const TopkArgs& a, size_t sm, cudaStream_t st) {
     e = cudaFuncSetAttribute(topk_cluster_kernel<C>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  topk_cluster_kernel<C><<<dim3(C, a.n), kTopkThreads, sm, st>>>(a);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, a.n);
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<C>, a);
   note_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -292,10 +292,12 @@ csa_status csa_index_topk(const csa_cache_t* cache, int32_t layer, int32_t n,
  *
  * Reduction order: the rows are cut into tiles of 128; each tile yields
  * (max, sum of exponentials, weighted sum of V).  The tiles are grouped
- * into chunks of consecutive tiles (one tile per chunk on CSA layers, 8 on
- * HCA layers); the tiles of a chunk are folded in order into the chunk's
- * result and the chunk results are folded in order, the sink last.  The
- * order depends on the query and the layer kind alone, never on the batch.
+ * into chunks of consecutive tiles (one tile per chunk on CSA layers; on
+ * HCA layers a query's tiles are cut into at most 8 chunks of
+ * ceil(tiles / 8) tiles); the tiles of a chunk are folded in order into the
+ * chunk's result and the chunk results are folded in order, the sink last.
+ * The order depends on the query and the layer kind alone, never on the
+ * batch.
  *
  * Launch variants (page "DeepSeek不惜代价保住它！V4关键特性被挖出来了",
  * section "牺牲了什么": two decode-attention kernels for a well-fed and an
@@ -340,11 +342,9 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
  *     (4 D + 8) bytes; with H = 128 and D = 512 that allows
  *     n x chunks <= 63.  On CSA layers a chunk is one tile and chunks =
  *     ceil((k + 128) / 128) (k = 1024: up to 7 queries; 4 queries need about
- *     9.5 MiB).  On HCA layers a chunk is 8 tiles and, the host not knowing
- *     the lengths, the count follows the cache's capacity: chunks =
- *     ceil((ceil(P / 32) + 1) / 8) for P = max_pages_per_request; at H = 128,
- *     D = 512 a cache sized for 1M tokens (P = 2048, 9 chunks) fits up to 7
- *     queries, and one query fits up to P = 16,096 (8.2M tokens);
+ *     9.5 MiB).  On HCA layers a query has at most 8 chunks (fewer when the
+ *     cache's capacity holds fewer tiles), so at H = 128, D = 512 up to 7
+ *     queries fit whatever the capacity;
  *   - the first call on each device looks up the array's device address;
  *     make that first call before any stream capture;
  *   - all calls share the array: calls whose kernels may overlap on the GPU
@@ -357,6 +357,42 @@ csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* cache, int32_t layer, 
                                        const int32_t* req_ids, const void* q,
                                        const int32_t* topk_idx, int32_t k, const float* sink,
                                        float scale, void* out, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------
+ * One decode step with host buffers: the step's inputs are copied from host
+ * memory, the step runs, and its output is copied back to host memory, all
+ * on `stream`.  Source: the same four steps as above (page
+ * "V4终于终于终于终于是来了", sections "CSA——压缩稀疏注意力" and
+ * "HCA——重度压缩注意力"): csa_compress_append of one token, on a CSA layer
+ * csa_index_scores and csa_topk (variant AUTO), then csa_hca_decode_attn
+ * (variant AUTO, with CSA_ATTN_STATE_READY on a CSA layer).
+ *
+ *   host_in   pinned host buffer of csa_decode_step_input_bytes(cache,
+ *             layer, n) bytes holding, each field on a 256-byte boundary and
+ *             in this order:  c [n][D] fp32, z [n][D] fp32 (the token's KV
+ *             candidate and gate logits); on a CSA layer c_I [n][d_I] fp32,
+ *             z_I [n][d_I] fp32, q_I [n][H_I][d_I] fp32, w [n][H_I] fp32;
+ *             last q [n][H][D] (BF16, or fp32 in the fp32 format).
+ *   host_out  pinned host buffer [n][H][D], the type of q.
+ *   req_ids   device int32 [n]; sink device fp32 [H]; scale as for
+ *             csa_hca_decode_attn; k the top-k size (CSA layers, 1..8192).
+ *   dev_buf   caller device scratch of csa_decode_step_dev_bytes(cache,
+ *             layer, n, k) bytes, 256-byte aligned (the inputs' copy, the
+ *             scores, counts and indices, the attention workspace, the
+ *             output before its copy), owned by the caller.
+ * The inputs before q travel in one copy; q travels on a second stream owned
+ * by the cache, beside the append and the selection, and the attention
+ * waits for it.  The call is asynchronous: host_in must not change, and
+ * host_out must not be read, until the stream has passed the call.  It can
+ * be captured in a CUDA graph (the host pointers are then fixed).  Calls on
+ * one cache must not run concurrently from several host threads (the
+ * second stream is shared).  Errors: as the four calls it makes.
+ * ------------------------------------------------------------------- */
+size_t     csa_decode_step_input_bytes(const csa_cache_t* cache, int32_t layer, int32_t n);
+size_t     csa_decode_step_dev_bytes(const csa_cache_t* cache, int32_t layer, int32_t n, int32_t k);
+csa_status csa_decode_step(csa_cache_t* cache, int32_t layer, int32_t n, const int32_t* req_ids, int32_t k,
+                           const float* sink, float scale, const void* host_in, void* host_out,
+                           void* dev_buf, size_t dev_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------
  * Batch-invariant projection GEMM:  Y[t][o] = sum_k X[t][k] W[o][k]

@@ -117,3 +117,6 @@ def test_cache_calls_on_a_null_handle_fail_on_the_host(cuda_lib):
     assert cuda_lib.csa_request_free(None, 0) == -1
     assert cuda_lib.csa_check_device_error(None, None) == -1
     assert cuda_lib.csa_debug_wait_timeout(None, 1000, None) == -1
+    assert cuda_lib.csa_decode_step_input_bytes(None, 0, 1) == 0
+    assert cuda_lib.csa_decode_step_dev_bytes(None, 0, 1, 16) == 0
+    assert cuda_lib.csa_decode_step(None, 0, 1, P, 16, P, 1.0, P, P, P, 1 << 20, None) == -1

@@ -46,8 +46,11 @@ def _eager(pair, layer, reqs, k, sink, v):
     return out.cpu(), (idx.cpu() if idx is not None else None)
 
 
-@pytest.mark.parametrize("layer", [0, 1])
-def test_decode_step_graph_matches_individual_calls(layer):
+@pytest.mark.parametrize("layer,fused", [(0, False), (1, False), (0, True)])
+def test_decode_step_graph_matches_individual_calls(layer, fused):
+    """fused=False: the graph of one csa_decode_step call (host buffers);
+    fused=True: the step composed from csa_compress_append, csa_index_topk
+    and csa_hca_decode_attn."""
     from compressed_sparse_long_hca_b200.api import DecodeStep
     wl = I.Workload("step", "csa", H=16, D=128, R=32, H_I=8, d_I=64, k=40, W=128, context=0, batch=0,
                     seed=4242)
@@ -62,10 +65,14 @@ def test_decode_step_graph_matches_individual_calls(layer):
     torch.cuda.synchronize()
     csa = layer == 0
     sink = pairs[0].params[layer]["sink"]
-    step = DecodeStep(pairs[0].cache, layer, reqs, wl.k if csa else 0, sink)
+    step = DecodeStep(pairs[0].cache, layer, reqs, wl.k if csa else 0, sink, fused_select=fused)
     rng = np.random.default_rng(17)
     for s in range(n_steps):
-        buf = step.new_host_inputs()
+        # even steps: a caller's own pinned buffer (copied into the step's on
+        # the host); odd steps: the step's own buffer, filled in place, and
+        # the replay that records the phase marks
+        own = s % 2 == 1
+        buf = step.host_in if own else step.new_host_inputs()
         v = step.views(buf)
         q = I.bf16_grid(rng.standard_normal((3, wl.H, wl.D)).astype(np.float32))
         v["q"].copy_(torch.from_numpy(q).to(torch.bfloat16))
@@ -77,11 +84,13 @@ def test_decode_step_graph_matches_individual_calls(layer):
             v["zi"].copy_(torch.from_numpy(np.stack([toks[r][3] for r in reqs])))
             v["q_idx"].copy_(torch.from_numpy(rng.standard_normal((3, wl.H_I, wl.d_I)).astype(np.float32)))
             v["w"].copy_(torch.from_numpy(rng.standard_normal((3, wl.H_I)).astype(np.float32)))
-        got = step(buf)
+        got = step(None, timed=True) if own else step(buf)
         torch.cuda.synchronize()
+        if own:
+            assert step.marks[0].elapsed_time(step.marks[1]) > 0
+        got_idx = step.topk_idx.cpu() if csa else None
         pairs[0].cache.check_device_error()
         got = got.clone()
-        got_idx = step.topk_idx.cpu() if csa else None
         ref, ref_idx = _eager(pairs[1], layer, reqs, wl.k, sink, {nm: t.clone() for nm, t in v.items()})
         assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), f"step {s}: output differs"
         if csa:
@@ -114,7 +123,7 @@ def test_decode_step_graph_matches_individual_calls(layer):
             Hp.check_attention(got[i].float().numpy(), res["out"], f"request {r}")
 
 
-def test_decode_step_rejects_unpinned_or_mis_sized_inputs():
+def test_decode_step_rejects_mis_sized_or_device_inputs():
     from compressed_sparse_long_hca_b200.api import DecodeStep
     wl = I.Workload("step-args", "hca", H=8, D=64, R=16, H_I=0, d_I=0, k=0, W=128, context=0, batch=0,
                     seed=4243)
@@ -122,8 +131,10 @@ def test_decode_step_rejects_unpinned_or_mis_sized_inputs():
     pair.cache.request_alloc(0, 256)
     step = DecodeStep(pair.cache, 0, [0], 0, pair.params[0]["sink"])
     with pytest.raises(ValueError):
-        step(torch.zeros(step.input_bytes, dtype=torch.uint8))            # not pinned
+        step(torch.zeros(step.input_bytes, dtype=torch.uint8, device="cuda"))   # not a host buffer
     with pytest.raises(ValueError):
         step(torch.zeros(step.input_bytes + 16, dtype=torch.uint8).pin_memory())
+    step(torch.zeros(step.input_bytes, dtype=torch.uint8))                    # pageable: copied on the host
+    torch.cuda.synchronize()
     with pytest.raises(ValueError):
         DecodeStep(pair.cache, 0, [], 0, pair.params[0]["sink"])
