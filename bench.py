@@ -516,6 +516,60 @@ def rooflines(wl, m: dict, steps: int, select: str = "separate") -> dict:
     return out
 
 
+def measure_projections(steps: int = 10, n_tok: int = 4) -> dict:
+    """The projections around the decode step at the Pro-like shapes (hidden
+    7168, query latent 1024, 128 heads x 512, indexer 64 x 128, 16 output
+    groups of 1024), for a batch of `n_tok` tokens, through csa_gemm_bf16:
+    each call timed with CUDA events after an L2 flush, against the HBM
+    roofline (at decode batch sizes a projection streams its weight)."""
+    import torch
+
+    from compressed_sparse_long_hca_b200.api import Linear
+    d, D, dI, HI, dc, H, G, dg, dm = 7168, 512, 128, 64, 1024, 128, 16, 1024, 7168
+    shapes = [  # name, n_out, k_in, groups, output dtype
+        ("h -> c, z, c_I, z_I, w, c_q", 2 * D + 2 * dI + HI + dc, d, 1, torch.float32),
+        ("c_q -> q, q_I", H * D + HI * dI, dc, 1, torch.bfloat16),
+        ("attention -> grouped (16 x 1024)", G * dg, H * D, G, torch.bfloat16),
+        ("grouped -> model width", dm, G * dg, 1, torch.float32),
+    ]
+    rng = np.random.default_rng(2026)
+    peak, peak_kind, _ = _peaks()
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(256 * 2**20 // 4, dtype=torch.int32, device="cuda")
+    calls, total_us, total_bytes = {}, 0.0, 0
+    for name, n_out, k_in, groups, odt in shapes:
+        w = (rng.standard_normal((n_out, k_in // groups), dtype=np.float32) / np.float32(np.sqrt(k_in // groups)))
+        lin = Linear(w, groups=groups)
+        del w
+        x = torch.randn((n_tok, k_in), device="cuda").to(torch.bfloat16)
+        y = torch.empty((n_tok, n_out), dtype=odt, device="cuda")
+        lin(x, y)                               # warm-up (workspace, launch set-up)
+        torch.cuda.synchronize()
+        ms = 0.0
+        for _ in range(steps):
+            flush.zero_()
+            flush_rd.sum()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            lin(x, y)
+            b.record()
+            b.synchronize()
+            ms += a.elapsed_time(b)
+        Linear.check_device_error()
+        us = ms / steps * 1e3
+        nbytes = n_out * (k_in // groups) * 2 + n_tok * k_in * 2 + n_tok * n_out * y.element_size()
+        calls[name] = {"us": round(us, 2), "weight_mb": round(n_out * (k_in // groups) * 2 / 1e6, 1),
+                       "achieved_gbs": round(nbytes / (us / 1e6) / 1e9, 1),
+                       "frac": round(nbytes / (us / 1e6) / 1e9 / peak, 3)}
+        total_us += us
+        total_bytes += nbytes
+        del lin, x, y
+    return {"tokens": n_tok, "calls": calls, "total_us": round(total_us, 2),
+            "roofline": {"bound": "hbm", "achieved": total_bytes / (total_us / 1e6) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": total_bytes / (total_us / 1e6) / 1e9 / peak,
+                         "algorithmic_bytes": total_bytes, "peak_source": peak_kind}}
+
+
 # Configurations measured beside the headline at N = 1 (fewer steps each):
 # the tiny fp32 CSA layer, HCA at 128K (batch 32), CSA Flash-like at 128K
 # (batch 32) and the HCA layer at 1M (batch 4).
@@ -570,6 +624,9 @@ def run_gpu(args):
             rec.update(rooflines(wo, mo, o_steps, args.select))
             others[name] = rec
         line["other_workloads"] = others
+        gc.collect()
+        torch.cuda.empty_cache()
+        line["projections"] = measure_projections()
     if rank == 0 and args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if rank == 0:

@@ -23,15 +23,15 @@ constexpr int kTileRows = 128;
 constexpr int kFoldBatch = 9;      // partials loaded at once by the fold kernel (a top-1024 query's 9 tiles)
 
 // Tiles per chunk of the reduction: 1 on CSA layers (a top-k query has a
-// handful of tiles, each a unit of parallel work); on HCA layers the
-// query's n_tiles are cut into at most kHcaChunks chunks of
-// ceil(n_tiles / kHcaChunks) tiles (a query at 1M tokens has 65 tiles: a
-// thread block folds 9 of them on chip and writes one partial).  A chunk of
-// one tile is that tile's partial exactly (folding into an empty result
-// scales by e^0 = 1).
-constexpr int kHcaChunks = 8;
+// handful of tiles, each a unit of parallel work); on HCA layers
+// max(1, n_tiles / 8) for the query's own tile count, so that a short query
+// keeps one tile per chunk (its tiles run in parallel) and a long one folds
+// runs of tiles on chip (a query at 1M tokens: 65 tiles, 9 chunks of 8).  A
+// chunk of one tile is that tile's partial exactly (folding into an empty
+// result scales by e^0 = 1).
+constexpr int kHcaChunkDiv = 8;
 __host__ __device__ inline int attn_chunk_tiles(bool csa, int n_tiles) {
-  return csa ? 1 : (n_tiles + kHcaChunks - 1) / kHcaChunks > 1 ? (n_tiles + kHcaChunks - 1) / kHcaChunks : 1;
+  return csa ? 1 : (n_tiles / kHcaChunkDiv > 1 ? n_tiles / kHcaChunkDiv : 1);
 }
 
 struct AttnArgs {

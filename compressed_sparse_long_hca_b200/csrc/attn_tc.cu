@@ -833,7 +833,13 @@ int attn_tiles_max(const Layout& L, int layer, int k) {
 
 int attn_chunks_max(const Layout& L, int layer, int k) {
   const int t = attn_tiles_max(L, layer, k);
-  return layer < L.n_csa ? t : (t < kHcaChunks ? t : kHcaChunks);
+  if (layer < L.n_csa) return t;
+  int m = 0;                     // the most chunks any query of at most t tiles has
+  for (int n = 1; n <= t; ++n) {
+    const int c = attn_chunk_tiles(false, n);
+    m = (n + c - 1) / c > m ? (n + c - 1) / c : m;
+  }
+  return m;
 }
 
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k) {

@@ -292,9 +292,9 @@ csa_status csa_index_topk(const csa_cache_t* cache, int32_t layer, int32_t n,
  *
  * Reduction order: the rows are cut into tiles of 128; each tile yields
  * (max, sum of exponentials, weighted sum of V).  The tiles are grouped
- * into chunks of consecutive tiles (one tile per chunk on CSA layers; on
- * HCA layers a query's tiles are cut into at most 8 chunks of
- * ceil(tiles / 8) tiles); the tiles of a chunk are folded in order into the
+ * into chunks of consecutive tiles (one tile per chunk on CSA layers,
+ * max(1, floor(tiles / 8)) on HCA layers for the query's own tile count);
+ * the tiles of a chunk are folded in order into the
  * chunk's result and the chunk results are folded in order, the sink last.
  * The order depends on the query and the layer kind alone, never on the
  * batch.
@@ -342,9 +342,9 @@ csa_status csa_hca_decode_attn(const csa_cache_t* cache, int32_t layer, int32_t 
  *     (4 D + 8) bytes; with H = 128 and D = 512 that allows
  *     n x chunks <= 63.  On CSA layers a chunk is one tile and chunks =
  *     ceil((k + 128) / 128) (k = 1024: up to 7 queries; 4 queries need about
- *     9.5 MiB).  On HCA layers a query has at most 8 chunks (fewer when the
- *     cache's capacity holds fewer tiles), so at H = 128, D = 512 up to 7
- *     queries fit whatever the capacity;
+ *     9.5 MiB).  On HCA layers a query has at most 15 chunks (fewer when
+ *     the cache's capacity holds fewer than 15 tiles), so at H = 128,
+ *     D = 512 up to 4 queries fit whatever the capacity;
  *   - the first call on each device looks up the array's device address;
  *     make that first call before any stream capture;
  *   - all calls share the array: calls whose kernels may overlap on the GPU

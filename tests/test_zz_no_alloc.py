@@ -107,14 +107,15 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
 
 
 def test_noalloc_hca_limit_follows_the_cache_capacity():
-    """On an HCA layer a query's tiles are cut into at most 8 chunks, one
-    partial each, so at H = 128, D = 512 the scratch fits 7 queries and not 8
-    whatever the cache's capacity (2048 pages = 1M tokens, or 16,128); a
-    batch that does not fit is refused before any launch."""
+    """On an HCA layer a query's tiles are cut into chunks of
+    max(1, tiles / 8), at most 15 chunks for any length, one partial each,
+    so at H = 128, D = 512 the scratch fits 4 queries and not 5 whatever the
+    cache's capacity (2048 pages = 1M tokens, or 16,128); a batch that does
+    not fit is refused before any launch."""
     wl = I.Workload("noalloc-hca", "hca", H=128, D=512, R=64, H_I=0, d_I=0, k=0, W=128, context=0,
                     batch=0, seed=779)
     sink = torch.zeros(wl.H, device="cuda")
-    for pages, n, expect in ((2048, 7, True), (2048, 8, False), (16128, 7, True), (16128, 8, False)):
+    for pages, n, expect in ((2048, 4, True), (2048, 5, False), (16128, 4, True), (16128, 5, False)):
         pair = Hp.Pair(wl, 0, 1, max_req=1, capacity=pages * 512)
         fits = pair.cache.attn_workspace_bytes(0, n, 0) <= 16 << 20
         assert fits == expect, (pages, n, pair.cache.attn_workspace_bytes(0, n, 0))
