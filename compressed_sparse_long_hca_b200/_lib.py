@@ -59,6 +59,9 @@ SIGNATURES = {
     "csa_decode_step_input_bytes": (_SZ, [_P, _I32, _I32]),
     "csa_decode_step_dev_bytes": (_SZ, [_P, _I32, _I32, _I32]),
     "csa_decode_step": (_I32, [_P, _I32, _I32, _P, _I32, _P, _F, _P, _P, _P, _SZ, _P]),
+    "csa_prefill_workspace_bytes": (_SZ, [_P, _I32, _I32, _I32, _I32, _I32]),
+    "csa_prefill_chunk": (_I32, [_P, _I32, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _F, _P, _P, _P,
+                                 _SZ, _I32, _P]),
     "csa_gemm_weight_bytes": (_SZ, [_I32, _I32, _I32]),
     "csa_gemm_pack_weight": (_I32, [_P, _I32, _I32, _I32, _P, _SZ]),
     "csa_gemm_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I32]),

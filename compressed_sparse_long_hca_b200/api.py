@@ -203,6 +203,59 @@ class Cache:
                                            k, _ptr(sink), scale, _ptr(out), ws_ptr, ws_bytes,
                                            VARIANTS[variant] | flags, _stream(stream)), "csa_hca_decode_attn")
 
+    def prefill_workspace_bytes(self, layer: int, n: int, n_tok: int, k: int = 0, variant="auto") -> int:
+        return int(self.lib.csa_prefill_workspace_bytes(self.handle, layer, n, n_tok, k, VARIANTS[variant]))
+
+    def prefill_chunk(self, layer: int, req_ids, kv_cand, kv_gate, idx_cand, idx_gate, q, q_idx, w, k: int,
+                      sink, out, topk_out=None, scale=None, variant="auto", stream=None,
+                      workspace: torch.Tensor | None = None) -> None:
+        """A chunk of n_tok (1 .. 128) new tokens per request, each also a
+        query with causal visibility (csa_prefill_chunk): the tokens are
+        appended, and query j of request b (at position len - n_tok + j)
+        attends to what a decode query there would.  kv_cand, kv_gate
+        [n, n_tok, D] fp32; idx_cand, idx_gate [n, n_tok, d_I] fp32, q_idx
+        [n, n_tok, H_I, d_I] and w [n, n_tok, H_I] fp32 (CSA layers, else
+        None); q and out [n, n_tok, H, D] (BF16, fp32 in the fp32 format);
+        topk_out [n, n_tok, k] int32 or None.  Unless `workspace` is given, a
+        buffer owned by this Cache object is grown to the size the library
+        asks for."""
+        n = req_ids.numel()
+        _need(req_ids, torch.int32, name="req_ids")
+        n_tok = kv_cand.shape[1] if kv_cand.dim() == 3 else -1
+        _need(kv_cand, torch.float32, (n, n_tok, self.D), "kv_cand")
+        _need(kv_gate, torch.float32, (n, n_tok, self.D), "kv_gate")
+        _need(q, self.qdtype, (n, n_tok, self.H, self.D), "q")
+        _need(out, self.qdtype, (n, n_tok, self.H, self.D), "out")
+        _need(sink, torch.float32, (self.H,), "sink")
+        csa = layer < self.n_csa
+        if csa:
+            _need(idx_cand, torch.float32, (n, n_tok, self.d_I), "idx_cand")
+            _need(idx_gate, torch.float32, (n, n_tok, self.d_I), "idx_gate")
+            _need(q_idx, torch.float32, (n, n_tok, self.H_I, self.d_I), "q_idx")
+            _need(w, torch.float32, (n, n_tok, self.H_I), "w")
+            if topk_out is not None:
+                _need(topk_out, torch.int32, (n, n_tok, k), "topk_out")
+        else:
+            k = 0
+        if scale is None:
+            scale = 1.0 / float(np.sqrt(self.D))
+        need = self.prefill_workspace_bytes(layer, n, n_tok, k, variant)
+        if need == 0:
+            raise ValueError("invalid chunk shape (n_tok must be in [1, 128], n * n_tok <= 65535)")
+        if workspace is None:
+            ws = getattr(self, "_pf_ws", None)
+            if ws is None or ws.numel() < need + 256 or ws.device != q.device:
+                ws = torch.empty(need + 256, dtype=torch.uint8, device=q.device)
+                self._pf_ws = ws
+            workspace = ws
+        _need(workspace, torch.uint8, name="workspace")
+        ws_ptr = (workspace.data_ptr() + 255) // 256 * 256
+        ws_bytes = workspace.numel() - (ws_ptr - workspace.data_ptr())
+        check(self.lib.csa_prefill_chunk(self.handle, layer, n, _ptr(req_ids), n_tok, _ptr(kv_cand), _ptr(kv_gate),
+                                         _ptr(idx_cand), _ptr(idx_gate), _ptr(q), _ptr(q_idx), _ptr(w), k,
+                                         _ptr(sink), scale, _ptr(out), _ptr(topk_out), ws_ptr, ws_bytes,
+                                         VARIANTS[variant], _stream(stream)), "csa_prefill_chunk")
+
     def check_device_error(self, stream=None) -> None:
         check(self.lib.csa_check_device_error(self.handle, _stream(stream)), "device")
 

@@ -393,4 +393,27 @@ cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_
   return cudaGetLastError();
 }
 
+// Set-up of a chunk of queries (csa_prefill_chunk), before the chunk's
+// append: block b copies request req_ids[b]'s window ring (the rows the
+// append is about to overwrite are still the pre-chunk ones) to
+// snap + b * ring_bytes and writes the request id once per query of the
+// chunk into req_exp[b * n_tok .. b * n_tok + n_tok - 1].
+__global__ void __launch_bounds__(256) chunk_prep_kernel(Layout L, int layer, const int32_t* req_ids, int n_tok,
+                                                       int32_t* req_exp, char* snap) {
+  const int b = blockIdx.x;
+  const int req = req_ids[b];
+  for (int j = threadIdx.x; j < n_tok; j += blockDim.x) req_exp[(int64_t)b * n_tok + j] = req;
+  if (req < 0 || req >= L.max_req) return;       // the append reports the bad id
+  const uint4* src = reinterpret_cast<const uint4*>(L.state(req, layer));
+  uint4* dst = reinterpret_cast<uint4*>(snap + (int64_t)b * L.ring_bytes);
+  for (int64_t x = threadIdx.x; x < L.ring_bytes / 16; x += blockDim.x) dst[x] = src[x];
+}
+
+cudaError_t launch_chunk_prep(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok, int32_t* req_exp,
+                              char* snap, cudaStream_t st) {
+  chunk_prep_kernel<<<n, 256, 0, st>>>(L, layer, req_ids, n_tok, req_exp, snap);
+  note_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace csa

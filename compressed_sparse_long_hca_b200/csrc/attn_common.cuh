@@ -55,11 +55,20 @@ struct AttnArgs {
   // on the stream ends (that grid writes none of them): they may be read
   // before griddepcontrol.wait.  Top-k lists and compressed entries never are.
   int state_ready;
+  // Chunk queries (q_per_req = C > 0, see visible_tokens): the C latest
+  // tokens of each request were appended together, which overwrote the ring
+  // rows of the C oldest window positions.  win_snap holds, per request of
+  // the chunk (query i: request slot i / C), a copy of its ring taken before
+  // that append; window positions below len - 128 are read from the copy.
+  int q_per_req;
+  const char* win_snap;
 };
 
 struct QueryGeom {
   int req;
   bool csa;
+  int64_t len;        // tokens of the request (the chunk included)
+  const char* snap;   // chunk queries: the request's ring before the chunk's append
   int64_t t;          // query position
   int64_t n_entries, w0, n_win, n_list, total;
   int n_tiles;
@@ -75,11 +84,14 @@ __device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& 
     return false;
   }
   g.csa = a.layer < L.n_csa;
-  const int64_t T = L.lengths()[(int64_t)a.layer * L.max_req + g.req];
+  g.len = L.lengths()[(int64_t)a.layer * L.max_req + g.req];
+  const int64_t T = visible_tokens(g.len, a.q_per_req, i);
   if (T <= 0) {
     if (report) set_err(L, kErrBounds, 1000000 + i);
     return false;
   }
+  g.snap = (a.q_per_req > 0 && a.win_snap != nullptr) ? a.win_snap + (int64_t)(i / a.q_per_req) * L.ring_bytes
+                                                      : nullptr;
   g.t = T - 1;
   g.n_entries = g.csa ? T / kCsaM : T / kHcaM;
   g.w0 = g.t - (kWindow - 1) > 0 ? g.t - (kWindow - 1) : 0;
@@ -90,6 +102,16 @@ __device__ __forceinline__ bool query_geom(const AttnArgs& a, int i, QueryGeom& 
   g.chunk = attn_chunk_tiles(g.csa, g.n_tiles);
   g.n_chunks = (g.n_tiles + g.chunk - 1) / g.chunk;
   return true;
+}
+
+// Base of the window ring that holds position p (a window position of the
+// query): the request's ring, or for a chunk query a position the chunk's
+// own append has overwritten there, the copy taken before it.  The ring
+// keeps positions len - 128 .. len - 1; the copy keeps the 128 positions
+// before the chunk, which cover the rest of every window of a chunk of at
+// most 128 queries.
+__device__ __forceinline__ const char* ring_base(const AttnArgs& a, const QueryGeom& g, int64_t p) {
+  return (g.snap != nullptr && p < g.len - kWindow) ? g.snap : a.L.state(g.req, a.layer);
 }
 
 // The fold of one partial into a running (m, l, O); shared by both launch

@@ -72,7 +72,10 @@ __device__ __forceinline__ const float* f32_row(const AttnArgs& a, const QueryGe
     }
     return j >= 0 ? L.entry_row_f32(g.req, a.layer, j) : nullptr;
   }
-  if (rr < g.total) return L.ring_row_f32(g.req, a.layer, (int)((g.w0 + (rr - g.n_list)) % kWindow));
+  if (rr < g.total) {
+    const int64_t p = g.w0 + (rr - g.n_list);
+    return reinterpret_cast<const float*>(ring_base(a, g, p)) + (p % kWindow) * L.D;
+  }
   return nullptr;
 }
 
@@ -292,9 +295,10 @@ __global__ void __launch_bounds__(kF32Threads) attn_f32_kernel(AttnArgs a) {
 
 cudaError_t launch_attn_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q,
                             const int32_t* topk, int k, const float* sink, float scale, float* out, void* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, int q_per_req, const char* win_snap) {
   const size_t sm = (size_t)f32_smem(L.D).total;
-  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, kF32Heads, nullptr, nullptr, 0, 1};
+  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, kF32Heads, nullptr, nullptr, 0, 1, 0,
+             q_per_req, win_snap};
   const int n_hg = (L.H + kF32Heads - 1) / kF32Heads;
   if (ws == nullptr) {
     cudaError_t e = cudaFuncSetAttribute(attn_f32_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

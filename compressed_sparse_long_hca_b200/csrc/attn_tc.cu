@@ -141,8 +141,9 @@ __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& 
       sc = reinterpret_cast<const float*>(pp + (g.csa ? L.pg_csa_scale : L.pg_hca_scale))[s];
     }
   } else if (rr < g.total) {
-    const char* st = L.state(g.req, a.layer);
-    const int slot = (int)((g.w0 + (rr - g.n_list)) % kWindow);
+    const int64_t p = g.w0 + (rr - g.n_list);
+    const char* st = ring_base(a, g, p);
+    const int slot = (int)(p % kWindow);
     f8 = reinterpret_cast<const uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (L.D - L.R);
     bf = reinterpret_cast<const uint16_t*>(st + L.ring_bf16) + (int64_t)slot * L.R;
     sc = reinterpret_cast<const float*>(st + L.ring_scale)[slot];
@@ -849,11 +850,12 @@ size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k) {
 
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
-                           void* ws, cudaStream_t st, bool state_ready) {
+                           void* ws, cudaStream_t st, bool state_ready, int q_per_req, const char* win_snap) {
   const size_t sm = attn_tc_smem_bytes(L.D, G);
   if (sm > 227 * 1024) return cudaErrorInvalidValue;
   const bool split = ws != nullptr;
-  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0, 0, state_ready ? 1 : 0};
+  AttnArgs a{L, layer, n, req_ids, q, topk, k, sink, scale, out, G, nullptr, nullptr, 0, 0, state_ready ? 1 : 0,
+             q_per_req, win_snap};
   const int n_hg = (L.H + G - 1) / G;
   // programmatic dependent launch: the kernel may start before the previous
   // grid on the stream ends and waits for it (griddepcontrol) where it must

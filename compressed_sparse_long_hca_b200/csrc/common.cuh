@@ -25,6 +25,16 @@ __device__ __forceinline__ void set_err(const Layout& L, int32_t code, int32_t d
   if (atomicCAS(e, 0, code) == 0) e[1] = detail;
 }
 
+// Tokens visible to query i of a launch (causal visibility).  A decode
+// launch (q_per_req == 0): query i is its request's latest token and sees
+// the request's whole length.  A chunk of queries (q_per_req = C > 0): the
+// queries come in runs of C per request, in position order, for the
+// request's C latest tokens, so query i sits at position len - C + i % C and
+// sees the tokens up to and including its own.
+__device__ __forceinline__ int64_t visible_tokens(int64_t len, int q_per_req, int i) {
+  return q_per_req > 0 ? len - q_per_req + (i % q_per_req) + 1 : len;
+}
+
 __device__ __forceinline__ uint8_t e4m3_rn(float y) {
   return (uint8_t)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
 }

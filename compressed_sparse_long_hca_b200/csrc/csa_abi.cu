@@ -20,12 +20,13 @@ cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_
                           cudaStream_t st);
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
-                            cudaStream_t st);
+                            cudaStream_t st, int q_per_req = 0);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st);
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
-                           void* ws, cudaStream_t st, bool state_ready = false);
+                           void* ws, cudaStream_t st, bool state_ready = false, int q_per_req = 0,
+                           const char* win_snap = nullptr);
 size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k);
 size_t attn_noalloc_scratch_bytes();
 cudaError_t attn_noalloc_scratch(void** out);
@@ -36,10 +37,12 @@ cudaError_t launch_index_topk(const Layout& L, int layer, int n, const int32_t* 
                               void* ws, int ctas, cudaStream_t st);
 cudaError_t launch_index_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                              const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas_per_query,
-                             cudaStream_t st);
+                             cudaStream_t st, int q_per_req = 0);
 cudaError_t launch_attn_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q,
                             const int32_t* topk, int k, const float* sink, float scale, float* out, void* ws,
-                            cudaStream_t st);
+                            cudaStream_t st, int q_per_req = 0, const char* win_snap = nullptr);
+cudaError_t launch_chunk_prep(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok, int32_t* req_exp,
+                              char* snap, cudaStream_t st);
 int gemm_row_tiles(int n_out);
 int gemm_k_tiles(int k_in, int groups);
 size_t gemm_weight_bytes(int n_out, int k_in, int groups);
@@ -300,9 +303,17 @@ csa_status csa_compress_append(csa_cache_t* c, int32_t layer, int32_t n, const i
   return CSA_OK;
 }
 
-csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
-                            const float* q_idx, const float* w, float* scores, int64_t ld,
-                            int32_t* n_valid, csa_variant variant, csa_stream_t stream) {
+// Chunk queries (csa_prefill_chunk): q_per_req queries per request for its
+// latest tokens, and the copy of each request's ring taken before the
+// chunk's append.  Zero for decode queries.
+struct ChunkQ {
+  int q_per_req;
+  const char* snap;
+};
+
+static csa_status index_scores_impl(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                                    const float* q_idx, const float* w, float* scores, int64_t ld,
+                                    int32_t* n_valid, csa_variant variant, csa_stream_t stream, ChunkQ cq) {
   if (!layer_ok(c, layer) || layer >= c->L.n_csa) return fail(CSA_ERR_ARG, "index scores need a CSA layer");
   if (n < 0 || n > 65535) return fail(CSA_ERR_ARG, "n must be in [0, 65535]");
   if (n == 0) return CSA_OK;
@@ -318,15 +329,21 @@ csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, cons
     const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < sms);
     const int per_q = low ? std::max(1, (4 * sms + n - 1) / n) : 1;
     e = csa::launch_index_f32(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, std::min(per_q, 1024),
-                              (cudaStream_t)stream);
+                              (cudaStream_t)stream, cq.q_per_req);
   } else {
     // Two persistent CTAs per SM for either variant; the per-key arithmetic
     // does not depend on the grid.
     e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, 2 * sms,
-                             (cudaStream_t)stream);
+                             (cudaStream_t)stream, cq.q_per_req);
   }
   if (e != cudaSuccess) return cuda_fail(e, "index launch");
   return CSA_OK;
+}
+
+csa_status csa_index_scores(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                            const float* q_idx, const float* w, float* scores, int64_t ld,
+                            int32_t* n_valid, csa_variant variant, csa_stream_t stream) {
+  return index_scores_impl(c, layer, n, req_ids, q_idx, w, scores, ld, n_valid, variant, stream, ChunkQ{0, nullptr});
 }
 
 csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int32_t n, int32_t k,
@@ -386,10 +403,17 @@ size_t csa_attn_workspace_bytes(const csa_cache_t* c, int32_t layer, int32_t n, 
   return csa::attn_workspace_bytes(c->L, layer, n, is_csa ? k : 0);
 }
 
-csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
-                               const void* q, const int32_t* topk_idx, int32_t k, const float* sink,
-                               float scale, void* out, void* workspace, size_t workspace_bytes,
-                               csa_variant variant_flags, csa_stream_t stream) {
+// Whether a launch of n queries takes the split attention (with a workspace).
+static bool attn_split(const Layout& L, int32_t n, csa_variant variant, bool ws_ok) {
+  const int G = L.H <= 16 ? 16 : 32;
+  const int ctas = n * ((L.H + G - 1) / G);
+  return variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && ws_ok && ctas < sm_count());
+}
+
+static csa_status decode_attn_impl(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                                   const void* q, const int32_t* topk_idx, int32_t k, const float* sink,
+                                   float scale, void* out, void* workspace, size_t workspace_bytes,
+                                   csa_variant variant_flags, csa_stream_t stream, ChunkQ cq) {
   const int flags = (int)variant_flags & ~0xFF;
   const csa_variant variant = (csa_variant)((int)variant_flags & 0xFF);
   if (flags & ~CSA_ATTN_STATE_READY) return fail(CSA_ERR_ARG, "unknown variant flag");
@@ -414,18 +438,25 @@ csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, c
   // (query, head group) already covers the SMs, split launch otherwise.  Both
   // compute the same tiles and fold them in the same order.
   const int G = c->L.H <= 16 ? 16 : 32;
-  const int ctas = n * ((c->L.H + G - 1) / G);
-  const bool split = variant == CSA_VARIANT_LOW_OCC ||
-                     (variant == CSA_VARIANT_AUTO && ws_ok && ctas < sm_count());
+  const bool split = attn_split(c->L, n, variant, ws_ok);
   cudaError_t e =
       c->L.fmt == csa::kFmtF32
           ? csa::launch_attn_f32(c->L, layer, n, req_ids, static_cast<const float*>(q), topk_idx, kk, sink, scale,
-                                 static_cast<float*>(out), split ? workspace : nullptr, (cudaStream_t)stream)
+                                 static_cast<float*>(out), split ? workspace : nullptr, (cudaStream_t)stream,
+                                 cq.q_per_req, cq.snap)
           : csa::launch_attn_tc(c->L, layer, n, req_ids, static_cast<const uint16_t*>(q), topk_idx, kk, sink,
                                 scale, static_cast<uint16_t*>(out), G, split ? workspace : nullptr,
-                                (cudaStream_t)stream, (flags & CSA_ATTN_STATE_READY) != 0);
+                                (cudaStream_t)stream, (flags & CSA_ATTN_STATE_READY) != 0, cq.q_per_req, cq.snap);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return CSA_OK;
+}
+
+csa_status csa_hca_decode_attn(const csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids,
+                               const void* q, const int32_t* topk_idx, int32_t k, const float* sink,
+                               float scale, void* out, void* workspace, size_t workspace_bytes,
+                               csa_variant variant_flags, csa_stream_t stream) {
+  return decode_attn_impl(c, layer, n, req_ids, q, topk_idx, k, sink, scale, out, workspace, workspace_bytes,
+                          variant_flags, stream, ChunkQ{0, nullptr});
 }
 
 csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* c, int32_t layer, int32_t n,
@@ -599,10 +630,96 @@ csa_status csa_decode_step(csa_cache_t* c, int32_t layer, int32_t n, const int32
   return CSA_OK;
 }
 
+// ---- a chunk of queries with causal visibility (prefill)
+
+namespace {
+
+struct ChunkLayout {
+  int64_t snap, req, scores, nv, idx, ws, total, ld;
+  size_t ws_bytes;
+};
+
+ChunkLayout chunk_layout(const csa_cache* c, int32_t layer, int32_t n, int32_t n_tok, int32_t k, csa_variant variant) {
+  const Layout& L = c->L;
+  const bool csa = layer < L.n_csa;
+  const int64_t Q = (int64_t)n * n_tok;
+  auto al = [](int64_t x) { return (x + 255) / 256 * 256; };
+  ChunkLayout s{};
+  int64_t o = 0;
+  s.snap = o;   o += al((int64_t)n * L.ring_bytes);
+  s.req = o;    o += al(Q * 4);
+  s.ld = csa ? std::max<int64_t>((int64_t)L.max_pages_per_req * csa::kCsaPerPage, 128) : 0;
+  s.scores = o; o += al(Q * s.ld * 4);
+  s.nv = o;     o += al(csa ? Q * 4 : 0);
+  s.idx = o;    o += al(csa ? Q * k * 4 : 0);
+  s.ws_bytes = attn_split(L, (int32_t)Q, variant, true) ? csa::attn_workspace_bytes(L, layer, (int)Q, csa ? k : 0) : 0;
+  s.ws = o;     o += al((int64_t)s.ws_bytes);
+  s.total = o;
+  return s;
+}
+
+bool chunk_shape_ok(const csa_cache* c, int32_t layer, int32_t n, int32_t n_tok, int32_t k, csa_variant variant,
+                    std::string* why) {
+  if (!layer_ok(c, layer)) { *why = "bad layer"; return false; }
+  if (n < 1 || n > 65535) { *why = "n must be in [1, 65535]"; return false; }
+  if (n_tok < 1 || n_tok > csa::kWindow) { *why = "n_tok must be in [1, 128]"; return false; }
+  if ((int64_t)n * n_tok > 65535) { *why = "n * n_tok must be <= 65535"; return false; }
+  if (layer < c->L.n_csa && (k < 1 || k > 8192)) { *why = "a CSA layer needs 1 <= k <= 8192"; return false; }
+  if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) { *why = "bad variant"; return false; }
+  return true;
+}
+
+}  // namespace
+
+size_t csa_prefill_workspace_bytes(const csa_cache_t* c, int32_t layer, int32_t n, int32_t n_tok, int32_t k,
+                                   csa_variant variant) {
+  std::string why;
+  if (!chunk_shape_ok(c, layer, n, n_tok, k, variant, &why)) return 0;
+  return (size_t)chunk_layout(c, layer, n, n_tok, layer < c->L.n_csa ? k : 0, variant).total;
+}
+
+csa_status csa_prefill_chunk(csa_cache_t* c, int32_t layer, int32_t n, const int32_t* req_ids, int32_t n_tok,
+                             const float* kv_cand, const float* kv_gate, const float* idx_cand,
+                             const float* idx_gate, const void* q, const float* q_idx, const float* w, int32_t k,
+                             const float* sink, float scale, void* out, int32_t* topk_out, void* workspace,
+                             size_t workspace_bytes, csa_variant variant, csa_stream_t stream) {
+  std::string why;
+  if (!chunk_shape_ok(c, layer, n, n_tok, k, variant, &why)) return fail(CSA_ERR_ARG, why);
+  const bool csa = layer < c->L.n_csa;
+  if (!req_ids || !kv_cand || !kv_gate || !q || !sink || !out || !workspace) return fail(CSA_ERR_ARG, "NULL argument");
+  if (csa && (!idx_cand || !idx_gate || !q_idx || !w)) return fail(CSA_ERR_ARG, "a CSA layer needs the index inputs");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(CSA_ERR_ARG, "workspace must be 256-byte aligned");
+  const int kk = csa ? k : 0;
+  const ChunkLayout cl = chunk_layout(c, layer, n, n_tok, kk, variant);
+  if (workspace_bytes < (size_t)cl.total) return fail(CSA_ERR_ARG, "workspace smaller than csa_prefill_workspace_bytes");
+  const int32_t Q = n * n_tok;
+  char* ws = static_cast<char*>(workspace);
+  char* snap = ws + cl.snap;
+  int32_t* req_exp = reinterpret_cast<int32_t*>(ws + cl.req);
+  // the rings as they are before the chunk, and one request id per query
+  cudaError_t e = csa::launch_chunk_prep(c->L, layer, n, req_ids, n_tok, req_exp, snap, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk set-up launch");
+  csa_status r = csa_compress_append(c, layer, n, req_ids, n_tok, kv_cand, kv_gate, idx_cand, idx_gate, stream);
+  if (r != CSA_OK) return r;
+  const ChunkQ cq{n_tok, snap};
+  int32_t* idx = nullptr;
+  if (csa) {
+    idx = topk_out ? topk_out : reinterpret_cast<int32_t*>(ws + cl.idx);
+    float* scores = reinterpret_cast<float*>(ws + cl.scores);
+    int32_t* nv = reinterpret_cast<int32_t*>(ws + cl.nv);
+    r = index_scores_impl(c, layer, Q, req_exp, q_idx, w, scores, cl.ld, nv, variant, stream, cq);
+    if (r == CSA_OK) r = csa_topk(scores, cl.ld, nv, Q, k, idx, variant, stream);
+    if (r != CSA_OK) return r;
+  }
+  return decode_attn_impl(c, layer, Q, req_exp, q, idx, kk, sink, scale, out, cl.ws_bytes ? ws + cl.ws : nullptr,
+                          cl.ws_bytes, variant, stream, cq);
+}
+
 // ---- batch-invariant projection GEMM
 
 static bool gemm_shape_ok(int32_t n_out, int32_t k_in, int32_t groups, std::string* why) {
   if (n_out < 1 || k_in < 1 || groups < 1) { *why = "n_out, k_in and groups must be >= 1"; return false; }
+  if (groups > 65535) { *why = "groups must be <= 65535"; return false; }
   if (n_out % groups || k_in % groups) { *why = "groups must divide n_out and k_in"; return false; }
   if (groups > 1 && (n_out / groups) % 128) { *why = "a grouped weight needs a multiple of 128 rows per group"; return false; }
   if ((k_in / groups) % 8) { *why = "k_in / groups must be a multiple of 8"; return false; }

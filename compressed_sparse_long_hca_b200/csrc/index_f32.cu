@@ -26,6 +26,7 @@ struct IndexF32Args {
   float* scores;          // [n][ld]
   int64_t ld;
   int32_t* n_valid;
+  int q_per_req;          // 0: decode queries; C > 0: chunk queries (visible_tokens)
 };
 
 }  // namespace
@@ -46,7 +47,8 @@ __global__ void __launch_bounds__(kIdxF32Threads) index_f32_kernel(IndexF32Args 
     }
     return;
   }
-  const int64_t N = L.lengths()[(int64_t)a.layer * L.max_req + req] / kCsaM;
+  const int64_t T = visible_tokens(L.lengths()[(int64_t)a.layer * L.max_req + req], a.q_per_req, i);
+  const int64_t N = T > 0 ? T / kCsaM : 0;
   if (blockIdx.x == 0 && tid == 0) {
     a.n_valid[i] = (int32_t)N;
     if (N > a.ld) set_err(L, kErrLd, i);
@@ -82,8 +84,8 @@ __global__ void __launch_bounds__(kIdxF32Threads) index_f32_kernel(IndexF32Args 
 
 cudaError_t launch_index_f32(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                              const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas_per_query,
-                             cudaStream_t st) {
-  IndexF32Args a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid};
+                             cudaStream_t st, int q_per_req) {
+  IndexF32Args a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, q_per_req};
   const size_t sm = (size_t)(L.HI * L.dI + L.HI) * 4;
   cudaError_t e = cudaFuncSetAttribute(index_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;

@@ -133,6 +133,7 @@ struct IndexTcArgs {
   uint32_t* hist2;        // [n][2048]       candidates in the k-th bin over key bits 9 .. 19
   int32_t* qcount;        // [n]             candidates appended so far
   uint2* cand;            // [n][ld]         candidates (key, index), in no particular order
+  int q_per_req;          // 0: decode queries; C > 0: chunk queries (visible_tokens)
 };
 
 // Number of 128-key tiles of query i (0 for an invalid query); N = its keys.
@@ -140,7 +141,8 @@ __device__ __forceinline__ int64_t query_tiles(const IndexTcArgs& a, int i, int6
   const int req = a.req_ids[i];
   *req_out = req;
   if (req < 0 || req >= a.L.max_req) { *n_keys = 0; return 0; }
-  const int64_t N = a.L.lengths()[(int64_t)a.layer * a.L.max_req + req] / kCsaM;
+  const int64_t T = visible_tokens(a.L.lengths()[(int64_t)a.layer * a.L.max_req + req], a.q_per_req, i);
+  const int64_t N = T > 0 ? T / kCsaM : 0;
   *n_keys = N;
   if (N > a.ld) return 0;
   return (N + kCsaPerPage - 1) / kCsaPerPage;
@@ -1076,7 +1078,7 @@ size_t index_tc_smem_bytes() { return kSmemPlain > 80 * 1024 ? kSmemPlain : 80 *
 
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
-                            cudaStream_t st) {
+                            cudaStream_t st, int q_per_req) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1085,6 +1087,7 @@ cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* re
     attr = true;
   }
   IndexTcArgs a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid};
+  a.q_per_req = q_per_req;
   index_tc_kernel<false><<<ctas, kThreads, index_tc_smem_bytes(), st>>>(a);
   note_launch();
   return cudaGetLastError();

@@ -53,7 +53,7 @@ constexpr int kKTile = 64;             // K per stage
 constexpr int kTokChunk = 32;          // tokens per MMA (N), fixed
 constexpr int kWTileBytes = kRowTile * kKTile * 2;     // 16 KB
 constexpr int kMaxTok = 256;           // tokens per call
-constexpr int kSmemBudget = 200 * 1024;
+constexpr int kSmemBudget = 100 * 1024;   // two CTAs per SM
 
 
 __device__ __forceinline__ void gemm_store(const GemmOut& out, int t, int o, float v) {
@@ -77,20 +77,22 @@ struct GemmArgs {
   float* part;            // [splits][n_tok][n_out] fp32 partials (splits > 1)
 };
 
-__device__ __forceinline__ int gemm_stages(int n_pad) {
+__host__ __device__ __forceinline__ int gemm_stages(int n_pad) {
   const int st = kSmemBudget / (kWTileBytes + n_pad * 128);
   return st > 8 ? 8 : (st < 2 ? 2 : st);
 }
 
 }  // namespace
 
-// Pack one group's columns of X (BF16, rows of `row_len` elements, the
-// group's first column at x) into the per-k-tile blocks the MMA's B operand
-// reads: block b holds rows 0 .. n_pad-1 of the group's columns
-// [64 b, 64 b + 64), 16-byte chunk c of row t at (t/8)*1024 + c*128 + (t%8)*16.
-// Rows >= n_tok and columns >= kg are zero.
+// Pack the columns of X (BF16 [n_tok][row_len]) into the per-k-tile blocks
+// the MMA's B operand reads, one group per grid row y (the group's columns
+// start at y * kg): block b of a group holds rows 0 .. n_pad-1 of its
+// columns [64 b, 64 b + 64), 16-byte chunk c of row t at
+// (t/8)*1024 + c*128 + (t%8)*16.  Rows >= n_tok and columns >= kg are zero.
 __global__ void gemm_pack_x_strided_kernel(const uint16_t* x, int n_tok, int kg, int row_len, int n_pad, int k_tiles,
                                            uint8_t* xp) {
+  x += (int64_t)blockIdx.y * kg;
+  xp += (int64_t)blockIdx.y * k_tiles * n_pad * 128;
   const int64_t total = (int64_t)k_tiles * n_pad * 8;
   for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
     const int c = (int)(u % 8);
@@ -109,7 +111,7 @@ __global__ void gemm_pack_x_strided_kernel(const uint16_t* x, int n_tok, int kg,
 }
 
 // grid (row_tiles, splits)
-__global__ void __launch_bounds__(kGThreads, 1) gemm_bf16_kernel(GemmArgs a) {
+__global__ void __launch_bounds__(kGThreads, 2) gemm_bf16_kernel(GemmArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -248,12 +250,13 @@ size_t gemm_weight_bytes(int n_out, int k_in, int groups) {
 }
 int gemm_max_tokens() { return kMaxTok; }
 
-// K parts of a weight: enough CTAs to cover the SMs when the row tiles are
-// few, each part at least 8 K tiles.  A function of the weight's shape only.
+// K parts of a weight: as many as keep every CTA resident at once (two per
+// SM), each part at least 4 K tiles.  A function of the weight's shape (and
+// the device) only.
 int gemm_splits(int n_out, int k_in, int groups, int sms) {
   const int rt = gemm_row_tiles(n_out), kt = gemm_k_tiles(k_in, groups);
-  int s = (sms + rt - 1) / rt;
-  if (s > kt / 8) s = kt / 8;
+  int s = 2 * sms / rt;
+  if (s > kt / 4) s = kt / 4;
   return s < 1 ? 1 : s;
 }
 
@@ -302,20 +305,17 @@ cudaError_t launch_gemm_bf16(const void* w_packed, int n_out, int k_in, int grou
     const int kg = k_in / groups;
     const int64_t chunks = (int64_t)kt * n_pad * 8;
     const int blocks = (int)((chunks + 255) / 256 < 2048 ? (chunks + 255) / 256 : 2048);
-    for (int g = 0; g < groups; ++g) {
-      gemm_pack_x_strided_kernel<<<blocks, 256, 0, st>>>(x + (size_t)g * kg, n_tok, kg, k_in, n_pad, kt,
-                                                         xp + (size_t)g * kt * n_pad * 128);
-      note_launch();
-    }
+    gemm_pack_x_strided_kernel<<<dim3(blocks, groups), 256, 0, st>>>(x, n_tok, kg, k_in, n_pad, kt, xp);
+    note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const int stages = (kSmemBudget / (kWTileBytes + n_pad * 128)) > 8 ? 8
-                     : ((kSmemBudget / (kWTileBytes + n_pad * 128)) < 2 ? 2 : kSmemBudget / (kWTileBytes + n_pad * 128));
-  const size_t smem = (size_t)stages * (kWTileBytes + n_pad * 128) + 256 + 128;
+  const size_t smem = (size_t)gemm_stages(n_pad) * (kWTileBytes + n_pad * 128) + 256 + 128;
   static bool attr = false;
   if (!attr) {
     e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr = true;
   }

@@ -395,6 +395,61 @@ csa_status csa_decode_step(csa_cache_t* cache, int32_t layer, int32_t n, const i
                            void* dev_buf, size_t dev_bytes, csa_stream_t stream);
 
 /* ---------------------------------------------------------------------
+ * A chunk of queries with causal visibility (prefill): n requests each
+ * append n_tok (1 .. 128) new tokens together, and every one of those
+ * tokens is also a query.  Source: the data flow of page
+ * "V4终于终于终于终于是来了", section "CSA——压缩稀疏注意力" (compressor,
+ * indexer, top-k, attention over the selected entries and the 128-token
+ * window), applied to every token of a chunk; the pages describe the decode
+ * step, and the reading taken here is that the query at position t sees
+ * exactly what a decode query at t sees: the tokens 0 .. t, hence the
+ * compressed entries completed by token t (floor((t + 1) / 4) on CSA
+ * layers, floor((t + 1) / 128) on HCA layers), its own window
+ * max(0, t - 127) .. t and RoPE at position t.  The results are
+ * bit-identical to appending the chunk's tokens one at a time and running
+ * the decode calls after each (batch invariance), whatever n_tok and the
+ * chunk's other requests.
+ *
+ * Steps, all on `stream`: copy each request's window ring to the workspace
+ * (the chunk's append overwrites up to n_tok of its rows, which the chunk's
+ * early queries still see), csa_compress_append of the n_tok tokens, on a
+ * CSA layer the index scores of the n x n_tok queries over their visible
+ * keys and csa_topk, then the attention.
+ *
+ *   req_ids    device int32 [n], distinct requests
+ *   kv_cand, kv_gate, idx_cand, idx_gate   as csa_compress_append with
+ *              n_tok tokens: [n][n_tok][D] and [n][n_tok][d_I] fp32
+ *   q          device [n][n_tok][H][D], BF16 (fp32 in the fp32 format),
+ *              16-byte aligned, before RoPE
+ *   q_idx, w   CSA layers: device fp32 [n][n_tok][H_I][d_I] and [n][n_tok][H_I]
+ *   k          top-k size (CSA layers, 1 .. 8192)
+ *   sink, scale  as csa_hca_decode_attn
+ *   out        device [n][n_tok][H][D], the type of q
+ *   topk_out   CSA layers: device int32 [n][n_tok][k] for the selected
+ *              entries, as csa_topk writes them, or NULL (they then stay in
+ *              the workspace)
+ *   workspace  caller device scratch of csa_prefill_workspace_bytes(cache,
+ *              layer, n, n_tok, k, variant) bytes, 256-byte aligned (ring
+ *              copies, per-query request ids, scores [n n_tok][ld] with
+ *              ld = max(128 x max_pages_per_request, 128), counts, indices,
+ *              the split attention's partials when the variant takes it)
+ *   variant    AUTO / HIGH_OCC / LOW_OCC, as the three calls (no flags);
+ *              every variant returns identical bits
+ * Limits: n * n_tok <= 65535.  Errors: CSA_ERR_ARG for a bad shape, a NULL
+ * or a short or misaligned workspace (nothing launched); otherwise as the
+ * calls it makes.  Asynchronous.
+ * csa_prefill_workspace_bytes returns 0 for a bad shape.
+ * ------------------------------------------------------------------- */
+size_t     csa_prefill_workspace_bytes(const csa_cache_t* cache, int32_t layer, int32_t n, int32_t n_tok,
+                                       int32_t k, csa_variant variant);
+csa_status csa_prefill_chunk(csa_cache_t* cache, int32_t layer, int32_t n, const int32_t* req_ids,
+                             int32_t n_tok, const float* kv_cand, const float* kv_gate,
+                             const float* idx_cand, const float* idx_gate, const void* q,
+                             const float* q_idx, const float* w, int32_t k, const float* sink,
+                             float scale, void* out, int32_t* topk_out, void* workspace,
+                             size_t workspace_bytes, csa_variant variant, csa_stream_t stream);
+
+/* ---------------------------------------------------------------------
  * Batch-invariant projection GEMM:  Y[t][o] = sum_k X[t][k] W[o][k]
  * (BF16 operands, fp32 accumulation), for the projections around the path:
  * hidden state -> compressor candidates and gates, query down-projection to
@@ -408,10 +463,12 @@ csa_status csa_decode_step(csa_cache_t* cache, int32_t layer, int32_t n, const i
  * section "牺牲了什么"): a token's output never depends on the batch.  The
  * weight rows are the MMA's M (128 per tile), the tokens its N, always in
  * chunks of 32 (zero padded); the K order is fixed.  A weight with few row
- * tiles has its K range cut into a number of parts that depends on the
- * weight's shape alone, and the parts are summed in part order.
+ * tiles has its K range cut into a number of parts (enough to give every
+ * SM two CTAs, each part at least 256 K values) that depends on the
+ * weight's shape and the device's SM count alone, never on the batch, and
+ * the parts are summed in part order.
  *
- * Groups: with `groups` > 1 the weight is block diagonal; group g's rows
+ * Groups: with `groups` (1 .. 65535) > 1 the weight is block diagonal; group g's rows
  * (n_out / groups of them, a multiple of 128) read the columns
  * [g k_in / groups, (g + 1) k_in / groups) of X, and the host weight holds
  * only those k_in / groups columns per row: W is [n_out][k_in / groups].

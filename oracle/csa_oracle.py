@@ -551,3 +551,22 @@ def decode_query(p: LayerParams, st: RequestState | None, q, sink, k: int | None
     out["out"] = mqa_attention(qr, rows, sink, scale)
     out["n_rows"] = rows.shape[0]
     return out
+
+
+def chunk_queries(p: LayerParams, st: RequestState, c, z, ci=None, zi=None, q=None, sink=None,
+                  k: int | None = None, q_idx=None, w=None, scale: float | None = None):
+    """A chunk of n new tokens that are also queries (prefill).  The pages
+    describe the decode step ([V4-来了] section "CSA——压缩稀疏注意力": the
+    data flow for the latest token); the reading taken for a chunk is causal
+    visibility: the query at position t sees what a decode query at t sees,
+    i.e. the tokens 0 .. t and nothing after.  Written as that definition:
+    append the chunk's tokens one at a time and run the decode step after
+    each.  c, z: [n, D]; ci, zi: [n, d_I]; q: [n, H, D]; q_idx: [n, H_I, d_I];
+    w: [n, H_I].  Returns one decode_query result per token, in order."""
+    res = []
+    for j in range(np.asarray(c).shape[0]):
+        append_tokens(st, c[j:j + 1], z[j:j + 1], None if ci is None else ci[j:j + 1],
+                      None if zi is None else zi[j:j + 1])
+        res.append(decode_query(p, st, q[j], sink, k=k, q_idx=None if q_idx is None else q_idx[j],
+                                w=None if w is None else w[j], scale=scale))
+    return res

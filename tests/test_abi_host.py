@@ -120,3 +120,6 @@ def test_cache_calls_on_a_null_handle_fail_on_the_host(cuda_lib):
     assert cuda_lib.csa_decode_step_input_bytes(None, 0, 1) == 0
     assert cuda_lib.csa_decode_step_dev_bytes(None, 0, 1, 16) == 0
     assert cuda_lib.csa_decode_step(None, 0, 1, P, 16, P, 1.0, P, P, P, 1 << 20, None) == -1
+    assert cuda_lib.csa_prefill_workspace_bytes(None, 0, 1, 16, 16, 0) == 0
+    assert cuda_lib.csa_prefill_chunk(None, 0, 1, P, 16, P, P, P, P, P, P, P, 16, P, 1.0, P, None, P, 1 << 20, 0,
+                                      None) == -1

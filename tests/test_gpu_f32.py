@@ -196,3 +196,63 @@ def test_f32_index_and_attention_on_written_rows(H, D, R, HI, dI):
             rows = np.concatenate([rows, wins[i]], axis=0)
             ref = O.mqa_attention(O.rope(q[i].astype(np.float64), T - 1, R), rows, sink, 1.0 / math.sqrt(D))
             Hp.check_attention(outs[0][i], ref, f"layer {layer} len {T}", fmt="f32")
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_f32_decode_step_host_buffers_match_individual_calls(layer):
+    """csa_decode_step (through api.DecodeStep) on an fp32-format cache: fp32
+    q in the packed host buffer and an fp32 output, bit-identical to the
+    individual calls on a second cache filled the same way, step after step,
+    while CSA entries (every 4th token) and an HCA block (at 1024) complete."""
+    from compressed_sparse_long_hca_b200.api import DecodeStep
+    wl = I.Workload("f32-step", "csa", H=8, D=64, R=16, H_I=4, d_I=32, k=16, W=128, context=0, batch=0,
+                    seed=5151)
+    lens = [300, 1021]
+    reqs = [1, 0]
+    pairs = [Hp.Pair(wl, 1, 1, max_req=2, capacity=max(lens) + 64, fmt="f32") for _ in range(2)]
+    for pair in pairs:
+        for r, T in enumerate(lens):
+            pair.cache.request_alloc(r, T + 64)
+            pair.append(layer, [r], {r: pair.gen_tokens(layer, r, 0, T)}, T, oracle=False)
+    torch.cuda.synchronize()
+    csa = layer == 0
+    sink = pairs[0].params[layer]["sink"]
+    sink_d = _t(sink)
+    step = DecodeStep(pairs[0].cache, layer, reqs, wl.k if csa else 0, sink)
+    c2 = pairs[1].cache
+    rid = _t(np.array(reqs, np.int32))
+    rng = np.random.default_rng(23)
+    for s in range(6):
+        v = step.views(step.host_in)
+        v["q"].copy_(torch.from_numpy(rng.standard_normal((2, wl.H, wl.D)).astype(np.float32)))
+        toks = {r: pairs[0].gen_tokens(layer, r, lens[r] + s, 1) for r in reqs}
+        for x, name in enumerate(("c", "z", "ci", "zi")):
+            if name in v:
+                v[name].copy_(torch.from_numpy(np.stack([toks[r][x] for r in reqs])))
+        if csa:
+            v["q_idx"].copy_(torch.from_numpy(rng.standard_normal((2, wl.H_I, wl.d_I)).astype(np.float32)))
+            v["w"].copy_(torch.from_numpy(rng.standard_normal((2, wl.H_I)).astype(np.float32)))
+        got = step()
+        torch.cuda.synchronize()
+        pairs[0].cache.check_device_error()
+        assert got.dtype == torch.float32
+        got = got.clone()
+        got_idx = step.topk_idx.cpu() if csa else None
+        # the same step through the individual calls on the second cache
+        dv = {name: t.cuda() for name, t in v.items()}
+        c2.compress_append(layer, rid, dv["c"], dv["z"], dv.get("ci"), dv.get("zi"))
+        idx = None
+        if csa:
+            ld = max(c2.get_length(layer, r) for r in reqs) // 4 + 1
+            scores = torch.empty((2, ld), device="cuda")
+            nv = torch.empty(2, dtype=torch.int32, device="cuda")
+            c2.index_scores(layer, rid, dv["q_idx"], dv["w"], scores, nv)
+            idx = torch.empty((2, wl.k), dtype=torch.int32, device="cuda")
+            topk(scores, nv, wl.k, idx)
+        out = torch.empty((2, wl.H, wl.D), dtype=torch.float32, device="cuda")
+        c2.decode_attn(layer, rid, dv["q"], idx, sink_d, out)
+        torch.cuda.synchronize()
+        c2.check_device_error()
+        assert torch.equal(got.view(torch.int32), out.cpu().view(torch.int32)), f"step {s}: output differs"
+        if csa:
+            assert torch.equal(got_idx, idx.cpu()), f"step {s}: top-k differs"
