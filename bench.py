@@ -570,6 +570,72 @@ def measure_projections(steps: int = 10, n_tok: int = 4) -> dict:
                          "algorithmic_bytes": total_bytes, "peak_source": peak_kind}}
 
 
+def measure_prefill(wl, n_tok: int = 128, reps: int = 3) -> dict:
+    """Chunks of queries with causal visibility (csa_prefill_chunk) at the end
+    of the workload's context: each request of the batch appends n_tok new
+    tokens that are all queries.  The cache is filled through the append path
+    first; each chunk is timed with CUDA events after an L2 flush."""
+    import torch
+
+    from compressed_sparse_long_hca_b200.api import Cache
+    B, T0 = wl.batch, wl.context
+    csa = wl.kind == "csa"
+    cap = T0 + (reps + 1) * n_tok + 512
+    nb = (cap + 511) // 512
+    b_kv, b_idx, sink = I.layer_params(wl.seed, 0, wl.kind, wl.D, wl.d_I or 32, wl.H)
+    cache = Cache(n_csa=1 if csa else 0, n_hca=0 if csa else 1, H=wl.H, D=wl.D, D_rope=wl.R,
+                  H_I=wl.H_I or 1, d_I=wl.d_I or 32, max_requests=B, max_pages_per_request=nb,
+                  pool_pages=nb * B, b_pos_csa=b_kv[None] if csa else None,
+                  b_pos_idx=b_idx[None] if csa else None, b_pos_hca=None if csa else b_kv[None],
+                  fmt=workload_fmt(wl))
+    rid = torch.arange(B, dtype=torch.int32, device="cuda")
+    for r in range(B):
+        cache.request_alloc(r, cap)
+    dI = wl.d_I if csa else 0
+    t = 0
+    while t < T0:
+        n = min(I.CHUNK, T0 - t)
+        parts = [I.device_token_inputs(wl.seed, 0, r, t // I.CHUNK, wl.D, dI) for r in range(B)]
+        st = lambda k: torch.stack([p[k][:n] for p in parts]).contiguous() if parts[0][k] is not None else None
+        cache.compress_append(0, rid, st(0), st(1), st(2), st(3))
+        t += n
+    torch.cuda.synchronize()
+    cache.check_device_error()
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl.seed * 7 + 1)
+    shp = (B, n_tok)
+    c, z = torch.randn(shp + (wl.D,), generator=g, device="cuda"), torch.randn(shp + (wl.D,), generator=g, device="cuda")
+    ci = torch.randn(shp + (dI,), generator=g, device="cuda") if csa else None
+    zi = torch.randn(shp + (dI,), generator=g, device="cuda") if csa else None
+    q = torch.randn(shp + (wl.H, wl.D), generator=g, device="cuda").to(cache.qdtype)
+    qi = torch.randn(shp + (wl.H_I, dI), generator=g, device="cuda") if csa else None
+    w = torch.randn(shp + (wl.H_I,), generator=g, device="cuda") if csa else None
+    out = torch.empty(shp + (wl.H, wl.D), dtype=cache.qdtype, device="cuda")
+    sink_d = torch.from_numpy(sink).cuda()
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device="cuda")
+    flush_rd = torch.ones(256 * 2**20 // 4, dtype=torch.int32, device="cuda")
+    cache.prefill_chunk(0, rid, c, z, ci, zi, q, qi, w, wl.k if csa else 0, sink_d, out)    # warm-up chunk
+    torch.cuda.synchronize()
+    ms = 0.0
+    for _ in range(reps):
+        flush.zero_()
+        flush_rd.sum()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        cache.prefill_chunk(0, rid, c, z, ci, zi, q, qi, w, wl.k if csa else 0, sink_d, out)
+        b.record()
+        b.synchronize()
+        ms += a.elapsed_time(b)
+    cache.check_device_error()
+    us = ms / reps * 1e3
+    toks = B * n_tok
+    del cache
+    return {"workload": wl.name, "context": T0, "batch": B, "tokens_per_request": n_tok, "chunks": reps,
+            "us_per_chunk": round(us, 1), "tokens_per_s": toks / (us / 1e6),
+            "api": "Cache.prefill_chunk -> csa_prefill_chunk",
+            "l2": "flushed before each chunk (256 MiB write + read)"}
+
+
 # Configurations measured beside the headline at N = 1 (fewer steps each):
 # the tiny fp32 CSA layer, HCA at 128K (batch 32), CSA Flash-like at 128K
 # (batch 32) and the HCA layer at 1M (batch 4).
@@ -627,6 +693,9 @@ def run_gpu(args):
         gc.collect()
         torch.cuda.empty_cache()
         line["projections"] = measure_projections()
+        gc.collect()
+        torch.cuda.empty_cache()
+        line["prefill"] = measure_prefill(wl)
     if rank == 0 and args.cpu_baseline and ws == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if rank == 0:
