@@ -62,6 +62,10 @@ struct AttnArgs {
   // that append; window positions below len - 128 are read from the copy.
   int q_per_req;
   const char* win_snap;
+  // split launch only: the CTAs of one (query, head group) form a cluster
+  // (one CTA per chunk) and fold the chunks' partials through distributed
+  // shared memory instead of the workspace and attn_fold_kernel
+  int cluster_fold;
 };
 
 struct QueryGeom {

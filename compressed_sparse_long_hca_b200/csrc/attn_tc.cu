@@ -46,7 +46,10 @@
 //   * softmax statistics of the tile: one thread per (row, 16 heads);
 //   * PV: O_t^T[dims x G] = V^T P^T, P^T in BF16; the FP8 dims use
 //     (P * row scale)^T, the RoPE dims P^T, each into its own accumulator.
+#include <cooperative_groups.h>
+
 #include <mutex>
+#include <vector>
 
 #include "attn_common.cuh"
 #include "common.cuh"
@@ -114,17 +117,18 @@ __device__ __forceinline__ float warp_reduce16(const float (&v)[16], int lane) {
   return op(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
 }
 
-// Address of row `r` of tile `tt`; returns whether the row exists.  The
-// first n_pgt page-table entries of the request are read from `pgt`
-// (shared memory), the others from the arena.
+// Address of row `r` of tile `tt` and of its FP8 scale (*scp, null for no
+// row; the scale is loaded with the row's gather, off the address chain);
+// returns whether the row exists.  The first n_pgt page-table entries of the
+// request are read from `pgt` (shared memory), the others from the arena.
 __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& g, int i, int tt, int r,
-                                            uint64_t* rowf8, uint64_t* rowbf, float* rsc, const int32_t* pgt,
+                                            uint64_t* rowf8, uint64_t* rowbf, const float** scp, const int32_t* pgt,
                                             int n_pgt) {
   const Layout& L = a.L;
   const int64_t rr = (int64_t)tt * kTileRows + r;
   const uint8_t* f8 = nullptr;
   const uint16_t* bf = nullptr;
-  float sc = 0.f;
+  const float* sc = nullptr;
   if (rr < g.n_list) {
     int64_t j = g.csa ? (int64_t)a.topk[(int64_t)i * a.k + rr] : rr;
     if (j >= g.n_entries) {
@@ -138,7 +142,7 @@ __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& 
       const char* pp = L.page(pi < n_pgt ? pgt[pi] : L.page_table(g.req)[pi], a.layer);
       f8 = reinterpret_cast<const uint8_t*>(pp) + (int64_t)s * L.kv_fp8_bytes;
       bf = reinterpret_cast<const uint16_t*>(pp + (g.csa ? L.pg_csa_bf16 : L.pg_hca_bf16)) + (int64_t)s * L.R;
-      sc = reinterpret_cast<const float*>(pp + (g.csa ? L.pg_csa_scale : L.pg_hca_scale))[s];
+      sc = reinterpret_cast<const float*>(pp + (g.csa ? L.pg_csa_scale : L.pg_hca_scale)) + s;
     }
   } else if (rr < g.total) {
     const int64_t p = g.w0 + (rr - g.n_list);
@@ -146,12 +150,72 @@ __device__ __forceinline__ bool resolve_row(const AttnArgs& a, const QueryGeom& 
     const int slot = (int)(p % kWindow);
     f8 = reinterpret_cast<const uint8_t*>(st + L.ring_fp8) + (int64_t)slot * (L.D - L.R);
     bf = reinterpret_cast<const uint16_t*>(st + L.ring_bf16) + (int64_t)slot * L.R;
-    sc = reinterpret_cast<const float*>(st + L.ring_scale)[slot];
+    sc = reinterpret_cast<const float*>(st + L.ring_scale) + slot;
   }
   rowf8[r] = reinterpret_cast<uint64_t>(f8);
   rowbf[r] = reinterpret_cast<uint64_t>(bf);
-  rsc[r] = sc;
+  *scp = sc;
   return f8 != nullptr;
+}
+
+constexpr int kClusterFoldMax = 16;    // chunks per query the cluster fold serves (cluster size)
+
+// Split launch with the fold in the cluster.  The CTAs of one (query, head
+// group), one per chunk, form a thread-block cluster; each has staged its
+// chunk's (m_c, l_c) per head and O_c [G][D] in its own shared memory (an
+// empty chunk: m_c = -inf).  After a cluster barrier every CTA folds a slice
+// of the head group's outputs, reading the chunks' partials from the other
+// CTAs' shared memory in chunk order, with the arithmetic of
+// attn_fold_kernel, so the bits are the same as the workspace path's.  A
+// second cluster barrier keeps every CTA's shared memory alive until all
+// reads of it are done.
+__device__ __noinline__ void cluster_fold(int G, int H, int D, const float* sink, uint16_t* out, int n_chunks, int i,
+                                          int h0, const float* o_stage, const float2* ml_stage, float2* ml_all) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = (int)cl.num_blocks();
+  const int rank = (int)cl.block_rank();
+  const int nch = n_chunks < C ? n_chunks : C;
+  cl.sync();
+  for (int x = threadIdx.x; x < nch * G; x += blockDim.x)
+    ml_all[x] = *cl.map_shared_rank(ml_stage + x % G, (unsigned)(x / G));
+  __syncthreads();
+  tc::griddep_wait();          // (a CTA without rows has not waited yet) nothing is written before
+  const int n4 = G * D / 4;
+  const int per = (n4 + C - 1) / C;
+  const int u_end = (rank + 1) * per < n4 ? (rank + 1) * per : n4;
+  for (int u = rank * per + (int)threadIdx.x; u < u_end; u += blockDim.x) {
+    const int hh = (4 * u) / D, d = (4 * u) % D;
+    const int h = h0 + hh;
+    if (h >= H) continue;
+    float4 v[kClusterFoldMax];
+#pragma unroll
+    for (int c = 0; c < kClusterFoldMax; ++c)
+      if (c < nch) v[c] = *reinterpret_cast<const float4*>(cl.map_shared_rank(o_stage + hh * D + d, (unsigned)c));
+    float m = -INFINITY, l = 0.f;
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < kClusterFoldMax; ++c) {
+      if (c >= nch) break;
+      const float2 ml = ml_all[c * G + hh];
+      if (ml.x == -INFINITY) continue;
+      float mn, al, be;
+      fold_coef(m, ml.x, mn, al, be);
+      l = fold_val(l, al, ml.y, be);
+      o[0] = fold_val(o[0], al, v[c].x, be);
+      o[1] = fold_val(o[1], al, v[c].y, be);
+      o[2] = fold_val(o[2], al, v[c].z, be);
+      o[3] = fold_val(o[3], al, v[c].w, be);
+      m = mn;
+    }
+    float cm, dn;
+    finish_coef(m, sink[h], l, cm, dn);
+    uint2 pk;
+    pk.x = (uint32_t)finish_val(o[0], cm, dn) | ((uint32_t)finish_val(o[1], cm, dn) << 16);
+    pk.y = (uint32_t)finish_val(o[2], cm, dn) | ((uint32_t)finish_val(o[3], cm, dn) << 16);
+    *reinterpret_cast<uint2*>(out + ((int64_t)i * H + h) * D + d) = pk;
+  }
+  cl.sync();
 }
 
 }  // namespace
@@ -217,7 +281,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       if (reporter) set_err(L, kErrBounds, 4000000 + i);
       return;
     }
-    if (c0 >= g.n_chunks) return;
+    if (c0 >= g.n_chunks) {
+      if (a.cluster_fold) {      // no rows: an empty partial, and this CTA's share of the fold
+        float2* ml_stage = reinterpret_cast<float2*>(tile + (int64_t)G * D * 4);
+        for (int x = tid; x < G; x += kAttThreads) ml_stage[x] = make_float2(-INFINITY, 0.f);
+        cluster_fold(G, H, D, a.sink, static_cast<uint16_t*>(a.out), g.n_chunks, i, h0,
+                     reinterpret_cast<const float*>(tile), ml_stage, reinterpret_cast<float2*>(stage));
+      }
+      return;
+    }
   }
   const int tt0 = kSplit ? c0 * g.chunk : 0;
   const int tt_end = kSplit ? min(tt0 + g.chunk, g.n_tiles) : g.n_tiles;
@@ -322,9 +394,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   const bool list_rows = (int64_t)tt0 * kTileRows < g.n_list;   // the first tile holds top-k / entry rows
   if (early && list_rows) tc::griddep_wait();
   float2* cs = reinterpret_cast<float2*>(stage);
+  const float* scp = nullptr;         // warps 0-3: FP8 scale of row tid of the tile being fetched
+  float scv = 0.f;                    // its value, loaded with the tile's gather
   int any = 0;
   if (warp < 4) {
-    any = resolve_row(a, g, i, tt0, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
+    any = resolve_row(a, g, i, tt0, tid, rowf8, rowbf, &scp, pgt, n_pgt) ? 1 : 0;
   } else {
     const int qt = tid - 128;
     for (int p = qt; p < R / 2; p += 128) {
@@ -347,11 +421,13 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       const int it = warp + 8 * u;
       buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
     }
+    scv = scp != nullptr ? __ldg(scp) : 0.f;
 #pragma unroll
     for (int u = 0; u < kMaxLoads; ++u) {
       const int it = warp + 8 * u;
       if (it < n_items) gather_store(it, buf[u]);
     }
+    if (warp < 4) rsc[tid] = scv;
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();                                      // every thread's query copies have landed
@@ -479,6 +555,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
           const int it = warp + 8 * u;
           buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
         }
+        scv = scp != nullptr ? __ldg(scp) : 0.f;
         buf_tile = tt;
       }
       // -- fold the previous tile while the loads fly
@@ -490,6 +567,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
           const int it = warp + 8 * u;
           if (it < n_items) gather_store(it, buf[u]);
         }
+        if (warp < 4) rsc[tid] = scv;
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
@@ -581,7 +659,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
       //    them) and loads issued now
       if (tt + 1 < tt_end) {
         int nany = 0;
-        if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
+        if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, &scp, pgt, n_pgt) ? 1 : 0;
         tile_valid = __syncthreads_count(nany) > 0;
         next_resolved = true;
         if (tile_valid) {
@@ -590,6 +668,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
             const int it = warp + 8 * u;
             buf[u] = it < n_items ? gather_load(it) : make_uint4(0, 0, 0, 0);
           }
+          scv = scp != nullptr ? __ldg(scp) : 0.f;
           buf_tile = tt + 1;
         }
       }
@@ -606,7 +685,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     // -- addresses of the next tile's rows (after a tile without rows)
     if (tt + 1 < tt_end && !next_resolved) {
       int nany = 0;
-      if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, rsc, pgt, n_pgt) ? 1 : 0;
+      if (warp < 4) nany = resolve_row(a, g, i, tt + 1, tid, rowf8, rowbf, &scp, pgt, n_pgt) ? 1 : 0;
       tile_valid = __syncthreads_count(nany) > 0;
     }
     next_resolved = false;
@@ -614,18 +693,26 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
 
   if (ok && n_done > 0) ok = tc::mbar_wait(bar_pv, (n_done - 1) & 1);
   ok = __syncthreads_and(ok) != 0;
+  // split launch: where this chunk's partial goes -- the workspace, or (the
+  // cluster fold) this CTA's shared memory, the tile buffer being free now
+  // that the last PV has completed: O_c [G][D] then (m_c, l_c) [G]
+  const bool cfold = kSplit && a.cluster_fold != 0;
+  float* const o_stage = reinterpret_cast<float*>(tile);
+  float2* const ml_stage = reinterpret_cast<float2*>(tile + (int64_t)G * D * 4);
+  float* const wo = !kSplit ? nullptr
+                    : cfold ? o_stage : a.ws_o + (((int64_t)i * a.chunks_max + c0) * H + h0) * D;    // [head - h0][D]
+  float2* const wml = !kSplit ? nullptr
+                      : cfold ? ml_stage : a.ws_ml + ((int64_t)i * a.chunks_max + c0) * H + h0;     // [head - h0]
   if (ok && kSplit && n_done == 0) {
     // ---- split launch, a chunk without rows: an empty partial
-    if (tid < G && h0 + tid < H) a.ws_ml[((int64_t)i * a.chunks_max + c0) * H + h0 + tid] = make_float2(-INFINITY, 0.f);
+    if (tid < G && h0 + tid < H) wml[tid] = make_float2(-INFINITY, 0.f);
   } else if (ok && kSplit && multi) {
     // ---- split launch, a chunk of several tiles: fold its last tile, then
-    // the chunk's (m, l, O) to the workspace
+    // the chunk's (m, l, O)
     tc::tc_fence_after();
     if (pend_fold) fold_pending();
-    if (tid < G && h0 + tid < H)
-      a.ws_ml[((int64_t)i * a.chunks_max + c0) * H + h0 + tid] = make_float2(m_run[tid], l_run[tid]);
+    if (tid < G && h0 + tid < H) wml[tid] = make_float2(m_run[tid], l_run[tid]);
     if (tw) {
-      float* wo = a.ws_o + ((int64_t)i * a.chunks_max + c0) * H * D;
       for (int dc = 0; dc < n_dc; ++dc) {
         uint32_t orun[16];
         tc::tmem_ld_x16(tmem + lane_base + col_orun + dc * G + hb, orun);
@@ -634,7 +721,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int h = h0 + hb + e;
-          if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(orun[e]);
+          if (h < H && d < D) wo[(int64_t)(hb + e) * D + d] = __uint_as_float(orun[e]);
         }
       }
     }
@@ -642,11 +729,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
     // ---- split launch, a chunk of one tile: the tile's partial is the
     // chunk's (folding into an empty result is exact)
     tc::tc_fence_after();
-    if (tid < G && h0 + tid < H)
-      a.ws_ml[((int64_t)i * a.chunks_max + c0) * H + h0 + tid] = make_float2(m_t[tid], l_t[tid]);
+    if (tid < G && h0 + tid < H) wml[tid] = make_float2(m_t[tid], l_t[tid]);
     if (tw) {
       // two 128-dim blocks per TMEM wait
-      float* wo = a.ws_o + ((int64_t)i * a.chunks_max + c0) * H * D;
       for (int dc0 = 0; dc0 < n_dc; dc0 += 2) {
         uint32_t om[2][16], orp[2][16];
 #pragma unroll
@@ -666,7 +751,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int h = h0 + hb + e;
-            if (h < H && d < D) wo[(int64_t)h * D + d] = __uint_as_float(d < dmain ? om[q2][e] : orp[q2][e]);
+            if (h < H && d < D) wo[(int64_t)(hb + e) * D + d] = __uint_as_float(d < dmain ? om[q2][e] : orp[q2][e]);
           }
         }
       }
@@ -741,8 +826,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
         }
       }
     }
-  } else if (!ok && tid == 0) {
-    set_err(L, kErrTimeout, 3000000 + i);
+  } else if (!ok) {
+    if (tid == 0) set_err(L, kErrTimeout, 3000000 + i);
+    if (cfold && tid < G) ml_stage[tid] = make_float2(-INFINITY, 0.f);   // the fold still runs; the error stands
   }
   tc::griddep_launch_dependents();                      // the fold (or the next step) may start launching
   if (warp == 0) {   // no tcgen05 operation of this CTA is in flight when TMEM is released
@@ -753,6 +839,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, n_cols);
+  if (cfold)
+    cluster_fold(G, H, D, a.sink, static_cast<uint16_t*>(a.out), g.n_chunks, i, h0, o_stage, ml_stage,
+                 reinterpret_cast<float2*>(stage));
 }
 
 // Split launch, second step: fold the chunk partials of (query blockIdx.y,
@@ -848,6 +937,46 @@ size_t attn_workspace_bytes(const Layout& L, int layer, int n, int k) {
   return (size_t)(units * L.D * 4 + units * 8);
 }
 
+// How many clusters of C split-launch CTAs (smem bytes each) the device can
+// hold at once; asked once per (device, C, smem) and remembered.
+static cudaError_t cluster_fold_capacity(int C, size_t smem, int* out) {
+  static std::mutex mu;
+  struct Entry { int dev, C; size_t smem; int n; };
+  static std::vector<Entry> seen;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& x : seen)
+    if (x.dev == dev && x.C == C && x.smem == smem) { *out = x.n; return cudaSuccess; }
+  if (C > 8) {
+    e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)C;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)C, 1, 1);
+  cfg.blockDim = dim3(kAttThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel<true>, &cfg);
+  if (e != cudaSuccess) {       // not available: the workspace path
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  seen.push_back(Entry{dev, C, smem, n});
+  *out = n;
+  return cudaSuccess;
+}
+
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
                            const int32_t* topk, int k, const float* sink, float scale, uint16_t* out, int G,
                            void* ws, cudaStream_t st, bool state_ready, int q_per_req, const char* win_snap) {
@@ -883,6 +1012,30 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(a.chunks_max, n_hg, n);
+  // The fold in the cluster when every cluster of the launch (one per query
+  // and head group, a CTA per chunk) can be resident at once; otherwise the
+  // partials go through the workspace to attn_fold_kernel.  Both give the
+  // same bits.
+  int resident = 0;
+  if (a.chunks_max >= 2 && a.chunks_max <= kClusterFoldMax && (L.D % 4) == 0) {
+    e = cluster_fold_capacity(a.chunks_max, sm, &resident);
+    if (e != cudaSuccess) return e;
+  }
+  if (resident >= n_hg * n) {
+    cudaLaunchAttribute at2[2];
+    at2[0] = at[0];
+    at2[1].id = cudaLaunchAttributeClusterDimension;
+    at2[1].val.clusterDim.x = (unsigned)a.chunks_max;
+    at2[1].val.clusterDim.y = 1;
+    at2[1].val.clusterDim.z = 1;
+    cfg.attrs = at2;
+    cfg.numAttrs = 2;
+    a.cluster_fold = 1;
+    e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, a);
+    note_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
   e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, a);
   note_launch();
   if (e != cudaSuccess) return e;
