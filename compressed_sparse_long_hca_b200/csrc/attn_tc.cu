@@ -62,11 +62,11 @@ namespace {
 constexpr int kAttThreads = 256;
 constexpr int kMaxLoads = 18;      // 16-byte loads per thread per tile (D <= 512)
 
-constexpr int kPgtCache = 4096;    // page-table entries of the query's request kept in shared memory
+constexpr int kPgtCache = 2048;    // page-table entries of the query's request kept in shared memory (1M tokens)
 
 struct AttnSmem {
   int Dp;             // head dim padded to a multiple of 128
-  int64_t tile, qs, pt, stage, rowf8, rowbf, rsc, stats, pgt, bars, total;
+  int64_t tile, qs, pt, rowf8, rowbf, rsc, stats, pgt, bars, total;
 };
 
 __host__ __device__ inline AttnSmem attn_smem(int D, int G) {
@@ -75,8 +75,9 @@ __host__ __device__ inline AttnSmem attn_smem(int D, int G) {
   int64_t o = 0;
   s.tile = o;  o += (int64_t)kTileRows * s.Dp * 2;           // BF16 rows, core-matrix order
   s.qs = o;    o += (int64_t)G * s.Dp * 2;                   // BF16 query heads
-  s.pt = o;    o += (int64_t)kTileRows * G * 2 * 2;          // BF16 P^T and (P*scale)^T
-  s.stage = o; o += (int64_t)kTileRows * (G + 1) * 4;        // fp32 logits / p
+  s.pt = o;    o += (int64_t)kTileRows * G * 2 * 2;          // BF16 P^T and (P*scale)^T (before the first tile:
+                                                             // cos / sin of the RoPE pairs; after the last: the
+                                                             // cluster fold's (m, l) of every chunk)
   s.rowf8 = o; o += (int64_t)kTileRows * 8;                  // row addresses (FP8 part)
   s.rowbf = o; o += (int64_t)kTileRows * 8;                  // row addresses (BF16 part)
   s.rsc = o;   o += (int64_t)kTileRows * 4;                  // row FP8 scales
@@ -238,7 +239,6 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   uint8_t* qs = sm + S.qs;
   uint8_t* pt = sm + S.pt;
   uint8_t* ptm = pt + kTileRows * G * 2;               // (P * row scale)^T for the FP8 dims
-  float* stage = reinterpret_cast<float*>(sm + S.stage);
   uint64_t* rowf8 = reinterpret_cast<uint64_t*>(sm + S.rowf8);
   uint64_t* rowbf = reinterpret_cast<uint64_t*>(sm + S.rowbf);
   float* rsc = reinterpret_cast<float*>(sm + S.rsc);
@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
         float2* ml_stage = reinterpret_cast<float2*>(tile + (int64_t)G * D * 4);
         for (int x = tid; x < G; x += kAttThreads) ml_stage[x] = make_float2(-INFINITY, 0.f);
         cluster_fold(G, H, D, a.sink, static_cast<uint16_t*>(a.out), g.n_chunks, i, h0,
-                     reinterpret_cast<const float*>(tile), ml_stage, reinterpret_cast<float2*>(stage));
+                     reinterpret_cast<const float*>(tile), ml_stage, reinterpret_cast<float2*>(pt));
       }
       return;
     }
@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   __syncthreads();
   const bool list_rows = (int64_t)tt0 * kTileRows < g.n_list;   // the first tile holds top-k / entry rows
   if (early && list_rows) tc::griddep_wait();
-  float2* cs = reinterpret_cast<float2*>(stage);
+  float2* cs = reinterpret_cast<float2*>(pt);         // P^T is first written by the first tile's softmax
   const float* scp = nullptr;         // warps 0-3: FP8 scale of row tid of the tile being fetched
   float scv = 0.f;                    // its value, loaded with the tile's gather
   int any = 0;
@@ -841,7 +841,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
   if (warp == 0) tc::tmem_dealloc(tmem, n_cols);
   if (cfold)
     cluster_fold(G, H, D, a.sink, static_cast<uint16_t*>(a.out), g.n_chunks, i, h0, o_stage, ml_stage,
-                 reinterpret_cast<float2*>(stage));
+                 reinterpret_cast<float2*>(pt));
 }
 
 // Split launch, second step: fold the chunk partials of (query blockIdx.y,
@@ -916,6 +916,18 @@ cudaError_t launch_attn_fold(const AttnArgs& a, cudaStream_t st) {
 
 size_t attn_tc_smem_bytes(int D, int G) { return (size_t)attn_smem(D, G).total + 1024; }
 
+// Dynamic shared memory of an attention launch, and a carveout no larger
+// than it needs: what the carveout leaves is the SM's L1, which holds the
+// row gathers in flight.
+template <bool kSplit>
+static cudaError_t attn_smem_attrs(size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int pct = (int)(((smem + 1024) * 100 + 228 * 1024 - 1) / (228 * 1024));
+  return cudaFuncSetAttribute(attn_tc_kernel<kSplit>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              pct < 100 ? pct : 100);
+}
+
 int attn_tiles_max(const Layout& L, int layer, int k) {
   const int64_t rows = (layer < L.n_csa ? (int64_t)k : (int64_t)L.max_pages_per_req * kHcaPerPage) + kWindow;
   return (int)((rows + kTileRows - 1) / kTileRows);
@@ -953,7 +965,7 @@ static cudaError_t cluster_fold_capacity(int C, size_t smem, int* out) {
     e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = attn_smem_attrs<true>(smem);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -998,7 +1010,7 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   cfg.attrs = at;
   cfg.numAttrs = 1;
   if (!split) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = attn_smem_attrs<false>(sm);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3(n, n_hg);
     e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<false>, a);
@@ -1009,7 +1021,7 @@ cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req
   a.chunks_max = attn_chunks_max(L, layer, k);
   a.ws_o = static_cast<float*>(ws);
   a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + (int64_t)n * a.chunks_max * L.H * L.D * 4);
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  cudaError_t e = attn_smem_attrs<true>(sm);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(a.chunks_max, n_hg, n);
   // The fold in the cluster when every cluster of the launch (one per query
