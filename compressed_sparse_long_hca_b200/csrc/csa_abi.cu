@@ -331,9 +331,12 @@ static csa_status index_scores_impl(const csa_cache_t* c, int32_t layer, int32_t
     e = csa::launch_index_f32(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, std::min(per_q, 1024),
                               (cudaStream_t)stream, cq.q_per_req);
   } else {
-    // Two persistent CTAs per SM for either variant; the per-key arithmetic
-    // does not depend on the grid.
-    e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, 2 * sms,
+    // Persistent CTAs over the flattened (query, tile) list: two per SM (AUTO,
+    // HIGH_OCC: their tcgen05 issue latencies overlap), or one per SM
+    // (LOW_OCC).  The CTAs own different tile ranges in the two grids; a
+    // key's score does not depend on which CTA computes it.
+    const int ctas = variant == CSA_VARIANT_LOW_OCC ? sms : 2 * sms;
+    e = csa::launch_index_tc(c->L, layer, n, req_ids, q_idx, w, scores, ld, n_valid, ctas,
                              (cudaStream_t)stream, cq.q_per_req);
   }
   if (e != cudaSuccess) return cuda_fail(e, "index launch");

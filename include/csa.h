@@ -216,7 +216,11 @@ csa_status csa_compress_append(csa_cache_t* cache, int32_t layer, int32_t n,
  * kernel and k^_j the stored MXFP4 key (block-scaled FP4 tensor-core MMA,
  * fp32 accumulation); in the fp32 format q^_h = q_idx[i][h] and k^_j the
  * stored fp32 key (fp32 FMA, d ascending, heads ascending).  Entries j >= N
- * of the row are not written.  Both variants return identical bits.
+ * of the row are not written.  Both variants return identical bits: the
+ * mixed format's persistent grid is two CTAs per SM (AUTO, HIGH_OCC) or one
+ * (LOW_OCC), each owning a different range of the (query, tile) list; the
+ * fp32 format gives a query one CTA (HIGH_OCC) or several (LOW_OCC; AUTO
+ * when n is below the SM count).
  *   q_idx    device float [n][H_I][d_I]
  *   w        device float [n][H_I]
  *   scores   device float [n][ld]   (ld >= the largest N; checked on device)
