@@ -449,3 +449,83 @@ def test_c5_ragged_sweep_at_scale():
         for r in allr:
             lens[r] += 1
     assert 1 in sizes_seen and max(sizes_seen) > 64
+
+
+@pytest.mark.parametrize("name", ["csa-pro-1m", "hca-pro-1m"])
+def test_full_size_prefill_chunk_matches_decode(name):
+    """A chunk of 128 queries per request (csa_prefill_chunk) at the
+    production shapes (H = 128, D = 512, R = 64; CSA: H_I = 64, d_I = 128,
+    k = 1024) equals, bit for bit, the same 128 tokens appended one at a time
+    with a decode step after each, on a second cache filled identically;
+    contexts of 5,000 to 131,071 tokens, so the chunk crosses CSA entries, an
+    HCA block and (for the longest) the 2^17 boundary.  The chunk's last query
+    of every request is also checked against the oracle over the stored rows."""
+    wl = I.WORKLOADS[name]
+    csa = wl.kind == "csa"
+    lens = [70000, 131071, 5000]
+    reqs = [1, 2, 0]
+    n_tok = 128
+    cap = max(lens) + n_tok + 64
+    pairs = [Hp.Pair(wl, 1 if csa else 0, 0 if csa else 1, max_req=3, capacity=cap) for _ in range(2)]
+    dI = wl.d_I if csa else 0
+    for pair in pairs:
+        for r in range(3):
+            pair.cache.request_alloc(r, cap)
+        _fill(pair.cache, 0, list(range(3)), {r: lens[r] for r in range(3)}, wl.seed, wl.D, dI)
+    A, B = pairs[0].cache, pairs[1].cache
+    sink = pairs[0].params[0]["sink"]
+    sink_d = torch.from_numpy(sink).cuda()
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    c, z = _host(wl.seed + 11, 3, n_tok, wl.D), _host(wl.seed + 12, 3, n_tok, wl.D)
+    ci = _host(wl.seed + 13, 3, n_tok, dI) if csa else None
+    zi = _host(wl.seed + 14, 3, n_tok, dI) if csa else None
+    q = I.bf16_grid(_host(wl.seed + 15, 3, n_tok, wl.H, wl.D))
+    qi = _host(wl.seed + 16, 3, n_tok, wl.H_I, wl.d_I) if csa else None
+    w = _host(wl.seed + 17, 3, n_tok, wl.H_I) if csa else None
+    rid = torch.tensor(reqs, dtype=torch.int32, device="cuda")
+    # the batch rows follow `reqs`
+    sel = lambda a: a[reqs] if a is not None else None
+    out = torch.empty((3, n_tok, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((3, n_tok, wl.k), dtype=torch.int32, device="cuda") if csa else None
+    A.prefill_chunk(0, rid, dev(sel(c)), dev(sel(z)), dev(sel(ci)) if csa else None, dev(sel(zi)) if csa else None,
+                    dev(sel(q)).to(torch.bfloat16), dev(sel(qi)) if csa else None, dev(sel(w)) if csa else None,
+                    wl.k, sink_d, out, topk_out=idx)
+    torch.cuda.synchronize()
+    A.check_device_error()
+    got = out.cpu().view(torch.int16)
+    got_idx = idx.cpu() if csa else None
+    for j in range(n_tok):
+        B.compress_append(0, rid, dev(sel(c)[:, j:j + 1]), dev(sel(z)[:, j:j + 1]),
+                          dev(sel(ci)[:, j:j + 1]) if csa else None, dev(sel(zi)[:, j:j + 1]) if csa else None)
+        ref_idx = None
+        if csa:
+            ld = max(B.get_length(0, r) for r in reqs) // 4 + 128
+            scores = torch.empty((3, ld), device="cuda")
+            nv = torch.empty(3, dtype=torch.int32, device="cuda")
+            B.index_scores(0, rid, dev(sel(qi)[:, j]), dev(sel(w)[:, j]), scores, nv)
+            ref_idx = torch.empty((3, wl.k), dtype=torch.int32, device="cuda")
+            topk(scores, nv, wl.k, ref_idx)
+        ref = torch.empty((3, wl.H, wl.D), dtype=torch.bfloat16, device="cuda")
+        B.decode_attn(0, rid, dev(sel(q)[:, j]).to(torch.bfloat16), ref_idx, sink_d, ref)
+        torch.cuda.synchronize()
+        B.check_device_error()
+        assert torch.equal(got[:, j], ref.cpu().view(torch.int16)), f"token {j}: output differs"
+        if csa:
+            assert torch.equal(got_idx[:, j], ref_idx.cpu()), f"token {j}: top-k differs"
+    # the oracle on the chunk's last query of every request, over the rows
+    # the GPU stored (its whole window is in the ring after the chunk)
+    for b, r in enumerate(reqs):
+        T = lens[r] + n_tok
+        last = dict(out_f=out[b, -1].float().cpu().numpy())
+        qq = {r: q[r, -1]}
+        if csa:
+            N = T // 4
+            nvv = torch.empty(1, dtype=torch.int32, device="cuda")
+            sc = torch.empty((1, N + 128), device="cuda")
+            B.index_scores(0, torch.tensor([r], dtype=torch.int32, device="cuda"), dev(qi[r, -1][None]),
+                           dev(w[r, -1][None]), sc, nvv)
+            torch.cuda.synchronize()
+            last.update(scores=sc[0, :N].cpu().numpy(), idx=got_idx[b, -1].numpy())
+            _oracle_check(A, wl, 0, r, T, qq, {r: qi[r, -1]}, {r: w[r, -1]}, sink, last)
+        else:
+            _oracle_check(A, wl, 0, r, T, qq, None, None, sink, last)
