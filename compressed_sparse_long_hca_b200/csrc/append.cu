@@ -416,4 +416,22 @@ cudaError_t launch_chunk_prep(const Layout& L, int layer, int n, const int32_t* 
   return cudaGetLastError();
 }
 
+// 16-byte chunks from src to dst (csa_decode_step: the step's small inputs
+// read straight from page-locked host memory over the bus, one chunk per
+// thread, every load in flight at once).
+__global__ void __launch_bounds__(256) copy16_kernel(const uint4* src, uint4* dst, int64_t n16) {
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n16; x += (int64_t)gridDim.x * blockDim.x)
+    dst[x] = src[x];
+}
+
+cudaError_t launch_copy16(const void* src, void* dst, size_t bytes, cudaStream_t st) {
+  const int64_t n16 = (int64_t)(bytes / 16);
+  if (n16 == 0) return cudaSuccess;
+  const int64_t blocks = (n16 + 255) / 256;
+  copy16_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                                         static_cast<uint4*>(dst), n16);
+  note_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace csa

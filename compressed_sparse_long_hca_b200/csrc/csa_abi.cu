@@ -43,6 +43,7 @@ cudaError_t launch_attn_f32(const Layout& L, int layer, int n, const int32_t* re
                             cudaStream_t st, int q_per_req = 0, const char* win_snap = nullptr);
 cudaError_t launch_chunk_prep(const Layout& L, int layer, int n, const int32_t* req_ids, int n_tok, int32_t* req_exp,
                               char* snap, cudaStream_t st);
+cudaError_t launch_copy16(const void* src, void* dst, size_t bytes, cudaStream_t st);
 int gemm_row_tiles(int n_out);
 int gemm_k_tiles(int k_in, int groups);
 size_t gemm_weight_bytes(int n_out, int k_in, int groups);
@@ -543,6 +544,17 @@ struct StepLayout {
   size_t ws_bytes;
 };
 
+// The device's address of page-locked (pinned or registered) host memory,
+// or null for any other memory (pageable host memory, device memory).
+const void* mapped_host(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 StepLayout step_layout(const csa_cache* c, int32_t layer, int32_t n, int32_t k) {
   const Layout& L = c->L;
   const bool csa = layer < L.n_csa;
@@ -601,9 +613,16 @@ csa_status csa_decode_step(csa_cache_t* c, int32_t layer, int32_t n, const int32
   char* d = static_cast<char*>(dev_buf);
   const char* h = static_cast<const char*>(host_in);
   cudaStream_t st = (cudaStream_t)stream;
-  // inputs before q in one copy; q, which only the attention reads, on the
-  // cache's second stream beside the append and the selection
-  cudaError_t e = cudaMemcpyAsync(d, h, (size_t)sl.q, cudaMemcpyHostToDevice, st);
+  // Page-locked host buffers are read and written by the kernels over the
+  // bus (a copy kernel for the small inputs, the attention's own output
+  // stores): a copy-engine transfer costs about 12 us of fixed latency on the
+  // step's critical path.  Other host memory goes through copies.
+  const void* in_dev = mapped_host(host_in);
+  void* out_dev = const_cast<void*>(mapped_host(host_out));
+  // inputs before q (for the append and the selection) first; q, which only
+  // the attention reads, on the cache's second stream beside them
+  cudaError_t e = in_dev != nullptr ? csa::launch_copy16(in_dev, d, (size_t)sl.q, st)
+                                    : cudaMemcpyAsync(d, h, (size_t)sl.q, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaEventRecord(c->ev_fork, st);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(c->side, c->ev_fork, 0);
   if (e == cudaSuccess) e = cudaMemcpyAsync(d + sl.q, h + sl.q, (size_t)sl.q_bytes, cudaMemcpyHostToDevice, c->side);
@@ -624,12 +643,14 @@ csa_status csa_decode_step(csa_cache_t* c, int32_t layer, int32_t n, const int32
   if (r != CSA_OK) return r;
   e = cudaStreamWaitEvent(st, c->ev_q, 0);
   if (e != cudaSuccess) return cuda_fail(e, "decode step join");
-  r = csa_hca_decode_attn(c, layer, n, req_ids, d + sl.q, idx, csa ? k : 0, sink, scale, d + sl.d_out,
-                          d + sl.d_ws, sl.ws_bytes, (csa_variant)(CSA_VARIANT_AUTO | (csa ? CSA_ATTN_STATE_READY : 0)),
-                          stream);
+  r = csa_hca_decode_attn(c, layer, n, req_ids, d + sl.q, idx, csa ? k : 0, sink, scale,
+                          out_dev != nullptr ? out_dev : d + sl.d_out, d + sl.d_ws, sl.ws_bytes,
+                          (csa_variant)(CSA_VARIANT_AUTO | (csa ? CSA_ATTN_STATE_READY : 0)), stream);
   if (r != CSA_OK) return r;
-  e = cudaMemcpyAsync(host_out, d + sl.d_out, (size_t)sl.out_bytes, cudaMemcpyDeviceToHost, st);
-  if (e != cudaSuccess) return cuda_fail(e, "decode step output copy");
+  if (out_dev == nullptr) {
+    e = cudaMemcpyAsync(host_out, d + sl.d_out, (size_t)sl.out_bytes, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode step output copy");
+  }
   return CSA_OK;
 }
 

@@ -384,9 +384,13 @@ csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* cache, int32_t layer, 
  *             layer, n, k) bytes, 256-byte aligned (the inputs' copy, the
  *             scores, counts and indices, the attention workspace, the
  *             output before its copy), owned by the caller.
- * The inputs before q travel in one copy; q travels on a second stream owned
- * by the cache, beside the append and the selection, and the attention
- * waits for it.  The call is asynchronous: host_in must not change, and
+ * The inputs before q travel first; q travels on a second stream owned by
+ * the cache, beside the append and the selection, and the attention waits
+ * for it.  When host_in is page-locked (pinned or registered) the inputs
+ * before q are read by a copy kernel straight from host memory, and when
+ * host_out is, the attention writes the output straight into it: no
+ * copy-engine transfer (each costs about 12 us of fixed latency) on the
+ * step's critical path.  Other host memory goes through cudaMemcpyAsync.  The call is asynchronous: host_in must not change, and
  * host_out must not be read, until the stream has passed the call.  It can
  * be captured in a CUDA graph (the host pointers are then fixed).  Calls on
  * one cache must not run concurrently from several host threads (the
