@@ -625,7 +625,10 @@ csa_status csa_decode_step(csa_cache_t* c, int32_t layer, int32_t n, const int32
                                     : cudaMemcpyAsync(d, h, (size_t)sl.q, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaEventRecord(c->ev_fork, st);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(c->side, c->ev_fork, 0);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(d + sl.q, h + sl.q, (size_t)sl.q_bytes, cudaMemcpyHostToDevice, c->side);
+  if (e == cudaSuccess)
+    e = in_dev != nullptr
+            ? csa::launch_copy16(static_cast<const char*>(in_dev) + sl.q, d + sl.q, (size_t)sl.q_bytes, c->side)
+            : cudaMemcpyAsync(d + sl.q, h + sl.q, (size_t)sl.q_bytes, cudaMemcpyHostToDevice, c->side);
   if (e == cudaSuccess) e = cudaEventRecord(c->ev_q, c->side);
   if (e != cudaSuccess) return cuda_fail(e, "decode step input copies");
   csa_status r = csa_compress_append(c, layer, n, req_ids, 1, reinterpret_cast<const float*>(d + sl.c),

@@ -387,7 +387,7 @@ csa_status csa_hca_decode_attn_noalloc(const csa_cache_t* cache, int32_t layer, 
  * The inputs before q travel first; q travels on a second stream owned by
  * the cache, beside the append and the selection, and the attention waits
  * for it.  When host_in is page-locked (pinned or registered) the inputs
- * before q are read by a copy kernel straight from host memory, and when
+ * are read by copy kernels straight from host memory, and when
  * host_out is, the attention writes the output straight into it: no
  * copy-engine transfer (each costs about 12 us of fixed latency) on the
  * step's critical path.  Other host memory goes through cudaMemcpyAsync.  The call is asynchronous: host_in must not change, and
