@@ -138,3 +138,62 @@ def test_decode_step_rejects_mis_sized_or_device_inputs():
     torch.cuda.synchronize()
     with pytest.raises(ValueError):
         DecodeStep(pair.cache, 0, [], 0, pair.params[0]["sink"])
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_c_decode_step_pageable_and_pinned_buffers_agree(layer):
+    """csa_decode_step called through the C ABI: with page-locked host
+    buffers the step's kernels read the inputs and write the output over the
+    bus directly; with pageable host memory (numpy arrays) it copies them
+    through the copy engine.  Both, on two caches filled identically, give
+    the same bits, step after step."""
+    from compressed_sparse_long_hca_b200 import _lib
+    from compressed_sparse_long_hca_b200.api import decode_step_fields
+    lib = _lib.load()
+    wl = I.Workload("step-c", "csa", H=16, D=128, R=32, H_I=8, d_I=64, k=40, W=128, context=0, batch=0,
+                    seed=4343)
+    lens = [900, 131]
+    reqs = [1, 0]
+    pairs = [Hp.Pair(wl, 1, 1, max_req=2, capacity=max(lens) + 64) for _ in range(2)]
+    for pair in pairs:
+        for r, T in enumerate(lens):
+            pair.cache.request_alloc(r, T + 64)
+            pair.append(layer, [r], {r: pair.gen_tokens(layer, r, 0, T)}, T, oracle=False)
+    torch.cuda.synchronize()
+    csa = layer == 0
+    k = wl.k if csa else 0
+    sink = torch.from_numpy(pairs[0].params[layer]["sink"]).cuda()
+    rid = torch.tensor(reqs, dtype=torch.int32, device="cuda")
+    fields, in_bytes = decode_step_fields(2, wl.H, wl.D, wl.H_I, wl.d_I, csa)
+    assert lib.csa_decode_step_input_bytes(pairs[0].cache.handle, layer, 2) == in_bytes
+    dev_bytes = lib.csa_decode_step_dev_bytes(pairs[0].cache.handle, layer, 2, k)
+    bufs = [torch.zeros(dev_bytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    pinned_in = torch.zeros(in_bytes, dtype=torch.uint8).pin_memory()
+    pinned_out = torch.zeros((2, wl.H, wl.D), dtype=torch.bfloat16).pin_memory()
+    page_in = np.zeros(in_bytes, dtype=np.uint8)
+    page_out = np.zeros(2 * wl.H * wl.D, dtype=np.uint16)
+    rng = np.random.default_rng(29)
+    scale = 1.0 / float(np.sqrt(wl.D))
+    stream = torch.cuda.current_stream().cuda_stream
+    for s in range(4):
+        page_in[:] = rng.integers(0, 256, in_bytes, dtype=np.uint8)
+        # sane values: fp32 fields from N(0, 1), the bf16 q from the bf16 grid
+        for name, dtype, shape, off, nbytes in fields:
+            if dtype == torch.float32:
+                page_in[off: off + nbytes] = rng.standard_normal(nbytes // 4).astype(np.float32).view(np.uint8)
+            else:
+                q = I.bf16_grid(rng.standard_normal(nbytes // 2).astype(np.float32))
+                page_in[off: off + nbytes] = torch.from_numpy(q).to(torch.bfloat16).view(torch.uint8).numpy()
+        pinned_in.copy_(torch.from_numpy(page_in))
+        st = lib.csa_decode_step(pairs[0].cache.handle, layer, 2, rid.data_ptr(), k, sink.data_ptr(), scale,
+                                 pinned_in.data_ptr(), pinned_out.data_ptr(), bufs[0].data_ptr(), dev_bytes, stream)
+        assert st == 0, _lib.load().csa_last_error()
+        st = lib.csa_decode_step(pairs[1].cache.handle, layer, 2, rid.data_ptr(), k, sink.data_ptr(), scale,
+                                 page_in.ctypes.data, page_out.ctypes.data, bufs[1].data_ptr(), dev_bytes, stream)
+        assert st == 0, _lib.load().csa_last_error()
+        torch.cuda.synchronize()
+        pairs[0].cache.check_device_error()
+        pairs[1].cache.check_device_error()
+        assert np.array_equal(pinned_out.view(torch.int16).numpy().reshape(-1).view(np.uint16), page_out), \
+            f"step {s}: output differs"
+        assert np.any(page_out != 0)
