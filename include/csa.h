@@ -310,9 +310,15 @@ csa_status csa_index_topk(const csa_cache_t* cache, int32_t layer, int32_t n,
  *                         tiles; `workspace` is not used (may be NULL).
  *   CSA_VARIANT_LOW_OCC   one thread block per (query, 32 heads, chunk);
  *                         the chunks' results go to `workspace` and a second
- *                         kernel folds them.  Needs workspace_bytes >=
- *                         csa_attn_workspace_bytes(cache, layer, n, k) and a
- *                         16-byte aligned workspace, else CSA_ERR_ARG.
+ *                         kernel folds them -- or, when every (query, 32
+ *                         heads) group of blocks fits on the GPU at once as
+ *                         one thread-block cluster (at most 16 chunks), the
+ *                         blocks of a cluster fold the results through
+ *                         distributed shared memory instead, in the same
+ *                         order and with the same arithmetic.  Needs
+ *                         workspace_bytes >= csa_attn_workspace_bytes(cache,
+ *                         layer, n, k) and a 16-byte aligned workspace, else
+ *                         CSA_ERR_ARG (whichever fold runs).
  *   CSA_VARIANT_AUTO      LOW_OCC when the workspace suffices and HIGH_OCC
  *                         would leave SMs idle, else HIGH_OCC.
  * All three return identical bits.  Any of them may carry the flag
