@@ -358,11 +358,13 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
   if (k < 1 || ld < 1) return fail(CSA_ERR_ARG, "k and ld must be >= 1");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
   // One thread-block cluster per query: 16 CTAs for an under-fed GPU (8 where
-  // the device cannot co-schedule 16), 8 for a well-fed one.  The selection
-  // is exact, so both return identical indices.
+  // the device cannot co-schedule 16), 8 for a well-fed one.  A row of at
+  // most 4096 scores fits one thread block: AUTO and HIGH_OCC then select it
+  // in a single block (no cluster round trips), LOW_OCC in a cluster of 8.
+  // The selection is exact, so every form returns identical indices.
   const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 10);
-  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, low ? 16 : 8,
-                                   (cudaStream_t)stream);
+  const int cluster = ld <= 4096 ? (variant == CSA_VARIANT_LOW_OCC ? 8 : 1) : (low ? 16 : 8);
+  cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, cluster, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "topk launch");
   return CSA_OK;
 }

@@ -678,6 +678,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid,
     case 16: return launch_topk_c<16>(a, sm, st);
     case 8: return launch_topk_c<8>(a, sm, st);
     case 4: return launch_topk_c<4>(a, sm, st);
+    case 1: return launch_topk_c<1>(a, sm, st);
     default: return cudaErrorInvalidValue;
   }
 }
