@@ -25,8 +25,16 @@
 //
 // Fixed K split.  A weight with few row tiles cannot fill the SMs; its K
 // range is then cut into S parts, S chosen from the weight's shape alone
-// (never from the batch), and a second kernel adds the parts' fp32 partials
-// in part order.  The result is therefore still independent of the batch.
+// (never from the batch).  Each part's CTA writes its fp32 partial; the CTA
+// that finishes a row tile last (a counter per row tile) adds the S
+// partials in part order and writes the output.  The result is therefore
+// still independent of the batch, and of which CTA comes last.
+//
+// Launch.  The activations are packed by a small kernel first; the GEMM is
+// launched with programmatic dependent launch behind it, so its CTAs set up
+// and start streaming their first weight tiles (which do not depend on the
+// pack) while the pack runs, and wait for it before the first activation
+// block is copied.
 //
 // Groups.  With G groups the weight is block diagonal: the rows of group g
 // (n_out / G of them, a multiple of 128) read the activation columns
@@ -75,6 +83,7 @@ struct GemmArgs {
   int splits;             // fixed K split
   GemmOut out;
   float* part;            // [splits][n_tok][n_out] fp32 partials (splits > 1)
+  int32_t* done;          // [row_tiles] parts finished (splits > 1; zeroed by the pack kernel)
 };
 
 __host__ __device__ __forceinline__ int gemm_stages(int n_pad) {
@@ -89,8 +98,12 @@ __host__ __device__ __forceinline__ int gemm_stages(int n_pad) {
 // start at y * kg): block b of a group holds rows 0 .. n_pad-1 of its
 // columns [64 b, 64 b + 64), 16-byte chunk c of row t at
 // (t/8)*1024 + c*128 + (t%8)*16.  Rows >= n_tok and columns >= kg are zero.
+// Also clears the GEMM's row-tile counters (n_done of them, may be null).
 __global__ void gemm_pack_x_strided_kernel(const uint16_t* x, int n_tok, int kg, int row_len, int n_pad, int k_tiles,
-                                           uint8_t* xp) {
+                                           uint8_t* xp, int32_t* done, int n_done) {
+  tc::griddep_launch_dependents();      // the GEMM may become resident now; it waits for this grid's writes
+  if (done != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int u = threadIdx.x; u < n_done; u += blockDim.x) done[u] = 0;
   x += (int64_t)blockIdx.y * kg;
   xp += (int64_t)blockIdx.y * k_tiles * n_pad * 128;
   const int64_t total = (int64_t)k_tiles * n_pad * 8;
@@ -123,6 +136,7 @@ __global__ void __launch_bounds__(kGThreads, 2) gemm_bf16_kernel(GemmArgs a) {
   uint64_t* acc_full = empty + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
   const int rt = blockIdx.x, sp = blockIdx.y;
   // this CTA's K tiles (fixed split) and, for a grouped weight, the
   // activation blocks its rows read
@@ -149,9 +163,29 @@ __global__ void __launch_bounds__(kGThreads, 2) gemm_bf16_kernel(GemmArgs a) {
   const int nk = kt1 - kt0;
   bool ok = true;
   int issued = 0;                                    // producer: stages filled so far
+  if (warp != 0) tc::griddep_wait();                 // the pack kernel's writes (activations, counters)
   if (warp == 0) {
-    // ---- producer: weight tile + activation block per stage
-    for (int x = 0; x < nk && ok; ++x) {
+    // ---- producer: weight tile + activation block per stage.  The weight
+    //      tiles of the first stages do not depend on the pack kernel and
+    //      are issued before waiting for it.
+    const int pre = nk < S ? nk : S;
+    if (tc::elect_one()) {
+      for (int x = 0; x < pre; ++x) {
+        tc::mbar_arrive_expect_tx(&full[x], (uint32_t)stage_bytes);
+        tc::bulk_g2s(sm + (int64_t)x * stage_bytes, a.w + ((int64_t)rt * a.k_tiles + kt0 + x) * kWTileBytes,
+                     kWTileBytes, &full[x]);
+      }
+    }
+    __syncwarp();
+    tc::griddep_wait();
+    if (tc::elect_one()) {
+      for (int x = 0; x < pre; ++x)
+        tc::bulk_g2s(sm + (int64_t)x * stage_bytes + kWTileBytes, a.xp + (int64_t)(xblk0 + kt0 + x) * xb,
+                     (uint32_t)xb, &full[x]);
+    }
+    __syncwarp();
+    issued = pre;
+    for (int x = pre; x < nk && ok; ++x) {
       const int s = x % S;
       if (x >= S) ok = tc::mbar_wait(&empty[s], ((x / S) - 1) & 1, 1000000000ull);
       ok = __all_sync(0xffffffffu, ok);
@@ -214,6 +248,35 @@ __global__ void __launch_bounds__(kGThreads, 2) gemm_bf16_kernel(GemmArgs a) {
         }
       }
     }
+    if (a.splits > 1) {
+      // the last of the row tile's S CTAs adds the partials in part order
+      // (every CTA takes part, also after an abort, so the count completes)
+      __threadfence();
+      tc::named_bar_sync(1, 128);
+      if (tid == 64) last_flag[0] = atomicAdd(&a.done[rt], 1) == a.splits - 1 ? 1 : 0;
+      tc::named_bar_sync(1, 128);
+      if (last_flag[0] && ok && !*abort_flag) {
+        __threadfence();
+        if (o < a.n_out) {
+          // acc = part 0, then + part 1, + part 2, ...; the loads of up to
+          // 16 parts are in flight together
+          const int64_t n = (int64_t)a.n_tok * a.n_out;
+          for (int t = 0; t < a.n_tok; ++t) {
+            const float* p = a.part + (int64_t)t * a.n_out + o;
+            float acc = 0.f;
+            for (int q0 = 0; q0 < a.splits; q0 += 16) {
+              float v[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = q0 + j < a.splits ? __ldcg(p + (q0 + j) * n) : 0.f;
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (q0 + j < a.splits) acc = q0 + j == 0 ? v[j] : acc + v[j];
+            }
+            gemm_store(a.out, t, o, acc);
+          }
+        }
+      }
+    }
     if (!ok) *abort_flag = 1;
   }
   tc::tc_fence_before();
@@ -228,16 +291,6 @@ __global__ void __launch_bounds__(kGThreads, 2) gemm_bf16_kernel(GemmArgs a) {
     // barrier covers every MMA issued; after an abort, wait on it bounded)
     tc::mbar_wait(acc_full, 0, 200000000ull);
     tc::tmem_dealloc(tmem, ncols);
-  }
-}
-
-// Fixed-order sum of the K parts: Y[t][o] = sum over s ascending of part[s][t][o].
-__global__ void gemm_reduce_kernel(const float* part, int splits, int n_tok, int n_out, GemmOut out) {
-  const int64_t n = (int64_t)n_tok * n_out;
-  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < n; u += (int64_t)gridDim.x * blockDim.x) {
-    float acc = part[u];
-    for (int s = 1; s < splits; ++s) acc += part[(int64_t)s * n + u];
-    gemm_store(out, (int)(u / n_out), (int)(u % n_out), acc);
   }
 }
 
@@ -265,7 +318,8 @@ size_t gemm_workspace_bytes(int n_out, int k_in, int groups, int n_tok, int sms)
   const size_t xp = (size_t)gemm_k_tiles(k_in, groups) * groups * n_pad * 128;
   const int S = gemm_splits(n_out, k_in, groups, sms);
   const size_t part = S > 1 ? (size_t)S * n_tok * n_out * 4 : 0;
-  return (xp + 255) / 256 * 256 + part;
+  const size_t done = S > 1 ? (size_t)gemm_row_tiles(n_out) * 4 : 0;
+  return (xp + 255) / 256 * 256 + part + done;
 }
 
 // Row-major BF16 weight [n_out][k_in] (host) -> packed tiles (host buffer):
@@ -299,13 +353,14 @@ cudaError_t launch_gemm_bf16(const void* w_packed, int n_out, int k_in, int grou
   uint8_t* xp = static_cast<uint8_t*>(ws);
   const size_t xp_bytes = ((size_t)kt * groups * n_pad * 128 + 255) / 256 * 256;
   float* part = S > 1 ? reinterpret_cast<float*>(xp + xp_bytes) : nullptr;
+  int32_t* done = S > 1 ? reinterpret_cast<int32_t*>(part + (size_t)S * n_tok * n_out) : nullptr;
   // packed activations: group g's k tiles are blocks g kt .. g kt + kt - 1
   cudaError_t e = cudaSuccess;
   {
     const int kg = k_in / groups;
     const int64_t chunks = (int64_t)kt * n_pad * 8;
     const int blocks = (int)((chunks + 255) / 256 < 2048 ? (chunks + 255) / 256 : 2048);
-    gemm_pack_x_strided_kernel<<<dim3(blocks, groups), 256, 0, st>>>(x, n_tok, kg, k_in, n_pad, kt, xp);
+    gemm_pack_x_strided_kernel<<<dim3(blocks, groups), 256, 0, st>>>(x, n_tok, kg, k_in, n_pad, kt, xp, done, rt);
     note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -319,15 +374,21 @@ cudaError_t launch_gemm_bf16(const void* w_packed, int n_out, int k_in, int grou
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  GemmArgs a{static_cast<const uint8_t*>(w_packed), xp, n_out, k_in, n_tok, n_pad, rt, kt, groups, S, out, part};
-  gemm_bf16_kernel<<<dim3(rt, S), kGThreads, smem, st>>>(a);
+  GemmArgs a{static_cast<const uint8_t*>(w_packed), xp, n_out, k_in, n_tok, n_pad, rt, kt, groups, S, out, part,
+             done};
+  cudaLaunchConfig_t lc{};
+  lc.gridDim = dim3(rt, S);
+  lc.blockDim = dim3(kGThreads);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&lc, gemm_bf16_kernel, a);
   note_launch();
-  e = cudaGetLastError();
-  if (e != cudaSuccess || S == 1) return e;
-  const int64_t n = (int64_t)n_tok * n_out;
-  gemm_reduce_kernel<<<(int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(part, S, n_tok, n_out,
-                                                                                            out);
-  note_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

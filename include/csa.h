@@ -483,7 +483,8 @@ csa_status csa_prefill_chunk(csa_cache_t* cache, int32_t layer, int32_t n, const
  * tiles has its K range cut into a number of parts (enough to give every
  * SM two CTAs, each part at least 256 K values) that depends on the
  * weight's shape and the device's SM count alone, never on the batch, and
- * the parts are summed in part order.
+ * the parts are summed in part order (by whichever CTA of a row tile
+ * finishes last; the order of the sum does not depend on which one).
  *
  * Groups: with `groups` (1 .. 65535) > 1 the weight is block diagonal; group g's rows
  * (n_out / groups of them, a multiple of 128) read the columns
@@ -494,7 +495,8 @@ csa_status csa_prefill_chunk(csa_cache_t* cache, int32_t layer, int32_t n, const
  *   csa_gemm_pack_weight    host BF16 W (row-major, as above) -> packed
  *                           device tiles; synchronous
  *   csa_gemm_workspace_bytes  scratch of one call (packed activations, and
- *                           the parts' partials when K is split)
+ *                           when K is split the parts' partials and one
+ *                           counter per 128-row tile)
  *   csa_gemm_bf16           X device BF16 [n_tok][k_in], 1 <= n_tok <= 256.
  *                           Y is written as n_seg (1 .. 8) row segments:
  *                           rows [r_s, r_s + segs[s].rows) of Y go to the
