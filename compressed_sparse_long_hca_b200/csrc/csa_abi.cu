@@ -21,6 +21,7 @@ cudaError_t launch_append(const Layout& L, int layer, int n, const int32_t* req_
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
                             cudaStream_t st, int q_per_req = 0);
+int topk_cluster_one_wave(int64_t ld, int n);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st);
 cudaError_t launch_attn_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const uint16_t* q,
@@ -357,13 +358,18 @@ csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int
   if (!scores || !n_valid || !idx_out) return fail(CSA_ERR_ARG, "NULL argument");
   if (k < 1 || ld < 1) return fail(CSA_ERR_ARG, "k and ld must be >= 1");
   if (variant < CSA_VARIANT_AUTO || variant > CSA_VARIANT_LOW_OCC) return fail(CSA_ERR_ARG, "bad variant");
-  // One thread-block cluster per query: 16 CTAs for an under-fed GPU (8 where
-  // the device cannot co-schedule 16), 8 for a well-fed one.  A row of at
-  // most 4096 scores fits one thread block: AUTO and HIGH_OCC then select it
-  // in a single block (no cluster round trips), LOW_OCC in a cluster of 8.
-  // The selection is exact, so every form returns identical indices.
-  const bool low = variant == CSA_VARIANT_LOW_OCC || (variant == CSA_VARIANT_AUTO && n < 10);
-  const int cluster = ld <= 4096 ? (variant == CSA_VARIANT_LOW_OCC ? 8 : 1) : (low ? 16 : 8);
+  // One thread-block cluster per query: 16 CTAs for LOW_OCC (8 where the
+  // device cannot co-schedule 16), 8 for HIGH_OCC; AUTO takes the largest
+  // of 16, 8 and 4 whose n clusters the device holds at once (one CTA of
+  // 1024 threads per SM: 32 queries take clusters of 4 rather than two
+  // waves of 8).  A row of at most 4096 scores fits one thread block: AUTO
+  // and HIGH_OCC then select it in a single block (no cluster round trips),
+  // LOW_OCC in a cluster of 8.  The selection is exact, so every form
+  // returns identical indices.
+  int cluster = 8;
+  if (ld <= 4096) cluster = variant == CSA_VARIANT_LOW_OCC ? 8 : 1;
+  else if (variant == CSA_VARIANT_LOW_OCC) cluster = 16;
+  else if (variant == CSA_VARIANT_AUTO) cluster = csa::topk_cluster_one_wave(ld, n);
   cudaError_t e = csa::launch_topk(scores, ld, n_valid, n, k, idx_out, nullptr, cluster, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "topk launch");
   return CSA_OK;

@@ -661,7 +661,44 @@ bool cluster16_ok(size_t sm) {
   return ok;
 }
 
+// How many clusters of C CTAs of the kernel, with `sm` bytes of shared
+// memory each, the device holds at once (asked once per device, C and size).
+template <int C>
+int max_clusters(size_t sm) {
+  static int cached_dev = -1;
+  static size_t cached_sm = 0;
+  static int cached_n = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev == cached_dev && sm == cached_sm) return cached_n;
+  int n = 0;
+  if (cudaFuncSetAttribute(topk_cluster_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) ==
+      cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, 1, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = sm;
+    if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<C>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  cached_dev = dev;
+  cached_sm = sm;
+  cached_n = n;
+  return n;
+}
+
 }  // namespace
+
+// Cluster size for n rows of ld scores on a GPU that should take them in
+// one wave: the largest of 16, 8 and 4 whose n clusters are all resident at
+// once (16 only where the device co-schedules it), else 4.
+int topk_cluster_one_wave(int64_t ld, int n) {
+  bool cache = false;
+  const size_t sm16 = topk_smem_bytes(ld, 16, &cache);
+  if (cluster16_ok(sm16) && n <= max_clusters<16>(sm16)) return 16;
+  if (n <= max_clusters<8>(topk_smem_bytes(ld, 8, &cache))) return 8;
+  return 4;
+}
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* n_valid, int n, int k,
                         int32_t* out, int32_t* err, int cluster, cudaStream_t st) {

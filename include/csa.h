@@ -237,9 +237,10 @@ csa_status csa_index_scores(const csa_cache_t* cache, int32_t layer, int32_t n,
  * padded with -1 when n_valid[i] < k.
  *   idx_out  device int32 [n][k]
  * Scores must not be NaN (a NaN is ordered above +inf).  One thread-block
- * cluster per query: 16 blocks (LOW_OCC, and AUTO for fewer than 10
- * queries) or 8; rows of at most 4096 scores take a single block (AUTO,
- * HIGH_OCC) or 8 (LOW_OCC).  Every form returns identical indices.
+ * cluster per query: 16 blocks (LOW_OCC), 8 (HIGH_OCC), and for AUTO the
+ * largest of 16, 8 and 4 whose n clusters the device holds at once (else
+ * 4); rows of at most 4096 scores take a single block (AUTO, HIGH_OCC) or
+ * 8 (LOW_OCC).  Every form returns identical indices.
  */
 csa_status csa_topk(const float* scores, int64_t ld, const int32_t* n_valid, int32_t n,
                     int32_t k, int32_t* idx_out, csa_variant variant, csa_stream_t stream);
