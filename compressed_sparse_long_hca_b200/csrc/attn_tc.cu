@@ -847,14 +847,16 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(AttnArgs a) {
 // Split launch, second step: fold the chunk partials of (query blockIdx.y,
 // head blockIdx.x) in chunk order; thread x owns dims 4x .. 4x+3.
 __global__ void __launch_bounds__(128) attn_fold_kernel(AttnArgs a) {
-  tc::griddep_wait();                                   // the partials are complete from here on
   const Layout& L = a.L;
   const int h = blockIdx.x, i = blockIdx.y, H = L.H, D = L.D;
   const int d4 = threadIdx.x;
-  if (4 * d4 >= D) return;
+  // The request id and its length are final before the partial kernel
+  // (the previous grid) starts, so the query's geometry is read while that
+  // grid finishes; the partials only after the wait.
   QueryGeom g;
-  if (!query_geom(a, i, g, false)) return;             // recorded by the partial kernel
-  if (g.n_chunks > a.chunks_max) return;
+  const bool have = 4 * d4 < D && query_geom(a, i, g, false);   // a bad query is recorded by the partial kernel
+  tc::griddep_wait();                                   // the partials are complete from here on
+  if (!have || g.n_chunks > a.chunks_max) return;
   float m = -INFINITY, l = 0.f;
   float o[4] = {0.f, 0.f, 0.f, 0.f};
   const int64_t base = (int64_t)i * a.chunks_max;
