@@ -157,6 +157,18 @@ def test_kv_row_quantiser():
     assert np.array_equal(O.dequantize_kv(O.quantize_kv(xb, R))[:, -R:], xb[:, -R:])
 
 
+def test_kv_row_rope_dims_are_torch_bf16():
+    """The RoPE dims of a stored row are the BF16 round-to-nearest-even of
+    the fp32 value: torch's own cast, ties and all."""
+    r = _rng(8)
+    D, R = 128, 64
+    x = (r.standard_normal((30, D)) * 3.0).astype(np.float32)
+    x[:, -R:][:, :8] = (np.arange(1, 9, dtype=np.uint32) << 16 | 0x8000).view(np.float32)   # exact ties
+    kv = O.quantize_kv(x.astype(np.float64), R)
+    ref = torch.from_numpy(np.ascontiguousarray(x[:, -R:])).to(torch.bfloat16).view(torch.int16).numpy()
+    assert np.array_equal(kv.rope, ref.view(np.uint16))
+
+
 def test_kv_row_zero():
     kv = O.quantize_kv(np.zeros((1, 128)), 64)
     assert kv.scale[0] == 1.0 and np.all(kv.fp8 == 0)

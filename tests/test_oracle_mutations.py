@@ -15,7 +15,8 @@ from tests import test_oracle_math as TM
 
 _ORIG = {name: getattr(O, name) for name in (
     "rope", "pool", "csa_window", "csa_entries_all", "stored_window", "index_scores", "topk", "mqa_attention", "window_positions",
-    "e4m3_value", "bf16_bits_from_f32", "quantize_mxfp4", "e2m1_code", "grouped_linear", "linear")}
+    "e4m3_value", "bf16_bits_from_f32", "quantize_mxfp4", "e2m1_code", "grouped_linear", "linear",
+    "quantize_kv", "n_csa_entries", "n_hca_entries")}
 
 
 # ---------------------------------------------------------------- the mistakes
@@ -148,6 +149,40 @@ def e2m1_ties_away_from_zero(y):
     return _ORIG["e2m1_code"](y + np.sign(y) * 1e-9)
 
 
+def kv_scale_for_224(x, R):
+    """FP8 scale amax / 224 instead of amax / 448 (half the code range used)."""
+    x32 = O.f32(x)
+    nope = x32[..., :-R]
+    amax = np.max(np.abs(nope), axis=-1).astype(np.float32)
+    s = np.where(amax > 0, amax / np.float32(224.0), np.float32(1.0)).astype(np.float32)
+    y = (nope / s[..., None]).astype(np.float32)
+    return O.KVRow(fp8=O.e4m3_code(y), rope=O.bf16_bits_from_f32(x32[..., -R:]), scale=s)
+
+
+def kv_fp8_truncated(x, R):
+    """FP8 codes by truncation toward zero instead of to nearest."""
+    row = _ORIG["quantize_kv"](x, R)
+    y = (O.f32(x)[..., :-R] / row.scale[..., None]).astype(np.float64)
+    v = O.e4m3_value(row.fp8)
+    over = np.abs(v) > np.abs(y)                 # rounded away from zero: step one code down
+    codes = np.where(over & ((row.fp8 & 0x7F) > 0), row.fp8 - 1, row.fp8).astype(np.uint8)
+    return O.KVRow(fp8=codes, rope=row.rope, scale=row.scale)
+
+
+def kv_rope_truncated(x, R):
+    row = _ORIG["quantize_kv"](x, R)
+    u = O.f32(x)[..., -R:].view(np.uint32)
+    return O.KVRow(fp8=row.fp8, rope=(u >> np.uint32(16)).astype(np.uint16), scale=row.scale)
+
+
+def csa_count_partial_entry(T, m=4):
+    return T // m + 1
+
+
+def hca_count_ratio_127(T, m=128):
+    return T // (m - 1)
+
+
 def grouped_linear_groups_reversed(x, W, groups):
     """Row group g reads column block groups - 1 - g."""
     x = np.asarray(x, np.float64)
@@ -193,6 +228,11 @@ CASES = [
     ("quantize_mxfp4", mxfp4_exponent_off_by_one, TF.test_mxfp4_scale_rule_and_brute_force, ()),
     ("e2m1_code", e2m1_ties_away_from_zero, TF.test_e2m1_ties_to_even_and_saturation, (0.25, 0.0)),
     ("e2m1_code", e2m1_ties_away_from_zero, TF.test_e2m1_ties_to_even_and_saturation, (2.5, 2.0)),
+    ("quantize_kv", kv_scale_for_224, TF.test_kv_row_quantiser, ()),
+    ("quantize_kv", kv_fp8_truncated, TF.test_kv_row_quantiser, ()),
+    ("quantize_kv", kv_rope_truncated, TF.test_kv_row_rope_dims_are_torch_bf16, ()),
+    ("n_csa_entries", csa_count_partial_entry, TM.test_entry_counts_match_page_figures, ()),
+    ("n_hca_entries", hca_count_ratio_127, TM.test_entry_counts_match_page_figures, ()),
     ("grouped_linear", grouped_linear_groups_reversed, TM.test_grouped_linear_is_block_diagonal_dense, ()),
     ("linear", linear_drops_last_column, TM.test_linear_brute_force_and_one_hot, ()),
 ]
