@@ -6,6 +6,7 @@ protocol: per-rank device timings combine as a maximum over ranks, the job's
 rate counts every rank's queries, and only rank 0 prints."""
 import contextlib
 import io
+import json
 import os
 import socket
 import sys
@@ -79,6 +80,34 @@ def test_reference_arm_only_rank0_prints(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(Args())
     assert buf.getvalue() == ""
+
+
+def test_reference_arm_line_keeps_the_contract(monkeypatch):
+    """Rank 0 of the reference arm (the oracle on the host cores) prints one
+    JSON line with the contract's keys, the same metric and unit as the
+    CUDA arm, and its own cpu_baseline and e2e objects."""
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+
+    class Args:
+        workload, steps, warmup = "tiny-csa", 1, 3
+
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_reference(Args())
+    lines = [x for x in buf.getvalue().splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == bench.UNIT and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny-csa" and d["steps"] == 1 and d["warmup"] == 3
+    assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
 def test_bench_byte_counts_and_rooflines():
