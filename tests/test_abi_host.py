@@ -123,3 +123,38 @@ def test_cache_calls_on_a_null_handle_fail_on_the_host(cuda_lib):
     assert cuda_lib.csa_prefill_workspace_bytes(None, 0, 1, 16, 16, 0) == 0
     assert cuda_lib.csa_prefill_chunk(None, 0, 1, P, 16, P, P, P, P, P, P, P, 16, P, 1.0, P, None, P, 1 << 20, 0,
                                       None) == -1
+
+
+def test_gemm_shapes_and_argument_errors_on_the_host(cuda_lib):
+    """The projection GEMM's size function and its argument checks run on the
+    host: packed weight bytes are 128-row x 64-column tiles of 16 KB, a bad
+    shape gives 0 bytes, and csa_gemm_bf16 returns CSA_ERR_ARG for every bad
+    argument before any CUDA call (the pointers below are never touched)."""
+    wb = cuda_lib.csa_gemm_weight_bytes
+    tile = 128 * 64 * 2
+    assert wb(300, 1000, 1) == 3 * 16 * tile                    # ceil(300 / 128) row tiles x ceil(1000 / 64)
+    assert wb(16 * 128, 16 * 64, 16) == 16 * 1 * tile           # block diagonal: each row tile reads its group
+    for bad in ((0, 64, 1), (256, 0, 1), (256, 64, 0), (256, 63, 1), (300, 64, 2), (256, 96, 3),
+                (128 * 70000, 64 * 70000, 70000)):
+        assert wb(*bad) == 0, bad
+    P = 0x10000
+    seg = (_lib.GemmOut * 2)()
+    seg[0].rows, seg[0].bf16, seg[0].y = 100, 1, P
+    seg[1].rows, seg[1].bf16, seg[1].y = 156, 0, P
+    segs = ctypes.cast(seg, ctypes.c_void_p)
+    g = cuda_lib.csa_gemm_bf16
+    cases = [
+        ((P, 256, 63, 1, P, 4, 2, segs, P, 1 << 30, None), b"multiple of 8"),
+        ((P, 256, 64, 1, P, 257, 2, segs, P, 1 << 30, None), b"n_tok"),
+        ((P, 256, 64, 1, P, 4, 0, segs, P, 1 << 30, None), b"n_seg"),
+        ((P, 256, 64, 1, P, 4, 9, segs, P, 1 << 30, None), b"n_seg"),
+        ((P, 300, 64, 1, P, 4, 2, segs, P, 1 << 30, None), b"add up"),
+        ((None, 256, 64, 1, P, 4, 2, segs, P, 1 << 30, None), b"NULL"),
+        ((P, 256, 64, 1, P, 4, 2, segs, P + 16, 1 << 30, None), b"aligned"),
+    ]
+    for args, msg in cases:
+        assert g(*args) == -1, args
+        assert msg in cuda_lib.csa_last_error(), (args, cuda_lib.csa_last_error())
+    assert g(P, 256, 64, 1, P, 0, 2, segs, P, 1 << 30, None) == 0     # no tokens: nothing to do
+    seg[1].y = None
+    assert g(P, 256, 64, 1, P, 4, 2, segs, P, 1 << 30, None) == -1    # a segment without an output
