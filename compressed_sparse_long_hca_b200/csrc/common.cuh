@@ -16,6 +16,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "layout.cuh"
 
 namespace csa {
@@ -154,6 +156,17 @@ __device__ __forceinline__ void store_index_key(const Layout& L, const float* ke
       if (l == 0) sfchunk[Layout::idx_sf_off(s, c)] = 127;
     }
   }
+}
+
+// Host side: whether the kernel set-up marked by `done` (one bit per device)
+// still has to run on device `dev`; devices beyond 63 always run it.  Set-up
+// calls (function attributes, occupancy queries) are per device, and two
+// host threads may both run one (they are idempotent).
+inline bool setup_needed(const std::atomic<uint64_t>& done, int dev) {
+  return dev < 0 || dev >= 64 || !((done.load(std::memory_order_acquire) >> dev) & 1u);
+}
+inline void setup_done(std::atomic<uint64_t>& done, int dev) {
+  if (dev >= 0 && dev < 64) done.fetch_or(uint64_t(1) << dev, std::memory_order_release);
 }
 
 }  // namespace csa

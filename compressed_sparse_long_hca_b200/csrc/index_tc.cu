@@ -1079,12 +1079,15 @@ size_t index_tc_smem_bytes() { return kSmemPlain > 80 * 1024 ? kSmemPlain : 80 *
 cudaError_t launch_index_tc(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                             const float* w, float* scores, int64_t ld, int32_t* n_valid, int ctas,
                             cudaStream_t st, int q_per_req) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)index_tc_smem_bytes());
+  static std::atomic<uint64_t> attr_set{0};     // devices whose kernel attribute is set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (setup_needed(attr_set, dev)) {
+    e = cudaFuncSetAttribute(index_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)index_tc_smem_bytes());
     if (e != cudaSuccess) return e;
-    attr = true;
+    setup_done(attr_set, dev);
   }
   IndexTcArgs a{L, layer, n, req_ids, q_idx, w, scores, ld, n_valid};
   a.q_per_req = q_per_req;
@@ -1125,7 +1128,14 @@ int index_topk_max_ctas() { return kThreads; }
 cudaError_t launch_index_topk(const Layout& L, int layer, int n, const int32_t* req_ids, const float* q_idx,
                               const float* w, float* scores, int64_t ld, int32_t* n_valid, int k, int32_t* idx_out,
                               void* ws, int ctas, cudaStream_t st) {
-  static int occ = 0;                      // CTAs per SM that can be resident together
+  // CTAs per SM that can be resident together, per device (the attributes
+  // are set and the occupancy asked once on each device)
+  static std::atomic<int> occ_by_dev[64];
+  int dev = 0, sms = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e0 != cudaSuccess) return e0;
+  int occ = dev >= 0 && dev < 64 ? occ_by_dev[dev].load(std::memory_order_acquire) : 0;
   if (occ == 0) {
     cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)index_topk_smem_bytes());
@@ -1136,13 +1146,10 @@ cudaError_t launch_index_topk(const Layout& L, int layer, int n, const int32_t* 
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_tc_kernel<true>, kThreads, index_topk_smem_bytes());
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) occ_by_dev[dev].store(occ, std::memory_order_release);
   }
   // the CTAs of a query wait for one another, so the grid never exceeds what
   // is resident at once; the selection enumerates a query's CTAs one per thread
-  int dev = 0, sms = 0;
-  cudaError_t e0 = cudaGetDevice(&dev);
-  if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e0 != cudaSuccess) return e0;
   if (ctas > occ * sms) ctas = occ * sms;
   if (ctas > kThreads) ctas = kThreads;
   const TopkWs wl = topk_ws(n, ld);

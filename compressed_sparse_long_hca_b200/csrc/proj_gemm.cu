@@ -366,13 +366,16 @@ cudaError_t launch_gemm_bf16(const void* w_packed, int n_out, int k_in, int grou
     if (e != cudaSuccess) return e;
   }
   const size_t smem = (size_t)gemm_stages(n_pad) * (kWTileBytes + n_pad * 128) + 256 + 128;
-  static bool attr = false;
-  if (!attr) {
+  static std::atomic<uint64_t> attr_set{0};     // devices whose kernel attributes are set
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (setup_needed(attr_set, dev)) {
     e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    attr = true;
+    setup_done(attr_set, dev);
   }
   GemmArgs a{static_cast<const uint8_t*>(w_packed), xp, n_out, k_in, n_tok, n_pad, rt, kt, groups, S, out, part,
              done};

@@ -35,6 +35,8 @@
 // memory (the bulk copy's mbarrier) gives up after a time limit.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -634,9 +636,14 @@ cudaError_t launch_topk_c(const TopkArgs& a, size_t sm, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// The occupancy answers below are cached per (device, size); calls may come
+// from several host threads, so each cache is read and written under a lock.
+std::mutex g_occupancy_mu;
+
 // Whether this device can co-schedule a 16-CTA cluster of the kernel with
 // `sm` bytes of shared memory (asked once per device and size).
 bool cluster16_ok(size_t sm) {
+  std::lock_guard<std::mutex> lock(g_occupancy_mu);
   static int cached_dev = -1;
   static size_t cached_sm = 0;
   static bool cached_ok = false;
@@ -665,6 +672,7 @@ bool cluster16_ok(size_t sm) {
 // memory each, the device holds at once (asked once per device, C and size).
 template <int C>
 int max_clusters(size_t sm) {
+  std::lock_guard<std::mutex> lock(g_occupancy_mu);
   static int cached_dev = -1;
   static size_t cached_sm = 0;
   static int cached_n = 0;
